@@ -1,0 +1,17 @@
+"""Oracle — plain, slow, obviously-correct CPU restatement of the denoise path.
+
+TEST INFRASTRUCTURE ONLY.  Only `tests/`, `__graft_entry__.smoke()` and the
+CPU-baseline leg of `bench.py` may import anything under `oracle/`; the CUDA
+product path never does, and the two share no code (only the seeded input
+generators in `synth/`).
+
+Modules:
+  model     fp64 numpy forward: prefill, canvas forward, LM-head entropy
+  sampler   Entropy-Bound sampler step and block loop (integer decisions)
+  absorbing absorbing forward process (invariant checks)
+
+Every function is pinned by `tests/test_oracle_*.py` against closed forms,
+brute force or library routines it does not use.  The whole-model composition
+beyond its pinned parts is "parity unpinned": no logits, weights or
+trajectories for it are published.
+"""

@@ -1,0 +1,74 @@
+"""Names, shapes and seeded values of a workload's weights and inputs.
+
+Weight tensors (row-major, the leading index is the output row):
+  tok_emb        [V + 1, d]     token embedding; row V is the [MASK] embedding
+  lm_head        [V, d]         untied LM head (the [MASK] id is not a class)
+  l{l}.wqkv      [(Hq + 2 Hkv) h, d]  rows: the Hq query heads, then Hkv key heads,
+                                then Hkv value heads, head-major, h rows per head
+  l{l}.wo        [d, Hq h]
+  l{l}.router    [E, d]
+  l{l}.gate      [E, I, d]      routed experts, SwiGLU gate projection
+  l{l}.up        [E, I, d]      routed experts, SwiGLU up projection
+  l{l}.down      [E, d, I]      routed experts, down projection
+  l{l}.sgate     [I_s, d]       shared expert
+  l{l}.sup       [I_s, d]
+  l{l}.sdown     [d, I_s]
+Every tensor is drawn i.i.d. (approximately) N(0, init_std^2) and stored in the
+workload's dtype.  In the FP8-expert workloads the three routed-expert tensors are
+additionally quantised (see `synth.fp8`).
+
+Inputs: prompt[b] holds `prompt_len` tokens uniform in [0, V).
+"""
+from __future__ import annotations
+
+import torch
+
+from . import gen
+from .workloads import Workload
+
+
+def layer_specs(w: Workload, l: int):
+    d, h, E, I, Is = w.d_model, w.head_dim, w.n_experts, w.expert_inter, w.shared_inter
+    return [
+        (f"l{l}.wqkv", (w.qkv_rows, d)),
+        (f"l{l}.wo", (d, w.n_q_heads * h)),
+        (f"l{l}.router", (E, d)),
+        (f"l{l}.gate", (E, I, d)),
+        (f"l{l}.up", (E, I, d)),
+        (f"l{l}.down", (E, d, I)),
+        (f"l{l}.sgate", (Is, d)),
+        (f"l{l}.sup", (Is, d)),
+        (f"l{l}.sdown", (d, Is)),
+    ]
+
+
+def global_specs(w: Workload):
+    return [("tok_emb", (w.vocab + 1, w.d_model)), ("lm_head", (w.vocab, w.d_model))]
+
+
+def all_specs(w: Workload):
+    out = list(global_specs(w))
+    for l in range(w.n_layers):
+        out += layer_specs(w, l)
+    return out
+
+
+def store_dtype(w: Workload) -> str:
+    return "f32" if w.dtype == "f32" else "bf16"
+
+
+def weight(w: Workload, name: str, shape, device="cpu", start_row=0, n_rows=None):
+    """Stored (un-quantised) values of one weight tensor or a row range of it."""
+    return gen.weight(w.seed, name, shape, w.init_std, store_dtype(w), device,
+                      start_row, n_rows)
+
+
+def prompt(w: Workload, device="cpu") -> torch.Tensor:
+    """[B, P] int32 prompt tokens uniform in [0, V)."""
+    rows = [gen.tokens(w.seed, f"prompt.b{b}", w.prompt_len, w.vocab, device)
+            for b in range(w.batch)]
+    return torch.stack(rows) if rows else torch.empty(0, w.prompt_len, dtype=torch.int32)
+
+
+def is_fp8_expert(w: Workload, name: str) -> bool:
+    return w.dtype == "bf16_fp8exp" and name.split(".")[-1] in ("gate", "up", "down")

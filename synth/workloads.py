@@ -1,0 +1,92 @@
+"""Workload shapes for the masked-diffusion denoise forward.
+
+Each workload is a model stand-in (dimensions, precision) plus an input recipe
+(batch, prompt length, number of denoise steps T, entropy bound gamma, seed).
+The dimensions the pages fix come from the explainer page "DiffusionGemma
+深度解析", list "核心架构参数" (30 layers, sliding window 1024, 256-token
+canvas, 262K vocabulary, 128 experts with top-8 routing plus one shared
+expert); the hidden sizes are stand-ins the pages do not give.
+
+This module only describes shapes; it holds none of the model's arithmetic.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, replace
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    n_layers: int
+    d_model: int
+    n_q_heads: int
+    n_kv_heads: int
+    head_dim: int
+    n_experts: int
+    top_k: int
+    expert_inter: int
+    shared_inter: int
+    vocab: int            # real tokens; the [MASK] id equals vocab
+    window: int           # sliding attention window over the prompt
+    canvas: int           # C, tokens denoised in parallel
+    rope_base: float
+    rms_eps: float
+    logit_scale: float
+    dtype: str            # "f32" | "bf16" | "bf16_fp8exp"
+    batch: int
+    prompt_len: int
+    T: int                # denoise forwards per block
+    gamma: float          # entropy bound of the sampler
+    seed: int = 0
+    init_std: float = 0.02
+
+    @property
+    def mask_id(self) -> int:
+        return self.vocab
+
+    @property
+    def kv_window(self) -> int:
+        return min(self.prompt_len, self.window)
+
+    @property
+    def qkv_rows(self) -> int:
+        return (self.n_q_heads + 2 * self.n_kv_heads) * self.head_dim
+
+    def with_(self, **kw) -> "Workload":
+        return replace(self, **kw)
+
+
+# Tiny fp32 model: the exact-trajectory case (T = 4).
+TINY_F32 = Workload(
+    name="tiny-f32", n_layers=2, d_model=64, n_q_heads=4, n_kv_heads=2, head_dim=16,
+    n_experts=8, top_k=2, expert_inter=128, shared_inter=128, vocab=512, window=1024,
+    canvas=32, rope_base=10000.0, rms_eps=1e-6, logit_scale=8.0, dtype="f32",
+    batch=1, prompt_len=32, T=4, gamma=1.0)
+
+# One Gemma-4-26B-A4B-shaped layer plus the 262,144-token LM head, BF16.
+LAYER1_BF16 = Workload(
+    name="layer1-bf16", n_layers=1, d_model=2048, n_q_heads=16, n_kv_heads=8, head_dim=128,
+    n_experts=128, top_k=8, expert_inter=768, shared_inter=2048, vocab=262144, window=1024,
+    canvas=256, rope_base=10000.0, rms_eps=1e-6, logit_scale=8.0, dtype="bf16",
+    batch=1, prompt_len=1024, T=12, gamma=1.0)
+
+# Full 30-layer stand-in, batch 1, prompt 1024: the throughput workload.
+FULL30_BF16 = LAYER1_BF16.with_(name="full30-bf16", n_layers=30)
+
+# Same model, 8 independent canvases with 8192-token prompts (window 1024).
+FULL30_B8_P8192 = FULL30_BF16.with_(name="full30-b8-p8192", batch=8, prompt_len=8192)
+
+
+def full30_fp8exp(batch: int) -> Workload:
+    """Same model with FP8 E4M3 expert weights, prompt 4096, the given batch."""
+    return FULL30_BF16.with_(name=f"full30-fp8exp-b{batch}", dtype="bf16_fp8exp",
+                             batch=batch, prompt_len=4096)
+
+
+WORKLOADS = {w.name: w for w in (TINY_F32, LAYER1_BF16, FULL30_BF16, FULL30_B8_P8192)}
+for _b in (1, 4, 16, 32, 64):
+    WORKLOADS[f"full30-fp8exp-b{_b}"] = full30_fp8exp(_b)
+
+
+def get(name: str) -> Workload:
+    return WORKLOADS[name]

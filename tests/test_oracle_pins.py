@@ -1,0 +1,389 @@
+"""Pins of the oracle against what the pages and the mathematics fix.
+
+Each test checks one oracle function against something other than itself: a
+closed form, a brute-force loop, a special case that reduces to a library
+routine the oracle does not call, an invariant, or values the pages print.
+"""
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import scipy.special
+import scipy.stats
+
+from oracle import absorbing, model, sampler
+from synth import gen, workloads
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+rng = np.random.default_rng(1234)
+
+
+# --------------------------------------------------------------- attention
+def brute_attention(q, k, v, allowed):
+    nq, Hq, h = q.shape
+    Hkv = k.shape[1]
+    out = np.zeros_like(q)
+    for i in range(nq):
+        for j in range(Hq):
+            kv = j // (Hq // Hkv)
+            keys = [t for t in range(k.shape[0]) if allowed[i, t]]
+            sc = [sum(q[i, j, c] * k[t, kv, c] for c in range(h)) / math.sqrt(h) for t in keys]
+            mx = max(sc)
+            ex = [math.exp(s - mx) for s in sc]
+            z = sum(ex)
+            for c in range(h):
+                out[i, j, c] = sum(e * v[t, kv, c] for e, t in zip(ex, keys)) / z
+    return out
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(4, 2), (2, 2), (4, 1)])
+def test_attention_matches_bruteforce(Hq, Hkv):
+    nq, nk, h = 5, 7, 4
+    q = rng.normal(size=(nq, Hq, h))
+    k = rng.normal(size=(nk, Hkv, h))
+    v = rng.normal(size=(nk, Hkv, h))
+    allowed = rng.random((nq, nk)) < 0.6
+    allowed[:, 0] = True
+    np.testing.assert_allclose(model.attention(q, k, v, allowed),
+                               brute_attention(q, k, v, allowed), rtol=1e-12, atol=1e-12)
+
+
+def test_attention_special_cases():
+    q = rng.normal(size=(3, 2, 4))
+    k = np.tile(rng.normal(size=(1, 1, 4)), (6, 1, 1))     # all keys equal
+    v = rng.normal(size=(6, 1, 4))
+    out = model.attention(q, k, v, np.ones((3, 6), bool))
+    np.testing.assert_allclose(out, np.broadcast_to(v.mean(axis=0), out.shape), atol=1e-14)
+    allowed = np.zeros((3, 6), bool)
+    allowed[:, 4] = True                                     # a single key
+    out = model.attention(q, rng.normal(size=(6, 1, 4)), v, allowed)
+    np.testing.assert_allclose(out, np.broadcast_to(v[4], out.shape), atol=1e-14)
+
+
+# --------------------------------------------------------------- RoPE
+def test_rope_identity_norm_relative():
+    h, base = 16, 10000.0
+    x = rng.normal(size=(1, 3, h))
+    np.testing.assert_allclose(model.rope(x, np.array([0]), base), x, atol=0)
+    pos = np.array([5, 37, 1000])
+    y = model.rope(np.repeat(x, 3, 0), pos, base)
+    # every rotated pair keeps its length
+    half = h // 2
+    n0 = x[..., :half] ** 2 + x[..., half:] ** 2
+    n1 = y[..., :half] ** 2 + y[..., half:] ** 2
+    np.testing.assert_allclose(n1, np.broadcast_to(n0, n1.shape), rtol=1e-12)
+    # q(m) . k(n) depends on m - n only
+    q, k = rng.normal(size=(1, 1, h)), rng.normal(size=(1, 1, h))
+    for m, n, d in [(3, 1, 10), (100, 7, 250)]:
+        a = (model.rope(q, np.array([m]), base) * model.rope(k, np.array([n]), base)).sum()
+        b = (model.rope(q, np.array([m + d]), base) * model.rope(k, np.array([n + d]), base)).sum()
+        assert abs(a - b) < 1e-9
+
+
+def test_rope_pair_frequencies():
+    """Unit vector on pair i at position p ends up at angle p * base^(-2i/h)."""
+    h, base, p = 8, 10000.0, 3
+    for i in range(h // 2):
+        e = np.zeros((1, 1, h))
+        e[0, 0, i] = 1.0
+        y = model.rope(e, np.array([p]), base)[0, 0]
+        ang = math.atan2(y[i + h // 2], y[i])
+        want = math.remainder(p * base ** (-2 * i / h), 2 * math.pi)
+        assert abs(math.remainder(ang - want, 2 * math.pi)) < 1e-12
+        others = [c for c in range(h) if c not in (i, i + h // 2)]
+        assert np.all(y[others] == 0)
+
+
+# --------------------------------------------------------------- RMSNorm
+def test_rmsnorm_closed_form():
+    x = rng.normal(size=(4, 64)) * 3.0
+    eps = 1e-6
+    y = model.rmsnorm(x, eps)
+    ms = (x * x).mean(axis=1)
+    np.testing.assert_allclose((y * y).mean(axis=1), ms / (ms + eps), rtol=1e-12)
+    assert np.all(np.sign(y) == np.sign(x))
+
+
+# --------------------------------------------------------------- timestep embedding
+def test_timestep_embedding_pins():
+    d = 64
+    e = model.timestep_embedding(math.pi / 2000.0, d)     # 1000*tau*w_0 = pi/2
+    assert abs(e[0] - 1.0) < 1e-15 and abs(e[d // 2]) < 1e-15
+    for tau in (0.25, 1.0):
+        e = model.timestep_embedding(tau, d)
+        np.testing.assert_allclose(e[:d // 2] ** 2 + e[d // 2:] ** 2, 1.0, rtol=1e-14)
+        # the slowest pair turns at 1000*tau*10000^(-(d/2-1)/(d/2))
+        w_last = 10000.0 ** (-(d // 2 - 1) / (d // 2))
+        assert abs(math.atan2(e[d // 2 - 1], e[-1]) - 1000 * tau * w_last) < 1e-12
+
+
+# --------------------------------------------------------------- MoE
+class _FakeLayer:
+    def __init__(self, E, d, I, Is, w):
+        self.w = w
+        self.router = rng.normal(size=(E, d))
+        self.experts = [(rng.normal(size=(I, d)) * 0.3, rng.normal(size=(I, d)) * 0.3,
+                         rng.normal(size=(d, I)) * 0.3) for _ in range(E)]
+        self.sgate, self.sup = rng.normal(size=(Is, d)) * 0.3, rng.normal(size=(Is, d)) * 0.3
+        self.sdown = rng.normal(size=(d, Is)) * 0.3
+
+    def expert(self, e):
+        return self.experts[e]
+
+
+def _dense_moe(u, L, top_k):
+    """All experts evaluated for every row; non-selected gates are zero."""
+    n, E = u.shape[0], len(L.experts)
+    logits = u @ L.router.T
+    p = scipy.special.softmax(logits, axis=1)
+    y = np.zeros_like(u)
+    for t in range(n):
+        top = np.lexsort((np.arange(E), -p[t]))[:top_k]
+        gates = np.zeros(E)
+        gates[top] = p[t, top] / p[t, top].sum()
+        for e in range(E):
+            wg, wu, wd = L.experts[e]
+            a = u[t] @ wg.T
+            hdn = a * scipy.special.expit(a) * (u[t] @ wu.T)
+            y[t] += gates[e] * (wd @ hdn)
+        a = u[t] @ L.sgate.T
+        y[t] += L.sdown @ (a * scipy.special.expit(a) * (u[t] @ L.sup.T))
+    return y
+
+
+@pytest.mark.parametrize("E,k", [(8, 2), (6, 6), (1, 1)])
+def test_moe_topk_equals_dense(E, k):
+    d, I, Is = 12, 10, 9
+    w = workloads.TINY_F32.with_(n_experts=E, top_k=k)
+    L = _FakeLayer(E, d, I, Is, w)
+    u = rng.normal(size=(7, d))
+    y, idx, g, _ = model.moe(u, L, k)
+    np.testing.assert_allclose(y, _dense_moe(u, L, k), rtol=1e-11, atol=1e-12)
+    if k == E:   # full mixture: gates are the plain softmax
+        for t in range(7):
+            full = scipy.special.softmax(u[t] @ L.router.T)
+            np.testing.assert_allclose(g[t][np.argsort(idx[t])], full, rtol=1e-12)
+
+
+def test_router_ties_go_to_lower_expert():
+    router = np.zeros((6, 2))
+    router[[1, 3, 4]] = [1.0, 0.0]
+    idx, g, _ = model.route(np.array([[2.0, 0.0]]), router, 2)
+    assert list(idx[0]) == [1, 3]
+    np.testing.assert_allclose(g[0], [0.5, 0.5])
+
+
+# --------------------------------------------------------------- entropy / LM-head statistics
+def test_entropy_uniform_two_level_gap():
+    V = 512
+    st = model.entropy_stats(np.full((1, V), 3.25))
+    assert abs(st["H64"][0] - math.log(V)) < 1e-12
+    assert st["argmax"][0] == 0
+    # two-level logits: n_a entries at a, n_b at b
+    a, b, na = 2.0, -1.0, 5
+    lg = np.full((1, V), b)
+    lg[0, 100:100 + na] = a
+    Z = na * math.exp(a) + (V - na) * math.exp(b)
+    Hc = math.log(Z) - (a * na * math.exp(a) + b * (V - na) * math.exp(b)) / Z
+    st = model.entropy_stats(lg)
+    assert abs(st["H64"][0] - Hc) < 1e-12 and st["argmax"][0] == 100
+    # a 100-nat gap leaves essentially no uncertainty
+    lg = np.zeros((1, V))
+    lg[0, 7] = 100.0
+    st = model.entropy_stats(lg)
+    assert 0.0 <= st["H64"][0] < 1e-38 and st["argmax"][0] == 7
+
+
+def test_entropy_matches_library_and_bounds():
+    lg = rng.normal(size=(6, 300)) * 4.0
+    st = model.entropy_stats(lg)
+    want = scipy.stats.entropy(scipy.special.softmax(lg, axis=1), axis=1)
+    np.testing.assert_allclose(st["H64"], want, rtol=1e-12)
+    assert np.all(st["H64"] >= 0) and np.all(st["H64"] <= math.log(300) + 1e-12)
+    np.testing.assert_allclose(st["lse"], scipy.special.logsumexp(lg, axis=1), rtol=1e-13)
+    assert st["H"].dtype == np.float32
+
+
+# --------------------------------------------------------------- sampler
+def _brute_sampler(H, am, canvas, mask, s, gamma):
+    """Independent restatement with exact rational prefix sums."""
+    masked = [i for i in range(len(mask)) if mask[i]]
+    m = len(masked)
+    if m == 0:
+        return list(canvas), list(mask), 0
+    keys = {i: max(float(np.float32(H[i])), 0.0) for i in masked}
+    order = sorted(masked, key=lambda i: (keys[i], i))
+    g = Fraction(float(np.float32(gamma)))
+    best = 0
+    for n in range(m + 1):
+        if sum((Fraction(keys[i]) for i in order[:n]), Fraction(0)) <= g:
+            best = n
+        else:
+            break
+    n = min(m, max(best, math.ceil(m / s)))
+    c2, m2 = list(canvas), list(mask)
+    for i in order[:n]:
+        c2[i], m2[i] = am[i], 0
+    return c2, m2, n
+
+
+@pytest.mark.parametrize("trial", range(40))
+def test_sampler_matches_bruteforce(trial):
+    r = np.random.default_rng(100 + trial)
+    C = int(r.integers(1, 13))
+    H = (r.random(C) * r.choice([0.05, 0.3, 2.0])).astype(np.float32)
+    if trial % 3 == 0:
+        H = np.round(H * 8).astype(np.float32) / 8           # force exact ties
+    am = r.integers(0, 50, C)
+    mask = (r.random(C) < 0.8).astype(np.uint8)
+    canvas = np.where(mask == 1, 50, r.integers(0, 50, C))
+    s = int(r.integers(1, 6))
+    gamma = float(r.choice([0.0, 0.1, 0.5, 1.0, 3.0]))
+    c, mk, n, _ = sampler.eb_step(H, am, canvas, mask, s, gamma)
+    c2, m2, n2 = _brute_sampler(H, am, canvas, mask, s, gamma)
+    assert n == n2 and list(c) == c2 and list(mk) == m2
+
+
+def test_sampler_special_cases():
+    C = 20
+    H = (np.arange(C, dtype=np.float32) + 1) / 7
+    am = np.arange(C) + 100
+    mask = np.ones(C, np.uint8)
+    canvas = np.full(C, 999)
+    for s in (1, 2, 3, 7):
+        _, _, n, _ = sampler.eb_step(H, am, canvas, mask, s, 0.0)
+        assert n == (C if s == 1 else math.ceil(C / s))        # gamma = 0 -> the minimum
+    _, mk, n, _ = sampler.eb_step(H, am, canvas, mask, 9, float("inf"))
+    assert n == C and not mk.any()
+    # equal entropies: lower positions first
+    c, mk, n, _ = sampler.eb_step(np.full(C, 0.5, np.float32), am, canvas, mask, 4, 0.0)
+    assert n == 5 and list(np.nonzero(mk == 0)[0]) == [0, 1, 2, 3, 4]
+    # nothing masked: no-op
+    c, mk, n, _ = sampler.eb_step(H, am, canvas, np.zeros(C, np.uint8), 3, 1.0)
+    assert n == 0 and list(c) == list(canvas)
+
+
+def test_block_invariants_with_synthetic_entropies():
+    C, T, V = 64, 6, 1000
+    step = {"k": 0}
+
+    def fake_forward(canvas, s):
+        step["k"] += 1
+        u = gen.uniform_u16(7, f"fake.{step['k']}", 2 * C).numpy()
+        return (u[:C] / 4096.0).astype(np.float32), u[C:] % V
+
+    canvas, traj = sampler.generate_block(fake_forward, C, V, T, 1.0)
+    prev_mask = np.ones(C, np.uint8)
+    prev_canvas = np.full(C, V)
+    for s, H, am, c, mk, n in traj:
+        assert np.all(mk <= prev_mask)                                   # never re-masked
+        kept = prev_mask == 0
+        assert np.all(c[kept] == prev_canvas[kept])                      # committed stay put
+        new = (prev_mask == 1) & (mk == 0)
+        assert np.all(c[new] == am[new])                                 # commits take argmax
+        assert mk.sum() <= C * (s - 1) // T                              # masked <= C(s-1)/T
+        order = sorted(np.nonzero(prev_mask)[0], key=lambda i: (H[i], i))
+        assert set(order[:n]) == set(np.nonzero(new)[0])                 # a sorted prefix
+        prev_mask, prev_canvas = mk, c
+    assert not (canvas == V).any() and len(traj) <= T
+
+
+# --------------------------------------------------------------- absorbing process
+def test_absorbing_example_endpoints():
+    g = json.load(open(os.path.join(GOLDEN, "absorbing_example.json")))
+    u = gen.uniform_u16(0, "absorb.example", len(g["sentence"])).numpy()
+    x0, _ = absorbing.absorb(g["sentence"], 0, g["T"], g["vocab"], u)
+    xT, _ = absorbing.absorb(g["sentence"], g["T"], g["T"], g["vocab"], u)
+    assert list(x0) == g["at_t0"] and list(xT) == g["at_tT"]
+
+
+def test_absorbing_fraction_and_monotone():
+    n, T = 200000, 10
+    u = gen.uniform_u16(3, "absorb.frac", n).numpy()
+    prev = np.zeros(n, bool)
+    for t in range(T + 1):
+        _, a = absorbing.absorb(np.zeros(n, np.int64), t, T, 99, u)
+        p = t / T
+        assert abs(a.mean() - p) <= 4 * math.sqrt(p * (1 - p) / n) + 1e-12
+        assert np.all(a >= prev)
+        prev = a
+
+
+# --------------------------------------------------------------- masks and composition
+def _tiny(**kw):
+    return model.Weights(workloads.TINY_F32.with_(**kw), keep_layers=True)
+
+
+def test_prefill_causal_and_window():
+    P = 12
+    base = np.arange(P) * 7 % 500
+    ws = _tiny()                                       # window 1024: all P rows are kept
+    kv = model.prefill(ws, base)
+    for j in (5, 9):
+        alt = base.copy()
+        alt[j] = (alt[j] + 1) % 500
+        kv2 = model.prefill(ws, alt)
+        K1, K2 = kv[1][0], kv2[1][0]                  # layer 1 keys
+        assert np.array_equal(K1[:j], K2[:j])          # causal: earlier rows unchanged
+        assert not np.allclose(K1[j:j + 2], K2[j:j + 2])
+    # window 4: the cache keeps positions 8..11; layer-1 row i depends on tokens i-3 .. i
+    ws4 = _tiny(window=4)
+    kv = model.prefill(ws4, base)
+    assert kv[1][0].shape[0] == 4
+    alt = base.copy()
+    alt[4] = (alt[4] + 1) % 500
+    assert np.array_equal(kv[1][0], model.prefill(ws4, alt)[1][0])
+    alt = base.copy()
+    alt[7] = (alt[7] + 1) % 500
+    K2 = model.prefill(ws4, alt)[1][0]
+    assert np.array_equal(kv[1][0][3], K2[3])          # position 11 is 4 away from 7
+    assert not np.allclose(kv[1][0][:3], K2[:3])
+
+
+def test_canvas_is_bidirectional():
+    ws = _tiny()
+    w = ws.w
+    prompt = np.arange(w.prompt_len) % w.vocab
+    kv = model.prefill(ws, prompt)
+    c = np.full(w.canvas, w.mask_id)
+    a = model.denoise_forward(ws, kv, c, 3, w.T, w.prompt_len)["H64"]
+    c2 = c.copy()
+    c2[20] = 5
+    b = model.denoise_forward(ws, kv, c2, 3, w.T, w.prompt_len)["H64"]
+    assert np.all(a[:20] != b[:20]) and np.all(a[21:] != b[21:])
+
+
+def test_zero_blocks_reduce_to_embedding_head():
+    """With Wo and all FFN outputs zero every layer is the identity."""
+    ws = _tiny()
+    w = ws.w
+    for l in range(w.n_layers):
+        for name, shape in [(f"l{l}.wo", (w.d_model, w.n_q_heads * w.head_dim)),
+                            (f"l{l}.sdown", (w.d_model, w.shared_inter)),
+                            (f"l{l}.down", (w.n_experts, w.d_model, w.expert_inter))]:
+            ws._cache[name] = np.zeros(shape)
+    prompt = np.arange(w.prompt_len) % w.vocab
+    kv = model.prefill(ws, prompt)
+    c = (np.arange(w.canvas) * 3) % (w.vocab + 1)
+    st = model.denoise_forward(ws, kv, c, 2, w.T, w.prompt_len, want_logits=True)
+    E = ws.get("tok_emb", (w.vocab + 1, w.d_model))
+    x = E[c] + model.timestep_embedding(2 / w.T, w.d_model)
+    xn = x / np.sqrt((x * x).mean(1, keepdims=True) + w.rms_eps)
+    want = w.logit_scale * xn @ ws.get("lm_head", (w.vocab, w.d_model)).T
+    np.testing.assert_allclose(st["logits"], want, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(st["H64"], scipy.stats.entropy(scipy.special.softmax(want, 1), axis=1),
+                               rtol=1e-11)
+
+
+# --------------------------------------------------------------- metric formulas (pages' numbers)
+def test_tps_formula_reproduces_pages():
+    from masked_discrete_diffusion_b200 import metrics
+    g = json.load(open(os.path.join(GOLDEN, "tps_h100_fp8.json")))
+    tps = metrics.tokens_per_second(g["tpf"], g["t_fwd_ms"] / 1000.0)
+    assert round(tps) == g["tps_reported"]
+    # tokens per forward counts one extra forward between consecutive canvases
+    assert metrics.tokens_per_forward([256, 256, 100], [12, 12, 5]) == 612 / (29 + 2)
+    assert metrics.effective_steps([256, 100], [12, 4]) == (256 * 12 + 100 * 4) / 356
