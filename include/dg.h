@@ -1,0 +1,195 @@
+/*
+ * dg.h — C-ABI of the masked (absorbing) discrete-diffusion denoise path.
+ *
+ * The operations follow the problem statement of "DiffusionGemma 技术报告"
+ * (full translation page):
+ *   - §3.1 "块自回归生成", KV-cache initialisation: the context is encoded once
+ *     by a causal pass, H = Encoder(h), and its keys/values are kept
+ *     (dg_prefill);
+ *   - §3.1 / §3.2 "推理时的去噪框架": a 256-token canvas is denoised by a decoder
+ *     that attends bidirectionally inside the canvas and to the KV cache, and
+ *     produces logits per canvas position (dg_denoise_step, without ever writing
+ *     the logits);
+ *   - §3.3 "DiffusionGemma 采样器", entropy-bounded refinement: positions are
+ *     accepted in ascending order of entropy (dg_eb_sample, also run inside
+ *     dg_denoise_step);
+ *   - §3.1: one canvas is denoised to completion before it is committed
+ *     (dg_generate_block).
+ * Architecture numbers (30 layers, sliding window 1024, 256-token canvas, 262K
+ * vocabulary, 128 experts top-8 plus a shared expert, timestep embedding) come
+ * from the explainer page "DiffusionGemma 深度解析", list "核心架构参数".
+ *
+ * Conventions
+ *   - Every data pointer is a DEVICE pointer owned by the caller unless stated.
+ *     Handles (dg_model, dg_kv) are owned by the library and released with their
+ *     destroy call.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Calls enqueue work and return without synchronising, except where noted.
+ *   - Every call returns a dg_status; nothing is thrown across the ABI and
+ *     nothing aborts.  Arguments are validated before any launch.  Errors of
+ *     kernels already enqueued surface on a later call or on dg_sync_status.
+ *   - Row-major layouts; [a, b] means a rows of b contiguous elements.
+ *   - Model dimensions: d = d_model, Hq / Hkv query / key-value heads of size h,
+ *     E experts with top_k routing and intermediate I, shared expert
+ *     intermediate Is, vocabulary V (the [MASK] id is V), canvas C, window Wn.
+ *     For a prefilled prompt of length P the cached window is W = min(P, Wn).
+ */
+#ifndef DG_H
+#define DG_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum dg_status {
+  DG_OK = 0,
+  DG_ERR_INVALID_ARG = 1, /* a null pointer, a size out of range, a bad value */
+  DG_ERR_UNSUPPORTED = 2, /* a valid request this build does not implement    */
+  DG_ERR_OOM = 3,         /* device allocation failed                          */
+  DG_ERR_CUDA = 4,        /* a CUDA runtime/driver error (message kept)         */
+  DG_ERR_TIMEOUT = 5,     /* a bounded device-side wait gave up                 */
+  DG_ERR_INTERNAL = 6
+} dg_status;
+
+typedef enum dg_dtype {
+  DG_F32 = 0,        /* fp32 weights; the SIMT path carries activations in fp64 */
+  DG_BF16 = 1,       /* bf16 weights and activations, fp32 accumulation          */
+  DG_BF16_FP8EXP = 2 /* as DG_BF16 but routed-expert weights in FP8 E4M3         */
+} dg_dtype;
+
+typedef struct dg_config {
+  int32_t n_layers, d_model, n_q_heads, n_kv_heads, head_dim;
+  int32_t n_experts, top_k, expert_inter, shared_inter;
+  int32_t vocab;       /* V; the [MASK] token id is V                       */
+  int32_t window;      /* sliding window Wn of the causal prompt pass        */
+  int32_t canvas;      /* C                                                   */
+  float rope_base;     /* rotary base (pairs (i, i + h/2), angle p*base^(-2i/h)) */
+  float rms_eps;
+  float logit_scale;   /* logits = logit_scale * RMSNorm(x) W_lm^T          */
+  int32_t dtype;       /* dg_dtype                                            */
+  int32_t max_batch;   /* largest B any call on this model will pass          */
+  int32_t max_prompt;  /* largest P any dg_prefill on this model will pass    */
+} dg_config;
+
+/* Weights of one layer (device pointers, borrowed for the model's lifetime).
+ * Element type: fp32 for DG_F32, bf16 otherwise; for DG_BF16_FP8EXP the three
+ * routed-expert tensors are FP8 E4M3 bytes with fp32 scales, one per
+ * (row, 128 consecutive input columns): w = q * scale.                       */
+typedef struct dg_layer_weights {
+  const void* wqkv;   /* [(Hq + 2 Hkv) h, d]: query heads, key heads, value heads */
+  const void* wo;     /* [d, Hq h]                                                */
+  const void* router; /* [E, d]                                                   */
+  const void* gate;   /* [E, I, d]                                                */
+  const void* up;     /* [E, I, d]                                                */
+  const void* down;   /* [E, d, I]                                                */
+  const float* gate_scale; /* [E, I, d/128]  FP8 only, else NULL                  */
+  const float* up_scale;   /* [E, I, d/128]                                       */
+  const float* down_scale; /* [E, d, I/128]                                       */
+  const void* sgate;  /* [Is, d]                                                  */
+  const void* sup;    /* [Is, d]                                                  */
+  const void* sdown;  /* [d, Is]                                                  */
+} dg_layer_weights;
+
+typedef struct dg_weights {
+  const void* tok_emb;            /* [V + 1, d]; row V embeds [MASK]           */
+  const void* lm_head;            /* [V, d] (untied)                           */
+  const dg_layer_weights* layers; /* HOST array of n_layers entries, copied    */
+} dg_weights;
+
+typedef struct dg_model dg_model;
+typedef struct dg_kv dg_kv;
+
+/* Human-readable name of a status code (static storage). */
+const char* dg_status_str(dg_status s);
+
+/* Detail of the last error raised on the calling thread ("" if none). */
+const char* dg_last_error(void);
+
+/* Validates the configuration and weight pointers, plans the kernels and
+ * allocates the library's device workspace for max_batch canvases and prompts
+ * up to max_prompt tokens, on the current CUDA device.  Synchronous.
+ * Errors: DG_ERR_INVALID_ARG (null, non-positive or inconsistent sizes, C > 1024,
+ * Hq not a multiple of Hkv, h odd), DG_ERR_UNSUPPORTED (a shape the tensor-core
+ * kernels do not tile), DG_ERR_OOM, DG_ERR_CUDA. */
+dg_status dg_model_create(const dg_config* cfg, const dg_weights* w, dg_model** out);
+
+/* Synchronises the device and frees the model's workspace. NULL is a no-op. */
+dg_status dg_model_destroy(dg_model* m);
+
+/* Waits for the model's queued work and reports asynchronous failures: a CUDA
+ * error (DG_ERR_CUDA) or a device-side bounded wait that gave up
+ * (DG_ERR_TIMEOUT; the flag is cleared by this call). */
+dg_status dg_sync_status(dg_model* m, void* stream);
+
+/* Causal encoder pass over B prompts of P tokens (prompt: [B, P] int32 ids in
+ * [0, V)).  Rows attend to keys j with i - Wn < j <= i; no timestep embedding.
+ * The post-RoPE keys and the values of the last W = min(P, Wn) positions of every
+ * layer are kept in a new library-owned handle *out:
+ *   K, V: [n_layers, B, Hkv, W, h] (bf16; fp64 for DG_F32).
+ * Requires 1 <= B <= max_batch, 1 <= P <= max_prompt.  Ids are checked on the
+ * device; an id outside [0, V) yields DG_ERR_INVALID_ARG on the next status read. */
+dg_status dg_prefill(dg_model* m, const int32_t* prompt, int32_t B, int32_t P,
+                     dg_kv** out, void* stream);
+
+/* Frees a KV handle (after synchronising its stream). NULL is a no-op. */
+dg_status dg_kv_destroy(dg_kv* kv);
+
+/* Batch size, prompt length and window of a KV handle (host values). */
+dg_status dg_kv_info(const dg_kv* kv, int32_t* B, int32_t* P, int32_t* W);
+
+/* One denoise forward plus one Entropy-Bound sampler step on B = kv's batch
+ * canvases (canvas: [B, C] int32 ids in [0, V], V = [MASK]; mask: [B, C] uint8,
+ * 1 = still masked; both updated in place).
+ * The forward embeds the canvas, adds the sinusoidal embedding of
+ * tau = steps_left / T, runs the layers (queries at absolute positions P..P+C-1,
+ * keys = the cached window followed by all C canvas rows, one softmax) and the
+ * LM head, and writes per position the softmax entropy in nats (entropy: [B, C]
+ * fp32, clamped at 0) and the argmax id (argmax: [B, C] int32, lowest id on
+ * ties).  The logits are never stored.  The sampler then commits, per canvas, the
+ * n = min(m, max(k_gamma, ceil(m / steps_left))) masked positions of lowest
+ * (entropy, position), where m is the number masked and k_gamma the longest
+ * prefix whose entropies sum to <= gamma (sums in 2^-48 fixed point); committed
+ * positions take their argmax and are unmasked.  n_committed: [B] int32.
+ * A canvas with m = 0 is left unchanged (n = 0).
+ * Requires 1 <= steps_left <= T, gamma >= 0 (not NaN). */
+dg_status dg_denoise_step(dg_model* m, const dg_kv* kv, int32_t* canvas, uint8_t* mask,
+                          int32_t steps_left, int32_t T, float gamma,
+                          float* entropy, int32_t* argmax, int32_t* n_committed,
+                          void* stream);
+
+/* Denoises B = kv's batch canvases from all [MASK] with T forwards
+ * (steps_left = T, T-1, ..., 1), without synchronising the host between steps.
+ * canvas_out: [B, C] int32 (no [MASK] remains); n_forwards: [B] int32, the
+ * number of forwards after which that canvas had no [MASK] left (nullable);
+ * router_load: [n_layers, E] int32 counts of (token, expert) routings summed
+ * over the block (nullable).  Requires T >= 1, gamma >= 0. */
+dg_status dg_generate_block(dg_model* m, const dg_kv* kv, int32_t T, float gamma,
+                            int32_t* canvas_out, int32_t* n_forwards,
+                            int32_t* router_load, void* stream);
+
+/* The sampler step alone, on caller-provided statistics: entropy [B, C] fp32,
+ * argmax [B, C] int32, canvas/mask [B, C] updated in place, n_committed [B].
+ * Same rule as in dg_denoise_step (a NaN entropy sorts as +inf, a negative one
+ * as 0).  Requires 1 <= C <= 1024, 1 <= steps_left, gamma >= 0. */
+dg_status dg_eb_sample(const float* entropy, const int32_t* argmax, int32_t* canvas,
+                       uint8_t* mask, int32_t B, int32_t C, int32_t steps_left,
+                       float gamma, int32_t* n_committed, void* stream);
+
+/* Test hook: the forward of dg_denoise_step without the sampler.  Writes
+ * entropy/argmax as above and, when non-NULL, the logits [B*C, V] fp32 and the
+ * final residual stream [B*C, d] fp32 (before the final norm). */
+dg_status dg_debug_forward(dg_model* m, const dg_kv* kv, const int32_t* canvas,
+                           int32_t steps_left, int32_t T, float* entropy,
+                           int32_t* argmax, float* logits, float* hidden, void* stream);
+
+/* Copies a KV handle's cached keys and values into caller buffers
+ * (k, v: [n_layers, B, Hkv, W, h] of the cache's element type). */
+dg_status dg_kv_read(const dg_kv* kv, void* k, void* v, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DG_H */

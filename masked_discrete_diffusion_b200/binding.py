@@ -1,0 +1,244 @@
+"""ctypes binding of libdg (include/dg.h): argument marshalling only.
+
+Every function below forwards to the C entry point of the same name; device
+buffers are passed as torch CUDA tensors (PyTorch supplies device memory and
+streams).  There is no fallback: if libdg.so is missing or a call fails, an
+exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdg.so")
+
+DG_F32, DG_BF16, DG_BF16_FP8EXP = 0, 1, 2
+_DTYPES = {"f32": DG_F32, "bf16": DG_BF16, "bf16_fp8exp": DG_BF16_FP8EXP}
+
+
+class DGError(RuntimeError):
+    def __init__(self, status: int, name: str, detail: str):
+        super().__init__(f"{name}: {detail}")
+        self.status = status
+        self.name = name
+
+
+class dg_config(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "n_layers", "d_model", "n_q_heads", "n_kv_heads", "head_dim", "n_experts", "top_k",
+        "expert_inter", "shared_inter", "vocab", "window", "canvas")] + [
+        ("rope_base", ctypes.c_float), ("rms_eps", ctypes.c_float),
+        ("logit_scale", ctypes.c_float), ("dtype", ctypes.c_int32),
+        ("max_batch", ctypes.c_int32), ("max_prompt", ctypes.c_int32)]
+
+
+_LAYER_FIELDS = ("wqkv", "wo", "router", "gate", "up", "down", "gate_scale", "up_scale",
+                 "down_scale", "sgate", "sup", "sdown")
+
+
+class dg_layer_weights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in _LAYER_FIELDS]
+
+
+class dg_weights(ctypes.Structure):
+    _fields_ = [("tok_emb", ctypes.c_void_p), ("lm_head", ctypes.c_void_p),
+                ("layers", ctypes.POINTER(dg_layer_weights))]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libdg.so (built in-tree by build.py); raise if it is absent."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libdg.so not built ({LIB_PATH}); run "
+                               "`python -m masked_discrete_diffusion_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float
+        L.dg_status_str.restype = ctypes.c_char_p
+        L.dg_status_str.argtypes = [ctypes.c_int]
+        L.dg_last_error.restype = ctypes.c_char_p
+        L.dg_last_error.argtypes = []
+        sigs = {
+            "dg_model_create": [ctypes.POINTER(dg_config), ctypes.POINTER(dg_weights),
+                                ctypes.POINTER(vp)],
+            "dg_model_destroy": [vp],
+            "dg_sync_status": [vp, vp],
+            "dg_prefill": [vp, vp, i32, i32, ctypes.POINTER(vp), vp],
+            "dg_kv_destroy": [vp],
+            "dg_kv_info": [vp, ctypes.POINTER(i32), ctypes.POINTER(i32), ctypes.POINTER(i32)],
+            "dg_kv_read": [vp, vp, vp, vp],
+            "dg_denoise_step": [vp, vp, vp, vp, i32, i32, f32, vp, vp, vp, vp],
+            "dg_generate_block": [vp, vp, i32, f32, vp, vp, vp, vp],
+            "dg_eb_sample": [vp, vp, vp, vp, i32, i32, i32, f32, vp, vp],
+            "dg_debug_forward": [vp, vp, vp, i32, i32, vp, vp, vp, vp, vp],
+        }
+        for name, args in sigs.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def exported_symbols():
+    return [n for n in ("dg_status_str", "dg_last_error", "dg_model_create", "dg_model_destroy",
+                        "dg_sync_status", "dg_prefill", "dg_kv_destroy", "dg_kv_info",
+                        "dg_kv_read", "dg_denoise_step", "dg_generate_block", "dg_eb_sample",
+                        "dg_debug_forward") if hasattr(lib(), n)]
+
+
+def _check(status: int):
+    if status != 0:
+        L = lib()
+        raise DGError(status, L.dg_status_str(status).decode(), L.dg_last_error().decode())
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return t.data_ptr()
+
+
+def _stream(stream=None) -> int | None:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream or None
+
+
+def make_config(w, max_batch: int | None = None, max_prompt: int | None = None) -> dg_config:
+    """dg_config from a workload description (any object with the workload fields)."""
+    return dg_config(
+        n_layers=w.n_layers, d_model=w.d_model, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads,
+        head_dim=w.head_dim, n_experts=w.n_experts, top_k=w.top_k, expert_inter=w.expert_inter,
+        shared_inter=w.shared_inter, vocab=w.vocab, window=w.window, canvas=w.canvas,
+        rope_base=w.rope_base, rms_eps=w.rms_eps, logit_scale=w.logit_scale,
+        dtype=_DTYPES[w.dtype], max_batch=max_batch or w.batch,
+        max_prompt=max_prompt or w.prompt_len)
+
+
+class Model:
+    """A dg_model handle; `tensors` maps weight names (see include/dg.h) to CUDA tensors
+    and must stay alive as long as the model (the library borrows them)."""
+
+    def __init__(self, cfg: dg_config, tensors: dict):
+        self.cfg = cfg
+        self.tensors = tensors
+        n = cfg.n_layers
+        self._layers = (dg_layer_weights * n)()
+        for l in range(n):
+            for f in _LAYER_FIELDS:
+                setattr(self._layers[l], f, _ptr(tensors.get(f"l{l}.{f}")))
+        self._w = dg_weights(tok_emb=_ptr(tensors["tok_emb"]), lm_head=_ptr(tensors["lm_head"]),
+                             layers=self._layers)
+        h = ctypes.c_void_p()
+        _check(lib().dg_model_create(ctypes.byref(cfg), ctypes.byref(self._w), ctypes.byref(h)))
+        self.handle = h
+
+    def close(self):
+        if getattr(self, "handle", None):
+            _check(lib().dg_model_destroy(self.handle))
+            self.handle = None
+
+    def __del__(self):  # pragma: no cover
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class KV:
+    def __init__(self, model: Model, handle):
+        self.model = model
+        self.handle = handle
+        B, P, W = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+        _check(lib().dg_kv_info(handle, ctypes.byref(B), ctypes.byref(P), ctypes.byref(W)))
+        self.B, self.P, self.W = B.value, P.value, W.value
+
+    def close(self):
+        if getattr(self, "handle", None):
+            _check(lib().dg_kv_destroy(self.handle))
+            self.handle = None
+
+    def __del__(self):  # pragma: no cover
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def dg_sync_status(model: Model, stream=None):
+    _check(lib().dg_sync_status(model.handle, _stream(stream)))
+
+
+def dg_prefill(model: Model, prompt: torch.Tensor, stream=None) -> KV:
+    assert prompt.dtype == torch.int32 and prompt.dim() == 2
+    h = ctypes.c_void_p()
+    _check(lib().dg_prefill(model.handle, _ptr(prompt), prompt.shape[0], prompt.shape[1],
+                            ctypes.byref(h), _stream(stream)))
+    return KV(model, h)
+
+
+def dg_kv_read(kv: KV, stream=None):
+    c = kv.model.cfg
+    dt = torch.float64 if c.dtype == DG_F32 else torch.bfloat16
+    shape = (c.n_layers, kv.B, c.n_kv_heads, kv.W, c.head_dim)
+    k = torch.empty(shape, dtype=dt, device="cuda")
+    v = torch.empty(shape, dtype=dt, device="cuda")
+    _check(lib().dg_kv_read(kv.handle, _ptr(k), _ptr(v), _stream(stream)))
+    return k, v
+
+
+def dg_denoise_step(model: Model, kv: KV, canvas, mask, steps_left: int, T: int, gamma: float,
+                    entropy=None, argmax=None, n_committed=None, stream=None):
+    B, C = canvas.shape
+    entropy = entropy if entropy is not None else torch.empty(B, C, dtype=torch.float32, device="cuda")
+    argmax = argmax if argmax is not None else torch.empty(B, C, dtype=torch.int32, device="cuda")
+    n_committed = (n_committed if n_committed is not None
+                   else torch.empty(B, dtype=torch.int32, device="cuda"))
+    _check(lib().dg_denoise_step(model.handle, kv.handle, _ptr(canvas), _ptr(mask), steps_left,
+                                 T, gamma, _ptr(entropy), _ptr(argmax), _ptr(n_committed),
+                                 _stream(stream)))
+    return entropy, argmax, n_committed
+
+
+def dg_generate_block(model: Model, kv: KV, T: int, gamma: float, canvas_out=None,
+                      n_forwards=None, router_load=None, stream=None):
+    c = model.cfg
+    canvas_out = (canvas_out if canvas_out is not None
+                  else torch.empty(kv.B, c.canvas, dtype=torch.int32, device="cuda"))
+    _check(lib().dg_generate_block(model.handle, kv.handle, T, gamma, _ptr(canvas_out),
+                                   _ptr(n_forwards), _ptr(router_load), _stream(stream)))
+    return canvas_out
+
+
+def dg_eb_sample(entropy, argmax, canvas, mask, steps_left: int, gamma: float,
+                 n_committed=None, stream=None):
+    B, C = entropy.shape
+    n_committed = (n_committed if n_committed is not None
+                   else torch.empty(B, dtype=torch.int32, device="cuda"))
+    _check(lib().dg_eb_sample(_ptr(entropy), _ptr(argmax), _ptr(canvas), _ptr(mask), B, C,
+                              steps_left, gamma, _ptr(n_committed), _stream(stream)))
+    return n_committed
+
+
+def dg_debug_forward(model: Model, kv: KV, canvas, steps_left: int, T: int, logits=False,
+                     hidden=False, stream=None):
+    c = model.cfg
+    B, C = canvas.shape
+    n = B * C
+    ent = torch.empty(B, C, dtype=torch.float32, device="cuda")
+    am = torch.empty(B, C, dtype=torch.int32, device="cuda")
+    lg = torch.empty(n, c.vocab, dtype=torch.float32, device="cuda") if logits else None
+    hd = torch.empty(n, c.d_model, dtype=torch.float32, device="cuda") if hidden else None
+    _check(lib().dg_debug_forward(model.handle, kv.handle, _ptr(canvas), steps_left, T,
+                                  _ptr(ent), _ptr(am), _ptr(lg), _ptr(hd), _stream(stream)))
+    return ent, am, lg, hd

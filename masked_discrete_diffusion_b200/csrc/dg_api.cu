@@ -1,0 +1,616 @@
+// libdg: host side of the C-ABI (include/dg.h) — validation, workspace, and
+// the launch sequence of the causal prompt pass and the canvas denoise forward.
+//
+// Launch sequence of one canvas forward (batch B, canvas C, prompt window W):
+//   embed + timestep  ->  per layer { RMSNorm -> QKV GEMM -> RoPE/scatter ->
+//   attention over [window | canvas] -> O GEMM (+residual) -> RMSNorm ->
+//   router -> permute -> grouped gate/up GEMM (SwiGLU) -> grouped down GEMM
+//   (x gate) -> shared expert -> combine (+residual) }  ->  RMSNorm -> LM-head
+//   statistics -> merge  ->  EB sampler.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "dg_internal.h"
+#include "k_sampler.cuh"
+#include "k_simt.cuh"
+#include "k_tc_gemm.cuh"
+
+namespace dg {
+
+static thread_local std::string g_err;
+
+void set_error(const char* fmt, ...) {
+  char buf[1024];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+}
+
+static dg_status check_launch(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_error("%s: %s", what, cudaGetErrorString(e));
+    return DG_ERR_CUDA;
+  }
+  return DG_OK;
+}
+
+// ---------------------------------------------------------------------------
+// precision paths
+// ---------------------------------------------------------------------------
+struct PathTiny {  // fp32 weights, fp64 activations and sums
+  typedef float TW;
+  typedef double TA, Acc, TR, TKV;
+  static constexpr bool kTensorCores = false;
+};
+struct PathBF16 {  // bf16 weights/activations, fp32 residual and sums
+  typedef bf16 TW, TA, TKV;
+  typedef float Acc, TR;
+  static constexpr bool kTensorCores = false;
+};
+
+static int ceil_div(long a, long b) { return (int)((a + b - 1) / b); }
+
+template <class T> static dg_status ws_alloc(Workspace& ws, T** p, size_t n) {
+  void* q = nullptr;
+  const size_t bytes = std::max<size_t>(n, 1) * sizeof(T);
+  cudaError_t e = cudaMalloc(&q, bytes);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    set_error("workspace allocation of %zu bytes failed: %s", bytes, cudaGetErrorString(e));
+    return DG_ERR_OOM;
+  }
+  ws.bufs.push_back({q, bytes});
+  *p = static_cast<T*>(q);
+  return DG_OK;
+}
+template <class T> static dg_status ws_alloc_v(Workspace& ws, void** p, size_t n) {
+  T* q = nullptr;
+  DG_TRY(ws_alloc(ws, &q, n));
+  *p = q;
+  return DG_OK;
+}
+
+static void ws_free(Workspace& ws) {
+  for (auto& b : ws.bufs) cudaFree(b.p);
+  ws.bufs.clear();
+}
+
+__global__ void rope_table_kernel(double base, int h, int max_pos, void* out, int as_double) {
+  const int half = h / 2;
+  const long n = (long)max_pos * half;
+  for (long e = blockIdx.x * (long)blockDim.x + threadIdx.x; e < n;
+       e += (long)gridDim.x * blockDim.x) {
+    const int pos = (int)(e / half), j = (int)(e % half);
+    const double theta = pow(base, -2.0 * (double)j / (double)h);
+    const double a = (double)pos * theta;
+    const double c = cos(a), s = sin(a);
+    if (as_double) {
+      ((double*)out)[e] = c;
+      ((double*)out)[n + e] = s;
+    } else {
+      ((float*)out)[e] = (float)c;
+      ((float*)out)[n + e] = (float)s;
+    }
+  }
+}
+
+template <class Path> static dg_status alloc_workspace(dg_model* m) {
+  typedef typename Path::TA TA;
+  typedef typename Path::Acc Acc;
+  typedef typename Path::TR TR;
+  typedef typename Path::TKV TKV;
+  const dg_config& c = m->cfg;
+  Workspace& ws = m->ws;
+  const size_t d = c.d_model, h = c.head_dim;
+  const size_t T = std::max<size_t>((size_t)c.max_batch * c.canvas, (size_t)c.max_prompt);
+  const size_t R = T * c.top_k;
+  ws.max_tok = T;
+  ws.max_rows = R;
+  ws.max_tiles = ceil_div((long)R, SG_BM) + c.n_experts + 1;
+  ws.n_vtiles = ceil_div(c.vocab, SG_BN);
+  ws.max_pos = c.max_prompt + c.canvas;
+  const size_t qkv = (size_t)(c.n_q_heads + 2 * c.n_kv_heads) * h;
+  DG_TRY(ws_alloc_v<TR>(ws, &ws.x, T * d));
+  DG_TRY(ws_alloc_v<TA>(ws, &ws.xn, T * d));
+  DG_TRY(ws_alloc_v<Acc>(ws, &ws.qkv, T * qkv));
+  DG_TRY(ws_alloc_v<TA>(ws, &ws.q, T * c.n_q_heads * h));
+  DG_TRY(ws_alloc_v<TA>(ws, &ws.o, T * c.n_q_heads * h));
+  DG_TRY(ws_alloc_v<TKV>(ws, &ws.kc, T * c.n_kv_heads * h));
+  DG_TRY(ws_alloc_v<TKV>(ws, &ws.vc, T * c.n_kv_heads * h));
+  DG_TRY(ws_alloc_v<Acc>(ws, &ws.ys, T * d));
+  DG_TRY(ws_alloc_v<TA>(ws, &ws.sh, T * c.shared_inter));
+  DG_TRY(ws_alloc(ws, &ws.ridx, R));
+  DG_TRY(ws_alloc(ws, &ws.rank, R));
+  DG_TRY(ws_alloc(ws, &ws.row_of, R));
+  DG_TRY(ws_alloc(ws, &ws.tok_of, R));
+  DG_TRY(ws_alloc_v<Acc>(ws, &ws.rgate, R));
+  DG_TRY(ws_alloc_v<Acc>(ws, &ws.gate_of, R));
+  DG_TRY(ws_alloc(ws, &ws.counts, c.n_experts));
+  DG_TRY(ws_alloc(ws, &ws.offsets, c.n_experts + 1));
+  DG_TRY(ws_alloc(ws, &ws.tile_e, ws.max_tiles));
+  DG_TRY(ws_alloc(ws, &ws.tile_m0, ws.max_tiles));
+  DG_TRY(ws_alloc(ws, &ws.n_tiles, 1));
+  DG_TRY(ws_alloc_v<TA>(ws, &ws.up, R * d));
+  DG_TRY(ws_alloc_v<TA>(ws, &ws.hb, R * c.expert_inter));
+  DG_TRY(ws_alloc_v<Acc>(ws, &ws.yb, R * d));
+  const size_t lm_rows = (size_t)c.max_batch * c.canvas;
+  DG_TRY(ws_alloc_v<Acc>(ws, &ws.lm_part, (size_t)ws.n_vtiles * lm_rows * 4));
+  DG_TRY(ws_alloc(ws, &ws.err, 4));
+  DG_TRY(ws_alloc(ws, &ws.ids, T));
+  DG_TRY(ws_alloc_v<Acc>(ws, &ws.rope, (size_t)2 * ws.max_pos * (h / 2)));
+  DG_TRY(ws_alloc(ws, &ws.mask, lm_rows));
+  DG_TRY(ws_alloc(ws, &ws.ent, lm_rows));
+  DG_TRY(ws_alloc(ws, &ws.amax, lm_rows));
+  DG_TRY(ws_alloc(ws, &ws.ncommit, c.max_batch));
+  DG_TRY_CUDA(cudaMemset(ws.err, 0, 4 * sizeof(int32_t)));
+  rope_table_kernel<<<256, 256>>>((double)c.rope_base, (int)h, ws.max_pos, ws.rope,
+                                  sizeof(Acc) == 8 ? 1 : 0);
+  DG_TRY(check_launch("rope table"));
+  if constexpr (Path::kTensorCores) DG_TRY(tc_prepare(m));
+  DG_TRY_CUDA(cudaDeviceSynchronize());
+  return DG_OK;
+}
+
+// ---------------------------------------------------------------------------
+// GEMM dispatch: tcgen05 for bf16 dense contractions, CUDA cores otherwise
+// ---------------------------------------------------------------------------
+template <class TA, class TW, class Acc, bool G, bool D, class Epi>
+static void gemm_simt(const TA* A, int lda, const TW* W, const TW* W2, int ldw, int M, int N,
+                      int K, GroupInfo g, int grid_y, Epi epi, cudaStream_t st) {
+  dim3 grid(ceil_div(N, SG_BN), G ? grid_y : ceil_div(M, SG_BM));
+  gemm_simt_kernel<TA, TW, Acc, G, D, Epi><<<grid, 256, 0, st>>>(A, lda, W, W2, ldw, M, N, K, g, epi);
+}
+
+template <class Path> struct Runner {
+  typedef typename Path::TW TW;
+  typedef typename Path::TA TA;
+  typedef typename Path::Acc Acc;
+  typedef typename Path::TR TR;
+  typedef typename Path::TKV TKV;
+
+  dg_model* m;
+  const dg_config& c;
+  Workspace& ws;
+  cudaStream_t st;
+  Runner(dg_model* m_, cudaStream_t st_) : m(m_), c(m_->cfg), ws(m_->ws), st(st_) {}
+
+  TR* x() { return (TR*)ws.x; }
+  TA* xn() { return (TA*)ws.xn; }
+
+  void rmsnorm(int n) {
+    rmsnorm_kernel<TR, TA, Acc><<<n, 256, 0, st>>>(x(), xn(), n, c.d_model, c.rms_eps);
+  }
+
+  // y[n, N] (+)= xn W^T  with W [N, K]
+  template <class Epi> void dense(const TA* A, int lda, const void* W, int N, int K, int n,
+                                  Epi epi) {
+    gemm_simt<TA, TW, Acc, false, false>(A, lda, (const TW*)W, nullptr, K, n, N, K, GroupInfo(),
+                                         0, epi, st);
+  }
+
+  // One decoder layer on n tokens = B_ * n_seq rows at positions pos0 + i.
+  dg_status layer(int l, int n, int B_, int n_seq, int pos0, const TKV* kA, const TKV* vA,
+                  int nA, int kposA, bool causal, int32_t* load) {
+    const dg_layer_weights& L = m->layers[l];
+    const int d = c.d_model, h = c.head_dim, Hq = c.n_q_heads, Hkv = c.n_kv_heads;
+    const int qkv_n = (Hq + 2 * Hkv) * h;
+    rmsnorm(n);
+    if constexpr (Path::kTensorCores)
+      DG_TRY(tc_gemm_store_f32(m, xn(), L.wqkv, (float*)ws.qkv, n, qkv_n, d, st));
+    else
+      dense(xn(), d, L.wqkv, qkv_n, d, n, EpiStore<Acc, Acc>{(Acc*)ws.qkv, qkv_n});
+    rope_scatter_kernel<Acc, TA, TKV><<<n, 128, 0, st>>>(
+        (const Acc*)ws.qkv, (TA*)ws.q, (TKV*)ws.kc, (TKV*)ws.vc, n, n_seq, pos0, Hq, Hkv, h,
+        (const Acc*)ws.rope, ws.max_pos);
+    {
+      const long warps = (long)n * Hq;
+      const int blocks = ceil_div(warps, 4);
+      const TKV* kB = (const TKV*)ws.kc;
+      const TKV* vB = (const TKV*)ws.vc;
+#define DG_ATTN(DPL)                                                                         \
+  attention_simt_kernel<TA, TKV, Acc, DPL><<<blocks, 128, 0, st>>>(                          \
+      (const TA*)ws.q, (TA*)ws.o, kA, vA, nA, kposA, kB, vB, n_seq, pos0, B_, n_seq, pos0, Hq, \
+      Hkv, h, causal ? 1 : 0, c.window)
+      if (h <= 32) DG_ATTN(1);
+      else if (h <= 64) DG_ATTN(2);
+      else if (h <= 96) DG_ATTN(3);
+      else DG_ATTN(4);
+#undef DG_ATTN
+    }
+    if constexpr (Path::kTensorCores)
+      DG_TRY(tc_gemm_add_residual(m, (const TA*)ws.o, L.wo, (float*)x(), n, d, Hq * h, st));
+    else
+      dense((const TA*)ws.o, Hq * h, L.wo, d, Hq * h, n, EpiAddResidual<TR, Acc>{x(), d});
+    DG_TRY(moe(l, n, load));
+    return check_launch("decoder layer");
+  }
+
+  dg_status moe(int l, int n, int32_t* load) {
+    const dg_layer_weights& L = m->layers[l];
+    const int d = c.d_model, E = c.n_experts, k = c.top_k, I = c.expert_inter;
+    const int Is = c.shared_inter;
+    const int n_ent = n * k;
+    router_kernel<TR, TW, Acc><<<n, 256, E * sizeof(Acc), st>>>(
+        x(), (const TW*)L.router, n, d, E, k, c.rms_eps, ws.ridx, (Acc*)ws.rgate, load);
+    moe_rank_kernel<<<E, 256, 0, st>>>(ws.ridx, n_ent, ws.rank, ws.counts);
+    int bm = SG_BM;
+    if constexpr (Path::kTensorCores) bm = tc_group_rows();
+    moe_offsets_kernel<<<1, 32, 0, st>>>(ws.counts, E, bm, ws.offsets, ws.tile_e, ws.tile_m0,
+                                         ws.n_tiles, ws.max_tiles);
+    moe_scatter_kernel<Acc><<<ceil_div(n_ent, 256), 256, 0, st>>>(
+        ws.ridx, (const Acc*)ws.rgate, ws.rank, ws.offsets, n_ent, k, ws.row_of, ws.tok_of,
+        (Acc*)ws.gate_of);
+    rmsnorm(n);  // u = RMSNorm(x) after attention
+    gather_rows_kernel<TA><<<n_ent, 256, 0, st>>>(xn(), ws.tok_of, ws.offsets + E, d,
+                                                  (TA*)ws.up);
+    const int grid_y = ceil_div(n_ent, bm) + E;
+    if constexpr (Path::kTensorCores) {
+      DG_TRY(tc_moe_gate_up(m, l, (const TA*)ws.up, (TA*)ws.hb, grid_y, st));
+      DG_TRY(tc_moe_down(m, l, (const TA*)ws.hb, (float*)ws.yb, grid_y, st));
+      DG_TRY(tc_gemm_swiglu(m, xn(), L.sgate, L.sup, (TA*)ws.sh, n, Is, d, st));
+      DG_TRY(tc_gemm_store_f32(m, (const TA*)ws.sh, L.sdown, (float*)ws.ys, n, d, Is, st));
+    } else {
+      GroupInfo g;
+      g.tile_e = ws.tile_e;
+      g.tile_m0 = ws.tile_m0;
+      g.n_tiles = ws.n_tiles;
+      g.offsets = ws.offsets;
+      g.w_slab = (size_t)I * d;
+      gemm_simt<TA, TW, Acc, true, true>((const TA*)ws.up, d, (const TW*)L.gate,
+                                         (const TW*)L.up, d, n_ent, I, d, g, grid_y,
+                                         EpiSwiglu<TA, Acc>{(TA*)ws.hb, I}, st);
+      gemm_simt<TA, TW, Acc, true, false>(
+          (const TA*)ws.hb, I, (const TW*)L.down, nullptr, I, n_ent, d, I, g, grid_y,
+          EpiRowScale<Acc, Acc>{(Acc*)ws.yb, d, (const Acc*)ws.gate_of}, st);
+      gemm_simt<TA, TW, Acc, false, true>(xn(), d, (const TW*)L.sgate, (const TW*)L.sup, d, n,
+                                          Is, d, GroupInfo(), 0,
+                                          EpiSwiglu<TA, Acc>{(TA*)ws.sh, Is}, st);
+      dense((const TA*)ws.sh, Is, L.sdown, d, Is, n, EpiStore<Acc, Acc>{(Acc*)ws.ys, d});
+    }
+    moe_combine_kernel<TR, Acc, Acc><<<n, 256, 0, st>>>(x(), (const Acc*)ws.ys,
+                                                        (const Acc*)ws.yb, ws.row_of, n, d, k);
+    return check_launch("moe");
+  }
+
+  // Prompt pass for each batch element, keeping the last W keys/values per layer.
+  dg_status prefill(const int32_t* prompt, int B, int P, dg_kv* kv) {
+    const int d = c.d_model, h = c.head_dim, Hkv = c.n_kv_heads;
+    const int W = kv->W;
+    for (int b = 0; b < B; ++b) {
+      embed_kernel<TW, TR><<<P, 256, 0, st>>>(prompt + (size_t)b * P, (const TW*)m->w.tok_emb,
+                                             x(), P, d, c.vocab - 1, -1.0, ws.err);
+      for (int l = 0; l < c.n_layers; ++l) {
+        DG_TRY(layer(l, P, 1, P, 0, nullptr, nullptr, 0, 0, true, nullptr));
+        // keys/values of positions P-W .. P-1 -> cache [l, b, hkv, W, h]
+        const size_t es = sizeof(TKV);
+        for (int which = 0; which < 2; ++which) {
+          const char* src = (const char*)(which ? ws.vc : ws.kc) + (size_t)(P - W) * h * es;
+          char* dst = (char*)(which ? kv->v : kv->k) +
+                      (((size_t)l * kv->B + b) * Hkv) * (size_t)W * h * es;
+          DG_TRY_CUDA(cudaMemcpy2DAsync(dst, (size_t)W * h * es, src, (size_t)P * h * es,
+                                        (size_t)W * h * es, Hkv, cudaMemcpyDeviceToDevice, st));
+        }
+      }
+    }
+    return check_launch("prefill");
+  }
+
+  // Canvas forward: statistics into ent/amax; optional logits/hidden (test hook).
+  dg_status forward(const dg_kv* kv, const int32_t* canvas, int s, int T, float* ent,
+                    int32_t* amax, float* logits, float* hidden, int32_t* load) {
+    const int B = kv->B, C = c.canvas, n = B * C, d = c.d_model;
+    const double tau = (double)s / (double)T;
+    embed_kernel<TW, TR><<<n, 256, 0, st>>>(canvas, (const TW*)m->w.tok_emb, x(), n, d, c.vocab,
+                                           tau, ws.err);
+    const size_t lstride = (size_t)B * c.n_kv_heads * kv->W * c.head_dim;
+    for (int l = 0; l < c.n_layers; ++l) {
+      const TKV* kA = (const TKV*)kv->k + l * lstride;
+      const TKV* vA = (const TKV*)kv->v + l * lstride;
+      DG_TRY(layer(l, n, B, C, kv->P, kA, vA, kv->W, kv->P - kv->W, false,
+                   load ? load + (size_t)l * c.n_experts : nullptr));
+    }
+    if (hidden) to_f32_kernel<TR><<<ceil_div((long)n * d, 256), 256, 0, st>>>(x(), hidden, (long)n * d);
+    rmsnorm(n);
+    bool done = false;
+    if constexpr (Path::kTensorCores) {
+      if (logits == nullptr) {
+        DG_TRY(tc_lmhead_stats(m, xn(), n, ent, amax, st));
+        done = true;
+      }
+    }
+    if (!done) {
+      dim3 grid(ws.n_vtiles, ceil_div(n, SG_BM));
+      lmhead_simt_kernel<TA, TW, Acc><<<grid, 256, 0, st>>>(xn(), (const TW*)m->w.lm_head, n,
+                                                           c.vocab, d, c.logit_scale,
+                                                           (Acc*)ws.lm_part, logits);
+      lm_merge_kernel<Acc><<<ceil_div(n, 4), 128, 0, st>>>((const Acc*)ws.lm_part, ws.n_vtiles,
+                                                          n, ent, amax);
+    }
+    return check_launch("forward");
+  }
+};
+
+}  // namespace dg
+
+using namespace dg;
+
+// ---------------------------------------------------------------------------
+// sampler launch (shared by dg_eb_sample, dg_denoise_step, dg_generate_block)
+// ---------------------------------------------------------------------------
+static dg_status gamma_fixed(float gamma, long long* out) {
+  DG_REQUIRE(!std::isnan(gamma) && gamma >= 0.0f, "gamma must be >= 0 and not NaN (got %g)",
+             (double)gamma);
+  const long long cap = 1LL << 62;
+  if (std::isinf(gamma)) {
+    *out = cap;
+    return DG_OK;
+  }
+  const double v = (double)gamma * 281474976710656.0;
+  *out = v >= (double)cap ? cap : (long long)std::floor(v);
+  return DG_OK;
+}
+
+static dg_status launch_sampler(const float* H, const int32_t* am, int32_t* canvas,
+                                uint8_t* mask, int B, int C, int s, long long gq,
+                                int32_t* ncommit, int32_t* nfwd, int step_no,
+                                cudaStream_t st) {
+#define DG_SAMP(NP)                                                                       \
+  eb_sample_kernel<NP><<<B, NP, 0, st>>>(H, am, canvas, mask, C, s, gq, ncommit, nfwd, \
+                                         step_no)
+  if (C <= 32) DG_SAMP(32);
+  else if (C <= 64) DG_SAMP(64);
+  else if (C <= 128) DG_SAMP(128);
+  else if (C <= 256) DG_SAMP(256);
+  else if (C <= 512) DG_SAMP(512);
+  else DG_SAMP(1024);
+#undef DG_SAMP
+  return check_launch("eb sampler");
+}
+
+extern "C" {
+
+const char* dg_status_str(dg_status s) {
+  switch (s) {
+    case DG_OK: return "DG_OK";
+    case DG_ERR_INVALID_ARG: return "DG_ERR_INVALID_ARG";
+    case DG_ERR_UNSUPPORTED: return "DG_ERR_UNSUPPORTED";
+    case DG_ERR_OOM: return "DG_ERR_OOM";
+    case DG_ERR_CUDA: return "DG_ERR_CUDA";
+    case DG_ERR_TIMEOUT: return "DG_ERR_TIMEOUT";
+    case DG_ERR_INTERNAL: return "DG_ERR_INTERNAL";
+  }
+  return "DG_ERR_UNKNOWN";
+}
+
+const char* dg_last_error(void) { return g_err.c_str(); }
+
+dg_status dg_model_create(const dg_config* cfg, const dg_weights* w, dg_model** out) {
+  g_err.clear();
+  DG_REQUIRE(cfg && w && out, "null argument");
+  *out = nullptr;
+  const dg_config& c = *cfg;
+  DG_REQUIRE(c.n_layers >= 1 && c.d_model >= 2 && c.d_model % 2 == 0, "bad n_layers/d_model");
+  DG_REQUIRE(c.n_q_heads >= 1 && c.n_kv_heads >= 1 && c.n_q_heads % c.n_kv_heads == 0,
+             "n_q_heads must be a positive multiple of n_kv_heads");
+  DG_REQUIRE(c.head_dim >= 2 && c.head_dim % 2 == 0 && c.head_dim <= 128,
+             "head_dim must be even and <= 128");
+  DG_REQUIRE(c.n_experts >= 1 && c.n_experts <= 1024, "n_experts must be in [1, 1024]");
+  DG_REQUIRE(c.top_k >= 1 && c.top_k <= c.n_experts && c.top_k <= 64, "bad top_k");
+  DG_REQUIRE(c.expert_inter >= 1 && c.shared_inter >= 1, "bad intermediate sizes");
+  DG_REQUIRE(c.vocab >= 2 && c.window >= 1, "bad vocab/window");
+  DG_REQUIRE(c.canvas >= 1 && c.canvas <= 1024, "canvas must be in [1, 1024]");
+  DG_REQUIRE(c.max_batch >= 1 && c.max_prompt >= 1, "bad max_batch/max_prompt");
+  DG_REQUIRE(c.rms_eps >= 0.0f && std::isfinite(c.logit_scale) && c.rope_base > 0.0f,
+             "bad eps/logit_scale/rope_base");
+  DG_REQUIRE(c.dtype == DG_F32 || c.dtype == DG_BF16 || c.dtype == DG_BF16_FP8EXP,
+             "unknown dtype %d", c.dtype);
+  if (c.dtype == DG_BF16_FP8EXP) {
+    set_error("FP8 expert weights are not implemented in this build");
+    return DG_ERR_UNSUPPORTED;
+  }
+  DG_REQUIRE(w->tok_emb && w->lm_head && w->layers, "null weight pointer");
+  for (int l = 0; l < c.n_layers; ++l) {
+    const dg_layer_weights& L = w->layers[l];
+    DG_REQUIRE(L.wqkv && L.wo && L.router && L.gate && L.up && L.down && L.sgate && L.sup &&
+                   L.sdown,
+               "null weight pointer in layer %d", l);
+  }
+  dg_model* m = new dg_model();
+  m->cfg = c;
+  m->w = *w;
+  m->layers.assign(w->layers, w->layers + c.n_layers);
+  m->w.layers = nullptr;
+  cudaGetDevice(&m->device);
+  dg_status s = c.dtype == DG_F32 ? alloc_workspace<PathTiny>(m) : alloc_workspace<PathBF16>(m);
+  if (s != DG_OK) {
+    std::string keep = g_err;
+    ws_free(m->ws);
+    delete m;
+    g_err = keep;
+    return s;
+  }
+  *out = m;
+  return DG_OK;
+}
+
+dg_status dg_model_destroy(dg_model* m) {
+  if (!m) return DG_OK;
+  cudaDeviceSynchronize();
+  tc_release(m);
+  ws_free(m->ws);
+  delete m;
+  return DG_OK;
+}
+
+dg_status dg_sync_status(dg_model* m, void* stream) {
+  DG_REQUIRE(m, "null model");
+  cudaStream_t st = (cudaStream_t)stream;
+  DG_TRY_CUDA(cudaStreamSynchronize(st));
+  int32_t err[4] = {0, 0, 0, 0};
+  DG_TRY_CUDA(cudaMemcpy(err, m->ws.err, sizeof(err), cudaMemcpyDeviceToHost));
+  DG_TRY_CUDA(cudaMemset(m->ws.err, 0, sizeof(err)));
+  if (err[0] & ERR_TIMEOUT) {
+    set_error("a device-side bounded wait gave up (error bits 0x%x)", err[0]);
+    return DG_ERR_TIMEOUT;
+  }
+  if (err[0] & ERR_BAD_TOKEN) {
+    set_error("a token id outside the vocabulary reached the embedding");
+    return DG_ERR_INVALID_ARG;
+  }
+  if (err[0]) {
+    set_error("device error bits 0x%x", err[0]);
+    return DG_ERR_INTERNAL;
+  }
+  return DG_OK;
+}
+
+dg_status dg_prefill(dg_model* m, const int32_t* prompt, int32_t B, int32_t P, dg_kv** out,
+                     void* stream) {
+  g_err.clear();
+  DG_REQUIRE(m && prompt && out, "null argument");
+  *out = nullptr;
+  const dg_config& c = m->cfg;
+  DG_REQUIRE(B >= 1 && B <= c.max_batch, "B=%d outside [1, max_batch=%d]", B, c.max_batch);
+  DG_REQUIRE(P >= 1 && P <= c.max_prompt, "P=%d outside [1, max_prompt=%d]", P, c.max_prompt);
+  dg_kv* kv = new dg_kv();
+  kv->m = m;
+  kv->B = B;
+  kv->P = P;
+  kv->W = std::min(P, c.window);
+  kv->elem = c.dtype == DG_F32 ? sizeof(double) : sizeof(bf16);
+  const size_t n = (size_t)c.n_layers * B * c.n_kv_heads * kv->W * c.head_dim * kv->elem;
+  if (cudaMalloc(&kv->k, n) != cudaSuccess || cudaMalloc(&kv->v, n) != cudaSuccess) {
+    cudaGetLastError();
+    cudaFree(kv->k);
+    cudaFree(kv->v);
+    delete kv;
+    set_error("KV cache allocation of 2 x %zu bytes failed", n);
+    return DG_ERR_OOM;
+  }
+  cudaStream_t st = (cudaStream_t)stream;
+  dg_status s = c.dtype == DG_F32 ? Runner<PathTiny>(m, st).prefill(prompt, B, P, kv)
+                                  : Runner<PathBF16>(m, st).prefill(prompt, B, P, kv);
+  if (s != DG_OK) {
+    cudaStreamSynchronize(st);
+    cudaFree(kv->k);
+    cudaFree(kv->v);
+    delete kv;
+    return s;
+  }
+  *out = kv;
+  return DG_OK;
+}
+
+dg_status dg_kv_destroy(dg_kv* kv) {
+  if (!kv) return DG_OK;
+  cudaDeviceSynchronize();
+  cudaFree(kv->k);
+  cudaFree(kv->v);
+  delete kv;
+  return DG_OK;
+}
+
+dg_status dg_kv_info(const dg_kv* kv, int32_t* B, int32_t* P, int32_t* W) {
+  DG_REQUIRE(kv, "null kv");
+  if (B) *B = kv->B;
+  if (P) *P = kv->P;
+  if (W) *W = kv->W;
+  return DG_OK;
+}
+
+dg_status dg_kv_read(const dg_kv* kv, void* k, void* v, void* stream) {
+  DG_REQUIRE(kv && k && v, "null argument");
+  const dg_config& c = kv->m->cfg;
+  const size_t n = (size_t)c.n_layers * kv->B * c.n_kv_heads * kv->W * c.head_dim * kv->elem;
+  cudaStream_t st = (cudaStream_t)stream;
+  DG_TRY_CUDA(cudaMemcpyAsync(k, kv->k, n, cudaMemcpyDeviceToDevice, st));
+  DG_TRY_CUDA(cudaMemcpyAsync(v, kv->v, n, cudaMemcpyDeviceToDevice, st));
+  return DG_OK;
+}
+
+static dg_status check_step_args(dg_model* m, const dg_kv* kv, int s, int T) {
+  DG_REQUIRE(m && kv, "null model/kv");
+  DG_REQUIRE(kv->m == m, "kv handle belongs to another model");
+  DG_REQUIRE(T >= 1 && s >= 1 && s <= T, "steps_left=%d must be in [1, T=%d]", s, T);
+  return DG_OK;
+}
+
+static dg_status run_forward(dg_model* m, const dg_kv* kv, const int32_t* canvas, int s, int T,
+                             float* ent, int32_t* am, float* logits, float* hidden,
+                             int32_t* load, cudaStream_t st) {
+  return m->cfg.dtype == DG_F32
+             ? Runner<PathTiny>(m, st).forward(kv, canvas, s, T, ent, am, logits, hidden, load)
+             : Runner<PathBF16>(m, st).forward(kv, canvas, s, T, ent, am, logits, hidden, load);
+}
+
+dg_status dg_denoise_step(dg_model* m, const dg_kv* kv, int32_t* canvas, uint8_t* mask,
+                          int32_t steps_left, int32_t T, float gamma, float* entropy,
+                          int32_t* argmax, int32_t* n_committed, void* stream) {
+  g_err.clear();
+  DG_TRY(check_step_args(m, kv, steps_left, T));
+  DG_REQUIRE(canvas && mask && entropy && argmax && n_committed, "null argument");
+  long long gq;
+  DG_TRY(gamma_fixed(gamma, &gq));
+  cudaStream_t st = (cudaStream_t)stream;
+  DG_TRY(run_forward(m, kv, canvas, steps_left, T, entropy, argmax, nullptr, nullptr, nullptr, st));
+  return launch_sampler(entropy, argmax, canvas, mask, kv->B, m->cfg.canvas, steps_left, gq,
+                        n_committed, nullptr, 0, st);
+}
+
+dg_status dg_generate_block(dg_model* m, const dg_kv* kv, int32_t T, float gamma,
+                            int32_t* canvas_out, int32_t* n_forwards, int32_t* router_load,
+                            void* stream) {
+  g_err.clear();
+  DG_TRY(check_step_args(m, kv, T, T));
+  DG_REQUIRE(canvas_out, "null canvas_out");
+  long long gq;
+  DG_TRY(gamma_fixed(gamma, &gq));
+  cudaStream_t st = (cudaStream_t)stream;
+  const dg_config& c = m->cfg;
+  const int B = kv->B, C = c.canvas;
+  Workspace& ws = m->ws;
+  fill_i32_kernel<<<ceil_div((long)B * C, 256), 256, 0, st>>>(canvas_out, B * C, c.vocab);
+  DG_TRY_CUDA(cudaMemsetAsync(ws.mask, 1, (size_t)B * C, st));
+  if (n_forwards) DG_TRY_CUDA(cudaMemsetAsync(n_forwards, 0, B * sizeof(int32_t), st));
+  if (router_load)
+    DG_TRY_CUDA(cudaMemsetAsync(router_load, 0,
+                                (size_t)c.n_layers * c.n_experts * sizeof(int32_t), st));
+  for (int k = 0; k < T; ++k) {
+    const int s = T - k;
+    DG_TRY(run_forward(m, kv, canvas_out, s, T, ws.ent, ws.amax, nullptr, nullptr, router_load,
+                       st));
+    DG_TRY(launch_sampler(ws.ent, ws.amax, canvas_out, ws.mask, B, C, s, gq, ws.ncommit,
+                          n_forwards, k + 1, st));
+  }
+  return DG_OK;
+}
+
+dg_status dg_eb_sample(const float* entropy, const int32_t* argmax, int32_t* canvas,
+                       uint8_t* mask, int32_t B, int32_t C, int32_t steps_left, float gamma,
+                       int32_t* n_committed, void* stream) {
+  g_err.clear();
+  DG_REQUIRE(entropy && argmax && canvas && mask, "null argument");
+  DG_REQUIRE(B >= 1 && C >= 1 && C <= 1024, "need B >= 1 and 1 <= C <= 1024");
+  DG_REQUIRE(steps_left >= 1, "steps_left must be >= 1");
+  long long gq;
+  DG_TRY(gamma_fixed(gamma, &gq));
+  return launch_sampler(entropy, argmax, canvas, mask, B, C, steps_left, gq, n_committed,
+                        nullptr, 0, (cudaStream_t)stream);
+}
+
+dg_status dg_debug_forward(dg_model* m, const dg_kv* kv, const int32_t* canvas,
+                           int32_t steps_left, int32_t T, float* entropy, int32_t* argmax,
+                           float* logits, float* hidden, void* stream) {
+  g_err.clear();
+  DG_TRY(check_step_args(m, kv, steps_left, T));
+  DG_REQUIRE(canvas && entropy && argmax, "null argument");
+  return run_forward(m, kv, canvas, steps_left, T, entropy, argmax, logits, hidden, nullptr,
+                     (cudaStream_t)stream);
+}
+
+}  // extern "C"

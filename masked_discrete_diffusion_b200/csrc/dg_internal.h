@@ -1,0 +1,93 @@
+// Internal declarations of libdg: model/KV structs, workspace, error helpers.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <string>
+#include <vector>
+
+#include "../../include/dg.h"
+
+namespace dg {
+
+void set_error(const char* fmt, ...);
+
+#define DG_TRY_CUDA(call)                                                            \
+  do {                                                                               \
+    cudaError_t e_ = (call);                                                         \
+    if (e_ != cudaSuccess) {                                                         \
+      ::dg::set_error("%s failed: %s (%s:%d)", #call, cudaGetErrorString(e_), __FILE__, \
+                      __LINE__);                                                     \
+      return e_ == cudaErrorMemoryAllocation ? DG_ERR_OOM : DG_ERR_CUDA;             \
+    }                                                                                \
+  } while (0)
+
+#define DG_REQUIRE(cond, ...)        \
+  do {                               \
+    if (!(cond)) {                   \
+      ::dg::set_error(__VA_ARGS__);  \
+      return DG_ERR_INVALID_ARG;     \
+    }                                \
+  } while (0)
+
+#define DG_TRY(expr)                 \
+  do {                               \
+    dg_status s_ = (expr);           \
+    if (s_ != DG_OK) return s_;      \
+  } while (0)
+
+// Device error bits (set by kernels, read and cleared by dg_sync_status).
+enum : int { ERR_BAD_TOKEN = 1, ERR_TIMEOUT = 2, ERR_BAD_SHAPE = 4 };
+
+// A typed device allocation owned by the workspace.
+struct DevBuf {
+  void* p = nullptr;
+  size_t bytes = 0;
+};
+
+struct Workspace {
+  size_t max_tok = 0;       // rows of every per-token buffer
+  size_t max_rows = 0;      // max_tok * top_k routed rows
+  std::vector<DevBuf> bufs; // for release
+  // per-token buffers (element types depend on the precision path)
+  void *x = nullptr, *xn = nullptr, *qkv = nullptr, *q = nullptr, *o = nullptr;
+  void *kc = nullptr, *vc = nullptr;          // current layer's own keys/values
+  void *ys = nullptr, *sh = nullptr;          // shared expert output / hidden
+  // routing
+  int32_t *ridx = nullptr, *rank = nullptr, *row_of = nullptr, *tok_of = nullptr;
+  void *rgate = nullptr, *gate_of = nullptr;
+  int32_t *counts = nullptr, *offsets = nullptr, *tile_e = nullptr, *tile_m0 = nullptr,
+          *n_tiles = nullptr;
+  void *up = nullptr, *hb = nullptr, *yb = nullptr; // routed rows
+  void* lm_part = nullptr;                          // [n_vtiles, max_tok, 4]
+  int32_t* load = nullptr;                          // [L, E] routing counts
+  int32_t* err = nullptr;                           // device error bits
+  int32_t* ids = nullptr;                           // [max_tok] token ids of the pass
+  void* rope = nullptr;                             // [max_pos, h/2] cos then sin
+  uint8_t* mask = nullptr;                          // [max_batch, C] block-loop mask
+  float* ent = nullptr;                             // [max_batch, C] entropies
+  int32_t *amax = nullptr, *ncommit = nullptr;      // [max_batch, C], [max_batch]
+  int max_pos = 0;
+  int max_tiles = 0;
+  int n_vtiles = 0;
+};
+
+}  // namespace dg
+
+struct dg_model {
+  dg_config cfg;
+  dg_weights w;
+  std::vector<dg_layer_weights> layers;
+  int device = 0;
+  dg::Workspace ws;
+};
+
+struct dg_kv {
+  dg_model* m = nullptr;
+  int B = 0, P = 0, W = 0;
+  void* k = nullptr;  // [L, B, Hkv, W, h]
+  void* v = nullptr;
+  size_t elem = 0;    // bytes per element
+};

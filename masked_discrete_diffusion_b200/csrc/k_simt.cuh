@@ -1,0 +1,626 @@
+// CUDA-core kernels of the denoise forward (all precisions).
+//
+// These carry the whole path for the fp32 tiny model (activations and sums in
+// fp64) and every step that is not a dense contraction for the bf16 models.
+// The dense contractions of the bf16 models run on tcgen05 (k_tc_gemm.cuh).
+//
+// Model passages: "DiffusionGemma 技术报告" (full translation page) §3.1-§3.2
+// (causal context pass, bidirectional canvas decoder, logits per position);
+// explainer page "DiffusionGemma 深度解析", list "核心架构参数" (MoE top-8 of 128
+// plus one shared expert, sliding window 1024, timestep embedding).
+#pragma once
+
+#include "k_common.cuh"
+
+namespace dg {
+
+// ---------------------------------------------------------------------------
+// a1: embedding gather (+ sinusoidal timestep embedding for canvas rows)
+// x[t, :] = E[ids[t], :] + temb(tau); temb[i] = sin(1000 tau w_i),
+// temb[d/2 + i] = cos(1000 tau w_i), w_i = 10000^(-i / (d/2)).  tau < 0: none.
+// ---------------------------------------------------------------------------
+template <class TW, class TR>
+__global__ void embed_kernel(const int32_t* __restrict__ ids, const TW* __restrict__ emb,
+                             TR* __restrict__ x, int n_tok, int d, int max_id, double tau,
+                             int32_t* err) {
+  const int t = blockIdx.x;
+  if (t >= n_tok) return;
+  int id = ids[t];
+  if (id < 0 || id > max_id) {
+    if (threadIdx.x == 0) atomicOr(err, 1);
+    id = 0;
+  }
+  const TW* row = emb + (size_t)id * d;
+  const int half = d / 2;
+  for (int c = threadIdx.x; c < d; c += blockDim.x) {
+    double v = (double)widen(row[c]);
+    if (tau >= 0.0) {
+      const int i = c < half ? c : c - half;
+      const double w = pow(10000.0, -(double)i / (double)half);
+      const double a = 1000.0 * tau * w;
+      v += c < half ? sin(a) : cos(a);
+    }
+    x[(size_t)t * d + c] = narrow<TR>(v);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// RMSNorm, gain 1: y = x / sqrt(mean(x^2) + eps)
+// ---------------------------------------------------------------------------
+template <class TR, class TA, class Acc>
+__global__ void rmsnorm_kernel(const TR* __restrict__ x, TA* __restrict__ y, int n, int d,
+                               float eps) {
+  __shared__ Acc red[32];
+  const int t = blockIdx.x;
+  if (t >= n) return;
+  const TR* r = x + (size_t)t * d;
+  Acc ss = 0;
+  for (int c = threadIdx.x; c < d; c += blockDim.x) {
+    Acc v = (Acc)widen(r[c]);
+    ss += v * v;
+  }
+  ss = block_sum(ss, red);
+  const Acc inv = Acc(1) / dsqrt(ss / (Acc)d + (Acc)eps);
+  for (int c = threadIdx.x; c < d; c += blockDim.x)
+    y[(size_t)t * d + c] = narrow<TA>((Acc)widen(r[c]) * inv);
+}
+
+// ---------------------------------------------------------------------------
+// Tiled CUDA-core GEMM  C[M, N] = A[M, K] W[N, K]^T with an epilogue functor.
+// GROUPED: blockIdx.y walks a tile table (expert e, first permuted row m0);
+// rows [m0, min(m0 + 64, offsets[e + 1])) use weight slab W + e * w_slab.
+// DUAL: a second weight W2 is accumulated alongside (gate and up projections).
+// ---------------------------------------------------------------------------
+struct GroupInfo {
+  const int32_t* tile_e = nullptr;
+  const int32_t* tile_m0 = nullptr;
+  const int32_t* n_tiles = nullptr;
+  const int32_t* offsets = nullptr;
+  size_t w_slab = 0;
+};
+
+constexpr int SG_BM = 64, SG_BN = 64, SG_BK = 16;
+
+template <class TA, class TW, class Acc, bool GROUPED, bool DUAL, class Epi>
+__global__ void __launch_bounds__(256)
+    gemm_simt_kernel(const TA* __restrict__ A, int lda, const TW* __restrict__ W,
+                     const TW* __restrict__ W2, int ldw, int M, int N, int K, GroupInfo g,
+                     Epi epi) {
+  __shared__ Acc As[SG_BK][SG_BM + 1];
+  __shared__ Acc Ws[SG_BK][SG_BN + 1];
+  __shared__ Acc Ws2[DUAL ? SG_BK : 1][DUAL ? SG_BN + 1 : 1];
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  const int n0 = blockIdx.x * SG_BN;
+  int m0 = blockIdx.y * SG_BM, m_end = M;
+  int e = 0;
+  if (GROUPED) {
+    if ((int)blockIdx.y >= *g.n_tiles) return;
+    e = g.tile_e[blockIdx.y];
+    m0 = g.tile_m0[blockIdx.y];
+    m_end = g.offsets[e + 1];
+    W += (size_t)e * g.w_slab;
+    if (DUAL) W2 += (size_t)e * g.w_slab;
+  }
+  const int m_lim = min(m0 + SG_BM, m_end);
+  Acc acc[4][4], acc2[DUAL ? 4 : 1][DUAL ? 4 : 1];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      acc[i][j] = 0;
+      if (DUAL) acc2[DUAL ? i : 0][DUAL ? j : 0] = 0;
+    }
+  for (int k0 = 0; k0 < K; k0 += SG_BK) {
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+      const int el = tid + it * 256, r = el >> 4, kk = el & 15;
+      const int gm = m0 + r, gk = k0 + kk, gn = n0 + r;
+      As[kk][r] = (gm < m_lim && gk < K) ? (Acc)widen(A[(size_t)gm * lda + gk]) : Acc(0);
+      Ws[kk][r] = (gn < N && gk < K) ? (Acc)widen(W[(size_t)gn * ldw + gk]) : Acc(0);
+      if (DUAL)
+        Ws2[DUAL ? kk : 0][DUAL ? r : 0] =
+            (gn < N && gk < K) ? (Acc)widen(W2[(size_t)gn * ldw + gk]) : Acc(0);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < SG_BK; ++kk) {
+      Acc a[4], b[4], b2[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = As[kk][ty + 16 * i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        b[j] = Ws[kk][tx + 16 * j];
+        if (DUAL) b2[j] = Ws2[DUAL ? kk : 0][DUAL ? tx + 16 * j : 0];
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          acc[i][j] += a[i] * b[j];
+          if (DUAL) acc2[DUAL ? i : 0][DUAL ? j : 0] += a[i] * b2[j];
+        }
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int r = m0 + ty + 16 * i, c = n0 + tx + 16 * j;
+      if (r < m_lim && c < N) {
+        if (DUAL)
+          epi(r, c, acc[i][j], acc2[DUAL ? i : 0][DUAL ? j : 0]);
+        else
+          epi(r, c, acc[i][j], acc[i][j]);
+      }
+    }
+}
+
+template <class TO, class Acc> struct EpiStore {
+  TO* out;
+  int ldo;
+  __device__ void operator()(int r, int c, Acc v, Acc) const {
+    out[(size_t)r * ldo + c] = narrow<TO>(v);
+  }
+};
+
+template <class TR, class Acc> struct EpiAddResidual {
+  TR* res;
+  int ldr;
+  __device__ void operator()(int r, int c, Acc v, Acc) const {
+    TR* p = res + (size_t)r * ldr + c;
+    *p = narrow<TR>((Acc)widen(*p) + v);
+  }
+};
+
+template <class TO, class Acc> struct EpiSwiglu {
+  TO* out;
+  int ldo;
+  __device__ void operator()(int r, int c, Acc g, Acc u) const {
+    out[(size_t)r * ldo + c] = narrow<TO>(silu(g) * u);
+  }
+};
+
+template <class TO, class Acc> struct EpiRowScale {
+  TO* out;
+  int ldo;
+  const Acc* scale;
+  __device__ void operator()(int r, int c, Acc v, Acc) const {
+    out[(size_t)r * ldo + c] = narrow<TO>(scale[r] * v);
+  }
+};
+
+// ---------------------------------------------------------------------------
+// a2 (RoPE part): rotate q and k of the raw projection, scatter q / k / v.
+// qkv: [n_tok, (Hq + 2 Hkv) h] raw projections.  Token t = b * n_seq + i sits at
+// absolute position pos0 + i.  q -> q_out [n_tok, Hq, h];
+// k, v -> kc / vc [b, Hkv, n_seq, h].  Pair (j, j + h/2) rotates by pos*theta_j.
+// rope: [max_pos, h/2] cos values followed by [max_pos, h/2] sin values.
+// ---------------------------------------------------------------------------
+template <class Acc, class TA, class TKV>
+__global__ void rope_scatter_kernel(const Acc* __restrict__ qkv, TA* __restrict__ q_out,
+                                    TKV* __restrict__ kc, TKV* __restrict__ vc, int n_tok,
+                                    int n_seq, int pos0, int Hq, int Hkv, int h,
+                                    const Acc* __restrict__ rope, int max_pos) {
+  const int t = blockIdx.x;
+  if (t >= n_tok) return;
+  const int b = t / n_seq, i = t % n_seq, pos = pos0 + i;
+  const int half = h / 2, heads = Hq + 2 * Hkv;
+  const Acc* row = qkv + (size_t)t * heads * h;
+  const Acc* cs = rope + (size_t)pos * half;
+  const Acc* sn = rope + (size_t)max_pos * half + (size_t)pos * half;
+  for (int e = threadIdx.x; e < heads * half; e += blockDim.x) {
+    const int hd = e / half, j = e % half;
+    const Acc x1 = row[hd * h + j], x2 = row[hd * h + j + half];
+    if (hd < Hq + Hkv) {
+      const Acc c = cs[j], s = sn[j];
+      const Acc y1 = x1 * c - x2 * s, y2 = x2 * c + x1 * s;
+      if (hd < Hq) {
+        TA* qo = q_out + ((size_t)t * Hq + hd) * h;
+        qo[j] = narrow<TA>(y1);
+        qo[j + half] = narrow<TA>(y2);
+      } else {
+        TKV* ko = kc + (((size_t)b * Hkv + (hd - Hq)) * n_seq + i) * h;
+        ko[j] = narrow<TKV>(y1);
+        ko[j + half] = narrow<TKV>(y2);
+      }
+    } else {
+      TKV* vo = vc + (((size_t)b * Hkv + (hd - Hq - Hkv)) * n_seq + i) * h;
+      vo[j] = narrow<TKV>(x1);
+      vo[j + half] = narrow<TKV>(x2);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// a3: attention, one warp per (batch b, query i, query head j).
+// Keys: segment A (the cached prompt window, nA keys, absolute positions
+// kposA..) followed by segment B (the pass's own keys, nB keys at kposB..).
+// causal != 0: key at position p is visible to the query at position qp iff
+// qp - window < p <= qp; otherwise every key is visible.  One online softmax
+// over both segments; scores scaled by 1/sqrt(h).  DPL = ceil(h / 32).
+// K/V layouts: [b, Hkv, n, h]; q/o: [b * nq + i, Hq, h].
+// ---------------------------------------------------------------------------
+template <class TA, class TKV, class Acc, int DPL>
+__global__ void attention_simt_kernel(const TA* __restrict__ q, TA* __restrict__ o,
+                                      const TKV* __restrict__ kA, const TKV* __restrict__ vA,
+                                      int nA, int kposA, const TKV* __restrict__ kB,
+                                      const TKV* __restrict__ vB, int nB, int kposB, int B,
+                                      int nq, int qpos0, int Hq, int Hkv, int h, int causal,
+                                      int window) {
+  const int lane = threadIdx.x & 31;
+  const long wid = (long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const long total = (long)B * nq * Hq;
+  if (wid >= total) return;
+  const int j = (int)(wid % Hq);
+  const long ti = wid / Hq;  // b * nq + i
+  const int b = (int)(ti / nq), i = (int)(ti % nq);
+  const int kvh = j / (Hq / Hkv);
+  const int qp = qpos0 + i;
+  const Acc scale = Acc(1) / dsqrt((Acc)h);
+  Acc qv[DPL], acc[DPL];
+  const TA* qrow = q + ((size_t)ti * Hq + j) * h;
+#pragma unroll
+  for (int u = 0; u < DPL; ++u) {
+    const int dd = lane + 32 * u;
+    qv[u] = dd < h ? (Acc)widen(qrow[dd]) * scale : Acc(0);
+    acc[u] = 0;
+  }
+  Acc mrun = -INFINITY, lrun = 0;
+  for (int seg = 0; seg < 2; ++seg) {
+    const TKV* K = seg == 0 ? kA : kB;
+    const TKV* V = seg == 0 ? vA : vB;
+    const int n = seg == 0 ? nA : nB;
+    const int p0 = seg == 0 ? kposA : kposB;
+    if (n == 0 || K == nullptr) continue;
+    const size_t base = ((size_t)b * Hkv + kvh) * n * h;
+    int lo = 0, hi = n;
+    if (causal) {
+      lo = max(0, qp - window + 1 - p0);
+      hi = min(n, qp - p0 + 1);
+    }
+    for (int t = lo; t < hi; ++t) {
+      const TKV* kr = K + base + (size_t)t * h;
+      Acc s = 0;
+#pragma unroll
+      for (int u = 0; u < DPL; ++u) {
+        const int dd = lane + 32 * u;
+        if (dd < h) s += qv[u] * (Acc)widen(kr[dd]);
+      }
+      s = warp_sum(s);
+      const Acc mnew = max(mrun, s);
+      const Acc corr = dexp(mrun - mnew), pexp = dexp(s - mnew);
+      lrun = lrun * corr + pexp;
+      const TKV* vr = V + base + (size_t)t * h;
+#pragma unroll
+      for (int u = 0; u < DPL; ++u) {
+        const int dd = lane + 32 * u;
+        if (dd < h) acc[u] = acc[u] * corr + pexp * (Acc)widen(vr[dd]);
+      }
+      mrun = mnew;
+    }
+  }
+  TA* orow = o + ((size_t)ti * Hq + j) * h;
+  const Acc inv = Acc(1) / lrun;
+#pragma unroll
+  for (int u = 0; u < DPL; ++u) {
+    const int dd = lane + 32 * u;
+    if (dd < h) orow[dd] = narrow<TA>(acc[u] * inv);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// a5: router.  u = RMSNorm(x) (recomputed from the residual at the accumulation
+// precision), logits = u Wr^T, p = softmax over all E, top-k by p (ties -> lower
+// expert id), gates renormalised to sum 1.  One block per token.
+// ---------------------------------------------------------------------------
+template <class TR, class TW, class Acc>
+__global__ void router_kernel(const TR* __restrict__ x, const TW* __restrict__ wr, int n_tok,
+                              int d, int E, int top_k, float eps, int32_t* __restrict__ idx,
+                              Acc* __restrict__ gate, int32_t* __restrict__ load) {
+  extern __shared__ unsigned char smem_raw[];
+  Acc* p = reinterpret_cast<Acc*>(smem_raw);  // [E]
+  __shared__ Acc red[32];
+  const int t = blockIdx.x;
+  if (t >= n_tok) return;
+  const TR* xr = x + (size_t)t * d;
+  Acc ss = 0;
+  for (int c = threadIdx.x; c < d; c += blockDim.x) {
+    const Acc v = (Acc)widen(xr[c]);
+    ss += v * v;
+  }
+  ss = block_sum(ss, red);
+  const Acc inv = Acc(1) / dsqrt(ss / (Acc)d + (Acc)eps);
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int e = wid; e < E; e += nw) {
+    const TW* w = wr + (size_t)e * d;
+    Acc s = 0;
+    for (int c = lane; c < d; c += 32) s += ((Acc)widen(xr[c]) * inv) * (Acc)widen(w[c]);
+    s = warp_sum(s);
+    if (lane == 0) p[e] = s;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    Acc mx = p[0];
+    for (int e = 1; e < E; ++e) mx = max(mx, p[e]);
+    Acc z = 0;
+    for (int e = 0; e < E; ++e) {
+      p[e] = dexp(p[e] - mx);
+      z += p[e];
+    }
+    for (int e = 0; e < E; ++e) p[e] /= z;
+    int sel[64];
+    Acc gs = 0;
+    for (int k = 0; k < top_k; ++k) {
+      int best = -1;
+      for (int e = 0; e < E; ++e) {
+        bool taken = false;
+        for (int q2 = 0; q2 < k; ++q2) taken |= (sel[q2] == e);
+        if (taken) continue;
+        if (best < 0 || p[e] > p[best]) best = e;
+      }
+      sel[k] = best;
+      gs += p[best];
+    }
+    for (int k = 0; k < top_k; ++k) {
+      idx[(size_t)t * top_k + k] = sel[k];
+      gate[(size_t)t * top_k + k] = p[sel[k]] / gs;
+      if (load) atomicAdd(&load[sel[k]], 1);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Deterministic permutation of (token, slot) entries into expert-contiguous
+// rows.  Entry j = t * k + slot belongs to expert idx[j]; within an expert the
+// entries keep their j order.  Block e computes the rank of each of its entries
+// and counts[e].
+// ---------------------------------------------------------------------------
+__global__ void moe_rank_kernel(const int32_t* __restrict__ idx, int n_entries,
+                                int32_t* __restrict__ rank, int32_t* __restrict__ counts) {
+  __shared__ int warp_tot[32];
+  __shared__ int carry;
+  const int e = blockIdx.x;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  for (int base = 0; base < n_entries; base += blockDim.x) {
+    const int j = base + threadIdx.x;
+    const bool f = j < n_entries && idx[j] == e;
+    const unsigned bal = __ballot_sync(0xffffffffu, f);
+    const int before = __popc(bal & ((1u << lane) - 1u));
+    if (lane == 0) warp_tot[wid] = __popc(bal);
+    __syncthreads();
+    int off = carry;
+    for (int w2 = 0; w2 < wid; ++w2) off += warp_tot[w2];
+    if (f) rank[j] = off + before;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int s = 0;
+      for (int w2 = 0; w2 < nw; ++w2) s += warp_tot[w2];
+      carry += s;
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) counts[e] = carry;
+}
+
+// offsets = exclusive scan of counts; tile table with `bm` rows per tile.
+__global__ void moe_offsets_kernel(const int32_t* __restrict__ counts, int E, int bm,
+                                   int32_t* __restrict__ offsets, int32_t* __restrict__ tile_e,
+                                   int32_t* __restrict__ tile_m0, int32_t* __restrict__ n_tiles,
+                                   int max_tiles) {
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  int off = 0, nt = 0;
+  for (int e = 0; e < E; ++e) {
+    offsets[e] = off;
+    const int c = counts[e];
+    for (int r = 0; r < c; r += bm) {
+      if (nt < max_tiles) {
+        tile_e[nt] = e;
+        tile_m0[nt] = off + r;
+      }
+      ++nt;
+    }
+    off += c;
+  }
+  offsets[E] = off;
+  *n_tiles = min(nt, max_tiles);
+}
+
+template <class Acc>
+__global__ void moe_scatter_kernel(const int32_t* __restrict__ idx, const Acc* __restrict__ gate,
+                                   const int32_t* __restrict__ rank,
+                                   const int32_t* __restrict__ offsets, int n_entries, int top_k,
+                                   int32_t* __restrict__ row_of, int32_t* __restrict__ tok_of,
+                                   Acc* __restrict__ gate_of) {
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= n_entries) return;
+  const int pos = offsets[idx[j]] + rank[j];
+  row_of[j] = pos;
+  tok_of[pos] = j / top_k;
+  gate_of[pos] = gate[j];
+}
+
+template <class TA>
+__global__ void gather_rows_kernel(const TA* __restrict__ src, const int32_t* __restrict__ tok_of,
+                                   const int32_t* __restrict__ n_rows_dev, int d,
+                                   TA* __restrict__ dst) {
+  const int r = blockIdx.x;
+  if (r >= *n_rows_dev) return;
+  const TA* s = src + (size_t)tok_of[r] * d;
+  TA* o = dst + (size_t)r * d;
+  for (int c = threadIdx.x; c < d; c += blockDim.x) o[c] = s[c];
+}
+
+// x[t] += ys[t] + sum over slots of yb[row_of[t * k + slot]] (slot order fixed).
+template <class TR, class TY, class Acc>
+__global__ void moe_combine_kernel(TR* __restrict__ x, const TY* __restrict__ ys,
+                                   const TY* __restrict__ yb, const int32_t* __restrict__ row_of,
+                                   int n_tok, int d, int top_k) {
+  const int t = blockIdx.x;
+  if (t >= n_tok) return;
+  for (int c = threadIdx.x; c < d; c += blockDim.x) {
+    Acc y = (Acc)widen(ys[(size_t)t * d + c]);
+    for (int k = 0; k < top_k; ++k)
+      y += (Acc)widen(yb[(size_t)row_of[(size_t)t * top_k + k] * d + c]);
+    TR* p = x + (size_t)t * d + c;
+    *p = narrow<TR>((Acc)widen(*p) + y);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// a8 (CUDA-core form): logits tile = scale * xn W_lm^T for 64 rows x 64 vocab
+// entries, reduced per row to partial statistics over the tile:
+//   m = max logit, s = sum exp(l - m), u = sum exp(l - m) (l - m), a = argmax
+// (lowest id among equal maxima).  Partials: [n_vtiles, n_rows, 4].
+// Optional logits output [n_rows, V] (test hook).
+// ---------------------------------------------------------------------------
+template <class TA, class TW, class Acc>
+__global__ void __launch_bounds__(256)
+    lmhead_simt_kernel(const TA* __restrict__ xn, const TW* __restrict__ wlm, int n_rows, int V,
+                       int d, float scale, Acc* __restrict__ part, float* __restrict__ logits) {
+  // the logits tile T reuses the operand staging buffers once the K loop is done
+  constexpr int kStage = 2 * SG_BK * (SG_BM + 1), kTile = SG_BM * (SG_BN + 1);
+  __shared__ Acc smem[kStage > kTile ? kStage : kTile];
+  Acc(*As)[SG_BM + 1] = reinterpret_cast<Acc(*)[SG_BM + 1]>(smem);
+  Acc(*Ws)[SG_BN + 1] = reinterpret_cast<Acc(*)[SG_BN + 1]>(smem + SG_BK * (SG_BM + 1));
+  Acc(*T)[SG_BN + 1] = reinterpret_cast<Acc(*)[SG_BN + 1]>(smem);
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  const int n0 = blockIdx.x * SG_BN, m0 = blockIdx.y * SG_BM;
+  Acc acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0;
+  for (int k0 = 0; k0 < d; k0 += SG_BK) {
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+      const int el = tid + it * 256, r = el >> 4, kk = el & 15;
+      const int gm = m0 + r, gk = k0 + kk, gn = n0 + r;
+      As[kk][r] = (gm < n_rows && gk < d) ? (Acc)widen(xn[(size_t)gm * d + gk]) : Acc(0);
+      Ws[kk][r] = (gn < V && gk < d) ? (Acc)widen(wlm[(size_t)gn * d + gk]) : Acc(0);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < SG_BK; ++kk) {
+      Acc a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = As[kk][ty + 16 * i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) b[j] = Ws[kk][tx + 16 * j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] += a[i] * b[j];
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const Acc l = (Acc)scale * acc[i][j];
+      T[ty + 16 * i][tx + 16 * j] = l;
+      const int r = m0 + ty + 16 * i, c = n0 + tx + 16 * j;
+      if (logits && r < n_rows && c < V) logits[(size_t)r * V + c] = (float)l;
+    }
+  __syncthreads();
+  const int lane = tid & 31, wid = tid >> 5;
+  for (int rr = wid; rr < SG_BM; rr += 8) {
+    const int r = m0 + rr;
+    if (r >= n_rows) continue;
+    Acc mx = -INFINITY;
+    int am = 0x7fffffff;
+    for (int c = lane; c < SG_BN; c += 32) {
+      if (n0 + c >= V) continue;
+      const Acc l = T[rr][c];
+      if (l > mx || (l == mx && n0 + c < am)) {
+        mx = l;
+        am = n0 + c;
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const Acc om = __shfl_xor_sync(0xffffffffu, mx, off);
+      const int oa = __shfl_xor_sync(0xffffffffu, am, off);
+      if (om > mx || (om == mx && oa < am)) {
+        mx = om;
+        am = oa;
+      }
+    }
+    Acc s = 0, u = 0;
+    for (int c = lane; c < SG_BN; c += 32) {
+      if (n0 + c >= V) continue;
+      const Acc z = T[rr][c] - mx, e = dexp(z);
+      s += e;
+      u += e * z;
+    }
+    s = warp_sum(s);
+    u = warp_sum(u);
+    if (lane == 0) {
+      Acc* pp = part + ((size_t)blockIdx.x * n_rows + r) * 4;
+      pp[0] = mx;
+      pp[1] = s;
+      pp[2] = u;
+      pp[3] = (Acc)am;
+    }
+  }
+}
+
+// Merge of per-tile statistics (fixed order and shape), one warp per row:
+//   M = max m_i, S = sum s_i e^(m_i - M),
+//   H = log S - (1/S) sum e^(m_i - M) (u_i + (m_i - M) s_i)   (clamped at 0),
+//   argmax = the id of the first tile (lowest vocab) attaining M.
+template <class Acc>
+__global__ void lm_merge_kernel(const Acc* __restrict__ part, int n_vt, int n_rows,
+                                float* __restrict__ H, int32_t* __restrict__ amax) {
+  const int lane = threadIdx.x & 31;
+  const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (r >= n_rows) return;
+  Acc M = -INFINITY;
+  Acc best_id = 0;
+  for (int i = lane; i < n_vt; i += 32) {
+    const Acc* p = part + ((size_t)i * n_rows + r) * 4;
+    if (p[0] > M) {
+      M = p[0];
+      best_id = p[3];
+    }
+  }
+  for (int off = 16; off > 0; off >>= 1) {
+    const Acc om = __shfl_xor_sync(0xffffffffu, M, off);
+    const Acc oi = __shfl_xor_sync(0xffffffffu, best_id, off);
+    if (om > M || (om == M && oi < best_id)) {
+      M = om;
+      best_id = oi;
+    }
+  }
+  Acc S = 0, U = 0;
+  for (int i = lane; i < n_vt; i += 32) {
+    const Acc* p = part + ((size_t)i * n_rows + r) * 4;
+    const Acc w = dexp(p[0] - M);
+    S += p[1] * w;
+    U += w * (p[2] + (p[0] - M) * p[1]);
+  }
+  S = warp_sum(S);
+  U = warp_sum(U);
+  if (lane == 0) {
+    Acc h = dlog(S) - U / S;
+    if (!(h > Acc(0))) h = 0;
+    H[r] = (float)h;
+    amax[r] = (int32_t)best_id;
+  }
+}
+
+template <class T>
+__global__ void to_f32_kernel(const T* __restrict__ src, float* __restrict__ dst, long n) {
+  const long i = blockIdx.x * (long)blockDim.x + threadIdx.x;
+  if (i < n) dst[i] = (float)widen(src[i]);
+}
+
+__global__ void fill_i32_kernel(int32_t* __restrict__ p, int n, int32_t v) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) p[i] = v;
+}
+
+}  // namespace dg

@@ -72,3 +72,19 @@ def prompt(w: Workload, device="cpu") -> torch.Tensor:
 
 def is_fp8_expert(w: Workload, name: str) -> bool:
     return w.dtype == "bf16_fp8exp" and name.split(".")[-1] in ("gate", "up", "down")
+
+
+def weight_set(w: Workload, device="cpu") -> dict:
+    """Every weight tensor of the workload, keyed by name, in its stored dtype."""
+    dt = torch.float32 if store_dtype(w) == "f32" else torch.bfloat16
+    out = {}
+    for name, shape in all_specs(w):
+        if is_fp8_expert(w, name):
+            from . import fp8
+            q, s = fp8.quantised(w, name, shape, device)
+            out[name], out[name.rsplit(".", 1)[0] + "." + name.split(".")[-1] + "_scale"] = q, s
+            continue
+        t = torch.empty(shape, dtype=dt, device=device)
+        gen.fill_weight_(t, w.seed, name, w.init_std)
+        out[name] = t
+    return out

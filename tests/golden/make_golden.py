@@ -1,0 +1,63 @@
+"""Writes the oracle's expected outputs for the full-size workloads to tests/golden/.
+
+Calls only `oracle/` and `synth/` (never the CUDA path).  Usage:
+    python tests/golden/make_golden.py layer1-bf16 [full30-bf16 ...]
+Each file <workload>.npz holds, for canvas 0 of the workload's first forward
+(all [MASK], steps_left = T):
+  H [C] fp32 entropies, H64 [C], argmax [C], margin [C] (top-1 minus top-2 logit),
+  lse [C]; logit_rows [R] row ids and logit_cols [Vs] vocab ids with
+  logits [R, Vs]; kv_last [L?, 2, Hkv, 8, h] post-RoPE keys / values of the last 8
+  prompt positions of layers 0 and L-1; router margins per layer (min over rows of
+  the gap between the k-th and (k+1)-th router logits); the sampler step's canvas,
+  mask and count on these entropies.
+"""
+from __future__ import annotations
+
+import os
+import sys
+import time
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, os.path.dirname(os.path.dirname(HERE)))
+
+from oracle import model as om  # noqa: E402
+from oracle import sampler as osamp  # noqa: E402
+from synth import model_inputs, workloads  # noqa: E402
+
+LOGIT_ROWS = [0, 1, 77, 128, 255]
+
+
+def make(name: str):
+    w = workloads.get(name)
+    t0 = time.time()
+    ws = om.Weights(w, keep_layers=False)
+    prompt = model_inputs.prompt(w)[0].numpy()
+    canvas = np.full(w.canvas, w.mask_id)
+    st = om.prefill_then_forward(ws, prompt, canvas, w.T, w.T, want_logits=True)
+    cols = np.arange(0, w.vocab, max(1, w.vocab // 4096))
+    rows = [r for r in LOGIT_ROWS if r < w.canvas]
+    kv_last = np.stack([np.stack([st["kv"][l][0][-8:].transpose(1, 0, 2),
+                                  st["kv"][l][1][-8:].transpose(1, 0, 2)])
+                        for l in sorted({0, w.n_layers - 1})])
+    rmarg = []
+    for idx, g, rl in st["routes"]:
+        srt = np.sort(rl, axis=1)[:, ::-1]
+        rmarg.append((srt[:, w.top_k - 1] - srt[:, w.top_k]).min())
+    c2, m2, n2, kg = osamp.eb_step(st["H"], st["argmax"], canvas, np.ones(w.canvas, np.uint8),
+                                   w.T, w.gamma)
+    out = os.path.join(HERE, f"{name}.npz")
+    np.savez_compressed(out, H=st["H"], H64=st["H64"], argmax=st["argmax"], margin=st["margin"],
+                        lse=st["lse"], logit_rows=np.array(rows), logit_cols=cols,
+                        logits=st["logits"][rows][:, cols].astype(np.float64), kv_last=kv_last,
+                        router_margin=np.array(rmarg), step_canvas=c2, step_mask=m2,
+                        step_n=np.array(n2), step=np.array(w.T))
+    print(f"{name}: wrote {out} in {time.time() - t0:.0f} s; H range "
+          f"[{st['H'].min():.4f}, {st['H'].max():.4f}], min margin {st['margin'].min():.4g}, "
+          f"min router gap {min(rmarg):.3g}, sampler n {n2}")
+
+
+if __name__ == "__main__":
+    for n in sys.argv[1:] or ["layer1-bf16"]:
+        make(n)

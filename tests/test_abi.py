@@ -1,0 +1,61 @@
+"""The C-ABI library builds, loads and exports every entry point include/*.h declares;
+host-side argument validation rejects bad calls before touching the device."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+from masked_discrete_diffusion_b200 import binding, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return binding.lib()
+
+
+def declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        names |= set(re.findall(r"^\s*(?:const\s+)?[\w]+\s*\*?\s*(dg_\w+)\s*\(", src, flags=re.M))
+    return sorted(names)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    assert lib.dg_status_str(0) == b"DG_OK"
+    assert lib.dg_status_str(1) == b"DG_ERR_INVALID_ARG"
+    assert lib.dg_status_str(5) == b"DG_ERR_TIMEOUT"
+
+
+def test_host_validation_without_device(lib):
+    vp = ctypes.c_void_p
+    # null pointers and bad scalars are rejected before any CUDA call
+    assert lib.dg_eb_sample(None, None, None, None, 1, 8, 1, 1.0, None, None) == 1
+    fake = vp(16)
+    assert lib.dg_eb_sample(fake, fake, fake, fake, 1, 8, 0, 1.0, None, None) == 1   # steps 0
+    assert lib.dg_eb_sample(fake, fake, fake, fake, 1, 2048, 1, 1.0, None, None) == 1
+    assert lib.dg_eb_sample(fake, fake, fake, fake, 1, 8, 1, float("nan"), None, None) == 1
+    assert lib.dg_eb_sample(fake, fake, fake, fake, 1, 8, 1, -0.5, None, None) == 1
+    assert b"gamma" in lib.dg_last_error()
+    out = vp()
+    assert lib.dg_model_create(None, None, ctypes.byref(out)) == 1
+    cfg = binding.dg_config(n_layers=1, d_model=64, n_q_heads=3, n_kv_heads=2, head_dim=16,
+                            n_experts=8, top_k=2, expert_inter=8, shared_inter=8, vocab=16,
+                            window=4, canvas=8, rope_base=1e4, rms_eps=1e-6, logit_scale=8,
+                            dtype=0, max_batch=1, max_prompt=8)
+    w = binding.dg_weights()
+    assert lib.dg_model_create(ctypes.byref(cfg), ctypes.byref(w), ctypes.byref(out)) == 1
+    assert b"multiple" in lib.dg_last_error()
+    assert lib.dg_model_destroy(None) == 0 and lib.dg_kv_destroy(None) == 0
