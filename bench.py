@@ -1,0 +1,334 @@
+#!/usr/bin/env python
+"""Throughput of block-parallel canvas denoising on B200.
+
+One step = one 256-token block per canvas: `dg_generate_block` runs T denoise
+forwards (all layers, LM head with online entropy, EB sampler) from an all
+[MASK] canvas.  Metric: canvas tokens per second = canvases x 256 / block time.
+Default workload: the 30-layer stand-in, batch 1, prompt 1024 (prefilled once),
+T = 12, gamma = 1.0.  Weights (40 GB) exceed L2, so no flush is needed.
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Multi-GPU: one process per GPU (torchrun); every rank denoises its own canvases
+(weak scaling, no collective on the data path); time = max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms in the background."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.p = None
+
+    def start(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--id={self.index}",
+                                       f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                       "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.p.terminate()
+        self.p.wait()
+        self.f.seek(0)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.f.read().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.f.name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+def dist_setup():
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the oracle, as it stands, on a bounded sample of the workload
+# ---------------------------------------------------------------------------
+class OracleSample:
+    """The oracle's canvas forward on layer 0 and on 1/vocab_frac of the LM head, one
+    canvas, scaled to a block (T forwards of all layers); weights generated once."""
+
+    def __init__(self, w, vocab_frac: int = 16):
+        import numpy as np
+
+        from oracle import model as om
+        from synth import model_inputs
+        self.om, self.w, self.vf = om, w, vocab_frac
+        self.ws = om.Weights(w, keep_layers=True)
+        self.lw = self.ws.layer(0)
+        prompt = model_inputs.prompt(w.with_(batch=1))[0].numpy()
+        P = len(prompt)
+        empty = np.zeros((0, w.n_kv_heads, w.head_dim))
+        _, k, v, _ = om.decoder_layer(om.embed(self.ws, prompt), np.arange(P), self.lw,
+                                      (empty, empty), om.causal_window_mask(P, w.window), w)
+        W = min(P, w.window)
+        self.kv = (k[P - W:], v[P - W:])
+        self.x = om.canvas_input(self.ws, np.full(w.canvas, w.mask_id), w.T, w.T)
+        self.Wl = self.ws.rows("lm_head", (w.vocab, w.d_model), 0, w.vocab // vocab_frac)
+
+    def run(self):
+        from threadpoolctl import threadpool_info
+        om, w = self.om, self.w
+        t0 = time.perf_counter()
+        x1, _, _, _ = om.canvas_layer(self.x, self.lw, self.kv, w.prompt_len, w)
+        t_layer = time.perf_counter() - t0
+        t0 = time.perf_counter()
+        om.entropy_stats(w.logit_scale * (om.rmsnorm(x1, w.rms_eps) @ self.Wl.T))
+        t_lm = time.perf_counter() - t0
+        fwd = w.n_layers * t_layer + self.vf * t_lm
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+        desc = (f"oracle canvas forward of layer 0 ({t_layer:.2f} s, x{w.n_layers} layers) and "
+                f"LM head over 1/{self.vf} of the vocabulary ({t_lm:.2f} s, x{self.vf}), "
+                f"one canvas, scaled to a block of {w.T} forwards x {w.batch} canvases; "
+                f"weight generation excluded")
+        return fwd * w.T * w.batch, desc, threads
+
+
+def run_reference(args, w, world, rank):
+    if rank != 0:
+        return
+    times = []
+    desc, threads = "", 1
+    smp = OracleSample(w)
+    for _ in range(args.warmup):
+        smp.run()
+    for _ in range(args.steps):
+        t, desc, threads = smp.run()
+        times.append(t)
+    block = statistics.mean(times)
+    val = w.batch * w.canvas / block
+    line = {"impl": "reference", "metric": "canvas tokens/sec at 1 B200 (256-tok block)",
+            "value": val, "unit": "canvas tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": block * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "batch": w.batch, "canvas": w.canvas,
+                       "prompt": w.prompt_len, "layers": w.n_layers, "T": w.T},
+            "cpu_baseline": {"value": val, "unit": "canvas tokens/s", "cores": threads,
+                             "kind": "oracle", "sample": desc},
+            "e2e": {"value": val, "unit": "canvas tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# our path
+# ---------------------------------------------------------------------------
+def run_ours(args, w, world, rank, local):
+    import numpy as np
+    import torch
+
+    from masked_discrete_diffusion_b200 import binding, build, metrics
+    from synth import model_inputs
+
+    build.build()
+    peaks, peak_src = load_peaks()
+    tensors = model_inputs.weight_set(w, "cuda")
+    model = binding.Model(binding.make_config(w), tensors)
+    prompt = model_inputs.prompt(w, "cuda", first=rank * w.batch)
+    kv = binding.dg_prefill(model, prompt)
+    binding.dg_sync_status(model)
+    B, C, T = w.batch, w.canvas, w.T
+    canvas = torch.empty(B, C, dtype=torch.int32, device="cuda")
+    nfwd = torch.zeros(B, dtype=torch.int32, device="cuda")
+    load = torch.zeros(w.n_layers, w.n_experts, dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    for _ in range(args.warmup):
+        binding.dg_generate_block(model, kv, T, w.gamma, canvas, nfwd, load)
+    binding.dg_sync_status(model)
+    barrier(world)
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    n0 = binding.dg_launch_count(model)
+    binding.dg_profile_start(model)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        binding.dg_generate_block(model, kv, T, w.gamma, canvas, nfwd, load)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    prof = binding.dg_profile_stop(model)
+    launches = binding.dg_launch_count(model) - n0
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    binding.dg_sync_status(model)
+    barrier(world)
+    ms_max = max_over_ranks(ms, world)
+    value = world * B * C * args.steps / (ms_max / 1e3)
+    ms_step = ms_max / args.steps
+    assert not bool((canvas == w.mask_id).any()), "a [MASK] survived the block"
+
+    # end to end through the public API: pinned prompt -> prefill -> block -> canvas to host
+    h_prompt = prompt.cpu().pin_memory()
+    h_canvas = torch.empty(B, C, dtype=torch.int32).pin_memory()
+    d_prompt = torch.empty_like(prompt)
+    kv.close()
+    torch.cuda.synchronize()
+    barrier(world)
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(args.steps):
+        d_prompt.copy_(h_prompt, non_blocking=True)
+        kv2 = binding.dg_prefill(model, d_prompt)
+        binding.dg_generate_block(model, kv2, T, w.gamma, canvas)
+        h_canvas.copy_(canvas, non_blocking=True)
+        f1.record(stream)
+        f1.synchronize()
+        kv2.close()
+    f1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1), world)
+    e2e_val = world * B * C * args.steps / (e2e_ms / 1e3)
+
+    # roofline of the dominant kernel group (routed-expert FFN)
+    load_np = load.cpu().numpy()
+    unique = [int((load_np[l] > 0).sum()) for l in range(w.n_layers)]
+    cost = metrics.forward_cost(model.cfg, B, kv.W, unique)
+    ex_ms, ex_groups = prof["experts"]
+    ex_bytes = statistics.mean(unique) * cost["expert_bytes"]
+    ex_avg_s = ex_ms / 1e3 / max(ex_groups, 1)
+    achieved = ex_bytes / ex_avg_s / 1e9
+    peak = float(peaks["hbm_gbs"])
+    fwd_ms = ms_step / T
+    t_roof = max(cost["bytes"] / (peak * 1e9), cost["flops"] / (float(peaks["bf16_tflops"]) * 1e12))
+    kinds = {k: {"ms_per_step": v[0] / args.steps, "groups_per_step": v[1] / args.steps}
+             for k, v in prof.items()}
+
+    line = {
+        "metric": "canvas tokens/sec at 1 B200 (256-tok block)", "value": value,
+        "unit": "canvas tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded random-init weights N(0,0.02), uniform prompt tokens)",
+        "config": {"workload": w.name, "batch": B, "canvas": C, "prompt": w.prompt_len,
+                   "layers": w.n_layers, "T": T, "gamma": w.gamma,
+                   "l2": "inputs larger than L2 (40 GB of weights streamed per forward)",
+                   "parallelism": f"replicas x{world}"},
+        "ms_per_forward": fwd_ms,
+        "tokens_per_forward": C / T,
+        "forward_roofline": {"ms": t_roof * 1e3, "frac": t_roof * 1e3 / fwd_ms,
+                             "alg_bytes": cost["bytes"], "alg_flops": cost["flops"],
+                             "peak_src": peak_src},
+        "roofline": {"kernel": "routed-expert FFN (gate/up SwiGLU + down) per layer",
+                     "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "alg_bytes_per_launch": ex_bytes, "avg_launch_ms": ex_avg_s * 1e3,
+                     "peak_src": f"{peak_src} hbm_gbs"},
+        "kernel_groups": kinds,
+        "gpu_launches": launches,
+        "clocks": clk,
+        "e2e": {"value": e2e_val, "unit": "canvas tokens/s",
+                "h2d_bytes_per_step": int(prompt.numel() * 4),
+                "d2h_bytes_per_step": int(canvas.numel() * 4),
+                "includes": "prompt H2D, dg_prefill, dg_generate_block, canvas D2H"},
+        "unique_experts_per_layer": statistics.mean(unique),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        t_block, desc, threads = OracleSample(w).run()
+        line["cpu_baseline"] = {"value": B * C / t_block, "unit": "canvas tokens/s",
+                                "cores": threads, "kind": "oracle", "sample": desc}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    model.close()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="full30-bf16")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    from synth import workloads
+    w = workloads.get(args.workload)
+    world, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            run_reference(args, w, world, rank)
+        else:
+            run_ours(args, w, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

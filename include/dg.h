@@ -189,6 +189,28 @@ dg_status dg_debug_forward(dg_model* m, const dg_kv* kv, const int32_t* canvas,
  * (k, v: [n_layers, B, Hkv, W, h] of the cache's element type). */
 dg_status dg_kv_read(const dg_kv* kv, void* k, void* v, void* stream);
 
+/* ---- measurement hooks (no counterpart on the pages) -------------------------
+ * Kernel groups whose device time can be recorded while the path runs. */
+typedef enum dg_kernel_kind {
+  DG_KIND_EXPERTS = 0,   /* routed-expert FFN: gate/up (SwiGLU) and down launches */
+  DG_KIND_LMHEAD = 1,    /* LM-head GEMM + online entropy statistics (+ merge)   */
+  DG_KIND_ATTENTION = 2, /* canvas / prompt attention                           */
+  DG_KIND_DENSE = 3,     /* QKV, O and shared-expert projections                */
+  DG_KIND_COUNT = 4
+} dg_kernel_kind;
+
+/* Starts recording a pair of CUDA events around every launch group of each
+ * kind, on the stream the launches use.  Costs one event record per launch. */
+dg_status dg_profile_start(dg_model* m);
+
+/* Synchronises the device, writes the summed device milliseconds
+ * (ms[DG_KIND_COUNT]) and the number of recorded launch groups
+ * (groups[DG_KIND_COUNT]) since dg_profile_start, and stops recording. */
+dg_status dg_profile_stop(dg_model* m, float* ms, int64_t* groups);
+
+/* Number of kernels this model has launched since it was created (host count). */
+dg_status dg_launch_count(const dg_model* m, int64_t* out);
+
 #ifdef __cplusplus
 }
 #endif

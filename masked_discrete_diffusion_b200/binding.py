@@ -77,6 +77,9 @@ def lib() -> ctypes.CDLL:
             "dg_generate_block": [vp, vp, i32, f32, vp, vp, vp, vp],
             "dg_eb_sample": [vp, vp, vp, vp, i32, i32, i32, f32, vp, vp],
             "dg_debug_forward": [vp, vp, vp, i32, i32, vp, vp, vp, vp, vp],
+            "dg_profile_start": [vp],
+            "dg_profile_stop": [vp, vp, vp],
+            "dg_launch_count": [vp, ctypes.POINTER(ctypes.c_int64)],
         }
         for name, args in sigs.items():
             fn = getattr(L, name)
@@ -90,7 +93,8 @@ def exported_symbols():
     return [n for n in ("dg_status_str", "dg_last_error", "dg_model_create", "dg_model_destroy",
                         "dg_sync_status", "dg_prefill", "dg_kv_destroy", "dg_kv_info",
                         "dg_kv_read", "dg_denoise_step", "dg_generate_block", "dg_eb_sample",
-                        "dg_debug_forward") if hasattr(lib(), n)]
+                        "dg_debug_forward", "dg_profile_start", "dg_profile_stop",
+                        "dg_launch_count") if hasattr(lib(), n)]
 
 
 def _check(status: int):
@@ -242,3 +246,24 @@ def dg_debug_forward(model: Model, kv: KV, canvas, steps_left: int, T: int, logi
     _check(lib().dg_debug_forward(model.handle, kv.handle, _ptr(canvas), steps_left, T,
                                   _ptr(ent), _ptr(am), _ptr(lg), _ptr(hd), _stream(stream)))
     return ent, am, lg, hd
+
+
+KINDS = ("experts", "lmhead", "attention", "dense")
+
+
+def dg_profile_start(model: Model):
+    _check(lib().dg_profile_start(model.handle))
+
+
+def dg_profile_stop(model: Model) -> dict:
+    """{kind: (device ms summed, launch groups)} since dg_profile_start."""
+    ms = (ctypes.c_float * len(KINDS))()
+    groups = (ctypes.c_int64 * len(KINDS))()
+    _check(lib().dg_profile_stop(model.handle, ms, groups))
+    return {k: (float(ms[i]), int(groups[i])) for i, k in enumerate(KINDS)}
+
+
+def dg_launch_count(model: Model) -> int:
+    out = ctypes.c_int64()
+    _check(lib().dg_launch_count(model.handle, ctypes.byref(out)))
+    return out.value

@@ -161,9 +161,11 @@ template <class Path> static dg_status alloc_workspace(dg_model* m) {
 // ---------------------------------------------------------------------------
 template <class TA, class TW, class Acc, bool G, bool D, class Epi>
 static void gemm_simt(const TA* A, int lda, const TW* W, const TW* W2, int ldw, int M, int N,
-                      int K, GroupInfo g, int grid_y, Epi epi, cudaStream_t st) {
+                      int K, GroupInfo g, int grid_y, Epi epi, cudaStream_t st,
+                      long long* count) {
   dim3 grid(ceil_div(N, SG_BN), G ? grid_y : ceil_div(M, SG_BM));
   gemm_simt_kernel<TA, TW, Acc, G, D, Epi><<<grid, 256, 0, st>>>(A, lda, W, W2, ldw, M, N, K, g, epi);
+  ++*count;
 }
 
 template <class Path> struct Runner {
@@ -184,13 +186,14 @@ template <class Path> struct Runner {
 
   void rmsnorm(int n) {
     rmsnorm_kernel<TR, TA, Acc><<<n, 256, 0, st>>>(x(), xn(), n, c.d_model, c.rms_eps);
+    ++m->launches;
   }
 
   // y[n, N] (+)= xn W^T  with W [N, K]
   template <class Epi> void dense(const TA* A, int lda, const void* W, int N, int K, int n,
                                   Epi epi) {
     gemm_simt<TA, TW, Acc, false, false>(A, lda, (const TW*)W, nullptr, K, n, N, K, GroupInfo(),
-                                         0, epi, st);
+                                         0, epi, st, &m->launches);
   }
 
   // One decoder layer on n tokens = B_ * n_seq rows at positions pos0 + i.
@@ -200,14 +203,19 @@ template <class Path> struct Runner {
     const int d = c.d_model, h = c.head_dim, Hq = c.n_q_heads, Hkv = c.n_kv_heads;
     const int qkv_n = (Hq + 2 * Hkv) * h;
     rmsnorm(n);
-    if constexpr (Path::kTensorCores)
-      DG_TRY(tc_gemm_store_f32(m, xn(), L.wqkv, (float*)ws.qkv, n, qkv_n, d, st));
-    else
-      dense(xn(), d, L.wqkv, qkv_n, d, n, EpiStore<Acc, Acc>{(Acc*)ws.qkv, qkv_n});
+    {
+      ProfScope ps(m, DG_KIND_DENSE, st);
+      if constexpr (Path::kTensorCores)
+        DG_TRY(tc_gemm_store_f32(m, xn(), L.wqkv, (float*)ws.qkv, n, qkv_n, d, st));
+      else
+        dense(xn(), d, L.wqkv, qkv_n, d, n, EpiStore<Acc, Acc>{(Acc*)ws.qkv, qkv_n});
+    }
     rope_scatter_kernel<Acc, TA, TKV><<<n, 128, 0, st>>>(
         (const Acc*)ws.qkv, (TA*)ws.q, (TKV*)ws.kc, (TKV*)ws.vc, n, n_seq, pos0, Hq, Hkv, h,
         (const Acc*)ws.rope, ws.max_pos);
+    ++m->launches;
     {
+      ProfScope ps(m, DG_KIND_ATTENTION, st);
       const long warps = (long)n * Hq;
       const int blocks = ceil_div(warps, 4);
       const TKV* kB = (const TKV*)ws.kc;
@@ -220,12 +228,16 @@ template <class Path> struct Runner {
       else if (h <= 64) DG_ATTN(2);
       else if (h <= 96) DG_ATTN(3);
       else DG_ATTN(4);
+      ++m->launches;
 #undef DG_ATTN
     }
-    if constexpr (Path::kTensorCores)
-      DG_TRY(tc_gemm_add_residual(m, (const TA*)ws.o, L.wo, (float*)x(), n, d, Hq * h, st));
-    else
-      dense((const TA*)ws.o, Hq * h, L.wo, d, Hq * h, n, EpiAddResidual<TR, Acc>{x(), d});
+    {
+      ProfScope ps(m, DG_KIND_DENSE, st);
+      if constexpr (Path::kTensorCores)
+        DG_TRY(tc_gemm_add_residual(m, (const TA*)ws.o, L.wo, (float*)x(), n, d, Hq * h, st));
+      else
+        dense((const TA*)ws.o, Hq * h, L.wo, d, Hq * h, n, EpiAddResidual<TR, Acc>{x(), d});
+    }
     DG_TRY(moe(l, n, load));
     return check_launch("decoder layer");
   }
@@ -237,21 +249,30 @@ template <class Path> struct Runner {
     const int n_ent = n * k;
     router_kernel<TR, TW, Acc><<<n, 256, E * sizeof(Acc), st>>>(
         x(), (const TW*)L.router, n, d, E, k, c.rms_eps, ws.ridx, (Acc*)ws.rgate, load);
+    ++m->launches;
     moe_rank_kernel<<<E, 256, 0, st>>>(ws.ridx, n_ent, ws.rank, ws.counts);
+    ++m->launches;
     int bm = SG_BM;
     if constexpr (Path::kTensorCores) bm = tc_group_rows();
     moe_offsets_kernel<<<1, 32, 0, st>>>(ws.counts, E, bm, ws.offsets, ws.tile_e, ws.tile_m0,
                                          ws.n_tiles, ws.max_tiles);
+    ++m->launches;
     moe_scatter_kernel<Acc><<<ceil_div(n_ent, 256), 256, 0, st>>>(
         ws.ridx, (const Acc*)ws.rgate, ws.rank, ws.offsets, n_ent, k, ws.row_of, ws.tok_of,
         (Acc*)ws.gate_of);
+    ++m->launches;
     rmsnorm(n);  // u = RMSNorm(x) after attention
     gather_rows_kernel<TA><<<n_ent, 256, 0, st>>>(xn(), ws.tok_of, ws.offsets + E, d,
                                                   (TA*)ws.up);
+    ++m->launches;
     const int grid_y = ceil_div(n_ent, bm) + E;
     if constexpr (Path::kTensorCores) {
-      DG_TRY(tc_moe_gate_up(m, l, (const TA*)ws.up, (TA*)ws.hb, grid_y, st));
-      DG_TRY(tc_moe_down(m, l, (const TA*)ws.hb, (float*)ws.yb, grid_y, st));
+      {
+        ProfScope ps(m, DG_KIND_EXPERTS, st);
+        DG_TRY(tc_moe_gate_up(m, l, (const TA*)ws.up, (TA*)ws.hb, grid_y, st));
+        DG_TRY(tc_moe_down(m, l, (const TA*)ws.hb, (float*)ws.yb, grid_y, st));
+      }
+      ProfScope ps(m, DG_KIND_DENSE, st);
       DG_TRY(tc_gemm_swiglu(m, xn(), L.sgate, L.sup, (TA*)ws.sh, n, Is, d, st));
       DG_TRY(tc_gemm_store_f32(m, (const TA*)ws.sh, L.sdown, (float*)ws.ys, n, d, Is, st));
     } else {
@@ -261,19 +282,23 @@ template <class Path> struct Runner {
       g.n_tiles = ws.n_tiles;
       g.offsets = ws.offsets;
       g.w_slab = (size_t)I * d;
+      ProfScope pe(m, DG_KIND_EXPERTS, st);
       gemm_simt<TA, TW, Acc, true, true>((const TA*)ws.up, d, (const TW*)L.gate,
                                          (const TW*)L.up, d, n_ent, I, d, g, grid_y,
-                                         EpiSwiglu<TA, Acc>{(TA*)ws.hb, I}, st);
+                                         EpiSwiglu<TA, Acc>{(TA*)ws.hb, I}, st, &m->launches);
       gemm_simt<TA, TW, Acc, true, false>(
           (const TA*)ws.hb, I, (const TW*)L.down, nullptr, I, n_ent, d, I, g, grid_y,
-          EpiRowScale<Acc, Acc>{(Acc*)ws.yb, d, (const Acc*)ws.gate_of}, st);
+          EpiRowScale<Acc, Acc>{(Acc*)ws.yb, d, (const Acc*)ws.gate_of}, st, &m->launches);
+      pe.end();
+      ProfScope pd(m, DG_KIND_DENSE, st);
       gemm_simt<TA, TW, Acc, false, true>(xn(), d, (const TW*)L.sgate, (const TW*)L.sup, d, n,
                                           Is, d, GroupInfo(), 0,
-                                          EpiSwiglu<TA, Acc>{(TA*)ws.sh, Is}, st);
+                                          EpiSwiglu<TA, Acc>{(TA*)ws.sh, Is}, st, &m->launches);
       dense((const TA*)ws.sh, Is, L.sdown, d, Is, n, EpiStore<Acc, Acc>{(Acc*)ws.ys, d});
     }
     moe_combine_kernel<TR, Acc, Acc><<<n, 256, 0, st>>>(x(), (const Acc*)ws.ys,
                                                         (const Acc*)ws.yb, ws.row_of, n, d, k);
+    ++m->launches;
     return check_launch("moe");
   }
 
@@ -284,6 +309,7 @@ template <class Path> struct Runner {
     for (int b = 0; b < B; ++b) {
       embed_kernel<TW, TR><<<P, 256, 0, st>>>(prompt + (size_t)b * P, (const TW*)m->w.tok_emb,
                                              x(), P, d, c.vocab - 1, -1.0, ws.err);
+      ++m->launches;
       for (int l = 0; l < c.n_layers; ++l) {
         DG_TRY(layer(l, P, 1, P, 0, nullptr, nullptr, 0, 0, true, nullptr));
         // keys/values of positions P-W .. P-1 -> cache [l, b, hkv, W, h]
@@ -307,6 +333,7 @@ template <class Path> struct Runner {
     const double tau = (double)s / (double)T;
     embed_kernel<TW, TR><<<n, 256, 0, st>>>(canvas, (const TW*)m->w.tok_emb, x(), n, d, c.vocab,
                                            tau, ws.err);
+    ++m->launches;
     const size_t lstride = (size_t)B * c.n_kv_heads * kv->W * c.head_dim;
     for (int l = 0; l < c.n_layers; ++l) {
       const TKV* kA = (const TKV*)kv->k + l * lstride;
@@ -315,7 +342,9 @@ template <class Path> struct Runner {
                    load ? load + (size_t)l * c.n_experts : nullptr));
     }
     if (hidden) to_f32_kernel<TR><<<ceil_div((long)n * d, 256), 256, 0, st>>>(x(), hidden, (long)n * d);
+    ++m->launches;
     rmsnorm(n);
+    ProfScope ps(m, DG_KIND_LMHEAD, st);
     bool done = false;
     if constexpr (Path::kTensorCores) {
       if (logits == nullptr) {
@@ -328,8 +357,10 @@ template <class Path> struct Runner {
       lmhead_simt_kernel<TA, TW, Acc><<<grid, 256, 0, st>>>(xn(), (const TW*)m->w.lm_head, n,
                                                            c.vocab, d, c.logit_scale,
                                                            (Acc*)ws.lm_part, logits);
+      ++m->launches;
       lm_merge_kernel<Acc><<<ceil_div(n, 4), 128, 0, st>>>((const Acc*)ws.lm_part, ws.n_vtiles,
                                                           n, ent, amax);
+      ++m->launches;
     }
     return check_launch("forward");
   }
@@ -358,7 +389,7 @@ static dg_status gamma_fixed(float gamma, long long* out) {
 static dg_status launch_sampler(const float* H, const int32_t* am, int32_t* canvas,
                                 uint8_t* mask, int B, int C, int s, long long gq,
                                 int32_t* ncommit, int32_t* nfwd, int step_no,
-                                cudaStream_t st) {
+                                cudaStream_t st, long long* counter_) {
 #define DG_SAMP(NP)                                                                       \
   eb_sample_kernel<NP><<<B, NP, 0, st>>>(H, am, canvas, mask, C, s, gq, ncommit, nfwd, \
                                          step_no)
@@ -368,6 +399,7 @@ static dg_status launch_sampler(const float* H, const int32_t* am, int32_t* canv
   else if (C <= 256) DG_SAMP(256);
   else if (C <= 512) DG_SAMP(512);
   else DG_SAMP(1024);
+  if (counter_) ++*counter_;
 #undef DG_SAMP
   return check_launch("eb sampler");
 }
@@ -441,6 +473,11 @@ dg_status dg_model_create(const dg_config* cfg, const dg_weights* w, dg_model** 
 dg_status dg_model_destroy(dg_model* m) {
   if (!m) return DG_OK;
   cudaDeviceSynchronize();
+  for (int k = 0; k < DG_KIND_COUNT; ++k)
+    for (auto& e : m->prof[k]) {
+      cudaEventDestroy(e.first);
+      cudaEventDestroy(e.second);
+    }
   tc_release(m);
   ws_free(m->ws);
   delete m;
@@ -559,7 +596,7 @@ dg_status dg_denoise_step(dg_model* m, const dg_kv* kv, int32_t* canvas, uint8_t
   cudaStream_t st = (cudaStream_t)stream;
   DG_TRY(run_forward(m, kv, canvas, steps_left, T, entropy, argmax, nullptr, nullptr, nullptr, st));
   return launch_sampler(entropy, argmax, canvas, mask, kv->B, m->cfg.canvas, steps_left, gq,
-                        n_committed, nullptr, 0, st);
+                        n_committed, nullptr, 0, st, &m->launches);
 }
 
 dg_status dg_generate_block(dg_model* m, const dg_kv* kv, int32_t T, float gamma,
@@ -575,6 +612,7 @@ dg_status dg_generate_block(dg_model* m, const dg_kv* kv, int32_t T, float gamma
   const int B = kv->B, C = c.canvas;
   Workspace& ws = m->ws;
   fill_i32_kernel<<<ceil_div((long)B * C, 256), 256, 0, st>>>(canvas_out, B * C, c.vocab);
+  ++m->launches;
   DG_TRY_CUDA(cudaMemsetAsync(ws.mask, 1, (size_t)B * C, st));
   if (n_forwards) DG_TRY_CUDA(cudaMemsetAsync(n_forwards, 0, B * sizeof(int32_t), st));
   if (router_load)
@@ -585,7 +623,7 @@ dg_status dg_generate_block(dg_model* m, const dg_kv* kv, int32_t T, float gamma
     DG_TRY(run_forward(m, kv, canvas_out, s, T, ws.ent, ws.amax, nullptr, nullptr, router_load,
                        st));
     DG_TRY(launch_sampler(ws.ent, ws.amax, canvas_out, ws.mask, B, C, s, gq, ws.ncommit,
-                          n_forwards, k + 1, st));
+                          n_forwards, k + 1, st, &m->launches));
   }
   return DG_OK;
 }
@@ -600,7 +638,38 @@ dg_status dg_eb_sample(const float* entropy, const int32_t* argmax, int32_t* can
   long long gq;
   DG_TRY(gamma_fixed(gamma, &gq));
   return launch_sampler(entropy, argmax, canvas, mask, B, C, steps_left, gq, n_committed,
-                        nullptr, 0, (cudaStream_t)stream);
+                        nullptr, 0, (cudaStream_t)stream, nullptr);
+}
+
+dg_status dg_profile_start(dg_model* m) {
+  DG_REQUIRE(m, "null model");
+  for (int k = 0; k < DG_KIND_COUNT; ++k) m->prof_used[k] = 0;
+  m->profiling = true;
+  return DG_OK;
+}
+
+dg_status dg_profile_stop(dg_model* m, float* ms, int64_t* groups) {
+  DG_REQUIRE(m, "null model");
+  m->profiling = false;
+  DG_TRY_CUDA(cudaDeviceSynchronize());
+  for (int k = 0; k < DG_KIND_COUNT; ++k) {
+    double tot = 0.0;
+    for (size_t i = 0; i < m->prof_used[k]; ++i) {
+      float t = 0.0f;
+      DG_TRY_CUDA(cudaEventElapsedTime(&t, m->prof[k][i].first, m->prof[k][i].second));
+      tot += t;
+    }
+    if (ms) ms[k] = (float)tot;
+    if (groups) groups[k] = (int64_t)m->prof_used[k];
+    m->prof_used[k] = 0;
+  }
+  return DG_OK;
+}
+
+dg_status dg_launch_count(const dg_model* m, int64_t* out) {
+  DG_REQUIRE(m && out, "null argument");
+  *out = m->launches;
+  return DG_OK;
 }
 
 dg_status dg_debug_forward(dg_model* m, const dg_kv* kv, const int32_t* canvas,

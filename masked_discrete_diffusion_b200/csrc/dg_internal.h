@@ -82,7 +82,41 @@ struct dg_model {
   std::vector<dg_layer_weights> layers;
   int device = 0;
   dg::Workspace ws;
+  long long launches = 0;  // kernels launched (host count)
+  // event recording around launch groups, per dg_kernel_kind
+  bool profiling = false;
+  std::vector<std::pair<cudaEvent_t, cudaEvent_t>> prof[DG_KIND_COUNT];
+  size_t prof_used[DG_KIND_COUNT] = {0, 0, 0, 0};
 };
+
+namespace dg {
+// RAII bracket recording a start/stop event pair around a launch group.
+struct ProfScope {
+  dg_model* m;
+  int kind;
+  cudaStream_t st;
+  cudaEvent_t stop = nullptr;
+  ProfScope(dg_model* m_, int kind_, cudaStream_t st_) : m(m_), kind(kind_), st(st_) {
+    if (!m->profiling) return;
+    auto& pool = m->prof[kind];
+    size_t& used = m->prof_used[kind];
+    if (used == pool.size()) {
+      cudaEvent_t a, b;
+      cudaEventCreate(&a);
+      cudaEventCreate(&b);
+      pool.push_back({a, b});
+    }
+    cudaEventRecord(pool[used].first, st);
+    stop = pool[used].second;
+    ++used;
+  }
+  void end() {
+    if (stop) cudaEventRecord(stop, st);
+    stop = nullptr;
+  }
+  ~ProfScope() { end(); }
+};
+}  // namespace dg
 
 struct dg_kv {
   dg_model* m = nullptr;

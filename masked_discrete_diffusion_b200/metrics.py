@@ -39,3 +39,34 @@ def canvas_tokens_per_second(batch: int, canvas: int, block_seconds: float) -> f
     """Canvas tokens completed per second when a block of `batch` canvases takes
     `block_seconds` of device time (all of its forwards and sampler steps)."""
     return batch * canvas / block_seconds
+
+
+def forward_cost(cfg, batch: int, window: int, unique_experts=None):
+    """Algorithmic bytes and FLOPs of one canvas forward (all layers + LM head).
+
+    Bytes: weights of the routed experts actually used (unique_experts[l] per layer,
+    all E if None), every dense weight (QKV, O, router, shared expert), the LM head,
+    the embedding rows gathered, and the cached prompt window's keys and values
+    read once.  Intermediate activations and the never-stored logits are not
+    counted.  FLOPs: 2 x multiply-adds of every projection over the B*C canvas
+    rows (k routed experts per row) plus 4 Hq C (W + C) h per layer for attention,
+    plus the LM head.
+    """
+    L, d, h = cfg.n_layers, cfg.d_model, cfg.head_dim
+    Hq, Hkv, E, k = cfg.n_q_heads, cfg.n_kv_heads, cfg.n_experts, cfg.top_k
+    I, Is, V, C = cfg.expert_inter, cfg.shared_inter, cfg.vocab, cfg.canvas
+    wb = 4 if cfg.dtype == 0 else 2
+    ewb = 1 if cfg.dtype == 2 else wb
+    expert_bytes = 3 * I * d * ewb + (3 * I * d // 128 * 4 if cfg.dtype == 2 else 0)
+    qkv = (Hq + 2 * Hkv) * h
+    dense = (qkv * d + d * Hq * h + E * d + 3 * Is * d) * wb
+    if unique_experts is None:
+        unique_experts = [E] * L
+    n = batch * C
+    kv_bytes = L * batch * Hkv * window * h * 2 * (8 if cfg.dtype == 0 else 2)
+    bytes_ = (sum(unique_experts) * expert_bytes + L * dense + V * d * wb + n * d * wb
+              + kv_bytes)
+    flops_layer = 2 * n * (qkv * d + d * Hq * h + E * d + k * 3 * I * d + 3 * Is * d) \
+        + 4 * Hq * C * (window + C) * h * batch
+    flops = L * flops_layer + 2 * n * d * V
+    return {"bytes": float(bytes_), "flops": float(flops), "expert_bytes": float(expert_bytes)}

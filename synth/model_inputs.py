@@ -63,10 +63,10 @@ def weight(w: Workload, name: str, shape, device="cpu", start_row=0, n_rows=None
                       start_row, n_rows)
 
 
-def prompt(w: Workload, device="cpu") -> torch.Tensor:
-    """[B, P] int32 prompt tokens uniform in [0, V)."""
+def prompt(w: Workload, device="cpu", first: int = 0) -> torch.Tensor:
+    """[B, P] int32 prompt tokens uniform in [0, V) for canvases first .. first + B - 1."""
     rows = [gen.tokens(w.seed, f"prompt.b{b}", w.prompt_len, w.vocab, device)
-            for b in range(w.batch)]
+            for b in range(first, first + w.batch)]
     return torch.stack(rows) if rows else torch.empty(0, w.prompt_len, dtype=torch.int32)
 
 
