@@ -80,6 +80,8 @@ def lib() -> ctypes.CDLL:
             "dg_profile_start": [vp],
             "dg_profile_stop": [vp, vp, vp],
             "dg_launch_count": [vp, ctypes.POINTER(ctypes.c_int64)],
+            "dg_op_gemm": [vp, vp, vp, vp, i32, i32, i32, vp],
+            "dg_op_moe": [vp, i32, vp, vp, i32, vp],
         }
         for name, args in sigs.items():
             fn = getattr(L, name)
@@ -94,7 +96,7 @@ def exported_symbols():
                         "dg_sync_status", "dg_prefill", "dg_kv_destroy", "dg_kv_info",
                         "dg_kv_read", "dg_denoise_step", "dg_generate_block", "dg_eb_sample",
                         "dg_debug_forward", "dg_profile_start", "dg_profile_stop",
-                        "dg_launch_count") if hasattr(lib(), n)]
+                        "dg_launch_count", "dg_op_gemm", "dg_op_moe") if hasattr(lib(), n)]
 
 
 def _check(status: int):
@@ -267,3 +269,19 @@ def dg_launch_count(model: Model) -> int:
     out = ctypes.c_int64()
     _check(lib().dg_launch_count(model.handle, ctypes.byref(out)))
     return out.value
+
+
+def dg_op_gemm(model: Model, A, W, stream=None):
+    """out[M, N] = A[M, K] W[N, K]^T (fp32) on the path's GEMM kernel."""
+    M, K = A.shape
+    N = W.shape[0]
+    out = torch.empty(M, N, dtype=torch.float32, device="cuda")
+    _check(lib().dg_op_gemm(model.handle, _ptr(A), _ptr(W), _ptr(out), M, N, K, _stream(stream)))
+    return out
+
+
+def dg_op_moe(model: Model, layer: int, x, stream=None):
+    """x + MoE_layer(RMSNorm(x)) for fp32 rows x [n, d]."""
+    out = torch.empty_like(x)
+    _check(lib().dg_op_moe(model.handle, layer, _ptr(x), _ptr(out), x.shape[0], _stream(stream)))
+    return out

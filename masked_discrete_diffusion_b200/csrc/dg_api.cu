@@ -13,6 +13,7 @@
 #include <cstring>
 
 #include "dg_internal.h"
+#include "../../include/dg_ops.h"
 #include "k_sampler.cuh"
 #include "k_simt.cuh"
 #include "k_tc_gemm.cuh"
@@ -50,7 +51,7 @@ struct PathTiny {  // fp32 weights, fp64 activations and sums
 struct PathBF16 {  // bf16 weights/activations, fp32 residual and sums
   typedef bf16 TW, TA, TKV;
   typedef float Acc, TR;
-  static constexpr bool kTensorCores = false;
+  static constexpr bool kTensorCores = true;
 };
 
 static int ceil_div(long a, long b) { return (int)((a + b - 1) / b); }
@@ -300,6 +301,20 @@ template <class Path> struct Runner {
                                                         (const Acc*)ws.yb, ws.row_of, n, d, k);
     ++m->launches;
     return check_launch("moe");
+  }
+
+  dg_status moe_op(int l, const float* x_in, float* out, int n) {
+    const size_t d = c.d_model;
+    if constexpr (sizeof(TR) == sizeof(float)) {
+      DG_TRY_CUDA(cudaMemcpyAsync(x(), x_in, n * d * sizeof(float), cudaMemcpyDeviceToDevice, st));
+    } else {
+      widen_f32_kernel<TR><<<ceil_div((long)n * d, 256), 256, 0, st>>>(x_in, x(), (long)n * d);
+      ++m->launches;
+    }
+    DG_TRY(moe(l, n, nullptr));
+    to_f32_kernel<TR><<<ceil_div((long)n * d, 256), 256, 0, st>>>(x(), out, (long)n * d);
+    ++m->launches;
+    return check_launch("moe op");
   }
 
   // Prompt pass for each batch element, keeping the last W keys/values per layer.
@@ -639,6 +654,34 @@ dg_status dg_eb_sample(const float* entropy, const int32_t* argmax, int32_t* can
   DG_TRY(gamma_fixed(gamma, &gq));
   return launch_sampler(entropy, argmax, canvas, mask, B, C, steps_left, gq, n_committed,
                         nullptr, 0, (cudaStream_t)stream, nullptr);
+}
+
+dg_status dg_op_gemm(dg_model* m, const void* A, const void* W, float* out, int32_t M, int32_t N,
+                     int32_t K, void* stream) {
+  g_err.clear();
+  DG_REQUIRE(m && A && W && out, "null argument");
+  DG_REQUIRE(M >= 1 && N >= 1 && K >= 1, "bad sizes");
+  cudaStream_t st = (cudaStream_t)stream;
+  if (m->cfg.dtype == DG_F32) {
+    gemm_simt<float, float, double, false, false>((const float*)A, K, (const float*)W, nullptr, K,
+                                                  M, N, K, GroupInfo(), 0,
+                                                  EpiStore<float, double>{out, N}, st,
+                                                  &m->launches);
+    return check_launch("op gemm");
+  }
+  DG_REQUIRE(N % 64 == 0 && K % 64 == 0, "bf16 GEMM needs N %% 64 == 0 and K %% 64 == 0");
+  return tc_gemm_f32_rows(m, (const bf16*)A, M, W, out, M, N, K, st);
+}
+
+dg_status dg_op_moe(dg_model* m, int32_t layer, const float* x, float* out, int32_t n,
+                    void* stream) {
+  g_err.clear();
+  DG_REQUIRE(m && x && out, "null argument");
+  DG_REQUIRE(layer >= 0 && layer < m->cfg.n_layers, "layer out of range");
+  DG_REQUIRE(n >= 1 && (size_t)n <= m->ws.max_tok, "n=%d outside [1, %zu]", n, m->ws.max_tok);
+  cudaStream_t st = (cudaStream_t)stream;
+  return m->cfg.dtype == DG_F32 ? Runner<PathTiny>(m, st).moe_op(layer, x, out, n)
+                                : Runner<PathBF16>(m, st).moe_op(layer, x, out, n);
 }
 
 dg_status dg_profile_start(dg_model* m) {

@@ -376,7 +376,7 @@ __global__ void router_kernel(const TR* __restrict__ x, const TW* __restrict__ w
 // entries keep their j order.  Block e computes the rank of each of its entries
 // and counts[e].
 // ---------------------------------------------------------------------------
-__global__ void moe_rank_kernel(const int32_t* __restrict__ idx, int n_entries,
+static __global__ void moe_rank_kernel(const int32_t* __restrict__ idx, int n_entries,
                                 int32_t* __restrict__ rank, int32_t* __restrict__ counts) {
   __shared__ int warp_tot[32];
   __shared__ int carry;
@@ -406,7 +406,7 @@ __global__ void moe_rank_kernel(const int32_t* __restrict__ idx, int n_entries,
 }
 
 // offsets = exclusive scan of counts; tile table with `bm` rows per tile.
-__global__ void moe_offsets_kernel(const int32_t* __restrict__ counts, int E, int bm,
+static __global__ void moe_offsets_kernel(const int32_t* __restrict__ counts, int E, int bm,
                                    int32_t* __restrict__ offsets, int32_t* __restrict__ tile_e,
                                    int32_t* __restrict__ tile_m0, int32_t* __restrict__ n_tiles,
                                    int max_tiles) {
@@ -613,12 +613,18 @@ __global__ void lm_merge_kernel(const Acc* __restrict__ part, int n_vt, int n_ro
 }
 
 template <class T>
+__global__ void widen_f32_kernel(const float* __restrict__ src, T* __restrict__ dst, long n) {
+  const long i = blockIdx.x * (long)blockDim.x + threadIdx.x;
+  if (i < n) dst[i] = (T)src[i];
+}
+
+template <class T>
 __global__ void to_f32_kernel(const T* __restrict__ src, float* __restrict__ dst, long n) {
   const long i = blockIdx.x * (long)blockDim.x + threadIdx.x;
   if (i < n) dst[i] = (float)widen(src[i]);
 }
 
-__global__ void fill_i32_kernel(int32_t* __restrict__ p, int n, int32_t v) {
+static __global__ void fill_i32_kernel(int32_t* __restrict__ p, int n, int32_t v) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) p[i] = v;
 }

@@ -1,0 +1,253 @@
+// Host side of the tcgen05 kernels: TMA tensor maps (cached per buffer) and
+// launch configuration of the dense, grouped-expert and LM-head GEMMs.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "dg_internal.h"
+#include "k_simt.cuh"
+#include "k_tc_gemm.cuh"
+
+namespace dg {
+
+namespace {
+
+struct MapKey {
+  const void* p;
+  uint64_t rows, cols;
+  uint32_t box_rows;
+  bool operator==(const MapKey& o) const {
+    return p == o.p && rows == o.rows && cols == o.cols && box_rows == o.box_rows;
+  }
+};
+struct MapKeyHash {
+  size_t operator()(const MapKey& k) const {
+    size_t h = std::hash<const void*>()(k.p);
+    h ^= std::hash<uint64_t>()(k.rows * 1315423911ull + k.cols) + 0x9e3779b9 + (h << 6) + (h >> 2);
+    return h ^ (k.box_rows * 2654435761u);
+  }
+};
+
+struct TcState {
+  PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  std::unordered_map<MapKey, CUtensorMap, MapKeyHash> maps;
+};
+
+std::mutex g_tc_mu;
+std::unordered_map<const dg_model*, TcState*> g_tc;
+
+TcState* state(const dg_model* m) {
+  std::lock_guard<std::mutex> lk(g_tc_mu);
+  auto it = g_tc.find(m);
+  return it == g_tc.end() ? nullptr : it->second;
+}
+
+int ceil_div_i(long a, long b) { return (int)((a + b - 1) / b); }
+
+// 2-D bf16 tensor [rows, cols] (row-major), box = 64 columns x box_rows rows,
+// 128-byte swizzle, out-of-range elements read as zero.
+dg_status tmap(const dg_model* m, const void* p, uint64_t rows, uint64_t cols, uint32_t box_rows,
+               CUtensorMap* out) {
+  TcState* s = state(m);
+  if (!s) {
+    set_error("tensor-core state missing");
+    return DG_ERR_INTERNAL;
+  }
+  MapKey key{p, rows, cols, box_rows};
+  auto it = s->maps.find(key);
+  if (it != s->maps.end()) {
+    *out = it->second;
+    return DG_OK;
+  }
+  if ((reinterpret_cast<uintptr_t>(p) & 15) || (cols * 2) % 16 || box_rows > 256) {
+    set_error("tensor map: base %p / row pitch %llu bytes not 16-byte aligned", p,
+              (unsigned long long)(cols * 2));
+    return DG_ERR_UNSUPPORTED;
+  }
+  CUtensorMap map;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = s->encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(p), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    set_error("cuTensorMapEncodeTiled failed (%d) for %p [%llu x %llu] box %u", (int)r, p,
+              (unsigned long long)rows, (unsigned long long)cols, box_rows);
+    return DG_ERR_CUDA;
+  }
+  s->maps.emplace(key, map);
+  *out = map;
+  return DG_OK;
+}
+
+template <class K> dg_status set_smem(K kern, size_t bytes) {
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e != cudaSuccess) {
+    set_error("cudaFuncSetAttribute(%zu bytes): %s", bytes, cudaGetErrorString(e));
+    return DG_ERR_CUDA;
+  }
+  return DG_OK;
+}
+
+template <int BN, int MT, bool DUAL, int ST, class Epi>
+dg_status launch_dense(dg_model* m, const CUtensorMap& a, const CUtensorMap& b,
+                       const CUtensorMap& b2, int M, int N, int K, Epi epi, cudaStream_t st) {
+  typedef DenseCfg<BN, MT, DUAL, ST> Cfg;
+  auto kern = tc_dense_kernel<BN, MT, DUAL, ST, Epi>;
+  static int ready_dev = -1;
+  if (ready_dev != m->device) {
+    DG_TRY(set_smem(kern, Cfg::SMEM));
+    ready_dev = m->device;
+  }
+  dim3 grid(ceil_div_i(M, 128 * MT), ceil_div_i(N, BN));
+  kern<<<grid, 128, Cfg::SMEM, st>>>(a, b, b2, M, K, epi, m->ws.err);
+  ++m->launches;
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_error("tc_dense launch: %s", cudaGetErrorString(e));
+    return DG_ERR_CUDA;
+  }
+  return DG_OK;
+}
+
+constexpr int DENSE_BN = 64, DENSE_MT = 2, DENSE_ST = 5, DUAL_ST = 4;
+constexpr int LM_BN = 256, LM_ST = 3;
+constexpr int GU_ST = 3, DN_ST = 4;
+
+}  // namespace
+
+dg_status tc_prepare(dg_model* m) {
+  const dg_config& c = m->cfg;
+  const int qkv_n = (c.n_q_heads + 2 * c.n_kv_heads) * c.head_dim;
+  if (c.d_model % 128 || c.expert_inter % 128 || c.shared_inter % 64 || qkv_n % 64 ||
+      (c.n_q_heads * c.head_dim) % 64) {
+    set_error("tensor-core tiling needs d %% 128, I %% 128, Is %% 64, (Hq+2Hkv)h %% 64 and Hq h %% 64");
+    return DG_ERR_UNSUPPORTED;
+  }
+  TcState* s = new TcState();
+  cudaDriverEntryPointQueryResult q;
+  void* fn = nullptr;
+  cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+  if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) {
+    delete s;
+    set_error("cuTensorMapEncodeTiled entry point unavailable");
+    return DG_ERR_CUDA;
+  }
+  s->encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  std::lock_guard<std::mutex> lk(g_tc_mu);
+  g_tc[m] = s;
+  return DG_OK;
+}
+
+void tc_release(dg_model* m) {
+  std::lock_guard<std::mutex> lk(g_tc_mu);
+  auto it = g_tc.find(m);
+  if (it != g_tc.end()) {
+    delete it->second;
+    g_tc.erase(it);
+  }
+}
+
+dg_status tc_gemm_store_f32(dg_model* m, const bf16* A, const void* W, float* out, int M, int N,
+                            int K, cudaStream_t st) {
+  CUtensorMap a, b;
+  DG_TRY(tmap(m, A, m->ws.max_tok, K, 128, &a));
+  DG_TRY(tmap(m, W, N, K, DENSE_BN, &b));
+  return launch_dense<DENSE_BN, DENSE_MT, false, DENSE_ST>(m, a, b, b, M, N, K,
+                                                           EpiStoreF32{out, N, N}, st);
+}
+
+dg_status tc_gemm_f32_rows(dg_model* m, const bf16* A, int a_rows, const void* W, float* out,
+                           int M, int N, int K, cudaStream_t st) {
+  CUtensorMap a, b;
+  DG_TRY(tmap(m, A, a_rows, K, 128, &a));
+  DG_TRY(tmap(m, W, N, K, DENSE_BN, &b));
+  return launch_dense<DENSE_BN, DENSE_MT, false, DENSE_ST>(m, a, b, b, M, N, K,
+                                                           EpiStoreF32{out, N, N}, st);
+}
+
+dg_status tc_gemm_add_residual(dg_model* m, const bf16* A, const void* W, float* x, int M, int N,
+                               int K, cudaStream_t st) {
+  CUtensorMap a, b;
+  DG_TRY(tmap(m, A, m->ws.max_tok, K, 128, &a));
+  DG_TRY(tmap(m, W, N, K, DENSE_BN, &b));
+  return launch_dense<DENSE_BN, DENSE_MT, false, DENSE_ST>(m, a, b, b, M, N, K,
+                                                           EpiAddF32{x, N, N}, st);
+}
+
+dg_status tc_gemm_swiglu(dg_model* m, const bf16* A, const void* Wg, const void* Wu, bf16* out,
+                         int M, int N, int K, cudaStream_t st) {
+  CUtensorMap a, b, b2;
+  DG_TRY(tmap(m, A, m->ws.max_tok, K, 128, &a));
+  DG_TRY(tmap(m, Wg, N, K, DENSE_BN, &b));
+  DG_TRY(tmap(m, Wu, N, K, DENSE_BN, &b2));
+  return launch_dense<DENSE_BN, DENSE_MT, true, DUAL_ST>(m, a, b, b2, M, N, K,
+                                                         EpiSwigluBf16{out, N, N}, st);
+}
+
+dg_status tc_lmhead_stats(dg_model* m, const bf16* xn, int M, float* ent, int32_t* amax,
+                          cudaStream_t st) {
+  const dg_config& c = m->cfg;
+  CUtensorMap a, b;
+  DG_TRY(tmap(m, xn, m->ws.max_tok, c.d_model, 128, &a));
+  DG_TRY(tmap(m, m->w.lm_head, c.vocab, c.d_model, LM_BN, &b));
+  float* part = (float*)m->ws.lm_part;
+  DG_TRY((launch_dense<LM_BN, 2, false, LM_ST>(m, a, b, b, M, c.vocab, c.d_model,
+                                               EpiLmStats{part, M, c.vocab, c.logit_scale}, st)));
+  const int n_vt = ceil_div_i(c.vocab, LM_BN);
+  lm_merge_kernel<float><<<ceil_div_i(M, 4), 128, 0, st>>>(part, n_vt, M, ent, amax);
+  ++m->launches;
+  return DG_OK;
+}
+
+template <bool GATEUP, int ST>
+static dg_status launch_expert(dg_model* m, const CUtensorMap& w, const CUtensorMap& w2,
+                               const CUtensorMap& x, int w_rows, int K, int FT, void* out, int ldo,
+                               const float* gate_of, cudaStream_t st) {
+  typedef ExpertCfg<GATEUP, ST> Cfg;
+  auto kern = tc_expert_kernel<GATEUP, ST>;
+  static int ready_dev = -1;
+  if (ready_dev != m->device) {
+    DG_TRY(set_smem(kern, Cfg::SMEM));
+    ready_dev = m->device;
+  }
+  int n_sm = 148;
+  cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, m->device);
+  const Workspace& ws = m->ws;
+  kern<<<n_sm, 192, Cfg::SMEM, st>>>(w, w2, x, ws.tile_e, ws.tile_m0, ws.n_tiles, ws.offsets,
+                                     w_rows, K, FT, out, ldo, gate_of, ws.err);
+  ++m->launches;
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_error("tc_expert launch: %s", cudaGetErrorString(e));
+    return DG_ERR_CUDA;
+  }
+  return DG_OK;
+}
+
+dg_status tc_moe_gate_up(dg_model* m, int l, const bf16* X, bf16* hb, int, cudaStream_t st) {
+  const dg_config& c = m->cfg;
+  const dg_layer_weights& L = m->layers[l];
+  const int E = c.n_experts, I = c.expert_inter, d = c.d_model;
+  CUtensorMap wg, wu, x;
+  DG_TRY(tmap(m, L.gate, (uint64_t)E * I, d, 128, &wg));
+  DG_TRY(tmap(m, L.up, (uint64_t)E * I, d, 128, &wu));
+  DG_TRY(tmap(m, X, m->ws.max_rows, d, 32, &x));
+  return launch_expert<true, GU_ST>(m, wg, wu, x, I, d, I / 128, hb, I, nullptr, st);
+}
+
+dg_status tc_moe_down(dg_model* m, int l, const bf16* H, float* yb, int, cudaStream_t st) {
+  const dg_config& c = m->cfg;
+  const dg_layer_weights& L = m->layers[l];
+  const int E = c.n_experts, I = c.expert_inter, d = c.d_model;
+  CUtensorMap wd, x;
+  DG_TRY(tmap(m, L.down, (uint64_t)E * d, I, 128, &wd));
+  DG_TRY(tmap(m, H, m->ws.max_rows, I, 32, &x));
+  return launch_expert<false, DN_ST>(m, wd, wd, x, d, I, d / 128, yb, d,
+                                     (const float*)m->ws.gate_of, st);
+}
+
+}  // namespace dg

@@ -83,7 +83,17 @@ def full30_fp8exp(batch: int) -> Workload:
                              batch=batch, prompt_len=4096)
 
 
-WORKLOADS = {w.name: w for w in (TINY_F32, LAYER1_BF16, FULL30_BF16, FULL30_B8_P8192)}
+# Small bf16 model for fast parity tests of the tensor-core path: several tiles per
+# GEMM with ragged tails (B*C = 288 rows), a prompt longer than the window
+# (160 > 128), experts receiving more than 256 rows, 4 vocabulary tiles.
+SMALL_BF16 = Workload(
+    name="small-bf16", n_layers=2, d_model=256, n_q_heads=4, n_kv_heads=2, head_dim=64,
+    n_experts=8, top_k=4, expert_inter=128, shared_inter=192, vocab=1024, window=128,
+    canvas=96, rope_base=10000.0, rms_eps=1e-6, logit_scale=8.0, dtype="bf16",
+    batch=3, prompt_len=160, T=6, gamma=1.0)
+
+WORKLOADS = {w.name: w for w in (TINY_F32, SMALL_BF16, LAYER1_BF16, FULL30_BF16,
+                                 FULL30_B8_P8192)}
 for _b in (1, 4, 16, 32, 64):
     WORKLOADS[f"full30-fp8exp-b{_b}"] = full30_fp8exp(_b)
 
