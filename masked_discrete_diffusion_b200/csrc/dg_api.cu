@@ -121,8 +121,15 @@ template <class Path> static dg_status alloc_workspace(dg_model* m) {
   DG_TRY(ws_alloc_v<Acc>(ws, &ws.qkv, T * qkv));
   DG_TRY(ws_alloc_v<TA>(ws, &ws.q, T * c.n_q_heads * h));
   DG_TRY(ws_alloc_v<TA>(ws, &ws.o, T * c.n_q_heads * h));
-  DG_TRY(ws_alloc_v<TKV>(ws, &ws.kc, T * c.n_kv_heads * h));
-  DG_TRY(ws_alloc_v<TKV>(ws, &ws.vc, T * c.n_kv_heads * h));
+  // own keys [B, Hkv, np, h] and transposed values [B, Hkv, h, np], np = n rounded up to 64
+  const size_t T_pad = T + 64 * (size_t)c.max_batch;
+  DG_TRY(ws_alloc_v<TKV>(ws, &ws.kc, T_pad * c.n_kv_heads * h));
+  DG_TRY(ws_alloc_v<TKV>(ws, &ws.vc, T_pad * c.n_kv_heads * h));
+  ws.kc_elems = T_pad * c.n_kv_heads * h;
+  if constexpr (Path::kTensorCores) {
+    DG_TRY(ws_alloc_v<float>(ws, &ws.attn_o, (size_t)ATT_MAX_SPLITS * T * c.n_q_heads * h));
+    DG_TRY(ws_alloc_v<float>(ws, &ws.attn_ml, (size_t)ATT_MAX_SPLITS * T * c.n_q_heads * 2));
+  }
   DG_TRY(ws_alloc_v<Acc>(ws, &ws.ys, T * d));
   DG_TRY(ws_alloc_v<TA>(ws, &ws.sh, T * c.shared_inter));
   DG_TRY(ws_alloc(ws, &ws.ridx, R));
@@ -198,8 +205,12 @@ template <class Path> struct Runner {
   }
 
   // One decoder layer on n tokens = B_ * n_seq rows at positions pos0 + i.
-  dg_status layer(int l, int n, int B_, int n_seq, int pos0, const TKV* kA, const TKV* vA,
-                  int nA, int kposA, bool causal, int32_t* load) {
+  // Segment A (the cached window, denoise only): keys [L, B, Hkv, WpA, h] and transposed
+  // values [L, B, Hkv, h, WpA] of `kv`, nA valid keys at positions kposA...
+  dg_status layer(int l, int n, int B_, int n_seq, int pos0, const dg_kv* kv, bool causal,
+                  int32_t* load) {
+    const int nA = kv ? kv->W : 0, kposA = kv ? kv->P - kv->W : 0, WpA = kv ? kv->Wp : 0;
+    const int np = (n_seq + 63) / 64 * 64;
     const dg_layer_weights& L = m->layers[l];
     const int d = c.d_model, h = c.head_dim, Hq = c.n_q_heads, Hkv = c.n_kv_heads;
     const int qkv_n = (Hq + 2 * Hkv) * h;
@@ -212,25 +223,38 @@ template <class Path> struct Runner {
         dense(xn(), d, L.wqkv, qkv_n, d, n, EpiStore<Acc, Acc>{(Acc*)ws.qkv, qkv_n});
     }
     rope_scatter_kernel<Acc, TA, TKV><<<n, 128, 0, st>>>(
-        (const Acc*)ws.qkv, (TA*)ws.q, (TKV*)ws.kc, (TKV*)ws.vc, n, n_seq, pos0, Hq, Hkv, h,
+        (const Acc*)ws.qkv, (TA*)ws.q, (TKV*)ws.kc, (TKV*)ws.vc, n, n_seq, np, pos0, Hq, Hkv, h,
         (const Acc*)ws.rope, ws.max_pos);
     ++m->launches;
     {
       ProfScope ps(m, DG_KIND_ATTENTION, st);
-      const long warps = (long)n * Hq;
-      const int blocks = ceil_div(warps, 4);
-      const TKV* kB = (const TKV*)ws.kc;
-      const TKV* vB = (const TKV*)ws.vc;
-#define DG_ATTN(DPL)                                                                         \
-  attention_simt_kernel<TA, TKV, Acc, DPL><<<blocks, 128, 0, st>>>(                          \
-      (const TA*)ws.q, (TA*)ws.o, kA, vA, nA, kposA, kB, vB, n_seq, pos0, B_, n_seq, pos0, Hq, \
-      Hkv, h, causal ? 1 : 0, c.window)
-      if (h <= 32) DG_ATTN(1);
-      else if (h <= 64) DG_ATTN(2);
-      else if (h <= 96) DG_ATTN(3);
-      else DG_ATTN(4);
-      ++m->launches;
+      bool done = false;
+      if constexpr (Path::kTensorCores) {
+        if (h == 128) {
+          DG_TRY(tc_attention(m, (const bf16*)ws.q, B_, n_seq, pos0, kv, l, (const bf16*)ws.kc,
+                              (const bf16*)ws.vc, n_seq, pos0, np, causal, (bf16*)ws.o, st));
+          done = true;
+        }
+      }
+      if (!done) {
+        const long warps = (long)n * Hq;
+        const int blocks = ceil_div(warps, 4);
+        const size_t lstride = kv ? (size_t)kv->B * Hkv * kv->Wp * h : 0;
+        const TKV* kA = kv ? (const TKV*)kv->k + l * lstride : nullptr;
+        const TKV* vA = kv ? (const TKV*)kv->v + l * lstride : nullptr;
+        const TKV* kB = (const TKV*)ws.kc;
+        const TKV* vB = (const TKV*)ws.vc;
+#define DG_ATTN(DPL)                                                                            \
+  attention_simt_kernel<TA, TKV, Acc, DPL><<<blocks, 128, 0, st>>>(                             \
+      (const TA*)ws.q, (TA*)ws.o, kA, vA, nA, WpA, kposA, kB, vB, n_seq, np, pos0, B_, n_seq,  \
+      pos0, Hq, Hkv, h, causal ? 1 : 0, c.window)
+        if (h <= 32) DG_ATTN(1);
+        else if (h <= 64) DG_ATTN(2);
+        else if (h <= 96) DG_ATTN(3);
+        else DG_ATTN(4);
+        ++m->launches;
 #undef DG_ATTN
+      }
     }
     {
       ProfScope ps(m, DG_KIND_DENSE, st);
@@ -320,22 +344,29 @@ template <class Path> struct Runner {
   // Prompt pass for each batch element, keeping the last W keys/values per layer.
   dg_status prefill(const int32_t* prompt, int B, int P, dg_kv* kv) {
     const int d = c.d_model, h = c.head_dim, Hkv = c.n_kv_heads;
-    const int W = kv->W;
+    const int W = kv->W, Wp = kv->Wp;
+    const int Pp = (P + 63) / 64 * 64;
+    const size_t es = sizeof(TKV);
     for (int b = 0; b < B; ++b) {
       embed_kernel<TW, TR><<<P, 256, 0, st>>>(prompt + (size_t)b * P, (const TW*)m->w.tok_emb,
                                              x(), P, d, c.vocab - 1, -1.0, ws.err);
       ++m->launches;
+      // padding columns of the transposed values must read as zero
+      DG_TRY_CUDA(cudaMemsetAsync(ws.vc, 0, (size_t)Hkv * h * Pp * es, st));
       for (int l = 0; l < c.n_layers; ++l) {
-        DG_TRY(layer(l, P, 1, P, 0, nullptr, nullptr, 0, 0, true, nullptr));
-        // keys/values of positions P-W .. P-1 -> cache [l, b, hkv, W, h]
-        const size_t es = sizeof(TKV);
-        for (int which = 0; which < 2; ++which) {
-          const char* src = (const char*)(which ? ws.vc : ws.kc) + (size_t)(P - W) * h * es;
-          char* dst = (char*)(which ? kv->v : kv->k) +
-                      (((size_t)l * kv->B + b) * Hkv) * (size_t)W * h * es;
-          DG_TRY_CUDA(cudaMemcpy2DAsync(dst, (size_t)W * h * es, src, (size_t)P * h * es,
-                                        (size_t)W * h * es, Hkv, cudaMemcpyDeviceToDevice, st));
-        }
+        DG_TRY(layer(l, P, 1, P, 0, nullptr, true, nullptr));
+        // keys [hkv, P-W .. P-1, :] -> cache K [l, b, hkv, 0 .. W-1, :]
+        char* kdst = (char*)kv->k + (((size_t)l * kv->B + b) * Hkv) * (size_t)Wp * h * es;
+        DG_TRY_CUDA(cudaMemcpy2DAsync(kdst, (size_t)Wp * h * es,
+                                      (const char*)ws.kc + (size_t)(P - W) * h * es,
+                                      (size_t)Pp * h * es, (size_t)W * h * es, Hkv,
+                                      cudaMemcpyDeviceToDevice, st));
+        // transposed values [hkv, :, P-W .. P-1] -> cache V^T [l, b, hkv, :, 0 .. W-1]
+        char* vdst = (char*)kv->v + (((size_t)l * kv->B + b) * Hkv) * (size_t)h * Wp * es;
+        DG_TRY_CUDA(cudaMemcpy2DAsync(vdst, (size_t)Wp * es,
+                                      (const char*)ws.vc + (size_t)(P - W) * es, (size_t)Pp * es,
+                                      (size_t)W * es, (size_t)Hkv * h, cudaMemcpyDeviceToDevice,
+                                      st));
       }
     }
     return check_launch("prefill");
@@ -349,13 +380,11 @@ template <class Path> struct Runner {
     embed_kernel<TW, TR><<<n, 256, 0, st>>>(canvas, (const TW*)m->w.tok_emb, x(), n, d, c.vocab,
                                            tau, ws.err);
     ++m->launches;
-    const size_t lstride = (size_t)B * c.n_kv_heads * kv->W * c.head_dim;
-    for (int l = 0; l < c.n_layers; ++l) {
-      const TKV* kA = (const TKV*)kv->k + l * lstride;
-      const TKV* vA = (const TKV*)kv->v + l * lstride;
-      DG_TRY(layer(l, n, B, C, kv->P, kA, vA, kv->W, kv->P - kv->W, false,
-                   load ? load + (size_t)l * c.n_experts : nullptr));
-    }
+    const int Cp = (C + 63) / 64 * 64;
+    if (Cp != C)
+      DG_TRY_CUDA(cudaMemsetAsync(ws.vc, 0, (size_t)B * c.n_kv_heads * c.head_dim * Cp * sizeof(TKV), st));
+    for (int l = 0; l < c.n_layers; ++l)
+      DG_TRY(layer(l, n, B, C, kv->P, kv, false, load ? load + (size_t)l * c.n_experts : nullptr));
     if (hidden) to_f32_kernel<TR><<<ceil_div((long)n * d, 256), 256, 0, st>>>(x(), hidden, (long)n * d);
     ++m->launches;
     rmsnorm(n);
@@ -534,9 +563,12 @@ dg_status dg_prefill(dg_model* m, const int32_t* prompt, int32_t B, int32_t P, d
   kv->B = B;
   kv->P = P;
   kv->W = std::min(P, c.window);
+  kv->Wp = (kv->W + 63) / 64 * 64;
   kv->elem = c.dtype == DG_F32 ? sizeof(double) : sizeof(bf16);
-  const size_t n = (size_t)c.n_layers * B * c.n_kv_heads * kv->W * c.head_dim * kv->elem;
-  if (cudaMalloc(&kv->k, n) != cudaSuccess || cudaMalloc(&kv->v, n) != cudaSuccess) {
+  const size_t n = (size_t)c.n_layers * B * c.n_kv_heads * kv->Wp * c.head_dim * kv->elem;
+  if (cudaMalloc(&kv->k, n) != cudaSuccess || cudaMalloc(&kv->v, n) != cudaSuccess ||
+      cudaMemsetAsync(kv->k, 0, n, (cudaStream_t)stream) != cudaSuccess ||
+      cudaMemsetAsync(kv->v, 0, n, (cudaStream_t)stream) != cudaSuccess) {
     cudaGetLastError();
     cudaFree(kv->k);
     cudaFree(kv->v);
@@ -578,11 +610,18 @@ dg_status dg_kv_info(const dg_kv* kv, int32_t* B, int32_t* P, int32_t* W) {
 dg_status dg_kv_read(const dg_kv* kv, void* k, void* v, void* stream) {
   DG_REQUIRE(kv && k && v, "null argument");
   const dg_config& c = kv->m->cfg;
-  const size_t n = (size_t)c.n_layers * kv->B * c.n_kv_heads * kv->W * c.head_dim * kv->elem;
   cudaStream_t st = (cudaStream_t)stream;
-  DG_TRY_CUDA(cudaMemcpyAsync(k, kv->k, n, cudaMemcpyDeviceToDevice, st));
-  DG_TRY_CUDA(cudaMemcpyAsync(v, kv->v, n, cudaMemcpyDeviceToDevice, st));
-  return DG_OK;
+  const size_t blocks = (size_t)c.n_layers * kv->B * c.n_kv_heads;
+  const size_t total = blocks * kv->W * c.head_dim;
+  if (kv->elem == sizeof(double))
+    kv_unpack_kernel<double><<<ceil_div(total, 256), 256, 0, st>>>(
+        (const double*)kv->k, (const double*)kv->v, (double*)k, (double*)v, blocks, kv->W, kv->Wp,
+        c.head_dim);
+  else
+    kv_unpack_kernel<bf16><<<ceil_div(total, 256), 256, 0, st>>>(
+        (const bf16*)kv->k, (const bf16*)kv->v, (bf16*)k, (bf16*)v, blocks, kv->W, kv->Wp,
+        c.head_dim);
+  return check_launch("kv read");
 }
 
 static dg_status check_step_args(dg_model* m, const dg_kv* kv, int s, int T) {

@@ -40,6 +40,7 @@ void set_error(const char* fmt, ...);
 
 // Device error bits (set by kernels, read and cleared by dg_sync_status).
 enum : int { ERR_BAD_TOKEN = 1, ERR_TIMEOUT = 2, ERR_BAD_SHAPE = 4 };
+constexpr int ATT_MAX_SPLITS = 8;
 
 // A typed device allocation owned by the workspace.
 struct DevBuf {
@@ -70,6 +71,8 @@ struct Workspace {
   float* ent = nullptr;                             // [max_batch, C] entropies
   int32_t *amax = nullptr, *ncommit = nullptr;      // [max_batch, C], [max_batch]
   int max_pos = 0;
+  size_t kc_elems = 0;
+  void *attn_o = nullptr, *attn_ml = nullptr;  // attention key-split partials
   int max_tiles = 0;
   int n_vtiles = 0;
 };
@@ -121,7 +124,8 @@ struct ProfScope {
 struct dg_kv {
   dg_model* m = nullptr;
   int B = 0, P = 0, W = 0;
-  void* k = nullptr;  // [L, B, Hkv, W, h]
-  void* v = nullptr;
+  int Wp = 0;         // W rounded up to 64 (padding reads as zero)
+  void* k = nullptr;  // keys [L, B, Hkv, Wp, h]
+  void* v = nullptr;  // values, transposed: [L, B, Hkv, h, Wp]
   size_t elem = 0;    // bytes per element
 };

@@ -193,14 +193,15 @@ template <class TO, class Acc> struct EpiRowScale {
 // ---------------------------------------------------------------------------
 // a2 (RoPE part): rotate q and k of the raw projection, scatter q / k / v.
 // qkv: [n_tok, (Hq + 2 Hkv) h] raw projections.  Token t = b * n_seq + i sits at
-// absolute position pos0 + i.  q -> q_out [n_tok, Hq, h];
-// k, v -> kc / vc [b, Hkv, n_seq, h].  Pair (j, j + h/2) rotates by pos*theta_j.
+// absolute position pos0 + i.  q -> q_out [n_tok, Hq, h]; k -> kc [b, Hkv, np, h];
+// v -> vc transposed [b, Hkv, h, np] (np >= n_seq, padded).
+// Pair (j, j + h/2) rotates by pos*theta_j.
 // rope: [max_pos, h/2] cos values followed by [max_pos, h/2] sin values.
 // ---------------------------------------------------------------------------
 template <class Acc, class TA, class TKV>
 __global__ void rope_scatter_kernel(const Acc* __restrict__ qkv, TA* __restrict__ q_out,
                                     TKV* __restrict__ kc, TKV* __restrict__ vc, int n_tok,
-                                    int n_seq, int pos0, int Hq, int Hkv, int h,
+                                    int n_seq, int np, int pos0, int Hq, int Hkv, int h,
                                     const Acc* __restrict__ rope, int max_pos) {
   const int t = blockIdx.x;
   if (t >= n_tok) return;
@@ -220,14 +221,14 @@ __global__ void rope_scatter_kernel(const Acc* __restrict__ qkv, TA* __restrict_
         qo[j] = narrow<TA>(y1);
         qo[j + half] = narrow<TA>(y2);
       } else {
-        TKV* ko = kc + (((size_t)b * Hkv + (hd - Hq)) * n_seq + i) * h;
+        TKV* ko = kc + (((size_t)b * Hkv + (hd - Hq)) * np + i) * h;
         ko[j] = narrow<TKV>(y1);
         ko[j + half] = narrow<TKV>(y2);
       }
     } else {
-      TKV* vo = vc + (((size_t)b * Hkv + (hd - Hq - Hkv)) * n_seq + i) * h;
-      vo[j] = narrow<TKV>(x1);
-      vo[j + half] = narrow<TKV>(x2);
+      TKV* vo = vc + ((size_t)b * Hkv + (hd - Hq - Hkv)) * h * np + i;
+      vo[(size_t)j * np] = narrow<TKV>(x1);
+      vo[(size_t)(j + half) * np] = narrow<TKV>(x2);
     }
   }
 }
@@ -239,13 +240,13 @@ __global__ void rope_scatter_kernel(const Acc* __restrict__ qkv, TA* __restrict_
 // causal != 0: key at position p is visible to the query at position qp iff
 // qp - window < p <= qp; otherwise every key is visible.  One online softmax
 // over both segments; scores scaled by 1/sqrt(h).  DPL = ceil(h / 32).
-// K/V layouts: [b, Hkv, n, h]; q/o: [b * nq + i, Hq, h].
+// K layout [b, Hkv, n_pad, h]; V transposed [b, Hkv, h, n_pad]; q/o: [b * nq + i, Hq, h].
 // ---------------------------------------------------------------------------
 template <class TA, class TKV, class Acc, int DPL>
 __global__ void attention_simt_kernel(const TA* __restrict__ q, TA* __restrict__ o,
                                       const TKV* __restrict__ kA, const TKV* __restrict__ vA,
-                                      int nA, int kposA, const TKV* __restrict__ kB,
-                                      const TKV* __restrict__ vB, int nB, int kposB, int B,
+                                      int nA, int padA, int kposA, const TKV* __restrict__ kB,
+                                      const TKV* __restrict__ vB, int nB, int padB, int kposB, int B,
                                       int nq, int qpos0, int Hq, int Hkv, int h, int causal,
                                       int window) {
   const int lane = threadIdx.x & 31;
@@ -271,9 +272,10 @@ __global__ void attention_simt_kernel(const TA* __restrict__ q, TA* __restrict__
     const TKV* K = seg == 0 ? kA : kB;
     const TKV* V = seg == 0 ? vA : vB;
     const int n = seg == 0 ? nA : nB;
+    const int npad = seg == 0 ? padA : padB;
     const int p0 = seg == 0 ? kposA : kposB;
     if (n == 0 || K == nullptr) continue;
-    const size_t base = ((size_t)b * Hkv + kvh) * n * h;
+    const size_t base = ((size_t)b * Hkv + kvh) * npad * h;
     int lo = 0, hi = n;
     if (causal) {
       lo = max(0, qp - window + 1 - p0);
@@ -291,11 +293,11 @@ __global__ void attention_simt_kernel(const TA* __restrict__ q, TA* __restrict__
       const Acc mnew = max(mrun, s);
       const Acc corr = dexp(mrun - mnew), pexp = dexp(s - mnew);
       lrun = lrun * corr + pexp;
-      const TKV* vr = V + base + (size_t)t * h;
+      const TKV* vr = V + base + t;
 #pragma unroll
       for (int u = 0; u < DPL; ++u) {
         const int dd = lane + 32 * u;
-        if (dd < h) acc[u] = acc[u] * corr + pexp * (Acc)widen(vr[dd]);
+        if (dd < h) acc[u] = acc[u] * corr + pexp * (Acc)widen(vr[(size_t)dd * npad]);
       }
       mrun = mnew;
     }
@@ -610,6 +612,19 @@ __global__ void lm_merge_kernel(const Acc* __restrict__ part, int n_vt, int n_ro
     H[r] = (float)h;
     amax[r] = (int32_t)best_id;
   }
+}
+
+// Cache K [blocks, Wp, h] and V^T [blocks, h, Wp] -> K, V [blocks, W, h].
+template <class T>
+__global__ void kv_unpack_kernel(const T* __restrict__ k, const T* __restrict__ vt,
+                                 T* __restrict__ ko, T* __restrict__ vo, size_t blocks, int W,
+                                 int Wp, int h) {
+  const size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
+  if (i >= blocks * W * h) return;
+  const size_t bl = i / ((size_t)W * h);
+  const int t = (int)(i / h % W), dd = (int)(i % h);
+  ko[i] = k[(bl * Wp + t) * h + dd];
+  vo[i] = vt[(bl * h + dd) * Wp + t];
 }
 
 template <class T>

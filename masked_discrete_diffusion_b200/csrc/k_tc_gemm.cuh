@@ -485,5 +485,8 @@ dg_status tc_moe_gate_up(dg_model* m, int l, const bf16* X, bf16* hb, int grid_y
 dg_status tc_moe_down(dg_model* m, int l, const bf16* H, float* yb, int grid_y, cudaStream_t st);
 dg_status tc_lmhead_stats(dg_model* m, const bf16* xn, int M, float* ent, int32_t* amax,
                           cudaStream_t st);
+dg_status tc_attention(dg_model* m, const bf16* q, int B, int nq, int qpos0, const dg_kv* kv,
+                       int l, const bf16* kB, const bf16* vB, int nB, int kposB, int npB,
+                       bool causal, bf16* out, cudaStream_t st);
 
 }  // namespace dg

@@ -6,6 +6,7 @@
 
 #include "dg_internal.h"
 #include "k_simt.cuh"
+#include "k_tc_attn.cuh"
 #include "k_tc_gemm.cuh"
 
 namespace dg {
@@ -248,6 +249,76 @@ dg_status tc_moe_down(dg_model* m, int l, const bf16* H, float* yb, int, cudaStr
   DG_TRY(tmap(m, H, m->ws.max_rows, I, 32, &x));
   return launch_expert<false, DN_ST>(m, wd, wd, x, d, I, d / 128, yb, d,
                                      (const float*)m->ws.gate_of, st);
+}
+
+dg_status tc_attention(dg_model* m, const bf16* q, int B, int nq, int qpos0, const dg_kv* kv,
+                       int l, const bf16* kB, const bf16* vB, int nB, int kposB, int npB,
+                       bool causal, bf16* out, cudaStream_t st) {
+  const dg_config& c = m->cfg;
+  const int Hq = c.n_q_heads, Hkv = c.n_kv_heads, h = c.head_dim;
+  if (h != 128) {
+    set_error("tensor-core attention needs head_dim 128");
+    return DG_ERR_UNSUPPORTED;
+  }
+  CUtensorMap mQ, mKA, mVA, mKB, mVB;
+  DG_TRY(tmap(m, q, m->ws.max_tok, (uint64_t)Hq * h, 128, &mQ));
+  DG_TRY(tmap(m, kB, (uint64_t)B * Hkv * npB, h, 128, &mKB));
+  DG_TRY(tmap(m, vB, (uint64_t)B * Hkv * h, npB, 128, &mVB));
+  AttnParams p{};
+  if (kv) {
+    DG_TRY(tmap(m, kv->k, (uint64_t)c.n_layers * kv->B * Hkv * kv->Wp, h, 128, &mKA));
+    DG_TRY(tmap(m, kv->v, (uint64_t)c.n_layers * kv->B * Hkv * h, kv->Wp, 128, &mVA));
+    p.nA = kv->W;
+    p.kposA = kv->P - kv->W;
+    p.rowsA = kv->Wp;
+    p.layer_rowA = l * kv->B * Hkv * kv->Wp;
+    p.layer_vrowA = l * kv->B * Hkv * h;
+  } else {
+    mKA = mKB;
+    mVA = mVB;
+  }
+  p.nq = nq;
+  p.qpos0 = qpos0;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.nB = nB;
+  p.kposB = kposB;
+  p.rowsB = npB;
+  p.causal = causal ? 1 : 0;
+  p.window = c.window;
+  p.B = B;
+  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)h));
+  p.part_o = (float*)m->ws.attn_o;
+  p.part_ml = (float*)m->ws.attn_ml;
+  const int TA = ceil_div_i(p.nA, AT_KT), TB = ceil_div_i(nB, AT_KT);
+  const int total = causal ? std::min(TB, ceil_div_i(c.window + 127, AT_KT) + 1) : TA + TB;
+  const int qtiles = ceil_div_i(nq, 128);
+  const int base = qtiles * Hq * B;
+  int n_sm = 148;
+  cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, m->device);
+  int splits = std::min(ceil_div_i(2 * n_sm, base), std::min((int)ATT_MAX_SPLITS, total));
+  splits = std::max(1, splits);
+  const int tps = ceil_div_i(total, splits);
+  splits = ceil_div_i(total, tps);
+  p.tiles_per_split = tps;
+  static int ready_dev = -1;
+  if (ready_dev != m->device) {
+    DG_TRY(set_smem(tc_attn_kernel, AT_SMEM));
+    ready_dev = m->device;
+  }
+  dim3 grid(qtiles * Hq, B, splits);
+  tc_attn_kernel<<<grid, 128, AT_SMEM, st>>>(mQ, mKA, mVA, mKB, mVB, p, m->ws.err);
+  ++m->launches;
+  const int ntok = B * nq;
+  attn_combine_kernel<<<ceil_div_i((long)ntok * Hq, 4), 128, 0, st>>>(
+      p.part_o, p.part_ml, splits, ntok, Hq, out);
+  ++m->launches;
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_error("tc_attention launch: %s", cudaGetErrorString(e));
+    return DG_ERR_CUDA;
+  }
+  return DG_OK;
 }
 
 }  // namespace dg
