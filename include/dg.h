@@ -208,6 +208,11 @@ dg_status dg_profile_start(dg_model* m);
  * (groups[DG_KIND_COUNT]) since dg_profile_start, and stops recording. */
 dg_status dg_profile_stop(dg_model* m, float* ms, int64_t* groups);
 
+/* Number of (MoE layer pass, expert) pairs in which the expert received at least
+ * one row — i.e. expert weight tiles streamed — since dg_profile_start (or model
+ * creation).  Synchronises the device. */
+dg_status dg_expert_units(dg_model* m, int64_t* units);
+
 /* Number of kernels this model has launched since it was created (host count). */
 dg_status dg_launch_count(const dg_model* m, int64_t* out);
 

@@ -80,6 +80,7 @@ def lib() -> ctypes.CDLL:
             "dg_profile_start": [vp],
             "dg_profile_stop": [vp, vp, vp],
             "dg_launch_count": [vp, ctypes.POINTER(ctypes.c_int64)],
+            "dg_expert_units": [vp, ctypes.POINTER(ctypes.c_int64)],
             "dg_op_gemm": [vp, vp, vp, vp, i32, i32, i32, vp],
             "dg_op_moe": [vp, i32, vp, vp, i32, vp],
         }
@@ -96,7 +97,8 @@ def exported_symbols():
                         "dg_sync_status", "dg_prefill", "dg_kv_destroy", "dg_kv_info",
                         "dg_kv_read", "dg_denoise_step", "dg_generate_block", "dg_eb_sample",
                         "dg_debug_forward", "dg_profile_start", "dg_profile_stop",
-                        "dg_launch_count", "dg_op_gemm", "dg_op_moe") if hasattr(lib(), n)]
+                        "dg_launch_count", "dg_op_gemm", "dg_op_moe", "dg_expert_units")
+            if hasattr(lib(), n)]
 
 
 def _check(status: int):
@@ -285,3 +287,9 @@ def dg_op_moe(model: Model, layer: int, x, stream=None):
     out = torch.empty_like(x)
     _check(lib().dg_op_moe(model.handle, layer, _ptr(x), _ptr(out), x.shape[0], _stream(stream)))
     return out
+
+
+def dg_expert_units(model: Model) -> int:
+    out = ctypes.c_int64()
+    _check(lib().dg_expert_units(model.handle, ctypes.byref(out)))
+    return out.value

@@ -138,6 +138,8 @@ template <class Path> static dg_status alloc_workspace(dg_model* m) {
   DG_TRY(ws_alloc(ws, &ws.tok_of, R));
   DG_TRY(ws_alloc_v<Acc>(ws, &ws.rgate, R));
   DG_TRY(ws_alloc_v<Acc>(ws, &ws.gate_of, R));
+  DG_TRY(ws_alloc_v<Acc>(ws, &ws.inv_rms, T));
+  DG_TRY(ws_alloc_v<Acc>(ws, &ws.rlog, std::max<size_t>(4096, T) * c.n_experts));
   DG_TRY(ws_alloc(ws, &ws.counts, c.n_experts));
   DG_TRY(ws_alloc(ws, &ws.offsets, c.n_experts + 1));
   DG_TRY(ws_alloc(ws, &ws.tile_e, ws.max_tiles));
@@ -149,6 +151,8 @@ template <class Path> static dg_status alloc_workspace(dg_model* m) {
   const size_t lm_rows = (size_t)c.max_batch * c.canvas;
   DG_TRY(ws_alloc_v<Acc>(ws, &ws.lm_part, (size_t)ws.n_vtiles * lm_rows * 4));
   DG_TRY(ws_alloc(ws, &ws.err, 4));
+  DG_TRY(ws_alloc(ws, &ws.units, 1));
+  DG_TRY_CUDA(cudaMemset(ws.units, 0, sizeof(unsigned long long)));
   DG_TRY(ws_alloc(ws, &ws.ids, T));
   DG_TRY(ws_alloc_v<Acc>(ws, &ws.rope, (size_t)2 * ws.max_pos * (h / 2)));
   DG_TRY(ws_alloc(ws, &ws.mask, lm_rows));
@@ -272,21 +276,33 @@ template <class Path> struct Runner {
     const int d = c.d_model, E = c.n_experts, k = c.top_k, I = c.expert_inter;
     const int Is = c.shared_inter;
     const int n_ent = n * k;
-    router_kernel<TR, TW, Acc><<<n, 256, E * sizeof(Acc), st>>>(
-        x(), (const TW*)L.router, n, d, E, k, c.rms_eps, ws.ridx, (Acc*)ws.rgate, load);
+    // u = RMSNorm(x) after attention (bf16 copy for the expert GEMMs, 1/rms for the router)
+    rmsnorm_kernel<TR, TA, Acc><<<n, 256, 0, st>>>(x(), xn(), n, d, c.rms_eps, (Acc*)ws.inv_rms);
     ++m->launches;
+    {
+      const int splits = std::max(1, std::min(16, 4096 / n));
+      const int kps = ceil_div(ceil_div(d, splits), 32) * 32;
+      const int ks = ceil_div(d, kps);
+      dim3 grid(ceil_div(n, 32), ks, ceil_div(E, 128));
+      router_logits_kernel<TR, TW, Acc><<<grid, 256, 0, st>>>(x(), (const TW*)L.router, n, d, E,
+                                                              kps, (Acc*)ws.rlog);
+      ++m->launches;
+      router_topk_kernel<Acc><<<ceil_div(n, 4), 128, 0, st>>>((const Acc*)ws.rlog, ks,
+                                                              (const Acc*)ws.inv_rms, n, E, k,
+                                                              ws.ridx, (Acc*)ws.rgate, load);
+      ++m->launches;
+    }
     moe_rank_kernel<<<E, 256, 0, st>>>(ws.ridx, n_ent, ws.rank, ws.counts);
     ++m->launches;
     int bm = SG_BM;
     if constexpr (Path::kTensorCores) bm = tc_group_rows();
-    moe_offsets_kernel<<<1, 32, 0, st>>>(ws.counts, E, bm, ws.offsets, ws.tile_e, ws.tile_m0,
-                                         ws.n_tiles, ws.max_tiles);
+    moe_offsets_kernel<<<1, 1024, 0, st>>>(ws.counts, E, bm, ws.offsets, ws.tile_e, ws.tile_m0,
+                                           ws.n_tiles, ws.max_tiles, ws.units);
     ++m->launches;
     moe_scatter_kernel<Acc><<<ceil_div(n_ent, 256), 256, 0, st>>>(
         ws.ridx, (const Acc*)ws.rgate, ws.rank, ws.offsets, n_ent, k, ws.row_of, ws.tok_of,
         (Acc*)ws.gate_of);
     ++m->launches;
-    rmsnorm(n);  // u = RMSNorm(x) after attention
     gather_rows_kernel<TA><<<n_ent, 256, 0, st>>>(xn(), ws.tok_of, ws.offsets + E, d,
                                                   (TA*)ws.up);
     ++m->launches;
@@ -726,7 +742,18 @@ dg_status dg_op_moe(dg_model* m, int32_t layer, const float* x, float* out, int3
 dg_status dg_profile_start(dg_model* m) {
   DG_REQUIRE(m, "null model");
   for (int k = 0; k < DG_KIND_COUNT; ++k) m->prof_used[k] = 0;
+  DG_TRY_CUDA(cudaDeviceSynchronize());
+  DG_TRY_CUDA(cudaMemset(m->ws.units, 0, sizeof(unsigned long long)));
   m->profiling = true;
+  return DG_OK;
+}
+
+dg_status dg_expert_units(dg_model* m, int64_t* units) {
+  DG_REQUIRE(m && units, "null argument");
+  unsigned long long u = 0;
+  DG_TRY_CUDA(cudaDeviceSynchronize());
+  DG_TRY_CUDA(cudaMemcpy(&u, m->ws.units, sizeof(u), cudaMemcpyDeviceToHost));
+  *units = (int64_t)u;
   return DG_OK;
 }
 

@@ -59,12 +59,14 @@ struct Workspace {
   // routing
   int32_t *ridx = nullptr, *rank = nullptr, *row_of = nullptr, *tok_of = nullptr;
   void *rgate = nullptr, *gate_of = nullptr;
+  void *inv_rms = nullptr, *rlog = nullptr;  // per-row 1/rms; split-K router partials
   int32_t *counts = nullptr, *offsets = nullptr, *tile_e = nullptr, *tile_m0 = nullptr,
           *n_tiles = nullptr;
   void *up = nullptr, *hb = nullptr, *yb = nullptr; // routed rows
   void* lm_part = nullptr;                          // [n_vtiles, max_tok, 4]
   int32_t* load = nullptr;                          // [L, E] routing counts
   int32_t* err = nullptr;                           // device error bits
+  unsigned long long* units = nullptr;              // (layer pass, expert) pairs with rows
   int32_t* ids = nullptr;                           // [max_tok] token ids of the pass
   void* rope = nullptr;                             // [max_pos, h/2] cos then sin
   uint8_t* mask = nullptr;                          // [max_batch, C] block-loop mask

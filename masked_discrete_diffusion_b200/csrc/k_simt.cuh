@@ -49,7 +49,7 @@ __global__ void embed_kernel(const int32_t* __restrict__ ids, const TW* __restri
 // ---------------------------------------------------------------------------
 template <class TR, class TA, class Acc>
 __global__ void rmsnorm_kernel(const TR* __restrict__ x, TA* __restrict__ y, int n, int d,
-                               float eps) {
+                               float eps, Acc* __restrict__ inv_out = nullptr) {
   __shared__ Acc red[32];
   const int t = blockIdx.x;
   if (t >= n) return;
@@ -61,6 +61,7 @@ __global__ void rmsnorm_kernel(const TR* __restrict__ x, TA* __restrict__ y, int
   }
   ss = block_sum(ss, red);
   const Acc inv = Acc(1) / dsqrt(ss / (Acc)d + (Acc)eps);
+  if (inv_out && threadIdx.x == 0) inv_out[t] = inv;
   for (int c = threadIdx.x; c < d; c += blockDim.x)
     y[(size_t)t * d + c] = narrow<TA>((Acc)widen(r[c]) * inv);
 }
@@ -312,63 +313,138 @@ __global__ void attention_simt_kernel(const TA* __restrict__ q, TA* __restrict__
 }
 
 // ---------------------------------------------------------------------------
-// a5: router.  u = RMSNorm(x) (recomputed from the residual at the accumulation
-// precision), logits = u Wr^T, p = softmax over all E, top-k by p (ties -> lower
-// expert id), gates renormalised to sum 1.  One block per token.
+// a5: router.  logits = RMSNorm(x) Wr^T computed at the accumulation precision
+// from the residual: router_logits_kernel forms split-K partial dot products
+// x . w (tile of 32 tokens x 128 experts per CTA, K range per blockIdx.y);
+// router_topk_kernel (one warp per token) sums the splits in a fixed order,
+// scales by the row's 1/rms, takes the softmax over all E experts, the top-k by
+// probability (ties -> lower expert id) and renormalises the k gates.
 // ---------------------------------------------------------------------------
 template <class TR, class TW, class Acc>
-__global__ void router_kernel(const TR* __restrict__ x, const TW* __restrict__ wr, int n_tok,
-                              int d, int E, int top_k, float eps, int32_t* __restrict__ idx,
-                              Acc* __restrict__ gate, int32_t* __restrict__ load) {
-  extern __shared__ unsigned char smem_raw[];
-  Acc* p = reinterpret_cast<Acc*>(smem_raw);  // [E]
-  __shared__ Acc red[32];
-  const int t = blockIdx.x;
-  if (t >= n_tok) return;
-  const TR* xr = x + (size_t)t * d;
-  Acc ss = 0;
-  for (int c = threadIdx.x; c < d; c += blockDim.x) {
-    const Acc v = (Acc)widen(xr[c]);
-    ss += v * v;
-  }
-  ss = block_sum(ss, red);
-  const Acc inv = Acc(1) / dsqrt(ss / (Acc)d + (Acc)eps);
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  for (int e = wid; e < E; e += nw) {
-    const TW* w = wr + (size_t)e * d;
-    Acc s = 0;
-    for (int c = lane; c < d; c += 32) s += ((Acc)widen(xr[c]) * inv) * (Acc)widen(w[c]);
-    s = warp_sum(s);
-    if (lane == 0) p[e] = s;
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    Acc mx = p[0];
-    for (int e = 1; e < E; ++e) mx = max(mx, p[e]);
-    Acc z = 0;
-    for (int e = 0; e < E; ++e) {
-      p[e] = dexp(p[e] - mx);
-      z += p[e];
+__global__ void __launch_bounds__(256)
+    router_logits_kernel(const TR* __restrict__ x, const TW* __restrict__ wr, int n, int d, int E,
+                         int k_per_split, Acc* __restrict__ part) {
+  __shared__ Acc Xs[32][33];
+  __shared__ Acc Ws[32][129];
+  const int tid = threadIdx.x, tx = tid & 31, ty = tid >> 5;
+  const int t0 = blockIdx.x * 32, e0 = blockIdx.z * 128;
+  const int k_lo = blockIdx.y * k_per_split, k_hi = min(d, k_lo + k_per_split);
+  Acc acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0;
+  for (int k0 = k_lo; k0 < k_hi; k0 += 32) {
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {  // x tile: 32 tokens x 32 k
+      const int el = tid + it * 256, r = el >> 5, kk = el & 31;
+      const int gt = t0 + r, gk = k0 + kk;
+      Xs[kk][r] = (gt < n && gk < k_hi) ? (Acc)widen(x[(size_t)gt * d + gk]) : Acc(0);
     }
-    for (int e = 0; e < E; ++e) p[e] /= z;
-    int sel[64];
-    Acc gs = 0;
-    for (int k = 0; k < top_k; ++k) {
-      int best = -1;
-      for (int e = 0; e < E; ++e) {
-        bool taken = false;
-        for (int q2 = 0; q2 < k; ++q2) taken |= (sel[q2] == e);
-        if (taken) continue;
-        if (best < 0 || p[e] > p[best]) best = e;
+#pragma unroll
+    for (int it = 0; it < 16; ++it) {  // w tile: 128 experts x 32 k
+      const int el = tid + it * 256, r = el >> 5, kk = el & 31;
+      const int ge = e0 + r, gk = k0 + kk;
+      Ws[kk][r] = (ge < E && gk < k_hi) ? (Acc)widen(wr[(size_t)ge * d + gk]) : Acc(0);
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int kk = 0; kk < 32; ++kk) {
+      Acc a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = Xs[kk][ty + 8 * i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) b[j] = Ws[kk][tx + 32 * j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] += a[i] * b[j];
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int t = t0 + ty + 8 * i, e = e0 + tx + 32 * j;
+      if (t < n && e < E) part[((size_t)blockIdx.y * n + t) * E + e] = acc[i][j];
+    }
+}
+
+template <class Acc>
+__global__ void router_topk_kernel(const Acc* __restrict__ part, int splits,
+                                   const Acc* __restrict__ inv_rms, int n, int E, int top_k,
+                                   int32_t* __restrict__ idx, Acc* __restrict__ gate,
+                                   int32_t* __restrict__ load) {
+  constexpr int MAXE = 32;  // experts per lane (E <= 1024)
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= n) return;
+  Acc pr[MAXE];
+  const Acc inv = inv_rms[t];
+  Acc mx = -INFINITY;
+#pragma unroll
+  for (int q = 0; q < MAXE; ++q) {
+    const int e = lane + 32 * q;
+    pr[q] = -INFINITY;
+    if (e < E) {
+      Acc s = 0;
+      for (int z = 0; z < splits; ++z) s += part[((size_t)z * n + t) * E + e];
+      pr[q] = s * inv;
+      mx = max(mx, pr[q]);
+    }
+  }
+  mx = warp_max(mx);
+  Acc z = 0;
+#pragma unroll
+  for (int q = 0; q < MAXE; ++q) {
+    const int e = lane + 32 * q;
+    pr[q] = e < E ? dexp(pr[q] - mx) : Acc(0);
+    z += pr[q];
+  }
+  z = warp_sum(z);
+#pragma unroll
+  for (int q = 0; q < MAXE; ++q) pr[q] /= z;
+  unsigned taken = 0;  // bit q: expert lane + 32 q already selected
+  Acc gsum = 0;
+  int sel_e[64];
+  Acc sel_p[64];
+  for (int k = 0; k < top_k; ++k) {
+    Acc bp = -1;
+    int be = 0x7fffffff;
+#pragma unroll
+    for (int q = 0; q < MAXE; ++q) {
+      const int e = lane + 32 * q;
+      if (e < E && !((taken >> q) & 1u) && (pr[q] > bp || (pr[q] == bp && e < be))) {
+        bp = pr[q];
+        be = e;
       }
-      sel[k] = best;
-      gs += p[best];
     }
-    for (int k = 0; k < top_k; ++k) {
-      idx[(size_t)t * top_k + k] = sel[k];
-      gate[(size_t)t * top_k + k] = p[sel[k]] / gs;
-      if (load) atomicAdd(&load[sel[k]], 1);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const Acc op = __shfl_xor_sync(0xffffffffu, bp, off);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+      if (op > bp || (op == bp && oe < be)) {
+        bp = op;
+        be = oe;
+      }
     }
+    if ((be & 31) == lane) taken |= 1u << (be >> 5);
+    sel_e[k] = be;
+    sel_p[k] = bp;
+    gsum += bp;
+  }
+  if (lane < top_k) {
+    int e = 0;
+    Acc pk = 0;
+    for (int k = 0; k < top_k; ++k)
+      if (k == lane) {
+        e = sel_e[k];
+        pk = sel_p[k];
+      }
+    idx[(size_t)t * top_k + lane] = e;
+    gate[(size_t)t * top_k + lane] = pk / gsum;
+    if (load) atomicAdd(&load[e], 1);
   }
 }
 
@@ -408,26 +484,41 @@ static __global__ void moe_rank_kernel(const int32_t* __restrict__ idx, int n_en
 }
 
 // offsets = exclusive scan of counts; tile table with `bm` rows per tile.
-static __global__ void moe_offsets_kernel(const int32_t* __restrict__ counts, int E, int bm,
-                                   int32_t* __restrict__ offsets, int32_t* __restrict__ tile_e,
-                                   int32_t* __restrict__ tile_m0, int32_t* __restrict__ n_tiles,
-                                   int max_tiles) {
-  if (threadIdx.x != 0 || blockIdx.x != 0) return;
-  int off = 0, nt = 0;
-  for (int e = 0; e < E; ++e) {
-    offsets[e] = off;
-    const int c = counts[e];
-    for (int r = 0; r < c; r += bm) {
-      if (nt < max_tiles) {
-        tile_e[nt] = e;
-        tile_m0[nt] = off + r;
-      }
-      ++nt;
-    }
-    off += c;
+// One block of 1024 threads, thread e handles expert e (E <= 1024).
+static __global__ void __launch_bounds__(1024)
+    moe_offsets_kernel(const int32_t* __restrict__ counts, int E, int bm,
+                       int32_t* __restrict__ offsets, int32_t* __restrict__ tile_e,
+                       int32_t* __restrict__ tile_m0, int32_t* __restrict__ n_tiles,
+                       int max_tiles, unsigned long long* __restrict__ used) {
+  __shared__ int sc[1024], st[1024];
+  const int e = threadIdx.x;
+  const int c = e < E ? counts[e] : 0;
+  // experts that received at least one row (their weights are streamed)
+  const unsigned bal = __ballot_sync(0xffffffffu, c > 0);
+  if (used && (e & 31) == 0 && bal) atomicAdd(used, (unsigned long long)__popc(bal));
+  const int nt = (c + bm - 1) / bm;
+  sc[e] = c;
+  st[e] = nt;
+  __syncthreads();
+  for (int off = 1; off < 1024; off <<= 1) {  // inclusive scans
+    const int a = e >= off ? sc[e - off] : 0, b = e >= off ? st[e - off] : 0;
+    __syncthreads();
+    sc[e] += a;
+    st[e] += b;
+    __syncthreads();
   }
-  offsets[E] = off;
-  *n_tiles = min(nt, max_tiles);
+  const int off_e = sc[e] - c, t_e = st[e] - nt;
+  if (e < E) offsets[e] = off_e;
+  if (e == E - 1) {
+    offsets[E] = off_e + c;
+    *n_tiles = min(t_e + nt, max_tiles);
+  }
+  if (e < E)
+    for (int r = 0; r < nt; ++r)
+      if (t_e + r < max_tiles) {
+        tile_e[t_e + r] = e;
+        tile_m0[t_e + r] = off_e + r * bm;
+      }
 }
 
 template <class Acc>
