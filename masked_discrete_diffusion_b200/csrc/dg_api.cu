@@ -464,6 +464,23 @@ static dg_status launch_sampler(const float* H, const int32_t* am, int32_t* canv
   return check_launch("eb sampler");
 }
 
+static void graph_free(dg::BlockGraph* g) {
+  if (g->exec) cudaGraphExecDestroy(g->exec);
+  for (int k = 0; k < DG_KIND_COUNT; ++k)
+    for (auto& e : g->ev[k]) {
+      cudaEventDestroy(e.first);
+      cudaEventDestroy(e.second);
+    }
+  delete g;
+}
+
+namespace dg {
+void release_graphs(dg_model* m) {
+  for (auto* g : m->graphs) graph_free(g);
+  m->graphs.clear();
+}
+}  // namespace dg
+
 extern "C" {
 
 const char* dg_status_str(dg_status s) {
@@ -518,6 +535,10 @@ dg_status dg_model_create(const dg_config* cfg, const dg_weights* w, dg_model** 
   m->layers.assign(w->layers, w->layers + c.n_layers);
   m->w.layers = nullptr;
   cudaGetDevice(&m->device);
+  {
+    const char* env = getenv("DG_NO_GRAPHS");
+    m->use_graphs = !(env && env[0] && env[0] != '0');
+  }
   dg_status s = c.dtype == DG_F32 ? alloc_workspace<PathTiny>(m) : alloc_workspace<PathBF16>(m);
   if (s != DG_OK) {
     std::string keep = g_err;
@@ -533,6 +554,7 @@ dg_status dg_model_create(const dg_config* cfg, const dg_weights* w, dg_model** 
 dg_status dg_model_destroy(dg_model* m) {
   if (!m) return DG_OK;
   cudaDeviceSynchronize();
+  release_graphs(m);
   for (int k = 0; k < DG_KIND_COUNT; ++k)
     for (auto& e : m->prof[k]) {
       cudaEventDestroy(e.first);
@@ -609,6 +631,16 @@ dg_status dg_prefill(dg_model* m, const int32_t* prompt, int32_t B, int32_t P, d
 dg_status dg_kv_destroy(dg_kv* kv) {
   if (!kv) return DG_OK;
   cudaDeviceSynchronize();
+  // graphs captured for this cache hold its pointers: drop them
+  auto& gs = kv->m->graphs;
+  for (size_t i = 0; i < gs.size();) {
+    if (gs[i]->kv == kv) {
+      graph_free(gs[i]);
+      gs.erase(gs.begin() + i);
+    } else {
+      ++i;
+    }
+  }
   cudaFree(kv->k);
   cudaFree(kv->v);
   delete kv;
@@ -669,15 +701,10 @@ dg_status dg_denoise_step(dg_model* m, const dg_kv* kv, int32_t* canvas, uint8_t
                         n_committed, nullptr, 0, st, &m->launches);
 }
 
-dg_status dg_generate_block(dg_model* m, const dg_kv* kv, int32_t T, float gamma,
-                            int32_t* canvas_out, int32_t* n_forwards, int32_t* router_load,
-                            void* stream) {
-  g_err.clear();
-  DG_TRY(check_step_args(m, kv, T, T));
-  DG_REQUIRE(canvas_out, "null canvas_out");
-  long long gq;
-  DG_TRY(gamma_fixed(gamma, &gq));
-  cudaStream_t st = (cudaStream_t)stream;
+// The launch sequence of one block (T forwards + sampler steps), enqueued on st.
+static dg_status generate_impl(dg_model* m, const dg_kv* kv, int32_t T, long long gq,
+                               int32_t* canvas_out, int32_t* n_forwards, int32_t* router_load,
+                               cudaStream_t st) {
   const dg_config& c = m->cfg;
   const int B = kv->B, C = c.canvas;
   Workspace& ws = m->ws;
@@ -696,6 +723,87 @@ dg_status dg_generate_block(dg_model* m, const dg_kv* kv, int32_t T, float gamma
                           n_forwards, k + 1, st, &m->launches));
   }
   return DG_OK;
+}
+
+// Captures the block's launch sequence once per (kv, T, gamma, output buffers,
+// profiling) and replays it: one host call per block instead of ~500 launches per
+// forward.  With profiling on, the graph also records an event pair around every
+// launch group, read back after each replay.
+static dg_status generate_graphed(dg_model* m, const dg_kv* kv, int32_t T, long long gq,
+                                  int32_t* canvas_out, int32_t* n_forwards,
+                                  int32_t* router_load, cudaStream_t st) {
+  dg::BlockGraph* g = nullptr;
+  for (auto* x : m->graphs)
+    if (x->kv == kv && x->T == T && x->gq == gq && x->canvas == canvas_out &&
+        x->nfwd == n_forwards && x->load == router_load && x->prof == m->profiling) {
+      g = x;
+      break;
+    }
+  if (!g) {
+    if (m->graphs.size() >= 8) {
+      graph_free(m->graphs.front());
+      m->graphs.erase(m->graphs.begin());
+    }
+    g = new dg::BlockGraph();
+    g->kv = kv;
+    g->T = T;
+    g->gq = gq;
+    g->canvas = canvas_out;
+    g->nfwd = n_forwards;
+    g->load = router_load;
+    g->prof = m->profiling;
+    const long long l0 = m->launches;
+    m->capture = g;
+    cudaGraph_t graph = nullptr;
+    cudaError_t e = cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal);
+    dg_status s = DG_OK;
+    if (e == cudaSuccess) {
+      s = generate_impl(m, kv, T, gq, canvas_out, n_forwards, router_load, st);
+      e = cudaStreamEndCapture(st, &graph);
+    }
+    m->capture = nullptr;
+    g->launches = m->launches - l0;
+    m->launches = l0;
+    if (s == DG_OK && e == cudaSuccess) e = cudaGraphInstantiate(&g->exec, graph, 0);
+    if (graph) cudaGraphDestroy(graph);
+    if (s != DG_OK || e != cudaSuccess) {
+      graph_free(g);
+      if (s == DG_OK) {
+        set_error("block graph capture failed: %s", cudaGetErrorString(e));
+        s = DG_ERR_CUDA;
+      }
+      cudaGetLastError();
+      return s;
+    }
+    m->graphs.push_back(g);
+  }
+  DG_TRY_CUDA(cudaGraphLaunch(g->exec, st));
+  m->launches += g->launches;
+  if (g->prof) {
+    DG_TRY_CUDA(cudaStreamSynchronize(st));
+    for (int k = 0; k < DG_KIND_COUNT; ++k)
+      for (auto& ev : g->ev[k]) {
+        float t = 0.f;
+        DG_TRY_CUDA(cudaEventElapsedTime(&t, ev.first, ev.second));
+        m->prof_acc_ms[k] += t;
+        m->prof_acc_n[k] += 1;
+      }
+  }
+  return DG_OK;
+}
+
+dg_status dg_generate_block(dg_model* m, const dg_kv* kv, int32_t T, float gamma,
+                            int32_t* canvas_out, int32_t* n_forwards, int32_t* router_load,
+                            void* stream) {
+  g_err.clear();
+  DG_TRY(check_step_args(m, kv, T, T));
+  DG_REQUIRE(canvas_out, "null canvas_out");
+  long long gq;
+  DG_TRY(gamma_fixed(gamma, &gq));
+  cudaStream_t st = (cudaStream_t)stream;
+  if (m->use_graphs)
+    return generate_graphed(m, kv, T, gq, canvas_out, n_forwards, router_load, st);
+  return generate_impl(m, kv, T, gq, canvas_out, n_forwards, router_load, st);
 }
 
 dg_status dg_eb_sample(const float* entropy, const int32_t* argmax, int32_t* canvas,
@@ -741,7 +849,11 @@ dg_status dg_op_moe(dg_model* m, int32_t layer, const float* x, float* out, int3
 
 dg_status dg_profile_start(dg_model* m) {
   DG_REQUIRE(m, "null model");
-  for (int k = 0; k < DG_KIND_COUNT; ++k) m->prof_used[k] = 0;
+  for (int k = 0; k < DG_KIND_COUNT; ++k) {
+    m->prof_used[k] = 0;
+    m->prof_acc_ms[k] = 0.0;
+    m->prof_acc_n[k] = 0;
+  }
   DG_TRY_CUDA(cudaDeviceSynchronize());
   DG_TRY_CUDA(cudaMemset(m->ws.units, 0, sizeof(unsigned long long)));
   m->profiling = true;
@@ -768,8 +880,8 @@ dg_status dg_profile_stop(dg_model* m, float* ms, int64_t* groups) {
       DG_TRY_CUDA(cudaEventElapsedTime(&t, m->prof[k][i].first, m->prof[k][i].second));
       tot += t;
     }
-    if (ms) ms[k] = (float)tot;
-    if (groups) groups[k] = (int64_t)m->prof_used[k];
+    if (ms) ms[k] = (float)(tot + m->prof_acc_ms[k]);
+    if (groups) groups[k] = (int64_t)m->prof_used[k] + m->prof_acc_n[k];
     m->prof_used[k] = 0;
   }
   return DG_OK;

@@ -81,6 +81,20 @@ struct Workspace {
 
 }  // namespace dg
 
+namespace dg {
+// A captured block (T forwards + sampler steps) and what it was captured for.
+struct BlockGraph {
+  cudaGraphExec_t exec = nullptr;
+  const dg_kv* kv = nullptr;
+  int T = 0;
+  long long gq = 0;
+  int32_t *canvas = nullptr, *nfwd = nullptr, *load = nullptr;
+  bool prof = false;
+  long long launches = 0;  // kernel launches the graph replays
+  std::vector<std::pair<cudaEvent_t, cudaEvent_t>> ev[DG_KIND_COUNT];
+};
+}  // namespace dg
+
 struct dg_model {
   dg_config cfg;
   dg_weights w;
@@ -92,7 +106,17 @@ struct dg_model {
   bool profiling = false;
   std::vector<std::pair<cudaEvent_t, cudaEvent_t>> prof[DG_KIND_COUNT];
   size_t prof_used[DG_KIND_COUNT] = {0, 0, 0, 0};
+  double prof_acc_ms[DG_KIND_COUNT] = {0, 0, 0, 0};  // from graph replays
+  int64_t prof_acc_n[DG_KIND_COUNT] = {0, 0, 0, 0};
+  // captured blocks
+  bool use_graphs = true;
+  std::vector<dg::BlockGraph*> graphs;
+  dg::BlockGraph* capture = nullptr;  // graph being captured (events go there)
 };
+
+namespace dg {
+void release_graphs(dg_model* m);
+}
 
 namespace dg {
 // RAII bracket recording a start/stop event pair around a launch group.
@@ -103,6 +127,15 @@ struct ProfScope {
   cudaEvent_t stop = nullptr;
   ProfScope(dg_model* m_, int kind_, cudaStream_t st_) : m(m_), kind(kind_), st(st_) {
     if (!m->profiling) return;
+    if (m->capture) {  // events owned by the graph being captured
+      cudaEvent_t a, b;
+      cudaEventCreate(&a);
+      cudaEventCreate(&b);
+      m->capture->ev[kind].push_back({a, b});
+      cudaEventRecord(a, st);
+      stop = b;
+      return;
+    }
     auto& pool = m->prof[kind];
     size_t& used = m->prof_used[kind];
     if (used == pool.size()) {

@@ -31,6 +31,7 @@ struct MapKeyHash {
 
 struct TcState {
   PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  int n_sm = 148;
   std::unordered_map<MapKey, CUtensorMap, MapKeyHash> maps;
 };
 
@@ -98,11 +99,6 @@ dg_status launch_dense(dg_model* m, const CUtensorMap& a, const CUtensorMap& b,
                        const CUtensorMap& b2, int M, int N, int K, Epi epi, cudaStream_t st) {
   typedef DenseCfg<BN, MT, DUAL, ST> Cfg;
   auto kern = tc_dense_kernel<BN, MT, DUAL, ST, Epi>;
-  static int ready_dev = -1;
-  if (ready_dev != m->device) {
-    DG_TRY(set_smem(kern, Cfg::SMEM));
-    ready_dev = m->device;
-  }
   dim3 grid(ceil_div_i(M, 128 * MT), ceil_div_i(N, BN));
   kern<<<grid, 128, Cfg::SMEM, st>>>(a, b, b2, M, K, epi, m->ws.err);
   ++m->launches;
@@ -138,8 +134,23 @@ dg_status tc_prepare(dg_model* m) {
     return DG_ERR_CUDA;
   }
   s->encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-  std::lock_guard<std::mutex> lk(g_tc_mu);
-  g_tc[m] = s;
+  {
+    std::lock_guard<std::mutex> lk(g_tc_mu);
+    g_tc[m] = s;
+  }
+  // dynamic shared-memory limits, set once here so that no attribute call happens
+  // while a launch sequence is being captured into a graph
+  typedef DenseCfg<DENSE_BN, DENSE_MT, false, DENSE_ST> Dn;
+  typedef DenseCfg<DENSE_BN, DENSE_MT, true, DUAL_ST> Du;
+  typedef DenseCfg<LM_BN, 2, false, LM_ST> Lm;
+  DG_TRY(set_smem(tc_dense_kernel<DENSE_BN, DENSE_MT, false, DENSE_ST, EpiStoreF32>, Dn::SMEM));
+  DG_TRY(set_smem(tc_dense_kernel<DENSE_BN, DENSE_MT, false, DENSE_ST, EpiAddF32>, Dn::SMEM));
+  DG_TRY(set_smem(tc_dense_kernel<DENSE_BN, DENSE_MT, true, DUAL_ST, EpiSwigluBf16>, Du::SMEM));
+  DG_TRY(set_smem(tc_dense_kernel<LM_BN, 2, false, LM_ST, EpiLmStats>, Lm::SMEM));
+  DG_TRY(set_smem(tc_expert_kernel<true, GU_ST>, ExpertCfg<true, GU_ST>::SMEM));
+  DG_TRY(set_smem(tc_expert_kernel<false, DN_ST>, ExpertCfg<false, DN_ST>::SMEM));
+  DG_TRY(set_smem(tc_attn_kernel, AT_SMEM));
+  cudaDeviceGetAttribute(&s->n_sm, cudaDevAttrMultiProcessorCount, m->device);
   return DG_OK;
 }
 
@@ -210,13 +221,7 @@ static dg_status launch_expert(dg_model* m, const CUtensorMap& w, const CUtensor
                                const float* gate_of, cudaStream_t st) {
   typedef ExpertCfg<GATEUP, ST> Cfg;
   auto kern = tc_expert_kernel<GATEUP, ST>;
-  static int ready_dev = -1;
-  if (ready_dev != m->device) {
-    DG_TRY(set_smem(kern, Cfg::SMEM));
-    ready_dev = m->device;
-  }
-  int n_sm = 148;
-  cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, m->device);
+  const int n_sm = state(m)->n_sm;
   const Workspace& ws = m->ws;
   kern<<<n_sm, 192, Cfg::SMEM, st>>>(w, w2, x, ws.tile_e, ws.tile_m0, ws.n_tiles, ws.offsets,
                                      w_rows, K, FT, out, ldo, gate_of, ws.err);
@@ -294,18 +299,12 @@ dg_status tc_attention(dg_model* m, const bf16* q, int B, int nq, int qpos0, con
   const int total = causal ? std::min(TB, ceil_div_i(c.window + 127, AT_KT) + 1) : TA + TB;
   const int qtiles = ceil_div_i(nq, 128);
   const int base = qtiles * Hq * B;
-  int n_sm = 148;
-  cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, m->device);
+  const int n_sm = state(m)->n_sm;
   int splits = std::min(ceil_div_i(2 * n_sm, base), std::min((int)ATT_MAX_SPLITS, total));
   splits = std::max(1, splits);
   const int tps = ceil_div_i(total, splits);
   splits = ceil_div_i(total, tps);
   p.tiles_per_split = tps;
-  static int ready_dev = -1;
-  if (ready_dev != m->device) {
-    DG_TRY(set_smem(tc_attn_kernel, AT_SMEM));
-    ready_dev = m->device;
-  }
   dim3 grid(qtiles * Hq, B, splits);
   tc_attn_kernel<<<grid, 128, AT_SMEM, st>>>(mQ, mKA, mVA, mKB, mVB, p, m->ws.err);
   ++m->launches;

@@ -92,3 +92,17 @@ def test_block_invariants(setup):
         prev = dm.clone()
     binding.dg_sync_status(model)
     assert torch.equal(dc, out)
+
+
+def test_block_graph_replay_is_deterministic(setup):
+    """The captured block replays to bit-identical canvases and routing counts."""
+    binding, model, kv, ws, okv = setup
+    outs = []
+    for _ in range(3):
+        load = torch.zeros(W.n_layers, W.n_experts, dtype=torch.int32, device="cuda")
+        out = torch.empty(W.batch, W.canvas, dtype=torch.int32, device="cuda")
+        binding.dg_generate_block(model, kv, W.T, W.gamma, canvas_out=out, router_load=load)
+        outs.append((out.clone(), load.clone()))
+    binding.dg_sync_status(model)
+    for o, l in outs[1:]:
+        assert torch.equal(o, outs[0][0]) and torch.equal(l, outs[0][1])
