@@ -555,6 +555,7 @@ dg_status dg_model_destroy(dg_model* m) {
   if (!m) return DG_OK;
   cudaDeviceSynchronize();
   release_graphs(m);
+  if (m->cap_stream) cudaStreamDestroy(m->cap_stream);
   for (int k = 0; k < DG_KIND_COUNT; ++k)
     for (auto& e : m->prof[k]) {
       cudaEventDestroy(e.first);
@@ -754,12 +755,16 @@ static dg_status generate_graphed(dg_model* m, const dg_kv* kv, int32_t T, long 
     g->prof = m->profiling;
     const long long l0 = m->launches;
     m->capture = g;
+    // capture on a library-owned stream (the caller's may be the legacy default
+    // stream, which cannot be captured); nothing executes during capture
     cudaGraph_t graph = nullptr;
-    cudaError_t e = cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal);
+    cudaError_t e = cudaSuccess;
+    if (!m->cap_stream) e = cudaStreamCreateWithFlags(&m->cap_stream, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamBeginCapture(m->cap_stream, cudaStreamCaptureModeThreadLocal);
     dg_status s = DG_OK;
     if (e == cudaSuccess) {
-      s = generate_impl(m, kv, T, gq, canvas_out, n_forwards, router_load, st);
-      e = cudaStreamEndCapture(st, &graph);
+      s = generate_impl(m, kv, T, gq, canvas_out, n_forwards, router_load, m->cap_stream);
+      e = cudaStreamEndCapture(m->cap_stream, &graph);
     }
     m->capture = nullptr;
     g->launches = m->launches - l0;

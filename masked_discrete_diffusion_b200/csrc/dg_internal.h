@@ -112,6 +112,7 @@ struct dg_model {
   bool use_graphs = true;
   std::vector<dg::BlockGraph*> graphs;
   dg::BlockGraph* capture = nullptr;  // graph being captured (events go there)
+  cudaStream_t cap_stream = nullptr;  // private stream used only for capturing
 };
 
 namespace dg {
