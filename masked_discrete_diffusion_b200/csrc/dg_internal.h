@@ -126,6 +126,7 @@ struct ProfScope {
   int kind;
   cudaStream_t st;
   cudaEvent_t stop = nullptr;
+  bool external = false;
   ProfScope(dg_model* m_, int kind_, cudaStream_t st_) : m(m_), kind(kind_), st(st_) {
     if (!m->profiling) return;
     if (m->capture) {  // events owned by the graph being captured
@@ -133,8 +134,10 @@ struct ProfScope {
       cudaEventCreate(&a);
       cudaEventCreate(&b);
       m->capture->ev[kind].push_back({a, b});
-      cudaEventRecord(a, st);
+      // "external" records become event-record nodes that fire on every replay
+      cudaEventRecordWithFlags(a, st, cudaEventRecordExternal);
       stop = b;
+      external = true;
       return;
     }
     auto& pool = m->prof[kind];
@@ -150,7 +153,12 @@ struct ProfScope {
     ++used;
   }
   void end() {
-    if (stop) cudaEventRecord(stop, st);
+    if (stop) {
+      if (external)
+        cudaEventRecordWithFlags(stop, st, cudaEventRecordExternal);
+      else
+        cudaEventRecord(stop, st);
+    }
     stop = nullptr;
   }
   ~ProfScope() { end(); }
