@@ -287,9 +287,15 @@ template <class Path> struct Runner {
       router_logits_kernel<TR, TW, Acc><<<grid, 256, 0, st>>>(x(), (const TW*)L.router, n, d, E,
                                                               kps, (Acc*)ws.rlog);
       ++m->launches;
-      router_topk_kernel<Acc><<<ceil_div(n, 4), 128, 0, st>>>((const Acc*)ws.rlog, ks,
-                                                              (const Acc*)ws.inv_rms, n, E, k,
-                                                              ws.ridx, (Acc*)ws.rgate, load);
+      if (E <= 32)
+        router_topk_kernel<Acc, 1><<<ceil_div(n, 4), 128, 0, st>>>(
+            (const Acc*)ws.rlog, ks, (const Acc*)ws.inv_rms, n, E, k, ws.ridx, (Acc*)ws.rgate, load);
+      else if (E <= 128)
+        router_topk_kernel<Acc, 4><<<ceil_div(n, 4), 128, 0, st>>>(
+            (const Acc*)ws.rlog, ks, (const Acc*)ws.inv_rms, n, E, k, ws.ridx, (Acc*)ws.rgate, load);
+      else
+        router_topk_kernel<Acc, 32><<<ceil_div(n, 4), 128, 0, st>>>(
+            (const Acc*)ws.rlog, ks, (const Acc*)ws.inv_rms, n, E, k, ws.ridx, (Acc*)ws.rgate, load);
       ++m->launches;
     }
     moe_rank_kernel<<<E, 256, 0, st>>>(ws.ridx, n_ent, ws.rank, ws.counts);
@@ -337,7 +343,7 @@ template <class Path> struct Runner {
                                           EpiSwiglu<TA, Acc>{(TA*)ws.sh, Is}, st, &m->launches);
       dense((const TA*)ws.sh, Is, L.sdown, d, Is, n, EpiStore<Acc, Acc>{(Acc*)ws.ys, d});
     }
-    moe_combine_kernel<TR, Acc, Acc><<<n, 256, 0, st>>>(x(), (const Acc*)ws.ys,
+    moe_combine_kernel<TR, Acc, Acc><<<dim3(n, ceil_div(d, 128)), 128, 0, st>>>(x(), (const Acc*)ws.ys,
                                                         (const Acc*)ws.yb, ws.row_of, n, d, k);
     ++m->launches;
     return check_launch("moe");

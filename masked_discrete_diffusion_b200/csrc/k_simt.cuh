@@ -371,12 +371,11 @@ __global__ void __launch_bounds__(256)
     }
 }
 
-template <class Acc>
+template <class Acc, int MAXE>  // MAXE experts per lane: E <= 32 * MAXE
 __global__ void router_topk_kernel(const Acc* __restrict__ part, int splits,
                                    const Acc* __restrict__ inv_rms, int n, int E, int top_k,
                                    int32_t* __restrict__ idx, Acc* __restrict__ gate,
                                    int32_t* __restrict__ load) {
-  constexpr int MAXE = 32;  // experts per lane (E <= 1024)
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= n) return;
@@ -407,8 +406,8 @@ __global__ void router_topk_kernel(const Acc* __restrict__ part, int splits,
   for (int q = 0; q < MAXE; ++q) pr[q] /= z;
   unsigned taken = 0;  // bit q: expert lane + 32 q already selected
   Acc gsum = 0;
-  int sel_e[64];
-  Acc sel_p[64];
+  int my_e = 0;   // lane k keeps the k-th selection
+  Acc my_p = 0;
   for (int k = 0; k < top_k; ++k) {
     Acc bp = -1;
     int be = 0x7fffffff;
@@ -430,21 +429,16 @@ __global__ void router_topk_kernel(const Acc* __restrict__ part, int splits,
       }
     }
     if ((be & 31) == lane) taken |= 1u << (be >> 5);
-    sel_e[k] = be;
-    sel_p[k] = bp;
+    if (lane == k) {
+      my_e = be;
+      my_p = bp;
+    }
     gsum += bp;
   }
   if (lane < top_k) {
-    int e = 0;
-    Acc pk = 0;
-    for (int k = 0; k < top_k; ++k)
-      if (k == lane) {
-        e = sel_e[k];
-        pk = sel_p[k];
-      }
-    idx[(size_t)t * top_k + lane] = e;
-    gate[(size_t)t * top_k + lane] = pk / gsum;
-    if (load) atomicAdd(&load[e], 1);
+    idx[(size_t)t * top_k + lane] = my_e;
+    gate[(size_t)t * top_k + lane] = my_p / gsum;
+    if (load) atomicAdd(&load[my_e], 1);
   }
 }
 
@@ -547,13 +541,16 @@ __global__ void gather_rows_kernel(const TA* __restrict__ src, const int32_t* __
 }
 
 // x[t] += ys[t] + sum over slots of yb[row_of[t * k + slot]] (slot order fixed).
+// grid (n_tok, ceil(d / blockDim)).
 template <class TR, class TY, class Acc>
 __global__ void moe_combine_kernel(TR* __restrict__ x, const TY* __restrict__ ys,
                                    const TY* __restrict__ yb, const int32_t* __restrict__ row_of,
                                    int n_tok, int d, int top_k) {
   const int t = blockIdx.x;
   if (t >= n_tok) return;
-  for (int c = threadIdx.x; c < d; c += blockDim.x) {
+  {
+    const int c = blockIdx.y * blockDim.x + threadIdx.x;
+    if (c >= d) return;
     Acc y = (Acc)widen(ys[(size_t)t * d + c]);
     for (int k = 0; k < top_k; ++k)
       y += (Acc)widen(yb[(size_t)row_of[(size_t)t * top_k + k] * d + c]);

@@ -6,7 +6,7 @@
 //     softmax statistics (the logits never leave the SM).
 //   * tc_expert_kernel — grouped routed-expert GEMM, weights as the MMA A operand
 //     (128 weight rows per tile) and the expert's gathered token rows as the B
-//     operand (N = tokens rounded up to 32, <= 256), persistent over work units
+//     operand (N = tokens rounded up to 32, <= 128), persistent over work units
 //     (token chunk, weight-row tile); SwiGLU or gate-weighted epilogue.
 // Operands are staged by TMA (no multicast) into 128-byte-swizzled K-major
 // tiles; accumulators live in TMEM and are read back with tcgen05.ld.
@@ -41,76 +41,71 @@ template <int COLS> struct TmemCols {
 // epilogues of the dense kernel: run(row, valid, n0, ld) with ld(acc, chunk, v)
 // loading 32 fp32 columns of accumulator `acc` (0, or 1 for the second weight).
 // ---------------------------------------------------------------------------
-struct EpiStoreF32 {
-  float* out;
-  int ldo, N;
+// Chunk epilogues: chunk(row, col, v, u) consumes 32 consecutive columns of one row
+// (v: the accumulator, u: the second weight's accumulator for dual GEMMs).
+template <class Derived, bool DUAL>
+struct EpiChunked {
+  static constexpr bool kChunked = true;
   template <int NCH, class Ld>
   __device__ void run(int row, bool valid, int n0, Ld&& ld) const {
 #pragma unroll 1
     for (int c = 0; c < NCH; ++c) {
-      float v[32];
+      float v[32], u[32];
       ld(0, c, v);
-      const int col = n0 + c * 32;
-      if (valid && col < N) {
-        float4* p = reinterpret_cast<float4*>(out + (size_t)row * ldo + col);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) p[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-      }
+      if (DUAL) ld(1, c, u);
+      static_cast<const Derived*>(this)->chunk(row, valid, n0 + c * 32, v, u);
     }
   }
 };
 
-struct EpiAddF32 {
+struct EpiStoreF32 : EpiChunked<EpiStoreF32, false> {
   float* out;
   int ldo, N;
-  template <int NCH, class Ld>
-  __device__ void run(int row, bool valid, int n0, Ld&& ld) const {
-#pragma unroll 1
-    for (int c = 0; c < NCH; ++c) {
-      float v[32];
-      ld(0, c, v);
-      const int col = n0 + c * 32;
-      if (valid && col < N) {
-        float4* p = reinterpret_cast<float4*>(out + (size_t)row * ldo + col);
+  EpiStoreF32(float* o, int l, int n) : out(o), ldo(l), N(n) {}
+  __device__ void chunk(int row, bool valid, int col, const float* v, const float*) const {
+    if (!valid || col >= N) return;
+    float4* p = reinterpret_cast<float4*>(out + (size_t)row * ldo + col);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          float4 o = p[j];
-          o.x += v[4 * j];
-          o.y += v[4 * j + 1];
-          o.z += v[4 * j + 2];
-          o.w += v[4 * j + 3];
-          p[j] = o;
-        }
-      }
+    for (int j = 0; j < 8; ++j) p[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+  }
+};
+
+struct EpiAddF32 : EpiChunked<EpiAddF32, false> {
+  float* out;
+  int ldo, N;
+  EpiAddF32(float* o, int l, int n) : out(o), ldo(l), N(n) {}
+  __device__ void chunk(int row, bool valid, int col, const float* v, const float*) const {
+    if (!valid || col >= N) return;
+    float4* p = reinterpret_cast<float4*>(out + (size_t)row * ldo + col);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      float4 o = p[j];
+      o.x += v[4 * j];
+      o.y += v[4 * j + 1];
+      o.z += v[4 * j + 2];
+      o.w += v[4 * j + 3];
+      p[j] = o;
     }
   }
 };
 
-struct EpiSwigluBf16 {
+struct EpiSwigluBf16 : EpiChunked<EpiSwigluBf16, true> {
   bf16* out;
   int ldo, N;
-  template <int NCH, class Ld>
-  __device__ void run(int row, bool valid, int n0, Ld&& ld) const {
-#pragma unroll 1
-    for (int c = 0; c < NCH; ++c) {
-      float g[32], u[32];
-      ld(0, c, g);
-      ld(1, c, u);
-      const int col = n0 + c * 32;
-      if (valid && col < N) {
-        uint4* p = reinterpret_cast<uint4*>(out + (size_t)row * ldo + col);
+  EpiSwigluBf16(bf16* o, int l, int n) : out(o), ldo(l), N(n) {}
+  __device__ void chunk(int row, bool valid, int col, const float* g, const float* u) const {
+    if (!valid || col >= N) return;
+    uint4* p = reinterpret_cast<uint4*>(out + (size_t)row * ldo + col);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint32_t w[4];
+    for (int j = 0; j < 4; ++j) {
+      uint32_t w[4];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int i = 8 * j + 2 * q;
-            __nv_bfloat162 b2 = __floats2bfloat162_rn(silu(g[i]) * u[i], silu(g[i + 1]) * u[i + 1]);
-            w[q] = *reinterpret_cast<uint32_t*>(&b2);
-          }
-          p[j] = make_uint4(w[0], w[1], w[2], w[3]);
-        }
+      for (int q = 0; q < 4; ++q) {
+        const int i = 8 * j + 2 * q;
+        __nv_bfloat162 b2 = __floats2bfloat162_rn(silu(g[i]) * u[i], silu(g[i + 1]) * u[i + 1]);
+        w[q] = *reinterpret_cast<uint32_t*>(&b2);
       }
+      p[j] = make_uint4(w[0], w[1], w[2], w[3]);
     }
   }
 };
@@ -119,6 +114,7 @@ struct EpiSwigluBf16 {
 // (columns n0 .. n0 + 32 NCH - 1, those < N): m = max, s = sum exp(l - m),
 // u = sum exp(l - m) (l - m), a = lowest id attaining m.  part[(tile, row)] = (m, s, u, a).
 struct EpiLmStats {
+  static constexpr bool kChunked = false;
   float* part;
   int M, N;
   float scale;
@@ -163,10 +159,37 @@ struct EpiLmStats {
 };
 
 // ---------------------------------------------------------------------------
-// dense kernel: grid (ceil(M / (128 MT)), ceil(N / BN)); 128 threads.
+// dense kernel: grid (ceil(M / (128 MT)), ceil(N / BN), ksplit); 128 threads.
 // warp 0 lane 0: TMA producer; warp 1 lane 0: MMA issuer; warp 2: TMEM owner;
 // all four warps: epilogue (warp w reads accumulator lanes 32w .. 32w + 31).
+// ksplit > 1 (launched as clusters of ksplit CTAs along z): CTA r accumulates the
+// r-th slice of K; the partial tiles are then reduced through distributed shared
+// memory: CTA r owns rows [r R, (r+1) R) of the tile (R = 128 MT / ksplit),
+// receives every CTA's partial rows into slot [source rank], sums the slots in
+// rank order (deterministic) and runs the epilogue for its rows.
 // ---------------------------------------------------------------------------
+namespace cl {
+__device__ __forceinline__ uint32_t ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+__device__ __forceinline__ uint32_t map(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void st4(uint32_t addr, float a, float b, float c, float d) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b),
+               "f"(c), "f"(d)
+               : "memory");
+}
+}  // namespace cl
+
 template <int BN, int MT, bool DUAL, int ST>
 struct DenseCfg {
   static constexpr int NACC = DUAL ? 2 : 1;
@@ -181,9 +204,11 @@ struct DenseCfg {
 template <int BN, int MT, bool DUAL, int ST, class Epi>
 __global__ void __launch_bounds__(128, 1)
     tc_dense_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mB,
-                    const __grid_constant__ CUtensorMap mB2, int M, int K, Epi epi,
+                    const __grid_constant__ CUtensorMap mB2, int M, int K, int ksplit, Epi epi,
                     int32_t* err) {
   typedef DenseCfg<BN, MT, DUAL, ST> Cfg;
+  // split-K needs the whole fp32 tile in the (drained) pipeline buffers and a chunk epilogue
+  constexpr bool kSplitOK = MT * 128 * Cfg::NACC * BN * 4 <= ST * Cfg::STAGE && Epi::kChunked;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + ST * Cfg::STAGE);
@@ -193,7 +218,10 @@ __global__ void __launch_bounds__(128, 1)
   int* abort_flag = reinterpret_cast<int*>(tslot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * (MT * 128), n0 = blockIdx.y * BN;
-  const int nk = (K + TC_KB - 1) / TC_KB;
+  const int nk_all = (K + TC_KB - 1) / TC_KB;
+  const int rank = ksplit > 1 ? (int)cl::ctarank() : 0;
+  const int kb_lo = (int)((long)nk_all * rank / ksplit);
+  const int nk = (int)((long)nk_all * (rank + 1) / ksplit) - kb_lo;
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -225,10 +253,11 @@ __global__ void __launch_bounds__(128, 1)
       uint8_t* st = smem + s * Cfg::STAGE;
       tc::mbar_expect_tx(full + s, Cfg::STAGE);
 #pragma unroll
+      const int kx = (kb_lo + kb) * TC_KB;
       for (int mt = 0; mt < MT; ++mt)
-        tc::tma_load_2d(st + mt * TC_SUB_A, &mA, full + s, kb * TC_KB, m0 + mt * 128);
-      tc::tma_load_2d(st + MT * TC_SUB_A, &mB, full + s, kb * TC_KB, n0);
-      if (DUAL) tc::tma_load_2d(st + MT * TC_SUB_A + Cfg::B_BYTES, &mB2, full + s, kb * TC_KB, n0);
+        tc::tma_load_2d(st + mt * TC_SUB_A, &mA, full + s, kx, m0 + mt * 128);
+      tc::tma_load_2d(st + MT * TC_SUB_A, &mB, full + s, kx, n0);
+      if (DUAL) tc::tma_load_2d(st + MT * TC_SUB_A + Cfg::B_BYTES, &mB2, full + s, kx, n0);
     }
   } else if (warp == 1 && lane == 0) {
     constexpr uint32_t idesc = tc::idesc_bf16(128, BN);
@@ -265,20 +294,69 @@ __global__ void __launch_bounds__(128, 1)
 
   // epilogue: wait for the accumulators
   bool ready = true;
-  if (lane == 0) ready = tc::mbar_wait(done, 0);
+  if (lane == 0) ready = nk == 0 || tc::mbar_wait(done, 0);
   ready = __shfl_sync(0xffffffffu, ready ? 1 : 0, 0) != 0;
-  if (!ready) {
-    if (lane == 0) atomicOr(err, ERR_TIMEOUT);
-  } else {
-    tc::fence_after_sync();
-    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+  if (!ready && lane == 0) atomicOr(err, ERR_TIMEOUT);
+  const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+  if (ksplit == 1) {
+    if (ready) {
+      tc::fence_after_sync();
 #pragma unroll 1
-    for (int mt = 0; mt < MT; ++mt) {
-      const int row = m0 + mt * 128 + 32 * warp + lane;
-      auto ld = [&](int a, int c, float* v) {
-        tc::tmem_ld32(tmem + lane_base + (mt * Cfg::NACC + a) * BN + c * 32, v);
-      };
-      epi.template run<BN / 32>(row, row < M, n0, ld);
+      for (int mt = 0; mt < MT; ++mt) {
+        const int row = m0 + mt * 128 + 32 * warp + lane;
+        auto ld = [&](int a, int c, float* v) {
+          tc::tmem_ld32(tmem + lane_base + (mt * Cfg::NACC + a) * BN + c * 32, v);
+        };
+        epi.template run<BN / 32>(row, row < M, n0, ld);
+      }
+    }
+  } else if constexpr (kSplitOK) {
+    // every thread of every CTA passes both cluster barriers, whatever happened above
+    constexpr int W = Cfg::NACC * BN;        // fp32 values per tile row
+    const int R = MT * 128 / ksplit;         // rows owned per CTA
+    cl::sync();                              // all pipelines drained: smem reusable
+    if (ready) {
+      tc::fence_after_sync();
+      const uint32_t recv = tc::smem_addr(smem);
+#pragma unroll 1
+      for (int mt = 0; mt < MT; ++mt) {
+        const int trow = mt * 128 + 32 * warp + lane;  // row within the tile
+        const int owner = trow / R, lr = trow % R;
+        const uint32_t dst = cl::map(recv, owner) + (uint32_t)(((rank * R + lr) * W) * 4);
+#pragma unroll 1
+        for (int a = 0; a < Cfg::NACC; ++a)
+#pragma unroll 1
+          for (int c = 0; c < BN / 32; ++c) {
+            float v[32];
+            tc::tmem_ld32(tmem + lane_base + (mt * Cfg::NACC + a) * BN + c * 32, v);
+            const uint32_t o = dst + (uint32_t)((a * BN + c * 32) * 4);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              cl::st4(o + 16 * j, v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+          }
+      }
+    }
+    cl::sync();                              // all partial rows delivered
+    const float* buf = reinterpret_cast<const float*>(smem);
+    for (int item = threadIdx.x; item < R * (BN / 32); item += blockDim.x) {
+      const int lr = item / (BN / 32), c = item % (BN / 32);
+      float v[32], u[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        v[j] = 0.f;
+        u[j] = 0.f;
+      }
+      for (int src = 0; src < ksplit; ++src) {
+        const float* p = buf + (size_t)(src * R + lr) * W + c * 32;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] += p[j];
+        if (DUAL) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) u[j] += p[BN + j];
+        }
+      }
+      const int row = m0 + rank * R + lr;
+      epi.chunk(row, row < M, n0 + c * 32, v, u);
     }
   }
   tc::fence_before_sync();
@@ -289,7 +367,7 @@ __global__ void __launch_bounds__(128, 1)
 // ---------------------------------------------------------------------------
 // grouped expert kernel (persistent).  Work unit u = chunk * FT + f: token chunk
 // `chunk` (expert e = chunk_e[chunk], permuted rows r0 = chunk_r0[chunk] ..
-// r0 + n - 1, n <= 256) times weight-row tile f (128 rows of the expert's
+// r0 + n - 1, n <= 128) times weight-row tile f (128 rows of the expert's
 // weight).  GATEUP: two weights (gate, up) [E*I, d] -> hb[r, f*128 + i] =
 // silu(g) * u (bf16).  Otherwise: down [E*d, I] -> yb[r, f*128 + i] =
 // gate_of[r] * acc (fp32).
@@ -300,9 +378,9 @@ __global__ void __launch_bounds__(128, 1)
 template <bool GATEUP, int ST>
 struct ExpertCfg {
   static constexpr int NW = GATEUP ? 2 : 1;
-  static constexpr uint32_t B_MAX = 256 * TC_KB * 2;
+  static constexpr uint32_t B_MAX = 128 * TC_KB * 2;
   static constexpr uint32_t STAGE = NW * TC_SUB_A + B_MAX;
-  static constexpr uint32_t TCOLS = GATEUP ? 512 : 256;
+  static constexpr uint32_t TCOLS = GATEUP ? 256 : 128;
   static constexpr size_t SMEM = 1024 + (size_t)ST * STAGE + 256;
 };
 
@@ -346,7 +424,7 @@ __global__ void __launch_bounds__(192, 1)
     f = u % FT;
     e = chunk_e[c];
     r0 = chunk_r0[c];
-    n = min(256, offsets[e + 1] - r0);
+    n = min(128, offsets[e + 1] - r0);
   };
 
   if (warp == 0) {
@@ -410,7 +488,7 @@ __global__ void __launch_bounds__(192, 1)
             const uint32_t acc = (kb | k) != 0;
             const uint64_t bd = tc::sdesc_k128(b0 + k * 32);
             tc::mma_bf16(tmem, tc::sdesc_k128(a0 + k * 32), bd, idesc, acc);
-            if (GATEUP) tc::mma_bf16(tmem + 256, tc::sdesc_k128(a0 + TC_SUB_A + k * 32), bd, idesc, acc);
+            if (GATEUP) tc::mma_bf16(tmem + 128, tc::sdesc_k128(a0 + TC_SUB_A + k * 32), bd, idesc, acc);
           }
           tc::mma_commit(empty + s);
         }
@@ -441,7 +519,7 @@ __global__ void __launch_bounds__(192, 1)
         tc::tmem_ld32(tmem + lane_base + c * 32, v);
         if (GATEUP) {
           float g2[32];
-          tc::tmem_ld32(tmem + lane_base + 256 + c * 32, g2);
+          tc::tmem_ld32(tmem + lane_base + 128 + c * 32, g2);
           bf16* o = reinterpret_cast<bf16*>(out);
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
@@ -472,7 +550,7 @@ __global__ void __launch_bounds__(192, 1)
 // ---------------------------------------------------------------------------
 dg_status tc_prepare(dg_model* m);
 void tc_release(dg_model* m);
-inline int tc_group_rows() { return 256; }
+inline int tc_group_rows() { return 128; }
 dg_status tc_gemm_store_f32(dg_model* m, const bf16* A, const void* W, float* out, int M, int N,
                             int K, cudaStream_t st);
 dg_status tc_gemm_f32_rows(dg_model* m, const bf16* A, int a_rows, const void* W, float* out,

@@ -94,15 +94,40 @@ template <class K> dg_status set_smem(K kern, size_t bytes) {
   return DG_OK;
 }
 
+// Split K over a cluster when the (M, N) tiles alone would leave most SMs idle.
 template <int BN, int MT, bool DUAL, int ST, class Epi>
 dg_status launch_dense(dg_model* m, const CUtensorMap& a, const CUtensorMap& b,
-                       const CUtensorMap& b2, int M, int N, int K, Epi epi, cudaStream_t st) {
+                       const CUtensorMap& b2, int M, int N, int K, Epi epi, cudaStream_t st,
+                       bool allow_split = true) {
   typedef DenseCfg<BN, MT, DUAL, ST> Cfg;
   auto kern = tc_dense_kernel<BN, MT, DUAL, ST, Epi>;
-  dim3 grid(ceil_div_i(M, 128 * MT), ceil_div_i(N, BN));
-  kern<<<grid, 128, Cfg::SMEM, st>>>(a, b, b2, M, K, epi, m->ws.err);
+  dim3 grid(ceil_div_i(M, 128 * MT), ceil_div_i(N, BN), 1);
+  const int tiles = grid.x * grid.y;
+  const int nk = ceil_div_i(K, TC_KB);
+  int ks = 1;
+  if (allow_split)
+    while (ks < 8 && tiles * ks * 2 <= state(m)->n_sm && nk >= ks * 2 * 2) ks *= 2;
+  cudaError_t e;
+  if (ks == 1) {
+    kern<<<grid, 128, Cfg::SMEM, st>>>(a, b, b2, M, K, 1, epi, m->ws.err);
+    e = cudaGetLastError();
+  } else {
+    grid.z = ks;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(128, 1, 1);
+    cfg.dynamicSmemBytes = Cfg::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = ks;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, a, b, b2, M, K, ks, epi, m->ws.err);
+  }
   ++m->launches;
-  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_error("tc_dense launch: %s", cudaGetErrorString(e));
     return DG_ERR_CUDA;
@@ -112,7 +137,7 @@ dg_status launch_dense(dg_model* m, const CUtensorMap& a, const CUtensorMap& b,
 
 constexpr int DENSE_BN = 64, DENSE_MT = 2, DENSE_ST = 5, DUAL_ST = 4;
 constexpr int LM_BN = 256, LM_ST = 3;
-constexpr int GU_ST = 3, DN_ST = 4;
+constexpr int GU_ST = 4, DN_ST = 6;
 
 }  // namespace
 
@@ -208,7 +233,8 @@ dg_status tc_lmhead_stats(dg_model* m, const bf16* xn, int M, float* ent, int32_
   DG_TRY(tmap(m, m->w.lm_head, c.vocab, c.d_model, LM_BN, &b));
   float* part = (float*)m->ws.lm_part;
   DG_TRY((launch_dense<LM_BN, 2, false, LM_ST>(m, a, b, b, M, c.vocab, c.d_model,
-                                               EpiLmStats{part, M, c.vocab, c.logit_scale}, st)));
+                                               EpiLmStats{part, M, c.vocab, c.logit_scale}, st,
+                                               false)));
   const int n_vt = ceil_div_i(c.vocab, LM_BN);
   lm_merge_kernel<float><<<ceil_div_i(M, 4), 128, 0, st>>>(part, n_vt, M, ent, amax);
   ++m->launches;

@@ -24,8 +24,11 @@ def small():
     m.close()
 
 
+# (256, 2048, 2048), (256, 4096, 2048) and (100, 1024, 512) run as clusters that split K
+# (4, 2 and 4 ways) and reduce the partial tiles through distributed shared memory.
 @pytest.mark.parametrize("M,N,K", [(256, 512, 256), (200, 192, 128), (300, 64, 64), (1, 64, 64),
-                                   (520, 4096, 2048)])
+                                   (520, 4096, 2048), (256, 2048, 2048), (256, 4096, 2048),
+                                   (100, 1024, 512)])
 def test_tc_gemm_matches_fp64(small, M, N, K):
     from masked_discrete_diffusion_b200 import binding
     A = gen.normal_values(1, f"A{M}", 0, M * K, 1.0, "cuda").reshape(M, K).to(torch.bfloat16)
