@@ -222,6 +222,7 @@ __global__ void __launch_bounds__(128, 1)
   const int rank = ksplit > 1 ? (int)cl::ctarank() : 0;
   const int kb_lo = (int)((long)nk_all * rank / ksplit);
   const int nk = (int)((long)nk_all * (rank + 1) / ksplit) - kb_lo;
+  const int rot = nk > 0 ? (int)(blockIdx.y % nk) : 0;
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -253,7 +254,9 @@ __global__ void __launch_bounds__(128, 1)
       uint8_t* st = smem + s * Cfg::STAGE;
       tc::mbar_expect_tx(full + s, Cfg::STAGE);
 #pragma unroll
-      const int kx = (kb_lo + kb) * TC_KB;
+      // CTAs start their K walk at different offsets so that they do not all read
+      // the same activation tile from the same L2 slices at the same time
+      const int kx = (kb_lo + (kb + rot) % nk) * TC_KB;
       for (int mt = 0; mt < MT; ++mt)
         tc::tma_load_2d(st + mt * TC_SUB_A, &mA, full + s, kx, m0 + mt * 128);
       tc::tma_load_2d(st + MT * TC_SUB_A, &mB, full + s, kx, n0);
@@ -448,12 +451,14 @@ __global__ void __launch_bounds__(192, 1)
             break;
           }
           uint8_t* st = smem + s * Cfg::STAGE;
+          // units of one token chunk start their K walk at different offsets
+          const int kx = ((kb + f) % nk) * TC_KB;
           tc::mbar_expect_tx(full + s, bytes);
-          tc::tma_load_2d(st, &mW, full + s, kb * TC_KB, wrow);
-          if (GATEUP) tc::tma_load_2d(st + TC_SUB_A, &mW2, full + s, kb * TC_KB, wrow);
+          tc::tma_load_2d(st, &mW, full + s, kx, wrow);
+          if (GATEUP) tc::tma_load_2d(st + TC_SUB_A, &mW2, full + s, kx, wrow);
           uint8_t* bt = st + Cfg::NW * TC_SUB_A;
           for (int j = 0; j < nb; ++j)
-            tc::tma_load_2d(bt + j * 32 * TC_KB * 2, &mX, full + s, kb * TC_KB, r0 + 32 * j);
+            tc::tma_load_2d(bt + j * 32 * TC_KB * 2, &mX, full + s, kx, r0 + 32 * j);
         }
       }
     }
