@@ -216,6 +216,29 @@ dg_status dg_expert_units(dg_model* m, int64_t* units);
 /* Number of kernels this model has launched since it was created (host count). */
 dg_status dg_launch_count(const dg_model* m, int64_t* out);
 
+/* ---- allocation-free entry point (no counterpart on the pages) --------------
+ * The LM-head entropy step of the forward (final RMSNorm, logits = logit_scale *
+ * xn W_lm^T, per-row softmax entropy and argmax; the logits are never stored),
+ * for callers that cannot allocate device memory: code whose allocator belongs
+ * to another runtime, real-time or embedded callers whose device memory is fixed
+ * up front, or callers that must not touch the allocator between steps.  It
+ * needs no model handle and calls no cudaMalloc, cudaFree or allocating library
+ * routine.  Its scratch is a file-scope device array of 6 MiB (256 rows x 4096
+ * columns of bf16, plus the per-tile statistics for up to 262,144 classes) that
+ * every GPU loading the library holds until the process exits.
+ *   hidden:  [M, d] fp32 residual rows (device);  lm_head: [V, d] bf16 (device,
+ *            16-byte aligned);  entropy: [M] fp32 out;  argmax: [M] int32 out.
+ *   Limits:  1 <= M <= 256, 1 <= V <= 262144, d a multiple of 64 in [64, 4096];
+ *            larger sizes return DG_ERR_INVALID_ARG before any launch.
+ * The first call on a device (with that device current) looks up the scratch
+ * array's device address, so make that first call before any stream capture.
+ * All calls on a device share the scratch: calls whose kernels may overlap on
+ * the GPU (other streams, other host threads) race and must be serialised.  A
+ * device-side wait that gives up marks the outputs (entropy NaN, argmax -1). */
+dg_status dg_lmhead_entropy_noalloc(const float* hidden, const void* lm_head, int32_t M,
+                                    int32_t V, int32_t d, float rms_eps, float logit_scale,
+                                    float* entropy, int32_t* argmax, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -81,6 +81,7 @@ def lib() -> ctypes.CDLL:
             "dg_profile_stop": [vp, vp, vp],
             "dg_launch_count": [vp, ctypes.POINTER(ctypes.c_int64)],
             "dg_expert_units": [vp, ctypes.POINTER(ctypes.c_int64)],
+            "dg_lmhead_entropy_noalloc": [vp, vp, i32, i32, i32, f32, f32, vp, vp, vp],
             "dg_op_gemm": [vp, vp, vp, vp, i32, i32, i32, vp],
             "dg_op_moe": [vp, i32, vp, vp, i32, vp],
         }
@@ -97,7 +98,8 @@ def exported_symbols():
                         "dg_sync_status", "dg_prefill", "dg_kv_destroy", "dg_kv_info",
                         "dg_kv_read", "dg_denoise_step", "dg_generate_block", "dg_eb_sample",
                         "dg_debug_forward", "dg_profile_start", "dg_profile_stop",
-                        "dg_launch_count", "dg_op_gemm", "dg_op_moe", "dg_expert_units")
+                        "dg_launch_count", "dg_op_gemm", "dg_op_moe", "dg_expert_units",
+                        "dg_lmhead_entropy_noalloc")
             if hasattr(lib(), n)]
 
 
@@ -293,3 +295,15 @@ def dg_expert_units(model: Model) -> int:
     out = ctypes.c_int64()
     _check(lib().dg_expert_units(model.handle, ctypes.byref(out)))
     return out.value
+
+
+def dg_lmhead_entropy_noalloc(hidden, lm_head, rms_eps: float, logit_scale: float, stream=None):
+    """Entropy [M] and argmax [M] of logit_scale * RMSNorm(hidden) lm_head^T, computed
+    without any device allocation by the library (static scratch)."""
+    M, d = hidden.shape
+    V = lm_head.shape[0]
+    ent = torch.empty(M, dtype=torch.float32, device="cuda")
+    am = torch.empty(M, dtype=torch.int32, device="cuda")
+    _check(lib().dg_lmhead_entropy_noalloc(_ptr(hidden), _ptr(lm_head), M, V, d, rms_eps,
+                                           logit_scale, _ptr(ent), _ptr(am), _stream(stream)))
+    return ent, am

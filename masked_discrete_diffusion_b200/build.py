@@ -8,7 +8,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 OUT = os.path.join(HERE, "libdg.so")
-SOURCES = ["dg_api.cu", "tc_host.cu"]
+SOURCES = ["dg_api.cu", "tc_host.cu", "noalloc.cu"]
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17", "-lineinfo",
          "-Xcompiler", "-fPIC", "-shared", "--expt-relaxed-constexpr"]
 
