@@ -82,6 +82,7 @@ static void ws_free(Workspace& ws) {
 }
 
 __global__ void rope_table_kernel(double base, int h, int max_pos, void* out, int as_double) {
+  pdl_enter();
   const int half = h / 2;
   const long n = (long)max_pos * half;
   for (long e = blockIdx.x * (long)blockDim.x + threadIdx.x; e < n;
@@ -160,7 +161,7 @@ template <class Path> static dg_status alloc_workspace(dg_model* m) {
   DG_TRY(ws_alloc(ws, &ws.amax, lm_rows));
   DG_TRY(ws_alloc(ws, &ws.ncommit, c.max_batch));
   DG_TRY_CUDA(cudaMemset(ws.err, 0, 4 * sizeof(int32_t)));
-  rope_table_kernel<<<256, 256>>>((double)c.rope_base, (int)h, ws.max_pos, ws.rope,
+  launch_pdl((rope_table_kernel), 256, 256, 0, cudaStream_t(0), 1, (double)c.rope_base, (int)h, ws.max_pos, ws.rope,
                                   sizeof(Acc) == 8 ? 1 : 0);
   DG_TRY(check_launch("rope table"));
   if constexpr (Path::kTensorCores) DG_TRY(tc_prepare(m));
@@ -176,7 +177,7 @@ static void gemm_simt(const TA* A, int lda, const TW* W, const TW* W2, int ldw, 
                       int K, GroupInfo g, int grid_y, Epi epi, cudaStream_t st,
                       long long* count) {
   dim3 grid(ceil_div(N, SG_BN), G ? grid_y : ceil_div(M, SG_BM));
-  gemm_simt_kernel<TA, TW, Acc, G, D, Epi><<<grid, 256, 0, st>>>(A, lda, W, W2, ldw, M, N, K, g, epi);
+  launch_pdl((gemm_simt_kernel<TA, TW, Acc, G, D, Epi>), grid, 256, 0, st, 1, A, lda, W, W2, ldw, M, N, K, g, epi);
   ++*count;
 }
 
@@ -197,7 +198,8 @@ template <class Path> struct Runner {
   TA* xn() { return (TA*)ws.xn; }
 
   void rmsnorm(int n) {
-    rmsnorm_kernel<TR, TA, Acc><<<n, 256, 0, st>>>(x(), xn(), n, c.d_model, c.rms_eps);
+    launch_pdl((rmsnorm_kernel<TR, TA, Acc>), n, 256, 0, st, 1, x(), xn(), n, c.d_model, c.rms_eps,
+               (Acc*)nullptr);
     ++m->launches;
   }
 
@@ -226,7 +228,7 @@ template <class Path> struct Runner {
       else
         dense(xn(), d, L.wqkv, qkv_n, d, n, EpiStore<Acc, Acc>{(Acc*)ws.qkv, qkv_n});
     }
-    rope_scatter_kernel<Acc, TA, TKV><<<n, 128, 0, st>>>(
+    launch_pdl((rope_scatter_kernel<Acc, TA, TKV>), n, 128, 0, st, 1, 
         (const Acc*)ws.qkv, (TA*)ws.q, (TKV*)ws.kc, (TKV*)ws.vc, n, n_seq, np, pos0, Hq, Hkv, h,
         (const Acc*)ws.rope, ws.max_pos);
     ++m->launches;
@@ -249,7 +251,7 @@ template <class Path> struct Runner {
         const TKV* kB = (const TKV*)ws.kc;
         const TKV* vB = (const TKV*)ws.vc;
 #define DG_ATTN(DPL)                                                                            \
-  attention_simt_kernel<TA, TKV, Acc, DPL><<<blocks, 128, 0, st>>>(                             \
+  launch_pdl((attention_simt_kernel<TA, TKV, Acc, DPL>), blocks, 128, 0, st, 1,                              \
       (const TA*)ws.q, (TA*)ws.o, kA, vA, nA, WpA, kposA, kB, vB, n_seq, np, pos0, B_, n_seq,  \
       pos0, Hq, Hkv, h, causal ? 1 : 0, c.window)
         if (h <= 32) DG_ATTN(1);
@@ -277,39 +279,39 @@ template <class Path> struct Runner {
     const int Is = c.shared_inter;
     const int n_ent = n * k;
     // u = RMSNorm(x) after attention (bf16 copy for the expert GEMMs, 1/rms for the router)
-    rmsnorm_kernel<TR, TA, Acc><<<n, 256, 0, st>>>(x(), xn(), n, d, c.rms_eps, (Acc*)ws.inv_rms);
+    launch_pdl((rmsnorm_kernel<TR, TA, Acc>), n, 256, 0, st, 1, x(), xn(), n, d, c.rms_eps, (Acc*)ws.inv_rms);
     ++m->launches;
     {
       const int splits = std::max(1, std::min(16, 4096 / n));
       const int kps = ceil_div(ceil_div(d, splits), 32) * 32;
       const int ks = ceil_div(d, kps);
       dim3 grid(ceil_div(n, 32), ks, ceil_div(E, 128));
-      router_logits_kernel<TR, TW, Acc><<<grid, 256, 0, st>>>(x(), (const TW*)L.router, n, d, E,
+      launch_pdl((router_logits_kernel<TR, TW, Acc>), grid, 256, 0, st, 1, x(), (const TW*)L.router, n, d, E,
                                                               kps, (Acc*)ws.rlog);
       ++m->launches;
       if (E <= 32)
-        router_topk_kernel<Acc, 1><<<ceil_div(n, 4), 128, 0, st>>>(
+        launch_pdl((router_topk_kernel<Acc, 1>), ceil_div(n, 4), 128, 0, st, 1, 
             (const Acc*)ws.rlog, ks, (const Acc*)ws.inv_rms, n, E, k, ws.ridx, (Acc*)ws.rgate, load);
       else if (E <= 128)
-        router_topk_kernel<Acc, 4><<<ceil_div(n, 4), 128, 0, st>>>(
+        launch_pdl((router_topk_kernel<Acc, 4>), ceil_div(n, 4), 128, 0, st, 1, 
             (const Acc*)ws.rlog, ks, (const Acc*)ws.inv_rms, n, E, k, ws.ridx, (Acc*)ws.rgate, load);
       else
-        router_topk_kernel<Acc, 32><<<ceil_div(n, 4), 128, 0, st>>>(
+        launch_pdl((router_topk_kernel<Acc, 32>), ceil_div(n, 4), 128, 0, st, 1, 
             (const Acc*)ws.rlog, ks, (const Acc*)ws.inv_rms, n, E, k, ws.ridx, (Acc*)ws.rgate, load);
       ++m->launches;
     }
-    moe_rank_kernel<<<E, 256, 0, st>>>(ws.ridx, n_ent, ws.rank, ws.counts);
+    launch_pdl((moe_rank_kernel), E, 256, 0, st, 1, ws.ridx, n_ent, ws.rank, ws.counts);
     ++m->launches;
     int bm = SG_BM;
     if constexpr (Path::kTensorCores) bm = tc_group_rows();
-    moe_offsets_kernel<<<1, 1024, 0, st>>>(ws.counts, E, bm, ws.offsets, ws.tile_e, ws.tile_m0,
+    launch_pdl((moe_offsets_kernel), 1, 1024, 0, st, 1, ws.counts, E, bm, ws.offsets, ws.tile_e, ws.tile_m0,
                                            ws.n_tiles, ws.max_tiles, ws.units);
     ++m->launches;
-    moe_scatter_kernel<Acc><<<ceil_div(n_ent, 256), 256, 0, st>>>(
+    launch_pdl((moe_scatter_kernel<Acc>), ceil_div(n_ent, 256), 256, 0, st, 1, 
         ws.ridx, (const Acc*)ws.rgate, ws.rank, ws.offsets, n_ent, k, ws.row_of, ws.tok_of,
         (Acc*)ws.gate_of);
     ++m->launches;
-    gather_rows_kernel<TA><<<n_ent, 256, 0, st>>>(xn(), ws.tok_of, ws.offsets + E, d,
+    launch_pdl((gather_rows_kernel<TA>), n_ent, 256, 0, st, 1, xn(), ws.tok_of, ws.offsets + E, d,
                                                   (TA*)ws.up);
     ++m->launches;
     const int grid_y = ceil_div(n_ent, bm) + E;
@@ -343,7 +345,7 @@ template <class Path> struct Runner {
                                           EpiSwiglu<TA, Acc>{(TA*)ws.sh, Is}, st, &m->launches);
       dense((const TA*)ws.sh, Is, L.sdown, d, Is, n, EpiStore<Acc, Acc>{(Acc*)ws.ys, d});
     }
-    moe_combine_kernel<TR, Acc, Acc><<<dim3(n, ceil_div(d, 128)), 128, 0, st>>>(x(), (const Acc*)ws.ys,
+    launch_pdl((moe_combine_kernel<TR, Acc, Acc>), dim3(n, ceil_div(d, 128)), 128, 0, st, 1, x(), (const Acc*)ws.ys,
                                                         (const Acc*)ws.yb, ws.row_of, n, d, k);
     ++m->launches;
     return check_launch("moe");
@@ -354,11 +356,11 @@ template <class Path> struct Runner {
     if constexpr (sizeof(TR) == sizeof(float)) {
       DG_TRY_CUDA(cudaMemcpyAsync(x(), x_in, n * d * sizeof(float), cudaMemcpyDeviceToDevice, st));
     } else {
-      widen_f32_kernel<TR><<<ceil_div((long)n * d, 256), 256, 0, st>>>(x_in, x(), (long)n * d);
+      launch_pdl((widen_f32_kernel<TR>), ceil_div((long)n * d, 256), 256, 0, st, 1, x_in, x(), (long)n * d);
       ++m->launches;
     }
     DG_TRY(moe(l, n, nullptr));
-    to_f32_kernel<TR><<<ceil_div((long)n * d, 256), 256, 0, st>>>(x(), out, (long)n * d);
+    launch_pdl((to_f32_kernel<TR>), ceil_div((long)n * d, 256), 256, 0, st, 1, x(), out, (long)n * d);
     ++m->launches;
     return check_launch("moe op");
   }
@@ -370,7 +372,7 @@ template <class Path> struct Runner {
     const int Pp = (P + 63) / 64 * 64;
     const size_t es = sizeof(TKV);
     for (int b = 0; b < B; ++b) {
-      embed_kernel<TW, TR><<<P, 256, 0, st>>>(prompt + (size_t)b * P, (const TW*)m->w.tok_emb,
+      launch_pdl((embed_kernel<TW, TR>), P, 256, 0, st, 1, prompt + (size_t)b * P, (const TW*)m->w.tok_emb,
                                              x(), P, d, c.vocab - 1, -1.0, ws.err);
       ++m->launches;
       // padding columns of the transposed values must read as zero
@@ -399,7 +401,7 @@ template <class Path> struct Runner {
                     int32_t* amax, float* logits, float* hidden, int32_t* load) {
     const int B = kv->B, C = c.canvas, n = B * C, d = c.d_model;
     const double tau = (double)s / (double)T;
-    embed_kernel<TW, TR><<<n, 256, 0, st>>>(canvas, (const TW*)m->w.tok_emb, x(), n, d, c.vocab,
+    launch_pdl((embed_kernel<TW, TR>), n, 256, 0, st, 1, canvas, (const TW*)m->w.tok_emb, x(), n, d, c.vocab,
                                            tau, ws.err);
     ++m->launches;
     const int Cp = (C + 63) / 64 * 64;
@@ -407,7 +409,7 @@ template <class Path> struct Runner {
       DG_TRY_CUDA(cudaMemsetAsync(ws.vc, 0, (size_t)B * c.n_kv_heads * c.head_dim * Cp * sizeof(TKV), st));
     for (int l = 0; l < c.n_layers; ++l)
       DG_TRY(layer(l, n, B, C, kv->P, kv, false, load ? load + (size_t)l * c.n_experts : nullptr));
-    if (hidden) to_f32_kernel<TR><<<ceil_div((long)n * d, 256), 256, 0, st>>>(x(), hidden, (long)n * d);
+    if (hidden) launch_pdl((to_f32_kernel<TR>), ceil_div((long)n * d, 256), 256, 0, st, 1, x(), hidden, (long)n * d);
     ++m->launches;
     rmsnorm(n);
     ProfScope ps(m, DG_KIND_LMHEAD, st);
@@ -420,11 +422,11 @@ template <class Path> struct Runner {
     }
     if (!done) {
       dim3 grid(ws.n_vtiles, ceil_div(n, SG_BM));
-      lmhead_simt_kernel<TA, TW, Acc><<<grid, 256, 0, st>>>(xn(), (const TW*)m->w.lm_head, n,
+      launch_pdl((lmhead_simt_kernel<TA, TW, Acc>), grid, 256, 0, st, 1, xn(), (const TW*)m->w.lm_head, n,
                                                            c.vocab, d, c.logit_scale,
                                                            (Acc*)ws.lm_part, logits);
       ++m->launches;
-      lm_merge_kernel<Acc><<<ceil_div(n, 4), 128, 0, st>>>((const Acc*)ws.lm_part, ws.n_vtiles,
+      launch_pdl((lm_merge_kernel<Acc>), ceil_div(n, 4), 128, 0, st, 1, (const Acc*)ws.lm_part, ws.n_vtiles,
                                                           n, ent, amax);
       ++m->launches;
     }
@@ -457,7 +459,7 @@ static dg_status launch_sampler(const float* H, const int32_t* am, int32_t* canv
                                 int32_t* ncommit, int32_t* nfwd, int step_no,
                                 cudaStream_t st, long long* counter_) {
 #define DG_SAMP(NP)                                                                       \
-  eb_sample_kernel<NP><<<B, NP, 0, st>>>(H, am, canvas, mask, C, s, gq, ncommit, nfwd, \
+  launch_pdl((eb_sample_kernel<NP>), B, NP, 0, st, 1, H, am, canvas, mask, C, s, gq, ncommit, nfwd, \
                                          step_no)
   if (C <= 32) DG_SAMP(32);
   else if (C <= 64) DG_SAMP(64);
@@ -669,11 +671,11 @@ dg_status dg_kv_read(const dg_kv* kv, void* k, void* v, void* stream) {
   const size_t blocks = (size_t)c.n_layers * kv->B * c.n_kv_heads;
   const size_t total = blocks * kv->W * c.head_dim;
   if (kv->elem == sizeof(double))
-    kv_unpack_kernel<double><<<ceil_div(total, 256), 256, 0, st>>>(
+    launch_pdl((kv_unpack_kernel<double>), ceil_div(total, 256), 256, 0, st, 1, 
         (const double*)kv->k, (const double*)kv->v, (double*)k, (double*)v, blocks, kv->W, kv->Wp,
         c.head_dim);
   else
-    kv_unpack_kernel<bf16><<<ceil_div(total, 256), 256, 0, st>>>(
+    launch_pdl((kv_unpack_kernel<bf16>), ceil_div(total, 256), 256, 0, st, 1, 
         (const bf16*)kv->k, (const bf16*)kv->v, (bf16*)k, (bf16*)v, blocks, kv->W, kv->Wp,
         c.head_dim);
   return check_launch("kv read");
@@ -715,7 +717,7 @@ static dg_status generate_impl(dg_model* m, const dg_kv* kv, int32_t T, long lon
   const dg_config& c = m->cfg;
   const int B = kv->B, C = c.canvas;
   Workspace& ws = m->ws;
-  fill_i32_kernel<<<ceil_div((long)B * C, 256), 256, 0, st>>>(canvas_out, B * C, c.vocab);
+  launch_pdl((fill_i32_kernel), ceil_div((long)B * C, 256), 256, 0, st, 1, canvas_out, B * C, c.vocab);
   ++m->launches;
   DG_TRY_CUDA(cudaMemsetAsync(ws.mask, 1, (size_t)B * C, st));
   if (n_forwards) DG_TRY_CUDA(cudaMemsetAsync(n_forwards, 0, B * sizeof(int32_t), st));

@@ -6,6 +6,7 @@
 
 #include <cstdint>
 #include <string>
+#include <utility>
 #include <vector>
 
 #include "../../include/dg.h"
@@ -13,6 +14,36 @@
 namespace dg {
 
 void set_error(const char* fmt, ...);
+
+// Launches `kern` with programmatic dependent launch allowed: the kernel may be
+// scheduled while its predecessor on the stream is still running; every kernel
+// of the library calls griddepcontrol.wait before touching global memory the
+// predecessor writes or reads, so only launch latency and prologues overlap.
+// cluster_z > 1 additionally groups CTAs into clusters of that size along z.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, int cluster_z, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[2];
+  int n = 0;
+  at[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster_z > 1) {
+    at[n].id = cudaLaunchAttributeClusterDimension;
+    at[n].val.clusterDim.x = 1;
+    at[n].val.clusterDim.y = 1;
+    at[n].val.clusterDim.z = cluster_z;
+    ++n;
+  }
+  cfg.attrs = at;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 #define DG_TRY_CUDA(call)                                                            \
   do {                                                                               \

@@ -10,6 +10,17 @@ namespace dg {
 
 typedef __nv_bfloat16 bf16;
 
+// Programmatic dependent launch: wait until the preceding kernel on the stream has
+// completed and its writes are visible, then let the next kernel be scheduled.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_enter() {
+  pdl_wait();
+  pdl_trigger();
+}
+
 __device__ __forceinline__ float widen(float x) { return x; }
 __device__ __forceinline__ float widen(bf16 x) { return __bfloat162float(x); }
 __device__ __forceinline__ double widen(double x) { return x; }

@@ -36,6 +36,7 @@ __global__ void __launch_bounds__(NP)
                      int32_t* __restrict__ canvas, uint8_t* __restrict__ mask, int C,
                      int steps_left, long long gamma_q, int32_t* __restrict__ n_commit,
                      int32_t* __restrict__ n_fwd, int step_no) {
+  pdl_enter();
   __shared__ unsigned long long key[NP];
   __shared__ long long pre[NP];
   __shared__ int cnt[NP / 32];

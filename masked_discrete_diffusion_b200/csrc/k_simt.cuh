@@ -23,6 +23,7 @@ template <class TW, class TR>
 __global__ void embed_kernel(const int32_t* __restrict__ ids, const TW* __restrict__ emb,
                              TR* __restrict__ x, int n_tok, int d, int max_id, double tau,
                              int32_t* err) {
+  pdl_enter();
   const int t = blockIdx.x;
   if (t >= n_tok) return;
   int id = ids[t];
@@ -50,6 +51,7 @@ __global__ void embed_kernel(const int32_t* __restrict__ ids, const TW* __restri
 template <class TR, class TA, class Acc>
 __global__ void rmsnorm_kernel(const TR* __restrict__ x, TA* __restrict__ y, int n, int d,
                                float eps, Acc* __restrict__ inv_out = nullptr) {
+  pdl_enter();
   __shared__ Acc red[32];
   const int t = blockIdx.x;
   if (t >= n) return;
@@ -87,6 +89,7 @@ __global__ void __launch_bounds__(256)
     gemm_simt_kernel(const TA* __restrict__ A, int lda, const TW* __restrict__ W,
                      const TW* __restrict__ W2, int ldw, int M, int N, int K, GroupInfo g,
                      Epi epi) {
+  pdl_enter();
   __shared__ Acc As[SG_BK][SG_BM + 1];
   __shared__ Acc Ws[SG_BK][SG_BN + 1];
   __shared__ Acc Ws2[DUAL ? SG_BK : 1][DUAL ? SG_BN + 1 : 1];
@@ -204,6 +207,7 @@ __global__ void rope_scatter_kernel(const Acc* __restrict__ qkv, TA* __restrict_
                                     TKV* __restrict__ kc, TKV* __restrict__ vc, int n_tok,
                                     int n_seq, int np, int pos0, int Hq, int Hkv, int h,
                                     const Acc* __restrict__ rope, int max_pos) {
+  pdl_enter();
   const int t = blockIdx.x;
   if (t >= n_tok) return;
   const int b = t / n_seq, i = t % n_seq, pos = pos0 + i;
@@ -250,6 +254,7 @@ __global__ void attention_simt_kernel(const TA* __restrict__ q, TA* __restrict__
                                       const TKV* __restrict__ vB, int nB, int padB, int kposB, int B,
                                       int nq, int qpos0, int Hq, int Hkv, int h, int causal,
                                       int window) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   const long wid = (long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const long total = (long)B * nq * Hq;
@@ -324,6 +329,7 @@ template <class TR, class TW, class Acc>
 __global__ void __launch_bounds__(256)
     router_logits_kernel(const TR* __restrict__ x, const TW* __restrict__ wr, int n, int d, int E,
                          int k_per_split, Acc* __restrict__ part) {
+  pdl_enter();
   __shared__ Acc Xs[32][33];
   __shared__ Acc Ws[32][129];
   const int tid = threadIdx.x, tx = tid & 31, ty = tid >> 5;
@@ -376,6 +382,7 @@ __global__ void router_topk_kernel(const Acc* __restrict__ part, int splits,
                                    const Acc* __restrict__ inv_rms, int n, int E, int top_k,
                                    int32_t* __restrict__ idx, Acc* __restrict__ gate,
                                    int32_t* __restrict__ load) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= n) return;
@@ -450,6 +457,7 @@ __global__ void router_topk_kernel(const Acc* __restrict__ part, int splits,
 // ---------------------------------------------------------------------------
 static __global__ void moe_rank_kernel(const int32_t* __restrict__ idx, int n_entries,
                                 int32_t* __restrict__ rank, int32_t* __restrict__ counts) {
+  pdl_enter();
   __shared__ int warp_tot[32];
   __shared__ int carry;
   const int e = blockIdx.x;
@@ -484,6 +492,7 @@ static __global__ void __launch_bounds__(1024)
                        int32_t* __restrict__ offsets, int32_t* __restrict__ tile_e,
                        int32_t* __restrict__ tile_m0, int32_t* __restrict__ n_tiles,
                        int max_tiles, unsigned long long* __restrict__ used) {
+  pdl_enter();
   __shared__ int sc[1024], st[1024];
   const int e = threadIdx.x;
   const int c = e < E ? counts[e] : 0;
@@ -521,6 +530,7 @@ __global__ void moe_scatter_kernel(const int32_t* __restrict__ idx, const Acc* _
                                    const int32_t* __restrict__ offsets, int n_entries, int top_k,
                                    int32_t* __restrict__ row_of, int32_t* __restrict__ tok_of,
                                    Acc* __restrict__ gate_of) {
+  pdl_enter();
   const int j = blockIdx.x * blockDim.x + threadIdx.x;
   if (j >= n_entries) return;
   const int pos = offsets[idx[j]] + rank[j];
@@ -533,6 +543,7 @@ template <class TA>
 __global__ void gather_rows_kernel(const TA* __restrict__ src, const int32_t* __restrict__ tok_of,
                                    const int32_t* __restrict__ n_rows_dev, int d,
                                    TA* __restrict__ dst) {
+  pdl_enter();
   const int r = blockIdx.x;
   if (r >= *n_rows_dev) return;
   const TA* s = src + (size_t)tok_of[r] * d;
@@ -546,6 +557,7 @@ template <class TR, class TY, class Acc>
 __global__ void moe_combine_kernel(TR* __restrict__ x, const TY* __restrict__ ys,
                                    const TY* __restrict__ yb, const int32_t* __restrict__ row_of,
                                    int n_tok, int d, int top_k) {
+  pdl_enter();
   const int t = blockIdx.x;
   if (t >= n_tok) return;
   {
@@ -570,6 +582,7 @@ template <class TA, class TW, class Acc>
 __global__ void __launch_bounds__(256)
     lmhead_simt_kernel(const TA* __restrict__ xn, const TW* __restrict__ wlm, int n_rows, int V,
                        int d, float scale, Acc* __restrict__ part, float* __restrict__ logits) {
+  pdl_enter();
   // the logits tile T reuses the operand staging buffers once the K loop is done
   constexpr int kStage = 2 * SG_BK * (SG_BM + 1), kTile = SG_BM * (SG_BN + 1);
   __shared__ Acc smem[kStage > kTile ? kStage : kTile];
@@ -665,6 +678,7 @@ __global__ void __launch_bounds__(256)
 template <class Acc>
 __global__ void lm_merge_kernel(const Acc* __restrict__ part, int n_vt, int n_rows,
                                 float* __restrict__ H, int32_t* __restrict__ amax) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (r >= n_rows) return;
@@ -707,6 +721,7 @@ template <class T>
 __global__ void kv_unpack_kernel(const T* __restrict__ k, const T* __restrict__ vt,
                                  T* __restrict__ ko, T* __restrict__ vo, size_t blocks, int W,
                                  int Wp, int h) {
+  pdl_enter();
   const size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
   if (i >= blocks * W * h) return;
   const size_t bl = i / ((size_t)W * h);
@@ -717,17 +732,20 @@ __global__ void kv_unpack_kernel(const T* __restrict__ k, const T* __restrict__ 
 
 template <class T>
 __global__ void widen_f32_kernel(const float* __restrict__ src, T* __restrict__ dst, long n) {
+  pdl_enter();
   const long i = blockIdx.x * (long)blockDim.x + threadIdx.x;
   if (i < n) dst[i] = (T)src[i];
 }
 
 template <class T>
 __global__ void to_f32_kernel(const T* __restrict__ src, float* __restrict__ dst, long n) {
+  pdl_enter();
   const long i = blockIdx.x * (long)blockDim.x + threadIdx.x;
   if (i < n) dst[i] = (float)widen(src[i]);
 }
 
 static __global__ void fill_i32_kernel(int32_t* __restrict__ p, int n, int32_t v) {
+  pdl_enter();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) p[i] = v;
 }

@@ -94,6 +94,7 @@ __global__ void __launch_bounds__(128, 1)
   const uint32_t tmem = *tslot;
   const uint32_t tS = tmem, tO = tmem + 128;
   const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+  pdl_enter();  // global memory is touched only from here on
 
   auto load_tile = [&](int i) {  // tile index i within this split -> stage i & 1
     const int t = my_lo + i;
@@ -280,6 +281,7 @@ __global__ void __launch_bounds__(128, 1)
 __global__ void attn_combine_kernel(const float* __restrict__ part_o,
                                     const float* __restrict__ part_ml, int splits, int ntok,
                                     int Hq, bf16* __restrict__ out) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   const long w = (long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (w >= (long)ntok * Hq) return;

@@ -208,7 +208,8 @@ __global__ void __launch_bounds__(128, 1)
                     int32_t* err) {
   typedef DenseCfg<BN, MT, DUAL, ST> Cfg;
   // split-K needs the whole fp32 tile in the (drained) pipeline buffers and a chunk epilogue
-  constexpr bool kSplitOK = MT * 128 * Cfg::NACC * BN * 4 <= ST * Cfg::STAGE && Epi::kChunked;
+  constexpr int RS = Cfg::NACC * BN + 4;  // reduction row stride (floats): padded against bank conflicts
+  constexpr bool kSplitOK = MT * 128 * RS * 4 <= ST * Cfg::STAGE && Epi::kChunked;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + ST * Cfg::STAGE);
@@ -238,6 +239,7 @@ __global__ void __launch_bounds__(128, 1)
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tslot;
+  pdl_enter();  // global memory is touched only from here on
 
   if (warp == 0 && lane == 0) {
     tc::prefetch_tmap(&mA);
@@ -315,7 +317,6 @@ __global__ void __launch_bounds__(128, 1)
     }
   } else if constexpr (kSplitOK) {
     // every thread of every CTA passes both cluster barriers, whatever happened above
-    constexpr int W = Cfg::NACC * BN;        // fp32 values per tile row
     const int R = MT * 128 / ksplit;         // rows owned per CTA
     cl::sync();                              // all pipelines drained: smem reusable
     if (ready) {
@@ -325,7 +326,7 @@ __global__ void __launch_bounds__(128, 1)
       for (int mt = 0; mt < MT; ++mt) {
         const int trow = mt * 128 + 32 * warp + lane;  // row within the tile
         const int owner = trow / R, lr = trow % R;
-        const uint32_t dst = cl::map(recv, owner) + (uint32_t)(((rank * R + lr) * W) * 4);
+        const uint32_t dst = cl::map(recv, owner) + (uint32_t)(((rank * R + lr) * RS) * 4);
 #pragma unroll 1
         for (int a = 0; a < Cfg::NACC; ++a)
 #pragma unroll 1
@@ -350,7 +351,7 @@ __global__ void __launch_bounds__(128, 1)
         u[j] = 0.f;
       }
       for (int src = 0; src < ksplit; ++src) {
-        const float* p = buf + (size_t)(src * R + lr) * W + c * 32;
+        const float* p = buf + (size_t)(src * R + lr) * RS + c * 32;
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] += p[j];
         if (DUAL) {
@@ -396,6 +397,7 @@ __global__ void __launch_bounds__(192, 1)
                      void* __restrict__ out, int ldo, const float* __restrict__ gate_of,
                      int32_t* err) {
   typedef ExpertCfg<GATEUP, ST> Cfg;
+  pdl_enter();  // the routing tables come from the preceding kernels
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + ST * Cfg::STAGE);

@@ -101,6 +101,7 @@ dg_status encode(const void* p, uint64_t rows, uint64_t cols, uint32_t box_rows,
 // A wait inside the GEMM that gave up leaves statistics unwritten: mark every row
 // (entropy NaN, argmax -1) so the caller sees the failure in the outputs.
 __global__ void noalloc_flag_kernel(const int32_t* err, int M, float* entropy, int32_t* argmax) {
+  pdl_enter();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < M && *err) {
     entropy[i] = __int_as_float(0x7fc00000);
@@ -134,7 +135,7 @@ extern "C" dg_status dg_lmhead_entropy_noalloc(const float* hidden, const void* 
   cudaStream_t st = (cudaStream_t)stream;
   DG_TRY_CUDA(cudaMemsetAsync(err, 0, sizeof(int32_t), st));
 
-  rmsnorm_kernel<float, bf16, float><<<M, 256, 0, st>>>(hidden, xn, M, d, rms_eps);
+  rmsnorm_kernel<float, bf16, float><<<M, 256, 0, st>>>(hidden, xn, M, d, rms_eps, nullptr);
   CUtensorMap ma, mb;
   DG_TRY(encode(xn, (uint64_t)M, (uint64_t)d, 128, &ma));
   DG_TRY(encode(lm_head, (uint64_t)V, (uint64_t)d, NA_BN, &mb));

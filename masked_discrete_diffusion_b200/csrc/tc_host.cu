@@ -109,23 +109,10 @@ dg_status launch_dense(dg_model* m, const CUtensorMap& a, const CUtensorMap& b,
     while (ks < 8 && tiles * ks * 2 <= state(m)->n_sm && nk >= ks * 2 * 2) ks *= 2;
   cudaError_t e;
   if (ks == 1) {
-    kern<<<grid, 128, Cfg::SMEM, st>>>(a, b, b2, M, K, 1, epi, m->ws.err);
-    e = cudaGetLastError();
+    e = launch_pdl(kern, grid, 128, Cfg::SMEM, st, 1, a, b, b2, M, K, 1, epi, m->ws.err);
   } else {
     grid.z = ks;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = dim3(128, 1, 1);
-    cfg.dynamicSmemBytes = Cfg::SMEM;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 1;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = ks;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, kern, a, b, b2, M, K, ks, epi, m->ws.err);
+    e = launch_pdl(kern, grid, 128, Cfg::SMEM, st, ks, a, b, b2, M, K, ks, epi, m->ws.err);
   }
   ++m->launches;
   if (e != cudaSuccess) {
@@ -236,7 +223,7 @@ dg_status tc_lmhead_stats(dg_model* m, const bf16* xn, int M, float* ent, int32_
                                                EpiLmStats{part, M, c.vocab, c.logit_scale}, st,
                                                false)));
   const int n_vt = ceil_div_i(c.vocab, LM_BN);
-  lm_merge_kernel<float><<<ceil_div_i(M, 4), 128, 0, st>>>(part, n_vt, M, ent, amax);
+  launch_pdl((lm_merge_kernel<float>), ceil_div_i(M, 4), 128, 0, st, 1, part, n_vt, M, ent, amax);
   ++m->launches;
   return DG_OK;
 }
@@ -249,7 +236,7 @@ static dg_status launch_expert(dg_model* m, const CUtensorMap& w, const CUtensor
   auto kern = tc_expert_kernel<GATEUP, ST>;
   const int n_sm = state(m)->n_sm;
   const Workspace& ws = m->ws;
-  kern<<<n_sm, 192, Cfg::SMEM, st>>>(w, w2, x, ws.tile_e, ws.tile_m0, ws.n_tiles, ws.offsets,
+  launch_pdl((kern), n_sm, 192, Cfg::SMEM, st, 1, w, w2, x, ws.tile_e, ws.tile_m0, ws.n_tiles, ws.offsets,
                                      w_rows, K, FT, out, ldo, gate_of, ws.err);
   ++m->launches;
   cudaError_t e = cudaGetLastError();
@@ -332,10 +319,10 @@ dg_status tc_attention(dg_model* m, const bf16* q, int B, int nq, int qpos0, con
   splits = ceil_div_i(total, tps);
   p.tiles_per_split = tps;
   dim3 grid(qtiles * Hq, B, splits);
-  tc_attn_kernel<<<grid, 128, AT_SMEM, st>>>(mQ, mKA, mVA, mKB, mVB, p, m->ws.err);
+  launch_pdl((tc_attn_kernel), grid, 128, AT_SMEM, st, 1, mQ, mKA, mVA, mKB, mVB, p, m->ws.err);
   ++m->launches;
   const int ntok = B * nq;
-  attn_combine_kernel<<<ceil_div_i((long)ntok * Hq, 4), 128, 0, st>>>(
+  launch_pdl((attn_combine_kernel), ceil_div_i((long)ntok * Hq, 4), 128, 0, st, 1, 
       p.part_o, p.part_ml, splits, ntok, Hq, out);
   ++m->launches;
   cudaError_t e = cudaGetLastError();
