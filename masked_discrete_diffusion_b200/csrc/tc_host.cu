@@ -313,7 +313,8 @@ dg_status tc_attention(dg_model* m, const bf16* q, int B, int nq, int qpos0, con
   const int qtiles = ceil_div_i(nq, 128);
   const int base = qtiles * Hq * B;
   const int n_sm = state(m)->n_sm;
-  int splits = std::min(ceil_div_i(2 * n_sm, base), std::min((int)ATT_MAX_SPLITS, total));
+  // one wave: CTAs (one per SM, ~194 KB of shared memory each) never exceed the SM count
+  int splits = std::min(std::max(1, n_sm / base), std::min((int)ATT_MAX_SPLITS, total));
   splits = std::max(1, splits);
   const int tps = ceil_div_i(total, splits);
   splits = ceil_div_i(total, tps);
