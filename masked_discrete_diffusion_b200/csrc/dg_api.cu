@@ -526,16 +526,17 @@ dg_status dg_model_create(const dg_config* cfg, const dg_weights* w, dg_model** 
              "bad eps/logit_scale/rope_base");
   DG_REQUIRE(c.dtype == DG_F32 || c.dtype == DG_BF16 || c.dtype == DG_BF16_FP8EXP,
              "unknown dtype %d", c.dtype);
-  if (c.dtype == DG_BF16_FP8EXP) {
-    set_error("FP8 expert weights are not implemented in this build");
-    return DG_ERR_UNSUPPORTED;
-  }
+  if (c.dtype == DG_BF16_FP8EXP)
+    DG_REQUIRE(c.d_model % 128 == 0 && c.expert_inter % 128 == 0,
+               "FP8 experts need d and I multiples of 128 (one scale per 128 columns)");
   DG_REQUIRE(w->tok_emb && w->lm_head && w->layers, "null weight pointer");
   for (int l = 0; l < c.n_layers; ++l) {
     const dg_layer_weights& L = w->layers[l];
     DG_REQUIRE(L.wqkv && L.wo && L.router && L.gate && L.up && L.down && L.sgate && L.sup &&
                    L.sdown,
                "null weight pointer in layer %d", l);
+    if (c.dtype == DG_BF16_FP8EXP)
+      DG_REQUIRE(L.gate_scale && L.up_scale && L.down_scale, "null FP8 scale pointer in layer %d", l);
   }
   dg_model* m = new dg_model();
   m->cfg = c;

@@ -7,6 +7,7 @@
 #include "dg_internal.h"
 #include "k_simt.cuh"
 #include "k_tc_attn.cuh"
+#include "k_tc_expert_fp8.cuh"
 #include "k_tc_gemm.cuh"
 
 namespace dg {
@@ -17,8 +18,10 @@ struct MapKey {
   const void* p;
   uint64_t rows, cols;
   uint32_t box_rows;
+  bool bytes = false;  // uint8 elements, 64-byte boxes, no swizzle (FP8 weights)
   bool operator==(const MapKey& o) const {
-    return p == o.p && rows == o.rows && cols == o.cols && box_rows == o.box_rows;
+    return p == o.p && rows == o.rows && cols == o.cols && box_rows == o.box_rows &&
+           bytes == o.bytes;
   }
 };
 struct MapKeyHash {
@@ -49,32 +52,34 @@ int ceil_div_i(long a, long b) { return (int)((a + b - 1) / b); }
 // 2-D bf16 tensor [rows, cols] (row-major), box = 64 columns x box_rows rows,
 // 128-byte swizzle, out-of-range elements read as zero.
 dg_status tmap(const dg_model* m, const void* p, uint64_t rows, uint64_t cols, uint32_t box_rows,
-               CUtensorMap* out) {
+               CUtensorMap* out, bool bytes = false) {
   TcState* s = state(m);
   if (!s) {
     set_error("tensor-core state missing");
     return DG_ERR_INTERNAL;
   }
-  MapKey key{p, rows, cols, box_rows};
+  MapKey key{p, rows, cols, box_rows, bytes};
   auto it = s->maps.find(key);
   if (it != s->maps.end()) {
     *out = it->second;
     return DG_OK;
   }
-  if ((reinterpret_cast<uintptr_t>(p) & 15) || (cols * 2) % 16 || box_rows > 256) {
+  const uint64_t esz = bytes ? 1 : 2;
+  if ((reinterpret_cast<uintptr_t>(p) & 15) || (cols * esz) % 16 || box_rows > 256) {
     set_error("tensor map: base %p / row pitch %llu bytes not 16-byte aligned", p,
-              (unsigned long long)(cols * 2));
+              (unsigned long long)(cols * esz));
     return DG_ERR_UNSUPPORTED;
   }
   CUtensorMap map;
   cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {cols * 2};
+  cuuint64_t strides[1] = {cols * esz};
   cuuint32_t box[2] = {64, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = s->encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(p), dims,
-                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = s->encode(&map, bytes ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                         2, const_cast<void*>(p), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         bytes ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     set_error("cuTensorMapEncodeTiled failed (%d) for %p [%llu x %llu] box %u", (int)r, p,
               (unsigned long long)rows, (unsigned long long)cols, box_rows);
@@ -125,6 +130,7 @@ dg_status launch_dense(dg_model* m, const CUtensorMap& a, const CUtensorMap& b,
 constexpr int DENSE_BN = 64, DENSE_MT = 2, DENSE_ST = 5, DUAL_ST = 4;
 constexpr int LM_BN = 256, LM_ST = 3;
 constexpr int GU_ST = 4, DN_ST = 6;
+constexpr int GU8_ST = 3, DN8_ST = 5;
 
 }  // namespace
 
@@ -162,6 +168,8 @@ dg_status tc_prepare(dg_model* m) {
   DG_TRY(set_smem(tc_expert_kernel<true, GU_ST>, ExpertCfg<true, GU_ST>::SMEM));
   DG_TRY(set_smem(tc_expert_kernel<false, DN_ST>, ExpertCfg<false, DN_ST>::SMEM));
   DG_TRY(set_smem(tc_attn_kernel, AT_SMEM));
+  DG_TRY(set_smem(tc_expert_f8_kernel<true, GU8_ST>, ExpertF8Cfg<true, GU8_ST>::SMEM));
+  DG_TRY(set_smem(tc_expert_f8_kernel<false, DN8_ST>, ExpertF8Cfg<false, DN8_ST>::SMEM));
   cudaDeviceGetAttribute(&s->n_sm, cudaDevAttrMultiProcessorCount, m->device);
   return DG_OK;
 }
@@ -247,10 +255,36 @@ static dg_status launch_expert(dg_model* m, const CUtensorMap& w, const CUtensor
   return DG_OK;
 }
 
+template <bool GATEUP, int ST>
+static dg_status launch_expert_f8(dg_model* m, const CUtensorMap& w, const CUtensorMap& w2,
+                                  const CUtensorMap& x, const float* s1, const float* s2,
+                                  int w_rows, int K, int FT, void* out, int ldo,
+                                  const float* gate_of, cudaStream_t st) {
+  typedef ExpertF8Cfg<GATEUP, ST> Cfg;
+  const Workspace& ws = m->ws;
+  cudaError_t e = launch_pdl((tc_expert_f8_kernel<GATEUP, ST>), state(m)->n_sm, 320, Cfg::SMEM, st, 1,
+                             w, w2, x, s1, s2, ws.tile_e, ws.tile_m0, ws.n_tiles, ws.offsets,
+                             w_rows, K, FT, out, ldo, gate_of, ws.err);
+  ++m->launches;
+  if (e != cudaSuccess) {
+    set_error("tc_expert_f8 launch: %s", cudaGetErrorString(e));
+    return DG_ERR_CUDA;
+  }
+  return DG_OK;
+}
+
 dg_status tc_moe_gate_up(dg_model* m, int l, const bf16* X, bf16* hb, int, cudaStream_t st) {
   const dg_config& c = m->cfg;
   const dg_layer_weights& L = m->layers[l];
   const int E = c.n_experts, I = c.expert_inter, d = c.d_model;
+  if (c.dtype == DG_BF16_FP8EXP) {
+    CUtensorMap wg, wu, x;
+    DG_TRY(tmap(m, L.gate, (uint64_t)E * I, d, 128, &wg, true));
+    DG_TRY(tmap(m, L.up, (uint64_t)E * I, d, 128, &wu, true));
+    DG_TRY(tmap(m, X, m->ws.max_rows, d, 32, &x));
+    return launch_expert_f8<true, GU8_ST>(m, wg, wu, x, L.gate_scale, L.up_scale, I, d, I / 128,
+                                          hb, I, nullptr, st);
+  }
   CUtensorMap wg, wu, x;
   DG_TRY(tmap(m, L.gate, (uint64_t)E * I, d, 128, &wg));
   DG_TRY(tmap(m, L.up, (uint64_t)E * I, d, 128, &wu));
@@ -262,6 +296,13 @@ dg_status tc_moe_down(dg_model* m, int l, const bf16* H, float* yb, int, cudaStr
   const dg_config& c = m->cfg;
   const dg_layer_weights& L = m->layers[l];
   const int E = c.n_experts, I = c.expert_inter, d = c.d_model;
+  if (c.dtype == DG_BF16_FP8EXP) {
+    CUtensorMap wd, x;
+    DG_TRY(tmap(m, L.down, (uint64_t)E * d, I, 128, &wd, true));
+    DG_TRY(tmap(m, H, m->ws.max_rows, I, 32, &x));
+    return launch_expert_f8<false, DN8_ST>(m, wd, wd, x, L.down_scale, L.down_scale, d, I,
+                                           d / 128, yb, d, (const float*)m->ws.gate_of, st);
+  }
   CUtensorMap wd, x;
   DG_TRY(tmap(m, L.down, (uint64_t)E * d, I, 128, &wd));
   DG_TRY(tmap(m, H, m->ws.max_rows, I, 32, &x));

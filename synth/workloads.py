@@ -92,8 +92,13 @@ SMALL_BF16 = Workload(
     canvas=96, rope_base=10000.0, rms_eps=1e-6, logit_scale=8.0, dtype="bf16",
     batch=3, prompt_len=160, T=6, gamma=1.0)
 
+# FP8-expert variants for parity tests: the small model, and one full-size layer with
+# the FP8 workload's 4096-token prompt.
+SMALL_FP8 = SMALL_BF16.with_(name="small-fp8exp", dtype="bf16_fp8exp")
+LAYER1_FP8 = LAYER1_BF16.with_(name="layer1-fp8exp-p4096", dtype="bf16_fp8exp", prompt_len=4096)
+
 WORKLOADS = {w.name: w for w in (TINY_F32, SMALL_BF16, LAYER1_BF16, FULL30_BF16,
-                                 FULL30_B8_P8192)}
+                                 FULL30_B8_P8192, SMALL_FP8, LAYER1_FP8)}
 for _b in (1, 4, 16, 32, 64):
     WORKLOADS[f"full30-fp8exp-b{_b}"] = full30_fp8exp(_b)
 

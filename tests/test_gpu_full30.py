@@ -1,0 +1,98 @@
+"""30-layer Gemma-4-26B-A4B-shaped stand-in (bf16, batch 1, prompt 1024, canvas 256, T 12):
+the throughput workload, in the launch configuration the bench times.
+
+Oracle values come from tests/golden/full30-bf16.npz (written by
+tests/golden/make_golden.py from the oracle alone): the first forward of the block
+(all [MASK], steps_left = T).  Checked: prefill window K/V of layers 0 and 29,
+entropies (2e-2 max-abs relative), argmax where decided, sampled logits.  The
+graph-replayed block itself is checked by properties that hold at any size: its
+first forward equals the stand-alone forward, it equals the step-by-step API
+bit for bit, and it ends with no [MASK] after exactly T forwards.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from synth import model_inputs, workloads
+
+from gpu_helpers import make_model, max_abs_rel
+
+pytestmark = pytest.mark.gpu
+W = workloads.FULL30_BF16
+TOL = 2e-2
+GOLD = os.path.join(os.path.dirname(__file__), "golden", "full30-bf16.npz")
+
+
+@pytest.fixture(scope="module")
+def run():
+    if not os.path.exists(GOLD):
+        pytest.skip("golden file missing")
+    from masked_discrete_diffusion_b200 import binding
+    g = np.load(GOLD)
+    model = make_model(W)
+    kv = binding.dg_prefill(model, model_inputs.prompt(W, "cuda"))
+    canvas = torch.full((1, W.canvas), W.mask_id, dtype=torch.int32, device="cuda")
+    ent, am, lg, _ = binding.dg_debug_forward(model, kv, canvas, W.T, W.T, logits=True)
+    ent2, am2, _, _ = binding.dg_debug_forward(model, kv, canvas, W.T, W.T)
+    k, v = binding.dg_kv_read(kv)
+    binding.dg_sync_status(model)
+    rows = torch.as_tensor(g["logit_rows"]).cuda()
+    cols = torch.as_tensor(g["logit_cols"]).cuda()
+    out = dict(g=g, ent=ent[0].cpu().numpy(), am=am[0].cpu().numpy(),
+               ent2=ent2[0].cpu().numpy(), am2=am2[0].cpu().numpy(),
+               lg=lg[rows][:, cols].cpu().numpy(),
+               k=k[[0, W.n_layers - 1], 0, :, -8:].float().cpu().numpy(),
+               v=v[[0, W.n_layers - 1], 0, :, -8:].float().cpu().numpy(),
+               binding=binding, model=model, kv=kv)
+    del lg, k, v
+    yield out
+    kv.close()
+    model.close()
+
+
+def test_prefill_window_kv(run):
+    kl = run["g"]["kv_last"]                # [2 layers, 2 (K, V), Hkv, 8, h]
+    for i in range(2):
+        assert max_abs_rel(run["k"][i], kl[i, 0]) < TOL
+        assert max_abs_rel(run["v"][i], kl[i, 1]) < TOL
+
+
+def test_logits_sampled(run):
+    assert max_abs_rel(run["lg"], run["g"]["logits"]) < TOL
+
+
+def test_entropies(run):
+    g = run["g"]
+    for ent in (run["ent"], run["ent2"]):
+        assert max_abs_rel(ent, g["H"]) < TOL
+        assert np.all(ent >= 0) and np.all(ent <= math.log(W.vocab) + 1e-3)
+
+
+def test_argmax_where_decided(run):
+    g = run["g"]
+    eps = float(np.abs(run["lg"] - g["logits"]).max())
+    decided = g["margin"] > 2 * eps + 1e-3
+    for am in (run["am"], run["am2"]):
+        assert np.array_equal(am[decided], g["argmax"][decided])
+
+
+def test_block_in_bench_configuration(run):
+    b, model, kv = run["binding"], run["model"], run["kv"]
+    nf = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = b.dg_generate_block(model, kv, W.T, W.gamma, n_forwards=nf)
+    out2 = b.dg_generate_block(model, kv, W.T, W.gamma)
+    dc = torch.full((1, W.canvas), W.mask_id, dtype=torch.int32, device="cuda")
+    dm = torch.ones_like(dc, dtype=torch.uint8)
+    first = None
+    for k in range(W.T):
+        ent, am, n = b.dg_denoise_step(model, kv, dc, dm, W.T - k, W.T, W.gamma)
+        if k == 0:
+            first = (ent.clone(), am.clone())
+    b.dg_sync_status(model)
+    assert int(nf[0]) == W.T and not (out == W.mask_id).any()
+    assert torch.equal(out, out2) and torch.equal(out, dc)
+    assert np.array_equal(first[0][0].cpu().numpy(), run["ent2"])
+    assert np.array_equal(first[1][0].cpu().numpy(), run["am2"])

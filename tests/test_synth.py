@@ -46,3 +46,40 @@ def test_weight_rows_and_prompt():
     assert int(p.min()) >= 0 and int(p.max()) < w.vocab
     wb = workloads.LAYER1_BF16
     assert model_inputs.weight(wb, "l0.wo", (4, 2048), n_rows=4).dtype == torch.bfloat16
+
+
+def test_e4m3_codes_roundtrip_and_rounding():
+    from synth import fp8
+    codes = torch.arange(256, dtype=torch.uint8)
+    finite = codes[(codes & 0x7F) != 0x7F]
+    vals = fp8.e4m3_decode(finite)
+    # every finite code decodes to a value that encodes back to itself (0x80 is -0)
+    back = fp8.e4m3_encode(vals)
+    keep = finite != 0x80
+    assert torch.equal(back[keep], finite[keep])
+    assert float(vals.max()) == 448.0 and float(vals[vals > 0].min()) == 2.0 ** -9
+    # known points of the format: 1.0 = 0x38, 448 = 0x7E, 2^-6 = 0x08, 2^-9 = 0x01
+    for v, c in [(1.0, 0x38), (448.0, 0x7E), (2.0 ** -6, 0x08), (2.0 ** -9, 0x01), (-1.5, 0xBC)]:
+        assert int(fp8.e4m3_encode(torch.tensor([v], dtype=torch.float64))[0]) == c
+    # rounding is to the nearest representable value, ties to even, saturating
+    x = torch.tensor([1.0625, 1.1875, 1.0624, 500.0, -3e-3, 2.0 ** -10], dtype=torch.float64)
+    r = fp8.e4m3_round(x)
+    assert r.tolist() == [1.0, 1.25, 1.0, 448.0, -2 * 2.0 ** -9, 0.0]
+    # brute force: nearest of all finite values
+    grid = torch.unique(torch.cat([vals, -vals]))
+    xs = torch.linspace(-460, 460, 20001, dtype=torch.float64)
+    rr = fp8.e4m3_round(xs)
+    d = (xs[:, None] - grid[None, :]).abs()
+    assert torch.all((rr - xs).abs() <= d.min(dim=1).values + 1e-12)
+
+
+def test_fp8_block_scales():
+    from synth import fp8
+    w = gen.normal_values(4, "fp8test", 0, 4 * 256, 0.02).reshape(4, 256)
+    codes, scales = fp8.quantize_rows(w)
+    assert scales.shape == (4, 2) and codes.dtype == torch.uint8
+    deq = fp8.e4m3_decode(codes).reshape(4, 2, 128) * scales.double()[..., None]
+    blk = w.double().reshape(4, 2, 128)
+    # the largest element of every block is represented (almost) exactly; error <= 1/16 relative
+    assert torch.allclose(deq.abs().amax(2), blk.abs().amax(2), rtol=1e-6)
+    assert float(((deq - blk).abs() / blk.abs().amax(2, keepdim=True)).max()) <= 2.0 ** -4
