@@ -1,8 +1,8 @@
 """Writes the oracle's expected outputs for the full-size workloads to tests/golden/.
 
 Calls only `oracle/` and `synth/` (never the CUDA path).  Usage:
-    python tests/golden/make_golden.py layer1-bf16 [full30-bf16 ...]
-Each file <workload>.npz holds, for canvas 0 of the workload's first forward
+    python tests/golden/make_golden.py layer1-bf16 [full30-bf16 full30-b8-p8192:7 ...]
+Each file <workload>[-c<canvas>].npz holds, for one canvas of the workload's first forward
 (all [MASK], steps_left = T):
   H [C] fp32 entropies, H64 [C], argmax [C], margin [C] (top-1 minus top-2 logit),
   lse [C]; logit_rows [R] row ids and logit_cols [Vs] vocab ids with
@@ -29,11 +29,12 @@ from synth import model_inputs, workloads  # noqa: E402
 LOGIT_ROWS = [0, 1, 77, 128, 255]
 
 
-def make(name: str):
+def make(name: str, canvas_index: int = 0):
+    """Oracle outputs of the first forward of canvas `canvas_index` of the workload."""
     w = workloads.get(name)
     t0 = time.time()
     ws = om.Weights(w, keep_layers=False)
-    prompt = model_inputs.prompt(w)[0].numpy()
+    prompt = model_inputs.prompt(w.with_(batch=1), first=canvas_index)[0].numpy()
     canvas = np.full(w.canvas, w.mask_id)
     st = om.prefill_then_forward(ws, prompt, canvas, w.T, w.T, want_logits=True)
     cols = np.arange(0, w.vocab, max(1, w.vocab // 4096))
@@ -47,7 +48,8 @@ def make(name: str):
         rmarg.append((srt[:, w.top_k - 1] - srt[:, w.top_k]).min())
     c2, m2, n2, kg = osamp.eb_step(st["H"], st["argmax"], canvas, np.ones(w.canvas, np.uint8),
                                    w.T, w.gamma)
-    out = os.path.join(HERE, f"{name}.npz")
+    suffix = f"-c{canvas_index}" if canvas_index else ""
+    out = os.path.join(HERE, f"{name}{suffix}.npz")
     np.savez_compressed(out, H=st["H"], H64=st["H64"], argmax=st["argmax"], margin=st["margin"],
                         lse=st["lse"], logit_rows=np.array(rows), logit_cols=cols,
                         logits=st["logits"][rows][:, cols].astype(np.float64), kv_last=kv_last,
@@ -59,5 +61,7 @@ def make(name: str):
 
 
 if __name__ == "__main__":
-    for n in sys.argv[1:] or ["layer1-bf16"]:
-        make(n)
+    # arguments: workload names, optionally "name:canvas" to pick a canvas of the batch
+    for arg in sys.argv[1:] or ["layer1-bf16"]:
+        name, _, c = arg.partition(":")
+        make(name, int(c) if c else 0)

@@ -1,0 +1,79 @@
+"""Batch of 8 canvases, each with its own 8192-token prompt (sliding window 1024):
+the same 30-layer model; oracle values for canvases 0 and 7 from
+tests/golden/full30-b8-p8192[-c7].npz (written by make_golden.py from the oracle).
+
+Also checks the per-expert router load the block reports (every routed row of
+every forward counted once) and the block's properties at this size.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from synth import model_inputs, workloads
+
+from gpu_helpers import make_model, max_abs_rel
+
+pytestmark = pytest.mark.gpu
+W = workloads.FULL30_B8_P8192
+TOL = 2e-2
+HERE = os.path.join(os.path.dirname(__file__), "golden")
+GOLD = {0: os.path.join(HERE, "full30-b8-p8192.npz"), 7: os.path.join(HERE, "full30-b8-p8192-c7.npz")}
+
+
+@pytest.fixture(scope="module")
+def run():
+    if not all(os.path.exists(p) for p in GOLD.values()):
+        pytest.skip("golden files missing")
+    from masked_discrete_diffusion_b200 import binding
+    model = make_model(W)
+    kv = binding.dg_prefill(model, model_inputs.prompt(W, "cuda"))
+    assert kv.W == 1024
+    canvas = torch.full((W.batch, W.canvas), W.mask_id, dtype=torch.int32, device="cuda")
+    ent, am, lg, _ = binding.dg_debug_forward(model, kv, canvas, W.T, W.T, logits=True)
+    ent2, am2, _, _ = binding.dg_debug_forward(model, kv, canvas, W.T, W.T)
+    k, v = binding.dg_kv_read(kv)
+    binding.dg_sync_status(model)
+    out = {"binding": binding, "model": model, "kv": kv, "ent": ent.cpu().numpy(),
+           "ent2": ent2.cpu().numpy(), "am2": am2.cpu().numpy(), "per": {}}
+    lg = lg.reshape(W.batch, W.canvas, W.vocab)
+    for b, path in GOLD.items():
+        g = np.load(path)
+        rows = torch.as_tensor(g["logit_rows"]).cuda()
+        cols = torch.as_tensor(g["logit_cols"]).cuda()
+        out["per"][b] = dict(g=g, lg=lg[b][rows][:, cols].cpu().numpy(),
+                             k=k[[0, W.n_layers - 1], b, :, -8:].float().cpu().numpy(),
+                             v=v[[0, W.n_layers - 1], b, :, -8:].float().cpu().numpy())
+    del lg, k, v
+    yield out
+    kv.close()
+    model.close()
+
+
+@pytest.mark.parametrize("b", [0, 7])
+def test_canvas_against_oracle(run, b):
+    p = run["per"][b]
+    g = p["g"]
+    for i in range(2):
+        assert max_abs_rel(p["k"][i], g["kv_last"][i, 0]) < TOL
+        assert max_abs_rel(p["v"][i], g["kv_last"][i, 1]) < TOL
+    assert max_abs_rel(p["lg"], g["logits"]) < TOL
+    assert max_abs_rel(run["ent"][b], g["H"]) < TOL
+    assert max_abs_rel(run["ent2"][b], g["H"]) < TOL
+    eps = float(np.abs(p["lg"] - g["logits"]).max())
+    decided = g["margin"] > 2 * eps + 1e-3
+    assert np.array_equal(run["am2"][b][decided], g["argmax"][decided])
+
+
+def test_block_and_router_load(run):
+    b, model, kv = run["binding"], run["model"], run["kv"]
+    nf = torch.zeros(W.batch, dtype=torch.int32, device="cuda")
+    load = torch.zeros(W.n_layers, W.n_experts, dtype=torch.int32, device="cuda")
+    out = b.dg_generate_block(model, kv, W.T, W.gamma, n_forwards=nf, router_load=load)
+    b.dg_sync_status(model)
+    assert not (out == W.mask_id).any() and nf.cpu().tolist() == [W.T] * W.batch
+    per_layer = load.sum(dim=1).cpu().tolist()
+    assert per_layer == [W.batch * W.canvas * W.top_k * W.T] * W.n_layers
+    assert np.all(run["ent2"] >= 0) and np.all(run["ent2"] <= math.log(W.vocab) + 1e-3)
