@@ -254,8 +254,12 @@ def run_ours(args, w, world, rank, local):
     e1.record(stream)
     torch.cuda.synchronize()
     torch.cuda.nvtx.range_pop()
-    launches = binding.dg_launch_count(model) - n0
     clk = clocks.stop()
+    # the block's device-side loop runs as many forwards as needed (at most T)
+    fwd_per_block = int(nfwd.max().item())
+    launches = args.steps * (1 + binding.dg_block_loop_launches(model) * fwd_per_block)
+    if binding.dg_block_loop_launches(model) == 0:
+        launches = binding.dg_launch_count(model) - n0
     ms = e0.elapsed_time(e1)
     binding.dg_sync_status(model)
     barrier(world)
@@ -288,7 +292,7 @@ def run_ours(args, w, world, rank, local):
     ex_avg_s = ex_ms / 1e3 / max(ex_groups, 1)
     achieved = ex_bytes / ex_avg_s / 1e9
     peak = float(peaks["hbm_gbs"])
-    fwd_ms = ms_step / T
+    fwd_ms = ms_step / max(fwd_per_block, 1)
     t_roof = max(cost["bytes"] / (peak * 1e9), cost["flops"] / (float(peaks["bf16_tflops"]) * 1e12))
     kinds = {k: {"ms_per_step": v[0] / args.steps, "groups_per_step": v[1] / args.steps}
              for k, v in prof.items()}
@@ -304,7 +308,8 @@ def run_ours(args, w, world, rank, local):
                    "l2": "inputs larger than L2 (40 GB of weights streamed per forward)",
                    "parallelism": f"replicas x{world}"},
         "ms_per_forward": fwd_ms,
-        "tokens_per_forward": C / T,
+        "forwards_per_block": fwd_per_block,
+        "tokens_per_forward": C / max(fwd_per_block, 1),
         "forward_roofline": {"ms": t_roof * 1e3, "frac": t_roof * 1e3 / fwd_ms,
                              "alg_bytes": cost["bytes"], "alg_flops": cost["flops"],
                              "peak_src": peak_src},

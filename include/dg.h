@@ -160,8 +160,9 @@ dg_status dg_denoise_step(dg_model* m, const dg_kv* kv, int32_t* canvas, uint8_t
                           float* entropy, int32_t* argmax, int32_t* n_committed,
                           void* stream);
 
-/* Denoises B = kv's batch canvases from all [MASK] with T forwards
- * (steps_left = T, T-1, ..., 1), without synchronising the host between steps.
+/* Denoises B = kv's batch canvases from all [MASK] with at most T forwards
+ * (steps_left = T, T-1, ..., 1), without synchronising the host between steps;
+ * the loop stops on the device as soon as no canvas has a masked position left.
  * canvas_out: [B, C] int32 (no [MASK] remains); n_forwards: [B] int32, the
  * number of forwards after which that canvas had no [MASK] left (nullable);
  * router_load: [n_layers, E] int32 counts of (token, expert) routings summed
@@ -212,6 +213,11 @@ dg_status dg_profile_stop(dg_model* m, float* ms, int64_t* groups);
  * one row — i.e. expert weight tiles streamed — since dg_profile_start (or model
  * creation).  Synchronises the device. */
 dg_status dg_expert_units(dg_model* m, int64_t* units);
+
+/* Kernels launched per loop iteration (one forward + sampler step + loop control) by
+ * the last dg_generate_block replay; its device-controlled loop runs as many
+ * iterations as forwards were needed (at most T), which n_forwards reports. */
+dg_status dg_block_loop_launches(const dg_model* m, int64_t* per_forward);
 
 /* Number of kernels this model has launched since it was created (host count). */
 dg_status dg_launch_count(const dg_model* m, int64_t* out);

@@ -81,6 +81,7 @@ def lib() -> ctypes.CDLL:
             "dg_profile_stop": [vp, vp, vp],
             "dg_launch_count": [vp, ctypes.POINTER(ctypes.c_int64)],
             "dg_expert_units": [vp, ctypes.POINTER(ctypes.c_int64)],
+            "dg_block_loop_launches": [vp, ctypes.POINTER(ctypes.c_int64)],
             "dg_lmhead_entropy_noalloc": [vp, vp, i32, i32, i32, f32, f32, vp, vp, vp],
             "dg_op_gemm": [vp, vp, vp, vp, i32, i32, i32, vp],
             "dg_op_moe": [vp, i32, vp, vp, i32, vp],
@@ -99,7 +100,7 @@ def exported_symbols():
                         "dg_kv_read", "dg_denoise_step", "dg_generate_block", "dg_eb_sample",
                         "dg_debug_forward", "dg_profile_start", "dg_profile_stop",
                         "dg_launch_count", "dg_op_gemm", "dg_op_moe", "dg_expert_units",
-                        "dg_lmhead_entropy_noalloc")
+                        "dg_lmhead_entropy_noalloc", "dg_block_loop_launches")
             if hasattr(lib(), n)]
 
 
@@ -307,3 +308,9 @@ def dg_lmhead_entropy_noalloc(hidden, lm_head, rms_eps: float, logit_scale: floa
     _check(lib().dg_lmhead_entropy_noalloc(_ptr(hidden), _ptr(lm_head), M, V, d, rms_eps,
                                            logit_scale, _ptr(ent), _ptr(am), _stream(stream)))
     return ent, am
+
+
+def dg_block_loop_launches(model: Model) -> int:
+    out = ctypes.c_int64()
+    _check(lib().dg_block_loop_launches(model.handle, ctypes.byref(out)))
+    return out.value

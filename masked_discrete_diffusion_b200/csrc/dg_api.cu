@@ -160,6 +160,8 @@ template <class Path> static dg_status alloc_workspace(dg_model* m) {
   DG_TRY(ws_alloc(ws, &ws.ent, lm_rows));
   DG_TRY(ws_alloc(ws, &ws.amax, lm_rows));
   DG_TRY(ws_alloc(ws, &ws.ncommit, c.max_batch));
+  DG_TRY(ws_alloc(ws, &ws.remaining, c.max_batch));
+  DG_TRY(ws_alloc(ws, &ws.loop_s, 1));
   DG_TRY_CUDA(cudaMemset(ws.err, 0, 4 * sizeof(int32_t)));
   launch_pdl((rope_table_kernel), 256, 256, 0, cudaStream_t(0), 1, (double)c.rope_base, (int)h, ws.max_pos, ws.rope,
                                   sizeof(Acc) == 8 ? 1 : 0);
@@ -192,7 +194,9 @@ template <class Path> struct Runner {
   const dg_config& c;
   Workspace& ws;
   cudaStream_t st;
-  Runner(dg_model* m_, cudaStream_t st_) : m(m_), c(m_->cfg), ws(m_->ws), st(st_) {}
+  const int32_t* s_dev = nullptr;  // steps left in device memory (captured block loop)
+  Runner(dg_model* m_, cudaStream_t st_, const int32_t* s_dev_ = nullptr)
+      : m(m_), c(m_->cfg), ws(m_->ws), st(st_), s_dev(s_dev_) {}
 
   TR* x() { return (TR*)ws.x; }
   TA* xn() { return (TA*)ws.xn; }
@@ -373,7 +377,8 @@ template <class Path> struct Runner {
     const size_t es = sizeof(TKV);
     for (int b = 0; b < B; ++b) {
       launch_pdl((embed_kernel<TW, TR>), P, 256, 0, st, 1, prompt + (size_t)b * P, (const TW*)m->w.tok_emb,
-                                             x(), P, d, c.vocab - 1, -1.0, ws.err);
+                                             x(), P, d, c.vocab - 1, -1.0, ws.err,
+                                             (const int32_t*)nullptr, 1);
       ++m->launches;
       // padding columns of the transposed values must read as zero
       DG_TRY_CUDA(cudaMemsetAsync(ws.vc, 0, (size_t)Hkv * h * Pp * es, st));
@@ -402,7 +407,7 @@ template <class Path> struct Runner {
     const int B = kv->B, C = c.canvas, n = B * C, d = c.d_model;
     const double tau = (double)s / (double)T;
     launch_pdl((embed_kernel<TW, TR>), n, 256, 0, st, 1, canvas, (const TW*)m->w.tok_emb, x(), n, d, c.vocab,
-                                           tau, ws.err);
+                                           tau, ws.err, (const int32_t*)s_dev, T);
     ++m->launches;
     const int Cp = (C + 63) / 64 * 64;
     if (Cp != C)
@@ -457,10 +462,12 @@ static dg_status gamma_fixed(float gamma, long long* out) {
 static dg_status launch_sampler(const float* H, const int32_t* am, int32_t* canvas,
                                 uint8_t* mask, int B, int C, int s, long long gq,
                                 int32_t* ncommit, int32_t* nfwd, int step_no,
-                                cudaStream_t st, long long* counter_) {
+                                cudaStream_t st, long long* counter_,
+                                const int32_t* s_dev = nullptr, int T = 0,
+                                int32_t* remaining = nullptr) {
 #define DG_SAMP(NP)                                                                       \
   launch_pdl((eb_sample_kernel<NP>), B, NP, 0, st, 1, H, am, canvas, mask, C, s, gq, ncommit, nfwd, \
-                                         step_no)
+                                         step_no, s_dev, T, remaining)
   if (C <= 32) DG_SAMP(32);
   else if (C <= 64) DG_SAMP(64);
   else if (C <= 128) DG_SAMP(128);
@@ -691,10 +698,10 @@ static dg_status check_step_args(dg_model* m, const dg_kv* kv, int s, int T) {
 
 static dg_status run_forward(dg_model* m, const dg_kv* kv, const int32_t* canvas, int s, int T,
                              float* ent, int32_t* am, float* logits, float* hidden,
-                             int32_t* load, cudaStream_t st) {
+                             int32_t* load, cudaStream_t st, const int32_t* s_dev = nullptr) {
   return m->cfg.dtype == DG_F32
-             ? Runner<PathTiny>(m, st).forward(kv, canvas, s, T, ent, am, logits, hidden, load)
-             : Runner<PathBF16>(m, st).forward(kv, canvas, s, T, ent, am, logits, hidden, load);
+             ? Runner<PathTiny>(m, st, s_dev).forward(kv, canvas, s, T, ent, am, logits, hidden, load)
+             : Runner<PathBF16>(m, st, s_dev).forward(kv, canvas, s, T, ent, am, logits, hidden, load);
 }
 
 dg_status dg_denoise_step(dg_model* m, const dg_kv* kv, int32_t* canvas, uint8_t* mask,
@@ -735,6 +742,78 @@ static dg_status generate_impl(dg_model* m, const dg_kv* kv, int32_t T, long lon
   return DG_OK;
 }
 
+static dg_status replay(dg_model* m, dg::BlockGraph* g, cudaStream_t st);
+
+// Builds the block as a graph with a device-controlled loop: an init kernel, then a
+// WHILE node whose body is one forward + sampler step + a control kernel that
+// decrements the device-side steps-left counter and stops the loop once the
+// counter reaches 0 or no canvas has a masked position left (the oracle's early
+// stop).  Returns false (nothing built) if this CUDA build refuses a step.
+static bool build_loop_graph(dg_model* m, const dg_kv* kv, int32_t T, long long gq,
+                             int32_t* canvas_out, int32_t* n_forwards, int32_t* router_load,
+                             dg::BlockGraph* g) {
+  const dg_config& c = m->cfg;
+  Workspace& ws = m->ws;
+  const int B = kv->B, C = c.canvas;
+  cudaStream_t cap = m->cap_stream;
+  cudaGraph_t graph = nullptr;
+  if (cudaGraphCreate(&graph, 0) != cudaSuccess) return false;
+  bool ok = false;
+  do {
+    cudaGraphConditionalHandle handle;
+    if (cudaGraphConditionalHandleCreate(&handle, graph, 1, cudaGraphCondAssignDefault) !=
+        cudaSuccess)
+      break;
+    if (cudaStreamBeginCaptureToGraph(cap, graph, nullptr, nullptr, 0,
+                                      cudaStreamCaptureModeThreadLocal) != cudaSuccess)
+      break;
+    const int n = B * C, n_load = router_load ? c.n_layers * c.n_experts : 0;
+    launch_pdl((block_init_kernel), ceil_div(std::max(n, n_load), 256), 256, 0, cap, 1, canvas_out,
+               ws.mask, n, (int32_t)c.vocab, n_forwards, B, router_load, n_load, ws.loop_s, T);
+    cudaGraph_t g1 = nullptr;
+    if (cudaStreamEndCapture(cap, &g1) != cudaSuccess) break;
+    size_t nn = 0;
+    cudaGraphGetNodes(graph, nullptr, &nn);
+    std::vector<cudaGraphNode_t> nodes(nn);
+    cudaGraphGetNodes(graph, nodes.data(), &nn);
+    cudaGraphNodeParams cp = {};
+    cp.type = cudaGraphNodeTypeConditional;
+    cp.conditional.handle = handle;
+    cp.conditional.type = cudaGraphCondTypeWhile;
+    cp.conditional.size = 1;
+    cudaGraphNode_t cnode;
+    if (cudaGraphAddNode(&cnode, graph, nodes.data(), nn, &cp) != cudaSuccess) break;
+    cudaGraph_t body = cp.conditional.phGraph_out[0];
+    if (cudaStreamBeginCaptureToGraph(cap, body, nullptr, nullptr, 0,
+                                      cudaStreamCaptureModeThreadLocal) != cudaSuccess)
+      break;
+    const long long l0 = m->launches;
+    dg_status s = run_forward(m, kv, canvas_out, T, T, ws.ent, ws.amax, nullptr, nullptr,
+                              router_load, cap, ws.loop_s);
+    if (s == DG_OK)
+      s = launch_sampler(ws.ent, ws.amax, canvas_out, ws.mask, B, C, T, gq, ws.ncommit,
+                         n_forwards, 1, cap, &m->launches, ws.loop_s, T, ws.remaining);
+    launch_pdl((block_step_kernel), 1, 32, 0, cap, 1, handle, ws.loop_s,
+               (const int32_t*)ws.remaining, B);
+    g->body_launches = m->launches - l0 + 1;
+    m->launches = l0;
+    cudaGraph_t g2 = nullptr;
+    const cudaError_t e = cudaStreamEndCapture(cap, &g2);
+    if (s != DG_OK || e != cudaSuccess) break;
+    if (cudaGraphInstantiate(&g->exec, graph, 0) != cudaSuccess) break;
+    g->launches = 1;
+    g->loop = true;
+    ok = true;
+  } while (false);
+  cudaGraphDestroy(graph);
+  if (!ok) {
+    cudaGetLastError();
+    if (g->exec) cudaGraphExecDestroy(g->exec);
+    g->exec = nullptr;
+  }
+  return ok;
+}
+
 // Captures the block's launch sequence once per (kv, T, gamma, output buffers,
 // profiling) and replays it: one host call per block instead of ~500 launches per
 // forward.  With profiling on, the graph also records an event pair around every
@@ -762,14 +841,17 @@ static dg_status generate_graphed(dg_model* m, const dg_kv* kv, int32_t T, long 
     g->nfwd = n_forwards;
     g->load = router_load;
     g->prof = m->profiling;
-    const long long l0 = m->launches;
-    m->capture = g;
     // capture on a library-owned stream (the caller's may be the legacy default
     // stream, which cannot be captured); nothing executes during capture
+    if (!m->cap_stream) DG_TRY_CUDA(cudaStreamCreateWithFlags(&m->cap_stream, cudaStreamNonBlocking));
+    if (!g->prof && build_loop_graph(m, kv, T, gq, canvas_out, n_forwards, router_load, g)) {
+      m->graphs.push_back(g);
+      return replay(m, g, st);
+    }
+    const long long l0 = m->launches;
+    m->capture = g;
     cudaGraph_t graph = nullptr;
-    cudaError_t e = cudaSuccess;
-    if (!m->cap_stream) e = cudaStreamCreateWithFlags(&m->cap_stream, cudaStreamNonBlocking);
-    if (e == cudaSuccess) e = cudaStreamBeginCapture(m->cap_stream, cudaStreamCaptureModeThreadLocal);
+    cudaError_t e = cudaStreamBeginCapture(m->cap_stream, cudaStreamCaptureModeThreadLocal);
     dg_status s = DG_OK;
     if (e == cudaSuccess) {
       s = generate_impl(m, kv, T, gq, canvas_out, n_forwards, router_load, m->cap_stream);
@@ -791,8 +873,13 @@ static dg_status generate_graphed(dg_model* m, const dg_kv* kv, int32_t T, long 
     }
     m->graphs.push_back(g);
   }
+  return replay(m, g, st);
+}
+
+static dg_status replay(dg_model* m, dg::BlockGraph* g, cudaStream_t st) {
   DG_TRY_CUDA(cudaGraphLaunch(g->exec, st));
   m->launches += g->launches;
+  m->last_body_launches = g->loop ? g->body_launches : 0;
   if (g->prof) {
     DG_TRY_CUDA(cudaStreamSynchronize(st));
     for (int k = 0; k < DG_KIND_COUNT; ++k)
@@ -904,6 +991,12 @@ dg_status dg_profile_stop(dg_model* m, float* ms, int64_t* groups) {
 dg_status dg_launch_count(const dg_model* m, int64_t* out) {
   DG_REQUIRE(m && out, "null argument");
   *out = m->launches;
+  return DG_OK;
+}
+
+dg_status dg_block_loop_launches(const dg_model* m, int64_t* per_forward) {
+  DG_REQUIRE(m && per_forward, "null argument");
+  *per_forward = m->last_body_launches;
   return DG_OK;
 }
 

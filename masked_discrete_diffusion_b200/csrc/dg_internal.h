@@ -103,6 +103,7 @@ struct Workspace {
   uint8_t* mask = nullptr;                          // [max_batch, C] block-loop mask
   float* ent = nullptr;                             // [max_batch, C] entropies
   int32_t *amax = nullptr, *ncommit = nullptr;      // [max_batch, C], [max_batch]
+  int32_t *remaining = nullptr, *loop_s = nullptr;  // [max_batch] masked left; steps left
   int max_pos = 0;
   size_t kc_elems = 0;
   void *attn_o = nullptr, *attn_ml = nullptr;  // attention key-split partials
@@ -121,7 +122,9 @@ struct BlockGraph {
   long long gq = 0;
   int32_t *canvas = nullptr, *nfwd = nullptr, *load = nullptr;
   bool prof = false;
-  long long launches = 0;  // kernel launches the graph replays
+  long long launches = 0;  // kernel launches the graph replays (1 for a loop graph: the init)
+  bool loop = false;       // device-controlled WHILE loop over forwards
+  long long body_launches = 0;  // kernels per loop iteration (forward + sampler + control)
   std::vector<std::pair<cudaEvent_t, cudaEvent_t>> ev[DG_KIND_COUNT];
 };
 }  // namespace dg
@@ -144,6 +147,7 @@ struct dg_model {
   std::vector<dg::BlockGraph*> graphs;
   dg::BlockGraph* capture = nullptr;  // graph being captured (events go there)
   cudaStream_t cap_stream = nullptr;  // private stream used only for capturing
+  long long last_body_launches = 0;   // kernels per forward of the last replayed loop graph
 };
 
 namespace dg {

@@ -35,8 +35,13 @@ __global__ void __launch_bounds__(NP)
     eb_sample_kernel(const float* __restrict__ H, const int32_t* __restrict__ amax,
                      int32_t* __restrict__ canvas, uint8_t* __restrict__ mask, int C,
                      int steps_left, long long gamma_q, int32_t* __restrict__ n_commit,
-                     int32_t* __restrict__ n_fwd, int step_no) {
+                     int32_t* __restrict__ n_fwd, int step_no, const int32_t* __restrict__ s_dev,
+                     int T, int32_t* __restrict__ remaining) {
   pdl_enter();
+  if (s_dev) {  // steps left read from device memory (captured block loop)
+    steps_left = *s_dev;
+    step_no = T - steps_left + 1;
+  }
   __shared__ unsigned long long key[NP];
   __shared__ long long pre[NP];
   __shared__ int cnt[NP / 32];
@@ -96,6 +101,7 @@ __global__ void __launch_bounds__(NP)
     mask[base + pos] = 0;
   }
   if (i == 0 && n_commit) n_commit[b] = n;
+  if (i == 0 && remaining) remaining[b] = m - n;
   // the forward after which this canvas has no [MASK] left
   if (i == 0 && n_fwd && m > 0 && n == m) n_fwd[b] = step_no;
 }

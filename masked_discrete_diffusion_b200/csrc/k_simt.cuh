@@ -18,12 +18,14 @@ namespace dg {
 // a1: embedding gather (+ sinusoidal timestep embedding for canvas rows)
 // x[t, :] = E[ids[t], :] + temb(tau); temb[i] = sin(1000 tau w_i),
 // temb[d/2 + i] = cos(1000 tau w_i), w_i = 10000^(-i / (d/2)).  tau < 0: none.
+// With s_dev set, tau = *s_dev / T (steps left read from device memory).
 // ---------------------------------------------------------------------------
 template <class TW, class TR>
 __global__ void embed_kernel(const int32_t* __restrict__ ids, const TW* __restrict__ emb,
                              TR* __restrict__ x, int n_tok, int d, int max_id, double tau,
-                             int32_t* err) {
+                             int32_t* err, const int32_t* __restrict__ s_dev, int T) {
   pdl_enter();
+  if (s_dev) tau = (double)*s_dev / (double)T;
   const int t = blockIdx.x;
   if (t >= n_tok) return;
   int id = ids[t];
@@ -742,6 +744,36 @@ __global__ void to_f32_kernel(const T* __restrict__ src, float* __restrict__ dst
   pdl_enter();
   const long i = blockIdx.x * (long)blockDim.x + threadIdx.x;
   if (i < n) dst[i] = (float)widen(src[i]);
+}
+
+// Start of a block: canvas all [MASK], mask all 1, counters cleared, steps left = T.
+static __global__ void block_init_kernel(int32_t* __restrict__ canvas, uint8_t* __restrict__ mask,
+                                         int n, int32_t mask_id, int32_t* __restrict__ nfwd,
+                                         int B, int32_t* __restrict__ load, int n_load,
+                                         int32_t* __restrict__ s_dev, int T) {
+  pdl_enter();
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) {
+    canvas[i] = mask_id;
+    mask[i] = 1;
+  }
+  if (nfwd && i < B) nfwd[i] = 0;
+  if (load && i < n_load) load[i] = 0;
+  if (i == 0) *s_dev = T;
+}
+
+// End of one loop iteration of the captured block: steps left -= 1; run the next
+// iteration only if steps remain and some canvas still has masked positions.
+static __global__ void block_step_kernel(cudaGraphConditionalHandle handle,
+                                         int32_t* __restrict__ s_dev,
+                                         const int32_t* __restrict__ remaining, int B) {
+  pdl_enter();
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  const int s = *s_dev - 1;
+  *s_dev = s;
+  int any = 0;
+  for (int b = 0; b < B; ++b) any |= remaining[b] > 0;
+  cudaGraphSetConditional(handle, (s > 0 && any) ? 1u : 0u);
 }
 
 static __global__ void fill_i32_kernel(int32_t* __restrict__ p, int n, int32_t v) {

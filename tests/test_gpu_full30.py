@@ -92,7 +92,9 @@ def test_block_in_bench_configuration(run):
         if k == 0:
             first = (ent.clone(), am.clone())
     b.dg_sync_status(model)
-    assert int(nf[0]) == W.T and not (out == W.mask_id).any()
+    # the loop stops once nothing is masked: at most T forwards (here the entropy bound
+    # commits the whole canvas before the ceil(m / s) minimum would)
+    assert 1 <= int(nf[0]) <= W.T and not (out == W.mask_id).any()
     assert torch.equal(out, out2) and torch.equal(out, dc)
     assert np.array_equal(first[0][0].cpu().numpy(), run["ent2"])
     assert np.array_equal(first[1][0].cpu().numpy(), run["am2"])
