@@ -9,6 +9,7 @@ from __future__ import annotations
 
 import ctypes
 import os
+import weakref
 
 import torch
 
@@ -153,8 +154,12 @@ class Model:
         h = ctypes.c_void_p()
         _check(lib().dg_model_create(ctypes.byref(cfg), ctypes.byref(self._w), ctypes.byref(h)))
         self.handle = h
+        self._kvs = weakref.WeakSet()
 
     def close(self):
+        """Destroys the model after every KV cache created from it."""
+        for kv in list(getattr(self, "_kvs", ())):
+            kv.close()
         if getattr(self, "handle", None):
             _check(lib().dg_model_destroy(self.handle))
             self.handle = None
@@ -170,6 +175,7 @@ class KV:
     def __init__(self, model: Model, handle):
         self.model = model
         self.handle = handle
+        model._kvs.add(self)
         B, P, W = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
         _check(lib().dg_kv_info(handle, ctypes.byref(B), ctypes.byref(P), ctypes.byref(W)))
         self.B, self.P, self.W = B.value, P.value, W.value

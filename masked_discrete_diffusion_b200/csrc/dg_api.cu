@@ -7,6 +7,7 @@
 //   router -> permute -> grouped gate/up GEMM (SwiGLU) -> grouped down GEMM
 //   (x gate) -> shared expert -> combine (+residual) }  ->  RMSNorm -> LM-head
 //   statistics -> merge  ->  EB sampler.
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -571,6 +572,8 @@ dg_status dg_model_destroy(dg_model* m) {
   if (!m) return DG_OK;
   cudaDeviceSynchronize();
   release_graphs(m);
+  for (dg_kv* kv : m->kvs) kv->m = nullptr;  // caches outlive the model only to be destroyed
+  m->kvs.clear();
   if (m->cap_stream) cudaStreamDestroy(m->cap_stream);
   for (int k = 0; k < DG_KIND_COUNT; ++k)
     for (auto& e : m->prof[k]) {
@@ -641,6 +644,7 @@ dg_status dg_prefill(dg_model* m, const int32_t* prompt, int32_t B, int32_t P, d
     delete kv;
     return s;
   }
+  m->kvs.push_back(kv);
   *out = kv;
   return DG_OK;
 }
@@ -648,15 +652,18 @@ dg_status dg_prefill(dg_model* m, const int32_t* prompt, int32_t B, int32_t P, d
 dg_status dg_kv_destroy(dg_kv* kv) {
   if (!kv) return DG_OK;
   cudaDeviceSynchronize();
-  // graphs captured for this cache hold its pointers: drop them
-  auto& gs = kv->m->graphs;
-  for (size_t i = 0; i < gs.size();) {
-    if (gs[i]->kv == kv) {
-      graph_free(gs[i]);
-      gs.erase(gs.begin() + i);
-    } else {
-      ++i;
+  if (kv->m) {  // the model is still alive: forget this cache and its captured graphs
+    dg_model* m = kv->m;
+    auto& gs = m->graphs;
+    for (size_t i = 0; i < gs.size();) {
+      if (gs[i]->kv == kv) {
+        graph_free(gs[i]);
+        gs.erase(gs.begin() + i);
+      } else {
+        ++i;
+      }
     }
+    m->kvs.erase(std::remove(m->kvs.begin(), m->kvs.end(), kv), m->kvs.end());
   }
   cudaFree(kv->k);
   cudaFree(kv->v);
@@ -674,6 +681,7 @@ dg_status dg_kv_info(const dg_kv* kv, int32_t* B, int32_t* P, int32_t* W) {
 
 dg_status dg_kv_read(const dg_kv* kv, void* k, void* v, void* stream) {
   DG_REQUIRE(kv && k && v, "null argument");
+  DG_REQUIRE(kv->m, "kv handle's model was destroyed");
   const dg_config& c = kv->m->cfg;
   cudaStream_t st = (cudaStream_t)stream;
   const size_t blocks = (size_t)c.n_layers * kv->B * c.n_kv_heads;
@@ -691,6 +699,7 @@ dg_status dg_kv_read(const dg_kv* kv, void* k, void* v, void* stream) {
 
 static dg_status check_step_args(dg_model* m, const dg_kv* kv, int s, int T) {
   DG_REQUIRE(m && kv, "null model/kv");
+  DG_REQUIRE(kv->m, "kv handle's model was destroyed");
   DG_REQUIRE(kv->m == m, "kv handle belongs to another model");
   DG_REQUIRE(T >= 1 && s >= 1 && s <= T, "steps_left=%d must be in [1, T=%d]", s, T);
   return DG_OK;

@@ -148,6 +148,7 @@ struct dg_model {
   dg::BlockGraph* capture = nullptr;  // graph being captured (events go there)
   cudaStream_t cap_stream = nullptr;  // private stream used only for capturing
   long long last_body_launches = 0;   // kernels per forward of the last replayed loop graph
+  std::vector<dg_kv*> kvs;            // live KV caches created from this model
 };
 
 namespace dg {

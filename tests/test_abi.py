@@ -59,3 +59,9 @@ def test_host_validation_without_device(lib):
     assert lib.dg_model_create(ctypes.byref(cfg), ctypes.byref(w), ctypes.byref(out)) == 1
     assert b"multiple" in lib.dg_last_error()
     assert lib.dg_model_destroy(None) == 0 and lib.dg_kv_destroy(None) == 0
+
+
+def test_kv_destroy_after_model_destroy_is_safe_without_device(lib):
+    # only null handles can be exercised without a GPU; the ordering itself is
+    # covered on the GPU by the model/KV lifetime test
+    assert lib.dg_kv_destroy(None) == 0 and lib.dg_model_destroy(None) == 0

@@ -95,3 +95,19 @@ def test_bad_token_reported(setup):
     with pytest.raises(binding.DGError) as e:
         binding.dg_sync_status(model)
     assert e.value.status == 1
+
+
+def test_kv_outlives_model():
+    """Destroying the model first leaves its caches destroyable, and unusable."""
+    from masked_discrete_diffusion_b200 import binding
+    model = make_model(W)
+    kv = binding.dg_prefill(model, model_inputs.prompt(W, "cuda"))
+    binding.dg_sync_status(model)
+    h = kv.handle
+    binding._check(binding.lib().dg_model_destroy(model.handle))
+    model.handle = None
+    n = torch.zeros(1, dtype=torch.int32, device="cuda")
+    st = binding.lib().dg_kv_read(h, n.data_ptr(), n.data_ptr(), None)
+    assert st == 1                                        # DG_ERR_INVALID_ARG
+    assert binding.lib().dg_kv_destroy(h) == 0
+    kv.handle = None
