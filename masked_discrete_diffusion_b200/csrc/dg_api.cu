@@ -226,17 +226,27 @@ template <class Path> struct Runner {
     const int d = c.d_model, h = c.head_dim, Hq = c.n_q_heads, Hkv = c.n_kv_heads;
     const int qkv_n = (Hq + 2 * Hkv) * h;
     rmsnorm(n);
+    bool fused_rope = false;
     {
       ProfScope ps(m, DG_KIND_DENSE, st);
-      if constexpr (Path::kTensorCores)
-        DG_TRY(tc_gemm_store_f32(m, xn(), L.wqkv, (float*)ws.qkv, n, qkv_n, d, st));
-      else
+      if constexpr (Path::kTensorCores) {
+        if (h == 128) {  // RoPE and the q / k / v scatter in the GEMM epilogue
+          DG_TRY(tc_gemm_qkv_rope(m, xn(), L.wqkv, n, n_seq, np, pos0, (bf16*)ws.q,
+                                  (bf16*)ws.kc, (bf16*)ws.vc, st));
+          fused_rope = true;
+        } else {
+          DG_TRY(tc_gemm_store_f32(m, xn(), L.wqkv, (float*)ws.qkv, n, qkv_n, d, st));
+        }
+      } else {
         dense(xn(), d, L.wqkv, qkv_n, d, n, EpiStore<Acc, Acc>{(Acc*)ws.qkv, qkv_n});
+      }
     }
-    launch_pdl((rope_scatter_kernel<Acc, TA, TKV>), n, 128, 0, st, 1, 
-        (const Acc*)ws.qkv, (TA*)ws.q, (TKV*)ws.kc, (TKV*)ws.vc, n, n_seq, np, pos0, Hq, Hkv, h,
-        (const Acc*)ws.rope, ws.max_pos);
-    ++m->launches;
+    if (!fused_rope) {
+      launch_pdl((rope_scatter_kernel<Acc, TA, TKV>), n, 128, 0, st, 1,
+          (const Acc*)ws.qkv, (TA*)ws.q, (TKV*)ws.kc, (TKV*)ws.vc, n, n_seq, np, pos0, Hq, Hkv, h,
+          (const Acc*)ws.rope, ws.max_pos);
+      ++m->launches;
+    }
     {
       ProfScope ps(m, DG_KIND_ATTENTION, st);
       bool done = false;

@@ -45,7 +45,7 @@ template <int COLS> struct TmemCols {
 // (v: the accumulator, u: the second weight's accumulator for dual GEMMs).
 template <class Derived, bool DUAL>
 struct EpiChunked {
-  static constexpr bool kChunked = true;
+  static constexpr bool kChunked = true, kRowWise = false;
   template <int NCH, class Ld>
   __device__ void run(int row, bool valid, int n0, Ld&& ld) const {
 #pragma unroll 1
@@ -110,11 +110,66 @@ struct EpiSwigluBf16 : EpiChunked<EpiSwigluBf16, true> {
   }
 };
 
+// QKV projection epilogue (N-tile = one head of h = 128): rotate query and key
+// heads (pairs (j, j + 64) by pos * theta_j, cos/sin from the table
+// rope[pos, 64] / rope[max_pos + pos, 64]) and scatter: q -> q[row, head, :],
+// k -> kc[b, g, i, :], v -> vc[b, g, :, i] (transposed); all bf16.  Row = b * n_seq + i
+// sits at position pos0 + i.
+struct EpiQkvRope {
+  static constexpr bool kChunked = false, kRowWise = true;
+  bf16 *q, *kc, *vc;
+  const float* rope;
+  int max_pos, n_seq, np, pos0, Hq, Hkv;
+  template <int NCH, class Ld>
+  __device__ void run(int row, bool valid, int n0, Ld&& ld) const {
+    static_assert(NCH == 4, "one head of 128 per tile");
+    const int head = n0 / 128;
+    const int b = valid ? row / n_seq : 0, i = valid ? row % n_seq : 0, pos = pos0 + i;
+#pragma unroll 1
+    for (int c = 0; c < 2; ++c) {
+      float lo[32], hi[32];
+      ld(0, c, lo);
+      ld(0, c + 2, hi);
+      if (!valid) continue;
+      if (head < Hq + Hkv) {
+        const float* cs = rope + (size_t)pos * 64 + c * 32;
+        const float* sn = rope + ((size_t)max_pos + pos) * 64 + c * 32;
+        bf16* dst = head < Hq ? q + ((size_t)row * Hq + head) * 128
+                              : kc + (((size_t)b * Hkv + (head - Hq)) * np + i) * 128;
+        uint32_t w1[16], w2[16];
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          const float c0 = cs[j], s0 = sn[j], c1 = cs[j + 1], s1 = sn[j + 1];
+          __nv_bfloat162 a = __floats2bfloat162_rn(lo[j] * c0 - hi[j] * s0, lo[j + 1] * c1 - hi[j + 1] * s1);
+          __nv_bfloat162 bb = __floats2bfloat162_rn(hi[j] * c0 + lo[j] * s0, hi[j + 1] * c1 + lo[j + 1] * s1);
+          w1[j >> 1] = *reinterpret_cast<uint32_t*>(&a);
+          w2[j >> 1] = *reinterpret_cast<uint32_t*>(&bb);
+        }
+        uint4* d1 = reinterpret_cast<uint4*>(dst + c * 32);
+        uint4* d2 = reinterpret_cast<uint4*>(dst + 64 + c * 32);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          d1[j] = make_uint4(w1[4 * j], w1[4 * j + 1], w1[4 * j + 2], w1[4 * j + 3]);
+          d2[j] = make_uint4(w2[4 * j], w2[4 * j + 1], w2[4 * j + 2], w2[4 * j + 3]);
+        }
+      } else {
+        const int g = head - Hq - Hkv;
+        bf16* vt = vc + ((size_t)b * Hkv + g) * 128 * np + i;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          vt[(size_t)(c * 32 + j) * np] = __float2bfloat16_rn(lo[j]);
+          vt[(size_t)(64 + c * 32 + j) * np] = __float2bfloat16_rn(hi[j]);
+        }
+      }
+    }
+  }
+};
+
 // Per-row statistics of logits l = scale * acc over this CTA's vocabulary tile
 // (columns n0 .. n0 + 32 NCH - 1, those < N): m = max, s = sum exp(l - m),
 // u = sum exp(l - m) (l - m), a = lowest id attaining m.  part[(tile, row)] = (m, s, u, a).
 struct EpiLmStats {
-  static constexpr bool kChunked = false;
+  static constexpr bool kChunked = false, kRowWise = false;
   float* part;
   int M, N;
   float scale;
@@ -209,7 +264,8 @@ __global__ void __launch_bounds__(128, 1)
   typedef DenseCfg<BN, MT, DUAL, ST> Cfg;
   // split-K needs the whole fp32 tile in the (drained) pipeline buffers and a chunk epilogue
   constexpr int RS = Cfg::NACC * BN + 4;  // reduction row stride (floats): padded against bank conflicts
-  constexpr bool kSplitOK = MT * 128 * RS * 4 <= ST * Cfg::STAGE && Epi::kChunked;
+  constexpr bool kSplitOK =
+      MT * 128 * RS * 4 <= ST * Cfg::STAGE && (Epi::kChunked || Epi::kRowWise);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + ST * Cfg::STAGE);
@@ -342,6 +398,21 @@ __global__ void __launch_bounds__(128, 1)
     }
     cl::sync();                              // all partial rows delivered
     const float* buf = reinterpret_cast<const float*>(smem);
+    if constexpr (Epi::kRowWise) {  // one thread per owned row, chunks summed on demand
+      for (int lr = threadIdx.x; lr < R; lr += blockDim.x) {
+        auto ld = [&](int a, int c, float* v) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = 0.f;
+          for (int src = 0; src < ksplit; ++src) {
+            const float* p = buf + (size_t)(src * R + lr) * RS + a * BN + c * 32;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] += p[j];
+          }
+        };
+        const int row = m0 + rank * R + lr;
+        epi.template run<BN / 32>(row, row < M, n0, ld);
+      }
+    } else
     for (int item = threadIdx.x; item < R * (BN / 32); item += blockDim.x) {
       const int lr = item / (BN / 32), c = item % (BN / 32);
       float v[32], u[32];
@@ -560,6 +631,8 @@ void tc_release(dg_model* m);
 inline int tc_group_rows() { return 128; }
 dg_status tc_gemm_store_f32(dg_model* m, const bf16* A, const void* W, float* out, int M, int N,
                             int K, cudaStream_t st);
+dg_status tc_gemm_qkv_rope(dg_model* m, const bf16* A, const void* W, int M, int n_seq, int np,
+                           int pos0, bf16* q, bf16* kc, bf16* vc, cudaStream_t st);
 dg_status tc_gemm_f32_rows(dg_model* m, const bf16* A, int a_rows, const void* W, float* out,
                            int M, int N, int K, cudaStream_t st);
 dg_status tc_gemm_add_residual(dg_model* m, const bf16* A, const void* W, float* x, int M, int N,

@@ -128,6 +128,7 @@ dg_status launch_dense(dg_model* m, const CUtensorMap& a, const CUtensorMap& b,
 }
 
 constexpr int DENSE_BN = 64, DENSE_MT = 2, DENSE_ST = 5, DUAL_ST = 4;
+constexpr int QKV_ST = 4;
 constexpr int LM_BN = 256, LM_ST = 3;
 constexpr int GU_ST = 4, DN_ST = 6;
 constexpr int GU8_ST = 3, DN8_ST = 5;
@@ -168,6 +169,8 @@ dg_status tc_prepare(dg_model* m) {
   DG_TRY(set_smem(tc_expert_kernel<true, GU_ST>, ExpertCfg<true, GU_ST>::SMEM));
   DG_TRY(set_smem(tc_expert_kernel<false, DN_ST>, ExpertCfg<false, DN_ST>::SMEM));
   DG_TRY(set_smem(tc_attn_kernel, AT_SMEM));
+  DG_TRY(set_smem(tc_dense_kernel<128, DENSE_MT, false, QKV_ST, EpiQkvRope>,
+                  DenseCfg<128, DENSE_MT, false, QKV_ST>::SMEM));
   DG_TRY(set_smem(tc_expert_f8_kernel<true, GU8_ST>, ExpertF8Cfg<true, GU8_ST>::SMEM));
   DG_TRY(set_smem(tc_expert_f8_kernel<false, DN8_ST>, ExpertF8Cfg<false, DN8_ST>::SMEM));
   cudaDeviceGetAttribute(&s->n_sm, cudaDevAttrMultiProcessorCount, m->device);
@@ -190,6 +193,27 @@ dg_status tc_gemm_store_f32(dg_model* m, const bf16* A, const void* W, float* ou
   DG_TRY(tmap(m, W, N, K, DENSE_BN, &b));
   return launch_dense<DENSE_BN, DENSE_MT, false, DENSE_ST>(m, a, b, b, M, N, K,
                                                            EpiStoreF32{out, N, N}, st);
+}
+
+dg_status tc_gemm_qkv_rope(dg_model* m, const bf16* A, const void* W, int M, int n_seq, int np,
+                           int pos0, bf16* q, bf16* kc, bf16* vc, cudaStream_t st) {
+  const dg_config& c = m->cfg;
+  const int N = (c.n_q_heads + 2 * c.n_kv_heads) * c.head_dim, K = c.d_model;
+  CUtensorMap a, b;
+  DG_TRY(tmap(m, A, m->ws.max_tok, K, 128, &a));
+  DG_TRY(tmap(m, W, N, K, 128, &b));
+  EpiQkvRope epi;
+  epi.q = q;
+  epi.kc = kc;
+  epi.vc = vc;
+  epi.rope = (const float*)m->ws.rope;
+  epi.max_pos = m->ws.max_pos;
+  epi.n_seq = n_seq;
+  epi.np = np;
+  epi.pos0 = pos0;
+  epi.Hq = c.n_q_heads;
+  epi.Hkv = c.n_kv_heads;
+  return launch_dense<128, DENSE_MT, false, QKV_ST>(m, a, b, b, M, N, K, epi, st);
 }
 
 dg_status tc_gemm_f32_rows(dg_model* m, const bf16* A, int a_rows, const void* W, float* out,
