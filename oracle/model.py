@@ -24,6 +24,14 @@ Precision: weights are read as their stored values (fp32 / bf16 / dequantised
 FP8) and widened to fp64; every activation and reduction is fp64.  Per-row
 entropies are rounded to fp32 at the end, which is the precision the sampler
 decides in.
+
+Storage variant (Weights(..., storage="bf16")): the same forward with the
+activations that a bf16 model keeps in memory rounded to bf16 where they are
+stored (normalised rows entering a projection, q / k / v after RoPE, the
+attention output, the SwiGLU hidden rows); residual stream, router and every
+sum stay fp64.  It measures how far bf16 storage alone moves the outputs of a
+workload (its sensitivity), from which the tolerances of the deep workloads are
+derived.
 """
 from __future__ import annotations
 
@@ -39,16 +47,35 @@ from synth.workloads import Workload
 # ----------------------------------------------------------------------------
 # weights
 # ----------------------------------------------------------------------------
+def round_bf16(a: np.ndarray) -> np.ndarray:
+    """Nearest bfloat16 value of fp64 values: 8 significant bits, ties to even.
+
+    a = m 2^e with 0.5 <= |m| < 1; m 2^8 rounded half-to-even to an integer keeps
+    8 significant bits (a carry to 256 gives the next power of two).  Exact in fp64;
+    the exponent range is not limited (the activations here are far from it).
+    """
+    m, e = np.frexp(np.asarray(a, dtype=np.float64))
+    return np.ldexp(np.round(m * 256.0), e - 8)
+
+
+def _keep(a: np.ndarray) -> np.ndarray:
+    return a
+
+
 class Weights:
     """Stored weight values as fp64 arrays, generated on demand from the seed.
 
     `keep_layers` caches every layer (tiny models); otherwise one layer at a
     time is held, so a 30-layer model never needs its full size in RAM.
+    `storage` = "fp64" (the oracle) or "bf16" (the storage variant).
     """
 
-    def __init__(self, w: Workload, keep_layers: bool = False):
+    def __init__(self, w: Workload, keep_layers: bool = False, storage: str = "fp64"):
+        if storage not in ("fp64", "bf16"):
+            raise ValueError(f"storage must be fp64 or bf16, not {storage!r}")
         self.w = w
         self.keep = keep_layers
+        self.store = round_bf16 if storage == "bf16" else _keep
         self._cache: dict[str, np.ndarray] = {}
 
     def _load(self, name, shape, start_row=0, n_rows=None) -> np.ndarray:
@@ -79,6 +106,7 @@ class LayerWeights:
     def __init__(self, ws: Weights, l: int):
         w = ws.w
         self.ws, self.l, self.w = ws, l, w
+        self.store = ws.store
         specs = dict(model_inputs.layer_specs(w, l))
         self.specs = specs
         qkv = ws.get(f"l{l}.wqkv", specs[f"l{l}.wqkv"])
@@ -155,9 +183,10 @@ def silu(z: np.ndarray) -> np.ndarray:
     return z / (1.0 + np.exp(-z))
 
 
-def swiglu(u: np.ndarray, wg: np.ndarray, wu: np.ndarray, wd: np.ndarray) -> np.ndarray:
-    """down(silu(gate u) * up u) for rows u [n, d]."""
-    return (silu(u @ wg.T) * (u @ wu.T)) @ wd.T
+def swiglu(u: np.ndarray, wg: np.ndarray, wu: np.ndarray, wd: np.ndarray,
+           store=_keep) -> np.ndarray:
+    """down(silu(gate u) * up u) for rows u [n, d] (hidden rows kept through `store`)."""
+    return store(silu(u @ wg.T) * (u @ wu.T)) @ wd.T
 
 
 def route(u: np.ndarray, router: np.ndarray, top_k: int):
@@ -180,15 +209,20 @@ def route(u: np.ndarray, router: np.ndarray, top_k: int):
 
 
 def moe(u: np.ndarray, lw: LayerWeights, top_k: int):
-    """Routed experts plus the shared expert (weight 1) on normalised rows u [n, d]."""
+    """Routed experts plus the shared expert (weight 1) on normalised rows u [n, d].
+
+    The router reads u itself; the expert inputs are u as stored (lw.store).
+    """
     idx, g, logits = route(u, lw.router, top_k)
-    y = swiglu(u, lw.sgate, lw.sup, lw.sdown)
+    st = lw.store
+    us = st(u)
+    y = swiglu(us, lw.sgate, lw.sup, lw.sdown, st)
     for e in range(lw.w.n_experts):
         rows, slot = np.nonzero(idx == e)
         if rows.size == 0:
             continue
         wg, wu, wd = lw.expert(e)
-        y[rows] += g[rows, slot][:, None] * swiglu(u[rows], wg, wu, wd)
+        y[rows] += g[rows, slot][:, None] * swiglu(us[rows], wg, wu, wd, st)
     return y, idx, g, logits
 
 
@@ -200,14 +234,15 @@ def decoder_layer(x, pos, lw: LayerWeights, kv_prev, allowed, w: Workload):
     """
     n = x.shape[0]
     H, Hk, h = w.n_q_heads, w.n_kv_heads, w.head_dim
-    xn = rmsnorm(x, w.rms_eps)
+    st = lw.store
+    xn = st(rmsnorm(x, w.rms_eps))
     q = (xn @ lw.wq.T).reshape(n, H, h)
     k = (xn @ lw.wk.T).reshape(n, Hk, h)
-    v = (xn @ lw.wv.T).reshape(n, Hk, h)
-    q, k = rope(q, pos, w.rope_base), rope(k, pos, w.rope_base)
+    v = st((xn @ lw.wv.T).reshape(n, Hk, h))
+    q, k = st(rope(q, pos, w.rope_base)), st(rope(k, pos, w.rope_base))
     K = np.concatenate([kv_prev[0], k], axis=0)
     V = np.concatenate([kv_prev[1], v], axis=0)
-    o = attention(q, K, V, allowed)
+    o = st(attention(q, K, V, allowed))
     x = x + o.reshape(n, H * h) @ lw.wo.T
     u = rmsnorm(x, w.rms_eps)
     y, idx, g, rlog = moe(u, lw, w.top_k)
@@ -275,7 +310,7 @@ def lm_head_stats(ws: Weights, x: np.ndarray, vocab_chunk: int = 16384, want_log
     optionally the logits [n, V].
     """
     w = ws.w
-    xn = rmsnorm(x, w.rms_eps)
+    xn = ws.store(rmsnorm(x, w.rms_eps))
     V = w.vocab
     logits = np.empty((x.shape[0], V))
     for c0 in range(0, V, vocab_chunk):
@@ -289,16 +324,20 @@ def lm_head_stats(ws: Weights, x: np.ndarray, vocab_chunk: int = 16384, want_log
 
 
 def entropy_stats(logits: np.ndarray):
-    """Per-row softmax entropy (nats), argmax, log-sum-exp and top-2 margin."""
+    """Per-row softmax entropy (nats), argmax, log-sum-exp, top-2 margin and sigma,
+    the standard deviation of the logits under the row's own softmax p (the
+    first-order gain of the entropy: dH = -Cov_p(l, dl), so |dH| <= sigma max|dl|)."""
     m = logits.max(axis=1, keepdims=True)
     lse = m + np.log(np.exp(logits - m).sum(axis=1, keepdims=True))
     logp = logits - lse
     p = np.exp(logp)
     H = -(p * logp).sum(axis=1)
+    mean = (p * logits).sum(axis=1, keepdims=True)
+    sigma = np.sqrt((p * (logits - mean) ** 2).sum(axis=1))
     am = logits.argmax(axis=1)
     top2 = np.partition(logits, -2, axis=1)[:, -2:]
     return {"H": H.astype(np.float32), "H64": H, "argmax": am.astype(np.int64),
-            "lse": lse[:, 0], "margin": top2[:, 1] - top2[:, 0]}
+            "lse": lse[:, 0], "margin": top2[:, 1] - top2[:, 0], "sigma": sigma}
 
 
 def denoise_forward(ws: Weights, kv_layers, canvas: np.ndarray, s: int, T: int, P: int,

@@ -1,15 +1,19 @@
 """Writes the oracle's expected outputs for the full-size workloads to tests/golden/.
 
 Calls only `oracle/` and `synth/` (never the CUDA path).  Usage:
-    python tests/golden/make_golden.py layer1-bf16 [full30-bf16 full30-b8-p8192:7 ...]
+    python tests/golden/make_golden.py layer1-bf16 [full30-bf16+s16 full30-b8-p8192:7 ...]
 Each file <workload>[-c<canvas>].npz holds, for one canvas of the workload's first forward
 (all [MASK], steps_left = T):
   H [C] fp32 entropies, H64 [C], argmax [C], margin [C] (top-1 minus top-2 logit),
-  lse [C]; logit_rows [R] row ids and logit_cols [Vs] vocab ids with
+  lse [C], sigma [C] (std of the logits under the row's softmax); logit_rows [R] row
+  ids and logit_cols [Vs] vocab ids with
   logits [R, Vs]; kv_last [L?, 2, Hkv, 8, h] post-RoPE keys / values of the last 8
   prompt positions of layers 0 and L-1; router margins per layer (min over rows of
   the gap between the k-th and (k+1)-th router logits); the sampler step's canvas,
   mask and count on these entropies.
+With the suffix "+s16" the file also holds the same outputs of the oracle's bf16
+storage variant (H_s16, argmax_s16, logits_s16, kv_last_s16): the sensitivity of the
+workload to bf16 activation storage, from which the deep workloads' tolerances follow.
 """
 from __future__ import annotations
 
@@ -29,7 +33,13 @@ from synth import model_inputs, workloads  # noqa: E402
 LOGIT_ROWS = [0, 1, 77, 128, 255]
 
 
-def make(name: str, canvas_index: int = 0):
+def _kv_last(w, st):
+    return np.stack([np.stack([st["kv"][l][0][-8:].transpose(1, 0, 2),
+                               st["kv"][l][1][-8:].transpose(1, 0, 2)])
+                     for l in sorted({0, w.n_layers - 1})])
+
+
+def make(name: str, canvas_index: int = 0, storage_variant: bool = False):
     """Oracle outputs of the first forward of canvas `canvas_index` of the workload."""
     w = workloads.get(name)
     t0 = time.time()
@@ -39,9 +49,13 @@ def make(name: str, canvas_index: int = 0):
     st = om.prefill_then_forward(ws, prompt, canvas, w.T, w.T, want_logits=True)
     cols = np.arange(0, w.vocab, max(1, w.vocab // 4096))
     rows = [r for r in LOGIT_ROWS if r < w.canvas]
-    kv_last = np.stack([np.stack([st["kv"][l][0][-8:].transpose(1, 0, 2),
-                                  st["kv"][l][1][-8:].transpose(1, 0, 2)])
-                        for l in sorted({0, w.n_layers - 1})])
+    kv_last = _kv_last(w, st)
+    extra = {}
+    if storage_variant:
+        ws16 = om.Weights(w, keep_layers=False, storage="bf16")
+        s16 = om.prefill_then_forward(ws16, prompt, canvas, w.T, w.T, want_logits=True)
+        extra = dict(H_s16=s16["H"], argmax_s16=s16["argmax"], kv_last_s16=_kv_last(w, s16),
+                     logits_s16=s16["logits"][rows][:, cols].astype(np.float64))
     rmarg = []
     for idx, g, rl in st["routes"]:
         srt = np.sort(rl, axis=1)[:, ::-1]
@@ -51,10 +65,11 @@ def make(name: str, canvas_index: int = 0):
     suffix = f"-c{canvas_index}" if canvas_index else ""
     out = os.path.join(HERE, f"{name}{suffix}.npz")
     np.savez_compressed(out, H=st["H"], H64=st["H64"], argmax=st["argmax"], margin=st["margin"],
-                        lse=st["lse"], logit_rows=np.array(rows), logit_cols=cols,
+                        lse=st["lse"], sigma=st["sigma"], logit_rows=np.array(rows),
+                        logit_cols=cols,
                         logits=st["logits"][rows][:, cols].astype(np.float64), kv_last=kv_last,
                         router_margin=np.array(rmarg), step_canvas=c2, step_mask=m2,
-                        step_n=np.array(n2), step=np.array(w.T))
+                        step_n=np.array(n2), step=np.array(w.T), **extra)
     print(f"{name}: wrote {out} in {time.time() - t0:.0f} s; H range "
           f"[{st['H'].min():.4f}, {st['H'].max():.4f}], min margin {st['margin'].min():.4g}, "
           f"min router gap {min(rmarg):.3g}, sampler n {n2}")
@@ -62,6 +77,8 @@ def make(name: str, canvas_index: int = 0):
 
 if __name__ == "__main__":
     # arguments: workload names, optionally "name:canvas" to pick a canvas of the batch
+    # and the suffix "+s16" for the bf16 storage variant as well
     for arg in sys.argv[1:] or ["layer1-bf16"]:
-        name, _, c = arg.partition(":")
-        make(name, int(c) if c else 0)
+        s16 = arg.endswith("+s16")
+        name, _, c = arg.removesuffix("+s16").partition(":")
+        make(name, int(c) if c else 0, storage_variant=s16)

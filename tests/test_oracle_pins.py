@@ -124,6 +124,7 @@ def test_timestep_embedding_pins():
 class _FakeLayer:
     def __init__(self, E, d, I, Is, w):
         self.w = w
+        self.store = lambda a: a   # the fp64 oracle keeps activations as computed
         self.router = rng.normal(size=(E, d))
         self.experts = [(rng.normal(size=(I, d)) * 0.3, rng.normal(size=(I, d)) * 0.3,
                          rng.normal(size=(d, I)) * 0.3) for _ in range(E)]
@@ -387,3 +388,61 @@ def test_tps_formula_reproduces_pages():
     # tokens per forward counts one extra forward between consecutive canvases
     assert metrics.tokens_per_forward([256, 256, 100], [12, 12, 5]) == 612 / (29 + 2)
     assert metrics.effective_steps([256, 100], [12, 4]) == (256 * 12 + 100 * 4) / 356
+
+
+# --------------------------------------------------------------- entropy gain and bf16 storage
+def test_entropy_sigma_two_point_and_first_order_gain():
+    """sigma = std of the logits under p: two-point closed form |a - b| sqrt(p (1 - p)),
+    zero for equal logits; and the entropy's first-order change is -Cov_p(l, dl)."""
+    a, b = 1.7, -0.4
+    st = model.entropy_stats(np.array([[a, b], [0.3, 0.3]]))
+    p = 1.0 / (1.0 + math.exp(b - a))
+    assert st["sigma"][0] == pytest.approx(abs(a - b) * math.sqrt(p * (1 - p)), rel=1e-12)
+    assert st["sigma"][1] == pytest.approx(0.0, abs=1e-15)
+    r = np.random.default_rng(5)
+    lg = r.normal(0, 3, (4, 300))
+    d = r.normal(0, 1, (4, 300))
+    delta = 1e-6
+    h0 = model.entropy_stats(lg)["H64"]
+    h1 = model.entropy_stats(lg + delta * d)["H64"]
+    p = scipy.special.softmax(lg, axis=1)
+    cov = (p * lg * d).sum(1) - (p * lg).sum(1) * (p * d).sum(1)
+    np.testing.assert_allclose((h1 - h0) / delta, -cov, rtol=1e-4, atol=1e-8)
+    sig = model.entropy_stats(lg)["sigma"]
+    assert np.all(np.abs(cov) <= sig * np.abs(d).max(1) * (1 + 1e-12))
+
+
+def test_round_bf16_ties_and_library():
+    """8 significant bits, ties to even; equals torch's fp32 -> bf16 rounding on fp32 values."""
+    import torch
+    f = model.round_bf16
+    assert f(np.array([1 + 2.0 ** -8]))[0] == 1.0                      # tie -> even (1.0)
+    assert f(np.array([1 + 3 * 2.0 ** -8]))[0] == 1 + 2.0 ** -6        # tie -> even (up)
+    assert f(np.array([1 + 2.0 ** -8 + 2.0 ** -30]))[0] == 1 + 2.0 ** -7
+    assert f(np.array([-3.0, 0.0, 255.5]))[:2].tolist() == [-3.0, 0.0]
+    assert f(np.array([255.5]))[0] == 256.0                            # carry into the exponent
+    x = np.random.default_rng(9).normal(0, 10, 20000).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(f(x.astype(np.float64)), ref)
+
+
+def test_bf16_storage_variant():
+    """storage="fp64" is the oracle itself; storage="bf16" keeps the cache keys/values
+    and entropies within bf16 distance of it, with every cached value bf16-exact."""
+    w = workloads.TINY_F32
+    prompt = np.arange(w.prompt_len) % w.vocab
+    c = np.full(w.canvas, w.mask_id)
+    ref = model.Weights(w, keep_layers=True)
+    same = model.Weights(w, keep_layers=True, storage="fp64")
+    s16 = model.Weights(w, keep_layers=True, storage="bf16")
+    kv_ref, kv_same, kv_16 = model.prefill(ref, prompt), model.prefill(same, prompt), model.prefill(s16, prompt)
+    for (k0, v0), (k1, v1), (k2, v2) in zip(kv_ref, kv_same, kv_16):
+        assert np.array_equal(k0, k1) and np.array_equal(v0, v1)
+        assert np.array_equal(model.round_bf16(k2), k2) and np.array_equal(model.round_bf16(v2), v2)
+        assert not np.array_equal(k0, k2)
+        assert np.abs(k2 - k0).max() <= 2.0 ** -6 * np.abs(k0).max()
+    h0 = model.denoise_forward(ref, kv_ref, c, w.T, w.T, w.prompt_len)["H64"]
+    h2 = model.denoise_forward(s16, kv_16, c, w.T, w.T, w.prompt_len)["H64"]
+    assert 0 < np.abs(h2 - h0).max() < 2e-2 * np.abs(h0).max()
+    with pytest.raises(ValueError):
+        model.Weights(w, storage="fp16")
