@@ -111,7 +111,8 @@ const char* dg_last_error(void);
 /* Validates the configuration and weight pointers, plans the kernels and
  * allocates the library's device workspace for max_batch canvases and prompts
  * up to max_prompt tokens, on the current CUDA device.  Synchronous.
- * Errors: DG_ERR_INVALID_ARG (null, non-positive or inconsistent sizes, C > 1024,
+ * Errors: DG_ERR_INVALID_ARG (null, non-positive or inconsistent sizes, d_model not a
+ * multiple of 8, C > 1024,
  * Hq not a multiple of Hkv, h odd), DG_ERR_UNSUPPORTED (a shape the tensor-core
  * kernels do not tile), DG_ERR_OOM, DG_ERR_CUDA. */
 dg_status dg_model_create(const dg_config* cfg, const dg_weights* w, dg_model** out);

@@ -141,6 +141,7 @@ template <class Path> static dg_status alloc_workspace(dg_model* m) {
   DG_TRY(ws_alloc_v<Acc>(ws, &ws.rgate, R));
   DG_TRY(ws_alloc_v<Acc>(ws, &ws.gate_of, R));
   DG_TRY(ws_alloc_v<Acc>(ws, &ws.inv_rms, T));
+  if constexpr (Path::kTensorCores) DG_TRY(ws_alloc_v<TA>(ws, &ws.u2, T * 2 * d));
   DG_TRY(ws_alloc_v<Acc>(ws, &ws.rlog, std::max<size_t>(4096, T) * c.n_experts));
   DG_TRY(ws_alloc(ws, &ws.counts, c.n_experts));
   DG_TRY(ws_alloc(ws, &ws.offsets, c.n_experts + 1));
@@ -167,7 +168,16 @@ template <class Path> static dg_status alloc_workspace(dg_model* m) {
   launch_pdl((rope_table_kernel), 256, 256, 0, cudaStream_t(0), 1, (double)c.rope_base, (int)h, ws.max_pos, ws.rope,
                                   sizeof(Acc) == 8 ? 1 : 0);
   DG_TRY(check_launch("rope table"));
-  if constexpr (Path::kTensorCores) DG_TRY(tc_prepare(m));
+  if constexpr (Path::kTensorCores) {
+    DG_TRY(tc_prepare(m));
+    DG_TRY_CUDA(cudaStreamCreateWithFlags(&m->side_stream, cudaStreamNonBlocking));
+    DG_TRY_CUDA(cudaEventCreateWithFlags(&m->fork_ev, cudaEventDisableTiming));
+    DG_TRY_CUDA(cudaEventCreateWithFlags(&m->join_ev, cudaEventDisableTiming));
+  }
+  const size_t perm_smem = (size_t)33 * c.n_experts * sizeof(int);
+  if (perm_smem > 48 * 1024)
+    DG_TRY_CUDA(cudaFuncSetAttribute(moe_permute_kernel<Acc>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)perm_smem));
   DG_TRY_CUDA(cudaDeviceSynchronize());
   return DG_OK;
 }
@@ -204,7 +214,7 @@ template <class Path> struct Runner {
 
   void rmsnorm(int n) {
     launch_pdl((rmsnorm_kernel<TR, TA, Acc>), n, 256, 0, st, 1, x(), xn(), n, c.d_model, c.rms_eps,
-               (Acc*)nullptr);
+               (Acc*)nullptr, (TA*)nullptr);
     ++m->launches;
   }
 
@@ -218,6 +228,7 @@ template <class Path> struct Runner {
   // One decoder layer on n tokens = B_ * n_seq rows at positions pos0 + i.
   // Segment A (the cached window, denoise only): keys [L, B, Hkv, WpA, h] and transposed
   // values [L, B, Hkv, h, WpA] of `kv`, nA valid keys at positions kposA...
+  // xn holds RMSNorm(x) on entry for l > 0 (the previous layer's combine writes it).
   dg_status layer(int l, int n, int B_, int n_seq, int pos0, const dg_kv* kv, bool causal,
                   int32_t* load) {
     const int nA = kv ? kv->W : 0, kposA = kv ? kv->P - kv->W : 0, WpA = kv ? kv->Wp : 0;
@@ -225,7 +236,7 @@ template <class Path> struct Runner {
     const dg_layer_weights& L = m->layers[l];
     const int d = c.d_model, h = c.head_dim, Hq = c.n_q_heads, Hkv = c.n_kv_heads;
     const int qkv_n = (Hq + 2 * Hkv) * h;
-    rmsnorm(n);
+    if (l == 0) rmsnorm(n);
     bool fused_rope = false;
     {
       ProfScope ps(m, DG_KIND_DENSE, st);
@@ -293,10 +304,30 @@ template <class Path> struct Runner {
     const int d = c.d_model, E = c.n_experts, k = c.top_k, I = c.expert_inter;
     const int Is = c.shared_inter;
     const int n_ent = n * k;
-    // u = RMSNorm(x) after attention (bf16 copy for the expert GEMMs, 1/rms for the router)
-    launch_pdl((rmsnorm_kernel<TR, TA, Acc>), n, 256, 0, st, 1, x(), xn(), n, d, c.rms_eps, (Acc*)ws.inv_rms);
+    // u = RMSNorm(x) after attention (bf16 copy for the expert GEMMs, 1/rms for the
+    // CUDA-core router, the two-term split for the tensor-core router)
+    bool tc_router = false;
+    if constexpr (Path::kTensorCores) tc_router = E <= 128 && k <= 8 && d % 64 == 0;
+    launch_pdl((rmsnorm_kernel<TR, TA, Acc>), n, 256, 0, st, 1, x(), xn(), n, d, c.rms_eps,
+               (Acc*)ws.inv_rms, tc_router ? (TA*)ws.u2 : (TA*)nullptr);
     ++m->launches;
-    {
+    if constexpr (Path::kTensorCores) {
+      // shared expert on the side stream, concurrent with routing and the routed experts
+      cudaStream_t side = m->side_stream;
+      DG_TRY_CUDA(cudaEventRecord(m->fork_ev, st));
+      DG_TRY_CUDA(cudaStreamWaitEvent(side, m->fork_ev, 0));
+      {
+        ProfScope ps(m, DG_KIND_DENSE, side);
+        DG_TRY(tc_gemm_swiglu(m, xn(), L.sgate, L.sup, (TA*)ws.sh, n, Is, d, side));
+        DG_TRY(tc_gemm_store_f32(m, (const TA*)ws.sh, L.sdown, (float*)ws.ys, n, d, Is, side));
+      }
+      DG_TRY_CUDA(cudaEventRecord(m->join_ev, side));
+      if (tc_router) {
+        ProfScope ps(m, DG_KIND_DENSE, st);
+        DG_TRY(tc_router_topk(m, (const bf16*)ws.u2, L.router, n, ws.ridx, (float*)ws.rgate, st));
+      }
+    }
+    if (!tc_router) {
       const int splits = std::max(1, std::min(16, 4096 / n));
       const int kps = ceil_div(ceil_div(d, splits), 32) * 32;
       const int ks = ceil_div(d, kps);
@@ -305,26 +336,25 @@ template <class Path> struct Runner {
                                                               kps, (Acc*)ws.rlog);
       ++m->launches;
       if (E <= 32)
-        launch_pdl((router_topk_kernel<Acc, 1>), ceil_div(n, 4), 128, 0, st, 1, 
-            (const Acc*)ws.rlog, ks, (const Acc*)ws.inv_rms, n, E, k, ws.ridx, (Acc*)ws.rgate, load);
+        launch_pdl((router_topk_kernel<Acc, 1>), ceil_div(n, 4), 128, 0, st, 1,
+            (const Acc*)ws.rlog, ks, (const Acc*)ws.inv_rms, n, E, k, ws.ridx, (Acc*)ws.rgate,
+            (int32_t*)nullptr);
       else if (E <= 128)
-        launch_pdl((router_topk_kernel<Acc, 4>), ceil_div(n, 4), 128, 0, st, 1, 
-            (const Acc*)ws.rlog, ks, (const Acc*)ws.inv_rms, n, E, k, ws.ridx, (Acc*)ws.rgate, load);
+        launch_pdl((router_topk_kernel<Acc, 4>), ceil_div(n, 4), 128, 0, st, 1,
+            (const Acc*)ws.rlog, ks, (const Acc*)ws.inv_rms, n, E, k, ws.ridx, (Acc*)ws.rgate,
+            (int32_t*)nullptr);
       else
-        launch_pdl((router_topk_kernel<Acc, 32>), ceil_div(n, 4), 128, 0, st, 1, 
-            (const Acc*)ws.rlog, ks, (const Acc*)ws.inv_rms, n, E, k, ws.ridx, (Acc*)ws.rgate, load);
+        launch_pdl((router_topk_kernel<Acc, 32>), ceil_div(n, 4), 128, 0, st, 1,
+            (const Acc*)ws.rlog, ks, (const Acc*)ws.inv_rms, n, E, k, ws.ridx, (Acc*)ws.rgate,
+            (int32_t*)nullptr);
       ++m->launches;
     }
-    launch_pdl((moe_rank_kernel), E, 256, 0, st, 1, ws.ridx, n_ent, ws.rank, ws.counts);
-    ++m->launches;
     int bm = SG_BM;
     if constexpr (Path::kTensorCores) bm = tc_group_rows();
-    launch_pdl((moe_offsets_kernel), 1, 1024, 0, st, 1, ws.counts, E, bm, ws.offsets, ws.tile_e, ws.tile_m0,
-                                           ws.n_tiles, ws.max_tiles, ws.units);
-    ++m->launches;
-    launch_pdl((moe_scatter_kernel<Acc>), ceil_div(n_ent, 256), 256, 0, st, 1, 
-        ws.ridx, (const Acc*)ws.rgate, ws.rank, ws.offsets, n_ent, k, ws.row_of, ws.tok_of,
-        (Acc*)ws.gate_of);
+    launch_pdl((moe_permute_kernel<Acc>), 1, 1024, (size_t)33 * E * sizeof(int), st, 1,
+               (const int32_t*)ws.ridx, (const Acc*)ws.rgate, n_ent, k, E, bm, ws.rank, ws.offsets,
+               ws.tile_e, ws.tile_m0, ws.n_tiles, ws.max_tiles, ws.units, load, ws.row_of,
+               ws.tok_of, (Acc*)ws.gate_of);
     ++m->launches;
     launch_pdl((gather_rows_kernel<TA>), n_ent, 256, 0, st, 1, xn(), ws.tok_of, ws.offsets + E, d,
                                                   (TA*)ws.up);
@@ -336,9 +366,7 @@ template <class Path> struct Runner {
         DG_TRY(tc_moe_gate_up(m, l, (const TA*)ws.up, (TA*)ws.hb, grid_y, st));
         DG_TRY(tc_moe_down(m, l, (const TA*)ws.hb, (float*)ws.yb, grid_y, st));
       }
-      ProfScope ps(m, DG_KIND_DENSE, st);
-      DG_TRY(tc_gemm_swiglu(m, xn(), L.sgate, L.sup, (TA*)ws.sh, n, Is, d, st));
-      DG_TRY(tc_gemm_store_f32(m, (const TA*)ws.sh, L.sdown, (float*)ws.ys, n, d, Is, st));
+      DG_TRY_CUDA(cudaStreamWaitEvent(st, m->join_ev, 0));  // shared expert done
     } else {
       GroupInfo g;
       g.tile_e = ws.tile_e;
@@ -360,8 +388,10 @@ template <class Path> struct Runner {
                                           EpiSwiglu<TA, Acc>{(TA*)ws.sh, Is}, st, &m->launches);
       dense((const TA*)ws.sh, Is, L.sdown, d, Is, n, EpiStore<Acc, Acc>{(Acc*)ws.ys, d});
     }
-    launch_pdl((moe_combine_kernel<TR, Acc, Acc>), dim3(n, ceil_div(d, 128)), 128, 0, st, 1, x(), (const Acc*)ws.ys,
-                                                        (const Acc*)ws.yb, ws.row_of, n, d, k);
+    // residual update fused with the next RMSNorm (next layer's input or the LM head's)
+    launch_pdl((moe_combine_norm_kernel<TR, TA, Acc, Acc>), n, 256, 0, st, 1, x(),
+               (const Acc*)ws.ys, (const Acc*)ws.yb, (const int32_t*)ws.row_of, n, d, k,
+               c.rms_eps, xn());
     ++m->launches;
     return check_launch("moe");
   }
@@ -425,9 +455,12 @@ template <class Path> struct Runner {
       DG_TRY_CUDA(cudaMemsetAsync(ws.vc, 0, (size_t)B * c.n_kv_heads * c.head_dim * Cp * sizeof(TKV), st));
     for (int l = 0; l < c.n_layers; ++l)
       DG_TRY(layer(l, n, B, C, kv->P, kv, false, load ? load + (size_t)l * c.n_experts : nullptr));
-    if (hidden) launch_pdl((to_f32_kernel<TR>), ceil_div((long)n * d, 256), 256, 0, st, 1, x(), hidden, (long)n * d);
-    ++m->launches;
-    rmsnorm(n);
+    if (hidden) {
+      launch_pdl((to_f32_kernel<TR>), ceil_div((long)n * d, 256), 256, 0, st, 1, x(), hidden,
+                 (long)n * d);
+      ++m->launches;
+    }
+    // xn = RMSNorm(x): written by the last layer's combine
     ProfScope ps(m, DG_KIND_LMHEAD, st);
     bool done = false;
     if constexpr (Path::kTensorCores) {
@@ -442,7 +475,7 @@ template <class Path> struct Runner {
                                                            c.vocab, d, c.logit_scale,
                                                            (Acc*)ws.lm_part, logits);
       ++m->launches;
-      launch_pdl((lm_merge_kernel<Acc>), ceil_div(n, 4), 128, 0, st, 1, (const Acc*)ws.lm_part, ws.n_vtiles,
+      launch_pdl((lm_merge_kernel<Acc>), n, 128, 0, st, 1, (const Acc*)ws.lm_part, ws.n_vtiles,
                                                           n, ent, amax);
       ++m->launches;
     }
@@ -529,7 +562,7 @@ dg_status dg_model_create(const dg_config* cfg, const dg_weights* w, dg_model** 
   DG_REQUIRE(cfg && w && out, "null argument");
   *out = nullptr;
   const dg_config& c = *cfg;
-  DG_REQUIRE(c.n_layers >= 1 && c.d_model >= 2 && c.d_model % 2 == 0, "bad n_layers/d_model");
+  DG_REQUIRE(c.n_layers >= 1 && c.d_model >= 8 && c.d_model % 8 == 0, "bad n_layers/d_model (d_model: a multiple of 8)");
   DG_REQUIRE(c.n_q_heads >= 1 && c.n_kv_heads >= 1 && c.n_q_heads % c.n_kv_heads == 0,
              "n_q_heads must be a positive multiple of n_kv_heads");
   DG_REQUIRE(c.head_dim >= 2 && c.head_dim % 2 == 0 && c.head_dim <= 128,
@@ -585,6 +618,9 @@ dg_status dg_model_destroy(dg_model* m) {
   for (dg_kv* kv : m->kvs) kv->m = nullptr;  // caches outlive the model only to be destroyed
   m->kvs.clear();
   if (m->cap_stream) cudaStreamDestroy(m->cap_stream);
+  if (m->side_stream) cudaStreamDestroy(m->side_stream);
+  if (m->fork_ev) cudaEventDestroy(m->fork_ev);
+  if (m->join_ev) cudaEventDestroy(m->join_ev);
   for (int k = 0; k < DG_KIND_COUNT; ++k)
     for (auto& e : m->prof[k]) {
       cudaEventDestroy(e.first);

@@ -91,6 +91,7 @@ struct Workspace {
   int32_t *ridx = nullptr, *rank = nullptr, *row_of = nullptr, *tok_of = nullptr;
   void *rgate = nullptr, *gate_of = nullptr;
   void *inv_rms = nullptr, *rlog = nullptr;  // per-row 1/rms; split-K router partials
+  void* u2 = nullptr;  // [rows, 2 d] two-term split of the normalised rows (tensor-core router)
   int32_t *counts = nullptr, *offsets = nullptr, *tile_e = nullptr, *tile_m0 = nullptr,
           *n_tiles = nullptr;
   void *up = nullptr, *hb = nullptr, *yb = nullptr; // routed rows
@@ -147,6 +148,10 @@ struct dg_model {
   std::vector<dg::BlockGraph*> graphs;
   dg::BlockGraph* capture = nullptr;  // graph being captured (events go there)
   cudaStream_t cap_stream = nullptr;  // private stream used only for capturing
+  // second stream for the shared expert, forked after the MoE RMSNorm and joined
+  // before the combine (concurrent graph branches when captured)
+  cudaStream_t side_stream = nullptr;
+  cudaEvent_t fork_ev = nullptr, join_ev = nullptr;
   long long last_body_launches = 0;   // kernels per forward of the last replayed loop graph
   std::vector<dg_kv*> kvs;            // live KV caches created from this model
 };

@@ -49,10 +49,15 @@ __global__ void embed_kernel(const int32_t* __restrict__ ids, const TW* __restri
 
 // ---------------------------------------------------------------------------
 // RMSNorm, gain 1: y = x / sqrt(mean(x^2) + eps)
+// Optional u2 [n, 2d]: the two-term split of u = x / rms into y (first d
+// columns) and lo = narrow(u - y) (last d columns); y + lo carries u to about
+// twice the precision of TA, so that a TA x TA contraction of [y | lo] against
+// [w | w] reproduces u . w at nearly fp32 accuracy (router logits on tensor cores).
 // ---------------------------------------------------------------------------
 template <class TR, class TA, class Acc>
 __global__ void rmsnorm_kernel(const TR* __restrict__ x, TA* __restrict__ y, int n, int d,
-                               float eps, Acc* __restrict__ inv_out = nullptr) {
+                               float eps, Acc* __restrict__ inv_out = nullptr,
+                               TA* __restrict__ u2 = nullptr) {
   pdl_enter();
   __shared__ Acc red[32];
   const int t = blockIdx.x;
@@ -66,8 +71,15 @@ __global__ void rmsnorm_kernel(const TR* __restrict__ x, TA* __restrict__ y, int
   ss = block_sum(ss, red);
   const Acc inv = Acc(1) / dsqrt(ss / (Acc)d + (Acc)eps);
   if (inv_out && threadIdx.x == 0) inv_out[t] = inv;
-  for (int c = threadIdx.x; c < d; c += blockDim.x)
-    y[(size_t)t * d + c] = narrow<TA>((Acc)widen(r[c]) * inv);
+  for (int c = threadIdx.x; c < d; c += blockDim.x) {
+    const Acc u = (Acc)widen(r[c]) * inv;
+    const TA hi = narrow<TA>(u);
+    y[(size_t)t * d + c] = hi;
+    if (u2) {
+      u2[(size_t)t * 2 * d + c] = hi;
+      u2[(size_t)t * 2 * d + d + c] = narrow<TA>(u - (Acc)widen(hi));
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -526,6 +538,91 @@ static __global__ void __launch_bounds__(1024)
       }
 }
 
+// The whole permutation in one block of 1024 threads (E <= 1024): ranks by
+// warp-level match + per-(warp, expert) counts scanned in warp order (entry
+// order is kept within an expert), counts, offsets, the tile table, the
+// streamed-expert counter, per-expert load, and the scatter of (row, token,
+// gate).  Dynamic shared memory: (32 + 1) * E ints.
+template <class Acc>
+__global__ void __launch_bounds__(1024)
+    moe_permute_kernel(const int32_t* __restrict__ idx, const Acc* __restrict__ gate,
+                       int n_entries, int top_k, int E, int bm, int32_t* __restrict__ rank,
+                       int32_t* __restrict__ offsets, int32_t* __restrict__ tile_e,
+                       int32_t* __restrict__ tile_m0, int32_t* __restrict__ n_tiles,
+                       int max_tiles, unsigned long long* __restrict__ used,
+                       int32_t* __restrict__ load, int32_t* __restrict__ row_of,
+                       int32_t* __restrict__ tok_of, Acc* __restrict__ gate_of) {
+  pdl_enter();
+  extern __shared__ int psm[];
+  int* hist = psm;            // [32][E]: counts, then exclusive offsets per warp
+  int* carry = psm + 32 * E;  // [E]: entries of each expert in earlier chunks
+  __shared__ int sc[1024], stl[1024];
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  for (int e = tid; e < E; e += blockDim.x) carry[e] = 0;
+  for (int base = 0; base < n_entries; base += blockDim.x) {
+    for (int i = tid; i < 32 * E; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    const int j = base + tid;
+    const bool valid = j < n_entries;
+    const int e = valid ? idx[j] : -1;
+    const unsigned same = __match_any_sync(0xffffffffu, e);
+    const int before = __popc(same & ((1u << lane) - 1u));
+    if (valid && before == 0) hist[w * E + e] = __popc(same);
+    __syncthreads();
+    for (int e2 = tid; e2 < E; e2 += blockDim.x) {
+      int s = carry[e2];
+      for (int w2 = 0; w2 < 32; ++w2) {
+        const int c = hist[w2 * E + e2];
+        hist[w2 * E + e2] = s;
+        s += c;
+      }
+      carry[e2] = s;
+    }
+    __syncthreads();
+    if (valid) rank[j] = hist[w * E + e] + before;
+    __syncthreads();
+  }
+  // counts -> offsets and tile table (inclusive scans over 1024 slots)
+  const int e = tid;
+  const int c = e < E ? carry[e] : 0;
+  const unsigned bal = __ballot_sync(0xffffffffu, c > 0);
+  if (used && lane == 0 && bal) atomicAdd(used, (unsigned long long)__popc(bal));
+  if (load && e < E) load[e] += c;
+  const int nt = (c + bm - 1) / bm;
+  sc[e] = c;
+  stl[e] = nt;
+  __syncthreads();
+  for (int off = 1; off < 1024; off <<= 1) {
+    const int a = e >= off ? sc[e - off] : 0, b = e >= off ? stl[e - off] : 0;
+    __syncthreads();
+    sc[e] += a;
+    stl[e] += b;
+    __syncthreads();
+  }
+  const int off_e = sc[e] - c, t_e = stl[e] - nt;
+  if (e < E) {
+    offsets[e] = off_e;
+    carry[e] = off_e;
+  }
+  if (e == E - 1) {
+    offsets[E] = off_e + c;
+    *n_tiles = min(t_e + nt, max_tiles);
+  }
+  if (e < E)
+    for (int r = 0; r < nt; ++r)
+      if (t_e + r < max_tiles) {
+        tile_e[t_e + r] = e;
+        tile_m0[t_e + r] = off_e + r * bm;
+      }
+  __syncthreads();
+  for (int j = tid; j < n_entries; j += blockDim.x) {
+    const int pos = carry[idx[j]] + rank[j];
+    row_of[j] = pos;
+    tok_of[pos] = j / top_k;
+    gate_of[pos] = gate[j];
+  }
+}
+
 template <class Acc>
 __global__ void moe_scatter_kernel(const int32_t* __restrict__ idx, const Acc* __restrict__ gate,
                                    const int32_t* __restrict__ rank,
@@ -571,6 +668,56 @@ __global__ void moe_combine_kernel(TR* __restrict__ x, const TY* __restrict__ ys
     TR* p = x + (size_t)t * d + c;
     *p = narrow<TR>((Acc)widen(*p) + y);
   }
+}
+
+// Combine fused with the next RMSNorm: x[t] += ys[t] + sum over slots of
+// yb[row_of[t * k + slot]] (slot order fixed), then y[t] = RMSNorm(x[t]).
+// One block per token; each thread owns 8 consecutive columns (d % 8 == 0) and
+// issues the loads of all slots before summing.
+template <class TR, class TA, class TY, class Acc>
+__global__ void moe_combine_norm_kernel(TR* __restrict__ x, const TY* __restrict__ ys,
+                                        const TY* __restrict__ yb,
+                                        const int32_t* __restrict__ row_of, int n_tok, int d,
+                                        int top_k, float eps, TA* __restrict__ y) {
+  pdl_enter();
+  constexpr int KB = 8;  // slots loaded together
+  __shared__ Acc red[32];
+  __shared__ int rows[64];
+  const int t = blockIdx.x;
+  if (t >= n_tok) return;
+  for (int k = threadIdx.x; k < top_k; k += blockDim.x) rows[k] = row_of[(size_t)t * top_k + k];
+  __syncthreads();
+  TR* xr = x + (size_t)t * d;
+  Acc ss = 0;
+  for (int c0 = threadIdx.x * 8; c0 < d; c0 += blockDim.x * 8) {
+    Acc v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = (Acc)widen(ys[(size_t)t * d + c0 + j]);
+    for (int k0 = 0; k0 < top_k; k0 += KB) {
+      TY u[KB][8];
+#pragma unroll
+      for (int k = 0; k < KB; ++k)
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          u[k][j] = k0 + k < top_k ? yb[(size_t)rows[k0 + k] * d + c0 + j] : TY(0);
+#pragma unroll
+      for (int k = 0; k < KB; ++k)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] += (Acc)widen(u[k][j]);
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const TR nx = narrow<TR>((Acc)widen(xr[c0 + j]) + v[j]);
+      xr[c0 + j] = nx;
+      const Acc a = (Acc)widen(nx);
+      ss += a * a;
+    }
+  }
+  ss = block_sum(ss, red);
+  const Acc inv = Acc(1) / dsqrt(ss / (Acc)d + (Acc)eps);
+  for (int c0 = threadIdx.x * 8; c0 < d; c0 += blockDim.x * 8)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) y[(size_t)t * d + c0 + j] = narrow<TA>((Acc)widen(xr[c0 + j]) * inv);
 }
 
 // ---------------------------------------------------------------------------
@@ -678,43 +825,98 @@ __global__ void __launch_bounds__(256)
 //   H = log S - (1/S) sum e^(m_i - M) (u_i + (m_i - M) s_i)   (clamped at 0),
 //   argmax = the id of the first tile (lowest vocab) attaining M.
 template <class Acc>
-__global__ void lm_merge_kernel(const Acc* __restrict__ part, int n_vt, int n_rows,
-                                float* __restrict__ H, int32_t* __restrict__ amax) {
+__global__ void __launch_bounds__(128)
+    lm_merge_kernel(const Acc* __restrict__ part, int n_vt, int n_rows, float* __restrict__ H,
+                    int32_t* __restrict__ amax) {
+  // one block per row; the tiles are split over the threads, each thread merges
+  // its tiles online (running max M_t; S and U rescaled when M_t rises), then the
+  // block merges the threads in a fixed order
   pdl_enter();
-  const int lane = threadIdx.x & 31;
-  const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  __shared__ Acc sm_m[128], sm_s[128], sm_u[128], sm_i[128];
+  const int r = blockIdx.x, tid = threadIdx.x;
   if (r >= n_rows) return;
-  Acc M = -INFINITY;
-  Acc best_id = 0;
-  for (int i = lane; i < n_vt; i += 32) {
-    const Acc* p = part + ((size_t)i * n_rows + r) * 4;
-    if (p[0] > M) {
-      M = p[0];
-      best_id = p[3];
+  Acc M = -INFINITY, S = 0, U = 0, id = 0;
+  for (int i0 = tid; i0 < n_vt; i0 += 4 * blockDim.x) {
+    Acc pm[4], ps[4], pu[4], pi[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {  // independent loads first
+      const int i = i0 + q * blockDim.x;
+      if (i < n_vt) {
+        const Acc* p = part + ((size_t)i * n_rows + r) * 4;
+        pm[q] = p[0];
+        ps[q] = p[1];
+        pu[q] = p[2];
+        pi[q] = p[3];
+      } else {
+        pm[q] = -INFINITY;
+        ps[q] = pu[q] = pi[q] = 0;
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (!(pm[q] > -INFINITY)) continue;
+      if (pm[q] > M) {  // tiles come in increasing id order per thread: ties keep the first
+        const Acc w = dexp(M - pm[q]);
+        U = w * (U + (M - pm[q]) * S);
+        S = w * S;
+        if (!(M > -INFINITY)) U = S = 0;
+        M = pm[q];
+        id = pi[q];
+      }
+      const Acc w = dexp(pm[q] - M);
+      S += ps[q] * w;
+      U += w * (pu[q] + (pm[q] - M) * ps[q]);
     }
   }
-  for (int off = 16; off > 0; off >>= 1) {
-    const Acc om = __shfl_xor_sync(0xffffffffu, M, off);
-    const Acc oi = __shfl_xor_sync(0xffffffffu, best_id, off);
-    if (om > M || (om == M && oi < best_id)) {
-      M = om;
-      best_id = oi;
+  sm_m[tid] = M;
+  sm_s[tid] = S;
+  sm_u[tid] = U;
+  sm_i[tid] = id;
+  __syncthreads();
+  if (tid < 32) {
+    // lane l merges threads l, l + 32, ... in order, then a fixed butterfly
+    Acc m2 = -INFINITY, s2 = 0, u2 = 0, i2 = 0;
+    for (int t = tid; t < blockDim.x; t += 32) {
+      const Acc mt = sm_m[t];
+      if (!(mt > -INFINITY)) continue;
+      if (mt > m2 || (mt == m2 && sm_i[t] < i2)) {
+        if (mt > m2) {
+          const Acc w = dexp(m2 - mt);
+          u2 = (m2 > -INFINITY) ? w * (u2 + (m2 - mt) * s2) : Acc(0);
+          s2 = (m2 > -INFINITY) ? w * s2 : Acc(0);
+          m2 = mt;
+        }
+        i2 = sm_i[t];
+      }
+      const Acc w = dexp(mt - m2);
+      s2 += sm_s[t] * w;
+      u2 += w * (sm_u[t] + (mt - m2) * sm_s[t]);
     }
-  }
-  Acc S = 0, U = 0;
-  for (int i = lane; i < n_vt; i += 32) {
-    const Acc* p = part + ((size_t)i * n_rows + r) * 4;
-    const Acc w = dexp(p[0] - M);
-    S += p[1] * w;
-    U += w * (p[2] + (p[0] - M) * p[1]);
-  }
-  S = warp_sum(S);
-  U = warp_sum(U);
-  if (lane == 0) {
-    Acc h = dlog(S) - U / S;
-    if (!(h > Acc(0))) h = 0;
-    H[r] = (float)h;
-    amax[r] = (int32_t)best_id;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const Acc om = __shfl_xor_sync(0xffffffffu, m2, off);
+      const Acc os = __shfl_xor_sync(0xffffffffu, s2, off);
+      const Acc ou = __shfl_xor_sync(0xffffffffu, u2, off);
+      const Acc oi = __shfl_xor_sync(0xffffffffu, i2, off);
+      const Acc mm = om > m2 ? om : m2;
+      if (mm > -INFINITY) {
+        const Acc wa = dexp(m2 - mm), wb = dexp(om - mm);
+        const Acc sa = m2 > -INFINITY ? s2 : Acc(0), sb = om > -INFINITY ? os : Acc(0);
+        const Acc ua = m2 > -INFINITY ? wa * (u2 + (m2 - mm) * s2) : Acc(0);
+        const Acc ub = om > -INFINITY ? wb * (ou + (om - mm) * os) : Acc(0);
+        const Acc ni = (om > m2 || (om == m2 && oi < i2)) ? oi : i2;
+        s2 = wa * sa + wb * sb;
+        u2 = ua + ub;
+        i2 = ni;
+        m2 = mm;
+      }
+    }
+    if (tid == 0) {
+      Acc h = dlog(s2) - u2 / s2;
+      if (!(h > Acc(0))) h = 0;
+      H[r] = (float)h;
+      amax[r] = (int32_t)i2;
+    }
   }
 }
 

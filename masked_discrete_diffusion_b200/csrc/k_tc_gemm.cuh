@@ -38,129 +38,204 @@ template <int COLS> struct TmemCols {
 };
 
 // ---------------------------------------------------------------------------
-// epilogues of the dense kernel: run(row, valid, n0, ld) with ld(acc, chunk, v)
-// loading 32 fp32 columns of accumulator `acc` (0, or 1 for the second weight).
+// Epilogues of the dense kernel.
+//
+// Staged epilogues (kStaged): the kernel stages the fp32 accumulator tile in
+// shared memory, sums the split-K partials of the cluster there in a fixed order
+// and hands the result over with lane = column, so that every store of a warp
+// covers consecutive columns:
+//   col4(row, col, v, u): four consecutive elements from col (a multiple of 4;
+//   u: the second weight's accumulator, DUAL);
+//   warp_rows<NQ, RB>(row0, M, n0, v, lane) (kWarpRows): RB whole rows, lane l
+//   holding columns n0 + l + 32 q.
+// Direct epilogues (!kStaged) read TMEM rows themselves: run(row, valid, n0, ld)
+// with ld(acc, chunk, v) loading 32 fp32 columns of one row; never split.
 // ---------------------------------------------------------------------------
-// Chunk epilogues: chunk(row, col, v, u) consumes 32 consecutive columns of one row
-// (v: the accumulator, u: the second weight's accumulator for dual GEMMs).
-template <class Derived, bool DUAL>
-struct EpiChunked {
-  static constexpr bool kChunked = true, kRowWise = false;
-  template <int NCH, class Ld>
-  __device__ void run(int row, bool valid, int n0, Ld&& ld) const {
-#pragma unroll 1
-    for (int c = 0; c < NCH; ++c) {
-      float v[32], u[32];
-      ld(0, c, v);
-      if (DUAL) ld(1, c, u);
-      static_cast<const Derived*>(this)->chunk(row, valid, n0 + c * 32, v, u);
-    }
-  }
-};
-
-struct EpiStoreF32 : EpiChunked<EpiStoreF32, false> {
+struct EpiStoreF32 {
+  static constexpr bool kStaged = true, kWarpRows = false;
   float* out;
   int ldo, N;
   EpiStoreF32(float* o, int l, int n) : out(o), ldo(l), N(n) {}
-  __device__ void chunk(int row, bool valid, int col, const float* v, const float*) const {
-    if (!valid || col >= N) return;
-    float4* p = reinterpret_cast<float4*>(out + (size_t)row * ldo + col);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) p[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+  __device__ void col4(int row, int c, float4 v, float4) const {
+    float* p = out + (size_t)row * ldo + c;
+    if (c + 4 <= N) {
+      *reinterpret_cast<float4*>(p) = v;
+    } else {
+      const float a[4] = {v.x, v.y, v.z, v.w};
+      for (int j = 0; j < 4 && c + j < N; ++j) p[j] = a[j];
+    }
   }
 };
 
-struct EpiAddF32 : EpiChunked<EpiAddF32, false> {
+struct EpiAddF32 {
+  static constexpr bool kStaged = true, kWarpRows = false;
   float* out;
   int ldo, N;
   EpiAddF32(float* o, int l, int n) : out(o), ldo(l), N(n) {}
-  __device__ void chunk(int row, bool valid, int col, const float* v, const float*) const {
-    if (!valid || col >= N) return;
-    float4* p = reinterpret_cast<float4*>(out + (size_t)row * ldo + col);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      float4 o = p[j];
-      o.x += v[4 * j];
-      o.y += v[4 * j + 1];
-      o.z += v[4 * j + 2];
-      o.w += v[4 * j + 3];
-      p[j] = o;
+  __device__ void col4(int row, int c, float4 v, float4) const {
+    float* p = out + (size_t)row * ldo + c;
+    if (c + 4 <= N) {
+      float4 o = *reinterpret_cast<float4*>(p);
+      o.x += v.x;
+      o.y += v.y;
+      o.z += v.z;
+      o.w += v.w;
+      *reinterpret_cast<float4*>(p) = o;
+    } else {
+      const float a[4] = {v.x, v.y, v.z, v.w};
+      for (int j = 0; j < 4 && c + j < N; ++j) p[j] += a[j];
     }
   }
 };
 
-struct EpiSwigluBf16 : EpiChunked<EpiSwigluBf16, true> {
+struct EpiSwigluBf16 {
+  static constexpr bool kStaged = true, kWarpRows = false;
   bf16* out;
   int ldo, N;
   EpiSwigluBf16(bf16* o, int l, int n) : out(o), ldo(l), N(n) {}
-  __device__ void chunk(int row, bool valid, int col, const float* g, const float* u) const {
-    if (!valid || col >= N) return;
-    uint4* p = reinterpret_cast<uint4*>(out + (size_t)row * ldo + col);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      uint32_t w[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int i = 8 * j + 2 * q;
-        __nv_bfloat162 b2 = __floats2bfloat162_rn(silu(g[i]) * u[i], silu(g[i + 1]) * u[i + 1]);
-        w[q] = *reinterpret_cast<uint32_t*>(&b2);
-      }
-      p[j] = make_uint4(w[0], w[1], w[2], w[3]);
+  __device__ void col4(int row, int c, float4 g, float4 u) const {
+    bf16* p = out + (size_t)row * ldo + c;
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(silu(g.x) * u.x, silu(g.y) * u.y);
+    const __nv_bfloat162 hi = __floats2bfloat162_rn(silu(g.z) * u.z, silu(g.w) * u.w);
+    if (c + 4 <= N) {
+      uint2 w;
+      w.x = *reinterpret_cast<const uint32_t*>(&lo);
+      w.y = *reinterpret_cast<const uint32_t*>(&hi);
+      *reinterpret_cast<uint2*>(p) = w;
+    } else {
+      const bf16 a[4] = {lo.x, lo.y, hi.x, hi.y};
+      for (int j = 0; j < 4 && c + j < N; ++j) p[j] = a[j];
     }
   }
 };
 
-// QKV projection epilogue (N-tile = one head of h = 128): rotate query and key
-// heads (pairs (j, j + 64) by pos * theta_j, cos/sin from the table
-// rope[pos, 64] / rope[max_pos + pos, 64]) and scatter: q -> q[row, head, :],
-// k -> kc[b, g, i, :], v -> vc[b, g, :, i] (transposed); all bf16.  Row = b * n_seq + i
-// sits at position pos0 + i.
+// Warp-row epilogues: a warp owns one output row; lane l holds the columns
+// n0 + l + 32 q (q < BN / 32) of the summed accumulator.  The kernel stages the
+// accumulator rows in shared memory (and sums split-K partials there) first.
+//
+// QKV projection (N-tile = one head of h = 128): rotate query and key heads
+// (pairs (j, j + 64) by pos * theta_j; cos / sin from the table rope[pos, 64] /
+// rope[max_pos + pos, 64]) and scatter: q -> q[row, head, :], k -> kc[b, g, i, :],
+// v -> vc[b, g, :, i] (transposed); all bf16.  Row = b * n_seq + i sits at
+// position pos0 + i.
 struct EpiQkvRope {
-  static constexpr bool kChunked = false, kRowWise = true;
+  static constexpr bool kStaged = true, kWarpRows = true;
   bf16 *q, *kc, *vc;
   const float* rope;
   int max_pos, n_seq, np, pos0, Hq, Hkv;
-  template <int NCH, class Ld>
-  __device__ void run(int row, bool valid, int n0, Ld&& ld) const {
-    static_assert(NCH == 4, "one head of 128 per tile");
+  // rows row0 .. row0 + RB - 1 (those < M); the table loads of all rows go first
+  template <int NQ, int RB>
+  __device__ void warp_rows(int row0, int M, int n0, const float (*v)[NQ], int lane) const {
+    static_assert(NQ == 4, "one head of 128 per tile");
     const int head = n0 / 128;
-    const int b = valid ? row / n_seq : 0, i = valid ? row % n_seq : 0, pos = pos0 + i;
-#pragma unroll 1
-    for (int c = 0; c < 2; ++c) {
-      float lo[32], hi[32];
-      ld(0, c, lo);
-      ld(0, c + 2, hi);
-      if (!valid) continue;
-      if (head < Hq + Hkv) {
-        const float* cs = rope + (size_t)pos * 64 + c * 32;
-        const float* sn = rope + ((size_t)max_pos + pos) * 64 + c * 32;
-        bf16* dst = head < Hq ? q + ((size_t)row * Hq + head) * 128
-                              : kc + (((size_t)b * Hkv + (head - Hq)) * np + i) * 128;
-        uint32_t w1[16], w2[16];
+    if (head < Hq + Hkv) {
+      float cs[RB][2], sn[RB][2];
 #pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-          const float c0 = cs[j], s0 = sn[j], c1 = cs[j + 1], s1 = sn[j + 1];
-          __nv_bfloat162 a = __floats2bfloat162_rn(lo[j] * c0 - hi[j] * s0, lo[j + 1] * c1 - hi[j + 1] * s1);
-          __nv_bfloat162 bb = __floats2bfloat162_rn(hi[j] * c0 + lo[j] * s0, hi[j + 1] * c1 + lo[j + 1] * s1);
-          w1[j >> 1] = *reinterpret_cast<uint32_t*>(&a);
-          w2[j >> 1] = *reinterpret_cast<uint32_t*>(&bb);
-        }
-        uint4* d1 = reinterpret_cast<uint4*>(dst + c * 32);
-        uint4* d2 = reinterpret_cast<uint4*>(dst + 64 + c * 32);
+      for (int r = 0; r < RB; ++r) {
+        const int pos = pos0 + (row0 + r < M ? (row0 + r) % n_seq : 0);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          d1[j] = make_uint4(w1[4 * j], w1[4 * j + 1], w1[4 * j + 2], w1[4 * j + 3]);
-          d2[j] = make_uint4(w2[4 * j], w2[4 * j + 1], w2[4 * j + 2], w2[4 * j + 3]);
-        }
-      } else {
-        const int g = head - Hq - Hkv;
-        bf16* vt = vc + ((size_t)b * Hkv + g) * 128 * np + i;
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          vt[(size_t)(c * 32 + j) * np] = __float2bfloat16_rn(lo[j]);
-          vt[(size_t)(64 + c * 32 + j) * np] = __float2bfloat16_rn(hi[j]);
+        for (int q2 = 0; q2 < 2; ++q2) {
+          cs[r][q2] = rope[(size_t)pos * 64 + lane + 32 * q2];
+          sn[r][q2] = rope[((size_t)max_pos + pos) * 64 + lane + 32 * q2];
         }
       }
+#pragma unroll
+      for (int r = 0; r < RB; ++r) {
+        const int row = row0 + r;
+        if (row >= M) break;
+        const int b = row / n_seq, i = row % n_seq;
+        bf16* dst = head < Hq ? q + ((size_t)row * Hq + head) * 128
+                              : kc + (((size_t)b * Hkv + (head - Hq)) * np + i) * 128;
+#pragma unroll
+        for (int q2 = 0; q2 < 2; ++q2) {
+          const int j = lane + 32 * q2;
+          const float x1 = v[r][q2], x2 = v[r][q2 + 2];
+          dst[j] = __float2bfloat16_rn(x1 * cs[r][q2] - x2 * sn[r][q2]);
+          dst[j + 64] = __float2bfloat16_rn(x2 * cs[r][q2] + x1 * sn[r][q2]);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int r = 0; r < RB; ++r) {
+        const int row = row0 + r;
+        if (row >= M) break;
+        const int b = row / n_seq, i = row % n_seq;
+        bf16* vt = vc + ((size_t)b * Hkv + (head - Hq - Hkv)) * 128 * np + i;
+#pragma unroll
+        for (int q2 = 0; q2 < 4; ++q2)
+          vt[(size_t)(lane + 32 * q2) * np] = __float2bfloat16_rn(v[r][q2]);
+      }
+    }
+  }
+};
+
+// Router (N-tile = all E <= 32 NQ experts of a row): softmax over the E logits,
+// the top_k experts by probability (ties -> lower id) and their gates
+// renormalised over the selection: idx / gate [row, top_k]; lane k keeps the
+// k-th selection.
+struct EpiRouterTopk {
+  static constexpr bool kStaged = true, kWarpRows = true;
+  int32_t* idx;
+  float* gate;
+  int E, top_k;
+  template <int NQ, int RB>
+  __device__ void warp_rows(int row0, int M, int n0, const float (*v)[NQ], int lane) const {
+#pragma unroll 1
+    for (int r = 0; r < RB; ++r)
+      if (row0 + r < M) warp_row<NQ>(row0 + r, v[r], lane);
+  }
+  template <int NQ>
+  __device__ void warp_row(int row, const float* v, int lane) const {
+    float p[NQ];
+    float mx = -INFINITY;
+#pragma unroll
+    for (int q2 = 0; q2 < NQ; ++q2) {
+      p[q2] = lane + 32 * q2 < E ? v[q2] : -INFINITY;
+      mx = fmaxf(mx, p[q2]);
+    }
+    mx = warp_max(mx);
+    float z = 0.f;
+#pragma unroll
+    for (int q2 = 0; q2 < NQ; ++q2) {
+      p[q2] = lane + 32 * q2 < E ? expf(p[q2] - mx) : 0.f;
+      z += p[q2];
+    }
+    z = warp_sum(z);
+#pragma unroll
+    for (int q2 = 0; q2 < NQ; ++q2) p[q2] /= z;
+    unsigned taken = 0;
+    float gsum = 0.f, my_p = 0.f;
+    int my_e = 0;
+    for (int k = 0; k < top_k; ++k) {
+      float bp = -1.f;
+      int be = 0x7fffffff;
+#pragma unroll
+      for (int q2 = 0; q2 < NQ; ++q2) {
+        const int e = lane + 32 * q2;
+        if (e < E && !((taken >> q2) & 1u) && (p[q2] > bp || (p[q2] == bp && e < be))) {
+          bp = p[q2];
+          be = e;
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const float op = __shfl_xor_sync(0xffffffffu, bp, off);
+        const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+        if (op > bp || (op == bp && oe < be)) {
+          bp = op;
+          be = oe;
+        }
+      }
+      if ((be & 31) == lane) taken |= 1u << (be >> 5);
+      if (lane == k) {
+        my_e = be;
+        my_p = bp;
+      }
+      gsum += bp;
+    }
+    if (lane < top_k) {
+      idx[(size_t)row * top_k + lane] = my_e;
+      gate[(size_t)row * top_k + lane] = my_p / gsum;
     }
   }
 };
@@ -169,7 +244,7 @@ struct EpiQkvRope {
 // (columns n0 .. n0 + 32 NCH - 1, those < N): m = max, s = sum exp(l - m),
 // u = sum exp(l - m) (l - m), a = lowest id attaining m.  part[(tile, row)] = (m, s, u, a).
 struct EpiLmStats {
-  static constexpr bool kChunked = false, kRowWise = false;
+  static constexpr bool kStaged = false, kWarpRows = false;
   float* part;
   int M, N;
   float scale;
@@ -238,6 +313,37 @@ __device__ __forceinline__ uint32_t map(uint32_t saddr, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
   return r;
 }
+__device__ __forceinline__ float lds(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ float ldc(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ float4 lds4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ float4 ldc4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ void sts4(uint32_t addr, float a, float b, float c, float d) {
+  asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c),
+               "f"(d)
+               : "memory");
+}
 __device__ __forceinline__ void st4(uint32_t addr, float a, float b, float c, float d) {
   asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b),
                "f"(c), "f"(d)
@@ -256,16 +362,21 @@ struct DenseCfg {
   static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
 };
 
+// 256 threads: warp 0 lane 0 issues the TMA loads, warp 1 lane 0 the MMAs; all eight
+// warps share the epilogue (warps w and w + 4 read the same TMEM lane quarter).
+constexpr int TC_DENSE_THREADS = 256;
+
 template <int BN, int MT, bool DUAL, int ST, class Epi>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(TC_DENSE_THREADS, 1)
     tc_dense_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mB,
                     const __grid_constant__ CUtensorMap mB2, int M, int K, int ksplit, Epi epi,
-                    int32_t* err) {
+                    int32_t* err, int kwrap) {
+  // kwrap > 0: the B operand's K coordinate is taken modulo kwrap (A = [a1 | a2]
+  // against B = [w | w] without storing w twice)
   typedef DenseCfg<BN, MT, DUAL, ST> Cfg;
-  // split-K needs the whole fp32 tile in the (drained) pipeline buffers and a chunk epilogue
-  constexpr int RS = Cfg::NACC * BN + 4;  // reduction row stride (floats): padded against bank conflicts
-  constexpr bool kSplitOK =
-      MT * 128 * RS * 4 <= ST * Cfg::STAGE && (Epi::kChunked || Epi::kRowWise);
+  // staged epilogues reuse the drained pipeline buffers for the fp32 tile
+  constexpr int RS = Cfg::NACC * BN + 4;  // staging row stride (floats): padded against bank conflicts
+  static_assert(!Epi::kStaged || MT * 128 * RS * 4 <= ST * Cfg::STAGE, "staging buffer");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + ST * Cfg::STAGE);
@@ -311,14 +422,15 @@ __global__ void __launch_bounds__(128, 1)
       }
       uint8_t* st = smem + s * Cfg::STAGE;
       tc::mbar_expect_tx(full + s, Cfg::STAGE);
-#pragma unroll
       // CTAs start their K walk at different offsets so that they do not all read
       // the same activation tile from the same L2 slices at the same time
       const int kx = (kb_lo + (kb + rot) % nk) * TC_KB;
+      const int kxb = kwrap > 0 ? kx % kwrap : kx;
+#pragma unroll
       for (int mt = 0; mt < MT; ++mt)
         tc::tma_load_2d(st + mt * TC_SUB_A, &mA, full + s, kx, m0 + mt * 128);
-      tc::tma_load_2d(st + MT * TC_SUB_A, &mB, full + s, kx, n0);
-      if (DUAL) tc::tma_load_2d(st + MT * TC_SUB_A + Cfg::B_BYTES, &mB2, full + s, kx, n0);
+      tc::tma_load_2d(st + MT * TC_SUB_A, &mB, full + s, kxb, n0);
+      if (DUAL) tc::tma_load_2d(st + MT * TC_SUB_A + Cfg::B_BYTES, &mB2, full + s, kxb, n0);
     }
   } else if (warp == 1 && lane == 0) {
     constexpr uint32_t idesc = tc::idesc_bf16(128, BN);
@@ -358,81 +470,132 @@ __global__ void __launch_bounds__(128, 1)
   if (lane == 0) ready = nk == 0 || tc::mbar_wait(done, 0);
   ready = __shfl_sync(0xffffffffu, ready ? 1 : 0, 0) != 0;
   if (!ready && lane == 0) atomicOr(err, ERR_TIMEOUT);
-  const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
-  if (ksplit == 1) {
-    if (ready) {
+  const int quarter = warp & 3, half = warp >> 2;  // TMEM lane quarter; column half
+  const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
+  if constexpr (!Epi::kStaged) {
+    if (ready && half == 0) {  // never split; thread per row
       tc::fence_after_sync();
 #pragma unroll 1
       for (int mt = 0; mt < MT; ++mt) {
-        const int row = m0 + mt * 128 + 32 * warp + lane;
+        const int row = m0 + mt * 128 + 32 * quarter + lane;
         auto ld = [&](int a, int c, float* v) {
           tc::tmem_ld32(tmem + lane_base + (mt * Cfg::NACC + a) * BN + c * 32, v);
         };
         epi.template run<BN / 32>(row, row < M, n0, ld);
       }
     }
-  } else if constexpr (kSplitOK) {
-    // every thread of every CTA passes both cluster barriers, whatever happened above
-    const int R = MT * 128 / ksplit;         // rows owned per CTA
-    cl::sync();                              // all pipelines drained: smem reusable
+  } else {
+    // 1. this CTA's partial tile -> its own shared memory, row-major (stride RS)
+    const uint32_t stg = tc::smem_addr(smem);
     if (ready) {
       tc::fence_after_sync();
-      const uint32_t recv = tc::smem_addr(smem);
 #pragma unroll 1
       for (int mt = 0; mt < MT; ++mt) {
-        const int trow = mt * 128 + 32 * warp + lane;  // row within the tile
-        const int owner = trow / R, lr = trow % R;
-        const uint32_t dst = cl::map(recv, owner) + (uint32_t)(((rank * R + lr) * RS) * 4);
+        const uint32_t dst = stg + (uint32_t)((mt * 128 + 32 * quarter + lane) * RS * 4);
 #pragma unroll 1
         for (int a = 0; a < Cfg::NACC; ++a)
 #pragma unroll 1
-          for (int c = 0; c < BN / 32; ++c) {
+          for (int c = half; c < BN / 32; c += 2) {
             float v[32];
             tc::tmem_ld32(tmem + lane_base + (mt * Cfg::NACC + a) * BN + c * 32, v);
             const uint32_t o = dst + (uint32_t)((a * BN + c * 32) * 4);
 #pragma unroll
             for (int j = 0; j < 8; ++j)
-              cl::st4(o + 16 * j, v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+              cl::sts4(o + 16 * j, v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
           }
       }
     }
-    cl::sync();                              // all partial rows delivered
-    const float* buf = reinterpret_cast<const float*>(smem);
-    if constexpr (Epi::kRowWise) {  // one thread per owned row, chunks summed on demand
-      for (int lr = threadIdx.x; lr < R; lr += blockDim.x) {
-        auto ld = [&](int a, int c, float* v) {
+    // every thread of every CTA passes the cluster barriers, whatever happened above
+    if (ksplit > 1) cl::sync();
+    else __syncthreads();
+    // 2. this CTA owns rows [rank R, rank R + R) of the tile: sum the partials of the
+    //    cluster's CTAs in rank order (lane = column), RB rows per warp at a time
+    // Every instruction latency is exposed here (two warps per scheduler), so a warp
+    // issues all loads of a pass (every source CTA) before it sums them.
+    constexpr int NW = TC_DENSE_THREADS / 32;
+    const int R = MT * 128 / ksplit;
+    if constexpr (Epi::kWarpRows) {
+      // lane = column; RB whole rows per warp at a time
+      constexpr int NQ = Cfg::NACC * BN / 32;
+      constexpr int RB = NQ >= 4 ? 2 : 4;
+      static_assert(16 % RB == 0, "warp-row tiling");  // R is a multiple of 16
+#pragma unroll 1
+      for (int lr0 = warp * RB; lr0 < R; lr0 += NW * RB) {
+        const int row0 = m0 + rank * R + lr0;
+        if (row0 >= M) break;
+        const uint32_t off = (uint32_t)(((rank * R + lr0) * RS + lane) * 4);
+        float t[8][RB][NQ];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = 0.f;
-          for (int src = 0; src < ksplit; ++src) {
-            const float* p = buf + (size_t)(src * R + lr) * RS + a * BN + c * 32;
+        for (int src = 0; src < 8; ++src) {
+          if (src < ksplit) {
+            const uint32_t rb = off + (src == rank ? stg : cl::map(stg, (uint32_t)src));
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] += p[j];
+            for (int r = 0; r < RB; ++r)
+#pragma unroll
+              for (int q = 0; q < NQ; ++q) {
+                const uint32_t ad = rb + (uint32_t)((r * RS + q * 32) * 4);
+                t[src][r][q] = src == rank ? cl::lds(ad) : cl::ldc(ad);
+              }
           }
-        };
-        const int row = m0 + rank * R + lr;
-        epi.template run<BN / 32>(row, row < M, n0, ld);
+        }
+        float v[RB][NQ];
+#pragma unroll
+        for (int r = 0; r < RB; ++r)
+#pragma unroll
+          for (int q = 0; q < NQ; ++q) {
+            v[r][q] = 0.f;  // sources in rank order
+#pragma unroll
+            for (int src = 0; src < 8; ++src)
+              if (src < ksplit) v[r][q] += t[src][r][q];
+          }
+        epi.template warp_rows<BN / 32, RB>(row0, M, n0, v, lane);
       }
-    } else
-    for (int item = threadIdx.x; item < R * (BN / 32); item += blockDim.x) {
-      const int lr = item / (BN / 32), c = item % (BN / 32);
-      float v[32], u[32];
+    } else {
+      // lane -> (row, 4 consecutive columns): a warp instruction covers RPW rows of BN
+      constexpr int LPR = BN / 4, RPW = 32 / LPR;
+      constexpr int IB = Cfg::NACC == 2 ? 1 : 2;  // warp instructions per pass
+      // R is a multiple of 16, so a warp's RPW * IB rows lie wholly inside or outside it
+      static_assert(BN <= 128 && 16 % (RPW * IB) == 0, "column epilogue tiling");
+      const int rsub = lane / LPR, c4 = (lane % LPR) * 4;
+#pragma unroll 1
+      for (int lr0 = warp * RPW * IB; lr0 < R; lr0 += NW * RPW * IB) {
+        if (m0 + rank * R + lr0 >= M) break;
+        const uint32_t off = (uint32_t)(((rank * R + lr0 + rsub) * RS + c4) * 4);
+        float4 t[8][IB][Cfg::NACC];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        v[j] = 0.f;
-        u[j] = 0.f;
-      }
-      for (int src = 0; src < ksplit; ++src) {
-        const float* p = buf + (size_t)(src * R + lr) * RS + c * 32;
+        for (int src = 0; src < 8; ++src) {
+          if (src < ksplit) {
+            const uint32_t rb = off + (src == rank ? stg : cl::map(stg, (uint32_t)src));
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] += p[j];
-        if (DUAL) {
+            for (int i = 0; i < IB; ++i)
 #pragma unroll
-          for (int j = 0; j < 32; ++j) u[j] += p[BN + j];
+              for (int a = 0; a < Cfg::NACC; ++a) {
+                const uint32_t ad = rb + (uint32_t)((i * RPW * RS + a * BN) * 4);
+                t[src][i][a] = src == rank ? cl::lds4(ad) : cl::ldc4(ad);
+              }
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < IB; ++i) {
+          float4 v[Cfg::NACC];
+#pragma unroll
+          for (int a = 0; a < Cfg::NACC; ++a) {
+            v[a] = make_float4(0.f, 0.f, 0.f, 0.f);  // sources in rank order
+#pragma unroll
+            for (int src = 0; src < 8; ++src)
+              if (src < ksplit) {
+                v[a].x += t[src][i][a].x;
+                v[a].y += t[src][i][a].y;
+                v[a].z += t[src][i][a].z;
+                v[a].w += t[src][i][a].w;
+              }
+          }
+          const int row = m0 + rank * R + lr0 + i * RPW + rsub;
+          if (row < M) epi.col4(row, n0 + c4, v[0], v[Cfg::NACC - 1]);
         }
       }
-      const int row = m0 + rank * R + lr;
-      epi.chunk(row, row < M, n0 + c * 32, v, u);
     }
+    if (ksplit > 1) cl::sync();  // peers may still read this CTA's tile
   }
   tc::fence_before_sync();
   __syncthreads();
@@ -459,8 +622,12 @@ struct ExpertCfg {
   static constexpr size_t SMEM = 1024 + (size_t)ST * STAGE + 256;
 };
 
+// 320 threads: warp 0 TMA, warp 1 MMA, warps 2..9 epilogue (warps w and w + 4 share
+// a TMEM lane quarter and split the token chunks).
+constexpr int TC_EXPERT_THREADS = 320;
+
 template <bool GATEUP, int ST>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(TC_EXPERT_THREADS, 1)
     tc_expert_kernel(const __grid_constant__ CUtensorMap mW, const __grid_constant__ CUtensorMap mW2,
                      const __grid_constant__ CUtensorMap mX, const int32_t* __restrict__ chunk_e,
                      const int32_t* __restrict__ chunk_r0, const int32_t* __restrict__ n_chunks,
@@ -474,7 +641,7 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + ST * Cfg::STAGE);
   uint64_t* empty = full + ST;
   uint64_t* tfull = empty + ST;   // accumulator ready (MMA -> epilogue)
-  uint64_t* tempty = tfull + 1;   // accumulator drained (epilogue -> MMA), 4 arrivals
+  uint64_t* tempty = tfull + 1;   // accumulator drained (epilogue -> MMA), 8 arrivals
   uint32_t* tslot = reinterpret_cast<uint32_t*>(tempty + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_units = *n_chunks * FT;
@@ -486,7 +653,7 @@ __global__ void __launch_bounds__(192, 1)
       tc::mbar_init(empty + s, 1);
     }
     tc::mbar_init(tfull, 1);
-    tc::mbar_init(tempty, 4);
+    tc::mbar_init(tempty, 8);
     tc::fence_mbar_init();
   }
   if (warp == 1) tc::tmem_alloc(tslot, Cfg::TCOLS);
@@ -574,8 +741,8 @@ __global__ void __launch_bounds__(192, 1)
       }
     }
   } else {
-    // epilogue warps 2..5 -> TMEM lane quarter (warp % 4)
-    const int q = warp & 3;
+    // epilogue warps 2..9 -> TMEM lane quarter (warp % 4), token chunks of parity hf
+    const int q = warp & 3, hf = (warp - 2) >> 2;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     int ui = 0;
     for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++ui) {
@@ -592,7 +759,7 @@ __global__ void __launch_bounds__(192, 1)
       const int fr = f * 128 + 32 * q + lane;  // weight row within the expert = output column
       const int nch = (n + 31) >> 5;
 #pragma unroll 1
-      for (int c = 0; c < nch; ++c) {
+      for (int c = hf; c < nch; c += 2) {
         float v[32];
         tc::tmem_ld32(tmem + lane_base + c * 32, v);
         if (GATEUP) {
@@ -633,6 +800,8 @@ dg_status tc_gemm_store_f32(dg_model* m, const bf16* A, const void* W, float* ou
                             int K, cudaStream_t st);
 dg_status tc_gemm_qkv_rope(dg_model* m, const bf16* A, const void* W, int M, int n_seq, int np,
                            int pos0, bf16* q, bf16* kc, bf16* vc, cudaStream_t st);
+dg_status tc_router_topk(dg_model* m, const bf16* u2, const void* Wr, int M, int32_t* idx,
+                         float* gate, cudaStream_t st);
 dg_status tc_gemm_f32_rows(dg_model* m, const bf16* A, int a_rows, const void* W, float* out,
                            int M, int N, int K, cudaStream_t st);
 dg_status tc_gemm_add_residual(dg_model* m, const bf16* A, const void* W, float* x, int M, int N,

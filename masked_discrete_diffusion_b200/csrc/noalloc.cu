@@ -141,9 +141,9 @@ extern "C" dg_status dg_lmhead_entropy_noalloc(const float* hidden, const void* 
   DG_TRY(encode(lm_head, (uint64_t)V, (uint64_t)d, NA_BN, &mb));
   typedef DenseCfg<NA_BN, 2, false, NA_ST> Cfg;
   dim3 grid((M + 255) / 256, (V + NA_BN - 1) / NA_BN, 1);
-  tc_dense_kernel<NA_BN, 2, false, NA_ST, EpiLmStats><<<grid, 128, Cfg::SMEM, st>>>(
-      ma, mb, mb, M, d, 1, EpiLmStats{part, M, V, logit_scale}, err);
-  lm_merge_kernel<float><<<(M + 3) / 4, 128, 0, st>>>(part, (V + NA_BN - 1) / NA_BN, M, entropy,
+  tc_dense_kernel<NA_BN, 2, false, NA_ST, EpiLmStats><<<grid, TC_DENSE_THREADS, Cfg::SMEM, st>>>(
+      ma, mb, mb, M, d, 1, EpiLmStats{part, M, V, logit_scale}, err, 0);
+  lm_merge_kernel<float><<<M, 128, 0, st>>>(part, (V + NA_BN - 1) / NA_BN, M, entropy,
                                                       argmax);
   noalloc_flag_kernel<<<(M + 127) / 128, 128, 0, st>>>(err, M, entropy, argmax);
   cudaError_t e = cudaGetLastError();

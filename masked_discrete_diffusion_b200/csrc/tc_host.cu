@@ -103,7 +103,7 @@ template <class K> dg_status set_smem(K kern, size_t bytes) {
 template <int BN, int MT, bool DUAL, int ST, class Epi>
 dg_status launch_dense(dg_model* m, const CUtensorMap& a, const CUtensorMap& b,
                        const CUtensorMap& b2, int M, int N, int K, Epi epi, cudaStream_t st,
-                       bool allow_split = true) {
+                       bool allow_split = true, int kwrap = 0) {
   typedef DenseCfg<BN, MT, DUAL, ST> Cfg;
   auto kern = tc_dense_kernel<BN, MT, DUAL, ST, Epi>;
   dim3 grid(ceil_div_i(M, 128 * MT), ceil_div_i(N, BN), 1);
@@ -114,10 +114,10 @@ dg_status launch_dense(dg_model* m, const CUtensorMap& a, const CUtensorMap& b,
     while (ks < 8 && tiles * ks * 2 <= state(m)->n_sm && nk >= ks * 2 * 2) ks *= 2;
   cudaError_t e;
   if (ks == 1) {
-    e = launch_pdl(kern, grid, 128, Cfg::SMEM, st, 1, a, b, b2, M, K, 1, epi, m->ws.err);
+    e = launch_pdl(kern, grid, TC_DENSE_THREADS, Cfg::SMEM, st, 1, a, b, b2, M, K, 1, epi, m->ws.err, kwrap);
   } else {
     grid.z = ks;
-    e = launch_pdl(kern, grid, 128, Cfg::SMEM, st, ks, a, b, b2, M, K, ks, epi, m->ws.err);
+    e = launch_pdl(kern, grid, TC_DENSE_THREADS, Cfg::SMEM, st, ks, a, b, b2, M, K, ks, epi, m->ws.err, kwrap);
   }
   ++m->launches;
   if (e != cudaSuccess) {
@@ -128,7 +128,7 @@ dg_status launch_dense(dg_model* m, const CUtensorMap& a, const CUtensorMap& b,
 }
 
 constexpr int DENSE_BN = 64, DENSE_MT = 2, DENSE_ST = 5, DUAL_ST = 4;
-constexpr int QKV_ST = 4;
+constexpr int QKV_ST = 4, RT_ST = 4;
 constexpr int LM_BN = 256, LM_ST = 3;
 constexpr int GU_ST = 4, DN_ST = 6;
 constexpr int GU8_ST = 3, DN8_ST = 5;
@@ -169,6 +169,8 @@ dg_status tc_prepare(dg_model* m) {
   DG_TRY(set_smem(tc_expert_kernel<true, GU_ST>, ExpertCfg<true, GU_ST>::SMEM));
   DG_TRY(set_smem(tc_expert_kernel<false, DN_ST>, ExpertCfg<false, DN_ST>::SMEM));
   DG_TRY(set_smem(tc_attn_kernel, AT_SMEM));
+  DG_TRY(set_smem(tc_dense_kernel<128, 1, false, RT_ST, EpiRouterTopk>,
+                  DenseCfg<128, 1, false, RT_ST>::SMEM));
   DG_TRY(set_smem(tc_dense_kernel<128, DENSE_MT, false, QKV_ST, EpiQkvRope>,
                   DenseCfg<128, DENSE_MT, false, QKV_ST>::SMEM));
   DG_TRY(set_smem(tc_expert_f8_kernel<true, GU8_ST>, ExpertF8Cfg<true, GU8_ST>::SMEM));
@@ -216,6 +218,23 @@ dg_status tc_gemm_qkv_rope(dg_model* m, const bf16* A, const void* W, int M, int
   return launch_dense<128, DENSE_MT, false, QKV_ST>(m, a, b, b, M, N, K, epi, st);
 }
 
+// Router logits u . w on tensor cores as [u_hi | u_lo] . [w | w] (K = 2 d), top-k
+// in the epilogue.  One N-tile holds all experts (E <= 128).
+dg_status tc_router_topk(dg_model* m, const bf16* u2, const void* Wr, int M, int32_t* idx,
+                         float* gate, cudaStream_t st) {
+  const dg_config& c = m->cfg;
+  const int d = c.d_model;
+  CUtensorMap a, b;
+  DG_TRY(tmap(m, u2, m->ws.max_tok, 2 * d, 128, &a));
+  DG_TRY(tmap(m, Wr, c.n_experts, d, 128, &b));
+  EpiRouterTopk epi;
+  epi.idx = idx;
+  epi.gate = gate;
+  epi.E = c.n_experts;
+  epi.top_k = c.top_k;
+  return launch_dense<128, 1, false, RT_ST>(m, a, b, b, M, 128, 2 * d, epi, st, true, d);
+}
+
 dg_status tc_gemm_f32_rows(dg_model* m, const bf16* A, int a_rows, const void* W, float* out,
                            int M, int N, int K, cudaStream_t st) {
   CUtensorMap a, b;
@@ -255,7 +274,7 @@ dg_status tc_lmhead_stats(dg_model* m, const bf16* xn, int M, float* ent, int32_
                                                EpiLmStats{part, M, c.vocab, c.logit_scale}, st,
                                                false)));
   const int n_vt = ceil_div_i(c.vocab, LM_BN);
-  launch_pdl((lm_merge_kernel<float>), ceil_div_i(M, 4), 128, 0, st, 1, part, n_vt, M, ent, amax);
+  launch_pdl((lm_merge_kernel<float>), M, 128, 0, st, 1, part, n_vt, M, ent, amax);
   ++m->launches;
   return DG_OK;
 }
@@ -268,7 +287,7 @@ static dg_status launch_expert(dg_model* m, const CUtensorMap& w, const CUtensor
   auto kern = tc_expert_kernel<GATEUP, ST>;
   const int n_sm = state(m)->n_sm;
   const Workspace& ws = m->ws;
-  launch_pdl((kern), n_sm, 192, Cfg::SMEM, st, 1, w, w2, x, ws.tile_e, ws.tile_m0, ws.n_tiles, ws.offsets,
+  launch_pdl((kern), n_sm, TC_EXPERT_THREADS, Cfg::SMEM, st, 1, w, w2, x, ws.tile_e, ws.tile_m0, ws.n_tiles, ws.offsets,
                                      w_rows, K, FT, out, ldo, gate_of, ws.err);
   ++m->launches;
   cudaError_t e = cudaGetLastError();
