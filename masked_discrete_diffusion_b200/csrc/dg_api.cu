@@ -128,10 +128,6 @@ template <class Path> static dg_status alloc_workspace(dg_model* m) {
   DG_TRY(ws_alloc_v<TKV>(ws, &ws.kc, T_pad * c.n_kv_heads * h));
   DG_TRY(ws_alloc_v<TKV>(ws, &ws.vc, T_pad * c.n_kv_heads * h));
   ws.kc_elems = T_pad * c.n_kv_heads * h;
-  if constexpr (Path::kTensorCores) {
-    DG_TRY(ws_alloc_v<float>(ws, &ws.attn_o, (size_t)ATT_MAX_SPLITS * T * c.n_q_heads * h));
-    DG_TRY(ws_alloc_v<float>(ws, &ws.attn_ml, (size_t)ATT_MAX_SPLITS * T * c.n_q_heads * 2));
-  }
   DG_TRY(ws_alloc_v<Acc>(ws, &ws.ys, T * d));
   DG_TRY(ws_alloc_v<TA>(ws, &ws.sh, T * c.shared_inter));
   DG_TRY(ws_alloc(ws, &ws.ridx, R));

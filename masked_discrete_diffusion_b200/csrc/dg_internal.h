@@ -107,7 +107,6 @@ struct Workspace {
   int32_t *remaining = nullptr, *loop_s = nullptr;  // [max_batch] masked left; steps left
   int max_pos = 0;
   size_t kc_elems = 0;
-  void *attn_o = nullptr, *attn_ml = nullptr;  // attention key-split partials
   int max_tiles = 0;
   int n_vtiles = 0;
 };

@@ -1,13 +1,18 @@
 // a3: attention on tcgen05.  One CTA = (query tile of 128 rows, query head j,
-// batch element b, key split z).  Keys are the concatenation of segment A (the
-// cached prompt window) and segment B (the pass's own keys: the canvas, or the
-// prompt itself in the causal prefill).  Per key tile of 128:
-//   S = Q K^T          (TMEM, fp32)             — tcgen05.mma, operands by TMA
-//   P = exp(S/sqrt(h) - m) (bf16, 128B-swizzled smem, written by the row's thread)
-//   O_t = P V          (TMEM)                   — V cached transposed (h x keys)
-//   O = O * e^(m_old - m_new) + O_t, l likewise (registers, one row per thread)
-// Each split writes its unnormalised O, m and l; attn_combine merges the splits
-// in a fixed order.  Grouped-query: head j reads key/value head j / (Hq/Hkv).
+// batch element b, key split z); the splits of a (tile, head, b) form one thread
+// block cluster.  Keys are the concatenation of segment A (the cached prompt
+// window) and segment B (the pass's own keys: the canvas, or the prompt itself
+// in the causal prefill).  Per key tile of 128:
+//   S = Q K^T          (TMEM, two buffers: S of the next tile is computed while
+//                       this tile's softmax runs)  — tcgen05.mma, operands by TMA
+//   P = exp(S/sqrt(h) - m) (bf16, 128B-swizzled smem)
+//   O_t = P V          (TMEM)                     — V cached transposed (h x keys)
+//   O = O * e^(m_old - m_new) + O_t, l likewise   (registers)
+// Eight warps: warps w and w + 4 share a TMEM lane quarter (32 query rows) and
+// split the tile's keys (softmax) and the head dimension (O) in halves.  At the
+// end the splits of the cluster merge through distributed shared memory in
+// rank order and the owning CTA writes the normalised bf16 output rows.
+// Grouped-query: head j reads key/value head j / (Hq/Hkv).
 //
 // Passages: bidirectional attention inside the canvas and attention to the
 // prompt's KV cache — "DiffusionGemma 技术报告" (full translation page), §3.1
@@ -24,24 +29,28 @@ struct AttnParams {
   int nq;          // queries per batch element (rows b*nq .. b*nq + nq - 1 of Q)
   int qpos0;       // absolute position of query 0
   int Hq, Hkv;
-  int nA, kposA, rowsA, vrowsA;  // segment A: keys, first position, K rows per (b,g), V^T rows base
-  int nB, kposB, rowsB;          // segment B
+  int nA, kposA, rowsA;  // segment A: keys, first position, K rows per (b, g)
+  int nB, kposB, rowsB;  // segment B
   int causal, window;
   int tiles_per_split;
   int layer_rowA;   // first K row of this layer's segment A for (b=0, g=0)
   int layer_vrowA;  // first V^T row of this layer's segment A for (b=0, g=0)
-  float* part_o;    // [splits, B*nq, Hq, 128]
-  float* part_ml;   // [splits, B*nq, Hq, 2]
   int B;
   float scale_log2;  // log2(e) / sqrt(h)
+  bf16* out;         // [B*nq, Hq, 128]
 };
 
 constexpr int AT_KT = 128;  // keys per tile
+constexpr int AT_THREADS = 256;
 constexpr uint32_t AT_SUB = 128 * 64 * 2;
-constexpr size_t AT_SMEM = 1024 + 2 * AT_SUB /*Q*/ + 2 * (4 * AT_SUB) /*K,V x2*/ + 2 * AT_SUB /*P*/ + 256;
+constexpr int AT_RS = 132;  // merge staging row stride (floats)
+constexpr size_t AT_SMEM =
+    1024 + 2 * AT_SUB /*Q*/ + 2 * (4 * AT_SUB) /*K,V x2*/ + 2 * AT_SUB /*P*/ + 256 /*barriers*/ +
+    2 * 128 * 4 /*row max halves*/ + 128 * 4 * 4 /*m, l halves for the merge*/;
+static_assert(128 * AT_RS * 4 <= 2 * 4 * AT_SUB, "merge staging fits the K/V buffers");
 
 // h = 128 only (two 64-wide swizzle atoms along the head dimension).
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(AT_THREADS, 1)
     tc_attn_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mKA,
                    const __grid_constant__ CUtensorMap mVA, const __grid_constant__ CUtensorMap mKB,
                    const __grid_constant__ CUtensorMap mVB, AttnParams p, int32_t* err) {
@@ -49,22 +58,26 @@ __global__ void __launch_bounds__(128, 1)
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sQ = smem;                       // 2 sub-tiles
   uint8_t* sKV = sQ + 2 * AT_SUB;           // stage s: K (2 sub) then V^T (2 sub)
-  uint8_t* sP = sKV + 2 * 4 * AT_SUB;       // 2 sub-tiles
+  uint8_t* sP = sKV + 2 * 4 * AT_SUB;       // 2 sub-tiles (keys 0..63, 64..127)
   uint64_t* bar = reinterpret_cast<uint64_t*>(sP + 2 * AT_SUB);
   uint64_t* q_full = bar;
   uint64_t* kv_full = bar + 1;  // [2]
-  uint64_t* s_done = bar + 3;
-  uint64_t* o_done = bar + 4;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 5);
+  uint64_t* s_done = bar + 3;   // [2]
+  uint64_t* o_done = bar + 5;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 6);
+  float* xmax = reinterpret_cast<float*>(smem + 2 * AT_SUB + 8 * AT_SUB + 2 * AT_SUB + 256);  // [2][128]
+  float* mlst = xmax + 256;  // [128][4]: m, l of half 0, l of half 1, unused
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int quarter = warp & 3, hf = warp >> 2;
   const int Hq = p.Hq;
   const int qt = blockIdx.x / Hq, j = blockIdx.x % Hq;
   const int b = blockIdx.y, z = blockIdx.z;
+  const int splits = gridDim.z;
   const int g = j / (Hq / p.Hkv);
   const int q0 = qt * 128;
-  const int row = q0 + tid;  // this thread's query (within the batch element)
-  const int qp = p.qpos0 + row;
+  const int r = 32 * quarter + lane;  // this thread's query row within the tile
+  const int qp = p.qpos0 + q0 + r;
 
   // key tiles of this split
   const int TA = (p.nA + AT_KT - 1) / AT_KT, TB = (p.nB + AT_KT - 1) / AT_KT;
@@ -81,19 +94,20 @@ __global__ void __launch_bounds__(128, 1)
 
   if (tid == 0) {
     tc::mbar_init(q_full, 1);
-    tc::mbar_init(kv_full, 1);
-    tc::mbar_init(kv_full + 1, 1);
-    tc::mbar_init(s_done, 1);
+    for (int k = 0; k < 2; ++k) {
+      tc::mbar_init(kv_full + k, 1);
+      tc::mbar_init(s_done + k, 1);
+    }
     tc::mbar_init(o_done, 1);
     tc::fence_mbar_init();
   }
-  if (warp == 1) tc::tmem_alloc(tslot, 256);
+  if (warp == 1) tc::tmem_alloc(tslot, 512);
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tslot;
-  const uint32_t tS = tmem, tO = tmem + 128;
-  const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+  const uint32_t tO = tmem + 256;  // S buffers at columns 0 and 128
+  const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
   pdl_enter();  // global memory is touched only from here on
 
   auto load_tile = [&](int i) {  // tile index i within this split -> stage i & 1
@@ -119,6 +133,29 @@ __global__ void __launch_bounds__(128, 1)
       tc::tma_load_2d(st + 3 * AT_SUB, &mVB, fb, t0 + 64, vrow);
     }
   };
+  constexpr uint32_t idesc = tc::idesc_bf16(128, 128);
+  // S(i) = Q K_i^T into S buffer i & 1 (thread 0); false on a timeout
+  auto issue_s = [&](int i) -> bool {
+    if (i == 0 && !tc::mbar_wait(q_full, 0)) return false;
+    if (!tc::mbar_wait(kv_full + (i & 1), (i >> 1) & 1)) return false;
+    tc::fence_after_sync();
+    const uint32_t qa = tc::smem_addr(sQ), ka = tc::smem_addr(sKV + (i & 1) * 4 * AT_SUB);
+#pragma unroll
+    for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        tc::mma_bf16(tmem + (i & 1) * 128, tc::sdesc_k128(qa + kb * AT_SUB + k * 32),
+                     tc::sdesc_k128(ka + kb * AT_SUB + k * 32), idesc, (kb | k) != 0);
+    tc::mma_commit(s_done + (i & 1));
+    return true;
+  };
+  // every warp's lane 0 waits on `bar`; false everywhere if any wait gave up
+  auto wait_all = [&](uint64_t* bar_, uint32_t ph) -> bool {
+    bool ok_ = true;
+    if (lane == 0) ok_ = tc::mbar_wait(bar_, ph);
+    ok_ = __shfl_sync(0xffffffffu, ok_ ? 1 : 0, 0) != 0;
+    return __syncthreads_and(ok_ ? 1 : 0) != 0;
+  };
 
   bool ok = true;
   if (tid == 0 && nt > 0) {
@@ -128,13 +165,13 @@ __global__ void __launch_bounds__(128, 1)
     tc::tma_load_2d(sQ + AT_SUB, &mQ, q_full, j * 128 + 64, qrow);
     load_tile(0);
     if (nt > 1) load_tile(1);
+    if (!issue_s(0)) atomicOr(err, ERR_TIMEOUT);
   }
 
-  float o[128];
+  float o[64];  // head dims 64 hf .. 64 hf + 63 of this row
 #pragma unroll
-  for (int d = 0; d < 128; ++d) o[d] = 0.f;
-  float m_run = -INFINITY, l_run = 0.f;
-  constexpr uint32_t idesc = tc::idesc_bf16(128, 128);
+  for (int d = 0; d < 64; ++d) o[d] = 0.f;
+  float m_run = -INFINITY, l_run = 0.f;  // l over this half's keys
 
   for (int i = 0; i < nt && ok; ++i) {
     const int t = my_lo + i;
@@ -142,56 +179,41 @@ __global__ void __launch_bounds__(128, 1)
     const int t0 = segA ? t * AT_KT : (t - TA) * AT_KT;
     const int nseg = segA ? p.nA : p.nB;
     const int kpos0 = (segA ? p.kposA : p.kposB) + t0;
-    uint8_t* st = sKV + (i & 1) * 4 * AT_SUB;
-    // ---- S = Q K^T
-    if (tid == 0) {
-      bool w1 = i > 0 || tc::mbar_wait(q_full, 0);
-      bool w2 = w1 && tc::mbar_wait(kv_full + (i & 1), (i >> 1) & 1);
-      if (!w2) {
-        atomicOr(err, ERR_TIMEOUT);
-      } else {
-        tc::fence_after_sync();
-        const uint32_t qa = tc::smem_addr(sQ), ka = tc::smem_addr(st);
-#pragma unroll
-        for (int kb = 0; kb < 2; ++kb)
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            tc::mma_bf16(tS, tc::sdesc_k128(qa + kb * AT_SUB + k * 32),
-                         tc::sdesc_k128(ka + kb * AT_SUB + k * 32), idesc, (kb | k) != 0);
-        tc::mma_commit(s_done);
-      }
-    }
+    // ---- S of the next tile runs on the tensor cores during this tile's softmax
+    if (tid == 0 && i + 1 < nt && !issue_s(i + 1)) atomicOr(err, ERR_TIMEOUT);
     __syncwarp();
-    bool ready = true;
-    if (lane == 0) ready = tc::mbar_wait(s_done, i & 1);
-    ready = __shfl_sync(0xffffffffu, ready ? 1 : 0, 0) != 0;
-    if (!__syncthreads_and(ready ? 1 : 0)) {
+    if (!wait_all(s_done + (i & 1), (i >> 1) & 1)) {
       if (tid == 0) atomicOr(err, ERR_TIMEOUT);
       ok = false;
       break;
     }
     tc::fence_after_sync();
-    // ---- softmax of this row over the tile (two passes over TMEM)
+    const uint32_t tS = tmem + (i & 1) * 128 + 64 * hf;
+    // ---- softmax over this half's 64 keys; the row max is shared with the other half
     float mt = -INFINITY;
 #pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < 2; ++c) {
       float v[32];
       tc::tmem_ld32(tS + lane_base + c * 32, v);
 #pragma unroll
       for (int q = 0; q < 32; ++q) {
-        const int kk = t0 + c * 32 + q;
-        const int kp = kpos0 + c * 32 + q;
+        const int kk = t0 + 64 * hf + c * 32 + q;
+        const int kp = kpos0 + 64 * hf + c * 32 + q;
         bool valid = kk < nseg;
         if (p.causal) valid = valid && kp <= qp && kp > qp - p.window;
         if (valid) mt = fmaxf(mt, v[q] * p.scale_log2);
       }
     }
+    xmax[hf * 128 + r] = mt;
+    __syncthreads();
+    mt = fmaxf(xmax[r], xmax[128 + r]);
     const float m_new = fmaxf(m_run, mt);
     const float alpha = (m_new == -INFINITY) ? 1.f : exp2f(m_run - m_new);
     float lsum = 0.f;
-    const int r7 = tid & 7;
+    const int r7 = r & 7;
+    uint8_t* prow = sP + hf * AT_SUB + r * 128;
 #pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < 2; ++c) {
       float v[32];
       tc::tmem_ld32(tS + lane_base + c * 32, v);
       uint32_t pk[16];
@@ -200,8 +222,8 @@ __global__ void __launch_bounds__(128, 1)
         float e2[2];
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
-          const int kk = t0 + c * 32 + q + u;
-          const int kp = kpos0 + c * 32 + q + u;
+          const int kk = t0 + 64 * hf + c * 32 + q + u;
+          const int kp = kpos0 + 64 * hf + c * 32 + q + u;
           bool valid = kk < nseg;
           if (p.causal) valid = valid && kp <= qp && kp > qp - p.window;
           e2[u] = valid ? exp2f(v[q + u] * p.scale_log2 - m_new) : 0.f;
@@ -210,12 +232,11 @@ __global__ void __launch_bounds__(128, 1)
         __nv_bfloat162 b2 = __floats2bfloat162_rn(e2[0], e2[1]);
         pk[q >> 1] = *reinterpret_cast<uint32_t*>(&b2);
       }
-      // keys c*32 .. c*32+31 -> sub-tile c/2, 16-byte chunks (c%2)*4 .. +3, swizzled by row
-      uint8_t* base = sP + (c >> 1) * AT_SUB + tid * 128;
+      // keys 32c .. 32c + 31 of this half -> 16-byte chunks 4c .. 4c + 3, swizzled by row
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const int chunk = (c & 1) * 4 + q;
-        *reinterpret_cast<uint4*>(base + ((chunk ^ r7) << 4)) =
+        const int chunk = c * 4 + q;
+        *reinterpret_cast<uint4*>(prow + ((chunk ^ r7) << 4)) =
             make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
       }
     }
@@ -227,7 +248,7 @@ __global__ void __launch_bounds__(128, 1)
     // ---- O_t = P V
     if (tid == 0) {
       tc::fence_after_sync();
-      const uint32_t pa = tc::smem_addr(sP), va = tc::smem_addr(st + 2 * AT_SUB);
+      const uint32_t pa = tc::smem_addr(sP), va = tc::smem_addr(sKV + (i & 1) * 4 * AT_SUB + 2 * AT_SUB);
 #pragma unroll
       for (int kb = 0; kb < 2; ++kb)
 #pragma unroll
@@ -237,73 +258,95 @@ __global__ void __launch_bounds__(128, 1)
       tc::mma_commit(o_done);
     }
     __syncwarp();
-    ready = true;
-    if (lane == 0) ready = tc::mbar_wait(o_done, i & 1);
-    ready = __shfl_sync(0xffffffffu, ready ? 1 : 0, 0) != 0;
-    if (!__syncthreads_and(ready ? 1 : 0)) {
+    if (!wait_all(o_done, i & 1)) {
       if (tid == 0) atomicOr(err, ERR_TIMEOUT);
       ok = false;
       break;
     }
     tc::fence_after_sync();
-    // stage i & 1 is free again: prefetch tile i + 2
+    // stage i & 1 is free again (S(i) and O_t(i) done): prefetch tile i + 2
     if (tid == 0 && i + 2 < nt) load_tile(i + 2);
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < 2; ++c) {
       float v[32];
-      tc::tmem_ld32(tO + lane_base + c * 32, v);
+      tc::tmem_ld32(tO + lane_base + 64 * hf + c * 32, v);
 #pragma unroll
       for (int q = 0; q < 32; ++q) o[c * 32 + q] = o[c * 32 + q] * alpha + v[q];
     }
     tc::fence_before_sync();
-    __syncthreads();
   }
 
-  // ---- partial results of this split
-  if (row < p.nq) {
-    const size_t tok = (size_t)b * p.nq + row;
-    const size_t ntok = (size_t)p.B * p.nq;
-    float* po = p.part_o + (((size_t)z * ntok + tok) * Hq + j) * 128;
+  // ---- merge of the cluster's splits: stage (m, l, O) rows in this CTA's K/V buffers
+  // (all loads were consumed, all MMAs are done), then the owner of each row sums the
+  // splits in rank order and writes the normalised bf16 row.
+  __syncthreads();
+  const uint32_t stg = tc::smem_addr(sKV);
+  {
+    const uint32_t dst = stg + (uint32_t)((r * AT_RS + 64 * hf) * 4);
 #pragma unroll
-    for (int d = 0; d < 128; d += 4)
-      *reinterpret_cast<float4*>(po + d) = make_float4(o[d], o[d + 1], o[d + 2], o[d + 3]);
-    float* pm = p.part_ml + (((size_t)z * ntok + tok) * Hq + j) * 2;
-    pm[0] = (nt > 0 && ok) ? m_run : -INFINITY;
-    pm[1] = (nt > 0 && ok) ? l_run : 0.f;
+    for (int d = 0; d < 64; d += 4) cl::sts4(dst + d * 4, o[d], o[d + 1], o[d + 2], o[d + 3]);
+    const bool have = nt > 0 && ok;
+    mlst[r * 4 + 1 + hf] = have ? l_run : 0.f;
+    if (hf == 0) mlst[r * 4] = have ? m_run : -INFINITY;
   }
+  if (splits > 1) cl::sync();
+  else __syncthreads();
+  {
+    const int R = 128 / splits;  // rows owned by this CTA (splits: 1, 2, 4 or 8)
+    const uint32_t mls = tc::smem_addr(mlst);
+#pragma unroll 1
+    for (int lr = warp; lr < R; lr += AT_THREADS / 32) {
+      const int row = z * R + lr;  // row within the tile
+      if (q0 + row >= p.nq) break;
+      float ms[8], ls[8];
+      float4 os[8];
+#pragma unroll
+      for (int s2 = 0; s2 < 8; ++s2) {
+        if (s2 < splits) {
+          const uint32_t base_ml = (splits > 1 ? cl::map(mls, (uint32_t)s2) : mls) + row * 16;
+          const uint32_t base_o = (splits > 1 ? cl::map(stg, (uint32_t)s2) : stg) +
+                                  (uint32_t)((row * AT_RS + 4 * lane) * 4);
+          if (splits > 1) {
+            ms[s2] = cl::ldc(base_ml);
+            ls[s2] = cl::ldc(base_ml + 4) + cl::ldc(base_ml + 8);
+            os[s2] = cl::ldc4(base_o);
+          } else {
+            ms[s2] = cl::lds(base_ml);
+            ls[s2] = cl::lds(base_ml + 4) + cl::lds(base_ml + 8);
+            os[s2] = cl::lds4(base_o);
+          }
+        }
+      }
+      float M = -INFINITY;
+#pragma unroll
+      for (int s2 = 0; s2 < 8; ++s2)
+        if (s2 < splits) M = fmaxf(M, ms[s2]);
+      float L = 0.f;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int s2 = 0; s2 < 8; ++s2)
+        if (s2 < splits && ms[s2] > -INFINITY) {
+          const float w = exp2f(ms[s2] - M);
+          L += w * ls[s2];
+          acc.x += w * os[s2].x;
+          acc.y += w * os[s2].y;
+          acc.z += w * os[s2].z;
+          acc.w += w * os[s2].w;
+        }
+      const float inv = L > 0.f ? 1.f / L : 0.f;
+      const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+      const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+      uint2 pk;
+      pk.x = *reinterpret_cast<const uint32_t*>(&lo);
+      pk.y = *reinterpret_cast<const uint32_t*>(&hi);
+      const size_t tok = (size_t)b * p.nq + q0 + row;
+      *reinterpret_cast<uint2*>(p.out + (tok * Hq + j) * 128 + 4 * lane) = pk;
+    }
+  }
+  if (splits > 1) cl::sync();  // peers may still read this CTA's staged rows
   tc::fence_before_sync();
   __syncthreads();
-  if (warp == 1) tc::tmem_dealloc(tmem, 256);
-}
-
-// Merge of the key splits (fixed order): out[tok, j, :] = sum_z e^(m_z - M) O_z /
-// sum_z e^(m_z - M) l_z  (m in log2 units).  One warp per (token, head).
-__global__ void attn_combine_kernel(const float* __restrict__ part_o,
-                                    const float* __restrict__ part_ml, int splits, int ntok,
-                                    int Hq, bf16* __restrict__ out) {
-  pdl_enter();
-  const int lane = threadIdx.x & 31;
-  const long w = (long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (w >= (long)ntok * Hq) return;
-  float M = -INFINITY;
-  for (int z = 0; z < splits; ++z) M = fmaxf(M, part_ml[((size_t)z * ntok * Hq + w) * 2]);
-  float L = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int z = 0; z < splits; ++z) {
-    const float mz = part_ml[((size_t)z * ntok * Hq + w) * 2];
-    if (mz == -INFINITY) continue;
-    const float s = exp2f(mz - M);
-    L += s * part_ml[((size_t)z * ntok * Hq + w) * 2 + 1];
-    const float4 v = reinterpret_cast<const float4*>(part_o + ((size_t)z * ntok * Hq + w) * 128)[lane];
-    acc[0] += s * v.x;
-    acc[1] += s * v.y;
-    acc[2] += s * v.z;
-    acc[3] += s * v.w;
-  }
-  const float inv = L > 0.f ? 1.f / L : 0.f;
-  __nv_bfloat162 a = __floats2bfloat162_rn(acc[0] * inv, acc[1] * inv);
-  __nv_bfloat162 c = __floats2bfloat162_rn(acc[2] * inv, acc[3] * inv);
-  uint2 pk = make_uint2(*reinterpret_cast<uint32_t*>(&a), *reinterpret_cast<uint32_t*>(&c));
-  reinterpret_cast<uint2*>(out + (size_t)w * 128)[lane] = pk;
+  if (warp == 1) tc::tmem_dealloc(tmem, 512);
 }
 
 }  // namespace dg

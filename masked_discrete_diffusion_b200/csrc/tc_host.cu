@@ -390,25 +390,22 @@ dg_status tc_attention(dg_model* m, const bf16* q, int B, int nq, int qpos0, con
   p.window = c.window;
   p.B = B;
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)h));
-  p.part_o = (float*)m->ws.attn_o;
-  p.part_ml = (float*)m->ws.attn_ml;
+  p.out = out;
   const int TA = ceil_div_i(p.nA, AT_KT), TB = ceil_div_i(nB, AT_KT);
   const int total = causal ? std::min(TB, ceil_div_i(c.window + 127, AT_KT) + 1) : TA + TB;
   const int qtiles = ceil_div_i(nq, 128);
   const int base = qtiles * Hq * B;
   const int n_sm = state(m)->n_sm;
-  // one wave: CTAs (one per SM, ~194 KB of shared memory each) never exceed the SM count
-  int splits = std::min(std::max(1, n_sm / base), std::min((int)ATT_MAX_SPLITS, total));
-  splits = std::max(1, splits);
-  const int tps = ceil_div_i(total, splits);
-  splits = ceil_div_i(total, tps);
-  p.tiles_per_split = tps;
+  // one wave: CTAs (one per SM, ~196 KB of shared memory each) never exceed the SM
+  // count; the key splits of a query tile form a cluster (a power of two <= 8, so
+  // that each owns 128 / splits rows of the merge)
+  const int cap = std::min(std::max(1, n_sm / base), std::min((int)ATT_MAX_SPLITS, total));
+  int splits = 1;
+  while (splits * 2 <= cap) splits *= 2;
+  p.tiles_per_split = ceil_div_i(total, splits);
   dim3 grid(qtiles * Hq, B, splits);
-  launch_pdl((tc_attn_kernel), grid, 128, AT_SMEM, st, 1, mQ, mKA, mVA, mKB, mVB, p, m->ws.err);
-  ++m->launches;
-  const int ntok = B * nq;
-  launch_pdl((attn_combine_kernel), ceil_div_i((long)ntok * Hq, 4), 128, 0, st, 1, 
-      p.part_o, p.part_ml, splits, ntok, Hq, out);
+  launch_pdl((tc_attn_kernel), grid, AT_THREADS, AT_SMEM, st, splits, mQ, mKA, mVA, mKB, mVB, p,
+             m->ws.err);
   ++m->launches;
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
