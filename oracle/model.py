@@ -25,11 +25,12 @@ FP8) and widened to fp64; every activation and reduction is fp64.  Per-row
 entropies are rounded to fp32 at the end, which is the precision the sampler
 decides in.
 
-Storage variant (Weights(..., storage="bf16")): the same forward with the
-activations that a bf16 model keeps in memory rounded to bf16 where they are
-stored (normalised rows entering a projection, q / k / v after RoPE, the
-attention output, the SwiGLU hidden rows); residual stream, router and every
-sum stay fp64.  It measures how far bf16 storage alone moves the outputs of a
+Storage variant (Weights(..., storage="bf16")): the same forward with every
+tensor a bf16 model multiplies kept in bf16: the activations rounded where they
+are stored (normalised rows entering a projection, q / k / v after RoPE, the
+attention output, the SwiGLU hidden rows) and FP8 expert weights dequantised to
+bf16 (bf16 weights are already exact); residual stream, router and every sum
+stay fp64.  It measures how far bf16 storage alone moves the outputs of a
 workload (its sensitivity), from which the tolerances of the deep workloads are
 derived.
 """
@@ -81,7 +82,8 @@ class Weights:
     def _load(self, name, shape, start_row=0, n_rows=None) -> np.ndarray:
         if model_inputs.is_fp8_expert(self.w, name):
             from synth import fp8
-            return fp8.dequantised(self.w, name, shape, start_row, n_rows).astype(np.float64)
+            a = fp8.dequantised(self.w, name, shape, start_row, n_rows).astype(np.float64)
+            return self.store(a)
         t = model_inputs.weight(self.w, name, shape, "cpu", start_row, n_rows)
         return t.to(torch.float64).numpy()
 

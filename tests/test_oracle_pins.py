@@ -446,3 +446,14 @@ def test_bf16_storage_variant():
     assert 0 < np.abs(h2 - h0).max() < 2e-2 * np.abs(h0).max()
     with pytest.raises(ValueError):
         model.Weights(w, storage="fp16")
+
+
+def test_bf16_storage_rounds_dequantised_fp8_weights():
+    """In the storage variant FP8 expert weights enter as bf16 values (code * scale
+    rounded); the fp64 oracle keeps code * scale exactly."""
+    w = workloads.SMALL_FP8
+    exact = model.Weights(w, keep_layers=True).layer(0).expert(1)[0]
+    s16 = model.Weights(w, keep_layers=True, storage="bf16").layer(0).expert(1)[0]
+    assert np.array_equal(model.round_bf16(exact), s16)
+    assert not np.array_equal(exact, s16)
+    assert np.all(np.abs(s16 - exact) <= 2.0 ** -8 * np.abs(exact))   # unit roundoff, 8 bits
