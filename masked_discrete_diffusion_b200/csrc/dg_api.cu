@@ -170,10 +170,20 @@ template <class Path> static dg_status alloc_workspace(dg_model* m) {
     DG_TRY_CUDA(cudaEventCreateWithFlags(&m->fork_ev, cudaEventDisableTiming));
     DG_TRY_CUDA(cudaEventCreateWithFlags(&m->join_ev, cudaEventDisableTiming));
   }
-  const size_t perm_smem = (size_t)33 * c.n_experts * sizeof(int);
-  if (perm_smem > 48 * 1024)
-    DG_TRY_CUDA(cudaFuncSetAttribute(moe_permute_kernel<Acc>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)perm_smem));
+  DG_REQUIRE(permute_smem_bytes(c.n_experts, 1024, 0) <= PERMUTE_FUSED_SMEM,
+             "n_experts too large for the permutation");
+  DG_TRY_CUDA(cudaFuncSetAttribute(moe_permute_gather_kernel<Acc, TA>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)PERMUTE_FUSED_SMEM));
+  DG_TRY_CUDA(cudaFuncSetAttribute(moe_permute_kernel<Acc>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)PERMUTE_FUSED_SMEM));
+  {
+    int dev = 0, n_sm = 0;
+    DG_TRY_CUDA(cudaGetDevice(&dev));
+    DG_TRY_CUDA(cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev));
+    m->n_sm_cache = n_sm;
+  }
   DG_TRY_CUDA(cudaDeviceSynchronize());
   return DG_OK;
 }
@@ -304,6 +314,10 @@ template <class Path> struct Runner {
     // CUDA-core router, the two-term split for the tensor-core router)
     bool tc_router = false;
     if constexpr (Path::kTensorCores) tc_router = E <= 128 && k <= 8 && d % 64 == 0;
+    int bm = SG_BM;
+    if constexpr (Path::kTensorCores) bm = tc_group_rows();
+    PermuteArgs pa{(const int32_t*)ws.ridx, n_ent, k, E, bm, ws.rank, ws.offsets, ws.tile_e,
+                   ws.tile_m0, ws.n_tiles, ws.max_tiles, ws.units, load, ws.row_of, ws.tok_of};
     launch_pdl((rmsnorm_kernel<TR, TA, Acc>), n, 256, 0, st, 1, x(), xn(), n, d, c.rms_eps,
                (Acc*)ws.inv_rms, tc_router ? (TA*)ws.u2 : (TA*)nullptr);
     ++m->launches;
@@ -345,16 +359,21 @@ template <class Path> struct Runner {
             (int32_t*)nullptr);
       ++m->launches;
     }
-    int bm = SG_BM;
-    if constexpr (Path::kTensorCores) bm = tc_group_rows();
-    launch_pdl((moe_permute_kernel<Acc>), 1, 1024, (size_t)33 * E * sizeof(int), st, 1,
-               (const int32_t*)ws.ridx, (const Acc*)ws.rgate, n_ent, k, E, bm, ws.rank, ws.offsets,
-               ws.tile_e, ws.tile_m0, ws.n_tiles, ws.max_tiles, ws.units, load, ws.row_of,
-               ws.tok_of, (Acc*)ws.gate_of);
-    ++m->launches;
-    launch_pdl((gather_rows_kernel<TA>), n_ent, 256, 0, st, 1, xn(), ws.tok_of, ws.offsets + E, d,
-                                                  (TA*)ws.up);
-    ++m->launches;
+    if (permute_smem_bytes(E, 1024, n_ent) <= PERMUTE_FUSED_SMEM) {
+      // every block derives the permutation in shared memory and gathers its rows
+      const int blocks = std::max(1, std::min(n_ent, m->n_sm_cache));
+      launch_pdl((moe_permute_gather_kernel<Acc, TA>), blocks, 1024,
+                 permute_smem_bytes(E, 1024, n_ent), st, 1, pa, (const Acc*)ws.rgate,
+                 (Acc*)ws.gate_of, (const TA*)xn(), d, (TA*)ws.up);
+      ++m->launches;
+    } else {
+      launch_pdl((moe_permute_kernel<Acc>), 1, 1024, permute_smem_bytes(E, 1024, 0), st, 1, pa,
+                 (const Acc*)ws.rgate, (Acc*)ws.gate_of);
+      ++m->launches;
+      launch_pdl((gather_rows_kernel<TA>), n_ent, 256, 0, st, 1, xn(), ws.tok_of,
+                 ws.offsets + E, d, (TA*)ws.up);
+      ++m->launches;
+    }
     const int grid_y = ceil_div(n_ent, bm) + E;
     if constexpr (Path::kTensorCores) {
       {

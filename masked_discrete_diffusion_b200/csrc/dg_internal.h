@@ -72,6 +72,9 @@ inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
 // Device error bits (set by kernels, read and cleared by dg_sync_status).
 enum : int { ERR_BAD_TOKEN = 1, ERR_TIMEOUT = 2, ERR_BAD_SHAPE = 4 };
 constexpr int ATT_MAX_SPLITS = 8;
+// shared memory of the fused permutation + gather (ranks and row tokens of all
+// (token, slot) entries kept on chip); above it the two steps run separately
+constexpr size_t PERMUTE_FUSED_SMEM = 200 * 1024;
 
 // A typed device allocation owned by the workspace.
 struct DevBuf {
@@ -150,6 +153,7 @@ struct dg_model {
   // second stream for the shared expert, forked after the MoE RMSNorm and joined
   // before the combine (concurrent graph branches when captured)
   cudaStream_t side_stream = nullptr;
+  int n_sm_cache = 148;  // multiprocessors of the model's device
   cudaEvent_t fork_ev = nullptr, join_ev = nullptr;
   long long last_body_launches = 0;   // kernels per forward of the last replayed loop graph
   std::vector<dg_kv*> kvs;            // live KV caches created from this model

@@ -538,88 +538,144 @@ static __global__ void __launch_bounds__(1024)
       }
 }
 
-// The whole permutation in one block of 1024 threads (E <= 1024): ranks by
-// warp-level match + per-(warp, expert) counts scanned in warp order (entry
-// order is kept within an expert), counts, offsets, the tile table, the
-// streamed-expert counter, per-expert load, and the scatter of (row, token,
-// gate).  Dynamic shared memory: (32 + 1) * E ints.
+// The whole permutation of the (token, slot) entries into expert-contiguous rows,
+// by one block (any multiple of 32 threads <= 1024): ranks by warp-level match
+// plus per-(warp, expert) counts scanned in warp order (entry order is kept within
+// an expert), counts, offsets, the tile table (bm rows per tile), the
+// streamed-expert counter, per-expert load, and the scatter of (row, token, gate).
+// Shared memory `psm`: (32 + 1) * E + 2 * blockDim.x ints.  rank [n_entries] and
+// tok [n_entries] (the token of every permuted row) are the caller's (shared or
+// global memory); `write` selects the block that stores the permutation.
+struct PermuteArgs {
+  const int32_t* idx;
+  int n_entries, top_k, E, bm;
+  int32_t *rank, *offsets, *tile_e, *tile_m0, *n_tiles;
+  int max_tiles;
+  unsigned long long* used;
+  int32_t *load, *row_of, *tok_of;
+};
+
 template <class Acc>
-__global__ void __launch_bounds__(1024)
-    moe_permute_kernel(const int32_t* __restrict__ idx, const Acc* __restrict__ gate,
-                       int n_entries, int top_k, int E, int bm, int32_t* __restrict__ rank,
-                       int32_t* __restrict__ offsets, int32_t* __restrict__ tile_e,
-                       int32_t* __restrict__ tile_m0, int32_t* __restrict__ n_tiles,
-                       int max_tiles, unsigned long long* __restrict__ used,
-                       int32_t* __restrict__ load, int32_t* __restrict__ row_of,
-                       int32_t* __restrict__ tok_of, Acc* __restrict__ gate_of) {
-  pdl_enter();
-  extern __shared__ int psm[];
-  int* hist = psm;            // [32][E]: counts, then exclusive offsets per warp
-  int* carry = psm + 32 * E;  // [E]: entries of each expert in earlier chunks
-  __shared__ int sc[1024], stl[1024];
+__device__ void block_permute(const PermuteArgs& a, const Acc* __restrict__ gate,
+                              Acc* __restrict__ gate_of, int* psm, int* rank, int* tok,
+                              bool write) {
+  const int E = a.E, nthr = blockDim.x, nw = nthr >> 5;
+  int* hist = psm;             // [nw][E]: counts, then exclusive offsets per warp
+  int* carry = psm + 32 * E;   // [E]: entries of each expert in earlier chunks, then offsets
+  int* sc = carry + E;         // [nthr] scan scratch (entries)
+  int* stl = sc + nthr;        // [nthr] scan scratch (tiles)
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-  for (int e = tid; e < E; e += blockDim.x) carry[e] = 0;
-  for (int base = 0; base < n_entries; base += blockDim.x) {
-    for (int i = tid; i < 32 * E; i += blockDim.x) hist[i] = 0;
+  for (int e = tid; e < E; e += nthr) carry[e] = 0;
+  for (int base = 0; base < a.n_entries; base += nthr) {
+    for (int i = tid; i < nw * E; i += nthr) hist[i] = 0;
     __syncthreads();
     const int j = base + tid;
-    const bool valid = j < n_entries;
-    const int e = valid ? idx[j] : -1;
+    const bool valid = j < a.n_entries;
+    const int e = valid ? __ldcg(a.idx + j) : -1;  // written by other blocks: read at L2
     const unsigned same = __match_any_sync(0xffffffffu, e);
     const int before = __popc(same & ((1u << lane) - 1u));
     if (valid && before == 0) hist[w * E + e] = __popc(same);
     __syncthreads();
-    for (int e2 = tid; e2 < E; e2 += blockDim.x) {
-      int s = carry[e2];
-      for (int w2 = 0; w2 < 32; ++w2) {
+    for (int e2 = tid; e2 < E; e2 += nthr) {
+      int s0 = carry[e2];
+      for (int w2 = 0; w2 < nw; ++w2) {
         const int c = hist[w2 * E + e2];
-        hist[w2 * E + e2] = s;
-        s += c;
+        hist[w2 * E + e2] = s0;
+        s0 += c;
       }
-      carry[e2] = s;
+      carry[e2] = s0;
     }
     __syncthreads();
     if (valid) rank[j] = hist[w * E + e] + before;
     __syncthreads();
   }
-  // counts -> offsets and tile table (inclusive scans over 1024 slots)
-  const int e = tid;
-  const int c = e < E ? carry[e] : 0;
-  const unsigned bal = __ballot_sync(0xffffffffu, c > 0);
-  if (used && lane == 0 && bal) atomicAdd(used, (unsigned long long)__popc(bal));
-  if (load && e < E) load[e] += c;
-  const int nt = (c + bm - 1) / bm;
-  sc[e] = c;
-  stl[e] = nt;
+  // counts -> offsets and tile table: thread t scans experts [t * per, t * per + per)
+  const int per = (E + nthr - 1) / nthr, e0 = tid * per;
+  int c_sum = 0, t_sum = 0, used_n = 0;
+  for (int e = e0; e < min(E, e0 + per); ++e) {
+    const int c = carry[e];
+    c_sum += c;
+    t_sum += (c + a.bm - 1) / a.bm;
+    used_n += c > 0;
+    if (write && a.load) a.load[e] += c;
+  }
+  if (write && a.used && used_n) atomicAdd(a.used, (unsigned long long)used_n);
+  sc[tid] = c_sum;
+  stl[tid] = t_sum;
   __syncthreads();
-  for (int off = 1; off < 1024; off <<= 1) {
-    const int a = e >= off ? sc[e - off] : 0, b = e >= off ? stl[e - off] : 0;
+  for (int off = 1; off < nthr; off <<= 1) {  // inclusive scans over the threads
+    const int x = tid >= off ? sc[tid - off] : 0, y = tid >= off ? stl[tid - off] : 0;
     __syncthreads();
-    sc[e] += a;
-    stl[e] += b;
+    sc[tid] += x;
+    stl[tid] += y;
     __syncthreads();
   }
-  const int off_e = sc[e] - c, t_e = stl[e] - nt;
-  if (e < E) {
-    offsets[e] = off_e;
+  int off_e = sc[tid] - c_sum, t_e = stl[tid] - t_sum;
+  for (int e = e0; e < min(E, e0 + per); ++e) {
+    const int c = carry[e], nt = (c + a.bm - 1) / a.bm;
     carry[e] = off_e;
+    if (write) {
+      a.offsets[e] = off_e;
+      for (int r = 0; r < nt; ++r)
+        if (t_e + r < a.max_tiles) {
+          a.tile_e[t_e + r] = e;
+          a.tile_m0[t_e + r] = off_e + r * a.bm;
+        }
+    }
+    off_e += c;
+    t_e += nt;
   }
-  if (e == E - 1) {
-    offsets[E] = off_e + c;
-    *n_tiles = min(t_e + nt, max_tiles);
+  if (write && tid == nthr - 1) {
+    a.offsets[E] = sc[tid];
+    *a.n_tiles = min(stl[tid], a.max_tiles);
   }
-  if (e < E)
-    for (int r = 0; r < nt; ++r)
-      if (t_e + r < max_tiles) {
-        tile_e[t_e + r] = e;
-        tile_m0[t_e + r] = off_e + r * bm;
-      }
   __syncthreads();
-  for (int j = tid; j < n_entries; j += blockDim.x) {
-    const int pos = carry[idx[j]] + rank[j];
-    row_of[j] = pos;
-    tok_of[pos] = j / top_k;
-    gate_of[pos] = gate[j];
+  for (int j = tid; j < a.n_entries; j += nthr) {
+    const int pos = carry[__ldcg(a.idx + j)] + rank[j];
+    tok[pos] = j / a.top_k;
+    if (write) {
+      a.row_of[j] = pos;
+      a.tok_of[pos] = j / a.top_k;
+      gate_of[pos] = __ldcg(gate + j);
+    }
+  }
+  __syncthreads();
+}
+
+inline size_t permute_smem_bytes(int E, int threads, int n_entries_in_smem) {
+  return ((size_t)33 * E + 2 * (size_t)threads + 2 * (size_t)n_entries_in_smem) * sizeof(int);
+}
+
+// The permutation alone (one block; rank scratch and tok_of in global memory), for
+// entry counts whose ranks do not fit in shared memory.
+template <class Acc>
+__global__ void __launch_bounds__(1024)
+    moe_permute_kernel(PermuteArgs a, const Acc* __restrict__ gate, Acc* __restrict__ gate_of) {
+  pdl_enter();
+  extern __shared__ int psm[];
+  block_permute(a, gate, gate_of, psm, a.rank, a.tok_of, true);
+}
+
+// Permutation and gather in one launch: every block derives the permutation (so that
+// no block waits for another), block 0 stores it, and block z copies its share of
+// the permuted rows dst[r] = src[token of row r] (rows of d elements, 16-byte units).
+template <class Acc, class TA>
+__global__ void __launch_bounds__(1024)
+    moe_permute_gather_kernel(PermuteArgs a, const Acc* __restrict__ gate,
+                              Acc* __restrict__ gate_of, const TA* __restrict__ src, int d,
+                              TA* __restrict__ dst) {
+  pdl_enter();
+  extern __shared__ int psm[];
+  int* rank = psm + 33 * a.E + 2 * blockDim.x;
+  int* tok = rank + a.n_entries;
+  block_permute(a, gate, gate_of, psm, rank, tok, blockIdx.x == 0);
+  const int units = d * (int)sizeof(TA) / 16;  // 16-byte units per row
+  const int per = (a.n_entries + gridDim.x - 1) / gridDim.x;
+  const int r0 = blockIdx.x * per, r1 = min(a.n_entries, r0 + per);
+  for (long u = threadIdx.x; u < (long)(r1 - r0) * units; u += blockDim.x) {
+    const int r = r0 + (int)(u / units), c = (int)(u % units);
+    reinterpret_cast<uint4*>(dst + (size_t)r * d)[c] =
+        reinterpret_cast<const uint4*>(src + (size_t)tok[r] * d)[c];
   }
 }
 

@@ -2,6 +2,12 @@
 the same 30-layer model; oracle values for canvases 0 and 7 from
 tests/golden/full30-b8-p8192[-c7].npz (written by make_golden.py from the oracle).
 
+Tolerances as for the single-canvas 30-layer workload (test_gpu_full30): 2e-2 on
+layer 0's keys and values; layer 29's K/V, logits and entropies within twice the
+distance between the oracle's bf16-storage and fp64 runs, taken from the
+single-canvas golden (the same weights and depth; the bf16-storage run of an
+8192-token prompt is not stored).
+
 Also checks the per-expert router load the block reports (every routed row of
 every forward counted once) and the block's properties at this size.
 """
@@ -14,18 +20,19 @@ import torch
 
 from synth import model_inputs, workloads
 
-from gpu_helpers import make_model, max_abs_rel
+from gpu_helpers import make_model, max_abs_rel, storage_tol
 
 pytestmark = pytest.mark.gpu
 W = workloads.FULL30_B8_P8192
 TOL = 2e-2
 HERE = os.path.join(os.path.dirname(__file__), "golden")
 GOLD = {0: os.path.join(HERE, "full30-b8-p8192.npz"), 7: os.path.join(HERE, "full30-b8-p8192-c7.npz")}
+SENS = os.path.join(HERE, "full30-bf16.npz")
 
 
 @pytest.fixture(scope="module")
 def run():
-    if not all(os.path.exists(p) for p in GOLD.values()):
+    if not all(os.path.exists(p) for p in list(GOLD.values()) + [SENS]):
         pytest.skip("golden files missing")
     from masked_discrete_diffusion_b200 import binding
     model = make_model(W)
@@ -37,6 +44,7 @@ def run():
     k, v = binding.dg_kv_read(kv)
     binding.dg_sync_status(model)
     out = {"binding": binding, "model": model, "kv": kv, "ent": ent.cpu().numpy(),
+           "sens": np.load(SENS),
            "ent2": ent2.cpu().numpy(), "am2": am2.cpu().numpy(), "per": {}}
     lg = lg.reshape(W.batch, W.canvas, W.vocab)
     for b, path in GOLD.items():
@@ -55,13 +63,14 @@ def run():
 @pytest.mark.parametrize("b", [0, 7])
 def test_canvas_against_oracle(run, b):
     p = run["per"][b]
-    g = p["g"]
-    for i in range(2):
-        assert max_abs_rel(p["k"][i], g["kv_last"][i, 0]) < TOL
-        assert max_abs_rel(p["v"][i], g["kv_last"][i, 1]) < TOL
-    assert max_abs_rel(p["lg"], g["logits"]) < TOL
-    assert max_abs_rel(run["ent"][b], g["H"]) < TOL
-    assert max_abs_rel(run["ent2"][b], g["H"]) < TOL
+    g, sens = p["g"], run["sens"]
+    assert max_abs_rel(p["k"][0], g["kv_last"][0, 0]) < TOL
+    assert max_abs_rel(p["v"][0], g["kv_last"][0, 1]) < TOL
+    assert max_abs_rel(p["k"][1], g["kv_last"][1, 0]) < storage_tol(sens, "kv_last", TOL, (1, 0))
+    assert max_abs_rel(p["v"][1], g["kv_last"][1, 1]) < storage_tol(sens, "kv_last", TOL, (1, 1))
+    assert max_abs_rel(p["lg"], g["logits"]) < storage_tol(sens, "logits", TOL)
+    assert max_abs_rel(run["ent"][b], g["H"]) < storage_tol(sens, "H", TOL)
+    assert max_abs_rel(run["ent2"][b], g["H"]) < storage_tol(sens, "H", TOL)
     eps = float(np.abs(p["lg"] - g["logits"]).max())
     decided = g["margin"] > 2 * eps + 1e-3
     assert np.array_equal(run["am2"][b][decided], g["argmax"][decided])
@@ -73,7 +82,9 @@ def test_block_and_router_load(run):
     load = torch.zeros(W.n_layers, W.n_experts, dtype=torch.int32, device="cuda")
     out = b.dg_generate_block(model, kv, W.T, W.gamma, n_forwards=nf, router_load=load)
     b.dg_sync_status(model)
-    assert not (out == W.mask_id).any() and nf.cpu().tolist() == [W.T] * W.batch
+    nfl = nf.cpu().tolist()
+    assert not (out == W.mask_id).any() and all(1 <= f <= W.T for f in nfl)
+    # every forward the loop ran routes every row of every canvas
     per_layer = load.sum(dim=1).cpu().tolist()
-    assert per_layer == [W.batch * W.canvas * W.top_k * W.T] * W.n_layers
+    assert per_layer == [W.batch * W.canvas * W.top_k * max(nfl)] * W.n_layers
     assert np.all(run["ent2"] >= 0) and np.all(run["ent2"] <= math.log(W.vocab) + 1e-3)

@@ -14,7 +14,7 @@ import torch
 from oracle import model as om
 from synth import gen, model_inputs, workloads
 
-from gpu_helpers import make_model, max_abs_rel
+from gpu_helpers import make_model, max_abs_rel, storage_tol
 
 pytestmark = pytest.mark.gpu
 TOL = 3e-2
@@ -107,8 +107,11 @@ def test_fp8_full_size_layer():
         cols = torch.as_tensor(g["logit_cols"]).cuda()
         lgs = lg[rows][:, cols].cpu().numpy()
         assert max_abs_rel(lgs, g["logits"]) < TOL
-        assert max_abs_rel(ent2[0].cpu().numpy(), g["H"]) < TOL
-        assert max_abs_rel(ent[0].cpu().numpy(), g["H"]) < TOL
+        # entropies: no stated tolerance; twice the oracle's bf16-storage distance
+        # (bf16 activations and the FP8 weights dequantised to bf16), at least TOL
+        tol_h = storage_tol(g, "H", TOL)
+        assert max_abs_rel(ent2[0].cpu().numpy(), g["H"]) < tol_h
+        assert max_abs_rel(ent[0].cpu().numpy(), g["H"]) < tol_h
         assert max_abs_rel(k[0, 0, :, -8:].float().cpu().numpy(), g["kv_last"][0, 0]) < TOL
         eps = float(np.abs(lgs - g["logits"]).max())
         decided = g["margin"] > 2 * eps + 1e-3
