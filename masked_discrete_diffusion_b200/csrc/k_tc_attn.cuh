@@ -108,7 +108,6 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   const uint32_t tmem = *tslot;
   const uint32_t tO = tmem + 256;  // S buffers at columns 0 and 128
   const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
-  pdl_enter();  // global memory is touched only from here on
 
   auto load_tile = [&](int i) {  // tile index i within this split -> stage i & 1
     const int t = my_lo + i;
@@ -157,14 +156,22 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     return __syncthreads_and(ok_ ? 1 : 0) != 0;
   };
 
+  // the cached prompt window (segment A) was written before this forward began, so its
+  // first tiles are requested before the preceding kernel has finished
+  const int n_first = min(nt, 2);
+  if (tid == 0)
+    for (int i = 0; i < n_first; ++i)
+      if (my_lo + i < TA) load_tile(i);
+  pdl_enter();  // q and the pass's own keys / values are read only from here on
+
   bool ok = true;
   if (tid == 0 && nt > 0) {
     tc::mbar_expect_tx(q_full, 2 * AT_SUB);
     const int qrow = b * p.nq + q0;
     tc::tma_load_2d(sQ, &mQ, q_full, j * 128, qrow);
     tc::tma_load_2d(sQ + AT_SUB, &mQ, q_full, j * 128 + 64, qrow);
-    load_tile(0);
-    if (nt > 1) load_tile(1);
+    for (int i = 0; i < n_first; ++i)
+      if (my_lo + i >= TA) load_tile(i);
     if (!issue_s(0)) atomicOr(err, ERR_TIMEOUT);
   }
 

@@ -370,9 +370,11 @@ template <int BN, int MT, bool DUAL, int ST, class Epi>
 __global__ void __launch_bounds__(TC_DENSE_THREADS, 1)
     tc_dense_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mB,
                     const __grid_constant__ CUtensorMap mB2, int M, int K, int ksplit, Epi epi,
-                    int32_t* err, int kwrap) {
+                    int32_t* err, int kwrap, int b_early) {
   // kwrap > 0: the B operand's K coordinate is taken modulo kwrap (A = [a1 | a2]
-  // against B = [w | w] without storing w twice)
+  // against B = [w | w] without storing w twice).
+  // b_early != 0: B is a model weight, constant while the model runs, so its first
+  // stages are requested before the preceding kernel has finished.
   typedef DenseCfg<BN, MT, DUAL, ST> Cfg;
   // staged epilogues reuse the drained pipeline buffers for the fp32 tile
   constexpr int RS = Cfg::NACC * BN + 4;  // staging row stride (floats): padded against bank conflicts
@@ -406,12 +408,32 @@ __global__ void __launch_bounds__(TC_DENSE_THREADS, 1)
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tslot;
-  pdl_enter();  // global memory is touched only from here on
+  // CTAs start their K walk at different offsets so that they do not all read the
+  // same activation tile from the same L2 slices at the same time
+  auto kcoord = [&](int kb) { return (kb_lo + (kb + rot) % nk) * TC_KB; };
+  auto load_b = [&](int kb, int s) {
+    const int kx = kcoord(kb), kxb = kwrap > 0 ? kx % kwrap : kx;
+    uint8_t* st = smem + s * Cfg::STAGE;
+    tc::tma_load_2d(st + MT * TC_SUB_A, &mB, full + s, kxb, n0);
+    if (DUAL) tc::tma_load_2d(st + MT * TC_SUB_A + Cfg::B_BYTES, &mB2, full + s, kxb, n0);
+  };
+  const int early = b_early ? min(ST, nk) : 0;
+  if (warp == 0 && lane == 0 && early > 0) {
+    tc::prefetch_tmap(&mB);
+    if (DUAL) tc::prefetch_tmap(&mB2);
+    for (int kb = 0; kb < early; ++kb) {
+      tc::mbar_expect_tx(full + kb, Cfg::STAGE);  // the whole stage: B now, A below
+      load_b(kb, kb);
+    }
+  }
+  pdl_enter();  // the activations (A) are read only from here on
 
   if (warp == 0 && lane == 0) {
     tc::prefetch_tmap(&mA);
-    tc::prefetch_tmap(&mB);
-    if (DUAL) tc::prefetch_tmap(&mB2);
+    if (early == 0) {
+      tc::prefetch_tmap(&mB);
+      if (DUAL) tc::prefetch_tmap(&mB2);
+    }
     for (int kb = 0; kb < nk; ++kb) {
       const int s = kb % ST;
       const uint32_t ph = (kb / ST) & 1;
@@ -421,16 +443,14 @@ __global__ void __launch_bounds__(TC_DENSE_THREADS, 1)
         break;
       }
       uint8_t* st = smem + s * Cfg::STAGE;
-      tc::mbar_expect_tx(full + s, Cfg::STAGE);
-      // CTAs start their K walk at different offsets so that they do not all read
-      // the same activation tile from the same L2 slices at the same time
-      const int kx = (kb_lo + (kb + rot) % nk) * TC_KB;
-      const int kxb = kwrap > 0 ? kx % kwrap : kx;
+      if (kb >= early) {
+        tc::mbar_expect_tx(full + s, Cfg::STAGE);
+        load_b(kb, s);
+      }
+      const int kx = kcoord(kb);
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt)
         tc::tma_load_2d(st + mt * TC_SUB_A, &mA, full + s, kx, m0 + mt * 128);
-      tc::tma_load_2d(st + MT * TC_SUB_A, &mB, full + s, kxb, n0);
-      if (DUAL) tc::tma_load_2d(st + MT * TC_SUB_A + Cfg::B_BYTES, &mB2, full + s, kxb, n0);
     }
   } else if (warp == 1 && lane == 0) {
     constexpr uint32_t idesc = tc::idesc_bf16(128, BN);

@@ -103,7 +103,7 @@ template <class K> dg_status set_smem(K kern, size_t bytes) {
 template <int BN, int MT, bool DUAL, int ST, class Epi>
 dg_status launch_dense(dg_model* m, const CUtensorMap& a, const CUtensorMap& b,
                        const CUtensorMap& b2, int M, int N, int K, Epi epi, cudaStream_t st,
-                       bool allow_split = true, int kwrap = 0) {
+                       bool allow_split = true, int kwrap = 0, bool b_weight = true) {
   typedef DenseCfg<BN, MT, DUAL, ST> Cfg;
   auto kern = tc_dense_kernel<BN, MT, DUAL, ST, Epi>;
   dim3 grid(ceil_div_i(M, 128 * MT), ceil_div_i(N, BN), 1);
@@ -114,10 +114,12 @@ dg_status launch_dense(dg_model* m, const CUtensorMap& a, const CUtensorMap& b,
     while (ks < 8 && tiles * ks * 2 <= state(m)->n_sm && nk >= ks * 2 * 2) ks *= 2;
   cudaError_t e;
   if (ks == 1) {
-    e = launch_pdl(kern, grid, TC_DENSE_THREADS, Cfg::SMEM, st, 1, a, b, b2, M, K, 1, epi, m->ws.err, kwrap);
+    e = launch_pdl(kern, grid, TC_DENSE_THREADS, Cfg::SMEM, st, 1, a, b, b2, M, K, 1, epi,
+                   m->ws.err, kwrap, b_weight ? 1 : 0);
   } else {
     grid.z = ks;
-    e = launch_pdl(kern, grid, TC_DENSE_THREADS, Cfg::SMEM, st, ks, a, b, b2, M, K, ks, epi, m->ws.err, kwrap);
+    e = launch_pdl(kern, grid, TC_DENSE_THREADS, Cfg::SMEM, st, ks, a, b, b2, M, K, ks, epi,
+                   m->ws.err, kwrap, b_weight ? 1 : 0);
   }
   ++m->launches;
   if (e != cudaSuccess) {
@@ -240,8 +242,10 @@ dg_status tc_gemm_f32_rows(dg_model* m, const bf16* A, int a_rows, const void* W
   CUtensorMap a, b;
   DG_TRY(tmap(m, A, a_rows, K, 128, &a));
   DG_TRY(tmap(m, W, N, K, DENSE_BN, &b));
+  // W is the caller's tensor, not a model weight: read only after the dependency wait
   return launch_dense<DENSE_BN, DENSE_MT, false, DENSE_ST>(m, a, b, b, M, N, K,
-                                                           EpiStoreF32{out, N, N}, st);
+                                                           EpiStoreF32{out, N, N}, st, true, 0,
+                                                           false);
 }
 
 dg_status tc_gemm_add_residual(dg_model* m, const bf16* A, const void* W, float* x, int M, int N,
