@@ -14,6 +14,8 @@ Each file <workload>[-c<canvas>].npz holds, for one canvas of the workload's fir
 With the suffix "+s16" the file also holds the same outputs of the oracle's bf16
 storage variant (H_s16, argmax_s16, logits_s16, kv_last_s16): the sensitivity of the
 workload to bf16 activation storage, from which the deep workloads' tolerances follow.
+The suffix "+s16only" adds those fields to an existing file (the fp64 run is not
+repeated).
 """
 from __future__ import annotations
 
@@ -37,6 +39,24 @@ def _kv_last(w, st):
     return np.stack([np.stack([st["kv"][l][0][-8:].transpose(1, 0, 2),
                                st["kv"][l][1][-8:].transpose(1, 0, 2)])
                      for l in sorted({0, w.n_layers - 1})])
+
+
+def add_storage_variant(name: str, canvas_index: int = 0):
+    """Adds the bf16-storage run's fields to an existing golden file."""
+    w = workloads.get(name)
+    t0 = time.time()
+    suffix = f"-c{canvas_index}" if canvas_index else ""
+    path = os.path.join(HERE, f"{name}{suffix}.npz")
+    old = dict(np.load(path))
+    prompt = model_inputs.prompt(w.with_(batch=1), first=canvas_index)[0].numpy()
+    canvas = np.full(w.canvas, w.mask_id)
+    ws16 = om.Weights(w, keep_layers=False, storage="bf16")
+    s16 = om.prefill_then_forward(ws16, prompt, canvas, w.T, w.T, want_logits=True)
+    rows, cols = old["logit_rows"], old["logit_cols"]
+    old.update(H_s16=s16["H"], argmax_s16=s16["argmax"], kv_last_s16=_kv_last(w, s16),
+               logits_s16=s16["logits"][rows][:, cols].astype(np.float64))
+    np.savez_compressed(path, **old)
+    print(f"{name}{suffix}: added the bf16-storage run in {time.time() - t0:.0f} s")
 
 
 def make(name: str, canvas_index: int = 0, storage_variant: bool = False):
@@ -77,8 +97,12 @@ def make(name: str, canvas_index: int = 0, storage_variant: bool = False):
 
 if __name__ == "__main__":
     # arguments: workload names, optionally "name:canvas" to pick a canvas of the batch
-    # and the suffix "+s16" for the bf16 storage variant as well
+    # and the suffix "+s16" for the bf16 storage variant as well ("+s16only": that alone)
     for arg in sys.argv[1:] or ["layer1-bf16"]:
+        if arg.endswith("+s16only"):
+            name, _, c = arg.removesuffix("+s16only").partition(":")
+            add_storage_variant(name, int(c) if c else 0)
+            continue
         s16 = arg.endswith("+s16")
         name, _, c = arg.removesuffix("+s16").partition(":")
         make(name, int(c) if c else 0, storage_variant=s16)

@@ -4,9 +4,8 @@ tests/golden/full30-b8-p8192[-c7].npz (written by make_golden.py from the oracle
 
 Tolerances as for the single-canvas 30-layer workload (test_gpu_full30): 2e-2 on
 layer 0's keys and values; layer 29's K/V, logits and entropies within twice the
-distance between the oracle's bf16-storage and fp64 runs, taken from the
-single-canvas golden (the same weights and depth; the bf16-storage run of an
-8192-token prompt is not stored).
+distance between the oracle's bf16-storage and fp64 runs of the same canvas (stored
+in its golden file; the single-canvas workload's distances if a file lacks them).
 
 Also checks the per-expert router load the block reports (every routed row of
 every forward counted once) and the block's properties at this size.
@@ -63,7 +62,8 @@ def run():
 @pytest.mark.parametrize("b", [0, 7])
 def test_canvas_against_oracle(run, b):
     p = run["per"][b]
-    g, sens = p["g"], run["sens"]
+    g = p["g"]
+    sens = g if "H_s16" in g.files else run["sens"]
     assert max_abs_rel(p["k"][0], g["kv_last"][0, 0]) < TOL
     assert max_abs_rel(p["v"][0], g["kv_last"][0, 1]) < TOL
     assert max_abs_rel(p["k"][1], g["kv_last"][1, 0]) < storage_tol(sens, "kv_last", TOL, (1, 0))
