@@ -142,6 +142,8 @@ template <class Path> static dg_status alloc_workspace(dg_model* m) {
   DG_TRY(ws_alloc(ws, &ws.counts, c.n_experts));
   DG_TRY(ws_alloc(ws, &ws.offsets, c.n_experts + 1));
   DG_TRY(ws_alloc(ws, &ws.tile_e, ws.max_tiles));
+  DG_TRY(ws_alloc(ws, &ws.ready, ws.max_tiles));
+  DG_TRY_CUDA(cudaMemset(ws.ready, 0, ws.max_tiles * sizeof(int32_t)));
   DG_TRY(ws_alloc(ws, &ws.tile_m0, ws.max_tiles));
   DG_TRY(ws_alloc(ws, &ws.n_tiles, 1));
   DG_TRY(ws_alloc_v<TA>(ws, &ws.up, R * d));
@@ -317,7 +319,8 @@ template <class Path> struct Runner {
     int bm = SG_BM;
     if constexpr (Path::kTensorCores) bm = tc_group_rows();
     PermuteArgs pa{(const int32_t*)ws.ridx, n_ent, k, E, bm, ws.rank, ws.offsets, ws.tile_e,
-                   ws.tile_m0, ws.n_tiles, ws.max_tiles, ws.units, load, ws.row_of, ws.tok_of};
+                   ws.tile_m0, ws.n_tiles, ws.max_tiles, ws.units, load, ws.row_of, ws.tok_of,
+                   ws.ready};
     launch_pdl((rmsnorm_kernel<TR, TA, Acc>), n, 256, 0, st, 1, x(), xn(), n, d, c.rms_eps,
                (Acc*)ws.inv_rms, tc_router ? (TA*)ws.u2 : (TA*)nullptr);
     ++m->launches;
@@ -378,8 +381,12 @@ template <class Path> struct Runner {
     if constexpr (Path::kTensorCores) {
       {
         ProfScope ps(m, DG_KIND_EXPERTS, st);
-        DG_TRY(tc_moe_gate_up(m, l, (const TA*)ws.up, (TA*)ws.hb, grid_y, st));
-        DG_TRY(tc_moe_down(m, l, (const TA*)ws.hb, (float*)ws.yb, grid_y, st));
+        if (c.dtype == DG_BF16_FP8EXP) {
+          DG_TRY(tc_moe_gate_up(m, l, (const TA*)ws.up, (TA*)ws.hb, grid_y, st));
+          DG_TRY(tc_moe_down(m, l, (const TA*)ws.hb, (float*)ws.yb, grid_y, st));
+        } else {
+          DG_TRY(tc_moe_experts(m, l, (const TA*)ws.up, (TA*)ws.hb, (float*)ws.yb, st));
+        }
       }
       DG_TRY_CUDA(cudaStreamWaitEvent(st, m->join_ev, 0));  // shared expert done
     } else {

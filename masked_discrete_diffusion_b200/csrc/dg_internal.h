@@ -95,6 +95,7 @@ struct Workspace {
   void *rgate = nullptr, *gate_of = nullptr;
   void *inv_rms = nullptr, *rlog = nullptr;  // per-row 1/rms; split-K router partials
   void* u2 = nullptr;  // [rows, 2 d] two-term split of the normalised rows (tensor-core router)
+  int32_t* ready = nullptr;  // [max_tiles] phase-1 units finished per token chunk (routed experts)
   int32_t *counts = nullptr, *offsets = nullptr, *tile_e = nullptr, *tile_m0 = nullptr,
           *n_tiles = nullptr;
   void *up = nullptr, *hb = nullptr, *yb = nullptr; // routed rows

@@ -21,6 +21,13 @@ __device__ __forceinline__ void pdl_enter() {
   pdl_trigger();
 }
 
+// Load with acquire semantics at GPU scope (pairs with a writer's fence + atomic).
+__device__ __forceinline__ int ld_acquire(const int32_t* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
 __device__ __forceinline__ float widen(float x) { return x; }
 __device__ __forceinline__ float widen(bf16 x) { return __bfloat162float(x); }
 __device__ __forceinline__ double widen(double x) { return x; }

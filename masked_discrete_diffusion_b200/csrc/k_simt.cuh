@@ -553,6 +553,7 @@ struct PermuteArgs {
   int max_tiles;
   unsigned long long* used;
   int32_t *load, *row_of, *tok_of;
+  int32_t* ready;  // per-tile counters of the routed-expert kernel, zeroed here (nullable)
 };
 
 template <class Acc>
@@ -629,6 +630,8 @@ __device__ void block_permute(const PermuteArgs& a, const Acc* __restrict__ gate
     a.offsets[E] = sc[tid];
     *a.n_tiles = min(stl[tid], a.max_tiles);
   }
+  if (write && a.ready)
+    for (int t = tid; t < a.max_tiles; t += nthr) a.ready[t] = 0;
   __syncthreads();
   for (int j = tid; j < a.n_entries; j += nthr) {
     const int pos = carry[__ldcg(a.idx + j)] + rank[j];

@@ -1,8 +1,8 @@
 // Grouped routed-expert GEMM with FP8 E4M3 expert weights (one fp32 scale per
 // weight row and 128 consecutive input columns) and bf16 activations.
 //
-// Same work decomposition as tc_expert_kernel (unit = token chunk x 128 weight
-// rows, weights on the MMA's M side, tokens on N).  Per stage of 64 input columns:
+// Work unit = token chunk x 128 weight rows, weights on the MMA's M side, tokens on
+// N (as in the bf16 routed-expert kernel), gate/up and down as two launches.  Per stage of 64 input columns:
 // TMA brings the FP8 weight tile(s) [128 rows x 64 bytes] and the bf16 token rows;
 // four converter warps turn each FP8 tile into the 128-byte-swizzled bf16 tile the
 // MMA reads (value = code * scale, rounded to bf16); the MMA warp then issues

@@ -4,10 +4,11 @@
 //     from HBM once), weights as the B operand; fused epilogues: fp32 store,
 //     residual add, SwiGLU (two weight operands), and the LM-head per-row
 //     softmax statistics (the logits never leave the SM).
-//   * tc_expert_kernel — grouped routed-expert GEMM, weights as the MMA A operand
-//     (128 weight rows per tile) and the expert's gathered token rows as the B
-//     operand (N = tokens rounded up to 32, <= 128), persistent over work units
-//     (token chunk, weight-row tile); SwiGLU or gate-weighted epilogue.
+//   * tc_moe_kernel — the routed experts (gate/up SwiGLU, then gate-weighted down)
+//     in one persistent launch: weights as the MMA A operand (two 128-row tiles
+//     per unit) and the expert's gathered token rows as the B operand (N = tokens
+//     rounded up to 32, <= 128); down units of a token chunk wait, on the device,
+//     for the chunk's gate/up units.
 // Operands are staged by TMA (no multicast) into 128-byte-swizzled K-major
 // tiles; accumulators live in TMEM and are read back with tcgen05.ld.
 //
@@ -623,49 +624,50 @@ __global__ void __launch_bounds__(TC_DENSE_THREADS, 1)
 }
 
 // ---------------------------------------------------------------------------
-// grouped expert kernel (persistent).  Work unit u = chunk * FT + f: token chunk
-// `chunk` (expert e = chunk_e[chunk], permuted rows r0 = chunk_r0[chunk] ..
-// r0 + n - 1, n <= 128) times weight-row tile f (128 rows of the expert's
-// weight).  GATEUP: two weights (gate, up) [E*I, d] -> hb[r, f*128 + i] =
-// silu(g) * u (bf16).  Otherwise: down [E*d, I] -> yb[r, f*128 + i] =
-// gate_of[r] * acc (fp32).
-// 192 threads: warp 0 TMA, warp 1 MMA, warps 2..5 epilogue (TMEM lanes
-// 32 (w % 4) .. +31).  One accumulator set; the MMA warp waits for the epilogue
-// to drain it before the next unit, while the producer keeps streaming.
+// Routed experts in one persistent launch.  Token chunk `c` = expert e =
+// chunk_e[c], permuted rows r0 = chunk_r0[c] .. r0 + n - 1 (n <= 128).
+//   phase 1, unit u = c * FT1 + f (FT1 = I / 128): gate and up rows f*128 .. +127
+//     of expert e against the chunk's rows X -> hb[r, f*128 + i] = silu(g) * u (bf16);
+//   phase 2, unit v = c * FT2 + f (FT2 = d / 256): down rows f*256 .. +255 of
+//     expert e (two 128-row tiles) against hb -> yb[r, f*256 + i] = gate_of[r] * acc.
+// A block takes units blockIdx.x, + gridDim.x, ... over phase 1 then phase 2, so
+// it waits (for a chunk's phase-1 units, counted in ready[c]) only after finishing
+// its own phase-1 units: no block waits for a block that waits.
+// Both phases run two MMAs per k-step (weights on the MMA's M side, tokens on N)
+// into TMEM columns 0 and 128.  320 threads: warp 0 TMA, warp 1 MMA, warps 2..9
+// epilogue (warps w and w + 4 share a TMEM lane quarter and split the token chunks).
 // ---------------------------------------------------------------------------
-template <bool GATEUP, int ST>
-struct ExpertCfg {
-  static constexpr int NW = GATEUP ? 2 : 1;
+template <int ST>
+struct MoeCfg {
   static constexpr uint32_t B_MAX = 128 * TC_KB * 2;
-  static constexpr uint32_t STAGE = NW * TC_SUB_A + B_MAX;
-  static constexpr uint32_t TCOLS = GATEUP ? 256 : 128;
+  static constexpr uint32_t STAGE = 2 * TC_SUB_A + B_MAX;
+  static constexpr uint32_t TCOLS = 256;
   static constexpr size_t SMEM = 1024 + (size_t)ST * STAGE + 256;
 };
+constexpr int TC_MOE_THREADS = 320;
 
-// 320 threads: warp 0 TMA, warp 1 MMA, warps 2..9 epilogue (warps w and w + 4 share
-// a TMEM lane quarter and split the token chunks).
-constexpr int TC_EXPERT_THREADS = 320;
-
-template <bool GATEUP, int ST>
-__global__ void __launch_bounds__(TC_EXPERT_THREADS, 1)
-    tc_expert_kernel(const __grid_constant__ CUtensorMap mW, const __grid_constant__ CUtensorMap mW2,
-                     const __grid_constant__ CUtensorMap mX, const int32_t* __restrict__ chunk_e,
-                     const int32_t* __restrict__ chunk_r0, const int32_t* __restrict__ n_chunks,
-                     const int32_t* __restrict__ offsets, int w_rows_per_expert, int K, int FT,
-                     void* __restrict__ out, int ldo, const float* __restrict__ gate_of,
-                     int32_t* err) {
-  typedef ExpertCfg<GATEUP, ST> Cfg;
+template <int ST>
+__global__ void __launch_bounds__(TC_MOE_THREADS, 1)
+    tc_moe_kernel(const __grid_constant__ CUtensorMap mWg, const __grid_constant__ CUtensorMap mWu,
+                  const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mWd,
+                  const __grid_constant__ CUtensorMap mH, const int32_t* __restrict__ chunk_e,
+                  const int32_t* __restrict__ chunk_r0, const int32_t* __restrict__ n_chunks,
+                  const int32_t* __restrict__ offsets, int I, int d, bf16* __restrict__ hb,
+                  float* __restrict__ yb, const float* __restrict__ gate_of,
+                  int32_t* __restrict__ ready, int32_t* err) {
+  typedef MoeCfg<ST> Cfg;
   pdl_enter();  // the routing tables come from the preceding kernels
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + ST * Cfg::STAGE);
   uint64_t* empty = full + ST;
-  uint64_t* tfull = empty + ST;   // accumulator ready (MMA -> epilogue)
-  uint64_t* tempty = tfull + 1;   // accumulator drained (epilogue -> MMA), 8 arrivals
+  uint64_t* tfull = empty + ST;   // accumulators ready (MMA -> epilogue)
+  uint64_t* tempty = tfull + 1;   // accumulators drained (epilogue -> MMA), 8 arrivals
   uint32_t* tslot = reinterpret_cast<uint32_t*>(tempty + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_units = *n_chunks * FT;
-  const int nk = (K + TC_KB - 1) / TC_KB;
+  const int nc = *n_chunks;
+  const int FT1 = I / 128, FT2 = d / 256;
+  const int U1 = nc * FT1, n_units = U1 + nc * FT2;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < ST; ++s) {
@@ -682,43 +684,74 @@ __global__ void __launch_bounds__(TC_EXPERT_THREADS, 1)
   tc::fence_after_sync();
   const uint32_t tmem = *tslot;
 
-  auto unit_rows = [&](int u, int& e, int& r0, int& n, int& f) {
-    const int c = u / FT;
-    f = u % FT;
-    e = chunk_e[c];
-    r0 = chunk_r0[c];
-    n = min(128, offsets[e + 1] - r0);
+  struct Unit {
+    bool down;
+    int c, e, r0, n, f;
+  };
+  auto unit_of = [&](int u) {
+    Unit x;
+    x.down = u >= U1;
+    const int v = x.down ? u - U1 : u, ft = x.down ? FT2 : FT1;
+    x.c = v / ft;
+    x.f = v % ft;
+    x.e = chunk_e[x.c];
+    x.r0 = chunk_r0[x.c];
+    x.n = min(128, offsets[x.e + 1] - x.r0);
+    return x;
   };
 
   if (warp == 0) {
     if (lane == 0) {
-      tc::prefetch_tmap(&mW);
-      if (GATEUP) tc::prefetch_tmap(&mW2);
+      tc::prefetch_tmap(&mWg);
+      tc::prefetch_tmap(&mWu);
       tc::prefetch_tmap(&mX);
+      tc::prefetch_tmap(&mWd);
+      tc::prefetch_tmap(&mH);
       int it = 0;
-      for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
-        int e, r0, n, f;
-        unit_rows(u, e, r0, n, f);
-        const int nb = (n + 31) >> 5;
-        const uint32_t bytes = Cfg::NW * TC_SUB_A + (uint32_t)nb * 32 * TC_KB * 2;
-        const int wrow = e * w_rows_per_expert + f * 128;
+      bool ok = true;
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+        const Unit x = unit_of(u);
+        if (x.down) {
+          // the chunk's hidden rows are complete once all its phase-1 units have counted
+          const uint64_t t0 = tc::global_ns();
+          while (ld_acquire(ready + x.c) < FT1) {
+            __nanosleep(64);
+            if (tc::global_ns() - t0 > 2000000000ull) {
+              atomicOr(err, ERR_TIMEOUT);
+              ok = false;
+              break;
+            }
+          }
+          if (!ok) break;
+          asm volatile("fence.proxy.async.global;" ::: "memory");  // before the TMA reads
+        }
+        const int nk = (x.down ? I : d) / TC_KB;
+        const int nb = (x.n + 31) >> 5;
+        const uint32_t bytes = 2 * TC_SUB_A + (uint32_t)nb * 32 * TC_KB * 2;
+        const int w1 = x.down ? x.e * d + x.f * 256 : x.e * I + x.f * 128;
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int s = it % ST;
           const uint32_t ph = (it / ST) & 1;
           if (it >= ST && !tc::mbar_wait(empty + s, ph ^ 1)) {
             atomicOr(err, ERR_TIMEOUT);
-            u = n_units;
+            ok = false;
             break;
           }
           uint8_t* st = smem + s * Cfg::STAGE;
-          // units of one token chunk start their K walk at different offsets
-          const int kx = ((kb + f) % nk) * TC_KB;
+          // units of one chunk start their K walk at different offsets
+          const int kx = ((kb + x.f) % nk) * TC_KB;
           tc::mbar_expect_tx(full + s, bytes);
-          tc::tma_load_2d(st, &mW, full + s, kx, wrow);
-          if (GATEUP) tc::tma_load_2d(st + TC_SUB_A, &mW2, full + s, kx, wrow);
-          uint8_t* bt = st + Cfg::NW * TC_SUB_A;
+          if (x.down) {
+            tc::tma_load_2d(st, &mWd, full + s, kx, w1);
+            tc::tma_load_2d(st + TC_SUB_A, &mWd, full + s, kx, w1 + 128);
+          } else {
+            tc::tma_load_2d(st, &mWg, full + s, kx, w1);
+            tc::tma_load_2d(st + TC_SUB_A, &mWu, full + s, kx, w1);
+          }
+          uint8_t* bt = st + 2 * TC_SUB_A;
           for (int j = 0; j < nb; ++j)
-            tc::tma_load_2d(bt + j * 32 * TC_KB * 2, &mX, full + s, kx, r0 + 32 * j);
+            tc::tma_load_2d(bt + j * 32 * TC_KB * 2, x.down ? &mH : &mX, full + s, kx,
+                            x.r0 + 32 * j);
         }
       }
     }
@@ -727,9 +760,9 @@ __global__ void __launch_bounds__(TC_EXPERT_THREADS, 1)
       int it = 0, ui = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++ui) {
-        int e, r0, n, f;
-        unit_rows(u, e, r0, n, f);
-        const int npad = ((n + 31) >> 5) << 5;
+        const Unit x = unit_of(u);
+        const int nk = (x.down ? I : d) / TC_KB;
+        const int npad = ((x.n + 31) >> 5) << 5;
         const uint32_t idesc = tc::idesc_bf16(128, npad);
         // wait until the epilogue has drained the previous unit's accumulators
         if (ui > 0 && !tc::mbar_wait(tempty, (ui - 1) & 1)) {
@@ -747,13 +780,13 @@ __global__ void __launch_bounds__(TC_EXPERT_THREADS, 1)
           }
           tc::fence_after_sync();
           const uint32_t a0 = tc::smem_addr(smem + s * Cfg::STAGE);
-          const uint32_t b0 = a0 + Cfg::NW * TC_SUB_A;
+          const uint32_t b0 = a0 + 2 * TC_SUB_A;
 #pragma unroll
           for (int k = 0; k < TC_KB / 16; ++k) {
             const uint32_t acc = (kb | k) != 0;
             const uint64_t bd = tc::sdesc_k128(b0 + k * 32);
             tc::mma_bf16(tmem, tc::sdesc_k128(a0 + k * 32), bd, idesc, acc);
-            if (GATEUP) tc::mma_bf16(tmem + 128, tc::sdesc_k128(a0 + TC_SUB_A + k * 32), bd, idesc, acc);
+            tc::mma_bf16(tmem + 128, tc::sdesc_k128(a0 + TC_SUB_A + k * 32), bd, idesc, acc);
           }
           tc::mma_commit(empty + s);
         }
@@ -766,43 +799,53 @@ __global__ void __launch_bounds__(TC_EXPERT_THREADS, 1)
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     int ui = 0;
     for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++ui) {
-      int e, r0, n, f;
-      unit_rows(u, e, r0, n, f);
-      bool ready = true;
-      if (lane == 0) ready = tc::mbar_wait(tfull, ui & 1);
-      ready = __shfl_sync(0xffffffffu, ready ? 1 : 0, 0) != 0;
-      if (!ready) {
-        if (lane == 0) atomicOr(err, ERR_TIMEOUT);
-        break;
-      }
+      const Unit x = unit_of(u);
+      bool rdy = true;
+      if (lane == 0) rdy = tc::mbar_wait(tfull, ui & 1);
+      rdy = __shfl_sync(0xffffffffu, rdy ? 1 : 0, 0) != 0;
+      // on a timeout the warp records it and keeps step with the other epilogue warps
+      // (same barriers, no TMEM reads), so that nothing waits forever
+      if (!rdy && lane == 0) atomicOr(err, ERR_TIMEOUT);
       tc::fence_after_sync();
-      const int fr = f * 128 + 32 * q + lane;  // weight row within the expert = output column
-      const int nch = (n + 31) >> 5;
+      const int nch = rdy ? (x.n + 31) >> 5 : 0;
+      if (!x.down) {
+        const int fr = x.f * 128 + 32 * q + lane;  // hidden column
 #pragma unroll 1
-      for (int c = hf; c < nch; c += 2) {
-        float v[32];
-        tc::tmem_ld32(tmem + lane_base + c * 32, v);
-        if (GATEUP) {
-          float g2[32];
-          tc::tmem_ld32(tmem + lane_base + 128 + c * 32, g2);
-          bf16* o = reinterpret_cast<bf16*>(out);
+        for (int c = hf; c < nch; c += 2) {
+          float g[32], v[32];
+          tc::tmem_ld32(tmem + lane_base + c * 32, g);
+          tc::tmem_ld32(tmem + lane_base + 128 + c * 32, v);
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const int t = c * 32 + j;
-            if (t < n) o[(size_t)(r0 + t) * ldo + fr] = __float2bfloat16_rn(silu(v[j]) * g2[j]);
+            if (t < x.n) hb[(size_t)(x.r0 + t) * I + fr] = __float2bfloat16_rn(silu(g[j]) * v[j]);
           }
-        } else {
-          float* o = reinterpret_cast<float*>(out);
+        }
+      } else {
+#pragma unroll 1
+        for (int half2 = 0; half2 < 2; ++half2) {
+          const int fr = x.f * 256 + half2 * 128 + 32 * q + lane;  // output column
+#pragma unroll 1
+          for (int c = hf; c < nch; c += 2) {
+            float v[32];
+            tc::tmem_ld32(tmem + lane_base + half2 * 128 + c * 32, v);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int t = c * 32 + j;
-            if (t < n) o[(size_t)(r0 + t) * ldo + fr] = gate_of[r0 + t] * v[j];
+            for (int j = 0; j < 32; ++j) {
+              const int t = c * 32 + j;
+              if (t < x.n) yb[(size_t)(x.r0 + t) * d + fr] = gate_of[x.r0 + t] * v[j];
+            }
           }
         }
       }
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(tc::smem_addr(tempty)) : "memory");
+      if (!x.down) {
+        // this unit's hidden columns are written: count it for the chunk's phase-2 units
+        __threadfence();
+        asm volatile("bar.sync 1, 256;" ::: "memory");  // the eight epilogue warps
+        if (warp == 2 && lane == 0) atomicAdd(ready + x.c, 1);
+      }
     }
   }
   tc::fence_before_sync();
@@ -830,6 +873,7 @@ dg_status tc_gemm_swiglu(dg_model* m, const bf16* A, const void* Wg, const void*
                          int M, int N, int K, cudaStream_t st);
 dg_status tc_moe_gate_up(dg_model* m, int l, const bf16* X, bf16* hb, int grid_y, cudaStream_t st);
 dg_status tc_moe_down(dg_model* m, int l, const bf16* H, float* yb, int grid_y, cudaStream_t st);
+dg_status tc_moe_experts(dg_model* m, int l, const bf16* X, bf16* hb, float* yb, cudaStream_t st);
 dg_status tc_lmhead_stats(dg_model* m, const bf16* xn, int M, float* ent, int32_t* amax,
                           cudaStream_t st);
 dg_status tc_attention(dg_model* m, const bf16* q, int B, int nq, int qpos0, const dg_kv* kv,

@@ -132,7 +132,7 @@ dg_status launch_dense(dg_model* m, const CUtensorMap& a, const CUtensorMap& b,
 constexpr int DENSE_BN = 64, DENSE_MT = 2, DENSE_ST = 5, DUAL_ST = 4;
 constexpr int QKV_ST = 4, RT_ST = 4;
 constexpr int LM_BN = 256, LM_ST = 3;
-constexpr int GU_ST = 4, DN_ST = 6;
+constexpr int MOE_ST = 4;
 constexpr int GU8_ST = 3, DN8_ST = 5;
 
 }  // namespace
@@ -140,9 +140,9 @@ constexpr int GU8_ST = 3, DN8_ST = 5;
 dg_status tc_prepare(dg_model* m) {
   const dg_config& c = m->cfg;
   const int qkv_n = (c.n_q_heads + 2 * c.n_kv_heads) * c.head_dim;
-  if (c.d_model % 128 || c.expert_inter % 128 || c.shared_inter % 64 || qkv_n % 64 ||
+  if (c.d_model % 256 || c.expert_inter % 128 || c.shared_inter % 64 || qkv_n % 64 ||
       (c.n_q_heads * c.head_dim) % 64) {
-    set_error("tensor-core tiling needs d %% 128, I %% 128, Is %% 64, (Hq+2Hkv)h %% 64 and Hq h %% 64");
+    set_error("tensor-core tiling needs d %% 256, I %% 128, Is %% 64, (Hq+2Hkv)h %% 64 and Hq h %% 64");
     return DG_ERR_UNSUPPORTED;
   }
   TcState* s = new TcState();
@@ -168,8 +168,7 @@ dg_status tc_prepare(dg_model* m) {
   DG_TRY(set_smem(tc_dense_kernel<DENSE_BN, DENSE_MT, false, DENSE_ST, EpiAddF32>, Dn::SMEM));
   DG_TRY(set_smem(tc_dense_kernel<DENSE_BN, DENSE_MT, true, DUAL_ST, EpiSwigluBf16>, Du::SMEM));
   DG_TRY(set_smem(tc_dense_kernel<LM_BN, 2, false, LM_ST, EpiLmStats>, Lm::SMEM));
-  DG_TRY(set_smem(tc_expert_kernel<true, GU_ST>, ExpertCfg<true, GU_ST>::SMEM));
-  DG_TRY(set_smem(tc_expert_kernel<false, DN_ST>, ExpertCfg<false, DN_ST>::SMEM));
+  DG_TRY(set_smem(tc_moe_kernel<MOE_ST>, MoeCfg<MOE_ST>::SMEM));
   DG_TRY(set_smem(tc_attn_kernel, AT_SMEM));
   DG_TRY(set_smem(tc_dense_kernel<128, 1, false, RT_ST, EpiRouterTopk>,
                   DenseCfg<128, 1, false, RT_ST>::SMEM));
@@ -284,25 +283,6 @@ dg_status tc_lmhead_stats(dg_model* m, const bf16* xn, int M, float* ent, int32_
 }
 
 template <bool GATEUP, int ST>
-static dg_status launch_expert(dg_model* m, const CUtensorMap& w, const CUtensorMap& w2,
-                               const CUtensorMap& x, int w_rows, int K, int FT, void* out, int ldo,
-                               const float* gate_of, cudaStream_t st) {
-  typedef ExpertCfg<GATEUP, ST> Cfg;
-  auto kern = tc_expert_kernel<GATEUP, ST>;
-  const int n_sm = state(m)->n_sm;
-  const Workspace& ws = m->ws;
-  launch_pdl((kern), n_sm, TC_EXPERT_THREADS, Cfg::SMEM, st, 1, w, w2, x, ws.tile_e, ws.tile_m0, ws.n_tiles, ws.offsets,
-                                     w_rows, K, FT, out, ldo, gate_of, ws.err);
-  ++m->launches;
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) {
-    set_error("tc_expert launch: %s", cudaGetErrorString(e));
-    return DG_ERR_CUDA;
-  }
-  return DG_OK;
-}
-
-template <bool GATEUP, int ST>
 static dg_status launch_expert_f8(dg_model* m, const CUtensorMap& w, const CUtensorMap& w2,
                                   const CUtensorMap& x, const float* s1, const float* s2,
                                   int w_rows, int K, int FT, void* out, int ldo,
@@ -320,41 +300,54 @@ static dg_status launch_expert_f8(dg_model* m, const CUtensorMap& w, const CUten
   return DG_OK;
 }
 
+// FP8 expert weights: gate/up, then down (two launches; bytes converted to bf16 in
+// shared memory)
 dg_status tc_moe_gate_up(dg_model* m, int l, const bf16* X, bf16* hb, int, cudaStream_t st) {
   const dg_config& c = m->cfg;
   const dg_layer_weights& L = m->layers[l];
   const int E = c.n_experts, I = c.expert_inter, d = c.d_model;
-  if (c.dtype == DG_BF16_FP8EXP) {
-    CUtensorMap wg, wu, x;
-    DG_TRY(tmap(m, L.gate, (uint64_t)E * I, d, 128, &wg, true));
-    DG_TRY(tmap(m, L.up, (uint64_t)E * I, d, 128, &wu, true));
-    DG_TRY(tmap(m, X, m->ws.max_rows, d, 32, &x));
-    return launch_expert_f8<true, GU8_ST>(m, wg, wu, x, L.gate_scale, L.up_scale, I, d, I / 128,
-                                          hb, I, nullptr, st);
-  }
   CUtensorMap wg, wu, x;
-  DG_TRY(tmap(m, L.gate, (uint64_t)E * I, d, 128, &wg));
-  DG_TRY(tmap(m, L.up, (uint64_t)E * I, d, 128, &wu));
+  DG_TRY(tmap(m, L.gate, (uint64_t)E * I, d, 128, &wg, true));
+  DG_TRY(tmap(m, L.up, (uint64_t)E * I, d, 128, &wu, true));
   DG_TRY(tmap(m, X, m->ws.max_rows, d, 32, &x));
-  return launch_expert<true, GU_ST>(m, wg, wu, x, I, d, I / 128, hb, I, nullptr, st);
+  return launch_expert_f8<true, GU8_ST>(m, wg, wu, x, L.gate_scale, L.up_scale, I, d, I / 128,
+                                        hb, I, nullptr, st);
 }
 
 dg_status tc_moe_down(dg_model* m, int l, const bf16* H, float* yb, int, cudaStream_t st) {
   const dg_config& c = m->cfg;
   const dg_layer_weights& L = m->layers[l];
   const int E = c.n_experts, I = c.expert_inter, d = c.d_model;
-  if (c.dtype == DG_BF16_FP8EXP) {
-    CUtensorMap wd, x;
-    DG_TRY(tmap(m, L.down, (uint64_t)E * d, I, 128, &wd, true));
-    DG_TRY(tmap(m, H, m->ws.max_rows, I, 32, &x));
-    return launch_expert_f8<false, DN8_ST>(m, wd, wd, x, L.down_scale, L.down_scale, d, I,
-                                           d / 128, yb, d, (const float*)m->ws.gate_of, st);
-  }
   CUtensorMap wd, x;
-  DG_TRY(tmap(m, L.down, (uint64_t)E * d, I, 128, &wd));
+  DG_TRY(tmap(m, L.down, (uint64_t)E * d, I, 128, &wd, true));
   DG_TRY(tmap(m, H, m->ws.max_rows, I, 32, &x));
-  return launch_expert<false, DN_ST>(m, wd, wd, x, d, I, d / 128, yb, d,
-                                     (const float*)m->ws.gate_of, st);
+  return launch_expert_f8<false, DN8_ST>(m, wd, wd, x, L.down_scale, L.down_scale, d, I,
+                                         d / 128, yb, d, (const float*)m->ws.gate_of, st);
+}
+
+// bf16 expert weights: both phases in one persistent launch (tc_moe_kernel)
+dg_status tc_moe_experts(dg_model* m, int l, const bf16* X, bf16* hb, float* yb,
+                         cudaStream_t st) {
+  const dg_config& c = m->cfg;
+  const dg_layer_weights& L = m->layers[l];
+  const int E = c.n_experts, I = c.expert_inter, d = c.d_model;
+  const Workspace& ws = m->ws;
+  CUtensorMap wg, wu, x, wd, h;
+  DG_TRY(tmap(m, L.gate, (uint64_t)E * I, d, 128, &wg));
+  DG_TRY(tmap(m, L.up, (uint64_t)E * I, d, 128, &wu));
+  DG_TRY(tmap(m, X, ws.max_rows, d, 32, &x));
+  DG_TRY(tmap(m, L.down, (uint64_t)E * d, I, 128, &wd));
+  DG_TRY(tmap(m, hb, ws.max_rows, I, 32, &h));
+  cudaError_t e = launch_pdl((tc_moe_kernel<MOE_ST>), state(m)->n_sm, TC_MOE_THREADS,
+                             MoeCfg<MOE_ST>::SMEM, st, 1, wg, wu, x, wd, h, ws.tile_e,
+                             ws.tile_m0, ws.n_tiles, ws.offsets, I, d, hb, yb,
+                             (const float*)ws.gate_of, ws.ready, ws.err);
+  ++m->launches;
+  if (e != cudaSuccess) {
+    set_error("tc_moe launch: %s", cudaGetErrorString(e));
+    return DG_ERR_CUDA;
+  }
+  return DG_OK;
 }
 
 dg_status tc_attention(dg_model* m, const bf16* q, int B, int nq, int qpos0, const dg_kv* kv,
