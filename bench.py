@@ -28,7 +28,7 @@ sys.path.insert(0, ROOT)
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # DRAM bytes per routed expert streamed by the gate/up + down kernels (ncu capture,
 # see the roofline computation below)
-DRAM_BYTES_PER_EXPERT = None  # not yet captured for the current routed-expert kernel
+DRAM_BYTES_PER_EXPERT = 98.38e6 / 9
 
 
 def load_peaks():
@@ -292,11 +292,11 @@ def run_ours(args, w, world, rank, local):
     unique_mean = units / max(ex_groups, 1)
     cost = metrics.forward_cost(model.cfg, B, kv_W, [unique_mean] * w.n_layers)
     ex_bytes = unique_mean * cost["expert_bytes"]
-    # DRAM traffic of the same two kernels: dram__bytes_read.sum + dram__bytes_write.sum of
-    # the gate/up and down launches in one ncu capture of the one-layer workload (same
-    # kernel shapes), 97.99 MB for 10.25 experts streamed, i.e. 9.56 MB per expert
-    # (algorithmic 9.44 MB); traffic grows with the experts streamed, so it is scaled
-    # by this run's count.  Valid for the expert kernels as captured.
+    # DRAM traffic of the routed-expert launch: dram__bytes_read.sum + dram__bytes_write.sum
+    # in one ncu capture of the one-layer workload (same kernel shapes; first forward of
+    # the block, 9 experts streamed): 98.38 MB = 85.0 MB of expert weights + the gathered
+    # rows and hidden rows, which ncu's cold cache sends to DRAM; scaled by this run's
+    # experts per launch.  Valid for the routed-expert kernel as captured.
     ex_traffic = (unique_mean * DRAM_BYTES_PER_EXPERT
                   if w.dtype == "bf16" and DRAM_BYTES_PER_EXPERT else None)
     ex_avg_s = ex_ms / 1e3 / max(ex_groups, 1)
