@@ -4,10 +4,11 @@
 // Work unit = token chunk x 128 weight rows, weights on the MMA's M side, tokens on
 // N (as in the bf16 routed-expert kernel), gate/up and down as two launches.  Per stage of 64 input columns:
 // TMA brings the FP8 weight tile(s) [128 rows x 64 bytes] and the bf16 token rows;
-// four converter warps turn each FP8 tile into the 128-byte-swizzled bf16 tile the
+// eight converter warps turn each FP8 tile into the 128-byte-swizzled bf16 tile the
 // MMA reads (value = code * scale, rounded to bf16); the MMA warp then issues
-// tcgen05.mma as in the bf16 kernel.  Roles (320 threads): warp 0 TMA, warp 1 MMA,
-// warps 2..5 epilogue, warps 6..9 converters.
+// tcgen05.mma as in the bf16 kernel.  Roles (576 threads): warp 0 TMA, warp 1 MMA,
+// warps 2..9 epilogue (warps w and w + 4 share a TMEM lane quarter and split the
+// token chunks), warps 10..17 converters.
 //
 // Passage: FP8 serving of the MoE experts — "DiffusionGemma 技术报告" (full
 // translation page), §6 (FP8 on H100, MoE memory-bound at batch 1).
@@ -37,8 +38,10 @@ __device__ __forceinline__ uint32_t f8x2_scaled(uint32_t two, float sc) {
   return *reinterpret_cast<uint32_t*>(&b);
 }
 
+constexpr int TC_F8_THREADS = 576;
+
 template <bool GATEUP, int ST>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(TC_F8_THREADS, 1)
     tc_expert_f8_kernel(const __grid_constant__ CUtensorMap mW, const __grid_constant__ CUtensorMap mW2,
                         const __grid_constant__ CUtensorMap mX, const float* __restrict__ sW,
                         const float* __restrict__ sW2, const int32_t* __restrict__ chunk_e,
@@ -51,7 +54,7 @@ __global__ void __launch_bounds__(320, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + ST * Cfg::STAGE);
-  uint64_t* conv = full + ST;     // converted tiles ready (4 converter warps)
+  uint64_t* conv = full + ST;     // converted tiles ready (8 converter warps)
   uint64_t* empty = conv + ST;
   uint64_t* tfull = empty + ST;
   uint64_t* tempty = tfull + 1;
@@ -64,11 +67,11 @@ __global__ void __launch_bounds__(320, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < ST; ++s) {
       tc::mbar_init(full + s, 1);
-      tc::mbar_init(conv + s, 4);
+      tc::mbar_init(conv + s, 8);
       tc::mbar_init(empty + s, 1);
     }
     tc::mbar_init(tfull, 1);
-    tc::mbar_init(tempty, 4);
+    tc::mbar_init(tempty, 8);
     tc::fence_mbar_init();
   }
   if (warp == 1) tc::tmem_alloc(tslot, Cfg::TCOLS);
@@ -159,9 +162,9 @@ __global__ void __launch_bounds__(320, 1)
         if (ok) tc::mma_commit(tfull);
       }
     }
-  } else if (warp >= 6) {
-    // converters: thread t handles 16-byte chunk (t % 4) of FP8 rows (t / 4) + 32 i
-    const int t = threadIdx.x - 192;  // 0..127
+  } else if (warp >= 10) {
+    // converters: thread t handles 16-byte chunk (t % 4) of FP8 rows (t / 4) + 64 i
+    const int t = threadIdx.x - 320;  // 0..255
     const int chunk = t & 3;
     int it = 0;
     for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
@@ -172,6 +175,14 @@ __global__ void __launch_bounds__(320, 1)
       for (int kb = 0; kb < nk; ++kb, ++it) {
         const int s = it % ST;
         const uint32_t ph = (it / ST) & 1;
+        const int kx = ((kb + f) % nk) * TC_KB;
+        // the scales do not depend on the staged tile: request them before waiting
+        float scl[Cfg::NW][2];
+#pragma unroll
+        for (int w = 0; w < Cfg::NW; ++w)
+#pragma unroll
+          for (int i = 0; i < 2; ++i)
+            scl[w][i] = (w == 0 ? sW : sW2)[(size_t)(wrow + (t >> 2) + 64 * i) * kscale + kx / 128];
         bool ready = true;
         if (lane == 0) ready = tc::mbar_wait(full + s, ph);
         ready = __shfl_sync(0xffffffffu, ready ? 1 : 0, 0) != 0;
@@ -180,16 +191,14 @@ __global__ void __launch_bounds__(320, 1)
           ok = false;
           break;
         }
-        const int kx = ((kb + f) % nk) * TC_KB;
 #pragma unroll
         for (int w = 0; w < Cfg::NW; ++w) {
-          const float* sc = w == 0 ? sW : sW2;
           const uint8_t* src = f8_at(s, w);
           uint8_t* dst = bf_at(s, w);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int r = (t >> 2) + 32 * i;
-            const float scale = sc[(size_t)(wrow + r) * kscale + kx / 128];
+          for (int i = 0; i < 2; ++i) {
+            const int r = (t >> 2) + 64 * i;
+            const float scale = scl[w][i];
             const uint4 q = *reinterpret_cast<const uint4*>(src + r * 64 + chunk * 16);
             const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
             uint32_t o[8];
@@ -214,8 +223,8 @@ __global__ void __launch_bounds__(320, 1)
       if (!ok) break;
     }
   } else {
-    // epilogue warps 2..5 -> TMEM lane quarter (warp % 4)
-    const int q = warp & 3;
+    // epilogue warps 2..9 -> TMEM lane quarter (warp % 4), token chunks of parity hf
+    const int q = warp & 3, hf = (warp - 2) >> 2;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     int ui = 0;
     for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++ui) {
@@ -232,7 +241,7 @@ __global__ void __launch_bounds__(320, 1)
       const int fr = f * 128 + 32 * q + lane;
       const int nch = (n + 31) >> 5;
 #pragma unroll 1
-      for (int c = 0; c < nch; ++c) {
+      for (int c = hf; c < nch; c += 2) {
         float v[32];
         tc::tmem_ld32(tmem + lane_base + c * 32, v);
         if (GATEUP) {

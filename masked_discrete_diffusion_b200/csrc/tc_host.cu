@@ -289,7 +289,8 @@ static dg_status launch_expert_f8(dg_model* m, const CUtensorMap& w, const CUten
                                   const float* gate_of, cudaStream_t st) {
   typedef ExpertF8Cfg<GATEUP, ST> Cfg;
   const Workspace& ws = m->ws;
-  cudaError_t e = launch_pdl((tc_expert_f8_kernel<GATEUP, ST>), state(m)->n_sm, 320, Cfg::SMEM, st, 1,
+  cudaError_t e = launch_pdl((tc_expert_f8_kernel<GATEUP, ST>), state(m)->n_sm, TC_F8_THREADS,
+                             Cfg::SMEM, st, 1,
                              w, w2, x, s1, s2, ws.tile_e, ws.tile_m0, ws.n_tiles, ws.offsets,
                              w_rows, K, FT, out, ldo, gate_of, ws.err);
   ++m->launches;
