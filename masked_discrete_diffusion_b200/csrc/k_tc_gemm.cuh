@@ -54,6 +54,7 @@ template <int COLS> struct TmemCols {
 // ---------------------------------------------------------------------------
 struct EpiStoreF32 {
   static constexpr bool kStaged = true, kWarpRows = false;
+  static constexpr size_t kExtraSmem = 0;
   float* out;
   int ldo, N;
   EpiStoreF32(float* o, int l, int n) : out(o), ldo(l), N(n) {}
@@ -70,6 +71,7 @@ struct EpiStoreF32 {
 
 struct EpiAddF32 {
   static constexpr bool kStaged = true, kWarpRows = false;
+  static constexpr size_t kExtraSmem = 0;
   float* out;
   int ldo, N;
   EpiAddF32(float* o, int l, int n) : out(o), ldo(l), N(n) {}
@@ -91,6 +93,7 @@ struct EpiAddF32 {
 
 struct EpiSwigluBf16 {
   static constexpr bool kStaged = true, kWarpRows = false;
+  static constexpr size_t kExtraSmem = 0;
   bf16* out;
   int ldo, N;
   EpiSwigluBf16(bf16* o, int l, int n) : out(o), ldo(l), N(n) {}
@@ -121,23 +124,74 @@ struct EpiSwigluBf16 {
 // position pos0 + i.
 struct EpiQkvRope {
   static constexpr bool kStaged = true, kWarpRows = true;
+  // cos / sin (fp32) of the positions of up to kCacheRows owned rows, filled by the
+  // warps that are idle during the main loop
+  static constexpr int kCacheRows = 64;
+  static constexpr size_t kExtraSmem = (size_t)kCacheRows * 64 * 2 * 4;
+  static constexpr int kVtStride = 66;  // bf16 per transposed row: conflict-free columns
   bf16 *q, *kc, *vc;
   const float* rope;
   int max_pos, n_seq, np, pos0, Hq, Hkv;
-  // rows row0 .. row0 + RB - 1 (those < M); the table loads of all rows go first
+
+  __device__ bool cached(int R) const { return R <= kCacheRows; }
+  // owned rows of a value head go through a transposed tile in shared memory
+  __device__ bool v_tile(int n0, int row_base, int R) const {
+    return n0 / 128 >= Hq + Hkv && R <= kCacheRows && (row_base % n_seq) + R <= n_seq &&
+           ((row_base % n_seq) & 1) == 0;
+  }
+  __device__ void prefill(uint8_t* extra, int row_base, int R, int M, int t, int nt) const {
+    if (!cached(R)) return;
+    // 16-byte units: rows of 64 floats = 16 units, cos then sin; all loads of a round
+    // are issued before its stores
+    float4* dst = reinterpret_cast<float4*>(extra);
+    const int units = R * 16 * 2;
+    constexpr int U = 8;
+    for (int base = t; base < units; base += nt * U) {
+      float4 x[U];
+#pragma unroll
+      for (int k = 0; k < U; ++k) {
+        const int idx = base + k * nt;
+        if (idx < units) {
+          const int tab = idx / (R * 16), rem = idx % (R * 16), r = rem >> 4, c = rem & 15;
+          const int row = row_base + r;
+          const int pos = pos0 + (row < M ? row % n_seq : 0);
+          x[k] = reinterpret_cast<const float4*>(rope + ((size_t)tab * max_pos + pos) * 64)[c];
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < U; ++k) {
+        const int idx = base + k * nt;
+        if (idx < units) {
+          const int tab = idx / (R * 16), rem = idx % (R * 16);
+          dst[tab * kCacheRows * 16 + rem] = x[k];
+        }
+      }
+    }
+  }
+  // rows row0 .. row0 + RB - 1 (those < M)
   template <int NQ, int RB>
-  __device__ void warp_rows(int row0, int M, int n0, const float (*v)[NQ], int lane) const {
+  __device__ void warp_rows(int row0, int M, int n0, const float (*v)[NQ], int lane,
+                            const uint8_t* extra, int row_base, int R, uint8_t* vt_s) const {
     static_assert(NQ == 4, "one head of 128 per tile");
     const int head = n0 / 128;
     if (head < Hq + Hkv) {
       float cs[RB][2], sn[RB][2];
+      const bool hit = cached(R);
+      const float* ccs = reinterpret_cast<const float*>(extra);
+      const float* csn = ccs + kCacheRows * 64;
 #pragma unroll
       for (int r = 0; r < RB; ++r) {
         const int pos = pos0 + (row0 + r < M ? (row0 + r) % n_seq : 0);
 #pragma unroll
         for (int q2 = 0; q2 < 2; ++q2) {
-          cs[r][q2] = rope[(size_t)pos * 64 + lane + 32 * q2];
-          sn[r][q2] = rope[((size_t)max_pos + pos) * 64 + lane + 32 * q2];
+          const int j = lane + 32 * q2;
+          if (hit) {
+            cs[r][q2] = ccs[(row0 + r - row_base) * 64 + j];
+            sn[r][q2] = csn[(row0 + r - row_base) * 64 + j];
+          } else {
+            cs[r][q2] = rope[(size_t)pos * 64 + j];
+            sn[r][q2] = rope[((size_t)max_pos + pos) * 64 + j];
+          }
         }
       }
 #pragma unroll
@@ -155,6 +209,15 @@ struct EpiQkvRope {
           dst[j + 64] = __float2bfloat16_rn(x2 * cs[r][q2] + x1 * sn[r][q2]);
         }
       }
+    } else if (v_tile(n0, row_base, R)) {
+      bf16* t = reinterpret_cast<bf16*>(vt_s);  // [128 dims][kVtStride]
+#pragma unroll
+      for (int r = 0; r < RB; ++r) {
+        if (row0 + r >= M) break;
+#pragma unroll
+        for (int q2 = 0; q2 < 4; ++q2)
+          t[(lane + 32 * q2) * kVtStride + (row0 + r - row_base)] = __float2bfloat16_rn(v[r][q2]);
+      }
     } else {
 #pragma unroll
       for (int r = 0; r < RB; ++r) {
@@ -168,6 +231,26 @@ struct EpiQkvRope {
       }
     }
   }
+  // after every warp's rows: the transposed value tile -> vc rows of 2 R contiguous bytes
+  __device__ void tail(uint8_t* vt_s, int row_base, int R, int M, int n0) const {
+    if (!v_tile(n0, row_base, R)) return;
+    const int g = n0 / 128 - Hq - Hkv;
+    const int b = row_base / n_seq, i0 = row_base % n_seq;
+    const int n_ok = min(R, M - row_base);
+    const uint32_t* t = reinterpret_cast<const uint32_t*>(vt_s);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int d = warp; d < 128; d += blockDim.x >> 5) {
+      bf16* dst = vc + (((size_t)b * Hkv + g) * 128 + d) * np + i0;
+      for (int pr = lane; 2 * pr < n_ok; pr += 32) {
+        const uint32_t two = t[(d * kVtStride) / 2 + pr];
+        if (2 * pr + 1 < n_ok) {
+          *reinterpret_cast<uint32_t*>(dst + 2 * pr) = two;
+        } else {
+          dst[2 * pr] = *reinterpret_cast<const bf16*>(&two);
+        }
+      }
+    }
+  }
 };
 
 // Router (N-tile = all E <= 32 NQ experts of a row): softmax over the E logits,
@@ -176,11 +259,15 @@ struct EpiQkvRope {
 // k-th selection.
 struct EpiRouterTopk {
   static constexpr bool kStaged = true, kWarpRows = true;
+  static constexpr size_t kExtraSmem = 0;
+  __device__ void prefill(uint8_t*, int, int, int, int, int) const {}
+  __device__ void tail(uint8_t*, int, int, int, int) const {}
   int32_t* idx;
   float* gate;
   int E, top_k;
   template <int NQ, int RB>
-  __device__ void warp_rows(int row0, int M, int n0, const float (*v)[NQ], int lane) const {
+  __device__ void warp_rows(int row0, int M, int n0, const float (*v)[NQ], int lane,
+                            const uint8_t*, int, int, uint8_t*) const {
 #pragma unroll 1
     for (int r = 0; r < RB; ++r)
       if (row0 + r < M) warp_row<NQ>(row0 + r, v[r], lane);
@@ -208,25 +295,23 @@ struct EpiRouterTopk {
     float gsum = 0.f, my_p = 0.f;
     int my_e = 0;
     for (int k = 0; k < top_k; ++k) {
+      // this lane's best untaken probability (lowest id on ties), then the warp's: the
+      // probabilities are >= 0, so their bit patterns order like the values
       float bp = -1.f;
       int be = 0x7fffffff;
 #pragma unroll
       for (int q2 = 0; q2 < NQ; ++q2) {
         const int e = lane + 32 * q2;
-        if (e < E && !((taken >> q2) & 1u) && (p[q2] > bp || (p[q2] == bp && e < be))) {
+        if (e < E && !((taken >> q2) & 1u) && p[q2] > bp) {
           bp = p[q2];
           be = e;
         }
       }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float op = __shfl_xor_sync(0xffffffffu, bp, off);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-        if (op > bp || (op == bp && oe < be)) {
-          bp = op;
-          be = oe;
-        }
-      }
+      const unsigned bits = bp >= 0.f ? __float_as_uint(bp) : 0u;
+      const unsigned top = __reduce_max_sync(0xffffffffu, bits);
+      be = (unsigned)__reduce_min_sync(0xffffffffu, bits == top && bp >= 0.f ? (unsigned)be
+                                                                              : 0x7fffffffu);
+      bp = __uint_as_float(top);
       if ((be & 31) == lane) taken |= 1u << (be >> 5);
       if (lane == k) {
         my_e = be;
@@ -246,6 +331,7 @@ struct EpiRouterTopk {
 // u = sum exp(l - m) (l - m), a = lowest id attaining m.  part[(tile, row)] = (m, s, u, a).
 struct EpiLmStats {
   static constexpr bool kStaged = false, kWarpRows = false;
+  static constexpr size_t kExtraSmem = 0;
   float* part;
   int M, N;
   float scale;
@@ -483,6 +569,11 @@ __global__ void __launch_bounds__(TC_DENSE_THREADS, 1)
       tc::mma_commit(empty + s);
     }
     if (ok) tc::mma_commit(done);
+  } else if constexpr (Epi::kExtraSmem > 0) {
+    // warps 2.. are idle during the main loop: they fill the epilogue's table cache
+    if (warp >= 2)
+      epi.prefill(smem + ST * Cfg::STAGE + 256, m0 + rank * (MT * 128 / ksplit),
+                  MT * 128 / ksplit, M, threadIdx.x - 64, TC_DENSE_THREADS - 64);
   }
   __syncwarp();
 
@@ -569,7 +660,13 @@ __global__ void __launch_bounds__(TC_DENSE_THREADS, 1)
             for (int src = 0; src < 8; ++src)
               if (src < ksplit) v[r][q] += t[src][r][q];
           }
-        epi.template warp_rows<BN / 32, RB>(row0, M, n0, v, lane);
+        epi.template warp_rows<BN / 32, RB>(row0, M, n0, v, lane, smem + ST * Cfg::STAGE + 256,
+                                            m0 + rank * R, R, smem + MT * 128 * RS * 4);
+      }
+      if constexpr (Epi::kExtraSmem > 0) {
+        static_assert(MT * 128 * RS * 4 + 128 * 66 * 2 <= ST * Cfg::STAGE, "transposed tile");
+        __syncthreads();  // every warp's rows are in the transposed tile
+        epi.tail(smem + MT * 128 * RS * 4, m0 + rank * R, R, M, n0);
       }
     } else {
       // lane -> (row, 4 consecutive columns): a warp instruction covers RPW rows of BN

@@ -114,11 +114,11 @@ dg_status launch_dense(dg_model* m, const CUtensorMap& a, const CUtensorMap& b,
     while (ks < 8 && tiles * ks * 2 <= state(m)->n_sm && nk >= ks * 2 * 2) ks *= 2;
   cudaError_t e;
   if (ks == 1) {
-    e = launch_pdl(kern, grid, TC_DENSE_THREADS, Cfg::SMEM, st, 1, a, b, b2, M, K, 1, epi,
+    e = launch_pdl(kern, grid, TC_DENSE_THREADS, Cfg::SMEM + Epi::kExtraSmem, st, 1, a, b, b2, M, K, 1, epi,
                    m->ws.err, kwrap, b_weight ? 1 : 0);
   } else {
     grid.z = ks;
-    e = launch_pdl(kern, grid, TC_DENSE_THREADS, Cfg::SMEM, st, ks, a, b, b2, M, K, ks, epi,
+    e = launch_pdl(kern, grid, TC_DENSE_THREADS, Cfg::SMEM + Epi::kExtraSmem, st, ks, a, b, b2, M, K, ks, epi,
                    m->ws.err, kwrap, b_weight ? 1 : 0);
   }
   ++m->launches;
@@ -173,7 +173,7 @@ dg_status tc_prepare(dg_model* m) {
   DG_TRY(set_smem(tc_dense_kernel<128, 1, false, RT_ST, EpiRouterTopk>,
                   DenseCfg<128, 1, false, RT_ST>::SMEM));
   DG_TRY(set_smem(tc_dense_kernel<128, DENSE_MT, false, QKV_ST, EpiQkvRope>,
-                  DenseCfg<128, DENSE_MT, false, QKV_ST>::SMEM));
+                  DenseCfg<128, DENSE_MT, false, QKV_ST>::SMEM + EpiQkvRope::kExtraSmem));
   DG_TRY(set_smem(tc_expert_f8_kernel<true, GU8_ST>, ExpertF8Cfg<true, GU8_ST>::SMEM));
   DG_TRY(set_smem(tc_expert_f8_kernel<false, DN8_ST>, ExpertF8Cfg<false, DN8_ST>::SMEM));
   cudaDeviceGetAttribute(&s->n_sm, cudaDevAttrMultiProcessorCount, m->device);
