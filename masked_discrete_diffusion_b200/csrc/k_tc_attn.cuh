@@ -197,19 +197,17 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     tc::fence_after_sync();
     const uint32_t tS = tmem + (i & 1) * 128 + 64 * hf;
     // ---- softmax over this half's 64 keys; the row max is shared with the other half
+    float sv[64];
+    tc::tmem_ld64(tS + lane_base, sv);
     float mt = -INFINITY;
-#pragma unroll 1
-    for (int c = 0; c < 2; ++c) {
-      float v[32];
-      tc::tmem_ld32(tS + lane_base + c * 32, v);
 #pragma unroll
-      for (int q = 0; q < 32; ++q) {
-        const int kk = t0 + 64 * hf + c * 32 + q;
-        const int kp = kpos0 + 64 * hf + c * 32 + q;
-        bool valid = kk < nseg;
-        if (p.causal) valid = valid && kp <= qp && kp > qp - p.window;
-        if (valid) mt = fmaxf(mt, v[q] * p.scale_log2);
-      }
+    for (int q = 0; q < 64; ++q) {
+      const int kk = t0 + 64 * hf + q;
+      const int kp = kpos0 + 64 * hf + q;
+      bool valid = kk < nseg;
+      if (p.causal) valid = valid && kp <= qp && kp > qp - p.window;
+      sv[q] = valid ? sv[q] * p.scale_log2 : -INFINITY;
+      mt = fmaxf(mt, sv[q]);
     }
     xmax[hf * 128 + r] = mt;
     __syncthreads();
@@ -219,21 +217,16 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     float lsum = 0.f;
     const int r7 = r & 7;
     uint8_t* prow = sP + hf * AT_SUB + r * 128;
-#pragma unroll 1
+#pragma unroll
     for (int c = 0; c < 2; ++c) {
-      float v[32];
-      tc::tmem_ld32(tS + lane_base + c * 32, v);
       uint32_t pk[16];
 #pragma unroll
       for (int q = 0; q < 32; q += 2) {
         float e2[2];
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
-          const int kk = t0 + 64 * hf + c * 32 + q + u;
-          const int kp = kpos0 + 64 * hf + c * 32 + q + u;
-          bool valid = kk < nseg;
-          if (p.causal) valid = valid && kp <= qp && kp > qp - p.window;
-          e2[u] = valid ? exp2f(v[q + u] * p.scale_log2 - m_new) : 0.f;
+          const float x = sv[c * 32 + q + u];
+          e2[u] = x == -INFINITY ? 0.f : exp2f(x - m_new);
           lsum += e2[u];
         }
         __nv_bfloat162 b2 = __floats2bfloat162_rn(e2[0], e2[1]);
@@ -273,12 +266,11 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     tc::fence_after_sync();
     // stage i & 1 is free again (S(i) and O_t(i) done): prefetch tile i + 2
     if (tid == 0 && i + 2 < nt) load_tile(i + 2);
+    {
+      float ov[64];
+      tc::tmem_ld64(tO + lane_base + 64 * hf, ov);
 #pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      float v[32];
-      tc::tmem_ld32(tO + lane_base + 64 * hf + c * 32, v);
-#pragma unroll
-      for (int q = 0; q < 32; ++q) o[c * 32 + q] = o[c * 32 + q] * alpha + v[q];
+      for (int q = 0; q < 64; ++q) o[q] = o[q] * alpha + ov[q];
     }
     tc::fence_before_sync();
   }
