@@ -55,6 +55,8 @@ template <int COLS> struct TmemCols {
 struct EpiStoreF32 {
   static constexpr bool kStaged = true, kWarpRows = false;
   static constexpr size_t kExtraSmem = 0;
+  __device__ void prefill(uint8_t*, int, int, int, int, int, int) const {}
+  __device__ const float* cache() const { return nullptr; }
   float* out;
   int ldo, N;
   EpiStoreF32(float* o, int l, int n) : out(o), ldo(l), N(n) {}
@@ -70,11 +72,50 @@ struct EpiStoreF32 {
 };
 
 struct EpiAddF32 {
+  // the residual rows this CTA owns ([R <= 64][64 columns] fp32) are read into shared
+  // memory by the warps idle during the main loop; col4 then adds from there
   static constexpr bool kStaged = true, kWarpRows = false;
-  static constexpr size_t kExtraSmem = 0;
+  static constexpr int kCacheRows = 64, kCacheCols = 64;
+  static constexpr size_t kExtraSmem = (size_t)kCacheRows * kCacheCols * 4;
   float* out;
   int ldo, N;
   EpiAddF32(float* o, int l, int n) : out(o), ldo(l), N(n) {}
+  __device__ void prefill(uint8_t* extra, int row_base, int R, int M, int n0, int t,
+                          int nt) const {
+    if (R > kCacheRows || n0 + kCacheCols > N) return;
+    float4* dst = reinterpret_cast<float4*>(extra);
+    const int units = R * (kCacheCols / 4);
+    constexpr int U = 8;
+    for (int base = t; base < units; base += nt * U) {
+      float4 x[U];
+#pragma unroll
+      for (int k = 0; k < U; ++k) {
+        const int idx = base + k * nt, r = idx / (kCacheCols / 4), c = idx % (kCacheCols / 4);
+        if (idx < units && row_base + r < M)
+          x[k] = reinterpret_cast<const float4*>(out + (size_t)(row_base + r) * ldo + n0)[c];
+      }
+#pragma unroll
+      for (int k = 0; k < U; ++k) {
+        const int idx = base + k * nt;
+        if (idx < units && row_base + idx / (kCacheCols / 4) < M) dst[idx] = x[k];
+      }
+    }
+  }
+  // residual rows from the cache when it holds them (R <= 64 and a full 64-column tile)
+  __device__ void col4_cached(const uint8_t* extra, int row_base, int R, int n0, int row, int c,
+                              float4 v) const {
+    if (R <= kCacheRows && n0 + kCacheCols <= N) {
+      float4 o = reinterpret_cast<const float4*>(extra)[(row - row_base) * (kCacheCols / 4) +
+                                                        (c - n0) / 4];
+      o.x += v.x;
+      o.y += v.y;
+      o.z += v.z;
+      o.w += v.w;
+      *reinterpret_cast<float4*>(out + (size_t)row * ldo + c) = o;
+    } else {
+      col4(row, c, v, v);
+    }
+  }
   __device__ void col4(int row, int c, float4 v, float4) const {
     float* p = out + (size_t)row * ldo + c;
     if (c + 4 <= N) {
@@ -94,6 +135,7 @@ struct EpiAddF32 {
 struct EpiSwigluBf16 {
   static constexpr bool kStaged = true, kWarpRows = false;
   static constexpr size_t kExtraSmem = 0;
+  __device__ void prefill(uint8_t*, int, int, int, int, int, int) const {}
   bf16* out;
   int ldo, N;
   EpiSwigluBf16(bf16* o, int l, int n) : out(o), ldo(l), N(n) {}
@@ -139,7 +181,7 @@ struct EpiQkvRope {
     return n0 / 128 >= Hq + Hkv && R <= kCacheRows && (row_base % n_seq) + R <= n_seq &&
            ((row_base % n_seq) & 1) == 0;
   }
-  __device__ void prefill(uint8_t* extra, int row_base, int R, int M, int t, int nt) const {
+  __device__ void prefill(uint8_t* extra, int row_base, int R, int M, int, int t, int nt) const {
     if (!cached(R)) return;
     // 16-byte units: rows of 64 floats = 16 units, cos then sin; all loads of a round
     // are issued before its stores
@@ -260,7 +302,7 @@ struct EpiQkvRope {
 struct EpiRouterTopk {
   static constexpr bool kStaged = true, kWarpRows = true;
   static constexpr size_t kExtraSmem = 0;
-  __device__ void prefill(uint8_t*, int, int, int, int, int) const {}
+  __device__ void prefill(uint8_t*, int, int, int, int, int, int) const {}
   __device__ void tail(uint8_t*, int, int, int, int) const {}
   int32_t* idx;
   float* gate;
@@ -573,7 +615,7 @@ __global__ void __launch_bounds__(TC_DENSE_THREADS, 1)
     // warps 2.. are idle during the main loop: they fill the epilogue's table cache
     if (warp >= 2)
       epi.prefill(smem + ST * Cfg::STAGE + 256, m0 + rank * (MT * 128 / ksplit),
-                  MT * 128 / ksplit, M, threadIdx.x - 64, TC_DENSE_THREADS - 64);
+                  MT * 128 / ksplit, M, n0, threadIdx.x - 64, TC_DENSE_THREADS - 64);
   }
   __syncwarp();
 
@@ -709,7 +751,13 @@ __global__ void __launch_bounds__(TC_DENSE_THREADS, 1)
               }
           }
           const int row = m0 + rank * R + lr0 + i * RPW + rsub;
-          if (row < M) epi.col4(row, n0 + c4, v[0], v[Cfg::NACC - 1]);
+          if (row < M) {
+            if constexpr (Epi::kExtraSmem > 0)
+              epi.col4_cached(smem + ST * Cfg::STAGE + 256, m0 + rank * R, R, n0, row, n0 + c4,
+                              v[0]);
+            else
+              epi.col4(row, n0 + c4, v[0], v[Cfg::NACC - 1]);
+          }
         }
       }
     }

@@ -165,7 +165,8 @@ dg_status tc_prepare(dg_model* m) {
   typedef DenseCfg<DENSE_BN, DENSE_MT, true, DUAL_ST> Du;
   typedef DenseCfg<LM_BN, 2, false, LM_ST> Lm;
   DG_TRY(set_smem(tc_dense_kernel<DENSE_BN, DENSE_MT, false, DENSE_ST, EpiStoreF32>, Dn::SMEM));
-  DG_TRY(set_smem(tc_dense_kernel<DENSE_BN, DENSE_MT, false, DENSE_ST, EpiAddF32>, Dn::SMEM));
+  DG_TRY(set_smem(tc_dense_kernel<DENSE_BN, DENSE_MT, false, DENSE_ST, EpiAddF32>,
+                  Dn::SMEM + EpiAddF32::kExtraSmem));
   DG_TRY(set_smem(tc_dense_kernel<DENSE_BN, DENSE_MT, true, DUAL_ST, EpiSwigluBf16>, Du::SMEM));
   DG_TRY(set_smem(tc_dense_kernel<LM_BN, 2, false, LM_ST, EpiLmStats>, Lm::SMEM));
   DG_TRY(set_smem(tc_moe_kernel<MOE_ST>, MoeCfg<MOE_ST>::SMEM));
