@@ -463,81 +463,6 @@ __global__ void router_topk_kernel(const Acc* __restrict__ part, int splits,
   }
 }
 
-// ---------------------------------------------------------------------------
-// Deterministic permutation of (token, slot) entries into expert-contiguous
-// rows.  Entry j = t * k + slot belongs to expert idx[j]; within an expert the
-// entries keep their j order.  Block e computes the rank of each of its entries
-// and counts[e].
-// ---------------------------------------------------------------------------
-static __global__ void moe_rank_kernel(const int32_t* __restrict__ idx, int n_entries,
-                                int32_t* __restrict__ rank, int32_t* __restrict__ counts) {
-  pdl_enter();
-  __shared__ int warp_tot[32];
-  __shared__ int carry;
-  const int e = blockIdx.x;
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  if (threadIdx.x == 0) carry = 0;
-  __syncthreads();
-  for (int base = 0; base < n_entries; base += blockDim.x) {
-    const int j = base + threadIdx.x;
-    const bool f = j < n_entries && idx[j] == e;
-    const unsigned bal = __ballot_sync(0xffffffffu, f);
-    const int before = __popc(bal & ((1u << lane) - 1u));
-    if (lane == 0) warp_tot[wid] = __popc(bal);
-    __syncthreads();
-    int off = carry;
-    for (int w2 = 0; w2 < wid; ++w2) off += warp_tot[w2];
-    if (f) rank[j] = off + before;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      int s = 0;
-      for (int w2 = 0; w2 < nw; ++w2) s += warp_tot[w2];
-      carry += s;
-    }
-    __syncthreads();
-  }
-  if (threadIdx.x == 0) counts[e] = carry;
-}
-
-// offsets = exclusive scan of counts; tile table with `bm` rows per tile.
-// One block of 1024 threads, thread e handles expert e (E <= 1024).
-static __global__ void __launch_bounds__(1024)
-    moe_offsets_kernel(const int32_t* __restrict__ counts, int E, int bm,
-                       int32_t* __restrict__ offsets, int32_t* __restrict__ tile_e,
-                       int32_t* __restrict__ tile_m0, int32_t* __restrict__ n_tiles,
-                       int max_tiles, unsigned long long* __restrict__ used) {
-  pdl_enter();
-  __shared__ int sc[1024], st[1024];
-  const int e = threadIdx.x;
-  const int c = e < E ? counts[e] : 0;
-  // experts that received at least one row (their weights are streamed)
-  const unsigned bal = __ballot_sync(0xffffffffu, c > 0);
-  if (used && (e & 31) == 0 && bal) atomicAdd(used, (unsigned long long)__popc(bal));
-  const int nt = (c + bm - 1) / bm;
-  sc[e] = c;
-  st[e] = nt;
-  __syncthreads();
-  for (int off = 1; off < 1024; off <<= 1) {  // inclusive scans
-    const int a = e >= off ? sc[e - off] : 0, b = e >= off ? st[e - off] : 0;
-    __syncthreads();
-    sc[e] += a;
-    st[e] += b;
-    __syncthreads();
-  }
-  const int off_e = sc[e] - c, t_e = st[e] - nt;
-  if (e < E) offsets[e] = off_e;
-  if (e == E - 1) {
-    offsets[E] = off_e + c;
-    *n_tiles = min(t_e + nt, max_tiles);
-  }
-  if (e < E)
-    for (int r = 0; r < nt; ++r)
-      if (t_e + r < max_tiles) {
-        tile_e[t_e + r] = e;
-        tile_m0[t_e + r] = off_e + r * bm;
-      }
-}
-
 // The whole permutation of the (token, slot) entries into expert-contiguous rows,
 // by one block (any multiple of 32 threads <= 1024): ranks by warp-level match
 // plus per-(warp, expert) counts scanned in warp order (entry order is kept within
@@ -682,21 +607,6 @@ __global__ void __launch_bounds__(1024)
   }
 }
 
-template <class Acc>
-__global__ void moe_scatter_kernel(const int32_t* __restrict__ idx, const Acc* __restrict__ gate,
-                                   const int32_t* __restrict__ rank,
-                                   const int32_t* __restrict__ offsets, int n_entries, int top_k,
-                                   int32_t* __restrict__ row_of, int32_t* __restrict__ tok_of,
-                                   Acc* __restrict__ gate_of) {
-  pdl_enter();
-  const int j = blockIdx.x * blockDim.x + threadIdx.x;
-  if (j >= n_entries) return;
-  const int pos = offsets[idx[j]] + rank[j];
-  row_of[j] = pos;
-  tok_of[pos] = j / top_k;
-  gate_of[pos] = gate[j];
-}
-
 template <class TA>
 __global__ void gather_rows_kernel(const TA* __restrict__ src, const int32_t* __restrict__ tok_of,
                                    const int32_t* __restrict__ n_rows_dev, int d,
@@ -707,26 +617,6 @@ __global__ void gather_rows_kernel(const TA* __restrict__ src, const int32_t* __
   const TA* s = src + (size_t)tok_of[r] * d;
   TA* o = dst + (size_t)r * d;
   for (int c = threadIdx.x; c < d; c += blockDim.x) o[c] = s[c];
-}
-
-// x[t] += ys[t] + sum over slots of yb[row_of[t * k + slot]] (slot order fixed).
-// grid (n_tok, ceil(d / blockDim)).
-template <class TR, class TY, class Acc>
-__global__ void moe_combine_kernel(TR* __restrict__ x, const TY* __restrict__ ys,
-                                   const TY* __restrict__ yb, const int32_t* __restrict__ row_of,
-                                   int n_tok, int d, int top_k) {
-  pdl_enter();
-  const int t = blockIdx.x;
-  if (t >= n_tok) return;
-  {
-    const int c = blockIdx.y * blockDim.x + threadIdx.x;
-    if (c >= d) return;
-    Acc y = (Acc)widen(ys[(size_t)t * d + c]);
-    for (int k = 0; k < top_k; ++k)
-      y += (Acc)widen(yb[(size_t)row_of[(size_t)t * top_k + k] * d + c]);
-    TR* p = x + (size_t)t * d + c;
-    *p = narrow<TR>((Acc)widen(*p) + y);
-  }
 }
 
 // Combine fused with the next RMSNorm: x[t] += ys[t] + sum over slots of
