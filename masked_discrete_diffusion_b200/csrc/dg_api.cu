@@ -382,8 +382,7 @@ template <class Path> struct Runner {
       {
         ProfScope ps(m, DG_KIND_EXPERTS, st);
         if (c.dtype == DG_BF16_FP8EXP) {
-          DG_TRY(tc_moe_gate_up(m, l, (const TA*)ws.up, (TA*)ws.hb, grid_y, st));
-          DG_TRY(tc_moe_down(m, l, (const TA*)ws.hb, (float*)ws.yb, grid_y, st));
+          DG_TRY(tc_moe_experts_f8(m, l, (const TA*)ws.up, (TA*)ws.hb, (float*)ws.yb, st));
         } else {
           DG_TRY(tc_moe_experts(m, l, (const TA*)ws.up, (TA*)ws.hb, (float*)ws.yb, st));
         }

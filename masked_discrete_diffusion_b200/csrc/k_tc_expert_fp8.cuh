@@ -1,14 +1,13 @@
-// Grouped routed-expert GEMM with FP8 E4M3 expert weights (one fp32 scale per
-// weight row and 128 consecutive input columns) and bf16 activations.
+// Routed experts with FP8 E4M3 expert weights (one fp32 scale per weight row and 128
+// consecutive input columns) and bf16 activations: gate/up SwiGLU and down in one
+// persistent launch, with the schedule and device-side chunk counters of the bf16
+// routed-expert kernel (tc_moe_kernel).
 //
-// Work unit = token chunk x 128 weight rows, weights on the MMA's M side, tokens on
-// N (as in the bf16 routed-expert kernel), gate/up and down as two launches.  Per stage of 64 input columns:
-// TMA brings the FP8 weight tile(s) [128 rows x 64 bytes] and the bf16 token rows;
-// eight converter warps turn each FP8 tile into the 128-byte-swizzled bf16 tile the
-// MMA reads (value = code * scale, rounded to bf16); the MMA warp then issues
-// tcgen05.mma as in the bf16 kernel.  Roles (576 threads): warp 0 TMA, warp 1 MMA,
-// warps 2..9 epilogue (warps w and w + 4 share a TMEM lane quarter and split the
-// token chunks), warps 10..17 converters.
+// Weights sit on the MMA's M side, tokens on N.  Per stage of 64 input columns TMA
+// brings two FP8 weight tiles [128 rows x 64 bytes] and the bf16 token rows; eight
+// converter warps turn each FP8 tile into the 128-byte-swizzled bf16 tile the MMA
+// reads (value = code * scale, rounded to bf16); the MMA warp then issues tcgen05.mma.
+// A unit's scales are staged in shared memory once per unit.
 //
 // Passage: FP8 serving of the MoE experts — "DiffusionGemma 技术报告" (full
 // translation page), §6 (FP8 on H100, MoE memory-bound at batch 1).
@@ -20,16 +19,6 @@
 
 namespace dg {
 
-template <bool GATEUP, int ST>
-struct ExpertF8Cfg {
-  static constexpr int NW = GATEUP ? 2 : 1;
-  static constexpr uint32_t F8_TILE = 128 * 64;           // 8 KB staging per weight
-  static constexpr uint32_t B_MAX = 128 * TC_KB * 2;      // token rows
-  static constexpr uint32_t STAGE = NW * F8_TILE + NW * TC_SUB_A + B_MAX;
-  static constexpr uint32_t TCOLS = GATEUP ? 256 : 128;
-  static constexpr size_t SMEM = 1024 + (size_t)ST * STAGE + 512;
-};
-
 // bf16 pair from two E4M3 bytes times a scale
 __device__ __forceinline__ uint32_t f8x2_scaled(uint32_t two, float sc) {
   __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)two, __NV_E4M3);
@@ -40,16 +29,39 @@ __device__ __forceinline__ uint32_t f8x2_scaled(uint32_t two, float sc) {
 
 constexpr int TC_F8_THREADS = 576;
 
-template <bool GATEUP, int ST>
+// ---------------------------------------------------------------------------
+// Both phases of the routed experts with FP8 weights in one persistent launch (the
+// schedule and the device-side chunk counters of tc_moe_kernel).  Per stage: TMA
+// brings two FP8 weight tiles [128 rows x 64 bytes] and the bf16 token rows; the
+// eight converter warps write the two bf16 tiles; the MMA warp issues two MMAs.
+//   phase 1, unit u = c * FT1 + f: gate rows and up rows f*128 .. +127 (K = d);
+//   phase 2, unit v = c * FT2 + f: down rows f*256 .. +127 and +128 .. +255 (K = I).
+// Roles (576 threads): warp 0 TMA, warp 1 MMA, warps 2..9 epilogue, warps 10..17
+// converters.
+// ---------------------------------------------------------------------------
+template <int ST>
+struct MoeF8Cfg {
+  static constexpr uint32_t F8_TILE = 128 * 64;
+  static constexpr uint32_t B_MAX = 128 * TC_KB * 2;
+  static constexpr uint32_t STAGE = 2 * F8_TILE + 2 * TC_SUB_A + B_MAX;
+  static constexpr uint32_t TCOLS = 256;
+  static constexpr size_t SMEM = 1024 + (size_t)ST * STAGE + 512;  // + the unit's scales
+  // a unit's scales: 256 weight rows (gate then up, or the two down tiles) x K / 128
+  static size_t smem_bytes(int d, int I) { return SMEM + (size_t)8 * (d > I ? d : I); }
+};
+
+template <int ST>
 __global__ void __launch_bounds__(TC_F8_THREADS, 1)
-    tc_expert_f8_kernel(const __grid_constant__ CUtensorMap mW, const __grid_constant__ CUtensorMap mW2,
-                        const __grid_constant__ CUtensorMap mX, const float* __restrict__ sW,
-                        const float* __restrict__ sW2, const int32_t* __restrict__ chunk_e,
-                        const int32_t* __restrict__ chunk_r0, const int32_t* __restrict__ n_chunks,
-                        const int32_t* __restrict__ offsets, int w_rows_per_expert, int K, int FT,
-                        void* __restrict__ out, int ldo, const float* __restrict__ gate_of,
-                        int32_t* err) {
-  typedef ExpertF8Cfg<GATEUP, ST> Cfg;
+    tc_moe_f8_kernel(const __grid_constant__ CUtensorMap mWg, const __grid_constant__ CUtensorMap mWu,
+                     const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mWd,
+                     const __grid_constant__ CUtensorMap mH, const float* __restrict__ sWg,
+                     const float* __restrict__ sWu, const float* __restrict__ sWd,
+                     const int32_t* __restrict__ chunk_e, const int32_t* __restrict__ chunk_r0,
+                     const int32_t* __restrict__ n_chunks, const int32_t* __restrict__ offsets,
+                     int I, int d, bf16* __restrict__ hb, float* __restrict__ yb,
+                     const float* __restrict__ gate_of, int32_t* __restrict__ ready,
+                     int32_t* err) {
+  typedef MoeF8Cfg<ST> Cfg;
   pdl_enter();  // the routing tables come from the preceding kernels
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -57,12 +69,13 @@ __global__ void __launch_bounds__(TC_F8_THREADS, 1)
   uint64_t* conv = full + ST;     // converted tiles ready (8 converter warps)
   uint64_t* empty = conv + ST;
   uint64_t* tfull = empty + ST;
-  uint64_t* tempty = tfull + 1;
+  uint64_t* tempty = tfull + 1;   // 8 epilogue arrivals
   uint32_t* tslot = reinterpret_cast<uint32_t*>(tempty + 1);
+  float* sscl = reinterpret_cast<float*>(smem + ST * Cfg::STAGE + 512);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_units = *n_chunks * FT;
-  const int nk = (K + TC_KB - 1) / TC_KB;
-  const int kscale = K / 128;  // scales per weight row
+  const int nc = *n_chunks;
+  const int FT1 = I / 128, FT2 = d / 256;
+  const int U1 = nc * FT1, n_units = U1 + nc * FT2;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < ST; ++s) {
@@ -80,48 +93,73 @@ __global__ void __launch_bounds__(TC_F8_THREADS, 1)
   tc::fence_after_sync();
   const uint32_t tmem = *tslot;
 
-  auto unit_rows = [&](int u, int& e, int& r0, int& n, int& f) {
-    const int c = u / FT;
-    f = u % FT;
-    e = chunk_e[c];
-    r0 = chunk_r0[c];
-    n = min(128, offsets[e + 1] - r0);
+  struct Unit {
+    bool down;
+    int c, e, r0, n, f, w1, nk;
   };
-  // per-stage buffers: [FP8 staging x NW][bf16 tile x NW][token rows]
+  auto unit_of = [&](int u) {
+    Unit x;
+    x.down = u >= U1;
+    const int v = x.down ? u - U1 : u, ft = x.down ? FT2 : FT1;
+    x.c = v / ft;
+    x.f = v % ft;
+    x.e = chunk_e[x.c];
+    x.r0 = chunk_r0[x.c];
+    x.n = min(128, offsets[x.e + 1] - x.r0);
+    x.w1 = x.down ? x.e * d + x.f * 256 : x.e * I + x.f * 128;  // first weight row of tile 0
+    x.nk = (x.down ? I : d) / TC_KB;
+    return x;
+  };
   auto f8_at = [&](int s, int w) { return smem + s * Cfg::STAGE + w * Cfg::F8_TILE; };
-  auto bf_at = [&](int s, int w) {
-    return smem + s * Cfg::STAGE + Cfg::NW * Cfg::F8_TILE + w * TC_SUB_A;
-  };
-  auto x_at = [&](int s) {
-    return smem + s * Cfg::STAGE + Cfg::NW * Cfg::F8_TILE + Cfg::NW * TC_SUB_A;
-  };
+  auto bf_at = [&](int s, int w) { return smem + s * Cfg::STAGE + 2 * Cfg::F8_TILE + w * TC_SUB_A; };
+  auto x_at = [&](int s) { return smem + s * Cfg::STAGE + 2 * Cfg::F8_TILE + 2 * TC_SUB_A; };
 
   if (warp == 0) {
     if (lane == 0) {
-      tc::prefetch_tmap(&mW);
-      if (GATEUP) tc::prefetch_tmap(&mW2);
+      tc::prefetch_tmap(&mWg);
+      tc::prefetch_tmap(&mWu);
       tc::prefetch_tmap(&mX);
+      tc::prefetch_tmap(&mWd);
+      tc::prefetch_tmap(&mH);
       int it = 0;
-      for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
-        int e, r0, n, f;
-        unit_rows(u, e, r0, n, f);
-        const int nb = (n + 31) >> 5;
-        const uint32_t bytes = Cfg::NW * Cfg::F8_TILE + (uint32_t)nb * 32 * TC_KB * 2;
-        const int wrow = e * w_rows_per_expert + f * 128;
-        for (int kb = 0; kb < nk; ++kb, ++it) {
+      bool ok = true;
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+        const Unit x = unit_of(u);
+        if (x.down) {
+          const uint64_t t0 = tc::global_ns();
+          while (ld_acquire(ready + x.c) < FT1) {
+            __nanosleep(64);
+            if (tc::global_ns() - t0 > 2000000000ull) {
+              atomicOr(err, ERR_TIMEOUT);
+              ok = false;
+              break;
+            }
+          }
+          if (!ok) break;
+          asm volatile("fence.proxy.async.global;" ::: "memory");  // before the TMA reads
+        }
+        const int nb = (x.n + 31) >> 5;
+        const uint32_t bytes = 2 * Cfg::F8_TILE + (uint32_t)nb * 32 * TC_KB * 2;
+        for (int kb = 0; kb < x.nk; ++kb, ++it) {
           const int s = it % ST;
           const uint32_t ph = (it / ST) & 1;
           if (it >= ST && !tc::mbar_wait(empty + s, ph ^ 1)) {
             atomicOr(err, ERR_TIMEOUT);
-            u = n_units;
+            ok = false;
             break;
           }
-          const int kx = ((kb + f) % nk) * TC_KB;
+          const int kx = ((kb + x.f) % x.nk) * TC_KB;
           tc::mbar_expect_tx(full + s, bytes);
-          tc::tma_load_2d(f8_at(s, 0), &mW, full + s, kx, wrow);
-          if (GATEUP) tc::tma_load_2d(f8_at(s, 1), &mW2, full + s, kx, wrow);
+          if (x.down) {
+            tc::tma_load_2d(f8_at(s, 0), &mWd, full + s, kx, x.w1);
+            tc::tma_load_2d(f8_at(s, 1), &mWd, full + s, kx, x.w1 + 128);
+          } else {
+            tc::tma_load_2d(f8_at(s, 0), &mWg, full + s, kx, x.w1);
+            tc::tma_load_2d(f8_at(s, 1), &mWu, full + s, kx, x.w1);
+          }
           for (int j = 0; j < nb; ++j)
-            tc::tma_load_2d(x_at(s) + j * 32 * TC_KB * 2, &mX, full + s, kx, r0 + 32 * j);
+            tc::tma_load_2d(x_at(s) + j * 32 * TC_KB * 2, x.down ? &mH : &mX, full + s, kx,
+                            x.r0 + 32 * j);
         }
       }
     }
@@ -130,16 +168,15 @@ __global__ void __launch_bounds__(TC_F8_THREADS, 1)
       int it = 0, ui = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++ui) {
-        int e, r0, n, f;
-        unit_rows(u, e, r0, n, f);
-        const int npad = ((n + 31) >> 5) << 5;
+        const Unit x = unit_of(u);
+        const int npad = ((x.n + 31) >> 5) << 5;
         const uint32_t idesc = tc::idesc_bf16(128, npad);
         if (ui > 0 && !tc::mbar_wait(tempty, (ui - 1) & 1)) {
           atomicOr(err, ERR_TIMEOUT);
           break;
         }
         tc::fence_after_sync();
-        for (int kb = 0; kb < nk; ++kb, ++it) {
+        for (int kb = 0; kb < x.nk; ++kb, ++it) {
           const int s = it % ST;
           const uint32_t ph = (it / ST) & 1;
           if (!tc::mbar_wait(conv + s, ph)) {
@@ -155,7 +192,7 @@ __global__ void __launch_bounds__(TC_F8_THREADS, 1)
             const uint32_t acc = (kb | k) != 0;
             const uint64_t bd = tc::sdesc_k128(b0 + k * 32);
             tc::mma_bf16(tmem, tc::sdesc_k128(a0 + k * 32), bd, idesc, acc);
-            if (GATEUP) tc::mma_bf16(tmem + 128, tc::sdesc_k128(a0 + TC_SUB_A + k * 32), bd, idesc, acc);
+            tc::mma_bf16(tmem + 128, tc::sdesc_k128(a0 + TC_SUB_A + k * 32), bd, idesc, acc);
           }
           tc::mma_commit(empty + s);
         }
@@ -163,55 +200,60 @@ __global__ void __launch_bounds__(TC_F8_THREADS, 1)
       }
     }
   } else if (warp >= 10) {
-    // converters: thread t handles 16-byte chunk (t % 4) of FP8 rows (t / 4) + 64 i
+    // converters: thread t handles 16-byte chunk (t % 4) of FP8 rows (t / 4) + 64 i.
+    // A unit's scales (256 rows x K/128) are brought into shared memory once; after a
+    // timed-out wait the warp skips the waits but keeps step with the other converters.
     const int t = threadIdx.x - 320;  // 0..255
     const int chunk = t & 3;
     int it = 0;
+    bool dead = false;
     for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
-      int e, r0, n, f;
-      unit_rows(u, e, r0, n, f);
-      const int wrow = e * w_rows_per_expert + f * 128;
-      bool ok = true;
-      for (int kb = 0; kb < nk; ++kb, ++it) {
+      const Unit x = unit_of(u);
+      const int kscale = (x.down ? I : d) / 128;
+      const int half = 128 * kscale;
+      asm volatile("bar.sync 2, 256;" ::: "memory");  // the previous unit's scales are read
+      for (int i = 4 * t; i < 2 * half; i += 1024) {
+        const float* src = x.down ? sWd + (size_t)x.w1 * kscale + i
+                           : i < half ? sWg + (size_t)x.w1 * kscale + i
+                                      : sWu + (size_t)x.w1 * kscale + (i - half);
+        *reinterpret_cast<float4*>(sscl + i) = __ldg(reinterpret_cast<const float4*>(src));
+      }
+      asm volatile("bar.sync 2, 256;" ::: "memory");
+      for (int kb = 0; kb < x.nk; ++kb, ++it) {
         const int s = it % ST;
         const uint32_t ph = (it / ST) & 1;
-        const int kx = ((kb + f) % nk) * TC_KB;
-        // the scales do not depend on the staged tile: request them before waiting
-        float scl[Cfg::NW][2];
-#pragma unroll
-        for (int w = 0; w < Cfg::NW; ++w)
-#pragma unroll
-          for (int i = 0; i < 2; ++i)
-            scl[w][i] = (w == 0 ? sW : sW2)[(size_t)(wrow + (t >> 2) + 64 * i) * kscale + kx / 128];
-        bool ready = true;
-        if (lane == 0) ready = tc::mbar_wait(full + s, ph);
-        ready = __shfl_sync(0xffffffffu, ready ? 1 : 0, 0) != 0;
-        if (!ready) {
-          if (lane == 0) atomicOr(err, ERR_TIMEOUT);
-          ok = false;
-          break;
+        const int kx = ((kb + x.f) % x.nk) * TC_KB;
+        if (!dead) {
+          bool rdy = true;
+          if (lane == 0) rdy = tc::mbar_wait(full + s, ph);
+          rdy = __shfl_sync(0xffffffffu, rdy ? 1 : 0, 0) != 0;
+          if (!rdy) {
+            if (lane == 0) atomicOr(err, ERR_TIMEOUT);
+            dead = true;
+          }
         }
+        if (!dead) {
 #pragma unroll
-        for (int w = 0; w < Cfg::NW; ++w) {
-          const uint8_t* src = f8_at(s, w);
-          uint8_t* dst = bf_at(s, w);
+          for (int w = 0; w < 2; ++w) {
+            const uint8_t* src = f8_at(s, w);
+            uint8_t* dst = bf_at(s, w);
 #pragma unroll
-          for (int i = 0; i < 2; ++i) {
-            const int r = (t >> 2) + 64 * i;
-            const float scale = scl[w][i];
-            const uint4 q = *reinterpret_cast<const uint4*>(src + r * 64 + chunk * 16);
-            const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
-            uint32_t o[8];
+            for (int i = 0; i < 2; ++i) {
+              const int r = (t >> 2) + 64 * i;
+              const float scale = sscl[(128 * w + r) * kscale + kx / 128];
+              const uint4 q = *reinterpret_cast<const uint4*>(src + r * 64 + chunk * 16);
+              const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
+              uint32_t o[8];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              o[2 * j] = f8x2_scaled(qw[j] & 0xffffu, scale);
-              o[2 * j + 1] = f8x2_scaled(qw[j] >> 16, scale);
+              for (int j = 0; j < 4; ++j) {
+                o[2 * j] = f8x2_scaled(qw[j] & 0xffffu, scale);
+                o[2 * j + 1] = f8x2_scaled(qw[j] >> 16, scale);
+              }
+              uint8_t* rowp = dst + r * 128;
+              const int c0 = (2 * chunk) ^ (r & 7), c1 = (2 * chunk + 1) ^ (r & 7);
+              *reinterpret_cast<uint4*>(rowp + c0 * 16) = make_uint4(o[0], o[1], o[2], o[3]);
+              *reinterpret_cast<uint4*>(rowp + c1 * 16) = make_uint4(o[4], o[5], o[6], o[7]);
             }
-            // 16 bf16 values = two 16-byte chunks (2 chunk, 2 chunk + 1) of row r
-            uint8_t* rowp = dst + r * 128;
-            const int c0 = (2 * chunk) ^ (r & 7), c1 = (2 * chunk + 1) ^ (r & 7);
-            *reinterpret_cast<uint4*>(rowp + c0 * 16) = make_uint4(o[0], o[1], o[2], o[3]);
-            *reinterpret_cast<uint4*>(rowp + c1 * 16) = make_uint4(o[4], o[5], o[6], o[7]);
           }
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -220,7 +262,6 @@ __global__ void __launch_bounds__(TC_F8_THREADS, 1)
           asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(tc::smem_addr(conv + s))
                        : "memory");
       }
-      if (!ok) break;
     }
   } else {
     // epilogue warps 2..9 -> TMEM lane quarter (warp % 4), token chunks of parity hf
@@ -228,45 +269,51 @@ __global__ void __launch_bounds__(TC_F8_THREADS, 1)
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     int ui = 0;
     for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++ui) {
-      int e, r0, n, f;
-      unit_rows(u, e, r0, n, f);
-      bool ready = true;
-      if (lane == 0) ready = tc::mbar_wait(tfull, ui & 1);
-      ready = __shfl_sync(0xffffffffu, ready ? 1 : 0, 0) != 0;
-      if (!ready) {
-        if (lane == 0) atomicOr(err, ERR_TIMEOUT);
-        break;
-      }
+      const Unit x = unit_of(u);
+      bool rdy = true;
+      if (lane == 0) rdy = tc::mbar_wait(tfull, ui & 1);
+      rdy = __shfl_sync(0xffffffffu, rdy ? 1 : 0, 0) != 0;
+      // on a timeout the warp records it and keeps step with the other epilogue warps
+      if (!rdy && lane == 0) atomicOr(err, ERR_TIMEOUT);
       tc::fence_after_sync();
-      const int fr = f * 128 + 32 * q + lane;
-      const int nch = (n + 31) >> 5;
+      const int nch = rdy ? (x.n + 31) >> 5 : 0;
+      if (!x.down) {
+        const int fr = x.f * 128 + 32 * q + lane;
 #pragma unroll 1
-      for (int c = hf; c < nch; c += 2) {
-        float v[32];
-        tc::tmem_ld32(tmem + lane_base + c * 32, v);
-        if (GATEUP) {
-          float g2[32];
-          tc::tmem_ld32(tmem + lane_base + 128 + c * 32, g2);
-          bf16* o = reinterpret_cast<bf16*>(out);
+        for (int c = hf; c < nch; c += 2) {
+          float g[32], v[32];
+          tc::tmem_ld32(tmem + lane_base + c * 32, g);
+          tc::tmem_ld32(tmem + lane_base + 128 + c * 32, v);
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const int tt = c * 32 + j;
-            if (tt < n) o[(size_t)(r0 + tt) * ldo + fr] = __float2bfloat16_rn(silu(v[j]) * g2[j]);
+            if (tt < x.n) hb[(size_t)(x.r0 + tt) * I + fr] = __float2bfloat16_rn(silu(g[j]) * v[j]);
           }
-        } else {
-          float* o = reinterpret_cast<float*>(out);
+        }
+      } else {
+#pragma unroll 1
+        for (int half2 = 0; half2 < 2; ++half2) {
+          const int fr = x.f * 256 + half2 * 128 + 32 * q + lane;
+#pragma unroll 1
+          for (int c = hf; c < nch; c += 2) {
+            float v[32];
+            tc::tmem_ld32(tmem + lane_base + half2 * 128 + c * 32, v);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int tt = c * 32 + j;
-            if (tt < n) o[(size_t)(r0 + tt) * ldo + fr] = gate_of[r0 + tt] * v[j];
+            for (int j = 0; j < 32; ++j) {
+              const int tt = c * 32 + j;
+              if (tt < x.n) yb[(size_t)(x.r0 + tt) * d + fr] = gate_of[x.r0 + tt] * v[j];
+            }
           }
         }
       }
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0)
-        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(tc::smem_addr(tempty))
-                     : "memory");
+      if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(tc::smem_addr(tempty)) : "memory");
+      if (!x.down) {
+        __threadfence();
+        asm volatile("bar.sync 1, 256;" ::: "memory");  // the eight epilogue warps
+        if (warp == 2 && lane == 0) atomicAdd(ready + x.c, 1);
+      }
     }
   }
   tc::fence_before_sync();

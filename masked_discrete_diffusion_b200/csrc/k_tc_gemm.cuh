@@ -1016,9 +1016,9 @@ dg_status tc_gemm_add_residual(dg_model* m, const bf16* A, const void* W, float*
                                int K, cudaStream_t st);
 dg_status tc_gemm_swiglu(dg_model* m, const bf16* A, const void* Wg, const void* Wu, bf16* out,
                          int M, int N, int K, cudaStream_t st);
-dg_status tc_moe_gate_up(dg_model* m, int l, const bf16* X, bf16* hb, int grid_y, cudaStream_t st);
-dg_status tc_moe_down(dg_model* m, int l, const bf16* H, float* yb, int grid_y, cudaStream_t st);
 dg_status tc_moe_experts(dg_model* m, int l, const bf16* X, bf16* hb, float* yb, cudaStream_t st);
+dg_status tc_moe_experts_f8(dg_model* m, int l, const bf16* X, bf16* hb, float* yb,
+                            cudaStream_t st);
 dg_status tc_lmhead_stats(dg_model* m, const bf16* xn, int M, float* ent, int32_t* amax,
                           cudaStream_t st);
 dg_status tc_attention(dg_model* m, const bf16* q, int B, int nq, int qpos0, const dg_kv* kv,

@@ -133,7 +133,7 @@ constexpr int DENSE_BN = 64, DENSE_MT = 2, DENSE_ST = 5, DUAL_ST = 4;
 constexpr int QKV_ST = 4, RT_ST = 4;
 constexpr int LM_BN = 256, LM_ST = 3;
 constexpr int MOE_ST = 4;
-constexpr int GU8_ST = 3, DN8_ST = 5;
+constexpr int MOE8_ST = 3;
 
 }  // namespace
 
@@ -143,6 +143,10 @@ dg_status tc_prepare(dg_model* m) {
   if (c.d_model % 256 || c.expert_inter % 128 || c.shared_inter % 64 || qkv_n % 64 ||
       (c.n_q_heads * c.head_dim) % 64) {
     set_error("tensor-core tiling needs d %% 256, I %% 128, Is %% 64, (Hq+2Hkv)h %% 64 and Hq h %% 64");
+    return DG_ERR_UNSUPPORTED;
+  }
+  if (c.dtype == DG_BF16_FP8EXP && (c.d_model > 4096 || c.expert_inter > 4096)) {
+    set_error("FP8 expert kernel keeps a unit's scales in shared memory: d and I <= 4096");
     return DG_ERR_UNSUPPORTED;
   }
   TcState* s = new TcState();
@@ -175,8 +179,7 @@ dg_status tc_prepare(dg_model* m) {
                   DenseCfg<128, 1, false, RT_ST>::SMEM));
   DG_TRY(set_smem(tc_dense_kernel<128, DENSE_MT, false, QKV_ST, EpiQkvRope>,
                   DenseCfg<128, DENSE_MT, false, QKV_ST>::SMEM + EpiQkvRope::kExtraSmem));
-  DG_TRY(set_smem(tc_expert_f8_kernel<true, GU8_ST>, ExpertF8Cfg<true, GU8_ST>::SMEM));
-  DG_TRY(set_smem(tc_expert_f8_kernel<false, DN8_ST>, ExpertF8Cfg<false, DN8_ST>::SMEM));
+  DG_TRY(set_smem(tc_moe_f8_kernel<MOE8_ST>, MoeF8Cfg<MOE8_ST>::smem_bytes(4096, 4096)));
   cudaDeviceGetAttribute(&s->n_sm, cudaDevAttrMultiProcessorCount, m->device);
   return DG_OK;
 }
@@ -283,48 +286,31 @@ dg_status tc_lmhead_stats(dg_model* m, const bf16* xn, int M, float* ent, int32_
   return DG_OK;
 }
 
-template <bool GATEUP, int ST>
-static dg_status launch_expert_f8(dg_model* m, const CUtensorMap& w, const CUtensorMap& w2,
-                                  const CUtensorMap& x, const float* s1, const float* s2,
-                                  int w_rows, int K, int FT, void* out, int ldo,
-                                  const float* gate_of, cudaStream_t st) {
-  typedef ExpertF8Cfg<GATEUP, ST> Cfg;
+// FP8 expert weights: both phases in one persistent launch (tc_moe_f8_kernel)
+dg_status tc_moe_experts_f8(dg_model* m, int l, const bf16* X, bf16* hb, float* yb,
+                            cudaStream_t st) {
+  const dg_config& c = m->cfg;
+  const dg_layer_weights& L = m->layers[l];
+  const int E = c.n_experts, I = c.expert_inter, d = c.d_model;
   const Workspace& ws = m->ws;
-  cudaError_t e = launch_pdl((tc_expert_f8_kernel<GATEUP, ST>), state(m)->n_sm, TC_F8_THREADS,
-                             Cfg::SMEM, st, 1,
-                             w, w2, x, s1, s2, ws.tile_e, ws.tile_m0, ws.n_tiles, ws.offsets,
-                             w_rows, K, FT, out, ldo, gate_of, ws.err);
+  CUtensorMap wg, wu, x, wd, h;
+  DG_TRY(tmap(m, L.gate, (uint64_t)E * I, d, 128, &wg, true));
+  DG_TRY(tmap(m, L.up, (uint64_t)E * I, d, 128, &wu, true));
+  DG_TRY(tmap(m, X, ws.max_rows, d, 32, &x));
+  DG_TRY(tmap(m, L.down, (uint64_t)E * d, I, 128, &wd, true));
+  DG_TRY(tmap(m, hb, ws.max_rows, I, 32, &h));
+  cudaError_t e = launch_pdl((tc_moe_f8_kernel<MOE8_ST>), state(m)->n_sm, TC_F8_THREADS,
+                             MoeF8Cfg<MOE8_ST>::smem_bytes(d, I), st, 1, wg, wu, x, wd, h,
+                             (const float*)L.gate_scale, (const float*)L.up_scale,
+                             (const float*)L.down_scale, ws.tile_e, ws.tile_m0, ws.n_tiles,
+                             ws.offsets, I, d, hb, yb, (const float*)ws.gate_of, ws.ready,
+                             ws.err);
   ++m->launches;
   if (e != cudaSuccess) {
-    set_error("tc_expert_f8 launch: %s", cudaGetErrorString(e));
+    set_error("tc_moe_f8 launch: %s", cudaGetErrorString(e));
     return DG_ERR_CUDA;
   }
   return DG_OK;
-}
-
-// FP8 expert weights: gate/up, then down (two launches; bytes converted to bf16 in
-// shared memory)
-dg_status tc_moe_gate_up(dg_model* m, int l, const bf16* X, bf16* hb, int, cudaStream_t st) {
-  const dg_config& c = m->cfg;
-  const dg_layer_weights& L = m->layers[l];
-  const int E = c.n_experts, I = c.expert_inter, d = c.d_model;
-  CUtensorMap wg, wu, x;
-  DG_TRY(tmap(m, L.gate, (uint64_t)E * I, d, 128, &wg, true));
-  DG_TRY(tmap(m, L.up, (uint64_t)E * I, d, 128, &wu, true));
-  DG_TRY(tmap(m, X, m->ws.max_rows, d, 32, &x));
-  return launch_expert_f8<true, GU8_ST>(m, wg, wu, x, L.gate_scale, L.up_scale, I, d, I / 128,
-                                        hb, I, nullptr, st);
-}
-
-dg_status tc_moe_down(dg_model* m, int l, const bf16* H, float* yb, int, cudaStream_t st) {
-  const dg_config& c = m->cfg;
-  const dg_layer_weights& L = m->layers[l];
-  const int E = c.n_experts, I = c.expert_inter, d = c.d_model;
-  CUtensorMap wd, x;
-  DG_TRY(tmap(m, L.down, (uint64_t)E * d, I, 128, &wd, true));
-  DG_TRY(tmap(m, H, m->ws.max_rows, I, 32, &x));
-  return launch_expert_f8<false, DN8_ST>(m, wd, wd, x, L.down_scale, L.down_scale, d, I,
-                                         d / 128, yb, d, (const float*)m->ws.gate_of, st);
 }
 
 // bf16 expert weights: both phases in one persistent launch (tc_moe_kernel)
