@@ -84,7 +84,9 @@ class ClockSampler:
                 "reasons": sorted(reasons)}
 
 
-def dist_setup():
+def dist_setup(backend: str | None = None):
+    """One process per GPU: RANK / LOCAL_RANK / WORLD_SIZE from the launcher, NCCL
+    between the ranks (gloo when no GPU is visible, for the host-side tests)."""
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -93,8 +95,11 @@ def dist_setup():
         import datetime
 
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        if backend is None:
+            backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
     elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return world, rank, local
@@ -105,7 +110,8 @@ def max_over_ranks(x: float, world: int) -> float:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -114,6 +120,20 @@ def barrier(world: int):
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
+
+
+def job_throughput(world: int, units_per_rank: int, steps: int, ms_max: float) -> float:
+    """Whole-job units per second: every rank processes units_per_rank per step (weak
+    scaling), timed as the slowest rank's device time over the steps."""
+    return world * units_per_rank * steps / (ms_max / 1e3)
+
+
+def build_once(world: int, local: int):
+    """The node's local rank 0 builds the library (if out of date); the others wait."""
+    from masked_discrete_diffusion_b200 import build
+    if local == 0:
+        build.build()
+    barrier(world)
 
 
 # ---------------------------------------------------------------------------
@@ -213,7 +233,7 @@ def run_e2e(args, w, world, model, prompt, canvas, stream):
     f1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(f0.elapsed_time(f1), world)
-    e2e_val = world * B * C * args.steps / (e2e_ms / 1e3)
+    e2e_val = job_throughput(world, B * C, args.steps, e2e_ms)
 
     return e2e_val
 
@@ -222,10 +242,10 @@ def run_ours(args, w, world, rank, local):
     import numpy as np
     import torch
 
-    from masked_discrete_diffusion_b200 import binding, build, metrics
+    from masked_discrete_diffusion_b200 import binding, metrics
     from synth import model_inputs
 
-    build.build()
+    build_once(world, local)
     peaks, peak_src = load_peaks()
     tensors = model_inputs.weight_set(w, "cuda")
     model = binding.Model(binding.make_config(w), tensors)
@@ -267,7 +287,7 @@ def run_ours(args, w, world, rank, local):
     binding.dg_sync_status(model)
     barrier(world)
     ms_max = max_over_ranks(ms, world)
-    value = world * B * C * args.steps / (ms_max / 1e3)
+    value = job_throughput(world, B * C, args.steps, ms_max)
     ms_step = ms_max / args.steps
 
     # second timed pass of the same K steps with CUDA events recorded around every

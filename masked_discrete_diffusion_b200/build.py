@@ -32,14 +32,17 @@ def needs_build() -> bool:
 def build(force: bool = False, verbose: bool = False) -> str:
     if not force and not needs_build():
         return OUT
-    cmd = [nvcc(), *FLAGS, "-o", OUT + ".tmp", *[os.path.join(CSRC, s) for s in SOURCES]]
+    # one temporary name per process: ranks that build at once each replace the
+    # library atomically with a complete file
+    tmp = f"{OUT}.{os.getpid()}.tmp"
+    cmd = [nvcc(), *FLAGS, "-o", tmp, *[os.path.join(CSRC, s) for s in SOURCES]]
     if verbose:
         print(" ".join(cmd))
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         sys.stderr.write(r.stdout + r.stderr)
         raise RuntimeError("nvcc failed building libdg.so")
-    os.replace(OUT + ".tmp", OUT)
+    os.replace(tmp, OUT)
     return OUT
 
 
