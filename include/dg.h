@@ -114,7 +114,8 @@ const char* dg_last_error(void);
  * Errors: DG_ERR_INVALID_ARG (null, non-positive or inconsistent sizes, d_model not a
  * multiple of 8, C > 1024,
  * Hq not a multiple of Hkv, h odd), DG_ERR_UNSUPPORTED (a shape the tensor-core
- * kernels do not tile), DG_ERR_OOM, DG_ERR_CUDA. */
+ * kernels do not tile: bf16 and FP8 need d % 256, I % 128, Is % 64, (Hq + 2 Hkv) h % 64
+ * and Hq h % 64; FP8 experts also d, I <= 4096), DG_ERR_OOM, DG_ERR_CUDA. */
 dg_status dg_model_create(const dg_config* cfg, const dg_weights* w, dg_model** out);
 
 /* Synchronises the device and frees the model's workspace. NULL is a no-op. */
