@@ -26,9 +26,11 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# DRAM bytes per routed expert streamed by the gate/up + down kernels (ncu capture,
-# see the roofline computation below)
-DRAM_BYTES_PER_EXPERT = 98.38e6 / 9
+# DRAM bytes per routed expert streamed by the routed-expert kernel, from an ncu capture
+# of that kernel as it now stands (see the roofline computation below).  None until
+# recaptured: the last capture (98.38 MB for the 9 experts of a first forward) predates
+# the bounded wait for in-flight copies added to the kernel's producer.
+DRAM_BYTES_PER_EXPERT = None
 
 
 def load_peaks():

@@ -109,8 +109,10 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   const uint32_t tO = tmem + 256;  // S buffers at columns 0 and 128
   const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
 
+  int n_loaded = 0;  // tiles requested so far (thread 0): tiles 0 .. n_loaded - 1
   auto load_tile = [&](int i) {  // tile index i within this split -> stage i & 1
     const int t = my_lo + i;
+    ++n_loaded;
     uint8_t* st = sKV + (i & 1) * 4 * AT_SUB;
     uint64_t* fb = kv_full + (i & 1);
     tc::mbar_expect_tx(fb, 4 * AT_SUB);
@@ -276,8 +278,12 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   }
 
   // ---- merge of the cluster's splits: stage (m, l, O) rows in this CTA's K/V buffers
-  // (all loads were consumed, all MMAs are done), then the owner of each row sums the
-  // splits in rank order and writes the normalised bf16 row.
+  // (all loads have landed, all MMAs are done), then the owner of each row sums the
+  // splits in rank order and writes the normalised bf16 row.  After a timed-out wait,
+  // thread 0 first waits (bounded) for the copies it requested.
+  if (tid == 0 && nt > 0 &&
+      !(tc::mbar_wait(q_full, 0) && tc::drain_slots(kv_full, 2, n_loaded)))
+    atomicOr(err, ERR_TIMEOUT);
   __syncthreads();
   const uint32_t stg = tc::smem_addr(sKV);
   {

@@ -162,6 +162,7 @@ __global__ void __launch_bounds__(TC_F8_THREADS, 1)
                             x.r0 + 32 * j);
         }
       }
+      if (!tc::drain_slots(full, ST, it)) atomicOr(err, ERR_TIMEOUT);
     }
   } else if (warp == 1) {
     if (lane == 0) {

@@ -563,7 +563,8 @@ __global__ void __launch_bounds__(TC_DENSE_THREADS, 1)
       tc::prefetch_tmap(&mB);
       if (DUAL) tc::prefetch_tmap(&mB2);
     }
-    for (int kb = 0; kb < nk; ++kb) {
+    int kb = 0;
+    for (; kb < nk; ++kb) {
       const int s = kb % ST;
       const uint32_t ph = (kb / ST) & 1;
       if (kb >= ST && !tc::mbar_wait(empty + s, ph ^ 1)) {
@@ -581,6 +582,7 @@ __global__ void __launch_bounds__(TC_DENSE_THREADS, 1)
       for (int mt = 0; mt < MT; ++mt)
         tc::tma_load_2d(st + mt * TC_SUB_A, &mA, full + s, kx, m0 + mt * 128);
     }
+    if (!tc::drain_slots(full, ST, kb)) atomicOr(err, ERR_TIMEOUT);
   } else if (warp == 1 && lane == 0) {
     constexpr uint32_t idesc = tc::idesc_bf16(128, BN);
     bool ok = true;
@@ -899,6 +901,7 @@ __global__ void __launch_bounds__(TC_MOE_THREADS, 1)
                             x.r0 + 32 * j);
         }
       }
+      if (!tc::drain_slots(full, ST, it)) atomicOr(err, ERR_TIMEOUT);
     }
   } else if (warp == 1) {
     if (lane == 0) {

@@ -66,6 +66,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
   }
 }
 
+// Before a CTA stops using a pipeline (end of its work, or a timed-out wait): bounded
+// wait until the last copy issued into each of the `slots` stage barriers has landed,
+// so that no TMA write reaches this CTA's shared memory after it has moved on.  Stage
+// loads are numbered 0 .. issued - 1 and load i completes on barrier i % slots in phase
+// (i / slots) & 1.  A slot whose last copy has already landed returns at once.
+__device__ __forceinline__ bool drain_slots(uint64_t* full, int slots, int issued) {
+  bool ok = true;
+  for (int s = 0; s < slots && s < issued; ++s) {
+    const int last = issued - 1 - (issued - 1 - s) % slots;
+    ok = mbar_wait(full + s, (uint32_t)(last / slots) & 1) && ok;
+  }
+  return ok;
+}
+
 // ---------------------------------------------------------------- TMA
 // 2-D tiled bulk tensor load global -> shared, completion counted on `bar`.
 // x = innermost (element) coordinate, must be a multiple of 8 for bf16.
