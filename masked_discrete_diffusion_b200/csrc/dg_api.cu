@@ -142,8 +142,8 @@ template <class Path> static dg_status alloc_workspace(dg_model* m) {
   DG_TRY(ws_alloc(ws, &ws.counts, c.n_experts));
   DG_TRY(ws_alloc(ws, &ws.offsets, c.n_experts + 1));
   DG_TRY(ws_alloc(ws, &ws.tile_e, ws.max_tiles));
-  DG_TRY(ws_alloc(ws, &ws.ready, ws.max_tiles));
-  DG_TRY_CUDA(cudaMemset(ws.ready, 0, ws.max_tiles * sizeof(int32_t)));
+  DG_TRY(ws_alloc(ws, &ws.ready, ws.max_tiles + 1));  // + the expert kernel's unit counter
+  DG_TRY_CUDA(cudaMemset(ws.ready, 0, (ws.max_tiles + 1) * sizeof(int32_t)));
   DG_TRY(ws_alloc(ws, &ws.tile_m0, ws.max_tiles));
   DG_TRY(ws_alloc(ws, &ws.n_tiles, 1));
   DG_TRY(ws_alloc_v<TA>(ws, &ws.up, R * d));

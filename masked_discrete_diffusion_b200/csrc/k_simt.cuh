@@ -478,7 +478,8 @@ struct PermuteArgs {
   int max_tiles;
   unsigned long long* used;
   int32_t *load, *row_of, *tok_of;
-  int32_t* ready;  // per-tile counters of the routed-expert kernel, zeroed here (nullable)
+  int32_t* ready;  // per-tile counters of the routed-expert kernel and, after them, its
+                   // unit counter; all zeroed here (nullable)
 };
 
 template <class Acc>
@@ -556,7 +557,7 @@ __device__ void block_permute(const PermuteArgs& a, const Acc* __restrict__ gate
     *a.n_tiles = min(stl[tid], a.max_tiles);
   }
   if (write && a.ready)
-    for (int t = tid; t < a.max_tiles; t += nthr) a.ready[t] = 0;
+    for (int t = tid; t <= a.max_tiles; t += nthr) a.ready[t] = 0;  // and the unit counter
   __syncthreads();
   for (int j = tid; j < a.n_entries; j += nthr) {
     const int pos = carry[__ldcg(a.idx + j)] + rank[j];

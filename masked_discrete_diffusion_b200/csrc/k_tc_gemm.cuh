@@ -801,7 +801,7 @@ __global__ void __launch_bounds__(TC_MOE_THREADS, 1)
                   const int32_t* __restrict__ chunk_r0, const int32_t* __restrict__ n_chunks,
                   const int32_t* __restrict__ offsets, int I, int d, bf16* __restrict__ hb,
                   float* __restrict__ yb, const float* __restrict__ gate_of,
-                  int32_t* __restrict__ ready, int32_t* err) {
+                  int32_t* __restrict__ ready, int32_t* __restrict__ next, int32_t* err) {
   typedef MoeCfg<ST> Cfg;
   pdl_enter();  // the routing tables come from the preceding kernels
   extern __shared__ uint8_t smem_raw[];
@@ -810,7 +810,13 @@ __global__ void __launch_bounds__(TC_MOE_THREADS, 1)
   uint64_t* empty = full + ST;
   uint64_t* tfull = empty + ST;   // accumulators ready (MMA -> epilogue)
   uint64_t* tempty = tfull + 1;   // accumulators drained (epilogue -> MMA), 8 arrivals
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(tempty + 1);
+  // units taken by the TMA thread, in order, for the MMA thread and the epilogue leader
+  constexpr int QD = 4;
+  uint64_t* qfull = tempty + 1;   // [QD] unit id written (TMA thread)
+  uint64_t* qempty = qfull + QD;  // [QD] unit id read (MMA thread + epilogue leader)
+  int32_t* qid = reinterpret_cast<int32_t*>(qempty + QD);  // [QD]
+  int32_t* ubc = qid + QD;        // the epilogue leader's broadcast of the unit id
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(ubc + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nc = *n_chunks;
   const int FT1 = I / 128, FT2 = d / 256;
@@ -823,6 +829,10 @@ __global__ void __launch_bounds__(TC_MOE_THREADS, 1)
     }
     tc::mbar_init(tfull, 1);
     tc::mbar_init(tempty, 8);
+    for (int k = 0; k < QD; ++k) {
+      tc::mbar_init(qfull + k, 1);
+      tc::mbar_init(qempty + k, 2);
+    }
     tc::fence_mbar_init();
   }
   if (warp == 1) tc::tmem_alloc(tslot, Cfg::TCOLS);
@@ -846,6 +856,18 @@ __global__ void __launch_bounds__(TC_MOE_THREADS, 1)
     x.n = min(128, offsets[x.e + 1] - x.r0);
     return x;
   };
+  // the ui-th unit id of this block (n_units when there is none, or on a timeout)
+  auto take = [&](int ui) -> int {
+    const int k = ui % QD;
+    if (!tc::mbar_wait(qfull + k, (ui / QD) & 1)) {
+      atomicOr(err, ERR_TIMEOUT);
+      return n_units;
+    }
+    const int u = *reinterpret_cast<volatile int32_t*>(qid + k);
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(tc::smem_addr(qempty + k))
+                 : "memory");
+    return u;
+  };
 
   if (warp == 0) {
     if (lane == 0) {
@@ -856,7 +878,19 @@ __global__ void __launch_bounds__(TC_MOE_THREADS, 1)
       tc::prefetch_tmap(&mH);
       int it = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      for (int qi = 0;; ++qi) {
+        // blocks take the next unit when they are ready for it (gate/up units first,
+        // so a down unit only ever waits for units that running blocks have taken)
+        const int k = qi % QD;
+        if (qi >= QD && !tc::mbar_wait(qempty + k, ((qi / QD) & 1) ^ 1)) {
+          atomicOr(err, ERR_TIMEOUT);
+          break;  // the readers give up on their own bounded waits
+        }
+        const int u = ok ? atomicAdd(next, 1) : n_units;
+        qid[k] = u < n_units ? u : n_units;
+        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(tc::smem_addr(qfull + k))
+                     : "memory");
+        if (u >= n_units) break;
         const Unit x = unit_of(u);
         if (x.down) {
           // the chunk's hidden rows are complete once all its phase-1 units have counted
@@ -869,7 +903,7 @@ __global__ void __launch_bounds__(TC_MOE_THREADS, 1)
               break;
             }
           }
-          if (!ok) break;
+          if (!ok) continue;  // publish the end of the work next
           asm volatile("fence.proxy.async.global;" ::: "memory");  // before the TMA reads
         }
         const int nk = (x.down ? I : d) / TC_KB;
@@ -905,9 +939,11 @@ __global__ void __launch_bounds__(TC_MOE_THREADS, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      int it = 0, ui = 0;
+      int it = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++ui) {
+      for (int ui = 0; ok; ++ui) {
+        const int u = take(ui);
+        if (u >= n_units) break;
         const Unit x = unit_of(u);
         const int nk = (x.down ? I : d) / TC_KB;
         const int npad = ((x.n + 31) >> 5) << 5;
@@ -945,8 +981,13 @@ __global__ void __launch_bounds__(TC_MOE_THREADS, 1)
     // epilogue warps 2..9 -> TMEM lane quarter (warp % 4), token chunks of parity hf
     const int q = warp & 3, hf = (warp - 2) >> 2;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-    int ui = 0;
-    for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++ui) {
+    for (int ui = 0;; ++ui) {
+      // warp 2 takes the unit id for the eight epilogue warps
+      if (warp == 2 && lane == 0) *reinterpret_cast<volatile int32_t*>(ubc) = take(ui);
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      const int u = *reinterpret_cast<volatile int32_t*>(ubc);
+      asm volatile("bar.sync 1, 256;" ::: "memory");  // read by all before the next take
+      if (u >= n_units) break;
       const Unit x = unit_of(u);
       bool rdy = true;
       if (lane == 0) rdy = tc::mbar_wait(tfull, ui & 1);

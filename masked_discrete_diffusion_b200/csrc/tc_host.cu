@@ -329,7 +329,8 @@ dg_status tc_moe_experts(dg_model* m, int l, const bf16* X, bf16* hb, float* yb,
   cudaError_t e = launch_pdl((tc_moe_kernel<MOE_ST>), state(m)->n_sm, TC_MOE_THREADS,
                              MoeCfg<MOE_ST>::SMEM, st, 1, wg, wu, x, wd, h, ws.tile_e,
                              ws.tile_m0, ws.n_tiles, ws.offsets, I, d, hb, yb,
-                             (const float*)ws.gate_of, ws.ready, ws.err);
+                             (const float*)ws.gate_of, ws.ready, ws.ready + ws.max_tiles,
+                             ws.err);
   ++m->launches;
   if (e != cudaSuccess) {
     set_error("tc_moe launch: %s", cudaGetErrorString(e));
