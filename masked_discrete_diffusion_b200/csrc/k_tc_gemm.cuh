@@ -777,9 +777,12 @@ __global__ void __launch_bounds__(TC_DENSE_THREADS, 1)
 //     of expert e against the chunk's rows X -> hb[r, f*128 + i] = silu(g) * u (bf16);
 //   phase 2, unit v = c * FT2 + f (FT2 = d / 256): down rows f*256 .. +255 of
 //     expert e (two 128-row tiles) against hb -> yb[r, f*256 + i] = gate_of[r] * acc.
-// A block takes units blockIdx.x, + gridDim.x, ... over phase 1 then phase 2, so
-// it waits (for a chunk's phase-1 units, counted in ready[c]) only after finishing
-// its own phase-1 units: no block waits for a block that waits.
+// Units are numbered phase 1 first.  A block's TMA thread takes the next number from
+// the device counter `next` (zeroed with `ready` before the launch) once it has issued
+// the loads of its current unit, and passes it to the MMA thread and the epilogue
+// through a small queue in shared memory.  A phase-2 unit waits for its chunk's
+// phase-1 units (counted in ready[c]); those were taken earlier by running blocks,
+// whose progress never depends on a waiting block, so every wait ends.
 // Both phases run two MMAs per k-step (weights on the MMA's M side, tokens on N)
 // into TMEM columns 0 and 128.  320 threads: warp 0 TMA, warp 1 MMA, warps 2..9
 // epilogue (warps w and w + 4 share a TMEM lane quarter and split the token chunks).
