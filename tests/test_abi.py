@@ -65,3 +65,43 @@ def test_kv_destroy_after_model_destroy_is_safe_without_device(lib):
     # only null handles can be exercised without a GPU; the ordering itself is
     # covered on the GPU by the model/KV lifetime test
     assert lib.dg_kv_destroy(None) == 0 and lib.dg_model_destroy(None) == 0
+
+
+def test_null_handles_and_bad_sizes_rejected_without_device(lib):
+    """Every entry point that takes a handle or buffers checks them before any CUDA call
+    (DG_ERR_INVALID_ARG = 1), so these run on a machine without a GPU."""
+    vp, i64 = ctypes.c_void_p, ctypes.c_int64
+    fake = vp(256)
+    n = i64()
+    calls = {
+        "dg_sync_status": (None, None),
+        "dg_prefill": (None, fake, 1, 8, ctypes.byref(vp()), None),
+        "dg_kv_info": (None, None, None, None),
+        "dg_kv_read": (None, fake, fake, None),
+        "dg_denoise_step": (None, None, fake, fake, 1, 4, 1.0, fake, fake, fake, None),
+        "dg_generate_block": (None, None, 4, 1.0, fake, None, None, None),
+        "dg_debug_forward": (None, None, fake, 1, 4, fake, fake, None, None, None),
+        "dg_profile_start": (None,),
+        "dg_profile_stop": (None, None, None),
+        "dg_launch_count": (None, ctypes.byref(n)),
+        "dg_expert_units": (None, ctypes.byref(n)),
+        "dg_block_loop_launches": (None, ctypes.byref(n)),
+        "dg_op_gemm": (None, fake, fake, fake, 1, 64, 64, None),
+        "dg_op_moe": (None, 0, fake, fake, 1, None),
+    }
+    for name, args in calls.items():
+        assert getattr(lib, name)(*args) == 1, name
+        assert lib.dg_last_error(), name
+    # the allocation-free LM head: pointers, ranges and alignment
+    na = lib.dg_lmhead_entropy_noalloc
+    ok = dict(h=fake, w=fake, M=256, V=262144, d=2048, eps=1e-6, s=8.0, e=fake, a=fake)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return na(a["h"], a["w"], a["M"], a["V"], a["d"], a["eps"], a["s"], a["e"], a["a"], None)
+
+    for bad in (dict(h=None), dict(w=None), dict(e=None), dict(a=None), dict(M=0),
+                dict(M=257), dict(V=0), dict(V=262145), dict(d=32), dict(d=100),
+                dict(d=4160), dict(w=vp(264)), dict(eps=-1.0), dict(s=float("inf")),
+                dict(s=float("nan"))):
+        assert call(**bad) == 1, bad
