@@ -1,0 +1,69 @@
+"""The golden files (written from the oracle alone by tests/golden/make_golden.py) on
+CPU: the fields the GPU parity tests read are present and consistent, and the
+distances between the oracle's bf16-storage run and its fp64 run behave as the
+tolerance reading for the deep workloads assumes — small after one layer, amplified
+through thirty."""
+import glob
+import os
+
+import numpy as np
+import pytest
+
+from gpu_helpers import max_abs_rel, storage_tol
+
+HERE = os.path.join(os.path.dirname(__file__), "golden")
+FILES = sorted(glob.glob(os.path.join(HERE, "*.npz")))
+STATED = 2e-2
+
+
+def _load(name):
+    path = os.path.join(HERE, name)
+    if not os.path.exists(path):
+        pytest.skip(f"{name} missing")
+    return np.load(path)
+
+
+@pytest.mark.parametrize("path", FILES, ids=[os.path.basename(f) for f in FILES])
+def test_fields_and_shapes(path):
+    g = np.load(path)
+    for k in ("H", "argmax", "logits", "logit_rows", "logit_cols", "margin", "kv_last",
+              "H_s16", "logits_s16", "kv_last_s16"):
+        assert k in g.files, k
+    C = g["H"].shape[0]
+    assert g["argmax"].shape == (C,) and g["margin"].shape == (C,)
+    assert g["logits"].shape == (len(g["logit_rows"]), len(g["logit_cols"]))
+    assert g["logits_s16"].shape == g["logits"].shape
+    assert g["kv_last_s16"].shape == g["kv_last"].shape and g["H_s16"].shape == g["H"].shape
+    assert np.all(g["H"] >= 0) and np.all(np.isfinite(g["logits"]))
+    assert np.all(g["margin"] >= 0)
+    # the sampled logit rows and columns index real canvas rows and vocabulary entries
+    assert g["logit_rows"].min() >= 0 and g["logit_rows"].max() < C
+    assert g["logit_cols"].min() >= 0
+
+
+def test_one_layer_storage_distance_within_stated_tolerance():
+    for name in ("layer1-bf16.npz", "layer1-fp8exp-p4096.npz"):
+        g = _load(name)
+        assert max_abs_rel(g["logits_s16"], g["logits"]) < STATED / 2
+        assert max_abs_rel(g["H_s16"], g["H"]) < STATED
+        for j in range(2):  # layer 0's keys and values
+            assert max_abs_rel(g["kv_last_s16"][0, j], g["kv_last"][0, j]) < STATED / 2
+
+
+def test_thirty_layers_amplify_storage_noise():
+    one, deep = _load("layer1-bf16.npz"), _load("full30-bf16.npz")
+    # same first layer: layer 0's K/V see the same storage noise in both workloads
+    for j in range(2):
+        a = max_abs_rel(one["kv_last_s16"][0, j], one["kv_last"][0, j])
+        b = max_abs_rel(deep["kv_last_s16"][0, j], deep["kv_last"][0, j])
+        assert 0.5 < b / a < 2.0
+    # the last layer's K/V, the logits and the entropies move several times further
+    assert max_abs_rel(deep["kv_last_s16"][1, 0], deep["kv_last"][1, 0]) > \
+        3 * max_abs_rel(deep["kv_last_s16"][0, 0], deep["kv_last"][0, 0])
+    assert max_abs_rel(deep["logits_s16"], deep["logits"]) > \
+        3 * max_abs_rel(one["logits_s16"], one["logits"])
+    assert max_abs_rel(deep["H_s16"], deep["H"]) > 3 * max_abs_rel(one["H_s16"], one["H"])
+    # so the deep tolerances come from the storage run, the shallow ones stay stated
+    assert storage_tol(deep, "H", STATED) > STATED
+    assert storage_tol(deep, "logits", STATED) > STATED
+    assert storage_tol(deep, "kv_last", STATED, (0, 0)) == STATED
