@@ -304,9 +304,28 @@ def dg_expert_units(model: Model) -> int:
     return out.value
 
 
+def _check_noalloc_args(hidden, lm_head):
+    """The C entry point reads hidden as fp32 [M, d] and lm_head as bf16 [V, d] on the
+    current device; anything else would be read out of bounds or misinterpreted, so it
+    is rejected here, before any launch."""
+    if hidden.dim() != 2 or hidden.dtype != torch.float32:
+        raise ValueError(f"hidden must be a 2-D float32 tensor, got {hidden.dtype} "
+                         f"{tuple(hidden.shape)}")
+    if lm_head.dim() != 2 or lm_head.dtype != torch.bfloat16:
+        raise ValueError(f"lm_head must be a 2-D bfloat16 tensor, got {lm_head.dtype} "
+                         f"{tuple(lm_head.shape)}")
+    if lm_head.shape[1] != hidden.shape[1]:
+        raise ValueError(f"lm_head has {lm_head.shape[1]} columns, hidden has "
+                         f"{hidden.shape[1]}")
+    for name, t in (("hidden", hidden), ("lm_head", lm_head)):
+        if not t.is_cuda or t.device.index != torch.cuda.current_device():
+            raise ValueError(f"{name} must be a CUDA tensor on the current device")
+
+
 def dg_lmhead_entropy_noalloc(hidden, lm_head, rms_eps: float, logit_scale: float, stream=None):
     """Entropy [M] and argmax [M] of logit_scale * RMSNorm(hidden) lm_head^T, computed
     without any device allocation by the library (static scratch)."""
+    _check_noalloc_args(hidden, lm_head)
     M, d = hidden.shape
     V = lm_head.shape[0]
     ent = torch.empty(M, dtype=torch.float32, device="cuda")

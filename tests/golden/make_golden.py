@@ -16,6 +16,18 @@ storage variant (H_s16, argmax_s16, logits_s16, kv_last_s16): the sensitivity of
 workload to bf16 activation storage, from which the deep workloads' tolerances follow.
 The suffix "+s16only" adds those fields to an existing file (the fp64 run is not
 repeated).
+
+Two further modes on a deep workload:
+  <name>@depths  -> <name>-depths.npz: the first forward of the models made of the
+     first k layers of the workload (k in DEPTHS; the weights are seeded per layer
+     name, so these are the same layers the full model holds), fp64 and bf16-storage
+     runs, at every k: H, argmax, margin, sampled logits and layer k-1's last keys and
+     values.  One pass through the layers serves every depth (the prompt pass and the
+     canvas pass interleave layer by layer, so the canvas state after layer k-1 is the
+     k-layer model's final residual).
+  <name>@block   -> <name>-block.npz: the oracle's whole block (all [MASK], up to T
+     forwards, the entropy-bound sampler after each): per step the input canvas, the
+     steps left, H, argmax, margin and the number committed; the number of forwards.
 """
 from __future__ import annotations
 
@@ -95,10 +107,89 @@ def make(name: str, canvas_index: int = 0, storage_variant: bool = False):
           f"min router gap {min(rmarg):.3g}, sampler n {n2}")
 
 
+DEPTHS = (1, 2, 4, 8, 16, 30)
+
+
+def depth_sweep(name: str, depths=DEPTHS):
+    """Oracle outputs of the first forward of the k-layer prefixes of the workload."""
+    w = workloads.get(name)
+    t0 = time.time()
+    prompt = model_inputs.prompt(w.with_(batch=1))[0].numpy()
+    canvas = np.full(w.canvas, w.mask_id)
+    P = prompt.shape[0]
+    cols = np.arange(0, w.vocab, max(1, w.vocab // 4096))
+    rows = [r for r in LOGIT_ROWS if r < w.canvas]
+    out = dict(depths=np.array([k for k in depths if k <= w.n_layers]),
+               logit_rows=np.array(rows), logit_cols=cols)
+    for storage, tag in (("fp64", ""), ("bf16", "_s16")):
+        ws = om.Weights(w, keep_layers=False, storage=storage)
+        x = om.canvas_input(ws, canvas, w.T, w.T)
+        for l, kw, vw, lw in om.prefill_layer_by_layer(ws, prompt):
+            x, _, _, _ = om.canvas_layer(x, lw, (kw, vw), P, w)
+            k = l + 1
+            if k not in depths:
+                continue
+            st = om.lm_head_stats(ws, x, want_logits=True)
+            kvl = np.stack([kw[-8:].transpose(1, 0, 2), vw[-8:].transpose(1, 0, 2)])
+            out.update({f"H{tag}_d{k}": st["H"], f"H64{tag}_d{k}": st["H64"],
+                        f"argmax{tag}_d{k}": st["argmax"], f"margin{tag}_d{k}": st["margin"],
+                        f"sigma{tag}_d{k}": st["sigma"],
+                        f"logits{tag}_d{k}": st["logits"][rows][:, cols].astype(np.float64),
+                        f"kv_last{tag}_d{k}": kvl})
+            print(f"{name} depth {k} ({storage}): H [{st['H'].min():.4f}, "
+                  f"{st['H'].max():.4f}] at {time.time() - t0:.0f} s", flush=True)
+            if k == max(depths):
+                break
+    path = os.path.join(HERE, f"{name}-depths.npz")
+    np.savez_compressed(path, **out)
+    print(f"{name}: wrote {path} in {time.time() - t0:.0f} s")
+
+
+def whole_block(name: str):
+    """The oracle's whole block on canvas 0 of the workload (steps as the sampler takes them)."""
+    w = workloads.get(name)
+    t0 = time.time()
+    ws = om.Weights(w, keep_layers=True)
+    prompt = model_inputs.prompt(w.with_(batch=1))[0].numpy()
+    P = prompt.shape[0]
+    kv = om.prefill(ws, prompt)
+    print(f"{name}: prefill done at {time.time() - t0:.0f} s", flush=True)
+    rec = []
+
+    def forward(canvas, s):
+        st = om.denoise_forward(ws, kv, canvas, s, w.T, P)
+        rec.append(dict(canvas=np.array(canvas, dtype=np.int64), s=s, H=st["H"],
+                        argmax=st["argmax"], margin=st["margin"], sigma=st["sigma"]))
+        print(f"{name}: forward s={s} at {time.time() - t0:.0f} s; H [{st['H'].min():.4f}, "
+              f"{st['H'].max():.4f}]", flush=True)
+        return st["H"], st["argmax"]
+
+    canvas, traj = osamp.generate_block(forward, w.canvas, w.mask_id, w.T, w.gamma)
+    n = len(traj)
+    out = dict(n_forwards=np.array(n), final_canvas=canvas,
+               s=np.array([r["s"] for r in rec]),
+               canvas_in=np.stack([r["canvas"] for r in rec]),
+               H=np.stack([r["H"] for r in rec]), argmax=np.stack([r["argmax"] for r in rec]),
+               margin=np.stack([r["margin"] for r in rec]),
+               sigma=np.stack([r["sigma"] for r in rec]),
+               n_committed=np.array([t[5] for t in traj]),
+               mask_after=np.stack([t[4] for t in traj]))
+    path = os.path.join(HERE, f"{name}-block.npz")
+    np.savez_compressed(path, **out)
+    print(f"{name}: wrote {path} in {time.time() - t0:.0f} s; {n} forwards, commits "
+          f"{[int(t[5]) for t in traj]}")
+
+
 if __name__ == "__main__":
     # arguments: workload names, optionally "name:canvas" to pick a canvas of the batch
     # and the suffix "+s16" for the bf16 storage variant as well ("+s16only": that alone)
     for arg in sys.argv[1:] or ["layer1-bf16"]:
+        if arg.endswith("@depths"):
+            depth_sweep(arg.removesuffix("@depths"))
+            continue
+        if arg.endswith("@block"):
+            whole_block(arg.removesuffix("@block"))
+            continue
         if arg.endswith("+s16only"):
             name, _, c = arg.removesuffix("+s16only").partition(":")
             add_storage_variant(name, int(c) if c else 0)

@@ -6,6 +6,7 @@ import os
 import re
 
 import pytest
+import torch
 
 from masked_discrete_diffusion_b200 import binding, build
 
@@ -105,3 +106,23 @@ def test_null_handles_and_bad_sizes_rejected_without_device(lib):
                 dict(d=4160), dict(w=vp(264)), dict(eps=-1.0), dict(s=float("inf")),
                 dict(s=float("nan"))):
         assert call(**bad) == 1, bad
+
+
+def test_noalloc_binding_rejects_bad_tensors_before_any_launch():
+    """The Python wrapper of the allocation-free entry point checks dtype, rank, the
+    shared width and the device before calling into the library (CPU tensors here:
+    no call can reach the GPU)."""
+    from masked_discrete_diffusion_b200 import binding
+    f32 = torch.zeros(4, 64, dtype=torch.float32)
+    b16 = torch.zeros(8, 64, dtype=torch.bfloat16)
+    bad = [
+        (f32.to(torch.bfloat16), b16, "hidden"),                         # hidden not fp32
+        (f32.reshape(-1), b16, "hidden"),                                # hidden not 2-D
+        (f32, b16.float(), "lm_head"),                                   # lm_head not bf16
+        (f32, b16.reshape(8, 8, 8), "lm_head"),                          # lm_head not 2-D
+        (f32, torch.zeros(8, 128, dtype=torch.bfloat16), "columns"),     # widths differ
+        (f32, b16, "CUDA"),                                              # not on a GPU
+    ]
+    for h, w, what in bad:
+        with pytest.raises(ValueError, match=what):
+            binding.dg_lmhead_entropy_noalloc(h, w, 1e-6, 8.0)

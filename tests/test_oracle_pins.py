@@ -379,6 +379,110 @@ def test_zero_blocks_reduce_to_embedding_head():
                                rtol=1e-11)
 
 
+# --------------------------------------------------------------- layer composition
+class _FixedWeights(model.Weights):
+    """Weights whose tensors are given (constructed by hand), not drawn from the seed."""
+
+    def __init__(self, w, tensors):
+        super().__init__(w, keep_layers=True)
+        self.t = tensors
+
+    def get(self, name, shape):
+        assert self.t[name].shape == tuple(shape), name
+        return self.t[name]
+
+    def rows(self, name, shape, start_row, n_rows):
+        return self.t[name][start_row:start_row + n_rows]
+
+
+def _composition_weights(swap_kv=False):
+    """d = 8, four query heads over two key/value heads (h = 2), one layer.
+
+    Query and router weights are zero, so every attention score is 0 (uniform
+    attention: the mean of V over the allowed keys) and the router ties; the key
+    rows are non-zero and differ from the value rows, so a q | k | v split that
+    read the key rows as values would change the output.  Values: head 0 = xn[0:2],
+    head 1 = xn[2:4]; Wo = I; routed experts zero; shared expert with gate = up =
+    down = I, so it adds silu(u) * u for u = RMSNorm(x) after attention."""
+    w = workloads.TINY_F32.with_(name="composition", n_layers=1, d_model=8, n_q_heads=4,
+                                 n_kv_heads=2, head_dim=2, n_experts=2, top_k=1,
+                                 expert_inter=4, shared_inter=8, vocab=16)
+    wq = np.zeros((8, 8))
+    wk = np.zeros((4, 8))
+    wk[:, 4:8] = 2.0 * np.eye(4)
+    wv = np.zeros((4, 8))
+    wv[:, 0:4] = np.eye(4)
+    if swap_kv:
+        wk, wv = wv, wk
+    t = {"l0.wqkv": np.concatenate([wq, wk, wv]), "l0.wo": np.eye(8),
+         "l0.router": np.zeros((2, 8)), "l0.gate": np.zeros((2, 4, 8)),
+         "l0.up": np.zeros((2, 4, 8)), "l0.down": np.zeros((2, 8, 4)),
+         "l0.sgate": np.eye(8), "l0.sup": np.eye(8), "l0.sdown": np.eye(8)}
+    return _FixedWeights(w, t)
+
+
+def _composition_expected(x, keys_xn, eps):
+    """Closed form of the constructed layer: pre-norm attention (mean of the value
+    heads over the keys, query heads 0, 1 -> kv head 0 and 2, 3 -> kv head 1), then
+    pre-norm shared expert silu(u) * u, each added to the residual."""
+    v0 = keys_xn[:, 0:2].mean(axis=0)
+    v1 = keys_xn[:, 2:4].mean(axis=0)
+    x1 = x + np.concatenate([v0, v0, v1, v1])[None, :]
+    u = x1 / np.sqrt((x1 * x1).mean(axis=1, keepdims=True) + eps)
+    return x1 + u * u / (1.0 + np.exp(-u))
+
+
+def _composition_rows():
+    # rows whose RMS is far from 1 (so a missing or misplaced norm shows)
+    return np.array([[3.0, -1.0, 0.5, 2.0, -4.0, 1.5, 0.25, -2.5],
+                     [0.1, 0.4, -0.3, 0.2, 0.05, -0.6, 0.7, -0.15],
+                     [-7.0, 2.0, 9.0, -1.0, 4.0, 3.0, -5.0, 6.0]])
+
+
+def test_decoder_layer_composition_closed_form():
+    """Pre-norm residual order, values from the normalised rows, the q | k | v row split
+    and the grouped-query head map, against a closed form (all rows see all rows)."""
+    ws = _composition_weights()
+    w = ws.w
+    x = _composition_rows()
+    xn = x / np.sqrt((x * x).mean(axis=1, keepdims=True) + w.rms_eps)
+    empty = np.zeros((0, 2, 2))
+    out, k, v, _ = model.decoder_layer(x, np.arange(3), ws.layer(0), (empty, empty),
+                                       np.ones((3, 3), dtype=bool), w)
+    np.testing.assert_allclose(out, _composition_expected(x, xn, w.rms_eps), rtol=1e-12,
+                               atol=1e-12)
+    np.testing.assert_allclose(v.reshape(3, 4), xn[:, 0:4], rtol=1e-12, atol=1e-12)
+    # variants a reading error would produce all differ from the constructed layer:
+    # values read from the key rows, a post-norm block, values from the raw rows
+    out_swap = model.decoder_layer(x, np.arange(3), _composition_weights(swap_kv=True).layer(0),
+                                   (empty, empty), np.ones((3, 3), dtype=bool), w)[0]
+    assert np.abs(out_swap - out).max() > 0.1
+    x1 = x + np.concatenate([xn[:, 0:2].mean(0)] * 2 + [xn[:, 2:4].mean(0)] * 2)
+    post = x1 / np.sqrt((x1 * x1).mean(1, keepdims=True) + w.rms_eps)
+    assert np.abs(_composition_expected(post, post, w.rms_eps) - out).max() > 0.1
+    assert np.abs(_composition_expected(x, x, w.rms_eps) - out).max() > 0.1
+
+
+def test_canvas_layer_one_softmax_over_window_and_canvas():
+    """Canvas rows attend to the cached window and every canvas row in ONE softmax: with
+    zero scores the value is the mean over all 2 + 3 keys (separate softmaxes over the
+    window and the canvas would average the two means instead)."""
+    ws = _composition_weights()
+    w = ws.w
+    x = _composition_rows()
+    xn = x / np.sqrt((x * x).mean(axis=1, keepdims=True) + w.rms_eps)
+    win_v = np.array([[[5.0, -3.0], [1.0, 8.0]], [[9.0, 1.0], [-6.0, 4.0]]])  # [W 2, Hkv 2, h 2]
+    win_k = np.ones_like(win_v)
+    out = model.canvas_layer(x, ws.layer(0), (win_k, win_v), 40, w)[0]
+    keys = np.concatenate([win_v.reshape(2, 4), xn[:, 0:4]])
+    np.testing.assert_allclose(out, _composition_expected(x, keys, w.rms_eps), rtol=1e-12,
+                               atol=1e-12)
+    two = 0.5 * (win_v.reshape(2, 4).mean(0) + xn[:, 0:4].mean(0))
+    x1 = x + np.concatenate([two[0:2], two[0:2], two[2:4], two[2:4]])
+    u = x1 / np.sqrt((x1 * x1).mean(1, keepdims=True) + w.rms_eps)
+    assert np.abs(x1 + u * u / (1 + np.exp(-u)) - out).max() > 0.1
+
+
 # --------------------------------------------------------------- metric formulas (pages' numbers)
 def test_tps_formula_reproduces_pages():
     from masked_discrete_diffusion_b200 import metrics
