@@ -297,9 +297,9 @@ def run_ours(args, w, world, rank, local):
     value = job_throughput(world, B * C, args.steps, ms_max)
     ms_step = ms_max / args.steps
 
-    # second timed pass of the same K steps with CUDA events recorded around every
-    # launch group inside the captured graph (per kernel-group device time)
-    binding.dg_profile_start(model)
+    # second pass of the same K steps with CUDA events recorded around every launch group
+    # (an unrolled graph of exactly the forwards the timed loop ran, on the same canvases)
+    binding.dg_profile_start(model, fwd_per_block)
     for _ in range(args.steps):
         binding.dg_generate_block(model, kv, T, w.gamma, canvas, nfwd, load)
     torch.cuda.synchronize()
@@ -331,8 +331,17 @@ def run_ours(args, w, world, rank, local):
     peak = float(peaks["hbm_gbs"])
     fwd_ms = ms_step / max(fwd_per_block, 1)
     t_roof = max(cost["bytes"] / (peak * 1e9), cost["flops"] / (float(peaks["bf16_tflops"]) * 1e12))
-    kinds = {k: {"ms_per_step": v[0] / args.steps, "groups_per_step": v[1] / args.steps}
+    kinds = {k: {"ms_per_forward": v[0] / args.steps / max(fwd_per_block, 1),
+                 "groups_per_forward": v[1] / args.steps / max(fwd_per_block, 1)}
              for k, v in prof.items()}
+    main_ms = sum(v["ms_per_forward"] for k, v in kinds.items() if k != "shared")
+    # router load of the last timed block: rows each expert received, summed over the
+    # block's forwards and layers; and how many experts received rows per layer
+    load_np = load.cpu().numpy()
+    router_load = {"per_expert_rows": [int(v) for v in load_np.sum(axis=0)],
+                   "experts_with_rows_per_layer": float((load_np > 0).sum(axis=1).mean()),
+                   "rows_per_layer_per_forward": B * C * w.top_k,
+                   "forwards": fwd_per_block}
 
     line = {
         "metric": "canvas tokens/sec at 1 B200 (256-tok block)", "value": value,
@@ -356,7 +365,11 @@ def run_ours(args, w, world, rank, local):
                      "alg_bytes_per_launch": ex_bytes, "avg_launch_ms": ex_avg_s * 1e3,
                      "peak_src": f"{peak_src} hbm_gbs"},
         "kernel_groups": kinds,
-        "kernel_groups_note": "second pass of the same steps with event records around each launch group",
+        "kernel_groups_main_stream_ms_per_forward": main_ms,
+        "kernel_groups_note": ("second pass of the same steps and forwards with event records "
+                               "around each launch group; 'shared' runs on a concurrent branch, "
+                               "the other groups sum to at most ms_per_forward"),
+        "router_load": router_load,
         "gpu_launches": launches,
         "clocks": clk,
         "e2e": None if e2e_val is None else {

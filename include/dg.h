@@ -195,16 +195,23 @@ dg_status dg_kv_read(const dg_kv* kv, void* k, void* v, void* stream);
 /* ---- measurement hooks (no counterpart on the pages) -------------------------
  * Kernel groups whose device time can be recorded while the path runs. */
 typedef enum dg_kernel_kind {
-  DG_KIND_EXPERTS = 0,   /* routed-expert FFN: gate/up (SwiGLU) and down launches */
-  DG_KIND_LMHEAD = 1,    /* LM-head GEMM + online entropy statistics (+ merge)   */
-  DG_KIND_ATTENTION = 2, /* canvas / prompt attention                           */
-  DG_KIND_DENSE = 3,     /* QKV, O and shared-expert projections                */
-  DG_KIND_COUNT = 4
+  DG_KIND_EXPERTS = 0,   /* routed-expert FFN: gate/up (SwiGLU) and down launches   */
+  DG_KIND_LMHEAD = 1,    /* LM-head GEMM + online entropy statistics (+ merge)     */
+  DG_KIND_ATTENTION = 2, /* canvas / prompt attention                             */
+  DG_KIND_DENSE = 3,     /* QKV and O projections (main stream)                   */
+  DG_KIND_SHARED = 4,    /* shared-expert projections (a concurrent graph branch) */
+  DG_KIND_ROUTING = 5,   /* RMSNorm, router, top-k and permutation launches       */
+  DG_KIND_GLUE = 6,      /* embedding, combine + RMSNorm, sampler                 */
+  DG_KIND_COUNT = 7
 } dg_kernel_kind;
 
 /* Starts recording a pair of CUDA events around every launch group of each
- * kind, on the stream the launches use.  Costs one event record per launch. */
-dg_status dg_profile_start(dg_model* m);
+ * kind, on the stream the launches use.  Costs one event record per launch.
+ * While recording, dg_generate_block runs an unrolled block of at most
+ * max_forwards forwards (0: T) instead of its device-controlled loop; given the
+ * number of forwards the loop ran (n_forwards), it replays the same forwards on the
+ * same canvases. */
+dg_status dg_profile_start(dg_model* m, int32_t max_forwards);
 
 /* Synchronises the device, writes the summed device milliseconds
  * (ms[DG_KIND_COUNT]) and the number of recorded launch groups

@@ -26,6 +26,17 @@ dg_status dg_op_gemm(dg_model* m, const void* A, const void* W, float* out, int3
 dg_status dg_op_moe(dg_model* m, int32_t layer, const float* x, float* out, int32_t n,
                     void* stream);
 
+/* Test hook for the device-side timeout path (no counterpart on the pages): the next
+ * routed-expert launch of this bf16 model makes its down units wait for one more
+ * gate/up unit than their token chunk has, and limits every wait of that launch to
+ * limit_ns nanoseconds (1e5 .. 1e9).  Each such wait runs out: the launch records
+ * DG_ERR_TIMEOUT in the model's device error word and unwinds (every role of the kernel
+ * keeps its waits bounded, so it ends within a few multiples of limit_ns), the next
+ * dg_sync_status returns DG_ERR_TIMEOUT, and later launches run normally.  Applies to
+ * one launch.  DG_ERR_UNSUPPORTED for models whose experts do not use that kernel
+ * (fp32, FP8 experts). */
+dg_status dg_debug_stall_experts(dg_model* m, int64_t limit_ns);
+
 #ifdef __cplusplus
 }
 #endif

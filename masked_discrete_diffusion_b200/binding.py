@@ -78,7 +78,7 @@ def lib() -> ctypes.CDLL:
             "dg_generate_block": [vp, vp, i32, f32, vp, vp, vp, vp],
             "dg_eb_sample": [vp, vp, vp, vp, i32, i32, i32, f32, vp, vp],
             "dg_debug_forward": [vp, vp, vp, i32, i32, vp, vp, vp, vp, vp],
-            "dg_profile_start": [vp],
+            "dg_profile_start": [vp, i32],
             "dg_profile_stop": [vp, vp, vp],
             "dg_launch_count": [vp, ctypes.POINTER(ctypes.c_int64)],
             "dg_expert_units": [vp, ctypes.POINTER(ctypes.c_int64)],
@@ -86,6 +86,7 @@ def lib() -> ctypes.CDLL:
             "dg_lmhead_entropy_noalloc": [vp, vp, i32, i32, i32, f32, f32, vp, vp, vp],
             "dg_op_gemm": [vp, vp, vp, vp, i32, i32, i32, vp],
             "dg_op_moe": [vp, i32, vp, vp, i32, vp],
+            "dg_debug_stall_experts": [vp, ctypes.c_int64],
         }
         for name, args in sigs.items():
             fn = getattr(L, name)
@@ -101,7 +102,8 @@ def exported_symbols():
                         "dg_kv_read", "dg_denoise_step", "dg_generate_block", "dg_eb_sample",
                         "dg_debug_forward", "dg_profile_start", "dg_profile_stop",
                         "dg_launch_count", "dg_op_gemm", "dg_op_moe", "dg_expert_units",
-                        "dg_lmhead_entropy_noalloc", "dg_block_loop_launches")
+                        "dg_lmhead_entropy_noalloc", "dg_block_loop_launches",
+                        "dg_debug_stall_experts")
             if hasattr(lib(), n)]
 
 
@@ -261,11 +263,13 @@ def dg_debug_forward(model: Model, kv: KV, canvas, steps_left: int, T: int, logi
     return ent, am, lg, hd
 
 
-KINDS = ("experts", "lmhead", "attention", "dense")
+KINDS = ("experts", "lmhead", "attention", "dense", "shared", "routing", "glue")
 
 
-def dg_profile_start(model: Model):
-    _check(lib().dg_profile_start(model.handle))
+def dg_profile_start(model: Model, max_forwards: int = 0):
+    """Event records around every launch group from now on; a profiled block runs at
+    most max_forwards forwards (0: T), unrolled."""
+    _check(lib().dg_profile_start(model.handle, max_forwards))
 
 
 def dg_profile_stop(model: Model) -> dict:
@@ -339,3 +343,8 @@ def dg_block_loop_launches(model: Model) -> int:
     out = ctypes.c_int64()
     _check(lib().dg_block_loop_launches(model.handle, ctypes.byref(out)))
     return out.value
+
+
+def dg_debug_stall_experts(model: Model, limit_ns: int):
+    """Test hook: the next routed-expert launch runs its waits out after limit_ns."""
+    _check(lib().dg_debug_stall_experts(model.handle, limit_ns))

@@ -244,7 +244,10 @@ template <class Path> struct Runner {
     const dg_layer_weights& L = m->layers[l];
     const int d = c.d_model, h = c.head_dim, Hq = c.n_q_heads, Hkv = c.n_kv_heads;
     const int qkv_n = (Hq + 2 * Hkv) * h;
-    if (l == 0) rmsnorm(n);
+    if (l == 0) {
+      ProfScope ps(m, DG_KIND_GLUE, st);
+      rmsnorm(n);
+    }
     bool fused_rope = false;
     {
       ProfScope ps(m, DG_KIND_DENSE, st);
@@ -321,22 +324,25 @@ template <class Path> struct Runner {
     PermuteArgs pa{(const int32_t*)ws.ridx, n_ent, k, E, bm, ws.rank, ws.offsets, ws.tile_e,
                    ws.tile_m0, ws.n_tiles, ws.max_tiles, ws.units, load, ws.row_of, ws.tok_of,
                    ws.ready};
-    launch_pdl((rmsnorm_kernel<TR, TA, Acc>), n, 256, 0, st, 1, x(), xn(), n, d, c.rms_eps,
-               (Acc*)ws.inv_rms, tc_router ? (TA*)ws.u2 : (TA*)nullptr);
-    ++m->launches;
+    {
+      ProfScope ps(m, DG_KIND_ROUTING, st);
+      launch_pdl((rmsnorm_kernel<TR, TA, Acc>), n, 256, 0, st, 1, x(), xn(), n, d, c.rms_eps,
+                 (Acc*)ws.inv_rms, tc_router ? (TA*)ws.u2 : (TA*)nullptr);
+      ++m->launches;
+    }
     if constexpr (Path::kTensorCores) {
       // shared expert on the side stream, concurrent with routing and the routed experts
       cudaStream_t side = m->side_stream;
       DG_TRY_CUDA(cudaEventRecord(m->fork_ev, st));
       DG_TRY_CUDA(cudaStreamWaitEvent(side, m->fork_ev, 0));
       {
-        ProfScope ps(m, DG_KIND_DENSE, side);
+        ProfScope ps(m, DG_KIND_SHARED, side);
         DG_TRY(tc_gemm_swiglu(m, xn(), L.sgate, L.sup, (TA*)ws.sh, n, Is, d, side));
         DG_TRY(tc_gemm_store_f32(m, (const TA*)ws.sh, L.sdown, (float*)ws.ys, n, d, Is, side));
       }
       DG_TRY_CUDA(cudaEventRecord(m->join_ev, side));
       if (tc_router) {
-        ProfScope ps(m, DG_KIND_DENSE, st);
+        ProfScope ps(m, DG_KIND_ROUTING, st);
         DG_TRY(tc_router_topk(m, (const bf16*)ws.u2, L.router, n, ws.ridx, (float*)ws.rgate, st));
       }
     }
@@ -362,6 +368,7 @@ template <class Path> struct Runner {
             (int32_t*)nullptr);
       ++m->launches;
     }
+    ProfScope pperm(m, DG_KIND_ROUTING, st);
     if (permute_smem_bytes(E, 1024, n_ent) <= PERMUTE_FUSED_SMEM) {
       // every block derives the permutation in shared memory and gathers its rows
       const int blocks = std::max(1, std::min(n_ent, m->n_sm_cache));
@@ -377,6 +384,7 @@ template <class Path> struct Runner {
                  ws.offsets + E, d, (TA*)ws.up);
       ++m->launches;
     }
+    pperm.end();
     const int grid_y = ceil_div(n_ent, bm) + E;
     if constexpr (Path::kTensorCores) {
       {
@@ -410,6 +418,7 @@ template <class Path> struct Runner {
       dense((const TA*)ws.sh, Is, L.sdown, d, Is, n, EpiStore<Acc, Acc>{(Acc*)ws.ys, d});
     }
     // residual update fused with the next RMSNorm (next layer's input or the LM head's)
+    ProfScope pg(m, DG_KIND_GLUE, st);
     launch_pdl((moe_combine_norm_kernel<TR, TA, Acc, Acc>), n, 256, 0, st, 1, x(),
                (const Acc*)ws.ys, (const Acc*)ws.yb, (const int32_t*)ws.row_of, n, d, k,
                c.rms_eps, xn());
@@ -468,9 +477,12 @@ template <class Path> struct Runner {
                     int32_t* amax, float* logits, float* hidden, int32_t* load) {
     const int B = kv->B, C = c.canvas, n = B * C, d = c.d_model;
     const double tau = (double)s / (double)T;
-    launch_pdl((embed_kernel<TW, TR>), n, 256, 0, st, 1, canvas, (const TW*)m->w.tok_emb, x(), n, d, c.vocab,
-                                           tau, ws.err, (const int32_t*)s_dev, T);
-    ++m->launches;
+    {
+      ProfScope ps(m, DG_KIND_GLUE, st);
+      launch_pdl((embed_kernel<TW, TR>), n, 256, 0, st, 1, canvas, (const TW*)m->w.tok_emb, x(), n,
+                 d, c.vocab, tau, ws.err, (const int32_t*)s_dev, T);
+      ++m->launches;
+    }
     const int Cp = (C + 63) / 64 * 64;
     if (Cp != C)
       DG_TRY_CUDA(cudaMemsetAsync(ws.vc, 0, (size_t)B * c.n_kv_heads * c.head_dim * Cp * sizeof(TKV), st));
@@ -797,7 +809,7 @@ dg_status dg_denoise_step(dg_model* m, const dg_kv* kv, int32_t* canvas, uint8_t
 // The launch sequence of one block (T forwards + sampler steps), enqueued on st.
 static dg_status generate_impl(dg_model* m, const dg_kv* kv, int32_t T, long long gq,
                                int32_t* canvas_out, int32_t* n_forwards, int32_t* router_load,
-                               cudaStream_t st) {
+                               cudaStream_t st, int fcap = 0) {
   const dg_config& c = m->cfg;
   const int B = kv->B, C = c.canvas;
   Workspace& ws = m->ws;
@@ -808,10 +820,12 @@ static dg_status generate_impl(dg_model* m, const dg_kv* kv, int32_t T, long lon
   if (router_load)
     DG_TRY_CUDA(cudaMemsetAsync(router_load, 0,
                                 (size_t)c.n_layers * c.n_experts * sizeof(int32_t), st));
-  for (int k = 0; k < T; ++k) {
+  const int nfw = fcap > 0 ? std::min(fcap, (int)T) : (int)T;
+  for (int k = 0; k < nfw; ++k) {
     const int s = T - k;
     DG_TRY(run_forward(m, kv, canvas_out, s, T, ws.ent, ws.amax, nullptr, nullptr, router_load,
                        st));
+    ProfScope ps(m, DG_KIND_GLUE, st);
     DG_TRY(launch_sampler(ws.ent, ws.amax, canvas_out, ws.mask, B, C, s, gq, ws.ncommit,
                           n_forwards, k + 1, st, &m->launches));
   }
@@ -900,7 +914,8 @@ static dg_status generate_graphed(dg_model* m, const dg_kv* kv, int32_t T, long 
   dg::BlockGraph* g = nullptr;
   for (auto* x : m->graphs)
     if (x->kv == kv && x->T == T && x->gq == gq && x->canvas == canvas_out &&
-        x->nfwd == n_forwards && x->load == router_load && x->prof == m->profiling) {
+        x->nfwd == n_forwards && x->load == router_load && x->prof == m->profiling &&
+        (!x->prof || x->fcap == m->prof_forwards)) {
       g = x;
       break;
     }
@@ -917,6 +932,7 @@ static dg_status generate_graphed(dg_model* m, const dg_kv* kv, int32_t T, long 
     g->nfwd = n_forwards;
     g->load = router_load;
     g->prof = m->profiling;
+    g->fcap = m->profiling ? m->prof_forwards : 0;
     // capture on a library-owned stream (the caller's may be the legacy default
     // stream, which cannot be captured); nothing executes during capture
     if (!m->cap_stream) DG_TRY_CUDA(cudaStreamCreateWithFlags(&m->cap_stream, cudaStreamNonBlocking));
@@ -930,7 +946,8 @@ static dg_status generate_graphed(dg_model* m, const dg_kv* kv, int32_t T, long 
     cudaError_t e = cudaStreamBeginCapture(m->cap_stream, cudaStreamCaptureModeThreadLocal);
     dg_status s = DG_OK;
     if (e == cudaSuccess) {
-      s = generate_impl(m, kv, T, gq, canvas_out, n_forwards, router_load, m->cap_stream);
+      s = generate_impl(m, kv, T, gq, canvas_out, n_forwards, router_load, m->cap_stream,
+                        g->fcap);
       e = cudaStreamEndCapture(m->cap_stream, &graph);
     }
     m->capture = nullptr;
@@ -1024,8 +1041,22 @@ dg_status dg_op_moe(dg_model* m, int32_t layer, const float* x, float* out, int3
                                 : Runner<PathBF16>(m, st).moe_op(layer, x, out, n);
 }
 
-dg_status dg_profile_start(dg_model* m) {
+dg_status dg_debug_stall_experts(dg_model* m, int64_t limit_ns) {
+  g_err.clear();
   DG_REQUIRE(m, "null model");
+  DG_REQUIRE(limit_ns >= 100000 && limit_ns <= 1000000000, "limit_ns outside [1e5, 1e9]");
+  if (m->cfg.dtype != DG_BF16) {
+    set_error("only the bf16 routed-expert kernel has this test path");
+    return DG_ERR_UNSUPPORTED;
+  }
+  m->stall_limit_ns = limit_ns;
+  return DG_OK;
+}
+
+dg_status dg_profile_start(dg_model* m, int32_t max_forwards) {
+  DG_REQUIRE(m, "null model");
+  DG_REQUIRE(max_forwards >= 0, "max_forwards must be >= 0");
+  m->prof_forwards = max_forwards;
   for (int k = 0; k < DG_KIND_COUNT; ++k) {
     m->prof_used[k] = 0;
     m->prof_acc_ms[k] = 0.0;

@@ -126,6 +126,7 @@ struct BlockGraph {
   long long gq = 0;
   int32_t *canvas = nullptr, *nfwd = nullptr, *load = nullptr;
   bool prof = false;
+  int fcap = 0;            // forwards of a profiled (unrolled) block, 0: T
   long long launches = 0;  // kernel launches the graph replays (1 for a loop graph: the init)
   bool loop = false;       // device-controlled WHILE loop over forwards
   long long body_launches = 0;  // kernels per loop iteration (forward + sampler + control)
@@ -143,9 +144,10 @@ struct dg_model {
   // event recording around launch groups, per dg_kernel_kind
   bool profiling = false;
   std::vector<std::pair<cudaEvent_t, cudaEvent_t>> prof[DG_KIND_COUNT];
-  size_t prof_used[DG_KIND_COUNT] = {0, 0, 0, 0};
-  double prof_acc_ms[DG_KIND_COUNT] = {0, 0, 0, 0};  // from graph replays
-  int64_t prof_acc_n[DG_KIND_COUNT] = {0, 0, 0, 0};
+  size_t prof_used[DG_KIND_COUNT] = {};
+  double prof_acc_ms[DG_KIND_COUNT] = {};  // from graph replays
+  int64_t prof_acc_n[DG_KIND_COUNT] = {};
+  int prof_forwards = 0;  // forwards of a profiled block (0: T)
   // captured blocks
   bool use_graphs = true;
   std::vector<dg::BlockGraph*> graphs;
@@ -158,6 +160,9 @@ struct dg_model {
   cudaEvent_t fork_ev = nullptr, join_ev = nullptr;
   long long last_body_launches = 0;   // kernels per forward of the last replayed loop graph
   std::vector<dg_kv*> kvs;            // live KV caches created from this model
+  // > 0: the next routed-expert launch stalls its down units on purpose, with every
+  // wait limited to this many ns (dg_debug_stall_experts; tests of the timeout path)
+  long long stall_limit_ns = 0;
 };
 
 namespace dg {

@@ -804,7 +804,11 @@ __global__ void __launch_bounds__(TC_MOE_THREADS, 1)
                   const int32_t* __restrict__ chunk_r0, const int32_t* __restrict__ n_chunks,
                   const int32_t* __restrict__ offsets, int I, int d, bf16* __restrict__ hb,
                   float* __restrict__ yb, const float* __restrict__ gate_of,
-                  int32_t* __restrict__ ready, int32_t* __restrict__ next, int32_t* err) {
+                  int32_t* __restrict__ ready, int32_t* __restrict__ next, int32_t* err,
+                  uint64_t limit_ns, int stall) {
+  // limit_ns: how long any wait of this launch may last before it gives up (records
+  // ERR_TIMEOUT and unwinds); stall != 0 (tests of that path only): a down unit waits for
+  // one more gate/up unit than its chunk has, so every such wait runs out
   typedef MoeCfg<ST> Cfg;
   pdl_enter();  // the routing tables come from the preceding kernels
   extern __shared__ uint8_t smem_raw[];
@@ -862,7 +866,7 @@ __global__ void __launch_bounds__(TC_MOE_THREADS, 1)
   // the ui-th unit id of this block (n_units when there is none, or on a timeout)
   auto take = [&](int ui) -> int {
     const int k = ui % QD;
-    if (!tc::mbar_wait(qfull + k, (ui / QD) & 1)) {
+    if (!tc::mbar_wait(qfull + k, (ui / QD) & 1, limit_ns)) {
       atomicOr(err, ERR_TIMEOUT);
       return n_units;
     }
@@ -885,7 +889,7 @@ __global__ void __launch_bounds__(TC_MOE_THREADS, 1)
         // blocks take the next unit when they are ready for it (gate/up units first,
         // so a down unit only ever waits for units that running blocks have taken)
         const int k = qi % QD;
-        if (qi >= QD && !tc::mbar_wait(qempty + k, ((qi / QD) & 1) ^ 1)) {
+        if (qi >= QD && !tc::mbar_wait(qempty + k, ((qi / QD) & 1) ^ 1, limit_ns)) {
           atomicOr(err, ERR_TIMEOUT);
           break;  // the readers give up on their own bounded waits
         }
@@ -898,9 +902,10 @@ __global__ void __launch_bounds__(TC_MOE_THREADS, 1)
         if (x.down) {
           // the chunk's hidden rows are complete once all its phase-1 units have counted
           const uint64_t t0 = tc::global_ns();
-          while (ld_acquire(ready + x.c) < FT1) {
+          const int need = FT1 + (stall ? 1 : 0);
+          while (ld_acquire(ready + x.c) < need) {
             __nanosleep(64);
-            if (tc::global_ns() - t0 > 2000000000ull) {
+            if (tc::global_ns() - t0 > limit_ns) {
               atomicOr(err, ERR_TIMEOUT);
               ok = false;
               break;
@@ -916,7 +921,7 @@ __global__ void __launch_bounds__(TC_MOE_THREADS, 1)
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int s = it % ST;
           const uint32_t ph = (it / ST) & 1;
-          if (it >= ST && !tc::mbar_wait(empty + s, ph ^ 1)) {
+          if (it >= ST && !tc::mbar_wait(empty + s, ph ^ 1, limit_ns)) {
             atomicOr(err, ERR_TIMEOUT);
             ok = false;
             break;
@@ -938,7 +943,7 @@ __global__ void __launch_bounds__(TC_MOE_THREADS, 1)
                             x.r0 + 32 * j);
         }
       }
-      if (!tc::drain_slots(full, ST, it)) atomicOr(err, ERR_TIMEOUT);
+      if (!tc::drain_slots(full, ST, it, limit_ns)) atomicOr(err, ERR_TIMEOUT);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -952,7 +957,7 @@ __global__ void __launch_bounds__(TC_MOE_THREADS, 1)
         const int npad = ((x.n + 31) >> 5) << 5;
         const uint32_t idesc = tc::idesc_bf16(128, npad);
         // wait until the epilogue has drained the previous unit's accumulators
-        if (ui > 0 && !tc::mbar_wait(tempty, (ui - 1) & 1)) {
+        if (ui > 0 && !tc::mbar_wait(tempty, (ui - 1) & 1, limit_ns)) {
           atomicOr(err, ERR_TIMEOUT);
           break;
         }
@@ -960,7 +965,7 @@ __global__ void __launch_bounds__(TC_MOE_THREADS, 1)
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int s = it % ST;
           const uint32_t ph = (it / ST) & 1;
-          if (!tc::mbar_wait(full + s, ph)) {
+          if (!tc::mbar_wait(full + s, ph, limit_ns)) {
             atomicOr(err, ERR_TIMEOUT);
             ok = false;
             break;
@@ -993,7 +998,7 @@ __global__ void __launch_bounds__(TC_MOE_THREADS, 1)
       if (u >= n_units) break;
       const Unit x = unit_of(u);
       bool rdy = true;
-      if (lane == 0) rdy = tc::mbar_wait(tfull, ui & 1);
+      if (lane == 0) rdy = tc::mbar_wait(tfull, ui & 1, limit_ns);
       rdy = __shfl_sync(0xffffffffu, rdy ? 1 : 0, 0) != 0;
       // on a timeout the warp records it and keeps step with the other epilogue warps
       // (same barriers, no TMEM reads), so that nothing waits forever

@@ -330,7 +330,10 @@ dg_status tc_moe_experts(dg_model* m, int l, const bf16* X, bf16* hb, float* yb,
                              MoeCfg<MOE_ST>::SMEM, st, 1, wg, wu, x, wd, h, ws.tile_e,
                              ws.tile_m0, ws.n_tiles, ws.offsets, I, d, hb, yb,
                              (const float*)ws.gate_of, ws.ready, ws.ready + ws.max_tiles,
-                             ws.err);
+                             ws.err, (uint64_t)(m->stall_limit_ns > 0 ? m->stall_limit_ns
+                                                                      : 2000000000ll),
+                             m->stall_limit_ns > 0 ? 1 : 0);
+  m->stall_limit_ns = 0;  // one launch only
   ++m->launches;
   if (e != cudaSuccess) {
     set_error("tc_moe launch: %s", cudaGetErrorString(e));

@@ -71,11 +71,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
 // so that no TMA write reaches this CTA's shared memory after it has moved on.  Stage
 // loads are numbered 0 .. issued - 1 and load i completes on barrier i % slots in phase
 // (i / slots) & 1.  A slot whose last copy has already landed returns at once.
-__device__ __forceinline__ bool drain_slots(uint64_t* full, int slots, int issued) {
+__device__ __forceinline__ bool drain_slots(uint64_t* full, int slots, int issued,
+                                            uint64_t limit_ns = 2000000000ull) {
   bool ok = true;
   for (int s = 0; s < slots && s < issued; ++s) {
     const int last = issued - 1 - (issued - 1 - s) % slots;
-    ok = mbar_wait(full + s, (uint32_t)(last / slots) & 1) && ok;
+    ok = mbar_wait(full + s, (uint32_t)(last / slots) & 1, limit_ns) && ok;
   }
   return ok;
 }

@@ -97,8 +97,20 @@ SMALL_BF16 = Workload(
 SMALL_FP8 = SMALL_BF16.with_(name="small-fp8exp", dtype="bf16_fp8exp")
 LAYER1_FP8 = LAYER1_BF16.with_(name="layer1-fp8exp-p4096", dtype="bf16_fp8exp", prompt_len=4096)
 
+# Ragged shapes of the full-size kernels: a prompt shorter than the window and not a
+# multiple of the 64-key tile (200), two canvases, and a canvas that is not a multiple
+# of the 128-row query tile (96).
+LAYER1_P200_B2 = LAYER1_BF16.with_(name="layer1-bf16-p200-b2", prompt_len=200, batch=2)
+LAYER1_P200_B2_C96 = LAYER1_P200_B2.with_(name="layer1-bf16-p200-b2-c96", canvas=96)
+
+# One FP8-expert layer at the batches where each expert holds several 128-row token
+# chunks (the tensor-bound part of the FP8 sweep).
+LAYER1_FP8_B16 = LAYER1_FP8.with_(name="layer1-fp8exp-p4096-b16", batch=16)
+LAYER1_FP8_B64 = LAYER1_FP8.with_(name="layer1-fp8exp-p4096-b64", batch=64)
+
 WORKLOADS = {w.name: w for w in (TINY_F32, SMALL_BF16, LAYER1_BF16, FULL30_BF16,
-                                 FULL30_B8_P8192, SMALL_FP8, LAYER1_FP8)}
+                                 FULL30_B8_P8192, SMALL_FP8, LAYER1_FP8, LAYER1_P200_B2,
+                                 LAYER1_P200_B2_C96, LAYER1_FP8_B16, LAYER1_FP8_B64)}
 for _b in (1, 4, 16, 32, 64):
     WORKLOADS[f"full30-fp8exp-b{_b}"] = full30_fp8exp(_b)
 

@@ -15,7 +15,9 @@ With the suffix "+s16" the file also holds the same outputs of the oracle's bf16
 storage variant (H_s16, argmax_s16, logits_s16, kv_last_s16): the sensitivity of the
 workload to bf16 activation storage, from which the deep workloads' tolerances follow.
 The suffix "+s16only" adds those fields to an existing file (the fp64 run is not
-repeated).
+repeated).  Files also hold router_margin_rows [C]: per row, the smallest gap over the
+layers between the top_k-th and (top_k+1)-th router logit ("+rmonly" adds it to an
+existing file).
 
 Two further modes on a deep workload:
   <name>@depths  -> <name>-depths.npz: the first forward of the models made of the
@@ -71,6 +73,34 @@ def add_storage_variant(name: str, canvas_index: int = 0):
     print(f"{name}{suffix}: added the bf16-storage run in {time.time() - t0:.0f} s")
 
 
+def _router_margin_rows(w, routes):
+    """Per canvas row, the smallest gap over the layers between the top_k-th and the
+    (top_k+1)-th router logit: a row whose gap is small may be routed differently by
+    any path that perturbs the router's input (bf16 storage included)."""
+    gaps = []
+    for _, _, rl in routes:
+        srt = np.sort(rl, axis=1)[:, ::-1]
+        gaps.append(srt[:, w.top_k - 1] - srt[:, w.top_k])
+    return np.min(np.stack(gaps), axis=0)
+
+
+def add_router_margins(name: str, canvas_index: int = 0):
+    """Adds router_margin_rows to an existing golden file (reruns the fp64 forward)."""
+    w = workloads.get(name)
+    t0 = time.time()
+    suffix = f"-c{canvas_index}" if canvas_index else ""
+    path = os.path.join(HERE, f"{name}{suffix}.npz")
+    old = dict(np.load(path))
+    prompt = model_inputs.prompt(w.with_(batch=1), first=canvas_index)[0].numpy()
+    canvas = np.full(w.canvas, w.mask_id)
+    st = om.prefill_then_forward(om.Weights(w, keep_layers=False), prompt, canvas, w.T, w.T)
+    assert np.array_equal(st["H"], old["H"]), "the oracle no longer reproduces this file"
+    old["router_margin_rows"] = _router_margin_rows(w, st["routes"])
+    np.savez_compressed(path, **old)
+    print(f"{name}{suffix}: added per-row router margins in {time.time() - t0:.0f} s; "
+          f"rows with margin < 1e-2: {(old['router_margin_rows'] < 1e-2).sum()}", flush=True)
+
+
 def make(name: str, canvas_index: int = 0, storage_variant: bool = False):
     """Oracle outputs of the first forward of canvas `canvas_index` of the workload."""
     w = workloads.get(name)
@@ -100,7 +130,9 @@ def make(name: str, canvas_index: int = 0, storage_variant: bool = False):
                         lse=st["lse"], sigma=st["sigma"], logit_rows=np.array(rows),
                         logit_cols=cols,
                         logits=st["logits"][rows][:, cols].astype(np.float64), kv_last=kv_last,
-                        router_margin=np.array(rmarg), step_canvas=c2, step_mask=m2,
+                        router_margin=np.array(rmarg),
+                        router_margin_rows=_router_margin_rows(w, st["routes"]),
+                        step_canvas=c2, step_mask=m2,
                         step_n=np.array(n2), step=np.array(w.T), **extra)
     print(f"{name}: wrote {out} in {time.time() - t0:.0f} s; H range "
           f"[{st['H'].min():.4f}, {st['H'].max():.4f}], min margin {st['margin'].min():.4g}, "
@@ -189,6 +221,10 @@ if __name__ == "__main__":
             continue
         if arg.endswith("@block"):
             whole_block(arg.removesuffix("@block"))
+            continue
+        if arg.endswith("+rmonly"):
+            name, _, c = arg.removesuffix("+rmonly").partition(":")
+            add_router_margins(name, int(c) if c else 0)
             continue
         if arg.endswith("+s16only"):
             name, _, c = arg.removesuffix("+s16only").partition(":")

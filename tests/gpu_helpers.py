@@ -20,11 +20,13 @@ def max_abs_rel(a, b):
 
 
 def storage_tol(g, key, stated, index=None):
-    """Tolerance for a deep workload's output `key`: the stated one, or twice the
-    distance between the oracle's bf16-storage run (key + "_s16") and its fp64 run,
-    whichever is larger.  A bf16 path's own rounding is a perturbation of the same
-    size as that run's, and both are amplified alike through the layers."""
+    """Tolerance for a deep workload's output `key`: the stated one where the oracle's
+    bf16-storage run (key + "_s16") stays within 1e-2 of its fp64 run (bf16 storage is
+    not amplified there), else 1.5x that distance (never below the stated one).  A bf16
+    path stores bf16 where that run does, so its error is a perturbation of the same
+    size, amplified alike through the layers."""
     a, b = g[key + "_s16"], g[key]
     if index is not None:
         a, b = a[index], b[index]
-    return max(stated, 2.0 * max_abs_rel(a, b))
+    dist = max_abs_rel(a, b)
+    return stated if dist < 1e-2 else max(stated, 1.5 * dist)

@@ -82,13 +82,14 @@ def test_null_handles_and_bad_sizes_rejected_without_device(lib):
         "dg_denoise_step": (None, None, fake, fake, 1, 4, 1.0, fake, fake, fake, None),
         "dg_generate_block": (None, None, 4, 1.0, fake, None, None, None),
         "dg_debug_forward": (None, None, fake, 1, 4, fake, fake, None, None, None),
-        "dg_profile_start": (None,),
+        "dg_profile_start": (None, 0),
         "dg_profile_stop": (None, None, None),
         "dg_launch_count": (None, ctypes.byref(n)),
         "dg_expert_units": (None, ctypes.byref(n)),
         "dg_block_loop_launches": (None, ctypes.byref(n)),
         "dg_op_gemm": (None, fake, fake, fake, 1, 64, 64, None),
         "dg_op_moe": (None, 0, fake, fake, 1, None),
+        "dg_debug_stall_experts": (None, 1000000),
     }
     for name, args in calls.items():
         assert getattr(lib, name)(*args) == 1, name

@@ -12,7 +12,9 @@ import pytest
 from gpu_helpers import max_abs_rel, storage_tol
 
 HERE = os.path.join(os.path.dirname(__file__), "golden")
-FILES = sorted(glob.glob(os.path.join(HERE, "*.npz")))
+# first-forward files (the depth sweep and the whole block have their own layouts)
+FILES = sorted(f for f in glob.glob(os.path.join(HERE, "*.npz"))
+               if not f.endswith(("-depths.npz", "-block.npz")))
 STATED = 2e-2
 
 
@@ -67,3 +69,46 @@ def test_thirty_layers_amplify_storage_noise():
     assert storage_tol(deep, "H", STATED) > STATED
     assert storage_tol(deep, "logits", STATED) > STATED
     assert storage_tol(deep, "kv_last", STATED, (0, 0)) == STATED
+
+
+def test_depth_sweep_file_matches_the_single_depth_files():
+    """Depth 1 of the sweep is the one-layer workload and depth 30 the 30-layer one
+    (weights seeded per layer name; the sweep runs the same oracle layer by layer), so
+    their fp64 and bf16-storage outputs are identical."""
+    d = _load("full30-bf16-depths.npz")
+    assert list(d["depths"]) == [1, 2, 4, 8, 16, 30]
+    for k, name in ((1, "layer1-bf16.npz"), (30, "full30-bf16.npz")):
+        g = _load(name)
+        for key in ("H", "argmax", "logits", "H_s16", "logits_s16"):
+            sweep_key = key.replace("_s16", "") + ("_s16" if key.endswith("_s16") else "")
+            np.testing.assert_array_equal(d[f"{sweep_key}_d{k}"], g[key], err_msg=f"{k} {key}")
+        # layer k-1's keys/values: the single-depth files keep layers 0 and L-1
+        np.testing.assert_array_equal(d[f"kv_last_d{k}"], g["kv_last"][-1])
+    # storage noise grows with depth on the logits (1 layer -> 30 layers)
+    assert max_abs_rel(d["logits_s16_d30"], d["logits_d30"]) > \
+        3 * max_abs_rel(d["logits_s16_d1"], d["logits_d1"])
+
+
+def test_whole_block_file_is_a_valid_trajectory():
+    """The oracle's block: steps left T, T-1, ...; each input canvas is the previous one
+    with exactly the committed positions set to their argmax; the committed counts obey
+    the rule's minimum ceil(masked / steps_left); the block ends with no [MASK]."""
+    import math
+    from synth import workloads
+    w = workloads.FULL30_BF16
+    b = _load("full30-bf16-block.npz")
+    n = int(b["n_forwards"])
+    assert 1 <= n <= w.T and list(b["s"]) == [w.T - i for i in range(n)]
+    assert np.all(b["canvas_in"][0] == w.mask_id)
+    assert int(b["n_committed"].sum()) == w.canvas
+    for i in range(n):
+        m = int((b["canvas_in"][i] == w.mask_id).sum())
+        assert int(b["n_committed"][i]) >= math.ceil(m / int(b["s"][i]))
+        assert np.all((b["H"][i] >= 0) & (b["H"][i] <= math.log(w.vocab) + 1e-3))
+        nxt = b["canvas_in"][i + 1] if i + 1 < n else b["final_canvas"]
+        changed = nxt != b["canvas_in"][i]
+        assert int(changed.sum()) == int(b["n_committed"][i])
+        assert np.all(b["canvas_in"][i][changed] == w.mask_id)
+        assert np.array_equal(nxt[changed], b["argmax"][i][changed])
+        assert np.array_equal(b["mask_after"][i] == 1, nxt == w.mask_id)
+    assert not np.any(b["final_canvas"] == w.mask_id)

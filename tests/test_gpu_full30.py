@@ -9,9 +9,10 @@ Tolerances.  The stated bf16 tolerance (2e-2 max-abs relative) holds for layer 0
 keys and values.  Through 30 random-init layers any perturbation of the size of bf16
 rounding grows: the oracle's own bf16-storage run (the same forward with bf16 kept
 where a bf16 model stores) moves the sampled logits by ~2 %, the entropies by ~11 %
-and layer 29's keys by ~3 % from the fp64 run.  So layer 29's K/V, the logits and the
-entropies are held to max(2e-2, twice that distance) (gpu_helpers.storage_tol);
-argmax is checked where the oracle's top-2 margin exceeds twice the logit error.
+and layer 29's keys by ~3 % from the fp64 run (tests/test_gpu_depth.py measures how
+this grows with depth).  So layer 29's K/V, the logits and the entropies are held to
+1.5x that distance (gpu_helpers.storage_tol); argmax is checked where the oracle's
+top-2 margin exceeds twice the logit error.
 The graph-replayed block is checked by properties that hold at any size: its first
 forward equals the stand-alone forward, it equals the step-by-step API bit for bit,
 and it ends with no [MASK] after at most T forwards.
