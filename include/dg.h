@@ -136,6 +136,15 @@ dg_status dg_sync_status(dg_model* m, void* stream);
 dg_status dg_prefill(dg_model* m, const int32_t* prompt, int32_t B, int32_t P,
                      dg_kv** out, void* stream);
 
+/* The same causal pass into an existing handle made by dg_prefill for this model
+ * with the same B and P: its buffers are overwritten in place (no allocation), so a
+ * serving loop can keep one handle per slot, and block graphs captured for the handle
+ * (dg_generate_block) stay valid.  The caller orders this call after every earlier
+ * use of the handle (same stream, or synchronised).  DG_ERR_INVALID_ARG if the handle
+ * belongs to another model or B / P differ. */
+dg_status dg_prefill_into(dg_model* m, const int32_t* prompt, int32_t B, int32_t P,
+                          dg_kv* kv, void* stream);
+
 /* Frees a KV handle (after synchronising its stream). NULL is a no-op. */
 dg_status dg_kv_destroy(dg_kv* kv);
 

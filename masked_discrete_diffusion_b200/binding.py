@@ -71,6 +71,7 @@ def lib() -> ctypes.CDLL:
             "dg_model_destroy": [vp],
             "dg_sync_status": [vp, vp],
             "dg_prefill": [vp, vp, i32, i32, ctypes.POINTER(vp), vp],
+            "dg_prefill_into": [vp, vp, i32, i32, vp, vp],
             "dg_kv_destroy": [vp],
             "dg_kv_info": [vp, ctypes.POINTER(i32), ctypes.POINTER(i32), ctypes.POINTER(i32)],
             "dg_kv_read": [vp, vp, vp, vp],
@@ -103,7 +104,7 @@ def exported_symbols():
                         "dg_debug_forward", "dg_profile_start", "dg_profile_stop",
                         "dg_launch_count", "dg_op_gemm", "dg_op_moe", "dg_expert_units",
                         "dg_lmhead_entropy_noalloc", "dg_block_loop_launches",
-                        "dg_debug_stall_experts")
+                        "dg_debug_stall_experts", "dg_prefill_into")
             if hasattr(lib(), n)]
 
 
@@ -204,6 +205,15 @@ def dg_prefill(model: Model, prompt: torch.Tensor, stream=None) -> KV:
     _check(lib().dg_prefill(model.handle, _ptr(prompt), prompt.shape[0], prompt.shape[1],
                             ctypes.byref(h), _stream(stream)))
     return KV(model, h)
+
+
+def dg_prefill_into(model: Model, prompt: torch.Tensor, kv: KV, stream=None) -> KV:
+    """Causal pass of prompt [B, P] into an existing handle of the same B and P."""
+    if prompt.dtype != torch.int32 or prompt.dim() != 2:
+        raise ValueError("prompt must be a 2-D int32 tensor")
+    B, P = prompt.shape
+    _check(lib().dg_prefill_into(model.handle, _ptr(prompt), B, P, kv.handle, _stream(stream)))
+    return kv
 
 
 def dg_kv_read(kv: KV, stream=None):

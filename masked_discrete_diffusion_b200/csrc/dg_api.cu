@@ -728,6 +728,18 @@ dg_status dg_prefill(dg_model* m, const int32_t* prompt, int32_t B, int32_t P, d
   return DG_OK;
 }
 
+dg_status dg_prefill_into(dg_model* m, const int32_t* prompt, int32_t B, int32_t P,
+                          dg_kv* kv, void* stream) {
+  g_err.clear();
+  DG_REQUIRE(m && prompt && kv, "null argument");
+  DG_REQUIRE(kv->m == m, "the KV handle belongs to another model (or its model is gone)");
+  DG_REQUIRE(B == kv->B && P == kv->P, "B=%d, P=%d differ from the handle's B=%d, P=%d", B, P,
+             kv->B, kv->P);
+  cudaStream_t st = (cudaStream_t)stream;
+  return m->cfg.dtype == DG_F32 ? Runner<PathTiny>(m, st).prefill(prompt, B, P, kv)
+                                : Runner<PathBF16>(m, st).prefill(prompt, B, P, kv);
+}
+
 dg_status dg_kv_destroy(dg_kv* kv) {
   if (!kv) return DG_OK;
   cudaDeviceSynchronize();

@@ -106,3 +106,26 @@ def test_block_graph_replay_is_deterministic(setup):
     binding.dg_sync_status(model)
     for o, l in outs[1:]:
         assert torch.equal(o, outs[0][0]) and torch.equal(l, outs[0][1])
+
+
+def test_prefill_into_reuses_the_handle(setup):
+    """Refilling a handle in place gives the cache a fresh dg_prefill of the same prompt
+    gives, and the block graph captured for the handle then denoises the new prompt
+    exactly as a fresh handle would."""
+    binding, model, kv, ws, okv = setup
+    other = model_inputs.prompt(W, "cuda", first=W.batch)            # canvases 3..5
+    fresh = binding.dg_prefill(model, other)
+    slot = binding.dg_prefill(model, model_inputs.prompt(W, "cuda"))
+    a = binding.dg_generate_block(model, slot, W.T, W.gamma)          # graph for the slot
+    binding.dg_prefill_into(model, other, slot)
+    k1, v1 = binding.dg_kv_read(slot)
+    k2, v2 = binding.dg_kv_read(fresh)
+    assert torch.equal(k1, k2) and torch.equal(v1, v2)
+    b = binding.dg_generate_block(model, slot, W.T, W.gamma)          # same graph, new cache
+    c = binding.dg_generate_block(model, fresh, W.T, W.gamma)
+    binding.dg_sync_status(model)
+    assert torch.equal(b, c) and not torch.equal(a, b)
+    with pytest.raises(binding.DGError):                              # shape must match
+        binding.dg_prefill_into(model, other[:2].contiguous(), slot)
+    slot.close()
+    fresh.close()
