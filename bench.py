@@ -246,6 +246,43 @@ def run_e2e(args, w, world, model, prompt, canvas, stream):
     return e2e_val
 
 
+def run_blocks(args, w, world, model, prompt):
+    """Block-autoregressive generation of args.blocks blocks per canvas (each finished
+    block joins the context through the causal pass before the next is denoised),
+    device-timed from the first block to the last, prompt pass excluded; tokens per
+    forward counts the K - 1 append passes of K blocks."""
+    import torch
+
+    from masked_discrete_diffusion_b200 import binding, metrics
+    K, B, C = args.blocks, w.batch, w.canvas
+    kv = binding.dg_prefill(model, prompt)
+    for _ in range(max(args.warmup, 1)):
+        binding.dg_prefill_into(model, prompt, kv)
+        binding.dg_generate_blocks(model, kv, K, w.T, w.gamma)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = 0.0
+    nf = None
+    for _ in range(args.steps):
+        binding.dg_prefill_into(model, prompt, kv)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        _, nf = binding.dg_generate_blocks(model, kv, K, w.T, w.gamma)
+        e1.record()
+        e1.synchronize()
+        ms += e0.elapsed_time(e1)
+    binding.dg_sync_status(model)
+    kv.close()
+    ms_max = max_over_ranks(ms, world)
+    per_block = nf.max(dim=1).values.cpu().tolist()
+    return {"n_blocks": K,
+            "canvas_tokens_per_s": job_throughput(world, B * K * C, args.steps, ms_max),
+            "ms_per_step": ms_max / args.steps,
+            "forwards_per_block": per_block,
+            "tokens_per_forward_eq10": metrics.tokens_per_forward([C] * K, per_block),
+            "includes": "dg_generate_blocks: K blocks, K - 1 dg_append_block causal passes"}
+
+
 def run_ours(args, w, world, rank, local):
     import numpy as np
     import torch
@@ -256,7 +293,9 @@ def run_ours(args, w, world, rank, local):
     build_once(world, local)
     peaks, peak_src = load_peaks()
     tensors = model_inputs.weight_set(w, "cuda")
-    model = binding.Model(binding.make_config(w), tensors)
+    # the context may grow by the appended blocks of the multi-block measurement
+    max_prompt = w.prompt_len + max(args.blocks - 1, 0) * w.canvas
+    model = binding.Model(binding.make_config(w, max_prompt=max_prompt), tensors)
     prompt = model_inputs.prompt(w, "cuda", first=rank * w.batch)
     kv = binding.dg_prefill(model, prompt)
     binding.dg_sync_status(model)
@@ -319,6 +358,7 @@ def run_ours(args, w, world, rank, local):
     kv.close()
     if not args.skip_e2e:
         e2e_val = run_e2e(args, w, world, model, prompt, canvas, stream)
+    blocks = run_blocks(args, w, world, model, prompt) if args.blocks > 1 else None
     # roofline of the dominant kernel group (routed-expert FFN); units = experts that
     # received rows, counted per (layer, forward) on the device
     ex_ms, ex_groups = prof["experts"]
@@ -385,6 +425,7 @@ def run_ours(args, w, world, rank, local):
             "includes": "prompt H2D, dg_prefill_into (the slot's KV handle refilled), "
                         "dg_generate_block, canvas D2H, every step"},
         "experts_streamed_per_layer_forward": unique_mean,
+        "blocks": blocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         t_block, desc, threads = OracleSample(w).run()
@@ -404,6 +445,8 @@ def main():
     ap.add_argument("--workload", default="full30-bf16")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--blocks", type=int, default=2,
+                    help="blocks of the multi-block measurement (1: skip it)")
     args = ap.parse_args()
     from synth import workloads
     w = workloads.get(args.workload)

@@ -137,11 +137,12 @@ dg_status dg_prefill(dg_model* m, const int32_t* prompt, int32_t B, int32_t P,
                      dg_kv** out, void* stream);
 
 /* The same causal pass into an existing handle made by dg_prefill for this model
- * with the same B and P: its buffers are overwritten in place (no allocation), so a
- * serving loop can keep one handle per slot, and block graphs captured for the handle
- * (dg_generate_block) stay valid.  The caller orders this call after every earlier
- * use of the handle (same stream, or synchronised).  DG_ERR_INVALID_ARG if the handle
- * belongs to another model or B / P differ. */
+ * with the same B (any 1 <= P <= max_prompt; a handle grown by dg_append_block returns
+ * to a prompt of P tokens): its buffers are overwritten in place (no allocation), so a
+ * serving loop can keep one handle per slot.  Block graphs are captured per (handle,
+ * context length), so a graph captured for the same P is replayed.  The caller orders
+ * this call after every earlier use of the handle (same stream, or synchronised).
+ * DG_ERR_INVALID_ARG if the handle belongs to another model or B differs. */
 dg_status dg_prefill_into(dg_model* m, const int32_t* prompt, int32_t B, int32_t P,
                           dg_kv* kv, void* stream);
 
@@ -181,6 +182,27 @@ dg_status dg_denoise_step(dg_model* m, const dg_kv* kv, int32_t* canvas, uint8_t
 dg_status dg_generate_block(dg_model* m, const dg_kv* kv, int32_t T, float gamma,
                             int32_t* canvas_out, int32_t* n_forwards,
                             int32_t* router_load, void* stream);
+
+/* Block-autoregressive continuation ("DiffusionGemma 技术报告", §3.1: each finished
+ * block joins the context through the causal encoder pass before the next block is
+ * denoised; §3.4, the K - 1 extra forwards of K blocks in the tokens-per-forward
+ * count).  tokens: [B, C] int32 ids in [0, V), the finished canvases of kv's batch.
+ * The block's rows run the causal pass at positions P .. P + C - 1 (keys: the cached
+ * window and the block's own rows within the sliding window, no timestep embedding);
+ * then every layer's cache keeps the last min(W + C, window) positions and kv's P grows
+ * by C.  (Block graphs are captured per context length, so none is invalidated.)
+ * Requires P + C <= max_prompt (the context a model is created for bounds the whole
+ * sequence, prompt and appended blocks) and no [MASK] in tokens (checked on the
+ * device: DG_ERR_INVALID_ARG on the next status read). */
+dg_status dg_append_block(dg_model* m, dg_kv* kv, const int32_t* tokens, void* stream);
+
+/* n_blocks blocks one after the other: dg_generate_block, then (except after the
+ * last) dg_append_block of the finished canvases.  out: [B, n_blocks C] int32, block k
+ * of canvas b in columns k C .. k C + C - 1; n_forwards: [n_blocks, B] int32 forwards
+ * per block and canvas (nullable).  kv ends extended by n_blocks - 1 blocks.
+ * Requires n_blocks >= 1 and P + (n_blocks - 1) C <= max_prompt. */
+dg_status dg_generate_blocks(dg_model* m, dg_kv* kv, int32_t n_blocks, int32_t T, float gamma,
+                             int32_t* out, int32_t* n_forwards, void* stream);
 
 /* The sampler step alone, on caller-provided statistics: entropy [B, C] fp32,
  * argmax [B, C] int32, canvas/mask [B, C] updated in place, n_committed [B].

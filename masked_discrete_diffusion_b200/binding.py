@@ -72,6 +72,8 @@ def lib() -> ctypes.CDLL:
             "dg_sync_status": [vp, vp],
             "dg_prefill": [vp, vp, i32, i32, ctypes.POINTER(vp), vp],
             "dg_prefill_into": [vp, vp, i32, i32, vp, vp],
+            "dg_append_block": [vp, vp, vp, vp],
+            "dg_generate_blocks": [vp, vp, i32, i32, f32, vp, vp, vp],
             "dg_kv_destroy": [vp],
             "dg_kv_info": [vp, ctypes.POINTER(i32), ctypes.POINTER(i32), ctypes.POINTER(i32)],
             "dg_kv_read": [vp, vp, vp, vp],
@@ -104,7 +106,8 @@ def exported_symbols():
                         "dg_debug_forward", "dg_profile_start", "dg_profile_stop",
                         "dg_launch_count", "dg_op_gemm", "dg_op_moe", "dg_expert_units",
                         "dg_lmhead_entropy_noalloc", "dg_block_loop_launches",
-                        "dg_debug_stall_experts", "dg_prefill_into")
+                        "dg_debug_stall_experts", "dg_prefill_into", "dg_append_block",
+                        "dg_generate_blocks")
             if hasattr(lib(), n)]
 
 
@@ -183,6 +186,12 @@ class KV:
         _check(lib().dg_kv_info(handle, ctypes.byref(B), ctypes.byref(P), ctypes.byref(W)))
         self.B, self.P, self.W = B.value, P.value, W.value
 
+    def refresh(self):
+        """Re-reads B, P and W (they change when blocks are appended)."""
+        B, P, W = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+        _check(lib().dg_kv_info(self.handle, ctypes.byref(B), ctypes.byref(P), ctypes.byref(W)))
+        self.B, self.P, self.W = B.value, P.value, W.value
+
     def close(self):
         if getattr(self, "handle", None):
             _check(lib().dg_kv_destroy(self.handle))
@@ -208,12 +217,35 @@ def dg_prefill(model: Model, prompt: torch.Tensor, stream=None) -> KV:
 
 
 def dg_prefill_into(model: Model, prompt: torch.Tensor, kv: KV, stream=None) -> KV:
-    """Causal pass of prompt [B, P] into an existing handle of the same B and P."""
+    """Causal pass of prompt [B, P] into an existing handle of the same B."""
     if prompt.dtype != torch.int32 or prompt.dim() != 2:
         raise ValueError("prompt must be a 2-D int32 tensor")
     B, P = prompt.shape
     _check(lib().dg_prefill_into(model.handle, _ptr(prompt), B, P, kv.handle, _stream(stream)))
+    kv.refresh()
     return kv
+
+
+def dg_append_block(model: Model, kv: KV, tokens: torch.Tensor, stream=None) -> KV:
+    """Causal pass of the finished blocks tokens [B, C] into kv (the context grows by C)."""
+    if tokens.dtype != torch.int32 or tokens.dim() != 2:
+        raise ValueError("tokens must be a 2-D int32 tensor")
+    _check(lib().dg_append_block(model.handle, kv.handle, _ptr(tokens), _stream(stream)))
+    kv.refresh()
+    return kv
+
+
+def dg_generate_blocks(model: Model, kv: KV, n_blocks: int, T: int, gamma: float,
+                       stream=None):
+    """n_blocks blocks one after the other; returns (tokens [B, n_blocks C],
+    forwards [n_blocks, B]); kv ends extended by n_blocks - 1 blocks."""
+    c = model.cfg
+    out = torch.empty(kv.B, n_blocks * c.canvas, dtype=torch.int32, device="cuda")
+    nf = torch.zeros(n_blocks, kv.B, dtype=torch.int32, device="cuda")
+    _check(lib().dg_generate_blocks(model.handle, kv.handle, n_blocks, T, gamma, _ptr(out),
+                                    _ptr(nf), _stream(stream)))
+    kv.refresh()
+    return out, nf
 
 
 def dg_kv_read(kv: KV, stream=None):

@@ -162,6 +162,7 @@ template <class Path> static dg_status alloc_workspace(dg_model* m) {
   DG_TRY(ws_alloc(ws, &ws.ncommit, c.max_batch));
   DG_TRY(ws_alloc(ws, &ws.remaining, c.max_batch));
   DG_TRY(ws_alloc(ws, &ws.loop_s, 1));
+  DG_TRY(ws_alloc(ws, &ws.blk, lm_rows));
   DG_TRY_CUDA(cudaMemset(ws.err, 0, 4 * sizeof(int32_t)));
   launch_pdl((rope_table_kernel), 256, 256, 0, cudaStream_t(0), 1, (double)c.rope_base, (int)h, ws.max_pos, ws.rope,
                                   sizeof(Acc) == 8 ? 1 : 0);
@@ -472,6 +473,59 @@ template <class Path> struct Runner {
     return check_launch("prefill");
   }
 
+  // Causal pass of B finished blocks (tokens [B, C], positions P .. P + C - 1) over the
+  // cached window: per layer the block's rows attend to the cached keys and to their
+  // own earlier rows within the sliding window (the same computation the prompt pass
+  // would have made had the block been part of the prompt); then each layer's window
+  // becomes the last min(W + C, window) positions of (window, block).  No LM head.
+  dg_status append(const int32_t* tokens, dg_kv* kv) {
+    const int B = kv->B, C = c.canvas, n = B * C, d = c.d_model, h = c.head_dim;
+    const int Hkv = c.n_kv_heads;
+    const int np = (C + 63) / 64 * 64;
+    const size_t es = sizeof(TKV);
+    launch_pdl((embed_kernel<TW, TR>), n, 256, 0, st, 1, tokens, (const TW*)m->w.tok_emb, x(), n,
+               d, c.vocab - 1, -1.0, ws.err, (const int32_t*)nullptr, 1);
+    ++m->launches;
+    // padding columns of the block's transposed values must read as zero
+    if (np != C) DG_TRY_CUDA(cudaMemsetAsync(ws.vc, 0, (size_t)B * Hkv * h * np * es, st));
+    const int W = kv->W, Wn = std::min(W + C, c.window);
+    const int keep = std::max(0, Wn - C);          // cached positions that stay
+    const int take = std::min(C, Wn);              // block positions that enter
+    const size_t slabK = (size_t)kv->Wp * h * es;  // one (b, g) slab of keys
+    const size_t rowV = (size_t)kv->Wp * es;       // one (b, g, dim) row of values^T
+    TKV* tmp = (TKV*)ws.up;                        // scratch: the kept part of a layer
+    for (int l = 0; l < c.n_layers; ++l) {
+      DG_TRY(layer(l, n, B, C, kv->P, kv, true, nullptr));
+      char* K = (char*)kv->k + (size_t)l * B * Hkv * slabK;
+      char* V = (char*)kv->v + (size_t)l * B * Hkv * h * rowV;
+      if (keep > 0 && W - keep > 0) {  // shift the kept positions to the front (via scratch)
+        DG_TRY_CUDA(cudaMemcpy2DAsync(tmp, (size_t)keep * h * es, K + (size_t)(W - keep) * h * es,
+                                      slabK, (size_t)keep * h * es, (size_t)B * Hkv,
+                                      cudaMemcpyDeviceToDevice, st));
+        DG_TRY_CUDA(cudaMemcpy2DAsync(K, slabK, tmp, (size_t)keep * h * es,
+                                      (size_t)keep * h * es, (size_t)B * Hkv,
+                                      cudaMemcpyDeviceToDevice, st));
+        DG_TRY_CUDA(cudaMemcpy2DAsync(tmp, (size_t)keep * es, V + (size_t)(W - keep) * es, rowV,
+                                      (size_t)keep * es, (size_t)B * Hkv * h,
+                                      cudaMemcpyDeviceToDevice, st));
+        DG_TRY_CUDA(cudaMemcpy2DAsync(V, rowV, tmp, (size_t)keep * es, (size_t)keep * es,
+                                      (size_t)B * Hkv * h, cudaMemcpyDeviceToDevice, st));
+      }
+      // the block's last `take` keys [B, Hkv, np, h] and values^T [B, Hkv, h, np] after them
+      DG_TRY_CUDA(cudaMemcpy2DAsync(K + (size_t)keep * h * es, slabK,
+                                    (const char*)ws.kc + (size_t)(C - take) * h * es,
+                                    (size_t)np * h * es, (size_t)take * h * es, (size_t)B * Hkv,
+                                    cudaMemcpyDeviceToDevice, st));
+      DG_TRY_CUDA(cudaMemcpy2DAsync(V + (size_t)keep * es, rowV,
+                                    (const char*)ws.vc + (size_t)(C - take) * es, (size_t)np * es,
+                                    (size_t)take * es, (size_t)B * Hkv * h,
+                                    cudaMemcpyDeviceToDevice, st));
+    }
+    kv->P += C;
+    kv->W = Wn;
+    return check_launch("append");
+  }
+
   // Canvas forward: statistics into ent/amax; optional logits/hidden (test hook).
   dg_status forward(const dg_kv* kv, const int32_t* canvas, int s, int T, float* ent,
                     int32_t* amax, float* logits, float* hidden, int32_t* load) {
@@ -700,7 +754,9 @@ dg_status dg_prefill(dg_model* m, const int32_t* prompt, int32_t B, int32_t P, d
   kv->B = B;
   kv->P = P;
   kv->W = std::min(P, c.window);
-  kv->Wp = (kv->W + 63) / 64 * 64;
+  // room for the window the cache can grow to by appended blocks (dg_append_block):
+  // the whole context stays within max_prompt positions
+  kv->Wp = (std::min(c.max_prompt, c.window) + 63) / 64 * 64;
   kv->elem = c.dtype == DG_F32 ? sizeof(double) : sizeof(bf16);
   const size_t n = (size_t)c.n_layers * B * c.n_kv_heads * kv->Wp * c.head_dim * kv->elem;
   if (cudaMalloc(&kv->k, n) != cudaSuccess || cudaMalloc(&kv->v, n) != cudaSuccess ||
@@ -733,8 +789,11 @@ dg_status dg_prefill_into(dg_model* m, const int32_t* prompt, int32_t B, int32_t
   g_err.clear();
   DG_REQUIRE(m && prompt && kv, "null argument");
   DG_REQUIRE(kv->m == m, "the KV handle belongs to another model (or its model is gone)");
-  DG_REQUIRE(B == kv->B && P == kv->P, "B=%d, P=%d differ from the handle's B=%d, P=%d", B, P,
-             kv->B, kv->P);
+  DG_REQUIRE(B == kv->B, "B=%d differs from the handle's B=%d", B, kv->B);
+  DG_REQUIRE(P >= 1 && P <= m->cfg.max_prompt, "P=%d outside [1, max_prompt=%d]", P,
+             m->cfg.max_prompt);
+  kv->P = P;  // a handle grown by appended blocks returns to a prompt of P tokens
+  kv->W = std::min(P, m->cfg.window);
   cudaStream_t st = (cudaStream_t)stream;
   return m->cfg.dtype == DG_F32 ? Runner<PathTiny>(m, st).prefill(prompt, B, P, kv)
                                 : Runner<PathBF16>(m, st).prefill(prompt, B, P, kv);
@@ -925,7 +984,8 @@ static dg_status generate_graphed(dg_model* m, const dg_kv* kv, int32_t T, long 
                                   int32_t* router_load, cudaStream_t st) {
   dg::BlockGraph* g = nullptr;
   for (auto* x : m->graphs)
-    if (x->kv == kv && x->T == T && x->gq == gq && x->canvas == canvas_out &&
+    if (x->kv == kv && x->kv_P == kv->P && x->kv_W == kv->W && x->T == T && x->gq == gq &&
+        x->canvas == canvas_out &&
         x->nfwd == n_forwards && x->load == router_load && x->prof == m->profiling &&
         (!x->prof || x->fcap == m->prof_forwards)) {
       g = x;
@@ -938,6 +998,8 @@ static dg_status generate_graphed(dg_model* m, const dg_kv* kv, int32_t T, long 
     }
     g = new dg::BlockGraph();
     g->kv = kv;
+    g->kv_P = kv->P;
+    g->kv_W = kv->W;
     g->T = T;
     g->gq = gq;
     g->canvas = canvas_out;
@@ -1010,6 +1072,46 @@ dg_status dg_generate_block(dg_model* m, const dg_kv* kv, int32_t T, float gamma
   if (m->use_graphs)
     return generate_graphed(m, kv, T, gq, canvas_out, n_forwards, router_load, st);
   return generate_impl(m, kv, T, gq, canvas_out, n_forwards, router_load, st);
+}
+
+dg_status dg_append_block(dg_model* m, dg_kv* kv, const int32_t* tokens, void* stream) {
+  g_err.clear();
+  DG_REQUIRE(m && kv && tokens, "null argument");
+  DG_REQUIRE(kv->m == m, "the KV handle belongs to another model (or its model is gone)");
+  const dg_config& c = m->cfg;
+  DG_REQUIRE(kv->P + c.canvas <= c.max_prompt,
+             "P + C = %d exceeds max_prompt = %d (the context the model was created for)",
+             kv->P + c.canvas, c.max_prompt);
+  // the kept part of a layer's window passes through the gathered-rows buffer
+  const size_t need = (size_t)kv->B * c.n_kv_heads * c.head_dim * std::min(kv->W, c.window) *
+                      kv->elem;
+  DG_REQUIRE(need <= m->ws.max_rows * (size_t)c.d_model * kv->elem,
+             "append scratch too small for this cache");
+  cudaStream_t st = (cudaStream_t)stream;
+  return c.dtype == DG_F32 ? Runner<PathTiny>(m, st).append(tokens, kv)
+                           : Runner<PathBF16>(m, st).append(tokens, kv);
+}
+
+dg_status dg_generate_blocks(dg_model* m, dg_kv* kv, int32_t n_blocks, int32_t T, float gamma,
+                             int32_t* out, int32_t* n_forwards, void* stream) {
+  g_err.clear();
+  DG_REQUIRE(m && kv && out, "null argument");
+  DG_REQUIRE(kv->m == m, "the KV handle belongs to another model (or its model is gone)");
+  DG_REQUIRE(n_blocks >= 1, "n_blocks must be >= 1");
+  const dg_config& c = m->cfg;
+  DG_REQUIRE(kv->P + (long long)(n_blocks - 1) * c.canvas <= c.max_prompt,
+             "P + (n_blocks - 1) C exceeds max_prompt = %d", c.max_prompt);
+  const int B = kv->B, C = c.canvas;
+  cudaStream_t st = (cudaStream_t)stream;
+  for (int k = 0; k < n_blocks; ++k) {
+    DG_TRY(dg_generate_block(m, kv, T, gamma, m->ws.blk, n_forwards ? n_forwards + k * B : nullptr,
+                             nullptr, stream));
+    DG_TRY_CUDA(cudaMemcpy2DAsync(out + (size_t)k * C, (size_t)n_blocks * C * sizeof(int32_t),
+                                  m->ws.blk, (size_t)C * sizeof(int32_t), C * sizeof(int32_t), B,
+                                  cudaMemcpyDeviceToDevice, st));
+    if (k + 1 < n_blocks) DG_TRY(dg_append_block(m, kv, m->ws.blk, stream));
+  }
+  return DG_OK;
 }
 
 dg_status dg_eb_sample(const float* entropy, const int32_t* argmax, int32_t* canvas,

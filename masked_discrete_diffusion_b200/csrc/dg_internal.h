@@ -109,6 +109,7 @@ struct Workspace {
   float* ent = nullptr;                             // [max_batch, C] entropies
   int32_t *amax = nullptr, *ncommit = nullptr;      // [max_batch, C], [max_batch]
   int32_t *remaining = nullptr, *loop_s = nullptr;  // [max_batch] masked left; steps left
+  int32_t* blk = nullptr;                           // [max_batch, C] a finished block
   int max_pos = 0;
   size_t kc_elems = 0;
   int max_tiles = 0;
@@ -122,6 +123,7 @@ namespace dg {
 struct BlockGraph {
   cudaGraphExec_t exec = nullptr;
   const dg_kv* kv = nullptr;
+  int kv_P = 0, kv_W = 0;  // the handle's context when captured (positions, window)
   int T = 0;
   long long gq = 0;
   int32_t *canvas = nullptr, *nfwd = nullptr, *load = nullptr;

@@ -82,10 +82,16 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   // key tiles of this split
   const int TA = (p.nA + AT_KT - 1) / AT_KT, TB = (p.nB + AT_KT - 1) / AT_KT;
   int t_lo = 0, t_hi = TA + TB;
-  if (p.causal) {  // only segment B; tiles meeting [q0 - window + 1, q0 + 127]
-    const int lo_pos = max(p.kposB, p.qpos0 + q0 - p.window + 1);
+  if (p.causal) {
+    // tiles meeting the key positions [q - window + 1, q] of the tile's queries: the
+    // cached segment A (positions before segment B) from its first tile in reach, then
+    // segment B up to the last query
+    const int lo_pos = p.qpos0 + q0 - p.window + 1;
     const int hi_pos = min(p.kposB + p.nB - 1, p.qpos0 + min(q0 + 127, p.nq - 1));
-    t_lo = TA + (lo_pos - p.kposB) / AT_KT;
+    if (TA > 0 && p.kposA + p.nA - 1 >= lo_pos)
+      t_lo = max(0, lo_pos - p.kposA) / AT_KT;
+    else
+      t_lo = TA + max(0, lo_pos - p.kposB) / AT_KT;
     t_hi = TA + (hi_pos - p.kposB) / AT_KT + 1;
   }
   const int my_lo = t_lo + z * p.tiles_per_split;

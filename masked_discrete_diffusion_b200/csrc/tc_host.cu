@@ -381,7 +381,9 @@ dg_status tc_attention(dg_model* m, const bf16* q, int B, int nq, int qpos0, con
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)h));
   p.out = out;
   const int TA = ceil_div_i(p.nA, AT_KT), TB = ceil_div_i(nB, AT_KT);
-  const int total = causal ? std::min(TB, ceil_div_i(c.window + 127, AT_KT) + 1) : TA + TB;
+  // causal: a query tile reaches window + 127 key positions, which meet at most that
+  // many tiles of each segment's grid plus one where the grids change
+  const int total = causal ? std::min(TA + TB, ceil_div_i(c.window + 127, AT_KT) + 2) : TA + TB;
   const int qtiles = ceil_div_i(nq, 128);
   const int base = qtiles * Hq * B;
   const int n_sm = state(m)->n_sm;

@@ -379,3 +379,30 @@ def prefill_then_forward(ws: Weights, prompt: np.ndarray, canvas: np.ndarray, s:
     st["routes"] = routes
     st["kv"] = kv_layers
     return st
+
+
+def generate_blocks(ws: Weights, prompt: np.ndarray, n_blocks: int, T: int, gamma: float):
+    """Block-autoregressive generation: block k is denoised from all [MASK] conditioned
+    on the causal pass over the prompt followed by blocks 0 .. k-1, and then joins the
+    context ("DiffusionGemma 技术报告" (full translation page), §3.1 "块自回归生成":
+    the context is encoded causally, each finished block is appended before the next).
+
+    Returns (blocks [n_blocks, C], trajectories per block as generate_block gives them).
+    """
+    from oracle import sampler
+    w = ws.w
+    context = np.asarray(prompt, dtype=np.int64)
+    blocks, trajs = [], []
+    for _ in range(n_blocks):
+        kv = prefill(ws, context)
+        P = len(context)
+
+        def forward(canvas, s, kv=kv, P=P):
+            st = denoise_forward(ws, kv, canvas, s, T, P)
+            return st["H"], st["argmax"]
+
+        canvas, traj = sampler.generate_block(forward, w.canvas, w.mask_id, T, gamma)
+        blocks.append(canvas)
+        trajs.append(traj)
+        context = np.concatenate([context, canvas])
+    return np.stack(blocks), trajs

@@ -70,6 +70,14 @@ def prompt(w: Workload, device="cpu", first: int = 0) -> torch.Tensor:
     return torch.stack(rows) if rows else torch.empty(0, w.prompt_len, dtype=torch.int32)
 
 
+def block_tokens(w: Workload, device="cpu", first: int = 0) -> torch.Tensor:
+    """[B, C] int32 tokens uniform in [0, V): finished blocks to append to canvases
+    first .. first + B - 1 (stand-ins for denoised canvases)."""
+    rows = [gen.tokens(w.seed, f"block.b{b}", w.canvas, w.vocab, device)
+            for b in range(first, first + w.batch)]
+    return torch.stack(rows)
+
+
 def is_fp8_expert(w: Workload, name: str) -> bool:
     return w.dtype == "bf16_fp8exp" and name.split(".")[-1] in ("gate", "up", "down")
 

@@ -27,6 +27,9 @@ Two further modes on a deep workload:
      values.  One pass through the layers serves every depth (the prompt pass and the
      canvas pass interleave layer by layer, so the canvas state after layer k-1 is the
      k-layer model's final residual).
+  <name>@append  -> <name>-append.npz: canvas 0's prompt and a block of seeded tokens
+     as one causal pass, layer 0's window keys / values at a few positions (the
+     reference for appending a finished block to the cache).
   <name>@block   -> <name>-block.npz: the oracle's whole block (all [MASK], up to T
      forwards, the entropy-bound sampler after each): per step the input canvas, the
      steps left, H, argmax, margin and the number committed; the number of forwards.
@@ -139,6 +142,30 @@ def make(name: str, canvas_index: int = 0, storage_variant: bool = False):
           f"min router gap {min(rmarg):.3g}, sampler n {n2}")
 
 
+APPEND_POS = (0, 8, 760, 776, 1016, 1024)   # window offsets: 8 positions from each
+
+
+def append_case(name: str):
+    """<name>-append.npz: canvas 0's prompt followed by a block of seeded tokens
+    (synth.model_inputs.block_tokens), as one causal pass: layer 0's keys and values
+    of 8 consecutive window positions from each offset in APPEND_POS (the window is
+    the last min(P + C, window) positions of the whole sequence)."""
+    w = workloads.get(name)
+    t0 = time.time()
+    prompt = model_inputs.prompt(w.with_(batch=1))[0].numpy()
+    block = model_inputs.block_tokens(w.with_(batch=1))[0].numpy()
+    seq = np.concatenate([prompt, block])
+    ws = om.Weights(w.with_(n_layers=1), keep_layers=False)
+    K, V = om.prefill(ws, seq)[0]                       # [W, Hkv, h]
+    Wn = K.shape[0]
+    sel = [o + i for o in APPEND_POS for i in range(8) if o + i < Wn]
+    out = dict(window=np.array(Wn), positions=np.array(sel),
+               k=K[sel].transpose(1, 0, 2), v=V[sel].transpose(1, 0, 2))
+    path = os.path.join(HERE, f"{name}-append.npz")
+    np.savez_compressed(path, **out)
+    print(f"{name}: wrote {path} in {time.time() - t0:.0f} s (window {Wn})")
+
+
 DEPTHS = (1, 2, 4, 8, 16, 30)
 
 
@@ -216,6 +243,9 @@ if __name__ == "__main__":
     # arguments: workload names, optionally "name:canvas" to pick a canvas of the batch
     # and the suffix "+s16" for the bf16 storage variant as well ("+s16only": that alone)
     for arg in sys.argv[1:] or ["layer1-bf16"]:
+        if arg.endswith("@append"):
+            append_case(arg.removesuffix("@append"))
+            continue
         if arg.endswith("@depths"):
             depth_sweep(arg.removesuffix("@depths"))
             continue

@@ -91,6 +91,8 @@ def test_null_handles_and_bad_sizes_rejected_without_device(lib):
         "dg_op_moe": (None, 0, fake, fake, 1, None),
         "dg_debug_stall_experts": (None, 1000000),
         "dg_prefill_into": (None, fake, 1, 1, fake, None),
+        "dg_append_block": (None, fake, fake, None),
+        "dg_generate_blocks": (None, fake, 1, 1, 1.0, fake, None, None),
     }
     for name, args in calls.items():
         assert getattr(lib, name)(*args) == 1, name

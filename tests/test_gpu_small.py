@@ -125,7 +125,7 @@ def test_prefill_into_reuses_the_handle(setup):
     c = binding.dg_generate_block(model, fresh, W.T, W.gamma)
     binding.dg_sync_status(model)
     assert torch.equal(b, c) and not torch.equal(a, b)
-    with pytest.raises(binding.DGError):                              # shape must match
+    with pytest.raises(binding.DGError):                              # batch must match
         binding.dg_prefill_into(model, other[:2].contiguous(), slot)
     slot.close()
     fresh.close()
