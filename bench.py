@@ -26,11 +26,13 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# DRAM bytes per routed expert streamed by the routed-expert kernel, from an ncu capture
-# of that kernel as it now stands (see the roofline computation below).  None until
-# recaptured: the last capture (98.38 MB for the 9 experts of a first forward) predates
-# the bounded wait for in-flight copies added to the kernel's producer.
-DRAM_BYTES_PER_EXPERT = None
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per routed expert streamed
+# by the routed-expert kernel as it now stands: one ncu capture of the 12 launches of
+# a one-layer block (layer1-bf16, same kernel shapes as one layer of the 30-layer
+# workload; profiles/tc_moe_kernel_layer1-bf16.md): 1,274.9 MB over 123 streamed
+# experts = 10,365,317 B each, 1.10x the 9,437,184 B of weights (the rest: gathered and
+# hidden rows, which ncu's cold cache sends to DRAM).
+DRAM_BYTES_PER_EXPERT = 10365317
 
 
 def load_peaks():
@@ -365,11 +367,8 @@ def run_ours(args, w, world, rank, local):
     unique_mean = units / max(ex_groups, 1)
     cost = metrics.forward_cost(model.cfg, B, kv_W, [unique_mean] * w.n_layers)
     ex_bytes = unique_mean * cost["expert_bytes"]
-    # DRAM traffic of the routed-expert launch: dram__bytes_read.sum + dram__bytes_write.sum
-    # in one ncu capture of the one-layer workload (same kernel shapes; first forward of
-    # the block, 9 experts streamed): 98.38 MB = 85.0 MB of expert weights + the gathered
-    # rows and hidden rows, which ncu's cold cache sends to DRAM; scaled by this run's
-    # experts per launch.  Valid for the routed-expert kernel as captured.
+    # DRAM traffic of the routed-expert launch: the captured bytes per streamed expert
+    # (DRAM_BYTES_PER_EXPERT) times this run's experts per launch
     ex_traffic = (unique_mean * DRAM_BYTES_PER_EXPERT
                   if w.dtype == "bf16" and DRAM_BYTES_PER_EXPERT else None)
     ex_avg_s = ex_ms / 1e3 / max(ex_groups, 1)
