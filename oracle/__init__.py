@@ -8,6 +8,8 @@ generators in `synth/`).
 Modules:
   model     fp64 numpy forward: prefill, canvas forward, LM-head entropy
   sampler   Entropy-Bound sampler step and block loop (integer decisions)
+  anneal    the Report's default sampler: annealed entropy-bounded refinement over a
+            uniform-noise canvas, adaptive stop, SplitMix64 draws
   absorbing absorbing forward process (invariant checks)
 
 Every function is pinned by `tests/test_oracle_*.py` against closed forms,

@@ -406,3 +406,22 @@ def generate_blocks(ws: Weights, prompt: np.ndarray, n_blocks: int, T: int, gamm
         trajs.append(traj)
         context = np.concatenate([context, canvas])
     return np.stack(blocks), trajs
+
+
+def generate_block_annealed(ws: Weights, prompt: np.ndarray, seed: int, params=None):
+    """One canvas denoised by the Report's default sampler (entropy-bounded refinement
+    with temperature annealing and adaptive stopping over a uniform-noise canvas,
+    "DiffusionGemma 技术报告" (full translation page), §3.2 and §3.3), conditioned on
+    the causal pass over the prompt.  Step k's forward takes the time input
+    t = (N - k) / N.  Returns oracle.anneal.generate_block's (result, trajectory).
+    """
+    from oracle import anneal
+    p = params or anneal.Params()
+    w = ws.w
+    kv = prefill(ws, np.asarray(prompt, dtype=np.int64))
+    P = len(prompt)
+
+    def forward(canvas, k):
+        return denoise_forward(ws, kv, canvas, p.N - k, p.N, P, want_logits=True)["logits"]
+
+    return anneal.generate_block(forward, w.canvas, w.vocab, seed, p)
