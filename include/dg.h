@@ -212,6 +212,62 @@ dg_status dg_eb_sample(const float* entropy, const int32_t* argmax, int32_t* can
                        uint8_t* mask, int32_t B, int32_t C, int32_t steps_left,
                        float gamma, int32_t* n_committed, void* stream);
 
+/* ---- the Report's default sampler ("DiffusionGemma 技术报告", §3.2 "画布初始化",
+ * "多项式扩散", §3.3 "熵有界的 token 精炼", "温度退火", "自适应停止启发式") ----------
+ * A canvas starts from uniformly drawn tokens and is refined for at most N steps:
+ * step k (0-based) runs the forward at t = (N - k) / N (timestep input t), tempers the
+ * logits by tau = tau_min + (tau_max - tau_min) t, draws a token at every position
+ * from softmax(l / tau) (Gumbel-max), and accepts, in ascending order of the tempered
+ * entropy (ties: lower position), the longest prefix whose entropies satisfy
+ * sum - max <= b (the mutual-information bound; at least one position); every other
+ * position is re-noised to a uniform token.  After a step the canvas stops when the
+ * mean tempered entropy is below e_stop (sum of 2^-48 fixed-point entropies
+ * < C floor(e_stop 2^48)) and the argmax sequence equals the previous step's; then,
+ * or after step N - 1, the canvas becomes that step's argmax sequence.
+ * Random draws: SplitMix64 used counter-wise, one seed per canvas (seeds: [B] uint64,
+ * device); stream keys mix64(seed + j G), j = 1 initial tokens, 2 Gumbel noise,
+ * 3 re-noising (the exact counters are stated in k_anneal.cuh and oracle/anneal.py). */
+typedef struct dg_anneal_params {
+  int32_t N;      /* maximum denoising steps, 1 .. 65536 (the Report: 48) */
+  float b;        /* mutual-information tolerance, >= 0, not NaN (0.1) */
+  float tau_max;  /* temperature at t = 1, finite > 0 (0.8) */
+  float tau_min;  /* temperature at t = 0, finite > 0 (0.4) */
+  float e_stop;   /* mean-entropy threshold of the adaptive stop, 0 .. 16 (0.005) */
+} dg_anneal_params;
+
+/* The whole annealed block for B = kv's batch canvases without host synchronisation
+ * (a device-controlled loop that ends once every canvas has stopped).
+ * params: host pointer; seeds: [B] uint64 device; canvas_out: [B, C] int32 in [0, V);
+ * n_forwards: [B] int32, the forward count at which each canvas stopped (nullable).
+ * Requires V <= 2^24. */
+dg_status dg_generate_block_annealed(dg_model* m, const dg_kv* kv,
+                                     const dg_anneal_params* params, const uint64_t* seeds,
+                                     int32_t* canvas_out, int32_t* n_forwards, void* stream);
+
+/* Step k's forward alone: canvas [B, C] int32 ids in [0, V); writes the tempered
+ * entropy [B, C] fp32, the argmax [B, C] int32 and the Gumbel-max draw sampled
+ * [B, C] int32.  Requires 0 <= k < N. */
+dg_status dg_anneal_forward(dg_model* m, const dg_kv* kv, const int32_t* canvas, int32_t k,
+                            const dg_anneal_params* params, const uint64_t* seeds,
+                            float* entropy, int32_t* argmax, int32_t* sampled, void* stream);
+
+/* Step k's refinement alone, on caller-provided statistics (entropy, argmax, sampled:
+ * [B, C]).  canvas [B, C] is rewritten; prev_argmax [B, C] holds the previous step's
+ * argmax sequence (read at k > 0) and receives this one; state [B] int32 is 0 while a
+ * canvas runs and becomes k + 1 when it stops (a canvas whose state is not 0 is left
+ * untouched); n_accepted [B] int32 (nullable).  The initial canvas of dg_anneal_init
+ * and state 0 start a block.  Requires 1 <= C <= 1024, 1 <= V <= 2^24, 0 <= k < N. */
+dg_status dg_anneal_sample(const float* entropy, const int32_t* argmax, const int32_t* sampled,
+                           int32_t* canvas, int32_t* prev_argmax, int32_t* state,
+                           int32_t* n_accepted, int32_t B, int32_t C, int32_t V, int32_t k,
+                           const dg_anneal_params* params, const uint64_t* seeds,
+                           void* stream);
+
+/* x_1 of every canvas: canvas [B, C] int32 uniform tokens in [0, V) from stream 1 of
+ * seeds [B]; prev_argmax [B, C] set to -1 and state [B] to 0 (both nullable). */
+dg_status dg_anneal_init(int32_t* canvas, int32_t* prev_argmax, int32_t* state, int32_t B,
+                         int32_t C, int32_t V, const uint64_t* seeds, void* stream);
+
 /* Test hook: the forward of dg_denoise_step without the sampler.  Writes
  * entropy/argmax as above and, when non-NULL, the logits [B*C, V] fp32 and the
  * final residual stream [B*C, d] fp32 (before the final norm). */

@@ -52,6 +52,35 @@ class dg_weights(ctypes.Structure):
 _lib = None
 
 
+class dg_anneal_params(ctypes.Structure):
+    """Constants of the annealed entropy-bounded sampler (defaults: the Report's)."""
+    _fields_ = [("N", ctypes.c_int32), ("b", ctypes.c_float), ("tau_max", ctypes.c_float),
+                ("tau_min", ctypes.c_float), ("e_stop", ctypes.c_float)]
+
+
+def anneal_params(N: int = 48, b: float = 0.1, tau_max: float = 0.8, tau_min: float = 0.4,
+                  e_stop: float = 0.005) -> dg_anneal_params:
+    return dg_anneal_params(N, b, tau_max, tau_min, e_stop)
+
+
+def _params(p) -> dg_anneal_params:
+    if p is None:
+        return anneal_params()
+    if isinstance(p, dg_anneal_params):
+        return p
+    return anneal_params(p.N, p.b, p.tau_max, p.tau_min, p.e_stop)   # any object with the fields
+
+
+def _seeds(seeds, B: int) -> torch.Tensor:
+    """[B] uint64 seeds on the device (int64 storage); ints or a tensor."""
+    if not torch.is_tensor(seeds):
+        seeds = torch.tensor([int(x) - (1 << 64) if int(x) >= (1 << 63) else int(x)
+                              for x in seeds], dtype=torch.int64)
+    if seeds.dtype not in (torch.int64, torch.uint64) or seeds.numel() != B:
+        raise ValueError(f"expected {B} 64-bit seeds")
+    return seeds.reshape(B).to("cuda").contiguous()
+
+
 def lib() -> ctypes.CDLL:
     """Load libdg.so (built in-tree by build.py); raise if it is absent."""
     global _lib
@@ -90,6 +119,13 @@ def lib() -> ctypes.CDLL:
             "dg_op_gemm": [vp, vp, vp, vp, i32, i32, i32, vp],
             "dg_op_moe": [vp, i32, vp, vp, i32, vp],
             "dg_debug_stall_experts": [vp, ctypes.c_int64],
+            "dg_generate_block_annealed": [vp, vp, ctypes.POINTER(dg_anneal_params), vp, vp,
+                                           vp, vp],
+            "dg_anneal_forward": [vp, vp, vp, i32, ctypes.POINTER(dg_anneal_params), vp, vp,
+                                  vp, vp, vp],
+            "dg_anneal_sample": [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32,
+                                 ctypes.POINTER(dg_anneal_params), vp, vp],
+            "dg_anneal_init": [vp, vp, vp, i32, i32, i32, vp, vp],
         }
         for name, args in sigs.items():
             fn = getattr(L, name)
@@ -107,7 +143,8 @@ def exported_symbols():
                         "dg_launch_count", "dg_op_gemm", "dg_op_moe", "dg_expert_units",
                         "dg_lmhead_entropy_noalloc", "dg_block_loop_launches",
                         "dg_debug_stall_experts", "dg_prefill_into", "dg_append_block",
-                        "dg_generate_blocks")
+                        "dg_generate_blocks", "dg_generate_block_annealed",
+                        "dg_anneal_forward", "dg_anneal_sample", "dg_anneal_init")
             if hasattr(lib(), n)]
 
 
@@ -289,6 +326,59 @@ def dg_eb_sample(entropy, argmax, canvas, mask, steps_left: int, gamma: float,
     _check(lib().dg_eb_sample(_ptr(entropy), _ptr(argmax), _ptr(canvas), _ptr(mask), B, C,
                               steps_left, gamma, _ptr(n_committed), _stream(stream)))
     return n_committed
+
+
+def dg_generate_block_annealed(model: Model, kv: KV, seeds, params=None, canvas_out=None,
+                               n_forwards=None, stream=None):
+    """The annealed block; returns (canvas [B, C] int32, n_forwards [B] int32)."""
+    c = model.cfg
+    p = _params(params)
+    sd = _seeds(seeds, kv.B)
+    canvas_out = (canvas_out if canvas_out is not None
+                  else torch.empty(kv.B, c.canvas, dtype=torch.int32, device="cuda"))
+    n_forwards = (n_forwards if n_forwards is not None
+                  else torch.empty(kv.B, dtype=torch.int32, device="cuda"))
+    _check(lib().dg_generate_block_annealed(model.handle, kv.handle, ctypes.byref(p), _ptr(sd),
+                                            _ptr(canvas_out), _ptr(n_forwards),
+                                            _stream(stream)))
+    return canvas_out, n_forwards
+
+
+def dg_anneal_forward(model: Model, kv: KV, canvas, k: int, seeds, params=None, stream=None):
+    """Step k's forward: (tempered entropy [B, C], argmax [B, C], Gumbel-max draw [B, C])."""
+    p = _params(params)
+    sd = _seeds(seeds, kv.B)
+    B, C = canvas.shape
+    H = torch.empty(B, C, dtype=torch.float32, device="cuda")
+    am = torch.empty(B, C, dtype=torch.int32, device="cuda")
+    smp = torch.empty(B, C, dtype=torch.int32, device="cuda")
+    _check(lib().dg_anneal_forward(model.handle, kv.handle, _ptr(canvas), k, ctypes.byref(p),
+                                   _ptr(sd), _ptr(H), _ptr(am), _ptr(smp), _stream(stream)))
+    return H, am, smp
+
+
+def dg_anneal_sample(entropy, argmax, sampled, canvas, prev_argmax, state, k: int, V: int,
+                     seeds, params=None, stream=None):
+    """Step k's refinement in place (canvas, prev_argmax, state); returns n_accepted [B]."""
+    p = _params(params)
+    B, C = entropy.shape
+    sd = _seeds(seeds, B)
+    nacc = torch.empty(B, dtype=torch.int32, device="cuda")
+    _check(lib().dg_anneal_sample(_ptr(entropy), _ptr(argmax), _ptr(sampled), _ptr(canvas),
+                                  _ptr(prev_argmax), _ptr(state), _ptr(nacc), B, C, V, k,
+                                  ctypes.byref(p), _ptr(sd), _stream(stream)))
+    return nacc
+
+
+def dg_anneal_init(B: int, C: int, V: int, seeds, stream=None):
+    """(x_1 [B, C] int32, prev_argmax [B, C] = -1, state [B] = 0)."""
+    sd = _seeds(seeds, B)
+    canvas = torch.empty(B, C, dtype=torch.int32, device="cuda")
+    prev = torch.empty(B, C, dtype=torch.int32, device="cuda")
+    state = torch.empty(B, dtype=torch.int32, device="cuda")
+    _check(lib().dg_anneal_init(_ptr(canvas), _ptr(prev), _ptr(state), B, C, V, _ptr(sd),
+                                _stream(stream)))
+    return canvas, prev, state
 
 
 def dg_debug_forward(model: Model, kv: KV, canvas, steps_left: int, T: int, logits=False,

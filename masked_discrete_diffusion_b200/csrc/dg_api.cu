@@ -163,6 +163,10 @@ template <class Path> static dg_status alloc_workspace(dg_model* m) {
   DG_TRY(ws_alloc(ws, &ws.remaining, c.max_batch));
   DG_TRY(ws_alloc(ws, &ws.loop_s, 1));
   DG_TRY(ws_alloc(ws, &ws.blk, lm_rows));
+  DG_TRY(ws_alloc(ws, &ws.sampled, lm_rows));
+  DG_TRY(ws_alloc(ws, &ws.prev, lm_rows));
+  DG_TRY(ws_alloc(ws, &ws.astate, c.max_batch));
+  DG_TRY(ws_alloc_v<Acc>(ws, &ws.gpart, (size_t)ws.n_vtiles * lm_rows * 2));
   DG_TRY_CUDA(cudaMemset(ws.err, 0, 4 * sizeof(int32_t)));
   launch_pdl((rope_table_kernel), 256, 256, 0, cudaStream_t(0), 1, (double)c.rope_base, (int)h, ws.max_pos, ws.rope,
                                   sizeof(Acc) == 8 ? 1 : 0);
@@ -527,8 +531,10 @@ template <class Path> struct Runner {
   }
 
   // Canvas forward: statistics into ent/amax; optional logits/hidden (test hook).
+  // With an.N > 0: tempered statistics and (an.seeds) the Gumbel-max draw into sampled.
   dg_status forward(const dg_kv* kv, const int32_t* canvas, int s, int T, float* ent,
-                    int32_t* amax, float* logits, float* hidden, int32_t* load) {
+                    int32_t* amax, float* logits, float* hidden, int32_t* load,
+                    const AnnealDev& an = AnnealDev{}, int32_t* sampled = nullptr) {
     const int B = kv->B, C = c.canvas, n = B * C, d = c.d_model;
     const double tau = (double)s / (double)T;
     {
@@ -552,7 +558,7 @@ template <class Path> struct Runner {
     bool done = false;
     if constexpr (Path::kTensorCores) {
       if (logits == nullptr) {
-        DG_TRY(tc_lmhead_stats(m, xn(), n, ent, amax, st));
+        DG_TRY(tc_lmhead_stats(m, xn(), n, ent, amax, st, an, sampled));
         done = true;
       }
     }
@@ -560,10 +566,12 @@ template <class Path> struct Runner {
       dim3 grid(ws.n_vtiles, ceil_div(n, SG_BM));
       launch_pdl((lmhead_simt_kernel<TA, TW, Acc>), grid, 256, 0, st, 1, xn(), (const TW*)m->w.lm_head, n,
                                                            c.vocab, d, c.logit_scale,
-                                                           (Acc*)ws.lm_part, logits);
+                                                           (Acc*)ws.lm_part, logits, an);
       ++m->launches;
       launch_pdl((lm_merge_kernel<Acc>), n, 128, 0, st, 1, (const Acc*)ws.lm_part, ws.n_vtiles,
-                                                          n, ent, amax);
+                                                          n, ent, amax,
+                                                          (const Acc*)(an.seeds ? an.gpart : nullptr),
+                                                          an.seeds ? sampled : nullptr);
       ++m->launches;
     }
     return check_launch("forward");
@@ -857,10 +865,13 @@ static dg_status check_step_args(dg_model* m, const dg_kv* kv, int s, int T) {
 
 static dg_status run_forward(dg_model* m, const dg_kv* kv, const int32_t* canvas, int s, int T,
                              float* ent, int32_t* am, float* logits, float* hidden,
-                             int32_t* load, cudaStream_t st, const int32_t* s_dev = nullptr) {
+                             int32_t* load, cudaStream_t st, const int32_t* s_dev = nullptr,
+                             const AnnealDev& an = AnnealDev{}, int32_t* sampled = nullptr) {
   return m->cfg.dtype == DG_F32
-             ? Runner<PathTiny>(m, st, s_dev).forward(kv, canvas, s, T, ent, am, logits, hidden, load)
-             : Runner<PathBF16>(m, st, s_dev).forward(kv, canvas, s, T, ent, am, logits, hidden, load);
+             ? Runner<PathTiny>(m, st, s_dev).forward(kv, canvas, s, T, ent, am, logits, hidden,
+                                                      load, an, sampled)
+             : Runner<PathBF16>(m, st, s_dev).forward(kv, canvas, s, T, ent, am, logits, hidden,
+                                                      load, an, sampled);
 }
 
 dg_status dg_denoise_step(dg_model* m, const dg_kv* kv, int32_t* canvas, uint8_t* mask,
@@ -905,17 +916,16 @@ static dg_status generate_impl(dg_model* m, const dg_kv* kv, int32_t T, long lon
 
 static dg_status replay(dg_model* m, dg::BlockGraph* g, cudaStream_t st);
 
-// Builds the block as a graph with a device-controlled loop: an init kernel, then a
-// WHILE node whose body is one forward + sampler step + a control kernel that
-// decrements the device-side steps-left counter and stops the loop once the
-// counter reaches 0 or no canvas has a masked position left (the oracle's early
-// stop).  Returns false (nothing built) if this CUDA build refuses a step.
-static bool build_loop_graph(dg_model* m, const dg_kv* kv, int32_t T, long long gq,
-                             int32_t* canvas_out, int32_t* n_forwards, int32_t* router_load,
-                             dg::BlockGraph* g) {
-  const dg_config& c = m->cfg;
+// Builds a block as a graph with a device-controlled loop: init(stream) captured first,
+// then a WHILE node whose body is body(stream) (one forward + sampler step) followed by
+// a control kernel that decrements the device-side steps-left counter and stops the
+// loop once it reaches 0 or no canvas of the batch is still running (remaining[b] > 0
+// marks a running canvas).  Returns false (nothing built) if this CUDA build refuses a
+// step.
+extern "C++" {
+template <class Init, class Body>
+static bool build_while_graph(dg_model* m, int B, dg::BlockGraph* g, Init&& init, Body&& body) {
   Workspace& ws = m->ws;
-  const int B = kv->B, C = c.canvas;
   cudaStream_t cap = m->cap_stream;
   cudaGraph_t graph = nullptr;
   if (cudaGraphCreate(&graph, 0) != cudaSuccess) return false;
@@ -928,9 +938,7 @@ static bool build_loop_graph(dg_model* m, const dg_kv* kv, int32_t T, long long 
     if (cudaStreamBeginCaptureToGraph(cap, graph, nullptr, nullptr, 0,
                                       cudaStreamCaptureModeThreadLocal) != cudaSuccess)
       break;
-    const int n = B * C, n_load = router_load ? c.n_layers * c.n_experts : 0;
-    launch_pdl((block_init_kernel), ceil_div(std::max(n, n_load), 256), 256, 0, cap, 1, canvas_out,
-               ws.mask, n, (int32_t)c.vocab, n_forwards, B, router_load, n_load, ws.loop_s, T);
+    init(cap);
     cudaGraph_t g1 = nullptr;
     if (cudaStreamEndCapture(cap, &g1) != cudaSuccess) break;
     size_t nn = 0;
@@ -944,16 +952,12 @@ static bool build_loop_graph(dg_model* m, const dg_kv* kv, int32_t T, long long 
     cp.conditional.size = 1;
     cudaGraphNode_t cnode;
     if (cudaGraphAddNode(&cnode, graph, nodes.data(), nn, &cp) != cudaSuccess) break;
-    cudaGraph_t body = cp.conditional.phGraph_out[0];
-    if (cudaStreamBeginCaptureToGraph(cap, body, nullptr, nullptr, 0,
+    cudaGraph_t bodyg = cp.conditional.phGraph_out[0];
+    if (cudaStreamBeginCaptureToGraph(cap, bodyg, nullptr, nullptr, 0,
                                       cudaStreamCaptureModeThreadLocal) != cudaSuccess)
       break;
     const long long l0 = m->launches;
-    dg_status s = run_forward(m, kv, canvas_out, T, T, ws.ent, ws.amax, nullptr, nullptr,
-                              router_load, cap, ws.loop_s);
-    if (s == DG_OK)
-      s = launch_sampler(ws.ent, ws.amax, canvas_out, ws.mask, B, C, T, gq, ws.ncommit,
-                         n_forwards, 1, cap, &m->launches, ws.loop_s, T, ws.remaining);
+    const dg_status s = body(cap);
     launch_pdl((block_step_kernel), 1, 32, 0, cap, 1, handle, ws.loop_s,
                (const int32_t*)ws.remaining, B);
     g->body_launches = m->launches - l0 + 1;
@@ -974,6 +978,33 @@ static bool build_loop_graph(dg_model* m, const dg_kv* kv, int32_t T, long long 
   }
   return ok;
 }
+}  // extern "C++"
+
+// The Entropy-Bound block: init kernel (all [MASK], steps left T), body = forward at
+// the device's steps-left + EB sampler step (remaining[b] = masked positions left).
+static bool build_loop_graph(dg_model* m, const dg_kv* kv, int32_t T, long long gq,
+                             int32_t* canvas_out, int32_t* n_forwards, int32_t* router_load,
+                             dg::BlockGraph* g) {
+  const dg_config& c = m->cfg;
+  Workspace& ws = m->ws;
+  const int B = kv->B, C = c.canvas;
+  const int n = B * C, n_load = router_load ? c.n_layers * c.n_experts : 0;
+  return build_while_graph(
+      m, B, g,
+      [&](cudaStream_t cap) {
+        launch_pdl((block_init_kernel), ceil_div(std::max(n, n_load), 256), 256, 0, cap, 1,
+                   canvas_out, ws.mask, n, (int32_t)c.vocab, n_forwards, B, router_load, n_load,
+                   ws.loop_s, T);
+      },
+      [&](cudaStream_t cap) {
+        dg_status s = run_forward(m, kv, canvas_out, T, T, ws.ent, ws.amax, nullptr, nullptr,
+                                  router_load, cap, ws.loop_s);
+        if (s == DG_OK)
+          s = launch_sampler(ws.ent, ws.amax, canvas_out, ws.mask, B, C, T, gq, ws.ncommit,
+                             n_forwards, 1, cap, &m->launches, ws.loop_s, T, ws.remaining);
+        return s;
+      });
+}
 
 // Captures the block's launch sequence once per (kv, T, gamma, output buffers,
 // profiling) and replays it: one host call per block instead of ~500 launches per
@@ -984,7 +1015,8 @@ static dg_status generate_graphed(dg_model* m, const dg_kv* kv, int32_t T, long 
                                   int32_t* router_load, cudaStream_t st) {
   dg::BlockGraph* g = nullptr;
   for (auto* x : m->graphs)
-    if (x->kv == kv && x->kv_P == kv->P && x->kv_W == kv->W && x->T == T && x->gq == gq &&
+    if (!x->anneal && x->kv == kv && x->kv_P == kv->P && x->kv_W == kv->W && x->T == T &&
+        x->gq == gq &&
         x->canvas == canvas_out &&
         x->nfwd == n_forwards && x->load == router_load && x->prof == m->profiling &&
         (!x->prof || x->fcap == m->prof_forwards)) {
@@ -1112,6 +1144,214 @@ dg_status dg_generate_blocks(dg_model* m, dg_kv* kv, int32_t n_blocks, int32_t T
     if (k + 1 < n_blocks) DG_TRY(dg_append_block(m, kv, m->ws.blk, stream));
   }
   return DG_OK;
+}
+
+// ---------------------------------------------------------------------------
+// The Report's default sampler: annealed entropy-bounded refinement over a
+// uniform-noise canvas (k_anneal.cuh states the rule and the readings).
+// ---------------------------------------------------------------------------
+struct AnnealQ {
+  unsigned long long bq = 0, eq = 0;  // min(floor(b 2^48), 2^62), floor(e_stop 2^48)
+};
+
+static dg_status anneal_check(const dg_anneal_params* p, int V, AnnealQ* q) {
+  DG_REQUIRE(p, "null params");
+  DG_REQUIRE(p->N >= 1 && p->N <= 65536, "N=%d outside [1, 65536]", p->N);
+  DG_REQUIRE(!std::isnan(p->b) && p->b >= 0.0f, "b must be >= 0 and not NaN (got %g)",
+             (double)p->b);
+  DG_REQUIRE(std::isfinite(p->tau_max) && p->tau_max > 0.0f && std::isfinite(p->tau_min) &&
+                 p->tau_min > 0.0f,
+             "temperatures must be finite and > 0 (got %g, %g)", (double)p->tau_max,
+             (double)p->tau_min);
+  DG_REQUIRE(p->e_stop >= 0.0f && p->e_stop <= 16.0f, "e_stop outside [0, 16] (got %g)",
+             (double)p->e_stop);
+  DG_REQUIRE(V >= 1 && V <= (1 << 24), "V=%d outside [1, 2^24]", V);
+  const double two48 = 281474976710656.0, cap = 4611686018427387904.0;  // 2^48, 2^62
+  const double bv = std::isinf(p->b) ? cap : std::floor((double)p->b * two48);
+  q->bq = bv >= cap ? (1ull << 62) : (unsigned long long)bv;
+  q->eq = (unsigned long long)std::floor((double)p->e_stop * two48);
+  return DG_OK;
+}
+
+static AnnealDev anneal_dev(dg_model* m, const dg_anneal_params* p, const uint64_t* seeds,
+                            int s, const int32_t* s_dev) {
+  AnnealDev a;
+  a.seeds = (const unsigned long long*)seeds;
+  a.s_dev = s_dev;
+  a.s = s;
+  a.N = p->N;
+  a.C = m->cfg.canvas;
+  a.tau_max = p->tau_max;
+  a.tau_min = p->tau_min;
+  a.gpart = m->ws.gpart;
+  return a;
+}
+
+static dg_status launch_anneal(const float* H, const int32_t* am, const int32_t* sampled,
+                               int32_t* canvas, int32_t* prev, int32_t* state, int32_t* nfwd,
+                               int32_t* nacc, int32_t* remaining, int B, int C, int V, int k,
+                               const int32_t* s_dev, int N, const AnnealQ& q,
+                               const uint64_t* seeds, cudaStream_t st, long long* counter) {
+  const unsigned long long* sd = (const unsigned long long*)seeds;
+#define DG_ANN(NP)                                                                          \
+  launch_pdl((anneal_sample_kernel<NP>), B, NP, 0, st, 1, H, am, sampled, canvas, prev, state, \
+             nfwd, nacc, remaining, C, V, k, s_dev, N, q.bq, q.eq, sd)
+  if (C <= 32) DG_ANN(32);
+  else if (C <= 64) DG_ANN(64);
+  else if (C <= 128) DG_ANN(128);
+  else if (C <= 256) DG_ANN(256);
+  else if (C <= 512) DG_ANN(512);
+  else DG_ANN(1024);
+#undef DG_ANN
+  if (counter) ++*counter;
+  return check_launch("annealed sampler");
+}
+
+// The annealed block as plain launches: N forwards (min(fcap, N) when profiling); a
+// canvas that has stopped is left alone by the later sampler steps.
+static dg_status anneal_impl(dg_model* m, const dg_kv* kv, const dg_anneal_params* p,
+                             const AnnealQ& q, const uint64_t* seeds, int32_t* canvas_out,
+                             int32_t* n_forwards, cudaStream_t st, int fcap) {
+  const dg_config& c = m->cfg;
+  Workspace& ws = m->ws;
+  const int B = kv->B, C = c.canvas, V = c.vocab;
+  {
+    ProfScope ps(m, DG_KIND_GLUE, st);
+    launch_pdl((anneal_init_kernel), ceil_div((long)B * C, 256), 256, 0, st, 1, canvas_out,
+               ws.prev, ws.astate, n_forwards, B, C, V, (const unsigned long long*)seeds,
+               (int32_t*)nullptr, p->N);
+    ++m->launches;
+  }
+  const int nfw = fcap > 0 ? std::min(fcap, (int)p->N) : (int)p->N;
+  for (int k = 0; k < nfw; ++k) {
+    const int s = p->N - k;
+    DG_TRY(run_forward(m, kv, canvas_out, s, p->N, ws.ent, ws.amax, nullptr, nullptr, nullptr,
+                       st, nullptr, anneal_dev(m, p, seeds, s, nullptr), ws.sampled));
+    ProfScope ps(m, DG_KIND_GLUE, st);
+    DG_TRY(launch_anneal(ws.ent, ws.amax, ws.sampled, canvas_out, ws.prev, ws.astate, n_forwards,
+                         ws.ncommit, (int32_t*)nullptr, B, C, V, k, (const int32_t*)nullptr,
+                         p->N, q, seeds, st, &m->launches));
+  }
+  return DG_OK;
+}
+
+// The annealed block as a device-controlled loop (see build_while_graph).
+static bool build_anneal_graph(dg_model* m, const dg_kv* kv, const dg_anneal_params* p,
+                               const AnnealQ& q, const uint64_t* seeds, int32_t* canvas_out,
+                               int32_t* n_forwards, dg::BlockGraph* g) {
+  const dg_config& c = m->cfg;
+  Workspace& ws = m->ws;
+  const int B = kv->B, C = c.canvas, V = c.vocab, N = p->N;
+  return build_while_graph(
+      m, B, g,
+      [&](cudaStream_t cap) {
+        launch_pdl((anneal_init_kernel), ceil_div((long)B * C, 256), 256, 0, cap, 1, canvas_out,
+                   ws.prev, ws.astate, n_forwards, B, C, V, (const unsigned long long*)seeds,
+                   ws.loop_s, N);
+      },
+      [&](cudaStream_t cap) {
+        dg_status s = run_forward(m, kv, canvas_out, N, N, ws.ent, ws.amax, nullptr, nullptr,
+                                  nullptr, cap, ws.loop_s, anneal_dev(m, p, seeds, N, ws.loop_s),
+                                  ws.sampled);
+        if (s == DG_OK)
+          s = launch_anneal(ws.ent, ws.amax, ws.sampled, canvas_out, ws.prev, ws.astate,
+                            n_forwards, ws.ncommit, ws.remaining, B, C, V, 0, ws.loop_s, N, q,
+                            seeds, cap, &m->launches);
+        return s;
+      });
+}
+
+dg_status dg_generate_block_annealed(dg_model* m, const dg_kv* kv, const dg_anneal_params* p,
+                                     const uint64_t* seeds, int32_t* canvas_out,
+                                     int32_t* n_forwards, void* stream) {
+  g_err.clear();
+  DG_TRY(check_step_args(m, kv, 1, 1));
+  DG_REQUIRE(seeds && canvas_out, "null argument");
+  AnnealQ q;
+  DG_TRY(anneal_check(p, m->cfg.vocab, &q));
+  DG_REQUIRE(m->cfg.canvas <= 1024, "canvas %d > 1024", m->cfg.canvas);
+  cudaStream_t st = (cudaStream_t)stream;
+  if (!m->use_graphs || m->profiling)
+    return anneal_impl(m, kv, p, q, seeds, canvas_out, n_forwards, st,
+                       m->profiling ? m->prof_forwards : 0);
+  dg::BlockGraph* g = nullptr;
+  for (auto* x : m->graphs)
+    if (x->anneal && x->kv == kv && x->kv_P == kv->P && x->kv_W == kv->W && x->aN == p->N &&
+        x->ab == p->b && x->atmax == p->tau_max && x->atmin == p->tau_min &&
+        x->aestop == p->e_stop && x->seeds == seeds && x->canvas == canvas_out &&
+        x->nfwd == n_forwards) {
+      g = x;
+      break;
+    }
+  if (!g) {
+    if (m->graphs.size() >= 8) {
+      graph_free(m->graphs.front());
+      m->graphs.erase(m->graphs.begin());
+    }
+    g = new dg::BlockGraph();
+    g->anneal = true;
+    g->kv = kv;
+    g->kv_P = kv->P;
+    g->kv_W = kv->W;
+    g->aN = p->N;
+    g->ab = p->b;
+    g->atmax = p->tau_max;
+    g->atmin = p->tau_min;
+    g->aestop = p->e_stop;
+    g->seeds = seeds;
+    g->canvas = canvas_out;
+    g->nfwd = n_forwards;
+    if (!m->cap_stream) DG_TRY_CUDA(cudaStreamCreateWithFlags(&m->cap_stream, cudaStreamNonBlocking));
+    if (!build_anneal_graph(m, kv, p, q, seeds, canvas_out, n_forwards, g)) {
+      graph_free(g);
+      return anneal_impl(m, kv, p, q, seeds, canvas_out, n_forwards, st, 0);
+    }
+    m->graphs.push_back(g);
+  }
+  return replay(m, g, st);
+}
+
+dg_status dg_anneal_forward(dg_model* m, const dg_kv* kv, const int32_t* canvas, int32_t k,
+                            const dg_anneal_params* p, const uint64_t* seeds, float* entropy,
+                            int32_t* argmax, int32_t* sampled, void* stream) {
+  g_err.clear();
+  DG_REQUIRE(canvas && seeds && entropy && argmax && sampled, "null argument");
+  AnnealQ q;
+  DG_REQUIRE(m, "null model");
+  DG_TRY(anneal_check(p, m->cfg.vocab, &q));
+  DG_REQUIRE(k >= 0 && k < p->N, "k=%d outside [0, N=%d)", k, p->N);
+  DG_TRY(check_step_args(m, kv, p->N - k, p->N));
+  return run_forward(m, kv, canvas, p->N - k, p->N, entropy, argmax, nullptr, nullptr, nullptr,
+                     (cudaStream_t)stream, nullptr, anneal_dev(m, p, seeds, p->N - k, nullptr),
+                     sampled);
+}
+
+dg_status dg_anneal_sample(const float* entropy, const int32_t* argmax, const int32_t* sampled,
+                           int32_t* canvas, int32_t* prev_argmax, int32_t* state,
+                           int32_t* n_accepted, int32_t B, int32_t C, int32_t V, int32_t k,
+                           const dg_anneal_params* p, const uint64_t* seeds, void* stream) {
+  g_err.clear();
+  DG_REQUIRE(entropy && argmax && sampled && canvas && prev_argmax && state && seeds,
+             "null argument");
+  DG_REQUIRE(B >= 1 && C >= 1 && C <= 1024, "need B >= 1 and 1 <= C <= 1024");
+  AnnealQ q;
+  DG_TRY(anneal_check(p, V, &q));
+  DG_REQUIRE(k >= 0 && k < p->N, "k=%d outside [0, N=%d)", k, p->N);
+  return launch_anneal(entropy, argmax, sampled, canvas, prev_argmax, state, (int32_t*)nullptr,
+                       n_accepted, (int32_t*)nullptr, B, C, V, k, (const int32_t*)nullptr, p->N,
+                       q, seeds, (cudaStream_t)stream, nullptr);
+}
+
+dg_status dg_anneal_init(int32_t* canvas, int32_t* prev_argmax, int32_t* state, int32_t B,
+                         int32_t C, int32_t V, const uint64_t* seeds, void* stream) {
+  g_err.clear();
+  DG_REQUIRE(canvas && seeds, "null argument");
+  DG_REQUIRE(B >= 1 && C >= 1 && (long long)B * C <= (1LL << 30), "bad B=%d, C=%d", B, C);
+  DG_REQUIRE(V >= 1 && V <= (1 << 24), "V=%d outside [1, 2^24]", V);
+  launch_pdl((anneal_init_kernel), ceil_div((long)B * C, 256), 256, 0, (cudaStream_t)stream, 1,
+             canvas, prev_argmax, state, (int32_t*)nullptr, B, C, V,
+             (const unsigned long long*)seeds, (int32_t*)nullptr, 1);
+  return check_launch("anneal init");
 }
 
 dg_status dg_eb_sample(const float* entropy, const int32_t* argmax, int32_t* canvas,

@@ -110,6 +110,10 @@ struct Workspace {
   int32_t *amax = nullptr, *ncommit = nullptr;      // [max_batch, C], [max_batch]
   int32_t *remaining = nullptr, *loop_s = nullptr;  // [max_batch] masked left; steps left
   int32_t* blk = nullptr;                           // [max_batch, C] a finished block
+  // annealed sampler: Gumbel-max draws [max_batch, C], previous argmax [max_batch, C],
+  // per-canvas stop state [max_batch], per-tile race winners [n_vtiles, max_batch C, 2]
+  int32_t *sampled = nullptr, *prev = nullptr, *astate = nullptr;
+  void* gpart = nullptr;
   int max_pos = 0;
   size_t kc_elems = 0;
   int max_tiles = 0;
@@ -129,6 +133,11 @@ struct BlockGraph {
   int32_t *canvas = nullptr, *nfwd = nullptr, *load = nullptr;
   bool prof = false;
   int fcap = 0;            // forwards of a profiled (unrolled) block, 0: T
+  // annealed block: its constants and seeds (anneal false: the Entropy-Bound block)
+  bool anneal = false;
+  int aN = 0;
+  float ab = 0.f, atmax = 0.f, atmin = 0.f, aestop = 0.f;
+  const void* seeds = nullptr;
   long long launches = 0;  // kernel launches the graph replays (1 for a loop graph: the init)
   bool loop = false;       // device-controlled WHILE loop over forwards
   long long body_launches = 0;  // kernels per loop iteration (forward + sampler + control)

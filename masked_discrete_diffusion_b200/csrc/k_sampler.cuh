@@ -43,7 +43,7 @@ __global__ void __launch_bounds__(NP)
     step_no = T - steps_left + 1;
   }
   __shared__ unsigned long long key[NP];
-  __shared__ long long pre[NP];
+  __shared__ unsigned long long pre[NP];
   __shared__ int cnt[NP / 32];
   const int b = blockIdx.x, i = threadIdx.x;
   const size_t base = (size_t)b * C;
@@ -74,19 +74,23 @@ __global__ void __launch_bounds__(NP)
       __syncthreads();
     }
   }
-  // inclusive prefix sum of the fixed-point entropies of the first m entries
-  long long q = 0;
-  if (i < m) q = eb_q48(__uint_as_float((unsigned)(key[i] >> 32)));
-  pre[i] = q;
+  // inclusive prefix sum of the fixed-point entropies of the first m entries, saturating
+  // at gamma_q + 1 (gamma_q <= 2^62: two saturated terms never wrap, and "<= gamma_q"
+  // is decided exactly however many capped entropies the canvas holds)
+  const unsigned long long cap = (unsigned long long)gamma_q + 1;
+  unsigned long long q = 0;
+  if (i < m) q = (unsigned long long)eb_q48(__uint_as_float((unsigned)(key[i] >> 32)));
+  pre[i] = q < cap ? q : cap;
   __syncthreads();
   for (int off = 1; off < NP; off <<= 1) {
-    const long long add = i >= off ? pre[i - off] : 0;
+    const unsigned long long add = i >= off ? pre[i - off] : 0;
     __syncthreads();
-    pre[i] += add;
+    const unsigned long long v = pre[i] + add;
+    pre[i] = v < cap ? v : cap;
     __syncthreads();
   }
   // k_gamma = number of prefixes within the bound (prefix sums are non-decreasing)
-  const int within = (i < m && pre[i] <= gamma_q) ? 1 : 0;
+  const int within = (i < m && pre[i] <= (unsigned long long)gamma_q) ? 1 : 0;
   const unsigned bw = __ballot_sync(0xffffffffu, within);
   __syncthreads();
   if ((i & 31) == 0) cnt[i >> 5] = __popc(bw);

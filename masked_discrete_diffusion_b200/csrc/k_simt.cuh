@@ -10,6 +10,7 @@
 // plus one shared expert, sliding window 1024, timestep embedding).
 #pragma once
 
+#include "k_anneal.cuh"
 #include "k_common.cuh"
 
 namespace dg {
@@ -675,13 +676,17 @@ __global__ void moe_combine_norm_kernel(TR* __restrict__ x, const TY* __restrict
 // entries, reduced per row to partial statistics over the tile:
 //   m = max logit, s = sum exp(l - m), u = sum exp(l - m) (l - m), a = argmax
 // (lowest id among equal maxima).  Partials: [n_vtiles, n_rows, 4].
-// Optional logits output [n_rows, V] (test hook).
+// Optional logits output [n_rows, V] (test hook).  With an.N > 0 the logits are
+// tempered (l = scale acc / tau) and, with an.seeds, each row's winner of the tile's
+// Gumbel-max race goes to an.gpart [n_vtiles, n_rows, 2] = (l / tau - log E, id).
 // ---------------------------------------------------------------------------
 template <class TA, class TW, class Acc>
 __global__ void __launch_bounds__(256)
     lmhead_simt_kernel(const TA* __restrict__ xn, const TW* __restrict__ wlm, int n_rows, int V,
-                       int d, float scale, Acc* __restrict__ part, float* __restrict__ logits) {
+                       int d, float scale, Acc* __restrict__ part, float* __restrict__ logits,
+                       AnnealDev an) {
   pdl_enter();
+  const Acc tau = an.N > 0 ? (Acc)an.tau() : Acc(1);
   // the logits tile T reuses the operand staging buffers once the K loop is done
   constexpr int kStage = 2 * SG_BK * (SG_BM + 1), kTile = SG_BM * (SG_BN + 1);
   __shared__ Acc smem[kStage > kTile ? kStage : kTile];
@@ -722,7 +727,8 @@ __global__ void __launch_bounds__(256)
   for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const Acc l = (Acc)scale * acc[i][j];
+      Acc l = (Acc)scale * acc[i][j];
+      if (an.N > 0) l = l / tau;
       T[ty + 16 * i][tx + 16 * j] = l;
       const int r = m0 + ty + 16 * i, c = n0 + tx + 16 * j;
       if (logits && r < n_rows && c < V) logits[(size_t)r * V + c] = (float)l;
@@ -767,6 +773,29 @@ __global__ void __launch_bounds__(256)
       pp[2] = u;
       pp[3] = (Acc)am;
     }
+    if (an.seeds) {  // this tile's winner of the race, lane by lane then across the warp
+      GumbelBest<Acc> gb;
+      const unsigned long long st = an.state0(r, V, n0);
+      for (int c = lane; c < SG_BN; c += 32) {
+        if (n0 + c >= V) continue;
+        const Acc z = T[rr][c] - mx;
+        gb.offer(dexp(z), (Acc)sm64_expo(sm64_mix(st + (unsigned long long)c * SM64_G), Acc(0)),
+                 z, n0 + c);
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const Acc oe = __shfl_xor_sync(0xffffffffu, gb.e, off);
+        const Acc oE = __shfl_xor_sync(0xffffffffu, gb.E, off);
+        const Acc oz = __shfl_xor_sync(0xffffffffu, gb.z, off);
+        const int oi = __shfl_xor_sync(0xffffffffu, gb.id, off);
+        gb.offer(oe, oE, oz, oi);
+      }
+      if (lane == 0) {
+        Acc* gp = reinterpret_cast<Acc*>(an.gpart) + ((size_t)blockIdx.x * n_rows + r) * 2;
+        gp[0] = gb.value(mx);
+        gp[1] = (Acc)gb.id;
+      }
+    }
   }
 }
 
@@ -774,10 +803,12 @@ __global__ void __launch_bounds__(256)
 //   M = max m_i, S = sum s_i e^(m_i - M),
 //   H = log S - (1/S) sum e^(m_i - M) (u_i + (m_i - M) s_i)   (clamped at 0),
 //   argmax = the id of the first tile (lowest vocab) attaining M.
+//   sampled (with gpart) = the id of the best (value, lowest id) race winner over tiles.
 template <class Acc>
 __global__ void __launch_bounds__(128)
     lm_merge_kernel(const Acc* __restrict__ part, int n_vt, int n_rows, float* __restrict__ H,
-                    int32_t* __restrict__ amax) {
+                    int32_t* __restrict__ amax, const Acc* __restrict__ gpart,
+                    int32_t* __restrict__ sampled) {
   // one block per row; the tiles are split over the threads, each thread merges
   // its tiles online (running max M_t; S and U rescaled when M_t rises), then the
   // block merges the threads in a fixed order
@@ -866,6 +897,45 @@ __global__ void __launch_bounds__(128)
       if (!(h > Acc(0))) h = 0;
       H[r] = (float)h;
       amax[r] = (int32_t)i2;
+    }
+  }
+  if (gpart) {  // (value, id) is a total order (ids are distinct): any merge order agrees
+    __syncthreads();
+    Acc bv = -INFINITY;
+    int bi = 0x7fffffff;
+    for (int i = tid; i < n_vt; i += blockDim.x) {
+      const Acc* g = gpart + ((size_t)i * n_rows + r) * 2;
+      const Acc v = g[0];
+      const int id = (int)g[1];
+      if (v > bv || (v == bv && id < bi)) {
+        bv = v;
+        bi = id;
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const Acc ov = __shfl_xor_sync(0xffffffffu, bv, off);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+      if (ov > bv || (ov == bv && oi < bi)) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    if ((tid & 31) == 0) {
+      sm_m[tid >> 5] = bv;
+      sm_i[tid >> 5] = (Acc)bi;
+    }
+    __syncthreads();
+    if (tid == 0) {
+      for (int w = 1; w < (int)(blockDim.x >> 5); ++w) {
+        const Acc ov = sm_m[w];
+        const int oi = (int)sm_i[w];
+        if (ov > bv || (ov == bv && oi < bi)) {
+          bv = ov;
+          bi = oi;
+        }
+      }
+      sampled[r] = bi;
     }
   }
 }

@@ -21,6 +21,7 @@
 #include <unordered_map>
 
 #include "dg_internal.h"
+#include "k_anneal.cuh"
 #include "k_common.cuh"
 #include "tc_ptx.cuh"
 
@@ -371,14 +372,19 @@ struct EpiRouterTopk {
 // Per-row statistics of logits l = scale * acc over this CTA's vocabulary tile
 // (columns n0 .. n0 + 32 NCH - 1, those < N): m = max, s = sum exp(l - m),
 // u = sum exp(l - m) (l - m), a = lowest id attaining m.  part[(tile, row)] = (m, s, u, a).
+// With an.N > 0 the logits are tempered (l = scale acc / tau) and, with an.seeds, the
+// tile's winner of the Gumbel-max race goes to an.gpart[(tile, row)] = (l / tau - log E,
+// id).
 struct EpiLmStats {
   static constexpr bool kStaged = false, kWarpRows = false;
   static constexpr size_t kExtraSmem = 0;
   float* part;
   int M, N;
   float scale;
+  AnnealDev an = {};
   template <int NCH, class Ld>
   __device__ void run(int row, bool valid, int n0, Ld&& ld) const {
+    const float scale = an.N > 0 ? (float)((double)this->scale / an.tau()) : this->scale;
     float mx = -INFINITY;
     int am = 0x7fffffff;
 #pragma unroll 1
@@ -396,24 +402,46 @@ struct EpiLmStats {
       }
     }
     float s = 0.f, u = 0.f;
+    const int tile = n0 / (NCH * 32);
+    if (an.seeds == nullptr) {
 #pragma unroll 1
-    for (int c = 0; c < NCH; ++c) {
-      float v[32];
-      ld(0, c, v);
+      for (int c = 0; c < NCH; ++c) {
+        float v[32];
+        ld(0, c, v);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const int col = n0 + c * 32 + j;
-        const float z = scale * v[j] - mx;
-        const float e = col < N ? __expf(z) : 0.f;
-        s += e;
-        u += e * z;
+        for (int j = 0; j < 32; ++j) {
+          const int col = n0 + c * 32 + j;
+          const float z = scale * v[j] - mx;
+          const float e = col < N ? __expf(z) : 0.f;
+          s += e;
+          u += e * z;
+        }
       }
+    } else {
+      GumbelBest<float> gb;
+      unsigned long long st = an.state0(valid ? row : 0, N, n0);
+#pragma unroll 1
+      for (int c = 0; c < NCH; ++c) {
+        float v[32];
+        ld(0, c, v);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int col = n0 + c * 32 + j;
+          const float z = scale * v[j] - mx;
+          const float e = col < N ? __expf(z) : 0.f;
+          s += e;
+          u += e * z;
+          if (col < N) gb.offer(e, sm64_expo(sm64_mix(st), 0.f), z, col);
+          st += SM64_G;
+        }
+      }
+      if (valid)
+        reinterpret_cast<float2*>(an.gpart)[(size_t)tile * M + row] =
+            make_float2(gb.value(mx), (float)gb.id);  // ids < 2^24: exact
     }
-    if (valid) {
-      const int tile = n0 / (NCH * 32);
+    if (valid)
       reinterpret_cast<float4*>(part)[(size_t)tile * M + row] =
           make_float4(mx, s, u, (float)am);
-    }
   }
 };
 
@@ -1072,7 +1100,8 @@ dg_status tc_moe_experts(dg_model* m, int l, const bf16* X, bf16* hb, float* yb,
 dg_status tc_moe_experts_f8(dg_model* m, int l, const bf16* X, bf16* hb, float* yb,
                             cudaStream_t st);
 dg_status tc_lmhead_stats(dg_model* m, const bf16* xn, int M, float* ent, int32_t* amax,
-                          cudaStream_t st);
+                          cudaStream_t st, const AnnealDev& an = AnnealDev{},
+                          int32_t* sampled = nullptr);
 dg_status tc_attention(dg_model* m, const bf16* q, int B, int nq, int qpos0, const dg_kv* kv,
                        int l, const bf16* kB, const bf16* vB, int nB, int kposB, int npB,
                        bool causal, bf16* out, cudaStream_t st);

@@ -271,17 +271,19 @@ dg_status tc_gemm_swiglu(dg_model* m, const bf16* A, const void* Wg, const void*
 }
 
 dg_status tc_lmhead_stats(dg_model* m, const bf16* xn, int M, float* ent, int32_t* amax,
-                          cudaStream_t st) {
+                          cudaStream_t st, const AnnealDev& an, int32_t* sampled) {
   const dg_config& c = m->cfg;
   CUtensorMap a, b;
   DG_TRY(tmap(m, xn, m->ws.max_tok, c.d_model, 128, &a));
   DG_TRY(tmap(m, m->w.lm_head, c.vocab, c.d_model, LM_BN, &b));
   float* part = (float*)m->ws.lm_part;
-  DG_TRY((launch_dense<LM_BN, 2, false, LM_ST>(m, a, b, b, M, c.vocab, c.d_model,
-                                               EpiLmStats{part, M, c.vocab, c.logit_scale}, st,
+  EpiLmStats epi{part, M, c.vocab, c.logit_scale};
+  epi.an = an;
+  DG_TRY((launch_dense<LM_BN, 2, false, LM_ST>(m, a, b, b, M, c.vocab, c.d_model, epi, st,
                                                false)));
   const int n_vt = ceil_div_i(c.vocab, LM_BN);
-  launch_pdl((lm_merge_kernel<float>), M, 128, 0, st, 1, part, n_vt, M, ent, amax);
+  launch_pdl((lm_merge_kernel<float>), M, 128, 0, st, 1, part, n_vt, M, ent, amax,
+             (const float*)(an.seeds ? an.gpart : nullptr), an.seeds ? sampled : nullptr);
   ++m->launches;
   return DG_OK;
 }

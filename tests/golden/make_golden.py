@@ -30,6 +30,10 @@ Two further modes on a deep workload:
   <name>@append  -> <name>-append.npz: canvas 0's prompt and a block of seeded tokens
      as one causal pass, layer 0's window keys / values at a few positions (the
      reference for appending a finished block to the cache).
+  <name>@anneal  -> <name>-anneal.npz: one forward of the annealed sampler (the Report's
+     default) for canvas 0 at step ANNEAL_K of N = 48 with seed ANNEAL_SEED, on the
+     uniform initial canvas x_1: tempered entropies H/H64, argmax, the Gumbel-max draw
+     `sampled` and its gap to the runner-up, the router margins of the rows.
   <name>@block   -> <name>-block.npz: the oracle's whole block (all [MASK], up to T
      forwards, the entropy-bound sampler after each): per step the input canvas, the
      steps left, H, argmax, margin and the number committed; the number of forwards.
@@ -166,6 +170,32 @@ def append_case(name: str):
     print(f"{name}: wrote {path} in {time.time() - t0:.0f} s (window {Wn})")
 
 
+ANNEAL_SEED, ANNEAL_K = 1234567, 5
+
+
+def anneal_case(name: str):
+    """<name>-anneal.npz: step ANNEAL_K's forward of the annealed sampler on canvas 0."""
+    from oracle import anneal
+    w = workloads.get(name)
+    t0 = time.time()
+    p = anneal.Params()
+    prompt = model_inputs.prompt(w.with_(batch=1))[0].numpy()
+    canvas = anneal.initial_canvas(ANNEAL_SEED, w.canvas, w.vocab)
+    ws = om.Weights(w, keep_layers=False)
+    st = om.prefill_then_forward(ws, prompt, canvas, p.N - ANNEAL_K, p.N, want_logits=True)
+    tau = anneal.temperature(ANNEAL_K, p)
+    ts = anneal.tempered_stats(st["logits"], tau)
+    sampled, gap = anneal.sample_tokens(st["logits"], tau, ANNEAL_SEED, ANNEAL_K)
+    out = dict(seed=np.array(ANNEAL_SEED, dtype=np.uint64), k=np.array(ANNEAL_K),
+               N=np.array(p.N), tau=np.array(tau), canvas=canvas, H=ts["H"], H64=ts["H64"],
+               argmax=ts["argmax"], sampled=sampled, gap=gap,
+               router_margin_rows=_router_margin_rows(w, st["routes"]))
+    path = os.path.join(HERE, f"{name}-anneal.npz")
+    np.savez_compressed(path, **out)
+    print(f"{name}: wrote {path} in {time.time() - t0:.0f} s; tau {tau:.4f}, H range "
+          f"[{ts['H'].min():.3f}, {ts['H'].max():.3f}], gaps > 0.05: {(gap > 0.05).mean():.3f}")
+
+
 DEPTHS = (1, 2, 4, 8, 16, 30)
 
 
@@ -251,6 +281,9 @@ if __name__ == "__main__":
             continue
         if arg.endswith("@block"):
             whole_block(arg.removesuffix("@block"))
+            continue
+        if arg.endswith("@anneal"):
+            anneal_case(arg.removesuffix("@anneal"))
             continue
         if arg.endswith("+rmonly"):
             name, _, c = arg.removesuffix("+rmonly").partition(":")

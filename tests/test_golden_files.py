@@ -14,7 +14,7 @@ from gpu_helpers import max_abs_rel, storage_tol
 HERE = os.path.join(os.path.dirname(__file__), "golden")
 # first-forward files (the depth sweep and the whole block have their own layouts)
 FILES = sorted(f for f in glob.glob(os.path.join(HERE, "*.npz"))
-               if not f.endswith(("-depths.npz", "-block.npz", "-append.npz")))
+               if not f.endswith(("-depths.npz", "-block.npz", "-append.npz", "-anneal.npz")))
 STATED = 2e-2
 
 
@@ -112,3 +112,16 @@ def test_whole_block_file_is_a_valid_trajectory():
         assert np.array_equal(nxt[changed], b["argmax"][i][changed])
         assert np.array_equal(b["mask_after"][i] == 1, nxt == w.mask_id)
     assert not np.any(b["final_canvas"] == w.mask_id)
+
+
+def test_anneal_file_is_consistent():
+    """The annealed forward file: its canvas is the seed's x_1, the draws are tokens, the
+    gaps are non-negative, the argmax and draw agree where the noise cannot move them."""
+    from oracle import anneal as an
+    g = _load("layer1-bf16-anneal.npz")
+    C, V = 256, 262144
+    assert np.array_equal(g["canvas"], an.initial_canvas(int(g["seed"]), C, V))
+    assert ((g["sampled"] >= 0) & (g["sampled"] < V)).all() and (g["gap"] >= 0).all()
+    assert abs(float(g["tau"]) - an.temperature(int(g["k"]), an.Params(N=int(g["N"])))) < 1e-15
+    assert np.allclose(g["H"], g["H64"], rtol=1e-6)
+    assert 0.9 < (g["gap"] > 0.05).mean() <= 1.0

@@ -1,0 +1,275 @@
+"""The Report's default sampler on the device (dg_anneal_*, dg_generate_block_annealed)
+against oracle/anneal.py.
+
+  * initial canvases and the refinement step, bit-exact on seeded synthetic statistics
+    (ragged and full-size shapes, ties, NaN / inf / negative entropies, saturated sums,
+    canvases that stop and canvases that do not);
+  * tiny fp32 model (fp64 activations on the device): the tempered entropy (1e-6, its
+    fp32 rounding), the argmax and the Gumbel-max draw of single forwards, and whole
+    blocks token for token with the same forward counts, at the Report's constants and
+    at a low temperature where every canvas stops early;
+  * small and full-size bf16 models: tempered entropies within 2e-2 and the draw equal
+    wherever the oracle's race is decided (best minus runner-up > 0.05, and for the
+    full-size layer a top-8 router gap > 1e-2 on the row);
+  * the block as a device-controlled loop equals the block as plain launches.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import anneal as an
+from oracle import model as om
+from synth import gen, model_inputs, workloads
+
+from gpu_helpers import make_model, max_abs_rel
+
+pytestmark = pytest.mark.gpu
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+DECIDED = 0.05
+
+
+def _seeds(n, base=1000):
+    return [base + 7919 * b for b in range(n)]
+
+
+def test_initial_canvas_matches_oracle():
+    from masked_discrete_diffusion_b200 import binding
+    for B, C, V in ((3, 256, 262144), (2, 96, 1024), (1, 1, 7)):
+        seeds = _seeds(B, 5)
+        canvas, prev, state = binding.dg_anneal_init(B, C, V, seeds)
+        torch.cuda.synchronize()
+        for b in range(B):
+            assert np.array_equal(canvas[b].cpu().numpy(), an.initial_canvas(seeds[b], C, V))
+        assert (prev == -1).all() and (state == 0).all()
+
+
+# --- the refinement step on synthetic statistics ----------------------------------------
+def _stats(tag, B, C, V, step, kind):
+    u = gen.uniform_u16(101, f"anneal.{tag}.{step}", 5 * B * C).numpy().reshape(5, B, C)
+    H = (u[0] / 65536.0 * 3.0).astype(np.float32)
+    for b in range(B):
+        r = b % 4
+        if r == 1:                                   # low entropies: long prefixes, stops
+            H[b] = (u[1, b] / 65536.0 * 0.008).astype(np.float32)
+        elif r == 2:                                 # ties
+            H[b] = (np.floor(u[1, b] / 65536.0 * 4) * 0.02).astype(np.float32)
+        elif r == 3 and kind == "special":
+            H[b, ::7] = 0.0
+            H[b, 3::11] = -0.5
+            H[b, 5::13] = np.nan
+            H[b, 6::17] = np.inf
+    am = (u[2] % V).astype(np.int32)
+    # canvases 1 mod 4 keep their argmax from step to step (so they may stop)
+    stable = (gen.uniform_u16(101, f"anneal.{tag}.am", B * C).numpy().reshape(B, C) % V)
+    am[1::4] = stable[1::4]
+    sampled = (u[3] % V).astype(np.int32)
+    return H, am, sampled
+
+
+def _oracle_step(H, am, sampled, canvas, prev, state, k, V, seed, p):
+    if state != 0:
+        return canvas, prev, state, None
+    stop = an.stop_test(H, am, prev if k > 0 else None, p.e_stop)
+    if stop or k == p.N - 1:
+        return am.astype(np.int64), am.astype(np.int64), k + 1, len(H)
+    c, n = an.refine(H, sampled, seed, k, V, p.b)
+    return c, am.astype(np.int64), 0, n
+
+
+@pytest.mark.parametrize("B,C,V", [(8, 256, 262144), (5, 96, 1024), (2, 1, 7), (1, 1024, 262144),
+                                   (3, 33, 50)])
+@pytest.mark.parametrize("kind", ["plain", "special"])
+@pytest.mark.parametrize("pset", ["report", "wide", "strict"])
+def test_refinement_steps_bit_exact(B, C, V, kind, pset):
+    from masked_discrete_diffusion_b200 import binding
+    p = {"report": an.Params(N=6),
+         "wide": an.Params(N=5, b=float("inf"), e_stop=16.0),
+         "strict": an.Params(N=4, b=0.0, e_stop=0.0)}[pset]
+    seeds = _seeds(B, 17)
+    canvas, prev, state = binding.dg_anneal_init(B, C, V, seeds)
+    oc = [an.initial_canvas(seeds[b], C, V) for b in range(B)]
+    op = [np.full(C, -1, np.int64) for _ in range(B)]
+    ost = [0] * B
+    tag = f"{B}.{C}.{V}.{kind}"
+    for k in range(p.N):
+        H, am, smp = _stats(tag, B, C, V, k, kind)
+        nacc = binding.dg_anneal_sample(torch.from_numpy(H).cuda(), torch.from_numpy(am).cuda(),
+                                        torch.from_numpy(smp).cuda(), canvas, prev, state, k, V,
+                                        seeds, p)
+        torch.cuda.synchronize()
+        for b in range(B):
+            was_running = ost[b] == 0
+            oc[b], op[b], ost[b], n = _oracle_step(H[b], am[b], smp[b], oc[b], op[b], ost[b], k,
+                                                   V, seeds[b], p)
+            assert np.array_equal(canvas[b].cpu().numpy(), oc[b]), (k, b)
+            assert int(state[b]) == ost[b], (k, b)
+            if was_running:
+                assert np.array_equal(prev[b].cpu().numpy(), op[b])
+                assert int(nacc[b]) == n, (k, b)
+    assert all(s > 0 for s in ost)                   # every canvas ended by step N - 1
+
+
+# --- forwards and whole blocks of the tiny fp32 model ------------------------------------
+def test_tiny_forward_tempered_and_drawn():
+    from masked_discrete_diffusion_b200 import binding
+    w = workloads.TINY_F32
+    model = make_model(w)
+    try:
+        prompt = model_inputs.prompt(w, "cuda")
+        kv = binding.dg_prefill(model, prompt)
+        ws = om.Weights(w, keep_layers=True)
+        okv = om.prefill(ws, prompt[0].cpu().numpy())
+        p, seed = an.Params(), 77
+        canvas = an.initial_canvas(seed, w.canvas, w.vocab)
+        dcanvas = torch.from_numpy(canvas.astype(np.int32)).reshape(1, -1).cuda()
+        for k in (0, 5, 47):
+            H, am, smp = binding.dg_anneal_forward(model, kv, dcanvas, k, [seed], p)
+            binding.dg_sync_status(model)
+            logits = om.denoise_forward(ws, okv, canvas, p.N - k, p.N, w.prompt_len,
+                                        want_logits=True)["logits"]
+            tau = an.temperature(k, p)
+            ts = an.tempered_stats(logits, tau)
+            sampled, gap = an.sample_tokens(logits, tau, seed, k)
+            assert max_abs_rel(H[0].cpu().numpy(), ts["H64"]) < 1e-6
+            assert np.array_equal(am[0].cpu().numpy(), ts["argmax"])
+            assert np.array_equal(smp[0].cpu().numpy(), sampled)
+            # the draw is not the argmax everywhere: the noise matters at this temperature
+            assert (sampled != ts["argmax"]).any()
+        kv.close()
+    finally:
+        model.close()
+
+
+@pytest.mark.parametrize("tau", [None, 0.02])
+def test_tiny_blocks_token_for_token(tau):
+    """Three canvases with their own prompts and seeds; at tau = 0.02 canvas 0 stops
+    early (after 29 forwards) while the others run all N steps, at the Report's constants
+    none stops early."""
+    from masked_discrete_diffusion_b200 import binding
+    w = workloads.TINY_F32.with_(batch=3)
+    p = an.Params() if tau is None else an.Params(tau_max=tau, tau_min=tau)
+    seeds = _seeds(3, 31)
+    model = make_model(w)
+    try:
+        prompt = model_inputs.prompt(w, "cuda")
+        kv = binding.dg_prefill(model, prompt)
+        out, nf = binding.dg_generate_block_annealed(model, kv, seeds, p)
+        binding.dg_sync_status(model)
+        ws = om.Weights(w, keep_layers=True)
+        early = []
+        for b in range(3):
+            res, traj = om.generate_block_annealed(ws, prompt[b].cpu().numpy(), seeds[b], p)
+            assert np.array_equal(out[b].cpu().numpy(), res), b
+            assert int(nf[b]) == len(traj), b
+            early.append(len(traj) < p.N)
+        assert any(early) == (tau is not None)
+        kv.close()
+    finally:
+        model.close()
+
+
+# --- bf16 models: entropies within tolerance, draws where the race is decided ------------
+def test_small_bf16_forward_decided_draws():
+    from masked_discrete_diffusion_b200 import binding
+    w = workloads.SMALL_BF16
+    p, k = an.Params(), 3
+    seeds = _seeds(w.batch, 3)
+    model = make_model(w)
+    try:
+        prompt = model_inputs.prompt(w, "cuda")
+        kv = binding.dg_prefill(model, prompt)
+        canvas = np.stack([an.initial_canvas(s, w.canvas, w.vocab) for s in seeds])
+        H, am, smp = binding.dg_anneal_forward(model, kv, torch.from_numpy(
+            canvas.astype(np.int32)).cuda(), k, seeds, p)
+        binding.dg_sync_status(model)
+        ws = om.Weights(w, keep_layers=True)
+        tau = an.temperature(k, p)
+        decided = total = 0
+        for b in range(w.batch):
+            st = om.prefill_then_forward(ws, prompt[b].cpu().numpy(), canvas[b], p.N - k, p.N,
+                                         want_logits=True)
+            ts = an.tempered_stats(st["logits"], tau)
+            sampled, gap = an.sample_tokens(st["logits"], tau, seeds[b], k)
+            assert max_abs_rel(H[b].cpu().numpy(), ts["H64"]) < 2e-2
+            z = np.sort(st["logits"] / tau, axis=1)
+            top = (z[:, -1] - z[:, -2]) > DECIDED
+            assert np.array_equal(am[b].cpu().numpy()[top], ts["argmax"][top])
+            ok = gap > DECIDED
+            assert np.array_equal(smp[b].cpu().numpy()[ok], sampled[ok])
+            decided += int(ok.sum())
+            total += len(ok)
+        assert decided >= 0.9 * total
+        kv.close()
+    finally:
+        model.close()
+
+
+def test_full_size_layer_forward_decided_draws():
+    path = os.path.join(GOLDEN, "layer1-bf16-anneal.npz")
+    if not os.path.exists(path):
+        pytest.skip("golden file missing")
+    from masked_discrete_diffusion_b200 import binding
+    w = workloads.LAYER1_BF16
+    g = np.load(path)
+    p, k, seed = an.Params(N=int(g["N"])), int(g["k"]), int(g["seed"])
+    model = make_model(w)
+    try:
+        kv = binding.dg_prefill(model, model_inputs.prompt(w, "cuda"))
+        H, am, smp = binding.dg_anneal_forward(
+            model, kv, torch.from_numpy(g["canvas"].astype(np.int32)).reshape(1, -1).cuda(), k,
+            [seed], p)
+        binding.dg_sync_status(model)
+        assert max_abs_rel(H[0].cpu().numpy(), g["H64"]) < 2e-2
+        ok = (g["gap"] > DECIDED) & (g["router_margin_rows"] > 1e-2)
+        assert ok.mean() > 0.8
+        assert np.array_equal(smp[0].cpu().numpy()[ok], g["sampled"][ok])
+        kv.close()
+    finally:
+        model.close()
+
+
+# --- the loop graph, the plain launches, validation ---------------------------------------
+def test_small_block_loop_equals_plain_launches(monkeypatch):
+    from masked_discrete_diffusion_b200 import binding
+    w = workloads.SMALL_BF16
+    seeds = _seeds(w.batch, 99)
+    outs = []
+    for no_graphs in ("0", "1"):
+        monkeypatch.setenv("DG_NO_GRAPHS", no_graphs)
+        model = make_model(w)
+        try:
+            kv = binding.dg_prefill(model, model_inputs.prompt(w, "cuda"))
+            out, nf = binding.dg_generate_block_annealed(model, kv, seeds, an.Params(N=12))
+            binding.dg_sync_status(model)
+            if no_graphs == "0":
+                assert binding.dg_block_loop_launches(model) > 0
+                again, nf2 = binding.dg_generate_block_annealed(model, kv, seeds,
+                                                                an.Params(N=12))
+                assert torch.equal(again, out) and torch.equal(nf2, nf)   # graph replay
+            outs.append((out.cpu(), nf.cpu()))
+            kv.close()
+        finally:
+            model.close()
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+    out, nf = outs[0]
+    assert ((out >= 0) & (out < w.vocab)).all() and ((nf >= 1) & (nf <= 12)).all()
+
+
+def test_parameters_are_validated():
+    from masked_discrete_diffusion_b200 import binding
+    H = torch.zeros(1, 8, device="cuda")
+    a = torch.zeros(1, 8, dtype=torch.int32, device="cuda")
+    canvas, prev, state = binding.dg_anneal_init(1, 8, 10, [1])
+    bad = [an.Params(N=0), an.Params(b=float("nan")), an.Params(b=-1.0),
+           an.Params(tau_min=0.0), an.Params(tau_max=float("inf")), an.Params(e_stop=17.0),
+           an.Params(e_stop=float("nan"))]
+    for p in bad:
+        with pytest.raises(binding.DGError) as e:
+            binding.dg_anneal_sample(H, a, a, canvas, prev, state, 0, 10, [1], p)
+        assert e.value.status == 1
+    with pytest.raises(binding.DGError):
+        binding.dg_anneal_sample(H, a, a, canvas, prev, state, 6, 10, [1], an.Params(N=6))
+    with pytest.raises(binding.DGError):
+        binding.dg_anneal_init(1, 8, (1 << 24) + 1, [1])

@@ -58,3 +58,23 @@ def test_sampler_nothing_masked_is_noop():
     n = binding.dg_eb_sample(torch.from_numpy(H).cuda(), torch.from_numpy(am).cuda(), dC,
                              torch.from_numpy(mask).cuda(), 3, 1.0)
     assert n.cpu().tolist() == [0, 0] and np.array_equal(dC.cpu().numpy(), canvas)
+
+
+@pytest.mark.parametrize("C,s", [(1024, 64), (512, 8), (1024, 1)])
+def test_sampler_saturated_prefix_sums(C, s):
+    """Every position masked with a NaN entropy (fixed point 2^54 each) and gamma = inf
+    (bound 2^62): the prefix sums pass 2^63 past position 511; the count within the bound
+    must still be exactly 256 (the oracle's unbounded integers)."""
+    from masked_discrete_diffusion_b200 import binding
+    H = np.full((1, C), np.nan, np.float32)
+    am = (np.arange(C, dtype=np.int32) * 7 % 1000).reshape(1, C)
+    canvas = np.full((1, C), 1000, np.int32)
+    mask = np.ones((1, C), np.uint8)
+    dC = torch.from_numpy(canvas).cuda()
+    dM = torch.from_numpy(mask).cuda()
+    n = binding.dg_eb_sample(torch.from_numpy(H).cuda(), torch.from_numpy(am).cuda(), dC, dM, s,
+                             float("inf"))
+    c2, m2, n2, kg = osamp.eb_step(H[0], am[0], canvas[0], mask[0], s, float("inf"))
+    assert kg == 256
+    assert int(n[0]) == n2 == max(256, -(-C // s))
+    assert np.array_equal(dC[0].cpu().numpy(), c2) and np.array_equal(dM[0].cpu().numpy(), m2)
