@@ -1271,7 +1271,7 @@ dg_status dg_generate_block_annealed(dg_model* m, const dg_kv* kv, const dg_anne
   DG_TRY(anneal_check(p, m->cfg.vocab, &q));
   DG_REQUIRE(m->cfg.canvas <= 1024, "canvas %d > 1024", m->cfg.canvas);
   cudaStream_t st = (cudaStream_t)stream;
-  if (!m->use_graphs || m->profiling)
+  if (!m->use_graphs)
     return anneal_impl(m, kv, p, q, seeds, canvas_out, n_forwards, st,
                        m->profiling ? m->prof_forwards : 0);
   dg::BlockGraph* g = nullptr;
@@ -1279,7 +1279,8 @@ dg_status dg_generate_block_annealed(dg_model* m, const dg_kv* kv, const dg_anne
     if (x->anneal && x->kv == kv && x->kv_P == kv->P && x->kv_W == kv->W && x->aN == p->N &&
         x->ab == p->b && x->atmax == p->tau_max && x->atmin == p->tau_min &&
         x->aestop == p->e_stop && x->seeds == seeds && x->canvas == canvas_out &&
-        x->nfwd == n_forwards) {
+        x->nfwd == n_forwards && x->prof == m->profiling &&
+        (!x->prof || x->fcap == m->prof_forwards)) {
       g = x;
       break;
     }
@@ -1301,8 +1302,36 @@ dg_status dg_generate_block_annealed(dg_model* m, const dg_kv* kv, const dg_anne
     g->seeds = seeds;
     g->canvas = canvas_out;
     g->nfwd = n_forwards;
+    g->prof = m->profiling;
+    g->fcap = m->profiling ? m->prof_forwards : 0;
     if (!m->cap_stream) DG_TRY_CUDA(cudaStreamCreateWithFlags(&m->cap_stream, cudaStreamNonBlocking));
-    if (!build_anneal_graph(m, kv, p, q, seeds, canvas_out, n_forwards, g)) {
+    if (g->prof) {
+      // profiling: the first fcap forwards unrolled, with an event pair around every
+      // launch group recorded by the graph (read back after each replay)
+      const long long l0 = m->launches;
+      m->capture = g;
+      cudaGraph_t graph = nullptr;
+      cudaError_t e = cudaStreamBeginCapture(m->cap_stream, cudaStreamCaptureModeThreadLocal);
+      dg_status s = DG_OK;
+      if (e == cudaSuccess) {
+        s = anneal_impl(m, kv, p, q, seeds, canvas_out, n_forwards, m->cap_stream, g->fcap);
+        e = cudaStreamEndCapture(m->cap_stream, &graph);
+      }
+      m->capture = nullptr;
+      g->launches = m->launches - l0;
+      m->launches = l0;
+      if (s == DG_OK && e == cudaSuccess) e = cudaGraphInstantiate(&g->exec, graph, 0);
+      if (graph) cudaGraphDestroy(graph);
+      if (s != DG_OK || e != cudaSuccess) {
+        graph_free(g);
+        if (s == DG_OK) {
+          set_error("annealed block capture failed: %s", cudaGetErrorString(e));
+          s = DG_ERR_CUDA;
+        }
+        cudaGetLastError();
+        return s;
+      }
+    } else if (!build_anneal_graph(m, kv, p, q, seeds, canvas_out, n_forwards, g)) {
       graph_free(g);
       return anneal_impl(m, kv, p, q, seeds, canvas_out, n_forwards, st, 0);
     }

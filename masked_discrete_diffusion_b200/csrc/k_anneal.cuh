@@ -17,9 +17,11 @@
 //  * draws: SplitMix64 (Steele, Lea and Flood, OOPSLA 2014) used counter-wise, the
 //    c-th output after state key being mix64(key + (c + 1) G); per canvas seed three
 //    stream keys mix64(seed + j G), j = 1 initial canvas (c = i), 2 Gumbel noise
-//    (c = (k C + i) V + v), 3 re-noising (c = k C + i); token = hi32(z) V >> 32;
-//    Gumbel noise -log E, E = -log u, u = (z >> 41 + 1/2) 2^-23; the drawn token is
-//    argmax_v (l_v / tau - log E_v), the lowest id on ties.
+//    (c = (k C + i) ceil(V / 2) + floor(v / 2): one output per token pair, the even
+//    token taking bits 63..41 and the odd one bits 31..9), 3 re-noising (c = k C + i);
+//    token = hi32(z) V >> 32; Gumbel noise -log E, E = -log u, u = (f + 1/2) 2^-23
+//    for the 23-bit field f; the drawn token is argmax_v (l_v / tau - log E_v), the
+//    lowest id on ties.
 #pragma once
 
 #include "k_common.cuh"
@@ -46,12 +48,16 @@ __host__ __device__ __forceinline__ unsigned long long sm64_draw(unsigned long l
 __device__ __forceinline__ int32_t sm64_token(unsigned long long z, int V) {
   return (int32_t)(((z >> 32) * (unsigned long long)(unsigned)V) >> 32);
 }
-// E = -log u with u = (floor(z / 2^41) + 1/2) 2^-23, exact in fp32 and fp64
-__device__ __forceinline__ float sm64_expo(unsigned long long z, float) {
-  return -logf(((float)(unsigned)(z >> 41) + 0.5f) * 1.1920928955078125e-07f);
+// the 23-bit field of output z for the even (odd = 0) or odd token of a pair
+__device__ __forceinline__ unsigned sm64_field(unsigned long long z, int odd) {
+  return odd ? (unsigned)(z >> 9) & 0x7FFFFFu : (unsigned)(z >> 41);
 }
-__device__ __forceinline__ double sm64_expo(unsigned long long z, double) {
-  return -log(((double)(unsigned)(z >> 41) + 0.5) * 1.1920928955078125e-07);
+// E = -log u with u = (f + 1/2) 2^-23, u exact in fp32 and fp64
+__device__ __forceinline__ float sm64_expo(unsigned f, float) {
+  return -logf(((float)f + 0.5f) * 1.1920928955078125e-07f);
+}
+__device__ __forceinline__ double sm64_expo(unsigned f, double) {
+  return -log(((double)f + 0.5) * 1.1920928955078125e-07);
 }
 
 // Per-launch parameters of the tempered LM-head statistics and the Gumbel-max draw.
@@ -67,13 +73,14 @@ struct AnnealDev {
     return (double)tau_min +
            ((double)tau_max - (double)tau_min) * ((double)steps_left() / (double)N);
   }
-  // the Gumbel stream's state before column col of row `row`: key + (c + 1) G with
-  // c = (k C + i) V + col
-  __device__ __forceinline__ unsigned long long state0(int row, int V, int col) const {
+  // the Gumbel stream's state for token pair `pair` of row `row`: key + (c + 1) G with
+  // c = (k C + i) ceil(V / 2) + pair
+  __device__ __forceinline__ unsigned long long pair_state(int row, int V, int pair) const {
     const int b = row / C, i = row - b * C;
     const unsigned long long key = sm64_key(seeds[b], SM64_GUMBEL);
     const unsigned long long k = (unsigned long long)(N - steps_left());
-    const unsigned long long c = (k * C + i) * (unsigned long long)V + (unsigned)col;
+    const unsigned long long c =
+        (k * C + i) * (unsigned long long)((V + 1) >> 1) + (unsigned)pair;
     return key + (c + 1) * SM64_G;
   }
 };
@@ -84,18 +91,25 @@ struct AnnealDev {
 template <class Acc> struct GumbelBest {
   Acc e = 0, E = 1, z = 0;
   int id = 0x7fffffff;
-  __device__ __forceinline__ void offer(Acc e2, Acc E2, Acc z2, int id2) {
+  __device__ __forceinline__ bool offer(Acc e2, Acc E2, Acc z2, int id2) {
     const Acc l = e2 * E, r = e * E2;
     if (l > r || (l == r && id2 < id)) {
       e = e2;
       E = E2;
       z = z2;
       id = id2;
+      return true;
     }
+    return false;
   }
   // the candidate's value on the absolute scale: m + z - log E = l / tau + Gumbel noise
   __device__ __forceinline__ Acc value(Acc m) const { return m + z - dlog(E); }
 };
+
+// The smallest E a draw can give is -log(1 - 2^-24) = 5.96e-8; a candidate with
+// e < e_best * SM64_EMIN_LO / E_best therefore cannot beat the best (SM64_EMIN_LO is a
+// little below that minimum, so the test never discards a possible winner).
+constexpr float SM64_EMIN_LO = 5.9e-8f;
 
 // x_1: uniform tokens (stream 1); previous argmax -1; per-canvas stop state 0; the
 // loop's steps-left counter N.

@@ -775,12 +775,13 @@ __global__ void __launch_bounds__(256)
     }
     if (an.seeds) {  // this tile's winner of the race, lane by lane then across the warp
       GumbelBest<Acc> gb;
-      const unsigned long long st = an.state0(r, V, n0);
+      const unsigned long long st = an.pair_state(r, V, 0);
       for (int c = lane; c < SG_BN; c += 32) {
-        if (n0 + c >= V) continue;
+        const int col = n0 + c;
+        if (col >= V) continue;
         const Acc z = T[rr][c] - mx;
-        gb.offer(dexp(z), (Acc)sm64_expo(sm64_mix(st + (unsigned long long)c * SM64_G), Acc(0)),
-                 z, n0 + c);
+        const unsigned long long zz = sm64_mix(st + (unsigned long long)(col >> 1) * SM64_G);
+        gb.offer(dexp(z), sm64_expo(sm64_field(zz, col & 1), Acc(0)), z, col);
       }
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) {

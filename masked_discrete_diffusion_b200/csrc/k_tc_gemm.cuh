@@ -375,6 +375,10 @@ struct EpiRouterTopk {
 // With an.N > 0 the logits are tempered (l = scale acc / tau) and, with an.seeds, the
 // tile's winner of the Gumbel-max race goes to an.gpart[(tile, row)] = (l / tau - log E,
 // id).
+// Pass 1 finds the largest accumulator (a max tree per 32-column chunk; the index is
+// searched only in a chunk that raises the maximum).  Pass 2 works in base-2 units,
+// z2 = (l - m) log2 e, e = 2^z2 (ex2.approx.ftz), with two interleaved sums; columns
+// >= N hold a large negative finite value, so that no column test is needed per element.
 struct EpiLmStats {
   static constexpr bool kStaged = false, kWarpRows = false;
   static constexpr size_t kExtraSmem = 0;
@@ -382,58 +386,122 @@ struct EpiLmStats {
   int M, N;
   float scale;
   AnnealDev an = {};
+
+  static __device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+  }
+
   template <int NCH, class Ld>
   __device__ void run(int row, bool valid, int n0, Ld&& ld) const {
-    const float scale = an.N > 0 ? (float)((double)this->scale / an.tau()) : this->scale;
-    float mx = -INFINITY;
+    constexpr float kLog2e = 1.4426950408889634f, kLn2 = 0.6931471805599453f;
+    const float sc = an.N > 0 ? (float)((double)scale / an.tau()) : scale;
+    const float sc2 = sc * kLog2e;
+    auto load = [&](int c, float* v) {
+      ld(0, c, v);
+      if (n0 + c * 32 + 32 > N) {  // the ragged last tile (uniform across the warp)
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (n0 + c * 32 + j >= N) v[j] = -1e30f;
+      }
+    };
+    // pass 1
+    float mv = -INFINITY;
     int am = 0x7fffffff;
 #pragma unroll 1
     for (int c = 0; c < NCH; ++c) {
       float v[32];
-      ld(0, c, v);
+      load(c, v);
+      float t[16];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const int col = n0 + c * 32 + j;
-        const float l = scale * v[j];
-        if (col < N && l > mx) {
-          mx = l;
-          am = col;
-        }
+      for (int j = 0; j < 16; ++j) t[j] = fmaxf(v[j], v[j + 16]);
+#pragma unroll
+      for (int w = 8; w > 0; w >>= 1)
+#pragma unroll
+        for (int j = 0; j < w; ++j) t[j] = fmaxf(t[j], t[j + w]);
+      if (t[0] > mv) {  // strict: an equal maximum in a later chunk keeps the earlier id
+        int idx = 31;
+#pragma unroll
+        for (int j = 30; j >= 0; --j)
+          if (v[j] == t[0]) idx = j;
+        mv = t[0];
+        am = n0 + c * 32 + idx;
       }
     }
-    float s = 0.f, u = 0.f;
+    const float mx = sc * mv, mx2 = sc2 * mv;
+    // pass 2
+    float s0 = 0.f, s1 = 0.f, u0 = 0.f, u1 = 0.f;
     const int tile = n0 / (NCH * 32);
     if (an.seeds == nullptr) {
 #pragma unroll 1
       for (int c = 0; c < NCH; ++c) {
         float v[32];
-        ld(0, c, v);
+        load(c, v);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int col = n0 + c * 32 + j;
-          const float z = scale * v[j] - mx;
-          const float e = col < N ? __expf(z) : 0.f;
-          s += e;
-          u += e * z;
+        for (int j = 0; j < 32; j += 2) {
+          const float z0 = fmaf(v[j], sc2, -mx2), z1 = fmaf(v[j + 1], sc2, -mx2);
+          const float e0 = ex2(z0), e1 = ex2(z1);
+          s0 += e0;
+          s1 += e1;
+          u0 = fmaf(e0, z0, u0);
+          u1 = fmaf(e1, z1, u1);
         }
       }
     } else {
+      // Gumbel-max race of this tile: it starts from the tile's argmax (z = 0, e = 1);
+      // a chunk where no row of the warp has e >= E_argmax^-1 E_min draws nothing (no
+      // column there can beat the argmax).  Otherwise each output of the stream serves a
+      // column pair, and since E = -log u >= 1 - u a column can beat the argmax (hence
+      // the best so far) only if 1 - u < e E_argmax (the margin 2^-10 covers every
+      // rounding): only those columns take the log, in a branch the warp skips when none
+      // of its rows has one.
       GumbelBest<float> gb;
-      unsigned long long st = an.state0(valid ? row : 0, N, n0);
+      const unsigned long long st = an.pair_state(valid ? row : 0, N, n0 >> 1);
+      if (am < N)
+        gb.offer(1.f,
+                 sm64_expo(sm64_field(sm64_mix(st + (unsigned long long)((am - n0) >> 1) * SM64_G),
+                                      am & 1),
+                           0.f),
+                 0.f, am);
+      const float lim = gb.e * SM64_EMIN_LO / gb.E;
+      const float tcap = gb.E * (1.f + 1.f / 1024.f);
 #pragma unroll 1
       for (int c = 0; c < NCH; ++c) {
         float v[32];
-        ld(0, c, v);
+        load(c, v);
+        bool cand = false;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int col = n0 + c * 32 + j;
-          const float z = scale * v[j] - mx;
-          const float e = col < N ? __expf(z) : 0.f;
-          s += e;
-          u += e * z;
-          if (col < N) gb.offer(e, sm64_expo(sm64_mix(st), 0.f), z, col);
-          st += SM64_G;
+        for (int j = 0; j < 32; j += 2) {
+          const float z0 = fmaf(v[j], sc2, -mx2), z1 = fmaf(v[j + 1], sc2, -mx2);
+          const float e0 = ex2(z0), e1 = ex2(z1);
+          s0 += e0;
+          s1 += e1;
+          u0 = fmaf(e0, z0, u0);
+          u1 = fmaf(e1, z1, u1);
+          v[j] = z0;
+          v[j + 1] = z1;
+          cand |= fmaxf(e0, e1) >= lim;
         }
+        if (!__any_sync(0xffffffffu, cand)) continue;
+        const unsigned long long stc = st + (unsigned long long)(c * 16) * SM64_G;
+        float uu[32];
+        unsigned fm = 0;
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          const unsigned long long zz = sm64_mix(stc + (unsigned long long)q * SM64_G);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int j = 2 * q + h;
+            const float uj = ((float)sm64_field(zz, h) + 0.5f) * 1.1920928955078125e-07f;
+            uu[j] = uj;
+            if (1.f - uj < ex2(v[j]) * tcap) fm |= 1u << j;
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (__any_sync(0xffffffffu, (fm >> j) & 1u) && ((fm >> j) & 1u))
+            gb.offer(ex2(v[j]), -logf(uu[j]), v[j] * kLn2, n0 + c * 32 + j);
       }
       if (valid)
         reinterpret_cast<float2*>(an.gpart)[(size_t)tile * M + row] =
@@ -441,7 +509,7 @@ struct EpiLmStats {
     }
     if (valid)
       reinterpret_cast<float4*>(part)[(size_t)tile * M + row] =
-          make_float4(mx, s, u, (float)am);
+          make_float4(mx, s0 + s1, (u0 + u1) * kLn2, (float)am);
   }
 };
 
@@ -657,10 +725,11 @@ __global__ void __launch_bounds__(TC_DENSE_THREADS, 1)
   const int quarter = warp & 3, half = warp >> 2;  // TMEM lane quarter; column half
   const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
   if constexpr (!Epi::kStaged) {
-    if (ready && half == 0) {  // never split; thread per row
+    // thread per row; with two 128-row blocks the two warp groups take one each
+    if (ready && (MT == 2 || half == 0)) {
       tc::fence_after_sync();
 #pragma unroll 1
-      for (int mt = 0; mt < MT; ++mt) {
+      for (int mt = MT == 2 ? half : 0; mt < MT; mt += MT == 2 ? 2 : 1) {
         const int row = m0 + mt * 128 + 32 * quarter + lane;
         auto ld = [&](int a, int c, float* v) {
           tc::tmem_ld32(tmem + lane_base + (mt * Cfg::NACC + a) * BN + c * 32, v);

@@ -45,12 +45,14 @@ Readings of what the pages leave open (the same list stands beside the CUDA path
     gives three stream keys, key_j = mix64(seed + j G) for j = 1 (initial canvas),
     2 (Gumbel noise), 3 (re-noising).
       initial token of position i:        stream 1, c = i
-      Gumbel noise of (k, i, token v):     stream 2, c = (k C + i) V + v
+      Gumbel noise of (k, i, tokens 2p, 2p + 1):
+                                           stream 2, c = (k C + i) ceil(V / 2) + p
       re-noise token of (k, i):            stream 3, c = k C + i
-    A token from 64 bits z is floor(hi32(z) V / 2^32) (multiply-shift).  A Gumbel
-    variate is -log(-log u) with u = (floor(z / 2^41) + 1/2) 2^-23 (exact in fp32).
-    The drawn token is argmax_v (l_v / tau + g_v), the lowest id on exact ties
-    (Gumbel-max: a draw from softmax(l / tau)).
+    A token from 64 bits z is floor(hi32(z) V / 2^32) (multiply-shift).  One output z
+    of stream 2 serves two tokens: the 23-bit field f = bits 63..41 of z for the even
+    token, bits 31..9 for the odd one; the Gumbel variate is -log(-log u) with
+    u = (f + 1/2) 2^-23 (exact in fp32).  The drawn token is argmax_v (l_v / tau + g_v),
+    the lowest id on exact ties (Gumbel-max: a draw from softmax(l / tau)).
 """
 from __future__ import annotations
 
@@ -118,10 +120,17 @@ def token_from_bits(z: np.ndarray, V: int) -> np.ndarray:
     return ((hi * np.uint64(V)) >> np.uint64(32)).astype(np.int64)   # V < 2^32: no wrap
 
 
-def gumbel_from_bits(z: np.ndarray) -> np.ndarray:
-    k = (np.asarray(z, dtype=np.uint64) >> np.uint64(41)).astype(np.float64)
-    u = (k + 0.5) * 2.0 ** -23
+def gumbel_from_field(f: np.ndarray) -> np.ndarray:
+    """Gumbel variate of a 23-bit field f: -log(-log u), u = (f + 1/2) 2^-23."""
+    u = (np.asarray(f, dtype=np.float64) + 0.5) * 2.0 ** -23
     return -np.log(-np.log(u))
+
+
+def fields_of_bits(z: np.ndarray) -> np.ndarray:
+    """The two 23-bit fields of each output: [..., 2] = (bits 63..41, bits 31..9)."""
+    z = np.asarray(z, dtype=np.uint64)
+    m = np.uint64((1 << 23) - 1)
+    return np.stack([z >> np.uint64(41), (z >> np.uint64(9)) & m], axis=-1)
 
 
 def initial_canvas(seed: int, C: int, V: int) -> np.ndarray:
@@ -130,9 +139,12 @@ def initial_canvas(seed: int, C: int, V: int) -> np.ndarray:
 
 
 def gumbel_row(seed: int, k: int, i: int, C: int, V: int) -> np.ndarray:
-    """Gumbel noise of all V tokens at step k, position i."""
-    c0 = (k * C + i) * V
-    return gumbel_from_bits(draw(stream_key(seed, STREAM_GUMBEL), np.arange(c0, c0 + V)))
+    """Gumbel noise of all V tokens at step k, position i (token v from output
+    (k C + i) ceil(V / 2) + floor(v / 2) of stream 2, field v mod 2)."""
+    half = (V + 1) // 2
+    c0 = (k * C + i) * half
+    f = fields_of_bits(draw(stream_key(seed, STREAM_GUMBEL), np.arange(c0, c0 + half)))
+    return gumbel_from_field(f.reshape(-1)[:V])
 
 
 def renoise_tokens(seed: int, k: int, C: int, V: int) -> np.ndarray:

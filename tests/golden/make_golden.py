@@ -33,7 +33,8 @@ Two further modes on a deep workload:
   <name>@anneal  -> <name>-anneal.npz: one forward of the annealed sampler (the Report's
      default) for canvas 0 at step ANNEAL_K of N = 48 with seed ANNEAL_SEED, on the
      uniform initial canvas x_1: tempered entropies H/H64, argmax, the Gumbel-max draw
-     `sampled` and its gap to the runner-up, the router margins of the rows.
+     `sampled` and its gap to the runner-up, the router margins of the rows, and the
+     bf16-storage run's H_s16 and sampled_s16.
   <name>@block   -> <name>-block.npz: the oracle's whole block (all [MASK], up to T
      forwards, the entropy-bound sampler after each): per step the input canvas, the
      steps left, H, argmax, margin and the number committed; the number of forwards.
@@ -186,10 +187,14 @@ def anneal_case(name: str):
     tau = anneal.temperature(ANNEAL_K, p)
     ts = anneal.tempered_stats(st["logits"], tau)
     sampled, gap = anneal.sample_tokens(st["logits"], tau, ANNEAL_SEED, ANNEAL_K)
+    ws16 = om.Weights(w, keep_layers=False, storage="bf16")
+    s16 = om.prefill_then_forward(ws16, prompt, canvas, p.N - ANNEAL_K, p.N, want_logits=True)
+    ts16 = anneal.tempered_stats(s16["logits"], tau)
     out = dict(seed=np.array(ANNEAL_SEED, dtype=np.uint64), k=np.array(ANNEAL_K),
                N=np.array(p.N), tau=np.array(tau), canvas=canvas, H=ts["H"], H64=ts["H64"],
                argmax=ts["argmax"], sampled=sampled, gap=gap,
-               router_margin_rows=_router_margin_rows(w, st["routes"]))
+               router_margin_rows=_router_margin_rows(w, st["routes"]), H_s16=ts16["H64"],
+               sampled_s16=anneal.sample_tokens(s16["logits"], tau, ANNEAL_SEED, ANNEAL_K)[0])
     path = os.path.join(HERE, f"{name}-anneal.npz")
     np.savez_compressed(path, **out)
     print(f"{name}: wrote {path} in {time.time() - t0:.0f} s; tau {tau:.4f}, H range "

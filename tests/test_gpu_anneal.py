@@ -8,9 +8,11 @@ against oracle/anneal.py.
     fp32 rounding), the argmax and the Gumbel-max draw of single forwards, and whole
     blocks token for token with the same forward counts, at the Report's constants and
     at a low temperature where every canvas stops early;
-  * small and full-size bf16 models: tempered entropies within 2e-2 and the draw equal
-    wherever the oracle's race is decided (best minus runner-up > 0.05, and for the
-    full-size layer a top-8 router gap > 1e-2 on the row);
+  * small and full-size bf16 models: tempered entropies within 2e-2 (for the full-size
+    layer on its uniform random canvas: the storage-noise bound, 1.5x the distance of
+    the oracle's bf16-storage run, on rows whose top-8 routing is decided) and the draw
+    equal wherever the oracle's race is decided (best minus runner-up > 0.05, and for
+    the full-size layer a top-8 router gap > 1e-2 on the row);
   * the block as a device-controlled loop equals the block as plain launches.
 """
 import os
@@ -221,8 +223,18 @@ def test_full_size_layer_forward_decided_draws():
             model, kv, torch.from_numpy(g["canvas"].astype(np.int32)).reshape(1, -1).cuda(), k,
             [seed], p)
         binding.dg_sync_status(model)
-        assert max_abs_rel(H[0].cpu().numpy(), g["H64"]) < 2e-2
-        ok = (g["gap"] > DECIDED) & (g["router_margin_rows"] > 1e-2)
+        # the uniform random canvas routes its rows diversely: 41 of 256 rows have a top-8
+        # router gap below 1e-2 and may route differently under any perturbation; on the
+        # others the storage-noise rule sets the bound (the oracle's bf16-storage run is
+        # 2.1e-2 from its fp64 run there, so 1.5x that)
+        route = g["router_margin_rows"] > 1e-2
+        dist = max_abs_rel(g["H_s16"][route], g["H64"][route])
+        tol = 2e-2 if dist < 1e-2 else max(2e-2, 1.5 * dist)
+        assert max_abs_rel(H[0].cpu().numpy()[route], g["H64"][route]) < tol
+        # every row, against the storage distance over every row
+        dist_all = max_abs_rel(g["H_s16"], g["H64"])
+        assert max_abs_rel(H[0].cpu().numpy(), g["H64"]) < max(2e-2, 1.5 * dist_all)
+        ok = (g["gap"] > DECIDED) & route
         assert ok.mean() > 0.8
         assert np.array_equal(smp[0].cpu().numpy()[ok], g["sampled"][ok])
         kv.close()

@@ -45,15 +45,30 @@ def test_token_draw_range_ends_and_uniformity():
 
 
 def test_gumbel_moments():
-    # Gumbel(0, 1): mean = Euler-Mascheroni constant, variance = pi^2 / 6
+    # Gumbel(0, 1): mean = Euler-Mascheroni constant, variance = pi^2 / 6, for the even
+    # and the odd field alike, and the two fields of one output uncorrelated
     z = an.draw(an.stream_key(3, 2), np.arange(400_000))
-    g = an.gumbel_from_bits(z)
-    assert np.isfinite(g).all()
-    assert abs(g.mean() - 0.5772156649015329) < 0.01
-    assert abs(g.var() - math.pi ** 2 / 6) < 0.03
+    f = an.fields_of_bits(z)
+    for h in (0, 1):
+        g = an.gumbel_from_field(f[:, h])
+        assert np.isfinite(g).all()
+        assert abs(g.mean() - 0.5772156649015329) < 0.01
+        assert abs(g.var() - math.pi ** 2 / 6) < 0.03
+    assert abs(np.corrcoef(f[:, 0], f[:, 1])[0, 1]) < 0.01
     # u stays strictly inside (0, 1): the extreme codes give finite noise
-    ext = an.gumbel_from_bits(np.array([0, (1 << 64) - 1], dtype=np.uint64))
+    ext = an.gumbel_from_field(np.array([0, (1 << 23) - 1]))
     assert np.isfinite(ext).all() and ext[0] < ext[1]
+
+
+def test_fields_are_the_stated_bits():
+    z = np.array([(0b1011 << 60) | (0x7FFFFF << 41) | (0x1234 << 9) | 0x1FF], dtype=np.uint64)
+    f = an.fields_of_bits(z)[0]
+    assert int(f[0]) == ((0b1011 << 60) | (0x7FFFFF << 41)) >> 41
+    assert int(f[1]) == 0x1234
+    # odd vocabulary: the last token takes the even field of its own output
+    g = an.gumbel_row(4, 1, 2, 3, 5)
+    zz = an.draw(an.stream_key(4, 2), [(1 * 3 + 2) * 3 + 2])
+    assert g[4] == an.gumbel_from_field(an.fields_of_bits(zz)[:, 0])[0]
 
 
 # --- temperature, tempered statistics, Gumbel-max ---------------------------------------
@@ -90,8 +105,8 @@ def test_gumbel_max_draws_follow_the_tempered_softmax():
     p = np.exp(l / tau) / np.exp(l / tau).sum()
     counts = np.zeros(len(l))
     key = an.stream_key(11, 2)
-    z = an.draw(key, np.arange(n * len(l))).reshape(n, len(l))
-    g = an.gumbel_from_bits(z)
+    z = an.draw(key, np.arange(n * len(l) // 2))
+    g = an.gumbel_from_field(an.fields_of_bits(z).reshape(n, len(l)))
     for r in range(n):
         counts[an.gumbel_max(l / tau, g[r])[0]] += 1
     sd = np.sqrt(n * p * (1 - p))
