@@ -6,7 +6,8 @@ product path never does, and the two share no code (only the seeded input
 generators in `synth/`).
 
 Modules:
-  model     fp64 numpy forward: prefill, canvas forward, LM-head entropy
+  model     fp64 numpy forward: prefill, canvas forward, LM-head entropy, the
+            self-conditioning signal z = FFW(p0 E) and the block loops that carry it
   sampler   Entropy-Bound sampler step and block loop (integer decisions)
   anneal    the Report's default sampler: annealed entropy-bounded refinement over a
             uniform-noise canvas, adaptive stop, SplitMix64 draws

@@ -298,10 +298,37 @@ def canvas_layer(x, lw, kv, P: int, w: Workload):
     return decoder_layer(x, pos, lw, kv, allowed, w)
 
 
-def canvas_input(ws: Weights, canvas: np.ndarray, s: int, T: int) -> np.ndarray:
-    """Embedding of the canvas tokens ([MASK] has its own row) plus temb(s / T)."""
+def canvas_input(ws: Weights, canvas: np.ndarray, s: int, T: int, z=None) -> np.ndarray:
+    """Embedding of the canvas tokens ([MASK] has its own row) plus temb(s / T), plus the
+    self-conditioning signal z [C, d] when given."""
     w = ws.w
-    return embed(ws, canvas) + timestep_embedding(s / T, w.d_model)[None, :]
+    x = embed(ws, canvas) + timestep_embedding(s / T, w.d_model)[None, :]
+    return x if z is None else x + z
+
+
+def selfcond_mix(ws: Weights, logits: np.ndarray) -> np.ndarray:
+    """y = p0 E: the clean-token probabilities p0 = softmax(logits) (temperature 1, the
+    V real tokens) times the token embedding rows of those tokens
+    ("DiffusionGemma 技术报告" (full translation page), §3.2 "去噪迭代": the
+    self-conditioning signal is a feed-forward network of p0 times the embedding matrix;
+    §6: the embedding product runs over the whole vocabulary in full precision)."""
+    w = ws.w
+    l = np.asarray(logits, dtype=np.float64)
+    m = l.max(axis=1, keepdims=True)
+    p = np.exp(l - m)
+    p /= p.sum(axis=1, keepdims=True)
+    E = ws.get("tok_emb", (w.vocab + 1, w.d_model))[:w.vocab]
+    return p @ E
+
+
+def selfcond(ws: Weights, logits: np.ndarray) -> np.ndarray:
+    """z = FFW(p0 E) with FFW(y) = W_down (silu(W_gate y) * W_up y), the next forward's
+    self-conditioning input (same section; the FFW's form is this model's SwiGLU)."""
+    w = ws.w
+    d, I = w.d_model, w.sc_inter
+    y = ws.store(selfcond_mix(ws, logits))
+    return swiglu(y, ws.get("sc.gate", (I, d)), ws.get("sc.up", (I, d)),
+                  ws.get("sc.down", (d, I)), ws.store)
 
 
 def lm_head_stats(ws: Weights, x: np.ndarray, vocab_chunk: int = 16384, want_logits=False):
@@ -343,10 +370,11 @@ def entropy_stats(logits: np.ndarray):
 
 
 def denoise_forward(ws: Weights, kv_layers, canvas: np.ndarray, s: int, T: int, P: int,
-                    want_logits=False, want_hidden=False):
-    """Decoder forward over one canvas [C] at steps-left s; returns lm_head_stats."""
+                    want_logits=False, want_hidden=False, z=None):
+    """Decoder forward over one canvas [C] at steps-left s (self-conditioning input z, or
+    none); returns lm_head_stats."""
     w = ws.w
-    x = canvas_input(ws, canvas, s, T)
+    x = canvas_input(ws, canvas, s, T, z)
     routes = []
     for l in range(w.n_layers):
         x, _, _, r = canvas_layer(x, ws.layer(l), kv_layers[l], P, w)
@@ -359,7 +387,7 @@ def denoise_forward(ws: Weights, kv_layers, canvas: np.ndarray, s: int, T: int, 
 
 
 def prefill_then_forward(ws: Weights, prompt: np.ndarray, canvas: np.ndarray, s: int,
-                         T: int, want_logits=False):
+                         T: int, want_logits=False, z=None):
     """Prefill of one prompt and one canvas forward, interleaved layer by layer.
 
     Layer l of the canvas forward needs only the canvas state after layer l-1
@@ -369,7 +397,7 @@ def prefill_then_forward(ws: Weights, prompt: np.ndarray, canvas: np.ndarray, s:
     """
     w = ws.w
     P = prompt.shape[0]
-    x = canvas_input(ws, canvas, s, T)
+    x = canvas_input(ws, canvas, s, T, z)
     kv_layers, routes = [], []
     for l, kw, vw, lw in prefill_layer_by_layer(ws, prompt):
         kv_layers.append((kw, vw))
@@ -379,6 +407,49 @@ def prefill_then_forward(ws: Weights, prompt: np.ndarray, canvas: np.ndarray, s:
     st["routes"] = routes
     st["kv"] = kv_layers
     return st
+
+
+class CanvasForwards:
+    """The successive forwards of one block over a fixed context (cache kv of P
+    positions), carrying the self-conditioning signal between them when the model has
+    one: z = 0 at the block's first forward, afterwards z = selfcond(the previous
+    forward's logits) ("DiffusionGemma 技术报告" (full translation page), §3.2
+    "解码器前向传播" and "去噪迭代").  `zs` records the z each forward received."""
+
+    def __init__(self, ws: Weights, kv, P: int):
+        self.ws, self.kv, self.P = ws, kv, P
+        self.z = None
+        self.zs = []
+
+    def logits(self, canvas, s: int, T: int):
+        w = self.ws.w
+        self.zs.append(self.z)
+        st = denoise_forward(self.ws, self.kv, canvas, s, T, self.P, want_logits=True, z=self.z)
+        if w.sc_inter > 0:
+            self.z = selfcond(self.ws, st["logits"])
+        return st
+
+    def entropy_bound(self, T: int):
+        """forward(canvas, s) -> (H, argmax) for oracle.sampler.generate_block."""
+        def forward(canvas, s):
+            st = self.logits(canvas, s, T)
+            return st["H"], st["argmax"]
+        return forward
+
+    def annealed(self, N: int):
+        """forward(canvas, k) -> logits for oracle.anneal.generate_block."""
+        return lambda canvas, k: self.logits(canvas, N - k, N)["logits"]
+
+
+def generate_block(ws: Weights, prompt: np.ndarray, T: int, gamma: float):
+    """One all-[MASK] canvas denoised by the Entropy-Bound block loop after the causal
+    pass over the prompt (with self-conditioning when the model has it).  Returns
+    oracle.sampler.generate_block's (canvas, trajectory)."""
+    from oracle import sampler
+    w = ws.w
+    kv = prefill(ws, np.asarray(prompt, dtype=np.int64))
+    fw = CanvasForwards(ws, kv, len(prompt))
+    return sampler.generate_block(fw.entropy_bound(T), w.canvas, w.mask_id, T, gamma)
 
 
 def generate_blocks(ws: Weights, prompt: np.ndarray, n_blocks: int, T: int, gamma: float):
@@ -395,13 +466,9 @@ def generate_blocks(ws: Weights, prompt: np.ndarray, n_blocks: int, T: int, gamm
     blocks, trajs = [], []
     for _ in range(n_blocks):
         kv = prefill(ws, context)
-        P = len(context)
-
-        def forward(canvas, s, kv=kv, P=P):
-            st = denoise_forward(ws, kv, canvas, s, T, P)
-            return st["H"], st["argmax"]
-
-        canvas, traj = sampler.generate_block(forward, w.canvas, w.mask_id, T, gamma)
+        fw = CanvasForwards(ws, kv, len(context))
+        canvas, traj = sampler.generate_block(fw.entropy_bound(T), w.canvas, w.mask_id, T,
+                                              gamma)
         blocks.append(canvas)
         trajs.append(traj)
         context = np.concatenate([context, canvas])
@@ -419,9 +486,5 @@ def generate_block_annealed(ws: Weights, prompt: np.ndarray, seed: int, params=N
     p = params or anneal.Params()
     w = ws.w
     kv = prefill(ws, np.asarray(prompt, dtype=np.int64))
-    P = len(prompt)
-
-    def forward(canvas, k):
-        return denoise_forward(ws, kv, canvas, p.N - k, p.N, P, want_logits=True)["logits"]
-
-    return anneal.generate_block(forward, w.canvas, w.vocab, seed, p)
+    fw = CanvasForwards(ws, kv, len(prompt))
+    return anneal.generate_block(fw.annealed(p.N), w.canvas, w.vocab, seed, p)

@@ -43,7 +43,11 @@ def layer_specs(w: Workload, l: int):
 
 
 def global_specs(w: Workload):
-    return [("tok_emb", (w.vocab + 1, w.d_model)), ("lm_head", (w.vocab, w.d_model))]
+    out = [("tok_emb", (w.vocab + 1, w.d_model)), ("lm_head", (w.vocab, w.d_model))]
+    if w.sc_inter > 0:  # the self-conditioning FFW
+        out += [("sc.gate", (w.sc_inter, w.d_model)), ("sc.up", (w.sc_inter, w.d_model)),
+                ("sc.down", (w.d_model, w.sc_inter))]
+    return out
 
 
 def all_specs(w: Workload):
@@ -57,9 +61,15 @@ def store_dtype(w: Workload) -> str:
     return "f32" if w.dtype == "f32" else "bf16"
 
 
+def std_of(w: Workload, name: str) -> float:
+    """Standard deviation a tensor is drawn with: the self-conditioning FFW's own (test
+    workloads raise it so that the signal reaches the next forward), else init_std."""
+    return w.sc_std if name.startswith("sc.") else w.init_std
+
+
 def weight(w: Workload, name: str, shape, device="cpu", start_row=0, n_rows=None):
     """Stored (un-quantised) values of one weight tensor or a row range of it."""
-    return gen.weight(w.seed, name, shape, w.init_std, store_dtype(w), device,
+    return gen.weight(w.seed, name, shape, std_of(w, name), store_dtype(w), device,
                       start_row, n_rows)
 
 
@@ -79,7 +89,8 @@ def block_tokens(w: Workload, device="cpu", first: int = 0) -> torch.Tensor:
 
 
 def is_fp8_expert(w: Workload, name: str) -> bool:
-    return w.dtype == "bf16_fp8exp" and name.split(".")[-1] in ("gate", "up", "down")
+    return (w.dtype == "bf16_fp8exp" and name.startswith("l")
+            and name.split(".")[-1] in ("gate", "up", "down"))
 
 
 def weight_set(w: Workload, device="cpu") -> dict:
@@ -93,6 +104,6 @@ def weight_set(w: Workload, device="cpu") -> dict:
             out[name], out[name.rsplit(".", 1)[0] + "." + name.split(".")[-1] + "_scale"] = q, s
             continue
         t = torch.empty(shape, dtype=dt, device=device)
-        gen.fill_weight_(t, w.seed, name, w.init_std)
+        gen.fill_weight_(t, w.seed, name, std_of(w, name))
         out[name] = t
     return out

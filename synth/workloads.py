@@ -39,6 +39,8 @@ class Workload:
     gamma: float          # entropy bound of the sampler
     seed: int = 0
     init_std: float = 0.02
+    sc_inter: int = 0     # self-conditioning FFW inner size (0: no self-conditioning)
+    sc_std: float = 0.02  # standard deviation of the self-conditioning FFW's weights
 
     @property
     def mask_id(self) -> int:
@@ -108,9 +110,17 @@ LAYER1_P200_B2_C96 = LAYER1_P200_B2.with_(name="layer1-bf16-p200-b2-c96", canvas
 LAYER1_FP8_B16 = LAYER1_FP8.with_(name="layer1-fp8exp-p4096-b16", batch=16)
 LAYER1_FP8_B64 = LAYER1_FP8.with_(name="layer1-fp8exp-p4096-b64", batch=64)
 
+# Self-conditioning variants (the Report's decoder input z = FFW(p0 E)): the FFW inner
+# size of the full-size model is the shared expert's.
+TINY_F32_SC = TINY_F32.with_(name="tiny-f32-sc", sc_inter=128, sc_std=4.0)
+SMALL_BF16_SC = SMALL_BF16.with_(name="small-bf16-sc", sc_inter=192, sc_std=1.0)
+LAYER1_BF16_SC = LAYER1_BF16.with_(name="layer1-bf16-sc", sc_inter=2048)
+FULL30_BF16_SC = FULL30_BF16.with_(name="full30-bf16-sc", sc_inter=2048)
+
 WORKLOADS = {w.name: w for w in (TINY_F32, SMALL_BF16, LAYER1_BF16, FULL30_BF16,
                                  FULL30_B8_P8192, SMALL_FP8, LAYER1_FP8, LAYER1_P200_B2,
-                                 LAYER1_P200_B2_C96, LAYER1_FP8_B16, LAYER1_FP8_B64)}
+                                 LAYER1_P200_B2_C96, LAYER1_FP8_B16, LAYER1_FP8_B64,
+                                 TINY_F32_SC, SMALL_BF16_SC, LAYER1_BF16_SC, FULL30_BF16_SC)}
 for _b in (1, 4, 16, 32, 64):
     WORKLOADS[f"full30-fp8exp-b{_b}"] = full30_fp8exp(_b)
 
