@@ -339,6 +339,63 @@ def run_annealed(args, w, world, model, prompt, eb_lmhead_ms):
                      "stop does not fire and every block runs N forwards")}
 
 
+def run_selfcond(args, w, world, tensors, prompt, eb):
+    """The same blocks with self-conditioning (the Report's decoder input z = FFW(p0 E),
+    p0 over the whole vocabulary): a second handle on the same weights plus the FFW's
+    three tensors (sc_inter = 2048, init std 0.02), device-timed graph replays of
+    dg_generate_block, then a profiled pass for the LM head's share (the p0 store, the
+    rescale, the K-sliced p0 E^T GEMM and the FFW run inside that group)."""
+    import torch
+
+    from masked_discrete_diffusion_b200 import binding
+    from synth import gen, model_inputs, workloads
+    ws = w.with_(name=w.name + "-sc", sc_inter=2048)
+    sc = {}
+    for name, shape in model_inputs.global_specs(ws):
+        if name.startswith("sc."):
+            t = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
+            gen.fill_weight_(t, ws.seed, name, model_inputs.std_of(ws, name))
+            sc[name] = t
+    model = binding.Model(binding.make_config(ws, max_prompt=w.prompt_len), dict(tensors, **sc))
+    try:
+        B, C = w.batch, w.canvas
+        kv = binding.dg_prefill(model, prompt)
+        out = torch.empty(B, C, dtype=torch.int32, device="cuda")
+        nf = torch.zeros(B, dtype=torch.int32, device="cuda")
+        for _ in range(max(args.warmup, 1)):
+            binding.dg_generate_block(model, kv, w.T, w.gamma, out, nf)
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.nvtx.range_push("selfcond")
+        e0.record()
+        for _ in range(args.steps):
+            binding.dg_generate_block(model, kv, w.T, w.gamma, out, nf)
+        e1.record()
+        e1.synchronize()
+        torch.cuda.nvtx.range_pop()
+        ms_max = max_over_ranks(e0.elapsed_time(e1), world)
+        fwd = int(nf.max().item())
+        binding.dg_profile_start(model, fwd)
+        binding.dg_generate_block(model, kv, w.T, w.gamma, out, nf)
+        torch.cuda.synchronize()
+        prof = binding.dg_profile_stop(model)
+        binding.dg_sync_status(model)
+        assert not bool((out == w.mask_id).any()), "a [MASK] survived the block"
+        kv.close()
+    finally:
+        model.close()
+    lm_ms, lm_n = prof["lmhead"]
+    return {"sc_inter": 2048, "steps": args.steps,
+            "canvas_tokens_per_s": job_throughput(world, B * C, args.steps, ms_max),
+            "ms_per_block": ms_max / args.steps, "forwards_per_block": fwd,
+            "ms_per_forward": ms_max / args.steps / max(fwd, 1),
+            "lmhead_with_selfcond_ms_per_forward": lm_ms / max(lm_n, 1),
+            "lmhead_ms_per_forward_without": eb,
+            "note": "the LM-head group also holds the p0 store and rescale, the p0 E^T GEMM "
+                    "(16 K slices) and the SwiGLU FFW of z"}
+
+
 def run_ours(args, w, world, rank, local):
     import numpy as np
     import torch
@@ -415,6 +472,10 @@ def run_ours(args, w, world, rank, local):
     if not args.skip_e2e:
         e2e_val = run_e2e(args, w, world, model, prompt, canvas, stream)
     blocks = run_blocks(args, w, world, model, prompt) if args.blocks > 1 else None
+    selfcond = None
+    if args.selfcond and w.dtype == "bf16":
+        selfcond = run_selfcond(args, w, world, tensors, prompt,
+                                prof["lmhead"][0] / max(prof["lmhead"][1], 1))
     annealed = None
     if args.annealed > 0:
         annealed = run_annealed(args, w, world, model, prompt,
@@ -484,6 +545,7 @@ def run_ours(args, w, world, rank, local):
         "experts_streamed_per_layer_forward": unique_mean,
         "blocks": blocks,
         "annealed": annealed,
+        "selfcond": selfcond,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         t_block, desc, threads = OracleSample(w).run()
@@ -503,6 +565,8 @@ def main():
     ap.add_argument("--workload", default="full30-bf16")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--selfcond", type=int, default=1,
+                    help="1: also time the blocks with self-conditioning (bf16 workloads)")
     ap.add_argument("--annealed", type=int, default=1,
                     help="timed blocks of the annealed sampler (0: skip that leg)")
     ap.add_argument("--blocks", type=int, default=2,

@@ -72,6 +72,7 @@ typedef struct dg_config {
   int32_t dtype;       /* dg_dtype                                            */
   int32_t max_batch;   /* largest B any call on this model will pass          */
   int32_t max_prompt;  /* largest P any dg_prefill on this model will pass    */
+  int32_t sc_inter;    /* inner size of the self-conditioning FFW; 0: none    */
 } dg_config;
 
 /* Weights of one layer (device pointers, borrowed for the model's lifetime).
@@ -97,6 +98,11 @@ typedef struct dg_weights {
   const void* tok_emb;            /* [V + 1, d]; row V embeds [MASK]           */
   const void* lm_head;            /* [V, d] (untied)                           */
   const dg_layer_weights* layers; /* HOST array of n_layers entries, copied    */
+  /* The self-conditioning FFW (sc_inter > 0; else ignored): z = sc_down (silu(sc_gate y)
+   * * (sc_up y)) for y = p0 E ("DiffusionGemma 技术报告", §3.2 "去噪迭代").        */
+  const void* sc_gate;            /* [sc_inter, d]                              */
+  const void* sc_up;              /* [sc_inter, d]                              */
+  const void* sc_down;            /* [d, sc_inter]                              */
 } dg_weights;
 
 typedef struct dg_model dg_model;
@@ -267,6 +273,27 @@ dg_status dg_anneal_sample(const float* entropy, const int32_t* argmax, const in
  * seeds [B]; prev_argmax [B, C] set to -1 and state [B] to 0 (both nullable). */
 dg_status dg_anneal_init(int32_t* canvas, int32_t* prev_argmax, int32_t* state, int32_t B,
                          int32_t C, int32_t V, const uint64_t* seeds, void* stream);
+
+/* ---- self-conditioning ("DiffusionGemma 技术报告", §3.2 "解码器前向传播", "去噪迭代";
+ * models created with sc_inter > 0) -------------------------------------------------
+ * After a forward the decoder's clean-token probabilities p0 = softmax(l) (temperature
+ * 1, the V real tokens) are mixed with the embedding rows, y = p0 E, and
+ * z = sc_down (silu(sc_gate y) * (sc_up y)) is added to the canvas rows' input of the
+ * next forward.  The block calls (dg_generate_block, dg_generate_blocks,
+ * dg_generate_block_annealed) carry z from forward to forward, 0 at a block's first, as
+ * long as it is switched on (the default for such models); dg_denoise_step,
+ * dg_debug_forward and dg_anneal_forward run without it (z = 0). */
+
+/* Switches the block calls' self-conditioning on (on != 0; needs sc_inter > 0) or off. */
+dg_status dg_set_selfcond(dg_model* m, int32_t on);
+
+/* One Entropy-Bound forward with self-conditioning: z_in [B, C, d] is added to the
+ * canvas rows' input (NULL: none), entropy/argmax as in dg_denoise_step, and the next
+ * forward's z written to z_out [B, C, d] (may equal z_in).  z is in the accumulate type:
+ * fp64 for DG_F32 models, fp32 otherwise.  Requires sc_inter > 0. */
+dg_status dg_selfcond_forward(dg_model* m, const dg_kv* kv, const int32_t* canvas,
+                              int32_t steps_left, int32_t T, const void* z_in, float* entropy,
+                              int32_t* argmax, void* z_out, void* stream);
 
 /* Test hook: the forward of dg_denoise_step without the sampler.  Writes
  * entropy/argmax as above and, when non-NULL, the logits [B*C, V] fp32 and the

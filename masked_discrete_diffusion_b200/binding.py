@@ -33,7 +33,8 @@ class dg_config(ctypes.Structure):
         "expert_inter", "shared_inter", "vocab", "window", "canvas")] + [
         ("rope_base", ctypes.c_float), ("rms_eps", ctypes.c_float),
         ("logit_scale", ctypes.c_float), ("dtype", ctypes.c_int32),
-        ("max_batch", ctypes.c_int32), ("max_prompt", ctypes.c_int32)]
+        ("max_batch", ctypes.c_int32), ("max_prompt", ctypes.c_int32),
+        ("sc_inter", ctypes.c_int32)]
 
 
 _LAYER_FIELDS = ("wqkv", "wo", "router", "gate", "up", "down", "gate_scale", "up_scale",
@@ -46,7 +47,8 @@ class dg_layer_weights(ctypes.Structure):
 
 class dg_weights(ctypes.Structure):
     _fields_ = [("tok_emb", ctypes.c_void_p), ("lm_head", ctypes.c_void_p),
-                ("layers", ctypes.POINTER(dg_layer_weights))]
+                ("layers", ctypes.POINTER(dg_layer_weights)), ("sc_gate", ctypes.c_void_p),
+                ("sc_up", ctypes.c_void_p), ("sc_down", ctypes.c_void_p)]
 
 
 _lib = None
@@ -126,6 +128,8 @@ def lib() -> ctypes.CDLL:
             "dg_anneal_sample": [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32,
                                  ctypes.POINTER(dg_anneal_params), vp, vp],
             "dg_anneal_init": [vp, vp, vp, i32, i32, i32, vp, vp],
+            "dg_set_selfcond": [vp, i32],
+            "dg_selfcond_forward": [vp, vp, vp, i32, i32, vp, vp, vp, vp, vp],
         }
         for name, args in sigs.items():
             fn = getattr(L, name)
@@ -144,7 +148,8 @@ def exported_symbols():
                         "dg_lmhead_entropy_noalloc", "dg_block_loop_launches",
                         "dg_debug_stall_experts", "dg_prefill_into", "dg_append_block",
                         "dg_generate_blocks", "dg_generate_block_annealed",
-                        "dg_anneal_forward", "dg_anneal_sample", "dg_anneal_init")
+                        "dg_anneal_forward", "dg_anneal_sample", "dg_anneal_init",
+                        "dg_set_selfcond", "dg_selfcond_forward")
             if hasattr(lib(), n)]
 
 
@@ -177,7 +182,7 @@ def make_config(w, max_batch: int | None = None, max_prompt: int | None = None) 
         shared_inter=w.shared_inter, vocab=w.vocab, window=w.window, canvas=w.canvas,
         rope_base=w.rope_base, rms_eps=w.rms_eps, logit_scale=w.logit_scale,
         dtype=_DTYPES[w.dtype], max_batch=max_batch or w.batch,
-        max_prompt=max_prompt or w.prompt_len)
+        max_prompt=max_prompt or w.prompt_len, sc_inter=getattr(w, "sc_inter", 0))
 
 
 class Model:
@@ -193,7 +198,8 @@ class Model:
             for f in _LAYER_FIELDS:
                 setattr(self._layers[l], f, _ptr(tensors.get(f"l{l}.{f}")))
         self._w = dg_weights(tok_emb=_ptr(tensors["tok_emb"]), lm_head=_ptr(tensors["lm_head"]),
-                             layers=self._layers)
+                             layers=self._layers, sc_gate=_ptr(tensors.get("sc.gate")),
+                             sc_up=_ptr(tensors.get("sc.up")), sc_down=_ptr(tensors.get("sc.down")))
         h = ctypes.c_void_p()
         _check(lib().dg_model_create(ctypes.byref(cfg), ctypes.byref(self._w), ctypes.byref(h)))
         self.handle = h
@@ -379,6 +385,27 @@ def dg_anneal_init(B: int, C: int, V: int, seeds, stream=None):
     _check(lib().dg_anneal_init(_ptr(canvas), _ptr(prev), _ptr(state), B, C, V, _ptr(sd),
                                 _stream(stream)))
     return canvas, prev, state
+
+
+def dg_set_selfcond(model: Model, on: bool):
+    _check(lib().dg_set_selfcond(model.handle, 1 if on else 0))
+
+
+def dg_selfcond_forward(model: Model, kv: KV, canvas, steps_left: int, T: int, z_in=None,
+                        stream=None):
+    """(entropy [B, C], argmax [B, C], z_out [B, C, d]); z in the model's accumulate type
+    (float64 for the fp32 model, float32 otherwise)."""
+    c = model.cfg
+    B, C = canvas.shape
+    zt = torch.float64 if c.dtype == _DTYPES["f32"] else torch.float32
+    if z_in is not None and (z_in.dtype != zt or tuple(z_in.shape) != (B, C, c.d_model)):
+        raise ValueError(f"z_in must be {zt} of shape {(B, C, c.d_model)}")
+    H = torch.empty(B, C, dtype=torch.float32, device="cuda")
+    am = torch.empty(B, C, dtype=torch.int32, device="cuda")
+    z_out = torch.empty(B, C, c.d_model, dtype=zt, device="cuda")
+    _check(lib().dg_selfcond_forward(model.handle, kv.handle, _ptr(canvas), steps_left, T,
+                                     _ptr(z_in), _ptr(H), _ptr(am), _ptr(z_out), _stream(stream)))
+    return H, am, z_out
 
 
 def dg_debug_forward(model: Model, kv: KV, canvas, steps_left: int, T: int, logits=False,

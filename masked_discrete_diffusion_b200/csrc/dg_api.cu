@@ -103,6 +103,7 @@ __global__ void rope_table_kernel(double base, int h, int max_pos, void* out, in
 }
 
 template <class Path> static dg_status alloc_workspace(dg_model* m) {
+  typedef typename Path::TW TW;
   typedef typename Path::TA TA;
   typedef typename Path::Acc Acc;
   typedef typename Path::TR TR;
@@ -167,6 +168,20 @@ template <class Path> static dg_status alloc_workspace(dg_model* m) {
   DG_TRY(ws_alloc(ws, &ws.prev, lm_rows));
   DG_TRY(ws_alloc(ws, &ws.astate, c.max_batch));
   DG_TRY(ws_alloc_v<Acc>(ws, &ws.gpart, (size_t)ws.n_vtiles * lm_rows * 2));
+  if (c.sc_inter > 0) {
+    DG_TRY(ws_alloc_v<TW>(ws, &ws.embT, d * c.vocab));
+    DG_TRY(ws_alloc_v<TA>(ws, &ws.scP, lm_rows * c.vocab));
+    DG_TRY(ws_alloc_v<Acc>(ws, &ws.scref, (size_t)ws.n_vtiles * lm_rows * 2));
+    DG_TRY(ws_alloc_v<TA>(ws, &ws.scy, T * d));  // max_tok rows: the GEMMs' A extent
+    DG_TRY(ws_alloc_v<TA>(ws, &ws.sch, T * c.sc_inter));
+    if constexpr (Path::kTensorCores)
+      DG_TRY(ws_alloc(ws, &ws.scpart, (size_t)SC_MAX_PARTS * lm_rows * d));
+    DG_TRY(ws_alloc_v<Acc>(ws, &ws.z, lm_rows * d));
+    dim3 tg(ceil_div(c.vocab, 32), ceil_div((long)d, 32));
+    transpose_emb_kernel<TW><<<tg, dim3(32, 8)>>>((const TW*)m->w.tok_emb, (TW*)ws.embT,
+                                                  c.vocab, (int)d);
+    DG_TRY(check_launch("embedding transpose"));
+  }
   DG_TRY_CUDA(cudaMemset(ws.err, 0, 4 * sizeof(int32_t)));
   launch_pdl((rope_table_kernel), 256, 256, 0, cudaStream_t(0), 1, (double)c.rope_base, (int)h, ws.max_pos, ws.rope,
                                   sizeof(Acc) == 8 ? 1 : 0);
@@ -452,9 +467,9 @@ template <class Path> struct Runner {
     const int Pp = (P + 63) / 64 * 64;
     const size_t es = sizeof(TKV);
     for (int b = 0; b < B; ++b) {
-      launch_pdl((embed_kernel<TW, TR>), P, 256, 0, st, 1, prompt + (size_t)b * P, (const TW*)m->w.tok_emb,
+      launch_pdl((embed_kernel<TW, TR, Acc>), P, 256, 0, st, 1, prompt + (size_t)b * P, (const TW*)m->w.tok_emb,
                                              x(), P, d, c.vocab - 1, -1.0, ws.err,
-                                             (const int32_t*)nullptr, 1);
+                                             (const int32_t*)nullptr, 1, (const Acc*)nullptr);
       ++m->launches;
       // padding columns of the transposed values must read as zero
       DG_TRY_CUDA(cudaMemsetAsync(ws.vc, 0, (size_t)Hkv * h * Pp * es, st));
@@ -487,8 +502,8 @@ template <class Path> struct Runner {
     const int Hkv = c.n_kv_heads;
     const int np = (C + 63) / 64 * 64;
     const size_t es = sizeof(TKV);
-    launch_pdl((embed_kernel<TW, TR>), n, 256, 0, st, 1, tokens, (const TW*)m->w.tok_emb, x(), n,
-               d, c.vocab - 1, -1.0, ws.err, (const int32_t*)nullptr, 1);
+    launch_pdl((embed_kernel<TW, TR, Acc>), n, 256, 0, st, 1, tokens, (const TW*)m->w.tok_emb, x(), n,
+               d, c.vocab - 1, -1.0, ws.err, (const int32_t*)nullptr, 1, (const Acc*)nullptr);
     ++m->launches;
     // padding columns of the block's transposed values must read as zero
     if (np != C) DG_TRY_CUDA(cudaMemsetAsync(ws.vc, 0, (size_t)B * Hkv * h * np * es, st));
@@ -532,15 +547,18 @@ template <class Path> struct Runner {
 
   // Canvas forward: statistics into ent/amax; optional logits/hidden (test hook).
   // With an.N > 0: tempered statistics and (an.seeds) the Gumbel-max draw into sampled.
+  // With z_in: the self-conditioning signal added to the canvas rows' input; with z_out
+  // (self-conditioned models): z = FFW(p0 E) of this forward's logits written there.
   dg_status forward(const dg_kv* kv, const int32_t* canvas, int s, int T, float* ent,
                     int32_t* amax, float* logits, float* hidden, int32_t* load,
-                    const AnnealDev& an = AnnealDev{}, int32_t* sampled = nullptr) {
+                    const AnnealDev& an = AnnealDev{}, int32_t* sampled = nullptr,
+                    const Acc* z_in = nullptr, Acc* z_out = nullptr) {
     const int B = kv->B, C = c.canvas, n = B * C, d = c.d_model;
     const double tau = (double)s / (double)T;
     {
       ProfScope ps(m, DG_KIND_GLUE, st);
-      launch_pdl((embed_kernel<TW, TR>), n, 256, 0, st, 1, canvas, (const TW*)m->w.tok_emb, x(), n,
-                 d, c.vocab, tau, ws.err, (const int32_t*)s_dev, T);
+      launch_pdl((embed_kernel<TW, TR, Acc>), n, 256, 0, st, 1, canvas, (const TW*)m->w.tok_emb, x(), n,
+                 d, c.vocab, tau, ws.err, (const int32_t*)s_dev, T, z_in);
       ++m->launches;
     }
     const int Cp = (C + 63) / 64 * 64;
@@ -555,10 +573,16 @@ template <class Path> struct Runner {
     }
     // xn = RMSNorm(x): written by the last layer's combine
     ProfScope ps(m, DG_KIND_LMHEAD, st);
+    ScDev sc;
+    if (z_out) {
+      sc.P = ws.scP;
+      sc.ref = ws.scref;
+      sc.ldp = c.vocab;
+    }
     bool done = false;
     if constexpr (Path::kTensorCores) {
       if (logits == nullptr) {
-        DG_TRY(tc_lmhead_stats(m, xn(), n, ent, amax, st, an, sampled));
+        DG_TRY(tc_lmhead_stats(m, xn(), n, ent, amax, st, an, sampled, sc));
         done = true;
       }
     }
@@ -566,15 +590,34 @@ template <class Path> struct Runner {
       dim3 grid(ws.n_vtiles, ceil_div(n, SG_BM));
       launch_pdl((lmhead_simt_kernel<TA, TW, Acc>), grid, 256, 0, st, 1, xn(), (const TW*)m->w.lm_head, n,
                                                            c.vocab, d, c.logit_scale,
-                                                           (Acc*)ws.lm_part, logits, an);
+                                                           (Acc*)ws.lm_part, logits, an, sc);
       ++m->launches;
-      launch_pdl((lm_merge_kernel<Acc>), n, 128, 0, st, 1, (const Acc*)ws.lm_part, ws.n_vtiles,
+      launch_pdl((lm_merge_kernel<Acc, TA>), n, 128, 0, st, 1, (const Acc*)ws.lm_part, ws.n_vtiles,
                                                           n, ent, amax,
                                                           (const Acc*)(an.seeds ? an.gpart : nullptr),
-                                                          an.seeds ? sampled : nullptr);
+                                                          an.seeds ? sampled : nullptr, sc, SG_BN);
       ++m->launches;
     }
+    if (z_out) DG_TRY(selfcond(n, z_out));
     return check_launch("forward");
+  }
+
+  // z = W_down (silu(W_gate y) * W_up y) for y = p0 E, p0 left by the LM head
+  dg_status selfcond(int n, Acc* z_out) {
+    const int d = c.d_model, V = c.vocab, I = c.sc_inter;
+    if constexpr (Path::kTensorCores) {
+      DG_TRY(tc_selfcond_mix(m, n, st));
+      DG_TRY(tc_gemm_swiglu(m, (const TA*)ws.scy, m->w.sc_gate, m->w.sc_up, (TA*)ws.sch, n, I, d,
+                            st));
+      DG_TRY(tc_gemm_store_f32(m, (const TA*)ws.sch, m->w.sc_down, (float*)z_out, n, d, I, st));
+    } else {
+      dense((const TA*)ws.scP, V, ws.embT, d, V, n, EpiStore<TA, Acc>{(TA*)ws.scy, d});
+      gemm_simt<TA, TW, Acc, false, true>((const TA*)ws.scy, d, (const TW*)m->w.sc_gate,
+                                          (const TW*)m->w.sc_up, d, n, I, d, GroupInfo(), 0,
+                                          EpiSwiglu<TA, Acc>{(TA*)ws.sch, I}, st, &m->launches);
+      dense((const TA*)ws.sch, I, m->w.sc_down, d, I, n, EpiStore<Acc, Acc>{z_out, d});
+    }
+    return check_launch("self-conditioning");
   }
 };
 
@@ -676,6 +719,16 @@ dg_status dg_model_create(const dg_config* cfg, const dg_weights* w, dg_model** 
     DG_REQUIRE(c.d_model % 128 == 0 && c.expert_inter % 128 == 0,
                "FP8 experts need d and I multiples of 128 (one scale per 128 columns)");
   DG_REQUIRE(w->tok_emb && w->lm_head && w->layers, "null weight pointer");
+  DG_REQUIRE(c.sc_inter >= 0, "sc_inter must be >= 0");
+  if (c.sc_inter > 0) {
+    DG_REQUIRE(w->sc_gate && w->sc_up && w->sc_down, "null self-conditioning weight pointer");
+    const int tile = c.dtype == DG_F32 ? SG_BN : 256;
+    DG_REQUIRE((c.vocab + tile - 1) / tile <= LM_SC_MAX_TILES,
+               "self-conditioning spans at most %d vocabulary tiles of %d", LM_SC_MAX_TILES, tile);
+    if (c.dtype != DG_F32)
+      DG_REQUIRE(c.sc_inter % 64 == 0 && c.vocab % 8 == 0,
+                 "self-conditioning on tensor cores needs sc_inter %% 64 == 0 and V %% 8 == 0");
+  }
   for (int l = 0; l < c.n_layers; ++l) {
     const dg_layer_weights& L = w->layers[l];
     DG_REQUIRE(L.wqkv && L.wo && L.router && L.gate && L.up && L.down && L.sgate && L.sup &&
@@ -690,6 +743,7 @@ dg_status dg_model_create(const dg_config* cfg, const dg_weights* w, dg_model** 
   m->layers.assign(w->layers, w->layers + c.n_layers);
   m->w.layers = nullptr;
   cudaGetDevice(&m->device);
+  m->selfcond = c.sc_inter > 0;
   {
     const char* env = getenv("DG_NO_GRAPHS");
     m->use_graphs = !(env && env[0] && env[0] != '0');
@@ -863,15 +917,30 @@ static dg_status check_step_args(dg_model* m, const dg_kv* kv, int s, int T) {
   return DG_OK;
 }
 
+// z_in / z_out: the self-conditioning signal in the path's accumulate type (fp64 for
+// the fp32 model, fp32 otherwise); nullptr: none in / none computed.
 static dg_status run_forward(dg_model* m, const dg_kv* kv, const int32_t* canvas, int s, int T,
                              float* ent, int32_t* am, float* logits, float* hidden,
                              int32_t* load, cudaStream_t st, const int32_t* s_dev = nullptr,
-                             const AnnealDev& an = AnnealDev{}, int32_t* sampled = nullptr) {
+                             const AnnealDev& an = AnnealDev{}, int32_t* sampled = nullptr,
+                             const void* z_in = nullptr, void* z_out = nullptr) {
   return m->cfg.dtype == DG_F32
              ? Runner<PathTiny>(m, st, s_dev).forward(kv, canvas, s, T, ent, am, logits, hidden,
-                                                      load, an, sampled)
+                                                      load, an, sampled, (const double*)z_in,
+                                                      (double*)z_out)
              : Runner<PathBF16>(m, st, s_dev).forward(kv, canvas, s, T, ent, am, logits, hidden,
-                                                      load, an, sampled);
+                                                      load, an, sampled, (const float*)z_in,
+                                                      (float*)z_out);
+}
+
+// The block loops' z buffer (nullptr when the model runs without self-conditioning).
+static void* loop_z(dg_model* m) { return m->selfcond ? m->ws.z : nullptr; }
+
+static dg_status zero_loop_z(dg_model* m, int B, cudaStream_t st) {
+  if (!m->selfcond) return DG_OK;
+  const size_t es = m->cfg.dtype == DG_F32 ? sizeof(double) : sizeof(float);
+  DG_TRY_CUDA(cudaMemsetAsync(m->ws.z, 0, (size_t)B * m->cfg.canvas * m->cfg.d_model * es, st));
+  return DG_OK;
 }
 
 dg_status dg_denoise_step(dg_model* m, const dg_kv* kv, int32_t* canvas, uint8_t* mask,
@@ -898,6 +967,7 @@ static dg_status generate_impl(dg_model* m, const dg_kv* kv, int32_t T, long lon
   launch_pdl((fill_i32_kernel), ceil_div((long)B * C, 256), 256, 0, st, 1, canvas_out, B * C, c.vocab);
   ++m->launches;
   DG_TRY_CUDA(cudaMemsetAsync(ws.mask, 1, (size_t)B * C, st));
+  DG_TRY(zero_loop_z(m, B, st));
   if (n_forwards) DG_TRY_CUDA(cudaMemsetAsync(n_forwards, 0, B * sizeof(int32_t), st));
   if (router_load)
     DG_TRY_CUDA(cudaMemsetAsync(router_load, 0,
@@ -906,7 +976,7 @@ static dg_status generate_impl(dg_model* m, const dg_kv* kv, int32_t T, long lon
   for (int k = 0; k < nfw; ++k) {
     const int s = T - k;
     DG_TRY(run_forward(m, kv, canvas_out, s, T, ws.ent, ws.amax, nullptr, nullptr, router_load,
-                       st));
+                       st, nullptr, AnnealDev{}, nullptr, loop_z(m), loop_z(m)));
     ProfScope ps(m, DG_KIND_GLUE, st);
     DG_TRY(launch_sampler(ws.ent, ws.amax, canvas_out, ws.mask, B, C, s, gq, ws.ncommit,
                           n_forwards, k + 1, st, &m->launches));
@@ -995,10 +1065,12 @@ static bool build_loop_graph(dg_model* m, const dg_kv* kv, int32_t T, long long 
         launch_pdl((block_init_kernel), ceil_div(std::max(n, n_load), 256), 256, 0, cap, 1,
                    canvas_out, ws.mask, n, (int32_t)c.vocab, n_forwards, B, router_load, n_load,
                    ws.loop_s, T);
+        zero_loop_z(m, B, cap);
       },
       [&](cudaStream_t cap) {
         dg_status s = run_forward(m, kv, canvas_out, T, T, ws.ent, ws.amax, nullptr, nullptr,
-                                  router_load, cap, ws.loop_s);
+                                  router_load, cap, ws.loop_s, AnnealDev{}, nullptr, loop_z(m),
+                                  loop_z(m));
         if (s == DG_OK)
           s = launch_sampler(ws.ent, ws.amax, canvas_out, ws.mask, B, C, T, gq, ws.ncommit,
                              n_forwards, 1, cap, &m->launches, ws.loop_s, T, ws.remaining);
@@ -1015,8 +1087,8 @@ static dg_status generate_graphed(dg_model* m, const dg_kv* kv, int32_t T, long 
                                   int32_t* router_load, cudaStream_t st) {
   dg::BlockGraph* g = nullptr;
   for (auto* x : m->graphs)
-    if (!x->anneal && x->kv == kv && x->kv_P == kv->P && x->kv_W == kv->W && x->T == T &&
-        x->gq == gq &&
+    if (!x->anneal && x->sc == m->selfcond && x->kv == kv && x->kv_P == kv->P &&
+        x->kv_W == kv->W && x->T == T && x->gq == gq &&
         x->canvas == canvas_out &&
         x->nfwd == n_forwards && x->load == router_load && x->prof == m->profiling &&
         (!x->prof || x->fcap == m->prof_forwards)) {
@@ -1039,6 +1111,7 @@ static dg_status generate_graphed(dg_model* m, const dg_kv* kv, int32_t T, long 
     g->load = router_load;
     g->prof = m->profiling;
     g->fcap = m->profiling ? m->prof_forwards : 0;
+    g->sc = m->selfcond;
     // capture on a library-owned stream (the caller's may be the legacy default
     // stream, which cannot be captured); nothing executes during capture
     if (!m->cap_stream) DG_TRY_CUDA(cudaStreamCreateWithFlags(&m->cap_stream, cudaStreamNonBlocking));
@@ -1221,12 +1294,14 @@ static dg_status anneal_impl(dg_model* m, const dg_kv* kv, const dg_anneal_param
                ws.prev, ws.astate, n_forwards, B, C, V, (const unsigned long long*)seeds,
                (int32_t*)nullptr, p->N);
     ++m->launches;
+    DG_TRY(zero_loop_z(m, B, st));
   }
   const int nfw = fcap > 0 ? std::min(fcap, (int)p->N) : (int)p->N;
   for (int k = 0; k < nfw; ++k) {
     const int s = p->N - k;
     DG_TRY(run_forward(m, kv, canvas_out, s, p->N, ws.ent, ws.amax, nullptr, nullptr, nullptr,
-                       st, nullptr, anneal_dev(m, p, seeds, s, nullptr), ws.sampled));
+                       st, nullptr, anneal_dev(m, p, seeds, s, nullptr), ws.sampled, loop_z(m),
+                       loop_z(m)));
     ProfScope ps(m, DG_KIND_GLUE, st);
     DG_TRY(launch_anneal(ws.ent, ws.amax, ws.sampled, canvas_out, ws.prev, ws.astate, n_forwards,
                          ws.ncommit, (int32_t*)nullptr, B, C, V, k, (const int32_t*)nullptr,
@@ -1248,11 +1323,12 @@ static bool build_anneal_graph(dg_model* m, const dg_kv* kv, const dg_anneal_par
         launch_pdl((anneal_init_kernel), ceil_div((long)B * C, 256), 256, 0, cap, 1, canvas_out,
                    ws.prev, ws.astate, n_forwards, B, C, V, (const unsigned long long*)seeds,
                    ws.loop_s, N);
+        zero_loop_z(m, B, cap);
       },
       [&](cudaStream_t cap) {
         dg_status s = run_forward(m, kv, canvas_out, N, N, ws.ent, ws.amax, nullptr, nullptr,
                                   nullptr, cap, ws.loop_s, anneal_dev(m, p, seeds, N, ws.loop_s),
-                                  ws.sampled);
+                                  ws.sampled, loop_z(m), loop_z(m));
         if (s == DG_OK)
           s = launch_anneal(ws.ent, ws.amax, ws.sampled, canvas_out, ws.prev, ws.astate,
                             n_forwards, ws.ncommit, ws.remaining, B, C, V, 0, ws.loop_s, N, q,
@@ -1276,7 +1352,8 @@ dg_status dg_generate_block_annealed(dg_model* m, const dg_kv* kv, const dg_anne
                        m->profiling ? m->prof_forwards : 0);
   dg::BlockGraph* g = nullptr;
   for (auto* x : m->graphs)
-    if (x->anneal && x->kv == kv && x->kv_P == kv->P && x->kv_W == kv->W && x->aN == p->N &&
+    if (x->anneal && x->sc == m->selfcond && x->kv == kv && x->kv_P == kv->P &&
+        x->kv_W == kv->W && x->aN == p->N &&
         x->ab == p->b && x->atmax == p->tau_max && x->atmin == p->tau_min &&
         x->aestop == p->e_stop && x->seeds == seeds && x->canvas == canvas_out &&
         x->nfwd == n_forwards && x->prof == m->profiling &&
@@ -1304,6 +1381,7 @@ dg_status dg_generate_block_annealed(dg_model* m, const dg_kv* kv, const dg_anne
     g->nfwd = n_forwards;
     g->prof = m->profiling;
     g->fcap = m->profiling ? m->prof_forwards : 0;
+    g->sc = m->selfcond;
     if (!m->cap_stream) DG_TRY_CUDA(cudaStreamCreateWithFlags(&m->cap_stream, cudaStreamNonBlocking));
     if (g->prof) {
       // profiling: the first fcap forwards unrolled, with an event pair around every
@@ -1381,6 +1459,25 @@ dg_status dg_anneal_init(int32_t* canvas, int32_t* prev_argmax, int32_t* state, 
              canvas, prev_argmax, state, (int32_t*)nullptr, B, C, V,
              (const unsigned long long*)seeds, (int32_t*)nullptr, 1);
   return check_launch("anneal init");
+}
+
+dg_status dg_set_selfcond(dg_model* m, int32_t on) {
+  g_err.clear();
+  DG_REQUIRE(m, "null model");
+  DG_REQUIRE(on == 0 || m->cfg.sc_inter > 0, "the model has no self-conditioning FFW");
+  m->selfcond = on != 0;
+  return DG_OK;
+}
+
+dg_status dg_selfcond_forward(dg_model* m, const dg_kv* kv, const int32_t* canvas,
+                              int32_t steps_left, int32_t T, const void* z_in, float* entropy,
+                              int32_t* argmax, void* z_out, void* stream) {
+  g_err.clear();
+  DG_TRY(check_step_args(m, kv, steps_left, T));
+  DG_REQUIRE(canvas && entropy && argmax && z_out, "null argument");
+  DG_REQUIRE(m->cfg.sc_inter > 0, "the model has no self-conditioning FFW");
+  return run_forward(m, kv, canvas, steps_left, T, entropy, argmax, nullptr, nullptr, nullptr,
+                     (cudaStream_t)stream, nullptr, AnnealDev{}, nullptr, z_in, z_out);
 }
 
 dg_status dg_eb_sample(const float* entropy, const int32_t* argmax, int32_t* canvas,

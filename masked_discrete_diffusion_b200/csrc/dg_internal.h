@@ -114,6 +114,13 @@ struct Workspace {
   // per-canvas stop state [max_batch], per-tile race winners [n_vtiles, max_batch C, 2]
   int32_t *sampled = nullptr, *prev = nullptr, *astate = nullptr;
   void* gpart = nullptr;
+  // self-conditioning (models with sc_inter > 0): the transposed embedding [d, V],
+  // p0 [max_batch C, V], per-tile (ref, sum) [n_vtiles, max_batch C, 2], y = p0 E
+  // [max_tok, d], the FFW hidden [max_tok, sc_inter], the K-sliced partials
+  // [parts, max_batch C, d] (tensor-core path) and z [max_batch C, d]
+  void *embT = nullptr, *scP = nullptr, *scref = nullptr, *scy = nullptr, *sch = nullptr;
+  float* scpart = nullptr;
+  void* z = nullptr;
   int max_pos = 0;
   size_t kc_elems = 0;
   int max_tiles = 0;
@@ -135,6 +142,7 @@ struct BlockGraph {
   int fcap = 0;            // forwards of a profiled (unrolled) block, 0: T
   // annealed block: its constants and seeds (anneal false: the Entropy-Bound block)
   bool anneal = false;
+  bool sc = false;  // captured with the self-conditioning signal carried
   int aN = 0;
   float ab = 0.f, atmax = 0.f, atmin = 0.f, aestop = 0.f;
   const void* seeds = nullptr;
@@ -174,6 +182,7 @@ struct dg_model {
   // > 0: the next routed-expert launch stalls its down units on purpose, with every
   // wait limited to this many ns (dg_debug_stall_experts; tests of the timeout path)
   long long stall_limit_ns = 0;
+  bool selfcond = false;  // block loops carry the self-conditioning signal (sc_inter > 0)
 };
 
 namespace dg {

@@ -12,6 +12,7 @@
 
 #include "k_anneal.cuh"
 #include "k_common.cuh"
+#include "k_selfcond.cuh"
 
 namespace dg {
 
@@ -19,12 +20,14 @@ namespace dg {
 // a1: embedding gather (+ sinusoidal timestep embedding for canvas rows)
 // x[t, :] = E[ids[t], :] + temb(tau); temb[i] = sin(1000 tau w_i),
 // temb[d/2 + i] = cos(1000 tau w_i), w_i = 10000^(-i / (d/2)).  tau < 0: none.
-// With s_dev set, tau = *s_dev / T (steps left read from device memory).
+// With s_dev set, tau = *s_dev / T (steps left read from device memory).  With z set
+// (self-conditioning), z[t, :] is added as well.
 // ---------------------------------------------------------------------------
-template <class TW, class TR>
+template <class TW, class TR, class TZ>
 __global__ void embed_kernel(const int32_t* __restrict__ ids, const TW* __restrict__ emb,
                              TR* __restrict__ x, int n_tok, int d, int max_id, double tau,
-                             int32_t* err, const int32_t* __restrict__ s_dev, int T) {
+                             int32_t* err, const int32_t* __restrict__ s_dev, int T,
+                             const TZ* __restrict__ z) {
   pdl_enter();
   if (s_dev) tau = (double)*s_dev / (double)T;
   const int t = blockIdx.x;
@@ -44,6 +47,7 @@ __global__ void embed_kernel(const int32_t* __restrict__ ids, const TW* __restri
       const double a = 1000.0 * tau * w;
       v += c < half ? sin(a) : cos(a);
     }
+    if (z) v += (double)z[(size_t)t * d + c];
     x[(size_t)t * d + c] = narrow<TR>(v);
   }
 }
@@ -684,7 +688,7 @@ template <class TA, class TW, class Acc>
 __global__ void __launch_bounds__(256)
     lmhead_simt_kernel(const TA* __restrict__ xn, const TW* __restrict__ wlm, int n_rows, int V,
                        int d, float scale, Acc* __restrict__ part, float* __restrict__ logits,
-                       AnnealDev an) {
+                       AnnealDev an, ScDev sc) {
   pdl_enter();
   const Acc tau = an.N > 0 ? (Acc)an.tau() : Acc(1);
   // the logits tile T reuses the operand staging buffers once the K loop is done
@@ -773,6 +777,22 @@ __global__ void __launch_bounds__(256)
       pp[2] = u;
       pp[3] = (Acc)am;
     }
+    if (sc.P) {  // self-conditioning: exp(l1 - ref) at temperature 1, ref = the tile's max
+      TA* prow = reinterpret_cast<TA*>(sc.P) + (size_t)r * sc.ldp;
+      Acc p = 0;
+      for (int c = lane; c < SG_BN; c += 32) {
+        if (n0 + c >= V) continue;
+        const Acc q = dexp((T[rr][c] - mx) * tau);
+        prow[n0 + c] = narrow<TA>(q);
+        p += q;
+      }
+      p = warp_sum(p);
+      if (lane == 0) {
+        Acc* rp = reinterpret_cast<Acc*>(sc.ref) + ((size_t)blockIdx.x * n_rows + r) * 2;
+        rp[0] = mx * tau;
+        rp[1] = p;
+      }
+    }
     if (an.seeds) {  // this tile's winner of the race, lane by lane then across the warp
       GumbelBest<Acc> gb;
       const unsigned long long st = an.pair_state(r, V, 0);
@@ -800,16 +820,20 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+constexpr int LM_SC_MAX_TILES = 1024;  // vocabulary tiles a self-conditioned row may span
+
 // Merge of per-tile statistics (fixed order and shape), one warp per row:
 //   M = max m_i, S = sum s_i e^(m_i - M),
 //   H = log S - (1/S) sum e^(m_i - M) (u_i + (m_i - M) s_i)   (clamped at 0),
 //   argmax = the id of the first tile (lowest vocab) attaining M.
-//   sampled (with gpart) = the id of the best (value, lowest id) race winner over tiles.
-template <class Acc>
+//   sampled (with gpart) = the id of the best (value, lowest id) race winner over tiles;
+//   with sc.P: the row's tile values become p0 = exp(l1 - M) / S (M = max ref_t,
+//   S = sum_t s_t exp(ref_t - M)) in place, tile t holding columns [t tw, (t + 1) tw).
+template <class Acc, class TP>
 __global__ void __launch_bounds__(128)
     lm_merge_kernel(const Acc* __restrict__ part, int n_vt, int n_rows, float* __restrict__ H,
                     int32_t* __restrict__ amax, const Acc* __restrict__ gpart,
-                    int32_t* __restrict__ sampled) {
+                    int32_t* __restrict__ sampled, ScDev sc, int tw) {
   // one block per row; the tiles are split over the threads, each thread merges
   // its tiles online (running max M_t; S and U rescaled when M_t rises), then the
   // block merges the threads in a fixed order
@@ -938,6 +962,38 @@ __global__ void __launch_bounds__(128)
       }
       sampled[r] = bi;
     }
+  }
+  if (sc.P) {
+    // M and S over the tiles (each thread its tiles, then thread 0 in a fixed order),
+    // the tiles' factors exp(ref_t - M) / S in shared memory (n_vt <= LM_SC_MAX_TILES),
+    // then every column of the row scaled by its tile's factor, threads on consecutive
+    // columns
+    __shared__ Acc sm_fac[LM_SC_MAX_TILES];
+    __syncthreads();
+    const Acc* rp = reinterpret_cast<const Acc*>(sc.ref);
+    Acc Mt = -INFINITY;
+    for (int i = tid; i < n_vt; i += blockDim.x) Mt = fmax(Mt, rp[((size_t)i * n_rows + r) * 2]);
+    sm_m[tid] = Mt;
+    __syncthreads();
+    if (tid == 0) {
+      Acc Mx = -INFINITY;
+      for (int t = 0; t < (int)blockDim.x; ++t) Mx = fmax(Mx, sm_m[t]);
+      Acc S = 0;
+      for (int i = 0; i < n_vt; ++i) {
+        const Acc* q = rp + ((size_t)i * n_rows + r) * 2;
+        S += q[1] * dexp(q[0] - Mx);
+      }
+      sm_s[0] = Mx;
+      sm_s[1] = Acc(1) / S;
+    }
+    __syncthreads();
+    const Acc Mx = sm_s[0], inv = sm_s[1];
+    for (int i = tid; i < n_vt; i += blockDim.x)
+      sm_fac[i] = dexp(rp[((size_t)i * n_rows + r) * 2] - Mx) * inv;
+    __syncthreads();
+    TP* prow = reinterpret_cast<TP*>(sc.P) + (size_t)r * sc.ldp;
+    for (int c = tid; c < sc.ldp; c += blockDim.x)
+      prow[c] = narrow<TP>((Acc)widen(prow[c]) * sm_fac[c / tw]);
   }
 }
 

@@ -23,6 +23,7 @@
 #include "dg_internal.h"
 #include "k_anneal.cuh"
 #include "k_common.cuh"
+#include "k_selfcond.cuh"
 #include "tc_ptx.cuh"
 
 namespace dg {
@@ -369,12 +370,42 @@ struct EpiRouterTopk {
   }
 };
 
+// Partial tiles of a K-sliced GEMM (launched with ksplit < 0): thread per row, the
+// CTA's accumulator rows stored to out + blockIdx.z * zstride ([M, N] fp32 per slice).
+struct EpiPartialRows {
+  static constexpr bool kStaged = false, kWarpRows = false;
+  static constexpr size_t kExtraSmem = 0;
+  float* out;
+  int M, N;
+  size_t zstride;
+  template <int NCH, class Ld>
+  __device__ void run(int row, bool valid, int n0, Ld&& ld) const {
+    float* o = out + (size_t)blockIdx.z * zstride + (size_t)row * N;
+#pragma unroll 1
+    for (int c = 0; c < NCH; ++c) {
+      float v[32];
+      ld(0, c, v);  // warp-collective: every lane loads
+      const int c0 = n0 + c * 32;
+      if (!valid || c0 >= N) continue;
+      if (c0 + 32 <= N) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          reinterpret_cast<float4*>(o + c0)[q] =
+              make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+      } else {
+        for (int j = 0; j < 32 && c0 + j < N; ++j) o[c0 + j] = v[j];
+      }
+    }
+  }
+};
+
 // Per-row statistics of logits l = scale * acc over this CTA's vocabulary tile
 // (columns n0 .. n0 + 32 NCH - 1, those < N): m = max, s = sum exp(l - m),
 // u = sum exp(l - m) (l - m), a = lowest id attaining m.  part[(tile, row)] = (m, s, u, a).
 // With an.N > 0 the logits are tempered (l = scale acc / tau) and, with an.seeds, the
 // tile's winner of the Gumbel-max race goes to an.gpart[(tile, row)] = (l / tau - log E,
-// id).
+// id).  With sc.P, the tile's values exp(l1 - ref) at temperature 1 (l1 = scale acc,
+// ref = its largest) go to sc.P as bf16 and (ref, their sum) to sc.ref (self-conditioning).
 // Pass 1 finds the largest accumulator (a max tree per 32-column chunk; the index is
 // searched only in a chunk that raises the maximum).  Pass 2 works in base-2 units,
 // z2 = (l - m) log2 e, e = 2^z2 (ex2.approx.ftz), with two interleaved sums; columns
@@ -386,6 +417,7 @@ struct EpiLmStats {
   int M, N;
   float scale;
   AnnealDev an = {};
+  ScDev sc = {};
 
   static __device__ __forceinline__ float ex2(float x) {
     float y;
@@ -395,9 +427,10 @@ struct EpiLmStats {
 
   template <int NCH, class Ld>
   __device__ void run(int row, bool valid, int n0, Ld&& ld) const {
-    constexpr float kLog2e = 1.4426950408889634f, kLn2 = 0.6931471805599453f;
-    const float sc = an.N > 0 ? (float)((double)scale / an.tau()) : scale;
-    const float sc2 = sc * kLog2e;
+    constexpr float kLog2e = 1.4426950408889634f;
+    const float tau = an.N > 0 ? (float)an.tau() : 1.f;
+    const float sc_ = an.N > 0 ? (float)((double)scale / an.tau()) : scale;
+    const float sc2 = sc_ * kLog2e;
     auto load = [&](int c, float* v) {
       ld(0, c, v);
       if (n0 + c * 32 + 32 > N) {  // the ragged last tile (uniform across the warp)
@@ -429,61 +462,98 @@ struct EpiLmStats {
         am = n0 + c * 32 + idx;
       }
     }
-    const float mx = sc * mv, mx2 = sc2 * mv;
-    // pass 2
-    float s0 = 0.f, s1 = 0.f, u0 = 0.f, u1 = 0.f;
+    const bool draw = an.seeds != nullptr, scp = sc.P != nullptr;
+    if (!draw && !scp) pass2<NCH, false, false>(row, valid, n0, load, mv, am, sc_, sc2, tau);
+    else if (!draw) pass2<NCH, false, true>(row, valid, n0, load, mv, am, sc_, sc2, tau);
+    else if (!scp) pass2<NCH, true, false>(row, valid, n0, load, mv, am, sc_, sc2, tau);
+    else pass2<NCH, true, true>(row, valid, n0, load, mv, am, sc_, sc2, tau);
+  }
+
+  template <int NCH, bool DRAW, bool SC, class Load>
+  __device__ void pass2(int row, bool valid, int n0, Load& load, float mv, int am, float sc_,
+                        float sc2, float tau) const {
+    constexpr float kLn2 = 0.6931471805599453f;
+    const float mx = sc_ * mv, mx2 = sc2 * mv;
     const int tile = n0 / (NCH * 32);
-    if (an.seeds == nullptr) {
-#pragma unroll 1
-      for (int c = 0; c < NCH; ++c) {
-        float v[32];
-        load(c, v);
-#pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-          const float z0 = fmaf(v[j], sc2, -mx2), z1 = fmaf(v[j + 1], sc2, -mx2);
-          const float e0 = ex2(z0), e1 = ex2(z1);
-          s0 += e0;
-          s1 += e1;
-          u0 = fmaf(e0, z0, u0);
-          u1 = fmaf(e1, z1, u1);
-        }
-      }
-    } else {
-      // Gumbel-max race of this tile: it starts from the tile's argmax (z = 0, e = 1);
-      // a chunk where no row of the warp has e >= E_argmax^-1 E_min draws nothing (no
-      // column there can beat the argmax).  Otherwise each output of the stream serves a
-      // column pair, and since E = -log u >= 1 - u a column can beat the argmax (hence
-      // the best so far) only if 1 - u < e E_argmax (the margin 2^-10 covers every
-      // rounding): only those columns take the log, in a branch the warp skips when none
-      // of its rows has one.
-      GumbelBest<float> gb;
-      const unsigned long long st = an.pair_state(valid ? row : 0, N, n0 >> 1);
+    float s0 = 0.f, s1 = 0.f, u0 = 0.f, u1 = 0.f, p0 = 0.f, p1 = 0.f;
+    // Gumbel-max race of this tile (DRAW): it starts from the tile's argmax (z = 0,
+    // e = 1); a chunk where no row of the warp has e >= E_argmax^-1 E_min draws nothing
+    // (no column there can beat the argmax).  Otherwise each output of the stream serves
+    // a column pair, and since E = -log u >= 1 - u a column can beat the argmax (hence
+    // the best so far) only if 1 - u < e E_argmax (the margin 2^-10 covers every
+    // rounding): only those columns take the log, in a branch the warp skips when none of
+    // its rows has one.
+    GumbelBest<float> gb;
+    unsigned long long st = 0;
+    float lim = 0.f, tcap = 0.f;
+    if constexpr (DRAW) {
+      st = an.pair_state(valid ? row : 0, N, n0 >> 1);
       if (am < N)
         gb.offer(1.f,
                  sm64_expo(sm64_field(sm64_mix(st + (unsigned long long)((am - n0) >> 1) * SM64_G),
                                       am & 1),
                            0.f),
                  0.f, am);
-      const float lim = gb.e * SM64_EMIN_LO / gb.E;
-      const float tcap = gb.E * (1.f + 1.f / 1024.f);
+      lim = gb.e * SM64_EMIN_LO / gb.E;
+      tcap = gb.E * (1.f + 1.f / 1024.f);
+    }
+    // p0 tile values at temperature 1: 2^(z2 tau) (= e when tau = 1)
+    bf16* prow = SC ? reinterpret_cast<bf16*>(sc.P) + (size_t)(valid ? row : 0) * sc.ldp : nullptr;
 #pragma unroll 1
-      for (int c = 0; c < NCH; ++c) {
-        float v[32];
-        load(c, v);
-        bool cand = false;
+    for (int c = 0; c < NCH; ++c) {
+      float v[32];
+      load(c, v);
+      bool cand = false;
 #pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-          const float z0 = fmaf(v[j], sc2, -mx2), z1 = fmaf(v[j + 1], sc2, -mx2);
-          const float e0 = ex2(z0), e1 = ex2(z1);
-          s0 += e0;
-          s1 += e1;
-          u0 = fmaf(e0, z0, u0);
-          u1 = fmaf(e1, z1, u1);
+      for (int j = 0; j < 32; j += 2) {
+        const float z0 = fmaf(v[j], sc2, -mx2), z1 = fmaf(v[j + 1], sc2, -mx2);
+        const float e0 = ex2(z0), e1 = ex2(z1);
+        s0 += e0;
+        s1 += e1;
+        u0 = fmaf(e0, z0, u0);
+        u1 = fmaf(e1, z1, u1);
+        if constexpr (SC) {
+          const float q0 = tau == 1.f ? e0 : ex2(z0 * tau), q1 = tau == 1.f ? e1 : ex2(z1 * tau);
+          p0 += q0;
+          p1 += q1;
+          v[j] = q0;  // the p0 values are stored below, then z is recomputed if drawing
+          v[j + 1] = q1;
+        } else if constexpr (DRAW) {
           v[j] = z0;
           v[j + 1] = z1;
-          cand |= fmaxf(e0, e1) >= lim;
         }
+        if constexpr (DRAW) cand |= fmaxf(e0, e1) >= lim;
+      }
+      if constexpr (SC) {
+        if (valid && n0 + c * 32 < N) {
+          uint4* dst = reinterpret_cast<uint4*>(prow + n0 + c * 32);
+          const bool full = n0 + c * 32 + 32 <= N;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint4 w;
+            uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              const __nv_bfloat162 b2 = __floats2bfloat162_rn(v[8 * q + 2 * h], v[8 * q + 2 * h + 1]);
+              wp[h] = *reinterpret_cast<const uint32_t*>(&b2);
+            }
+            if (full) {
+              dst[q] = w;
+            } else {
+              const bf16* wb = reinterpret_cast<const bf16*>(&w);
+              for (int h = 0; h < 8; ++h)
+                if (n0 + c * 32 + 8 * q + h < N) prow[n0 + c * 32 + 8 * q + h] = wb[h];
+            }
+          }
+        }
+      }
+      if constexpr (DRAW) {
         if (!__any_sync(0xffffffffu, cand)) continue;
+        if constexpr (SC) {  // v holds the p0 values: bring back the tempered z2
+          load(c, v);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = fmaf(v[j], sc2, -mx2);
+        }
         const unsigned long long stc = st + (unsigned long long)(c * 16) * SM64_G;
         float uu[32];
         unsigned fm = 0;
@@ -503,13 +573,16 @@ struct EpiLmStats {
           if (__any_sync(0xffffffffu, (fm >> j) & 1u) && ((fm >> j) & 1u))
             gb.offer(ex2(v[j]), -logf(uu[j]), v[j] * kLn2, n0 + c * 32 + j);
       }
-      if (valid)
+    }
+    if (valid) {
+      if constexpr (DRAW)
         reinterpret_cast<float2*>(an.gpart)[(size_t)tile * M + row] =
             make_float2(gb.value(mx), (float)gb.id);  // ids < 2^24: exact
-    }
-    if (valid)
+      if constexpr (SC)
+        reinterpret_cast<float2*>(sc.ref)[(size_t)tile * M + row] = make_float2(scale * mv, p0 + p1);
       reinterpret_cast<float4*>(part)[(size_t)tile * M + row] =
           make_float4(mx, s0 + s1, (u0 + u1) * kLn2, (float)am);
+    }
   }
 };
 
@@ -613,10 +686,14 @@ __global__ void __launch_bounds__(TC_DENSE_THREADS, 1)
   int* abort_flag = reinterpret_cast<int*>(tslot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * (MT * 128), n0 = blockIdx.y * BN;
+  // ksplit > 1: the K slices of a cluster, reduced through DSMEM; ksplit < 0: -ksplit
+  // independent K slices along grid z, each leaving its own partial tile (the epilogue
+  // writes it to slice blockIdx.z)
   const int nk_all = (K + TC_KB - 1) / TC_KB;
-  const int rank = ksplit > 1 ? (int)cl::ctarank() : 0;
-  const int kb_lo = (int)((long)nk_all * rank / ksplit);
-  const int nk = (int)((long)nk_all * (rank + 1) / ksplit) - kb_lo;
+  const int nparts = ksplit < 0 ? -ksplit : ksplit;
+  const int rank = ksplit > 1 ? (int)cl::ctarank() : (ksplit < 0 ? (int)blockIdx.z : 0);
+  const int kb_lo = (int)((long)nk_all * rank / nparts);
+  const int nk = (int)((long)nk_all * (rank + 1) / nparts) - kb_lo;
   const int rot = nk > 0 ? (int)(blockIdx.y % nk) : 0;
 
   if (threadIdx.x == 0) {
@@ -1170,7 +1247,10 @@ dg_status tc_moe_experts_f8(dg_model* m, int l, const bf16* X, bf16* hb, float* 
                             cudaStream_t st);
 dg_status tc_lmhead_stats(dg_model* m, const bf16* xn, int M, float* ent, int32_t* amax,
                           cudaStream_t st, const AnnealDev& an = AnnealDev{},
-                          int32_t* sampled = nullptr);
+                          int32_t* sampled = nullptr, const ScDev& sc = ScDev{});
+// y = p0 E for the n rows the LM head left in the workspace (self-conditioning): a
+// K-sliced tcgen05 GEMM against the transposed embedding, partials added in slice order.
+dg_status tc_selfcond_mix(dg_model* m, int n, cudaStream_t st);
 dg_status tc_attention(dg_model* m, const bf16* q, int B, int nq, int qpos0, const dg_kv* kv,
                        int l, const bf16* kB, const bf16* vB, int nB, int kposB, int npB,
                        bool causal, bf16* out, cudaStream_t st);

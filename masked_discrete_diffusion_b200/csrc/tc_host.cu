@@ -134,6 +134,7 @@ constexpr int QKV_ST = 4, RT_ST = 4;
 constexpr int LM_BN = 256, LM_ST = 3;
 constexpr int MOE_ST = 4;
 constexpr int MOE8_ST = 3;
+constexpr int SC_ST = 3;  // p0 E^T GEMM stages
 
 }  // namespace
 
@@ -173,6 +174,8 @@ dg_status tc_prepare(dg_model* m) {
                   Dn::SMEM + EpiAddF32::kExtraSmem));
   DG_TRY(set_smem(tc_dense_kernel<DENSE_BN, DENSE_MT, true, DUAL_ST, EpiSwigluBf16>, Du::SMEM));
   DG_TRY(set_smem(tc_dense_kernel<LM_BN, 2, false, LM_ST, EpiLmStats>, Lm::SMEM));
+  DG_TRY(set_smem(tc_dense_kernel<256, 2, false, SC_ST, EpiPartialRows>,
+                  DenseCfg<256, 2, false, SC_ST>::SMEM));
   DG_TRY(set_smem(tc_moe_kernel<MOE_ST>, MoeCfg<MOE_ST>::SMEM));
   DG_TRY(set_smem(tc_attn_kernel, AT_SMEM));
   DG_TRY(set_smem(tc_dense_kernel<128, 1, false, RT_ST, EpiRouterTopk>,
@@ -271,7 +274,8 @@ dg_status tc_gemm_swiglu(dg_model* m, const bf16* A, const void* Wg, const void*
 }
 
 dg_status tc_lmhead_stats(dg_model* m, const bf16* xn, int M, float* ent, int32_t* amax,
-                          cudaStream_t st, const AnnealDev& an, int32_t* sampled) {
+                          cudaStream_t st, const AnnealDev& an, int32_t* sampled,
+                          const ScDev& sc) {
   const dg_config& c = m->cfg;
   CUtensorMap a, b;
   DG_TRY(tmap(m, xn, m->ws.max_tok, c.d_model, 128, &a));
@@ -279,11 +283,41 @@ dg_status tc_lmhead_stats(dg_model* m, const bf16* xn, int M, float* ent, int32_
   float* part = (float*)m->ws.lm_part;
   EpiLmStats epi{part, M, c.vocab, c.logit_scale};
   epi.an = an;
+  epi.sc = sc;
   DG_TRY((launch_dense<LM_BN, 2, false, LM_ST>(m, a, b, b, M, c.vocab, c.d_model, epi, st,
                                                false)));
   const int n_vt = ceil_div_i(c.vocab, LM_BN);
-  launch_pdl((lm_merge_kernel<float>), M, 128, 0, st, 1, part, n_vt, M, ent, amax,
-             (const float*)(an.seeds ? an.gpart : nullptr), an.seeds ? sampled : nullptr);
+  launch_pdl((lm_merge_kernel<float, bf16>), M, 128, 0, st, 1, part, n_vt, M, ent, amax,
+             (const float*)(an.seeds ? an.gpart : nullptr), an.seeds ? sampled : nullptr, sc,
+             LM_BN);
+  ++m->launches;
+  return DG_OK;
+}
+
+dg_status tc_selfcond_mix(dg_model* m, int n, cudaStream_t st) {
+  const dg_config& c = m->cfg;
+  const int V = c.vocab, d = c.d_model;
+  const size_t lm_rows = (size_t)c.max_batch * c.canvas;
+  CUtensorMap a, b;
+  DG_TRY(tmap(m, m->ws.scP, lm_rows, V, 128, &a));
+  DG_TRY(tmap(m, m->ws.embT, d, V, 256, &b));
+  typedef DenseCfg<256, 2, false, SC_ST> Cfg;
+  const int tiles = ceil_div_i(n, 256) * ceil_div_i(d, 256);
+  const int nk = ceil_div_i(V, TC_KB);
+  const int S = std::max(1, std::min(std::min(SC_MAX_PARTS, state(m)->n_sm / tiles), nk));
+  dim3 grid(ceil_div_i(n, 256), ceil_div_i(d, 256), S);
+  EpiPartialRows epi{(float*)m->ws.scpart, n, d, (size_t)n * d};
+  cudaError_t e = launch_pdl(tc_dense_kernel<256, 2, false, SC_ST, EpiPartialRows>, grid,
+                             TC_DENSE_THREADS, Cfg::SMEM, st, 1, a, b, b, n, V, -S, epi,
+                             m->ws.err, 0, 1);
+  ++m->launches;
+  if (e != cudaSuccess) {
+    set_error("self-conditioning GEMM launch: %s", cudaGetErrorString(e));
+    return DG_ERR_CUDA;
+  }
+  const long total = (long)n * d;
+  launch_pdl((selfcond_reduce_kernel<bf16>), (int)((total + 255) / 256), 256, 0, st, 1,
+             (const float*)m->ws.scpart, S, n, d, (bf16*)m->ws.scy);
   ++m->launches;
   return DG_OK;
 }

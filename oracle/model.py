@@ -318,7 +318,7 @@ def selfcond_mix(ws: Weights, logits: np.ndarray) -> np.ndarray:
     p = np.exp(l - m)
     p /= p.sum(axis=1, keepdims=True)
     E = ws.get("tok_emb", (w.vocab + 1, w.d_model))[:w.vocab]
-    return p @ E
+    return ws.store(p) @ E           # p0 kept through `store` (a bf16 model stores it)
 
 
 def selfcond(ws: Weights, logits: np.ndarray) -> np.ndarray:

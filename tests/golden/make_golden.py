@@ -35,6 +35,10 @@ Two further modes on a deep workload:
      uniform initial canvas x_1: tempered entropies H/H64, argmax, the Gumbel-max draw
      `sampled` and its gap to the runner-up, the router margins of the rows, and the
      bf16-storage run's H_s16 and sampled_s16.
+  <name>@selfcond -> <name>-selfcond.npz (a self-conditioned workload): canvas 0's first
+     forward (all [MASK], steps_left = T), its entropies and the self-conditioning signal
+     z = FFW(p0 E) it hands to the next forward, with y = p0 E; and the bf16-storage
+     run's H64_s16 and z_s16.
   <name>@block   -> <name>-block.npz: the oracle's whole block (all [MASK], up to T
      forwards, the entropy-bound sampler after each): per step the input canvas, the
      steps left, H, argmax, margin and the number committed; the number of forwards.
@@ -201,6 +205,26 @@ def anneal_case(name: str):
           f"[{ts['H'].min():.3f}, {ts['H'].max():.3f}], gaps > 0.05: {(gap > 0.05).mean():.3f}")
 
 
+def selfcond_case(name: str):
+    """<name>-selfcond.npz: canvas 0's first forward and the z it produces."""
+    w = workloads.get(name)
+    t0 = time.time()
+    prompt = model_inputs.prompt(w.with_(batch=1))[0].numpy()
+    canvas = np.full(w.canvas, w.mask_id)
+    ws = om.Weights(w, keep_layers=False)
+    st = om.prefill_then_forward(ws, prompt, canvas, w.T, w.T, want_logits=True)
+    y = om.selfcond_mix(ws, st["logits"])
+    z = om.selfcond(ws, st["logits"])
+    ws16 = om.Weights(w, keep_layers=False, storage="bf16")
+    s16 = om.prefill_then_forward(ws16, prompt, canvas, w.T, w.T, want_logits=True)
+    out = dict(H=st["H"], H64=st["H64"], y=y, z=z, H64_s16=s16["H64"],
+               z_s16=om.selfcond(ws16, s16["logits"]))
+    path = os.path.join(HERE, f"{name}-selfcond.npz")
+    np.savez_compressed(path, **out)
+    print(f"{name}: wrote {path} in {time.time() - t0:.0f} s; |y| rms {np.sqrt((y * y).mean()):.3g},"
+          f" |z| rms {np.sqrt((z * z).mean()):.3g}")
+
+
 DEPTHS = (1, 2, 4, 8, 16, 30)
 
 
@@ -289,6 +313,9 @@ if __name__ == "__main__":
             continue
         if arg.endswith("@anneal"):
             anneal_case(arg.removesuffix("@anneal"))
+            continue
+        if arg.endswith("@selfcond"):
+            selfcond_case(arg.removesuffix("@selfcond"))
             continue
         if arg.endswith("+rmonly"):
             name, _, c = arg.removesuffix("+rmonly").partition(":")
