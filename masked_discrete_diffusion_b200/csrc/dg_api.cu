@@ -595,8 +595,15 @@ template <class Path> struct Runner {
       launch_pdl((lm_merge_kernel<Acc, TA>), n, 128, 0, st, 1, (const Acc*)ws.lm_part, ws.n_vtiles,
                                                           n, ent, amax,
                                                           (const Acc*)(an.seeds ? an.gpart : nullptr),
-                                                          an.seeds ? sampled : nullptr, sc, SG_BN);
+                                                          an.seeds ? sampled : nullptr, sc);
       ++m->launches;
+      if (sc.P) {  // the tile values become p0
+        static_assert(SG_BN == 64, "tile shift");
+        const long groups = (long)n * (c.vocab / (16 / (int)sizeof(TA)));
+        launch_pdl((selfcond_scale_kernel<TA, Acc>), ceil_div(groups, 256), 256, 0, st, 1,
+                   (TA*)sc.P, (const Acc*)sc.ref, n, c.vocab, 6);
+        ++m->launches;
+      }
     }
     if (z_out) DG_TRY(selfcond(n, z_out));
     return check_launch("forward");
@@ -722,9 +729,8 @@ dg_status dg_model_create(const dg_config* cfg, const dg_weights* w, dg_model** 
   DG_REQUIRE(c.sc_inter >= 0, "sc_inter must be >= 0");
   if (c.sc_inter > 0) {
     DG_REQUIRE(w->sc_gate && w->sc_up && w->sc_down, "null self-conditioning weight pointer");
-    const int tile = c.dtype == DG_F32 ? SG_BN : 256;
-    DG_REQUIRE((c.vocab + tile - 1) / tile <= LM_SC_MAX_TILES,
-               "self-conditioning spans at most %d vocabulary tiles of %d", LM_SC_MAX_TILES, tile);
+    DG_REQUIRE(c.vocab % (c.dtype == DG_F32 ? 2 : 8) == 0,
+               "self-conditioning needs V a multiple of 16 bytes of activations");
     if (c.dtype != DG_F32)
       DG_REQUIRE(c.sc_inter % 64 == 0 && c.vocab % 8 == 0,
                  "self-conditioning on tensor cores needs sc_inter %% 64 == 0 and V %% 8 == 0");

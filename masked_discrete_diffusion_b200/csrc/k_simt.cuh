@@ -820,20 +820,18 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-constexpr int LM_SC_MAX_TILES = 1024;  // vocabulary tiles a self-conditioned row may span
-
 // Merge of per-tile statistics (fixed order and shape), one warp per row:
 //   M = max m_i, S = sum s_i e^(m_i - M),
 //   H = log S - (1/S) sum e^(m_i - M) (u_i + (m_i - M) s_i)   (clamped at 0),
 //   argmax = the id of the first tile (lowest vocab) attaining M.
 //   sampled (with gpart) = the id of the best (value, lowest id) race winner over tiles;
-//   with sc.P: the row's tile values become p0 = exp(l1 - M) / S (M = max ref_t,
-//   S = sum_t s_t exp(ref_t - M)) in place, tile t holding columns [t tw, (t + 1) tw).
+//   with sc.P: each tile's factor exp(ref_t - M) / S (M = max ref_t,
+//   S = sum_t s_t exp(ref_t - M)) replaces ref_t, for selfcond_scale_kernel.
 template <class Acc, class TP>
 __global__ void __launch_bounds__(128)
     lm_merge_kernel(const Acc* __restrict__ part, int n_vt, int n_rows, float* __restrict__ H,
                     int32_t* __restrict__ amax, const Acc* __restrict__ gpart,
-                    int32_t* __restrict__ sampled, ScDev sc, int tw) {
+                    int32_t* __restrict__ sampled, ScDev sc) {
   // one block per row; the tiles are split over the threads, each thread merges
   // its tiles online (running max M_t; S and U rescaled when M_t rises), then the
   // block merges the threads in a fixed order
@@ -964,37 +962,51 @@ __global__ void __launch_bounds__(128)
     }
   }
   if (sc.P) {
-    // M and S over the tiles (each thread its tiles, then thread 0 in a fixed order),
-    // the tiles' factors exp(ref_t - M) / S in shared memory (n_vt <= LM_SC_MAX_TILES),
-    // then every column of the row scaled by its tile's factor, threads on consecutive
-    // columns
-    __shared__ Acc sm_fac[LM_SC_MAX_TILES];
+    // M = max ref_t, S = sum_t s_t exp(ref_t - M) (per-thread partial sums over strided
+    // tiles, then added in thread order), and each tile's factor exp(ref_t - M) / S
+    // written over its ref_t for selfcond_scale_kernel
     __syncthreads();
-    const Acc* rp = reinterpret_cast<const Acc*>(sc.ref);
+    Acc* rp = reinterpret_cast<Acc*>(sc.ref);
     Acc Mt = -INFINITY;
     for (int i = tid; i < n_vt; i += blockDim.x) Mt = fmax(Mt, rp[((size_t)i * n_rows + r) * 2]);
     sm_m[tid] = Mt;
     __syncthreads();
-    if (tid == 0) {
-      Acc Mx = -INFINITY;
-      for (int t = 0; t < (int)blockDim.x; ++t) Mx = fmax(Mx, sm_m[t]);
-      Acc S = 0;
-      for (int i = 0; i < n_vt; ++i) {
-        const Acc* q = rp + ((size_t)i * n_rows + r) * 2;
-        S += q[1] * dexp(q[0] - Mx);
-      }
-      sm_s[0] = Mx;
-      sm_s[1] = Acc(1) / S;
+    Acc Mx = -INFINITY;
+    for (int t = 0; t < (int)blockDim.x; ++t) Mx = fmax(Mx, sm_m[t]);
+    Acc St = 0;
+    for (int i = tid; i < n_vt; i += blockDim.x) {
+      const Acc* q = rp + ((size_t)i * n_rows + r) * 2;
+      St += q[1] * dexp(q[0] - Mx);
     }
+    sm_s[tid] = St;
     __syncthreads();
-    const Acc Mx = sm_s[0], inv = sm_s[1];
-    for (int i = tid; i < n_vt; i += blockDim.x)
-      sm_fac[i] = dexp(rp[((size_t)i * n_rows + r) * 2] - Mx) * inv;
-    __syncthreads();
-    TP* prow = reinterpret_cast<TP*>(sc.P) + (size_t)r * sc.ldp;
-    for (int c = tid; c < sc.ldp; c += blockDim.x)
-      prow[c] = narrow<TP>((Acc)widen(prow[c]) * sm_fac[c / tw]);
+    Acc S = 0;
+    for (int t = 0; t < (int)blockDim.x; ++t) S += sm_s[t];
+    const Acc inv = Acc(1) / S;
+    for (int i = tid; i < n_vt; i += blockDim.x) {
+      Acc* q = rp + ((size_t)i * n_rows + r) * 2;
+      q[0] = dexp(q[0] - Mx) * inv;
+    }
   }
+}
+
+// p0 from the tile values: P[r, c] *= factor of (row r, tile c >> tw_shift) (the
+// merge left the factors at ref[(tile, r)][0]).  One thread per 16 bytes of a row.
+template <class TP, class Acc>
+__global__ void selfcond_scale_kernel(TP* __restrict__ P, const Acc* __restrict__ ref, int n_rows,
+                                      int V, int tw_shift) {
+  pdl_enter();
+  constexpr int kVec = 16 / sizeof(TP);
+  const int per_row = V / kVec;  // V % kVec == 0
+  const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (size_t)n_rows * per_row) return;
+  const int r = (int)(i / per_row), c0 = (int)(i - (size_t)r * per_row) * kVec;
+  const Acc f = ref[((size_t)(c0 >> tw_shift) * n_rows + r) * 2];
+  uint4 w = *reinterpret_cast<const uint4*>(P + (size_t)r * V + c0);
+  TP* e = reinterpret_cast<TP*>(&w);
+#pragma unroll
+  for (int j = 0; j < kVec; ++j) e[j] = narrow<TP>((Acc)widen(e[j]) * f);
+  *reinterpret_cast<uint4*>(P + (size_t)r * V + c0) = w;
 }
 
 // Cache K [blocks, Wp, h] and V^T [blocks, h, Wp] -> K, V [blocks, W, h].

@@ -144,7 +144,7 @@ extern "C" dg_status dg_lmhead_entropy_noalloc(const float* hidden, const void* 
   tc_dense_kernel<NA_BN, 2, false, NA_ST, EpiLmStats><<<grid, TC_DENSE_THREADS, Cfg::SMEM, st>>>(
       ma, mb, mb, M, d, 1, EpiLmStats{part, M, V, logit_scale}, err, 0, 0);
   lm_merge_kernel<float, bf16><<<M, 128, 0, st>>>(part, (V + NA_BN - 1) / NA_BN, M, entropy,
-                                                 argmax, nullptr, nullptr, ScDev{}, NA_BN);
+                                                 argmax, nullptr, nullptr, ScDev{});
   noalloc_flag_kernel<<<(M + 127) / 128, 128, 0, st>>>(err, M, entropy, argmax);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {

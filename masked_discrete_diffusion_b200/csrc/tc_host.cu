@@ -288,9 +288,15 @@ dg_status tc_lmhead_stats(dg_model* m, const bf16* xn, int M, float* ent, int32_
                                                false)));
   const int n_vt = ceil_div_i(c.vocab, LM_BN);
   launch_pdl((lm_merge_kernel<float, bf16>), M, 128, 0, st, 1, part, n_vt, M, ent, amax,
-             (const float*)(an.seeds ? an.gpart : nullptr), an.seeds ? sampled : nullptr, sc,
-             LM_BN);
+             (const float*)(an.seeds ? an.gpart : nullptr), an.seeds ? sampled : nullptr, sc);
   ++m->launches;
+  if (sc.P) {  // the tile values become p0
+    static_assert(LM_BN == 256, "tile shift");
+    const long groups = (long)M * (c.vocab / 8);
+    launch_pdl((selfcond_scale_kernel<bf16, float>), (int)((groups + 255) / 256), 256, 0, st, 1,
+               (bf16*)sc.P, (const float*)sc.ref, M, c.vocab, 8);
+    ++m->launches;
+  }
   return DG_OK;
 }
 
