@@ -52,6 +52,19 @@ __device__ __forceinline__ double dsqrt(double x) { return sqrt(x); }
 
 template <class T> __device__ __forceinline__ T silu(T z) { return z / (T(1) + dexp(-z)); }
 
+// 8 consecutive elements moved with 16-byte accesses (p 16-byte aligned).
+template <class T> __device__ __forceinline__ void ld8(const T* p, T (&v)[8]) {
+  static_assert((sizeof(T) * 8) % 16 == 0, "16-byte vectors");
+#pragma unroll
+  for (int i = 0; i < (int)(sizeof(T) * 8 / 16); ++i)
+    reinterpret_cast<uint4*>(v)[i] = reinterpret_cast<const uint4*>(p)[i];
+}
+template <class T> __device__ __forceinline__ void st8(T* p, const T (&v)[8]) {
+#pragma unroll
+  for (int i = 0; i < (int)(sizeof(T) * 8 / 16); ++i)
+    reinterpret_cast<uint4*>(p)[i] = reinterpret_cast<const uint4*>(v)[i];
+}
+
 template <class T> __device__ __forceinline__ T warp_sum(T v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

@@ -644,35 +644,69 @@ __global__ void moe_combine_norm_kernel(TR* __restrict__ x, const TY* __restrict
   __syncthreads();
   TR* xr = x + (size_t)t * d;
   Acc ss = 0;
-  for (int c0 = threadIdx.x * 8; c0 < d; c0 += blockDim.x * 8) {
+  // rows are 16-byte aligned (d % 8 == 0): every access moves 8 columns at once; the
+  // sums keep their order (shared expert, then the slots in k order, then the residual)
+  TR keep[8];  // the thread's first column group, kept for the norm pass
+  int g = 0;
+  for (int c0 = threadIdx.x * 8; c0 < d; c0 += blockDim.x * 8, ++g) {
     Acc v[8];
+    {
+      TY a[8];
+      ld8(ys + (size_t)t * d + c0, a);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) v[j] = (Acc)widen(ys[(size_t)t * d + c0 + j]);
+      for (int j = 0; j < 8; ++j) v[j] = (Acc)widen(a[j]);
+    }
     for (int k0 = 0; k0 < top_k; k0 += KB) {
       TY u[KB][8];
 #pragma unroll
-      for (int k = 0; k < KB; ++k)
+      for (int k = 0; k < KB; ++k) {
+        if (k0 + k < top_k) {
+          ld8(yb + (size_t)rows[k0 + k] * d + c0, u[k]);
+        } else {
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          u[k][j] = k0 + k < top_k ? yb[(size_t)rows[k0 + k] * d + c0 + j] : TY(0);
+          for (int j = 0; j < 8; ++j) u[k][j] = TY(0);
+        }
+      }
 #pragma unroll
       for (int k = 0; k < KB; ++k)
 #pragma unroll
         for (int j = 0; j < 8; ++j) v[j] += (Acc)widen(u[k][j]);
     }
+    TR xo[8], nx[8];
+    ld8(xr + c0, xo);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      const TR nx = narrow<TR>((Acc)widen(xr[c0 + j]) + v[j]);
-      xr[c0 + j] = nx;
-      const Acc a = (Acc)widen(nx);
+      nx[j] = narrow<TR>((Acc)widen(xo[j]) + v[j]);
+      const Acc a = (Acc)widen(nx[j]);
       ss += a * a;
+    }
+    st8(xr + c0, nx);
+    if (g == 0) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) keep[j] = nx[j];
     }
   }
   ss = block_sum(ss, red);
   const Acc inv = Acc(1) / dsqrt(ss / (Acc)d + (Acc)eps);
-  for (int c0 = threadIdx.x * 8; c0 < d; c0 += blockDim.x * 8)
+  g = 0;
+  for (int c0 = threadIdx.x * 8; c0 < d; c0 += blockDim.x * 8, ++g) {
+    TR xv[8];
+    if (g == 0) {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) y[(size_t)t * d + c0 + j] = narrow<TA>((Acc)widen(xr[c0 + j]) * inv);
+      for (int j = 0; j < 8; ++j) xv[j] = keep[j];
+    } else {
+      ld8(xr + c0, xv);
+    }
+    TA o[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) o[j] = narrow<TA>((Acc)widen(xv[j]) * inv);
+    if constexpr ((sizeof(TA) * 8) % 16 == 0) {
+      st8(y + (size_t)t * d + c0, o);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) y[(size_t)t * d + c0 + j] = o[j];
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------
