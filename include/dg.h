@@ -252,10 +252,13 @@ dg_status dg_generate_block_annealed(dg_model* m, const dg_kv* kv,
 
 /* Step k's forward alone: canvas [B, C] int32 ids in [0, V); writes the tempered
  * entropy [B, C] fp32, the argmax [B, C] int32 and the Gumbel-max draw sampled
- * [B, C] int32.  Requires 0 <= k < N. */
+ * [B, C] int32.  Self-conditioning (nullable, as in dg_selfcond_forward): z_in [B, C, d]
+ * added to the canvas rows' input, z_out [B, C, d] the next forward's z (p0 at
+ * temperature 1; requires sc_inter > 0).  Requires 0 <= k < N. */
 dg_status dg_anneal_forward(dg_model* m, const dg_kv* kv, const int32_t* canvas, int32_t k,
                             const dg_anneal_params* params, const uint64_t* seeds,
-                            float* entropy, int32_t* argmax, int32_t* sampled, void* stream);
+                            float* entropy, int32_t* argmax, int32_t* sampled,
+                            const void* z_in, void* z_out, void* stream);
 
 /* Step k's refinement alone, on caller-provided statistics (entropy, argmax, sampled:
  * [B, C]).  canvas [B, C] is rewritten; prev_argmax [B, C] holds the previous step's

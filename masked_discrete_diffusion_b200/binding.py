@@ -124,7 +124,7 @@ def lib() -> ctypes.CDLL:
             "dg_generate_block_annealed": [vp, vp, ctypes.POINTER(dg_anneal_params), vp, vp,
                                            vp, vp],
             "dg_anneal_forward": [vp, vp, vp, i32, ctypes.POINTER(dg_anneal_params), vp, vp,
-                                  vp, vp, vp],
+                                  vp, vp, vp, vp, vp],
             "dg_anneal_sample": [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32,
                                  ctypes.POINTER(dg_anneal_params), vp, vp],
             "dg_anneal_init": [vp, vp, vp, i32, i32, i32, vp, vp],
@@ -350,17 +350,26 @@ def dg_generate_block_annealed(model: Model, kv: KV, seeds, params=None, canvas_
     return canvas_out, n_forwards
 
 
-def dg_anneal_forward(model: Model, kv: KV, canvas, k: int, seeds, params=None, stream=None):
-    """Step k's forward: (tempered entropy [B, C], argmax [B, C], Gumbel-max draw [B, C])."""
+def dg_anneal_forward(model: Model, kv: KV, canvas, k: int, seeds, params=None, z_in=None,
+                      want_z=False, stream=None):
+    """Step k's forward: (tempered entropy [B, C], argmax [B, C], Gumbel-max draw [B, C]),
+    and with want_z the self-conditioning signal it hands on [B, C, d] (z_in: the one
+    it receives, in the model's accumulate type)."""
     p = _params(params)
     sd = _seeds(seeds, kv.B)
     B, C = canvas.shape
+    c = model.cfg
+    zt = torch.float64 if c.dtype == _DTYPES["f32"] else torch.float32
+    if z_in is not None and (z_in.dtype != zt or tuple(z_in.shape) != (B, C, c.d_model)):
+        raise ValueError(f"z_in must be {zt} of shape {(B, C, c.d_model)}")
     H = torch.empty(B, C, dtype=torch.float32, device="cuda")
     am = torch.empty(B, C, dtype=torch.int32, device="cuda")
     smp = torch.empty(B, C, dtype=torch.int32, device="cuda")
+    z_out = torch.empty(B, C, c.d_model, dtype=zt, device="cuda") if want_z else None
     _check(lib().dg_anneal_forward(model.handle, kv.handle, _ptr(canvas), k, ctypes.byref(p),
-                                   _ptr(sd), _ptr(H), _ptr(am), _ptr(smp), _stream(stream)))
-    return H, am, smp
+                                   _ptr(sd), _ptr(H), _ptr(am), _ptr(smp), _ptr(z_in),
+                                   _ptr(z_out), _stream(stream)))
+    return (H, am, smp, z_out) if want_z else (H, am, smp)
 
 
 def dg_anneal_sample(entropy, argmax, sampled, canvas, prev_argmax, state, k: int, V: int,

@@ -1426,7 +1426,8 @@ dg_status dg_generate_block_annealed(dg_model* m, const dg_kv* kv, const dg_anne
 
 dg_status dg_anneal_forward(dg_model* m, const dg_kv* kv, const int32_t* canvas, int32_t k,
                             const dg_anneal_params* p, const uint64_t* seeds, float* entropy,
-                            int32_t* argmax, int32_t* sampled, void* stream) {
+                            int32_t* argmax, int32_t* sampled, const void* z_in, void* z_out,
+                            void* stream) {
   g_err.clear();
   DG_REQUIRE(canvas && seeds && entropy && argmax && sampled, "null argument");
   AnnealQ q;
@@ -1434,9 +1435,10 @@ dg_status dg_anneal_forward(dg_model* m, const dg_kv* kv, const int32_t* canvas,
   DG_TRY(anneal_check(p, m->cfg.vocab, &q));
   DG_REQUIRE(k >= 0 && k < p->N, "k=%d outside [0, N=%d)", k, p->N);
   DG_TRY(check_step_args(m, kv, p->N - k, p->N));
+  DG_REQUIRE(!z_out || m->cfg.sc_inter > 0, "the model has no self-conditioning FFW");
   return run_forward(m, kv, canvas, p->N - k, p->N, entropy, argmax, nullptr, nullptr, nullptr,
                      (cudaStream_t)stream, nullptr, anneal_dev(m, p, seeds, p->N - k, nullptr),
-                     sampled);
+                     sampled, z_in, z_out);
 }
 
 dg_status dg_anneal_sample(const float* entropy, const int32_t* argmax, const int32_t* sampled,

@@ -9,6 +9,8 @@ oracle.model.selfcond / CanvasForwards.
     relative, the next forward's entropies with the oracle's z fed in; the block as a
     loop graph equals the plain launches; switched off, the block equals that of the
     same weights without the FFW;
+  * the annealed forward with self-conditioning (tempered statistics and draws, p0 at
+    temperature 1): tiny exact, small bf16 within 2e-2 and on decided draws;
   * one full-size layer (V = 262,144: p0 over the whole vocabulary, 16 K slices):
     the entropies and z against the golden file (2e-2, or 1.5x the oracle's
     bf16-storage distance where that exceeds 1e-2).
@@ -213,6 +215,84 @@ def test_full_size_layer_z():
         # z ends a chain of bf16 stores (p0, y = p0 E, the FFW's hidden rows) and a
         # cancelling sum over d: the storage-noise rule of the deep tests applies
         assert max_abs_rel(z[0].cpu().numpy(), g["z"]) < storage_tol(g, "z", 2e-2)
+        kv.close()
+    finally:
+        model.close()
+
+
+# --- self-conditioning inside the annealed forward (p0 at temperature 1 while the
+# statistics and the draw are tempered) ---------------------------------------------------
+def _anneal_sc_oracle(ws, okv_or_prompt, canvas, k, seed, p, z, w, prefilled):
+    if prefilled:
+        st = om.denoise_forward(ws, okv_or_prompt, canvas, p.N - k, p.N, w.prompt_len,
+                                want_logits=True, z=z)
+    else:
+        st = om.prefill_then_forward(ws, okv_or_prompt, canvas, p.N - k, p.N,
+                                     want_logits=True, z=z)
+    tau = an.temperature(k, p)
+    ts = an.tempered_stats(st["logits"], tau)
+    drawn, gap = an.sample_tokens(st["logits"], tau, seed, k)
+    return ts, drawn, gap, om.selfcond(ws, st["logits"])
+
+
+def test_tiny_annealed_forward_with_selfcond():
+    from masked_discrete_diffusion_b200 import binding
+    w = workloads.TINY_F32_SC
+    model = make_model(w)
+    try:
+        prompt = model_inputs.prompt(w, "cuda")
+        kv = binding.dg_prefill(model, prompt)
+        ws = om.Weights(w, keep_layers=True)
+        okv = om.prefill(ws, prompt[0].cpu().numpy())
+        p, seed, k = an.Params(), 5, 3
+        canvas = an.initial_canvas(seed, w.canvas, w.vocab)
+        z0 = om.selfcond(ws, om.denoise_forward(ws, okv, canvas, p.N, p.N, w.prompt_len,
+                                                want_logits=True)["logits"])
+        H, am, smp, z = binding.dg_anneal_forward(
+            model, kv, torch.from_numpy(canvas.astype(np.int32)).reshape(1, -1).cuda(), k, [seed],
+            p, z_in=torch.from_numpy(z0).reshape(1, w.canvas, w.d_model).cuda(), want_z=True)
+        binding.dg_sync_status(model)
+        ts, drawn, _, oz = _anneal_sc_oracle(ws, okv, canvas, k, seed, p, z0, w, True)
+        assert max_abs_rel(H[0].cpu().numpy(), ts["H64"]) < 1e-6
+        assert np.array_equal(am[0].cpu().numpy(), ts["argmax"])
+        assert np.array_equal(smp[0].cpu().numpy(), drawn)
+        assert max_abs_rel(z[0].cpu().numpy(), oz) < 1e-9
+        kv.close()
+    finally:
+        model.close()
+
+
+def test_small_bf16_annealed_forward_with_selfcond():
+    """The tensor-core epilogue that both draws (tempered) and stores p0 (temperature
+    1): entropies and z within 2e-2, draws equal where the race is decided."""
+    from masked_discrete_diffusion_b200 import binding
+    w = workloads.SMALL_BF16_SC
+    model = make_model(w)
+    try:
+        prompt = model_inputs.prompt(w, "cuda")
+        kv = binding.dg_prefill(model, prompt)
+        ws = om.Weights(w, keep_layers=True)
+        p, k = an.Params(), 4
+        seeds = [41 + b for b in range(w.batch)]
+        canvas = np.stack([an.initial_canvas(s, w.canvas, w.vocab) for s in seeds])
+        z0 = [om.selfcond(ws, om.prefill_then_forward(ws, prompt[b].cpu().numpy(), canvas[b],
+                                                      p.N, p.N, want_logits=True)["logits"])
+              for b in range(w.batch)]
+        H, am, smp, z = binding.dg_anneal_forward(
+            model, kv, torch.from_numpy(canvas.astype(np.int32)).cuda(), k, seeds, p,
+            z_in=torch.from_numpy(np.stack(z0).astype(np.float32)).cuda(), want_z=True)
+        binding.dg_sync_status(model)
+        decided = total = 0
+        for b in range(w.batch):
+            ts, drawn, gap, oz = _anneal_sc_oracle(ws, prompt[b].cpu().numpy(), canvas[b], k,
+                                                   seeds[b], p, z0[b], w, False)
+            assert max_abs_rel(H[b].cpu().numpy(), ts["H64"]) < 2e-2
+            assert max_abs_rel(z[b].cpu().numpy(), oz) < 2e-2
+            ok = gap > 0.05
+            assert np.array_equal(smp[b].cpu().numpy()[ok], drawn[ok])
+            decided += int(ok.sum())
+            total += len(ok)
+        assert decided >= 0.9 * total
         kv.close()
     finally:
         model.close()
