@@ -173,9 +173,12 @@ def test_tiny_blocks_token_for_token(tau):
 
 
 # --- bf16 models: entropies within tolerance, draws where the race is decided ------------
-def test_small_bf16_forward_decided_draws():
+@pytest.mark.parametrize("vocab", [1024, 999])
+def test_small_bf16_forward_decided_draws(vocab):
+    """V = 999: the last vocabulary tile is partial and the last token owns half of a
+    stream output (odd V)."""
     from masked_discrete_diffusion_b200 import binding
-    w = workloads.SMALL_BF16
+    w = workloads.SMALL_BF16.with_(vocab=vocab)
     p, k = an.Params(), 3
     seeds = _seeds(w.batch, 3)
     model = make_model(w)

@@ -114,9 +114,11 @@ def test_tiny_annealed_block_token_for_token(tau):
         model.close()
 
 
-def test_small_bf16_z_and_next_forward():
+@pytest.mark.parametrize("vocab", [1024, 1000])
+def test_small_bf16_z_and_next_forward(vocab):
+    """V = 1000: p0's last vocabulary tile is partial."""
     from masked_discrete_diffusion_b200 import binding
-    w = workloads.SMALL_BF16_SC
+    w = workloads.SMALL_BF16_SC.with_(vocab=vocab)
     model = make_model(w)
     try:
         prompt = model_inputs.prompt(w, "cuda")
