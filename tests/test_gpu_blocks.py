@@ -108,3 +108,32 @@ def test_full_size_layer_append():
         kv.close()
     finally:
         model.close()
+
+
+@pytest.mark.parametrize("name", ["tiny-f32", "tiny-f32-sc"])
+def test_tiny_annealed_blocks_with_append_exact(name):
+    """Block-autoregressive generation with the Report's sampler: an annealed block, its
+    causal append, a second annealed block conditioned on prompt + first block; both
+    blocks token for token against the oracle's annealed blocks over the same contexts
+    (with self-conditioning: z starts from 0 again in the second block)."""
+    from masked_discrete_diffusion_b200 import binding
+    from oracle import anneal as an
+    w = workloads.get(name)
+    p = an.Params(tau_max=0.02, tau_min=0.02)      # canvas 0 of this prompt stops early
+    model = make_model(w, max_prompt=w.prompt_len + w.canvas)
+    try:
+        prompt = model_inputs.prompt(w, "cuda")
+        kv = binding.dg_prefill(model, prompt)
+        b1, nf1 = binding.dg_generate_block_annealed(model, kv, [7], p)
+        binding.dg_append_block(model, kv, b1)
+        b2, nf2 = binding.dg_generate_block_annealed(model, kv, [8], p)
+        binding.dg_sync_status(model)
+        ws = om.Weights(w, keep_layers=True)
+        ctx = prompt[0].cpu().numpy()
+        r1, t1 = om.generate_block_annealed(ws, ctx, 7, p)
+        r2, t2 = om.generate_block_annealed(ws, np.concatenate([ctx, r1]), 8, p)
+        assert np.array_equal(b1[0].cpu().numpy(), r1) and int(nf1[0]) == len(t1)
+        assert np.array_equal(b2[0].cpu().numpy(), r2) and int(nf2[0]) == len(t2)
+        kv.close()
+    finally:
+        model.close()
