@@ -116,10 +116,14 @@ const char* dg_last_error(void);
 
 /* Validates the configuration and weight pointers, plans the kernels and
  * allocates the library's device workspace for max_batch canvases and prompts
- * up to max_prompt tokens, on the current CUDA device.  Synchronous.
+ * up to max_prompt tokens, on the current CUDA device.  Synchronous.  With
+ * sc_inter > 0 it also builds the transposed embedding [d, V] the self-conditioning
+ * product reads and the workspace for p0 [max_batch C, V] (bf16 on the bf16 paths).
  * Errors: DG_ERR_INVALID_ARG (null, non-positive or inconsistent sizes, d_model not a
  * multiple of 8, C > 1024,
- * Hq not a multiple of Hkv, h odd), DG_ERR_UNSUPPORTED (a shape the tensor-core
+ * Hq not a multiple of Hkv, h odd; with sc_inter > 0: a null FFW pointer, V not a
+ * multiple of 2 (fp32) or 8 (bf16), sc_inter not a multiple of 64 (bf16)),
+ * DG_ERR_UNSUPPORTED (a shape the tensor-core
  * kernels do not tile: bf16 and FP8 need d % 256, I % 128, Is % 64, (Hq + 2 Hkv) h % 64
  * and Hq h % 64; FP8 experts also d, I <= 4096), DG_ERR_OOM, DG_ERR_CUDA. */
 dg_status dg_model_create(const dg_config* cfg, const dg_weights* w, dg_model** out);
