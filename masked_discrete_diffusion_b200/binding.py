@@ -4,6 +4,14 @@ Every function below forwards to the C entry point of the same name; device
 buffers are passed as torch CUDA tensors (PyTorch supplies device memory and
 streams).  There is no fallback: if libdg.so is missing or a call fails, an
 exception is raised.
+
+The calls come in four groups: model and batch set-up; one denoising forward
+with the entropy-bounded (EB) draw and the whole EB generation loop, for one
+block or with block appends; the annealed sampler (tempered Gumbel-max draws,
+acceptance of the lowest-entropy prefix, re-noising of the rest), as one forward
+or as the whole loop; and self-conditioning, where the tensor z that a forward
+leaves behind is fed into the canvas input of the next one.  Tensors for z hold
+the model's accumulate type: fp64 for the f32 model, fp32 for the bf16 ones.
 """
 from __future__ import annotations
 
