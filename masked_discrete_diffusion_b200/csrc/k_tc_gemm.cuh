@@ -958,8 +958,10 @@ __global__ void __launch_bounds__(TC_DENSE_THREADS, 1)
 // phase-1 units (counted in ready[c]); those were taken earlier by running blocks,
 // whose progress never depends on a waiting block, so every wait ends.
 // Both phases run two MMAs per k-step (weights on the MMA's M side, tokens on N)
-// into TMEM columns 0 and 128.  320 threads: warp 0 TMA, warp 1 MMA, warps 2..9
-// epilogue (warps w and w + 4 share a TMEM lane quarter and split the token chunks).
+// into TMEM columns 0 and 128.  576 threads: warp 0 TMA, warp 1 MMA, warps 2..17
+// epilogue (warps w, w + 4, w + 8 and w + 12 share a TMEM lane quarter and take one
+// 32-token chunk each, so that each thread's share of the SwiGLU and of the stores is
+// a quarter of a unit's).
 // ---------------------------------------------------------------------------
 template <int ST>
 struct MoeCfg {
@@ -968,7 +970,8 @@ struct MoeCfg {
   static constexpr uint32_t TCOLS = 256;
   static constexpr size_t SMEM = 1024 + (size_t)ST * STAGE + 256;
 };
-constexpr int TC_MOE_THREADS = 320;
+constexpr int MOE_EPI_WARPS = 16;
+constexpr int TC_MOE_THREADS = 64 + 32 * MOE_EPI_WARPS;
 
 template <int ST>
 __global__ void __launch_bounds__(TC_MOE_THREADS, 1)
@@ -990,7 +993,7 @@ __global__ void __launch_bounds__(TC_MOE_THREADS, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + ST * Cfg::STAGE);
   uint64_t* empty = full + ST;
   uint64_t* tfull = empty + ST;   // accumulators ready (MMA -> epilogue)
-  uint64_t* tempty = tfull + 1;   // accumulators drained (epilogue -> MMA), 8 arrivals
+  uint64_t* tempty = tfull + 1;   // accumulators drained (epilogue -> MMA), one per epilogue warp
   // units taken by the TMA thread, in order, for the MMA thread and the epilogue leader
   constexpr int QD = 4;
   uint64_t* qfull = tempty + 1;   // [QD] unit id written (TMA thread)
@@ -1009,7 +1012,7 @@ __global__ void __launch_bounds__(TC_MOE_THREADS, 1)
       tc::mbar_init(empty + s, 1);
     }
     tc::mbar_init(tfull, 1);
-    tc::mbar_init(tempty, 8);
+    tc::mbar_init(tempty, MOE_EPI_WARPS);
     for (int k = 0; k < QD; ++k) {
       tc::mbar_init(qfull + k, 1);
       tc::mbar_init(qempty + k, 2);
@@ -1160,15 +1163,16 @@ __global__ void __launch_bounds__(TC_MOE_THREADS, 1)
       }
     }
   } else {
-    // epilogue warps 2..9 -> TMEM lane quarter (warp % 4), token chunks of parity hf
-    const int q = warp & 3, hf = (warp - 2) >> 2;
+    // epilogue warps 2..17 -> TMEM lane quarter (warp % 4), token chunks part, part + 4, ..
+    constexpr int NP = MOE_EPI_WARPS / 4;
+    const int q = warp & 3, part = (warp - 2) >> 2;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     for (int ui = 0;; ++ui) {
-      // warp 2 takes the unit id for the eight epilogue warps
+      // warp 2 takes the unit id for the epilogue warps
       if (warp == 2 && lane == 0) *reinterpret_cast<volatile int32_t*>(ubc) = take(ui);
-      asm volatile("bar.sync 1, 256;" ::: "memory");
+      asm volatile("bar.sync 1, %0;" ::"n"(32 * MOE_EPI_WARPS) : "memory");
       const int u = *reinterpret_cast<volatile int32_t*>(ubc);
-      asm volatile("bar.sync 1, 256;" ::: "memory");  // read by all before the next take
+      asm volatile("bar.sync 1, %0;" ::"n"(32 * MOE_EPI_WARPS) : "memory");  // read by all before the next take
       if (u >= n_units) break;
       const Unit x = unit_of(u);
       bool rdy = true;
@@ -1182,7 +1186,7 @@ __global__ void __launch_bounds__(TC_MOE_THREADS, 1)
       if (!x.down) {
         const int fr = x.f * 128 + 32 * q + lane;  // hidden column
 #pragma unroll 1
-        for (int c = hf; c < nch; c += 2) {
+        for (int c = part; c < nch; c += NP) {
           float g[32], v[32];
           tc::tmem_ld32(tmem + lane_base + c * 32, g);
           tc::tmem_ld32(tmem + lane_base + 128 + c * 32, v);
@@ -1197,7 +1201,7 @@ __global__ void __launch_bounds__(TC_MOE_THREADS, 1)
         for (int half2 = 0; half2 < 2; ++half2) {
           const int fr = x.f * 256 + half2 * 128 + 32 * q + lane;  // output column
 #pragma unroll 1
-          for (int c = hf; c < nch; c += 2) {
+          for (int c = part; c < nch; c += NP) {
             float v[32];
             tc::tmem_ld32(tmem + lane_base + half2 * 128 + c * 32, v);
 #pragma unroll
@@ -1214,7 +1218,7 @@ __global__ void __launch_bounds__(TC_MOE_THREADS, 1)
       if (!x.down) {
         // this unit's hidden columns are written: count it for the chunk's phase-2 units
         __threadfence();
-        asm volatile("bar.sync 1, 256;" ::: "memory");  // the eight epilogue warps
+        asm volatile("bar.sync 1, %0;" ::"n"(32 * MOE_EPI_WARPS) : "memory");  // the epilogue warps
         if (warp == 2 && lane == 0) atomicAdd(ready + x.c, 1);
       }
     }
