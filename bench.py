@@ -27,12 +27,12 @@ sys.path.insert(0, ROOT)
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per routed expert streamed
-# by the routed-expert kernel as it now stands: one ncu capture of the 12 launches of
-# a one-layer block (layer1-bf16, same kernel shapes as one layer of the 30-layer
-# workload; profiles/tc_moe_kernel_layer1-bf16.md): 1,274.9 MB over 123 streamed
-# experts = 10,365,317 B each, 1.10x the 9,437,184 B of weights (the rest: gathered and
-# hidden rows, which ncu's cold cache sends to DRAM).
-DRAM_BYTES_PER_EXPERT = 10365317
+# by the routed-expert kernel as it now stands (sixteen epilogue warps): one ncu capture
+# of the 12 launches of a one-layer block (layer1-bf16, same kernel shapes as one layer
+# of the 30-layer workload; profiles/tc_moe_kernel_layer1-bf16.md): 1,272.8 MB over 123
+# streamed experts = 10,347,882 B each, 1.10x the 9,437,184 B of weights (the rest:
+# gathered and hidden rows, which ncu's cold cache sends to DRAM).
+DRAM_BYTES_PER_EXPERT = 10347882
 
 
 def load_peaks():
