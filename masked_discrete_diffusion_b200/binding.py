@@ -177,6 +177,30 @@ def _ptr(t) -> int | None:
     return t.data_ptr()
 
 
+def _arg(t, name: str, dtype, shape):
+    """Device pointer of a caller tensor after checking what the C entry point assumes
+    about it: a contiguous CUDA tensor on the current device with exactly this dtype and
+    shape (the library reads or writes that many elements of that type, so anything
+    else would be read or written out of bounds, or misread).  None stays None."""
+    if t is None:
+        return None
+    if not torch.is_tensor(t):
+        raise ValueError(f"{name} must be a tensor")
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must be {dtype} of shape {tuple(shape)}, got {t.dtype} "
+                         f"{tuple(t.shape)}")
+    if not t.is_cuda or t.device.index != torch.cuda.current_device():
+        raise ValueError(f"{name} must be a CUDA tensor on the current device")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _z_type(model) -> torch.dtype:
+    """Accumulate type of a model: that of its self-conditioning signal z."""
+    return torch.float64 if model.cfg.dtype == DG_F32 else torch.float32
+
+
 def _stream(stream=None) -> int | None:
     s = stream if stream is not None else torch.cuda.current_stream()
     return s.cuda_stream or None
@@ -260,28 +284,30 @@ def dg_sync_status(model: Model, stream=None):
 
 
 def dg_prefill(model: Model, prompt: torch.Tensor, stream=None) -> KV:
-    assert prompt.dtype == torch.int32 and prompt.dim() == 2
+    if not torch.is_tensor(prompt) or prompt.dim() != 2:
+        raise ValueError("prompt must be a 2-D int32 tensor")
+    pp = _arg(prompt, "prompt", torch.int32, prompt.shape)
     h = ctypes.c_void_p()
-    _check(lib().dg_prefill(model.handle, _ptr(prompt), prompt.shape[0], prompt.shape[1],
+    _check(lib().dg_prefill(model.handle, pp, prompt.shape[0], prompt.shape[1],
                             ctypes.byref(h), _stream(stream)))
     return KV(model, h)
 
 
 def dg_prefill_into(model: Model, prompt: torch.Tensor, kv: KV, stream=None) -> KV:
     """Causal pass of prompt [B, P] into an existing handle of the same B."""
-    if prompt.dtype != torch.int32 or prompt.dim() != 2:
+    if not torch.is_tensor(prompt) or prompt.dim() != 2:
         raise ValueError("prompt must be a 2-D int32 tensor")
     B, P = prompt.shape
-    _check(lib().dg_prefill_into(model.handle, _ptr(prompt), B, P, kv.handle, _stream(stream)))
+    pp = _arg(prompt, "prompt", torch.int32, (B, P))
+    _check(lib().dg_prefill_into(model.handle, pp, B, P, kv.handle, _stream(stream)))
     kv.refresh()
     return kv
 
 
 def dg_append_block(model: Model, kv: KV, tokens: torch.Tensor, stream=None) -> KV:
     """Causal pass of the finished blocks tokens [B, C] into kv (the context grows by C)."""
-    if tokens.dtype != torch.int32 or tokens.dim() != 2:
-        raise ValueError("tokens must be a 2-D int32 tensor")
-    _check(lib().dg_append_block(model.handle, kv.handle, _ptr(tokens), _stream(stream)))
+    tp = _arg(tokens, "tokens", torch.int32, (kv.B, model.cfg.canvas))
+    _check(lib().dg_append_block(model.handle, kv.handle, tp, _stream(stream)))
     kv.refresh()
     return kv
 
@@ -311,13 +337,17 @@ def dg_kv_read(kv: KV, stream=None):
 
 def dg_denoise_step(model: Model, kv: KV, canvas, mask, steps_left: int, T: int, gamma: float,
                     entropy=None, argmax=None, n_committed=None, stream=None):
-    B, C = canvas.shape
+    B, C = kv.B, model.cfg.canvas
+    cp = _arg(canvas, "canvas", torch.int32, (B, C))
+    mp = _arg(mask, "mask", torch.uint8, (B, C))
     entropy = entropy if entropy is not None else torch.empty(B, C, dtype=torch.float32, device="cuda")
     argmax = argmax if argmax is not None else torch.empty(B, C, dtype=torch.int32, device="cuda")
     n_committed = (n_committed if n_committed is not None
                    else torch.empty(B, dtype=torch.int32, device="cuda"))
-    _check(lib().dg_denoise_step(model.handle, kv.handle, _ptr(canvas), _ptr(mask), steps_left,
-                                 T, gamma, _ptr(entropy), _ptr(argmax), _ptr(n_committed),
+    _check(lib().dg_denoise_step(model.handle, kv.handle, cp, mp, steps_left, T, gamma,
+                                 _arg(entropy, "entropy", torch.float32, (B, C)),
+                                 _arg(argmax, "argmax", torch.int32, (B, C)),
+                                 _arg(n_committed, "n_committed", torch.int32, (B,)),
                                  _stream(stream)))
     return entropy, argmax, n_committed
 
@@ -327,17 +357,28 @@ def dg_generate_block(model: Model, kv: KV, T: int, gamma: float, canvas_out=Non
     c = model.cfg
     canvas_out = (canvas_out if canvas_out is not None
                   else torch.empty(kv.B, c.canvas, dtype=torch.int32, device="cuda"))
-    _check(lib().dg_generate_block(model.handle, kv.handle, T, gamma, _ptr(canvas_out),
-                                   _ptr(n_forwards), _ptr(router_load), _stream(stream)))
+    _check(lib().dg_generate_block(model.handle, kv.handle, T, gamma,
+                                   _arg(canvas_out, "canvas_out", torch.int32, (kv.B, c.canvas)),
+                                   _arg(n_forwards, "n_forwards", torch.int32, (kv.B,)),
+                                   _arg(router_load, "router_load", torch.int32,
+                                        (c.n_layers, c.n_experts)),
+                                   _stream(stream)))
     return canvas_out
 
 
 def dg_eb_sample(entropy, argmax, canvas, mask, steps_left: int, gamma: float,
                  n_committed=None, stream=None):
+    if not torch.is_tensor(entropy) or entropy.dim() != 2:
+        raise ValueError("entropy must be a 2-D float32 tensor")
     B, C = entropy.shape
+    ep = _arg(entropy, "entropy", torch.float32, (B, C))
+    ap = _arg(argmax, "argmax", torch.int32, (B, C))
+    cp = _arg(canvas, "canvas", torch.int32, (B, C))
+    mp = _arg(mask, "mask", torch.uint8, (B, C))
     n_committed = (n_committed if n_committed is not None
                    else torch.empty(B, dtype=torch.int32, device="cuda"))
-    _check(lib().dg_eb_sample(_ptr(entropy), _ptr(argmax), _ptr(canvas), _ptr(mask), B, C,
+    _arg(n_committed, "n_committed", torch.int32, (B,))
+    _check(lib().dg_eb_sample(ep, ap, cp, mp, B, C,
                               steps_left, gamma, _ptr(n_committed), _stream(stream)))
     return n_committed
 
@@ -352,9 +393,10 @@ def dg_generate_block_annealed(model: Model, kv: KV, seeds, params=None, canvas_
                   else torch.empty(kv.B, c.canvas, dtype=torch.int32, device="cuda"))
     n_forwards = (n_forwards if n_forwards is not None
                   else torch.empty(kv.B, dtype=torch.int32, device="cuda"))
-    _check(lib().dg_generate_block_annealed(model.handle, kv.handle, ctypes.byref(p), _ptr(sd),
-                                            _ptr(canvas_out), _ptr(n_forwards),
-                                            _stream(stream)))
+    _check(lib().dg_generate_block_annealed(
+        model.handle, kv.handle, ctypes.byref(p), _ptr(sd),
+        _arg(canvas_out, "canvas_out", torch.int32, (kv.B, c.canvas)),
+        _arg(n_forwards, "n_forwards", torch.int32, (kv.B,)), _stream(stream)))
     return canvas_out, n_forwards
 
 
@@ -363,19 +405,19 @@ def dg_anneal_forward(model: Model, kv: KV, canvas, k: int, seeds, params=None, 
     """Step k's forward: (tempered entropy [B, C], argmax [B, C], Gumbel-max draw [B, C]),
     and with want_z the self-conditioning signal it hands on [B, C, d] (z_in: the one
     it receives, in the model's accumulate type)."""
+    c = model.cfg
+    B, C = kv.B, c.canvas
+    zt = _z_type(model)
+    cp = _arg(canvas, "canvas", torch.int32, (B, C))
+    zp = _arg(z_in, "z_in", zt, (B, C, c.d_model))
     p = _params(params)
     sd = _seeds(seeds, kv.B)
-    B, C = canvas.shape
-    c = model.cfg
-    zt = torch.float64 if c.dtype == _DTYPES["f32"] else torch.float32
-    if z_in is not None and (z_in.dtype != zt or tuple(z_in.shape) != (B, C, c.d_model)):
-        raise ValueError(f"z_in must be {zt} of shape {(B, C, c.d_model)}")
     H = torch.empty(B, C, dtype=torch.float32, device="cuda")
     am = torch.empty(B, C, dtype=torch.int32, device="cuda")
     smp = torch.empty(B, C, dtype=torch.int32, device="cuda")
     z_out = torch.empty(B, C, c.d_model, dtype=zt, device="cuda") if want_z else None
-    _check(lib().dg_anneal_forward(model.handle, kv.handle, _ptr(canvas), k, ctypes.byref(p),
-                                   _ptr(sd), _ptr(H), _ptr(am), _ptr(smp), _ptr(z_in),
+    _check(lib().dg_anneal_forward(model.handle, kv.handle, cp, k, ctypes.byref(p),
+                                   _ptr(sd), _ptr(H), _ptr(am), _ptr(smp), zp,
                                    _ptr(z_out), _stream(stream)))
     return (H, am, smp, z_out) if want_z else (H, am, smp)
 
@@ -383,12 +425,22 @@ def dg_anneal_forward(model: Model, kv: KV, canvas, k: int, seeds, params=None, 
 def dg_anneal_sample(entropy, argmax, sampled, canvas, prev_argmax, state, k: int, V: int,
                      seeds, params=None, stream=None):
     """Step k's refinement in place (canvas, prev_argmax, state); returns n_accepted [B]."""
-    p = _params(params)
+    if not torch.is_tensor(entropy) or entropy.dim() != 2:
+        raise ValueError("entropy must be a 2-D float32 tensor")
     B, C = entropy.shape
+    ptrs = [_arg(entropy, "entropy", torch.float32, (B, C))]
+    for name, t in (("argmax", argmax), ("sampled", sampled), ("canvas", canvas),
+                    ("prev_argmax", prev_argmax)):
+        if t is None:
+            raise ValueError(f"{name} is required")
+        ptrs.append(_arg(t, name, torch.int32, (B, C)))
+    if state is None:
+        raise ValueError("state is required")
+    ptrs.append(_arg(state, "state", torch.int32, (B,)))
+    p = _params(params)
     sd = _seeds(seeds, B)
     nacc = torch.empty(B, dtype=torch.int32, device="cuda")
-    _check(lib().dg_anneal_sample(_ptr(entropy), _ptr(argmax), _ptr(sampled), _ptr(canvas),
-                                  _ptr(prev_argmax), _ptr(state), _ptr(nacc), B, C, V, k,
+    _check(lib().dg_anneal_sample(*ptrs[:6], _ptr(nacc), B, C, V, k,
                                   ctypes.byref(p), _ptr(sd), _stream(stream)))
     return nacc
 
@@ -413,28 +465,29 @@ def dg_selfcond_forward(model: Model, kv: KV, canvas, steps_left: int, T: int, z
     """(entropy [B, C], argmax [B, C], z_out [B, C, d]); z in the model's accumulate type
     (float64 for the fp32 model, float32 otherwise)."""
     c = model.cfg
-    B, C = canvas.shape
-    zt = torch.float64 if c.dtype == _DTYPES["f32"] else torch.float32
-    if z_in is not None and (z_in.dtype != zt or tuple(z_in.shape) != (B, C, c.d_model)):
-        raise ValueError(f"z_in must be {zt} of shape {(B, C, c.d_model)}")
+    B, C = kv.B, c.canvas
+    zt = _z_type(model)
+    cp = _arg(canvas, "canvas", torch.int32, (B, C))
+    zp = _arg(z_in, "z_in", zt, (B, C, c.d_model))
     H = torch.empty(B, C, dtype=torch.float32, device="cuda")
     am = torch.empty(B, C, dtype=torch.int32, device="cuda")
     z_out = torch.empty(B, C, c.d_model, dtype=zt, device="cuda")
-    _check(lib().dg_selfcond_forward(model.handle, kv.handle, _ptr(canvas), steps_left, T,
-                                     _ptr(z_in), _ptr(H), _ptr(am), _ptr(z_out), _stream(stream)))
+    _check(lib().dg_selfcond_forward(model.handle, kv.handle, cp, steps_left, T,
+                                     zp, _ptr(H), _ptr(am), _ptr(z_out), _stream(stream)))
     return H, am, z_out
 
 
 def dg_debug_forward(model: Model, kv: KV, canvas, steps_left: int, T: int, logits=False,
                      hidden=False, stream=None):
     c = model.cfg
-    B, C = canvas.shape
+    B, C = kv.B, c.canvas
+    cp = _arg(canvas, "canvas", torch.int32, (B, C))
     n = B * C
     ent = torch.empty(B, C, dtype=torch.float32, device="cuda")
     am = torch.empty(B, C, dtype=torch.int32, device="cuda")
     lg = torch.empty(n, c.vocab, dtype=torch.float32, device="cuda") if logits else None
     hd = torch.empty(n, c.d_model, dtype=torch.float32, device="cuda") if hidden else None
-    _check(lib().dg_debug_forward(model.handle, kv.handle, _ptr(canvas), steps_left, T,
+    _check(lib().dg_debug_forward(model.handle, kv.handle, cp, steps_left, T,
                                   _ptr(ent), _ptr(am), _ptr(lg), _ptr(hd), _stream(stream)))
     return ent, am, lg, hd
 
