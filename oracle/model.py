@@ -84,6 +84,11 @@ class Weights:
             from synth import fp8
             a = fp8.dequantised(self.w, name, shape, start_row, n_rows).astype(np.float64)
             return self.store(a)
+        if model_inputs.is_fp4_expert(self.w, name):
+            from synth import nvfp4
+            a = nvfp4.dequantised(self.w, name, shape, model_inputs.std_of(self.w, name),
+                                  start_row, n_rows)
+            return self.store(a)
         t = model_inputs.weight(self.w, name, shape, "cpu", start_row, n_rows)
         return t.to(torch.float64).numpy()
 

@@ -15,7 +15,7 @@ Weight tensors (row-major, the leading index is the output row):
   l{l}.sdown     [d, I_s]
 Every tensor is drawn i.i.d. (approximately) N(0, init_std^2) and stored in the
 workload's dtype.  In the FP8-expert workloads the three routed-expert tensors are
-additionally quantised (see `synth.fp8`).
+additionally quantised (see `synth.fp8` and `synth.nvfp4`).
 
 Inputs: prompt[b] holds `prompt_len` tokens uniform in [0, V).
 """
@@ -93,6 +93,11 @@ def is_fp8_expert(w: Workload, name: str) -> bool:
             and name.split(".")[-1] in ("gate", "up", "down"))
 
 
+def is_fp4_expert(w: Workload, name: str) -> bool:
+    return (w.dtype == "bf16_fp4exp" and name.startswith("l")
+            and name.split(".")[-1] in ("gate", "up", "down"))
+
+
 def weight_set(w: Workload, device="cpu") -> dict:
     """Every weight tensor of the workload, keyed by name, in its stored dtype."""
     dt = torch.float32 if store_dtype(w) == "f32" else torch.bfloat16
@@ -102,6 +107,11 @@ def weight_set(w: Workload, device="cpu") -> dict:
             from . import fp8
             q, s = fp8.quantised(w, name, shape, device)
             out[name], out[name.rsplit(".", 1)[0] + "." + name.split(".")[-1] + "_scale"] = q, s
+            continue
+        if is_fp4_expert(w, name):
+            from . import nvfp4
+            q, s, st = nvfp4.quantised(w, name, shape, std_of(w, name), device)
+            out[name], out[name + "_scale"], out[name + "_tscale"] = q, s, st
             continue
         t = torch.empty(shape, dtype=dt, device=device)
         gen.fill_weight_(t, w.seed, name, std_of(w, name))

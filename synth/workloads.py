@@ -32,7 +32,7 @@ class Workload:
     rope_base: float
     rms_eps: float
     logit_scale: float
-    dtype: str            # "f32" | "bf16" | "bf16_fp8exp"
+    dtype: str            # "f32" | "bf16" | "bf16_fp8exp" | "bf16_fp4exp"
     batch: int
     prompt_len: int
     T: int                # denoise forwards per block
@@ -105,6 +105,17 @@ LAYER1_FP8 = LAYER1_BF16.with_(name="layer1-fp8exp-p4096", dtype="bf16_fp8exp", 
 LAYER1_P200_B2 = LAYER1_BF16.with_(name="layer1-bf16-p200-b2", prompt_len=200, batch=2)
 LAYER1_P200_B2_C96 = LAYER1_P200_B2.with_(name="layer1-bf16-p200-b2-c96", canvas=96)
 
+# NVFP4-expert variants (E2M1 codes, an E4M3 scale per 16 input columns and a
+# power-of-two scale per tensor): the small model and one full-size layer.
+SMALL_FP4 = SMALL_BF16.with_(name="small-fp4exp", dtype="bf16_fp4exp")
+LAYER1_FP4 = LAYER1_BF16.with_(name="layer1-fp4exp", dtype="bf16_fp4exp")
+
+
+def full30_fp4exp(batch: int) -> Workload:
+    """The 30-layer model with NVFP4 expert weights, prompt 1024, the given batch."""
+    return FULL30_BF16.with_(name=f"full30-fp4exp-b{batch}", dtype="bf16_fp4exp", batch=batch)
+
+
 # One FP8-expert layer at the batches where each expert holds several 128-row token
 # chunks (the tensor-bound part of the FP8 sweep).
 LAYER1_FP8_B16 = LAYER1_FP8.with_(name="layer1-fp8exp-p4096-b16", batch=16)
@@ -120,9 +131,11 @@ FULL30_BF16_SC = FULL30_BF16.with_(name="full30-bf16-sc", sc_inter=2048)
 WORKLOADS = {w.name: w for w in (TINY_F32, SMALL_BF16, LAYER1_BF16, FULL30_BF16,
                                  FULL30_B8_P8192, SMALL_FP8, LAYER1_FP8, LAYER1_P200_B2,
                                  LAYER1_P200_B2_C96, LAYER1_FP8_B16, LAYER1_FP8_B64,
-                                 TINY_F32_SC, SMALL_BF16_SC, LAYER1_BF16_SC, FULL30_BF16_SC)}
+                                 TINY_F32_SC, SMALL_BF16_SC, LAYER1_BF16_SC, FULL30_BF16_SC,
+                                 SMALL_FP4, LAYER1_FP4)}
 for _b in (1, 4, 16, 32, 64):
     WORKLOADS[f"full30-fp8exp-b{_b}"] = full30_fp8exp(_b)
+    WORKLOADS[f"full30-fp4exp-b{_b}"] = full30_fp4exp(_b)
 
 
 def get(name: str) -> Workload:
