@@ -57,7 +57,8 @@ typedef enum dg_status {
 typedef enum dg_dtype {
   DG_F32 = 0,        /* fp32 weights; the SIMT path carries activations in fp64 */
   DG_BF16 = 1,       /* bf16 weights and activations, fp32 accumulation          */
-  DG_BF16_FP8EXP = 2 /* as DG_BF16 but routed-expert weights in FP8 E4M3         */
+  DG_BF16_FP8EXP = 2, /* as DG_BF16 but routed-expert weights in FP8 E4M3        */
+  DG_BF16_FP4EXP = 3  /* as DG_BF16 but routed-expert weights in NVFP4            */
 } dg_dtype;
 
 typedef struct dg_config {
@@ -78,7 +79,14 @@ typedef struct dg_config {
 /* Weights of one layer (device pointers, borrowed for the model's lifetime).
  * Element type: fp32 for DG_F32, bf16 otherwise; for DG_BF16_FP8EXP the three
  * routed-expert tensors are FP8 E4M3 bytes with fp32 scales, one per
- * (row, 128 consecutive input columns): w = q * scale.                       */
+ * (row, 128 consecutive input columns): w = q * scale.  For DG_BF16_FP4EXP
+ * ("NVFP4", the agentlenshq page on DiffusionGemma: NVFP4 kernels for Blackwell)
+ * they are E2M1 codes packed two per byte ([E, I, d/2] and [E, d, I/2] bytes,
+ * element 2i in the low nibble), one E4M3 block scale byte per (row, 16 consecutive
+ * input columns) in the *_scale fields and one fp32 tensor scale per tensor in the
+ * *_tscale fields: w = e2m1(code) * block scale * tensor scale.  The kernel widens
+ * the codes to bf16 in shared memory, so a weight must be exact in fp32: the
+ * tensor scale must be a power of two. */
 typedef struct dg_layer_weights {
   const void* wqkv;   /* [(Hq + 2 Hkv) h, d]: query heads, key heads, value heads */
   const void* wo;     /* [d, Hq h]                                                */
@@ -86,12 +94,15 @@ typedef struct dg_layer_weights {
   const void* gate;   /* [E, I, d]                                                */
   const void* up;     /* [E, I, d]                                                */
   const void* down;   /* [E, d, I]                                                */
-  const float* gate_scale; /* [E, I, d/128]  FP8 only, else NULL                  */
-  const float* up_scale;   /* [E, I, d/128]                                       */
-  const float* down_scale; /* [E, d, I/128]                                       */
+  const void* gate_scale;  /* FP8: fp32 [E, I, d/128]; NVFP4: E4M3 [E, I, d/16]; else NULL */
+  const void* up_scale;    /* FP8: fp32 [E, I, d/128]; NVFP4: E4M3 [E, I, d/16]           */
+  const void* down_scale;  /* FP8: fp32 [E, d, I/128]; NVFP4: E4M3 [E, d, I/16]           */
   const void* sgate;  /* [Is, d]                                                  */
   const void* sup;    /* [Is, d]                                                  */
   const void* sdown;  /* [d, Is]                                                  */
+  const float* gate_tscale; /* NVFP4 only: fp32 [1] tensor scale, else NULL       */
+  const float* up_tscale;   /* NVFP4 only: fp32 [1]                               */
+  const float* down_tscale; /* NVFP4 only: fp32 [1]                               */
 } dg_layer_weights;
 
 typedef struct dg_weights {

@@ -24,8 +24,9 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libdg.so")
 
-DG_F32, DG_BF16, DG_BF16_FP8EXP = 0, 1, 2
-_DTYPES = {"f32": DG_F32, "bf16": DG_BF16, "bf16_fp8exp": DG_BF16_FP8EXP}
+DG_F32, DG_BF16, DG_BF16_FP8EXP, DG_BF16_FP4EXP = 0, 1, 2, 3
+_DTYPES = {"f32": DG_F32, "bf16": DG_BF16, "bf16_fp8exp": DG_BF16_FP8EXP,
+           "bf16_fp4exp": DG_BF16_FP4EXP}
 
 
 class DGError(RuntimeError):
@@ -46,7 +47,8 @@ class dg_config(ctypes.Structure):
 
 
 _LAYER_FIELDS = ("wqkv", "wo", "router", "gate", "up", "down", "gate_scale", "up_scale",
-                 "down_scale", "sgate", "sup", "sdown")
+                 "down_scale", "sgate", "sup", "sdown", "gate_tscale", "up_tscale",
+                 "down_tscale")
 
 
 class dg_layer_weights(ctypes.Structure):

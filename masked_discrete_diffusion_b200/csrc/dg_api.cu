@@ -409,7 +409,9 @@ template <class Path> struct Runner {
     if constexpr (Path::kTensorCores) {
       {
         ProfScope ps(m, DG_KIND_EXPERTS, st);
-        if (c.dtype == DG_BF16_FP8EXP) {
+        if (c.dtype == DG_BF16_FP4EXP) {
+          DG_TRY(tc_moe_experts_f4(m, l, (const TA*)ws.up, (TA*)ws.hb, (float*)ws.yb, st));
+        } else if (c.dtype == DG_BF16_FP8EXP) {
           DG_TRY(tc_moe_experts_f8(m, l, (const TA*)ws.up, (TA*)ws.hb, (float*)ws.yb, st));
         } else {
           DG_TRY(tc_moe_experts(m, l, (const TA*)ws.up, (TA*)ws.hb, (float*)ws.yb, st));
@@ -720,8 +722,14 @@ dg_status dg_model_create(const dg_config* cfg, const dg_weights* w, dg_model** 
   DG_REQUIRE(c.max_batch >= 1 && c.max_prompt >= 1, "bad max_batch/max_prompt");
   DG_REQUIRE(c.rms_eps >= 0.0f && std::isfinite(c.logit_scale) && c.rope_base > 0.0f,
              "bad eps/logit_scale/rope_base");
-  DG_REQUIRE(c.dtype == DG_F32 || c.dtype == DG_BF16 || c.dtype == DG_BF16_FP8EXP,
+  DG_REQUIRE(c.dtype == DG_F32 || c.dtype == DG_BF16 || c.dtype == DG_BF16_FP8EXP ||
+                 c.dtype == DG_BF16_FP4EXP,
              "unknown dtype %d", c.dtype);
+  if (c.dtype == DG_BF16_FP4EXP)
+    DG_REQUIRE(c.d_model % 32 == 0 && c.expert_inter % 32 == 0 && c.d_model <= 2048 &&
+                   c.expert_inter <= 2048,
+               "NVFP4 experts need d and I multiples of 32 and at most 2048 (a unit's block "
+               "scales are staged in shared memory)");
   if (c.dtype == DG_BF16_FP8EXP)
     DG_REQUIRE(c.d_model % 128 == 0 && c.expert_inter % 128 == 0,
                "FP8 experts need d and I multiples of 128 (one scale per 128 columns)");
@@ -742,6 +750,10 @@ dg_status dg_model_create(const dg_config* cfg, const dg_weights* w, dg_model** 
                "null weight pointer in layer %d", l);
     if (c.dtype == DG_BF16_FP8EXP)
       DG_REQUIRE(L.gate_scale && L.up_scale && L.down_scale, "null FP8 scale pointer in layer %d", l);
+    if (c.dtype == DG_BF16_FP4EXP)
+      DG_REQUIRE(L.gate_scale && L.up_scale && L.down_scale && L.gate_tscale && L.up_tscale &&
+                     L.down_tscale,
+                 "null NVFP4 scale pointer in layer %d", l);
   }
   dg_model* m = new dg_model();
   m->cfg = c;

@@ -1,16 +1,23 @@
 // Routed experts with FP8 E4M3 expert weights (one fp32 scale per weight row and 128
-// consecutive input columns) and bf16 activations: gate/up SwiGLU and down in one
-// persistent launch, with the schedule and device-side chunk counters of the bf16
-// routed-expert kernel (tc_moe_kernel).
+// consecutive input columns), or NVFP4 expert weights (E2M1 codes two per byte, one
+// E4M3 scale per weight row and 16 consecutive input columns, one fp32 power-of-two
+// scale per tensor), and bf16 activations: gate/up SwiGLU and down in one persistent
+// launch, with the schedule and device-side chunk counters of the bf16 routed-expert
+// kernel (tc_moe_kernel).
 //
 // Weights sit on the MMA's M side, tokens on N.  Per stage of 64 input columns TMA
 // brings two FP8 weight tiles [128 rows x 64 bytes] and the bf16 token rows; eight
 // converter warps turn each FP8 tile into the 128-byte-swizzled bf16 tile the MMA
 // reads (value = code * scale, rounded to bf16); the MMA warp then issues tcgen05.mma.
-// A unit's scales are staged in shared memory once per unit.
+// A unit's scales are staged in shared memory once per unit.  NVFP4: TMA brings two
+// tiles [128 rows x 32 bytes] of packed codes and the converters write value =
+// e2m1(code) * (block scale * tensor scale), exact in fp32, rounded to bf16.
 //
-// Passage: FP8 serving of the MoE experts — "DiffusionGemma 技术报告" (full
-// translation page), §6 (FP8 on H100, MoE memory-bound at batch 1).
+// Passages: FP8 serving of the MoE experts — "DiffusionGemma 技术报告" (full
+// translation page), §6 (FP8 on H100, MoE memory-bound at batch 1); NVFP4 — the
+// agentlenshq page on DiffusionGemma (NVFP4 kernels for Hopper and Blackwell).  The
+// block-scaled tensor-core MMA is not used: the codes are widened to bf16 in shared
+// memory and the MMA is the bf16 one of the other expert kernels.
 #pragma once
 
 #include <cuda_fp8.h>
@@ -29,6 +36,24 @@ __device__ __forceinline__ uint32_t f8x2_scaled(uint32_t two, float sc) {
 
 constexpr int TC_F8_THREADS = 576;
 
+// NVFP4 scales of one layer: E4M3 block scales [rows, K / 16] and fp32 tensor scales [1]
+struct F4Scales {
+  const uint8_t *g = nullptr, *u = nullptr, *d = nullptr;
+  const float *tg = nullptr, *tu = nullptr, *td = nullptr;
+};
+
+// value of a 4-bit E2M1 code: magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6 for codes 0..7 (in
+// half units 0, 1, 2, 3, 4, 6, 8, 12, one nibble each of 0xC8643210), bit 3 the sign
+__device__ __forceinline__ float e2m1_value(uint32_t c) {
+  const float mag = (float)((0xC8643210u >> (4 * (c & 7u))) & 0xFu) * 0.5f;
+  return (c & 8u) ? -mag : mag;
+}
+
+__device__ __forceinline__ float e4m3_value(uint8_t b) {
+  __half_raw h = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)b, __NV_E4M3);
+  return __half2float(*reinterpret_cast<__half*>(&h));
+}
+
 // ---------------------------------------------------------------------------
 // Both phases of the routed experts with FP8 weights in one persistent launch (the
 // schedule and the device-side chunk counters of tc_moe_kernel).  Per stage: TMA
@@ -39,29 +64,34 @@ constexpr int TC_F8_THREADS = 576;
 // Roles (576 threads): warp 0 TMA, warp 1 MMA, warps 2..9 epilogue, warps 10..17
 // converters.
 // ---------------------------------------------------------------------------
-template <int ST>
-struct MoeF8Cfg {
-  static constexpr uint32_t F8_TILE = 128 * 64;
+template <int ST, bool FP4>
+struct MoeLowpCfg {
+  static constexpr uint32_t F8_TILE = FP4 ? 128 * 32 : 128 * 64;  // weight bytes per tile
   static constexpr uint32_t B_MAX = 128 * TC_KB * 2;
   static constexpr uint32_t STAGE = 2 * F8_TILE + 2 * TC_SUB_A + B_MAX;
+  static_assert(STAGE % 1024 == 0 && (2 * F8_TILE) % 1024 == 0, "swizzled tiles 1024-aligned");
   static constexpr uint32_t TCOLS = 256;
   static constexpr size_t SMEM = 1024 + (size_t)ST * STAGE + 512;  // + the unit's scales
   // a unit's scales: 256 weight rows (gate then up, or the two down tiles) x K / 128
-  static size_t smem_bytes(int d, int I) { return SMEM + (size_t)8 * (d > I ? d : I); }
+  // fp32 (FP8) or x K / 16 E4M3 bytes (NVFP4), then (NVFP4) the 256-entry table of a
+  // byte's two E2M1 values as a bf16 pair
+  static size_t smem_bytes(int d, int I) {
+    const size_t K = d > I ? d : I;
+    return SMEM + (FP4 ? 16 * K + 1024 : 8 * K);
+  }
 };
+template <int ST> using MoeF8Cfg = MoeLowpCfg<ST, false>;
 
-template <int ST>
-__global__ void __launch_bounds__(TC_F8_THREADS, 1)
-    tc_moe_f8_kernel(const __grid_constant__ CUtensorMap mWg, const __grid_constant__ CUtensorMap mWu,
-                     const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mWd,
-                     const __grid_constant__ CUtensorMap mH, const float* __restrict__ sWg,
-                     const float* __restrict__ sWu, const float* __restrict__ sWd,
-                     const int32_t* __restrict__ chunk_e, const int32_t* __restrict__ chunk_r0,
-                     const int32_t* __restrict__ n_chunks, const int32_t* __restrict__ offsets,
-                     int I, int d, bf16* __restrict__ hb, float* __restrict__ yb,
-                     const float* __restrict__ gate_of, int32_t* __restrict__ ready,
-                     int32_t* err) {
-  typedef MoeF8Cfg<ST> Cfg;
+template <int ST, bool FP4>
+__device__ __forceinline__ void moe_lowp_body(
+    const CUtensorMap& mWg, const CUtensorMap& mWu, const CUtensorMap& mX,
+    const CUtensorMap& mWd, const CUtensorMap& mH, const float* __restrict__ sWg,
+    const float* __restrict__ sWu, const float* __restrict__ sWd, const F4Scales& f4,
+    const int32_t* __restrict__ chunk_e, const int32_t* __restrict__ chunk_r0,
+    const int32_t* __restrict__ n_chunks, const int32_t* __restrict__ offsets, int I, int d,
+    bf16* __restrict__ hb, float* __restrict__ yb, const float* __restrict__ gate_of,
+    int32_t* __restrict__ ready, int32_t* err) {
+  typedef MoeLowpCfg<ST, FP4> Cfg;
   pdl_enter();  // the routing tables come from the preceding kernels
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -88,6 +118,14 @@ __global__ void __launch_bounds__(TC_F8_THREADS, 1)
     tc::fence_mbar_init();
   }
   if (warp == 1) tc::tmem_alloc(tslot, Cfg::TCOLS);
+  // NVFP4: byte b -> (e2m1(b & 15), e2m1(b >> 4)) as bf16, exact (at most 2 significant bits)
+  uint32_t* f4tab = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(sscl) +
+                                                16 * (size_t)(d > I ? d : I));
+  if (FP4 && threadIdx.x < 256) {
+    __nv_bfloat162 v2 = __floats2bfloat162_rn(e2m1_value(threadIdx.x & 15u),
+                                              e2m1_value(threadIdx.x >> 4));
+    f4tab[threadIdx.x] = *reinterpret_cast<uint32_t*>(&v2);
+  }
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
@@ -149,13 +187,14 @@ __global__ void __launch_bounds__(TC_F8_THREADS, 1)
             break;
           }
           const int kx = ((kb + x.f) % x.nk) * TC_KB;
+          const int kw = FP4 ? kx / 2 : kx;  // byte column of the weight tiles
           tc::mbar_expect_tx(full + s, bytes);
           if (x.down) {
-            tc::tma_load_2d(f8_at(s, 0), &mWd, full + s, kx, x.w1);
-            tc::tma_load_2d(f8_at(s, 1), &mWd, full + s, kx, x.w1 + 128);
+            tc::tma_load_2d(f8_at(s, 0), &mWd, full + s, kw, x.w1);
+            tc::tma_load_2d(f8_at(s, 1), &mWd, full + s, kw, x.w1 + 128);
           } else {
-            tc::tma_load_2d(f8_at(s, 0), &mWg, full + s, kx, x.w1);
-            tc::tma_load_2d(f8_at(s, 1), &mWu, full + s, kx, x.w1);
+            tc::tma_load_2d(f8_at(s, 0), &mWg, full + s, kw, x.w1);
+            tc::tma_load_2d(f8_at(s, 1), &mWu, full + s, kw, x.w1);
           }
           for (int j = 0; j < nb; ++j)
             tc::tma_load_2d(x_at(s) + j * 32 * TC_KB * 2, x.down ? &mH : &mX, full + s, kx,
@@ -208,16 +247,30 @@ __global__ void __launch_bounds__(TC_F8_THREADS, 1)
     const int chunk = t & 3;
     int it = 0;
     bool dead = false;
+    uint8_t* sscl8 = reinterpret_cast<uint8_t*>(sscl);
     for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
       const Unit x = unit_of(u);
-      const int kscale = (x.down ? I : d) / 128;
+      const int kscale = (x.down ? I : d) / (FP4 ? 16 : 128);
       const int half = 128 * kscale;
+      float tsc[2] = {1.f, 1.f};
       asm volatile("bar.sync 2, 256;" ::: "memory");  // the previous unit's scales are read
-      for (int i = 4 * t; i < 2 * half; i += 1024) {
-        const float* src = x.down ? sWd + (size_t)x.w1 * kscale + i
-                           : i < half ? sWg + (size_t)x.w1 * kscale + i
-                                      : sWu + (size_t)x.w1 * kscale + (i - half);
-        *reinterpret_cast<float4*>(sscl + i) = __ldg(reinterpret_cast<const float4*>(src));
+      if constexpr (FP4) {
+        // E4M3 bytes: gate rows then up rows, or the 256 down rows (16 bytes at a time)
+        for (int i = 16 * t; i < 2 * half; i += 4096) {
+          const uint8_t* src = x.down ? f4.d + (size_t)x.w1 * kscale + i
+                               : i < half ? f4.g + (size_t)x.w1 * kscale + i
+                                          : f4.u + (size_t)x.w1 * kscale + (i - half);
+          *reinterpret_cast<uint4*>(sscl8 + i) = __ldg(reinterpret_cast<const uint4*>(src));
+        }
+        tsc[0] = x.down ? __ldg(f4.td) : __ldg(f4.tg);
+        tsc[1] = x.down ? __ldg(f4.td) : __ldg(f4.tu);
+      } else {
+        for (int i = 4 * t; i < 2 * half; i += 1024) {
+          const float* src = x.down ? sWd + (size_t)x.w1 * kscale + i
+                             : i < half ? sWg + (size_t)x.w1 * kscale + i
+                                        : sWu + (size_t)x.w1 * kscale + (i - half);
+          *reinterpret_cast<float4*>(sscl + i) = __ldg(reinterpret_cast<const float4*>(src));
+        }
       }
       asm volatile("bar.sync 2, 256;" ::: "memory");
       for (int kb = 0; kb < x.nk; ++kb, ++it) {
@@ -233,7 +286,40 @@ __global__ void __launch_bounds__(TC_F8_THREADS, 1)
             dead = true;
           }
         }
-        if (!dead) {
+        if (!dead && FP4) {
+          // thread t (0..255) converts, in tile w = 0 and 1, row t / 2 and 16-byte chunk
+          // t % 2 of the row's 32 bytes (64 codes): codes 32 ch .. 32 ch + 31, scale
+          // blocks (kx + 32 ch) / 16 and the next
+#pragma unroll
+          for (int w = 0; w < 2; ++w) {
+            const int r = t >> 1, ch = t & 1;
+            const uint4 q = *reinterpret_cast<const uint4*>(f8_at(s, w) + r * 32 + ch * 16);
+            const uint8_t* srow = sscl8 + (size_t)(128 * w + r) * kscale + ((kx + 32 * ch) >> 4);
+            // block scale * tensor scale: at most 4 significant bits times a power of
+            // two, exact in bf16, so the bf16 products below are exact
+            const __nv_bfloat162 sc2[2] = {
+                __float2bfloat162_rn(e4m3_value(srow[0]) * tsc[w]),
+                __float2bfloat162_rn(e4m3_value(srow[1]) * tsc[w])};
+            const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
+            uint32_t o[16];
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const uint32_t t2 = f4tab[(qw[b] >> (8 * i)) & 0xffu];
+                __nv_bfloat162 v2 = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&t2),
+                                            sc2[b >> 1]);
+                o[4 * b + i] = *reinterpret_cast<uint32_t*>(&v2);
+              }
+            }
+            uint8_t* rowp = bf_at(s, w) + r * 128;
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              *reinterpret_cast<uint4*>(rowp + (((4 * ch + k) ^ (r & 7)) << 4)) =
+                  make_uint4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
+          }
+        }
+        if (!dead && !FP4) {
 #pragma unroll
           for (int w = 0; w < 2; ++w) {
             const uint8_t* src = f8_at(s, w);
@@ -320,6 +406,35 @@ __global__ void __launch_bounds__(TC_F8_THREADS, 1)
   tc::fence_before_sync();
   __syncthreads();
   if (warp == 1) tc::tmem_dealloc(tmem, Cfg::TCOLS);
+}
+
+template <int ST>
+__global__ void __launch_bounds__(TC_F8_THREADS, 1)
+    tc_moe_f8_kernel(const __grid_constant__ CUtensorMap mWg, const __grid_constant__ CUtensorMap mWu,
+                     const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mWd,
+                     const __grid_constant__ CUtensorMap mH, const float* __restrict__ sWg,
+                     const float* __restrict__ sWu, const float* __restrict__ sWd,
+                     const int32_t* __restrict__ chunk_e, const int32_t* __restrict__ chunk_r0,
+                     const int32_t* __restrict__ n_chunks, const int32_t* __restrict__ offsets,
+                     int I, int d, bf16* __restrict__ hb, float* __restrict__ yb,
+                     const float* __restrict__ gate_of, int32_t* __restrict__ ready,
+                     int32_t* err) {
+  moe_lowp_body<ST, false>(mWg, mWu, mX, mWd, mH, sWg, sWu, sWd, F4Scales{}, chunk_e, chunk_r0,
+                           n_chunks, offsets, I, d, hb, yb, gate_of, ready, err);
+}
+
+template <int ST>
+__global__ void __launch_bounds__(TC_F8_THREADS, 1)
+    tc_moe_f4_kernel(const __grid_constant__ CUtensorMap mWg, const __grid_constant__ CUtensorMap mWu,
+                     const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mWd,
+                     const __grid_constant__ CUtensorMap mH, const F4Scales f4,
+                     const int32_t* __restrict__ chunk_e, const int32_t* __restrict__ chunk_r0,
+                     const int32_t* __restrict__ n_chunks, const int32_t* __restrict__ offsets,
+                     int I, int d, bf16* __restrict__ hb, float* __restrict__ yb,
+                     const float* __restrict__ gate_of, int32_t* __restrict__ ready,
+                     int32_t* err) {
+  moe_lowp_body<ST, true>(mWg, mWu, mX, mWd, mH, nullptr, nullptr, nullptr, f4, chunk_e,
+                          chunk_r0, n_chunks, offsets, I, d, hb, yb, gate_of, ready, err);
 }
 
 }  // namespace dg

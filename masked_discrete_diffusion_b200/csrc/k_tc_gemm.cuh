@@ -1247,6 +1247,8 @@ dg_status tc_gemm_add_residual(dg_model* m, const bf16* A, const void* W, float*
 dg_status tc_gemm_swiglu(dg_model* m, const bf16* A, const void* Wg, const void* Wu, bf16* out,
                          int M, int N, int K, cudaStream_t st);
 dg_status tc_moe_experts(dg_model* m, int l, const bf16* X, bf16* hb, float* yb, cudaStream_t st);
+dg_status tc_moe_experts_f4(dg_model* m, int l, const bf16* X, bf16* hb, float* yb,
+                            cudaStream_t st);
 dg_status tc_moe_experts_f8(dg_model* m, int l, const bf16* X, bf16* hb, float* yb,
                             cudaStream_t st);
 dg_status tc_lmhead_stats(dg_model* m, const bf16* xn, int M, float* ent, int32_t* amax,

@@ -18,10 +18,11 @@ struct MapKey {
   const void* p;
   uint64_t rows, cols;
   uint32_t box_rows;
-  bool bytes = false;  // uint8 elements, 64-byte boxes, no swizzle (FP8 weights)
+  bool bytes = false;  // uint8 elements, no swizzle (FP8 weights, packed NVFP4 weights)
+  uint32_t box_cols = 64;  // inner box extent in elements (bytes for uint8 maps)
   bool operator==(const MapKey& o) const {
     return p == o.p && rows == o.rows && cols == o.cols && box_rows == o.box_rows &&
-           bytes == o.bytes;
+           bytes == o.bytes && box_cols == o.box_cols;
   }
 };
 struct MapKeyHash {
@@ -52,13 +53,13 @@ int ceil_div_i(long a, long b) { return (int)((a + b - 1) / b); }
 // 2-D bf16 tensor [rows, cols] (row-major), box = 64 columns x box_rows rows,
 // 128-byte swizzle, out-of-range elements read as zero.
 dg_status tmap(const dg_model* m, const void* p, uint64_t rows, uint64_t cols, uint32_t box_rows,
-               CUtensorMap* out, bool bytes = false) {
+               CUtensorMap* out, bool bytes = false, uint32_t box_cols = 64) {
   TcState* s = state(m);
   if (!s) {
     set_error("tensor-core state missing");
     return DG_ERR_INTERNAL;
   }
-  MapKey key{p, rows, cols, box_rows, bytes};
+  MapKey key{p, rows, cols, box_rows, bytes, box_cols};
   auto it = s->maps.find(key);
   if (it != s->maps.end()) {
     *out = it->second;
@@ -73,7 +74,11 @@ dg_status tmap(const dg_model* m, const void* p, uint64_t rows, uint64_t cols, u
   CUtensorMap map;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {cols * esz};
-  cuuint32_t box[2] = {64, box_rows};
+  if (box_cols * esz % 16 || box_cols > 256) {
+    set_error("tensor map: inner box of %u elements is not a multiple of 16 bytes", box_cols);
+    return DG_ERR_UNSUPPORTED;
+  }
+  cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = s->encode(&map, bytes ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
                          2, const_cast<void*>(p), dims, strides, box, estr,
@@ -183,6 +188,7 @@ dg_status tc_prepare(dg_model* m) {
   DG_TRY(set_smem(tc_dense_kernel<128, DENSE_MT, false, QKV_ST, EpiQkvRope>,
                   DenseCfg<128, DENSE_MT, false, QKV_ST>::SMEM + EpiQkvRope::kExtraSmem));
   DG_TRY(set_smem(tc_moe_f8_kernel<MOE8_ST>, MoeF8Cfg<MOE8_ST>::smem_bytes(4096, 4096)));
+  DG_TRY(set_smem(tc_moe_f4_kernel<MOE8_ST>, MoeLowpCfg<MOE8_ST, true>::smem_bytes(2048, 2048)));
   cudaDeviceGetAttribute(&s->n_sm, cudaDevAttrMultiProcessorCount, m->device);
   return DG_OK;
 }
@@ -350,6 +356,35 @@ dg_status tc_moe_experts_f8(dg_model* m, int l, const bf16* X, bf16* hb, float* 
   ++m->launches;
   if (e != cudaSuccess) {
     set_error("tc_moe_f8 launch: %s", cudaGetErrorString(e));
+    return DG_ERR_CUDA;
+  }
+  return DG_OK;
+}
+
+// NVFP4 expert weights (packed E2M1 codes [rows, K / 2] bytes, E4M3 block scales
+// [rows, K / 16], one fp32 tensor scale per matrix): the same persistent launch with the
+// NVFP4 converter
+dg_status tc_moe_experts_f4(dg_model* m, int l, const bf16* X, bf16* hb, float* yb,
+                            cudaStream_t st) {
+  const dg_config& c = m->cfg;
+  const dg_layer_weights& L = m->layers[l];
+  const int E = c.n_experts, I = c.expert_inter, d = c.d_model;
+  const Workspace& ws = m->ws;
+  CUtensorMap wg, wu, x, wd, h;
+  DG_TRY(tmap(m, L.gate, (uint64_t)E * I, d / 2, 128, &wg, true, 32));
+  DG_TRY(tmap(m, L.up, (uint64_t)E * I, d / 2, 128, &wu, true, 32));
+  DG_TRY(tmap(m, X, ws.max_rows, d, 32, &x));
+  DG_TRY(tmap(m, L.down, (uint64_t)E * d, I / 2, 128, &wd, true, 32));
+  DG_TRY(tmap(m, hb, ws.max_rows, I, 32, &h));
+  F4Scales sc{(const uint8_t*)L.gate_scale, (const uint8_t*)L.up_scale,
+              (const uint8_t*)L.down_scale, L.gate_tscale, L.up_tscale, L.down_tscale};
+  cudaError_t e = launch_pdl((tc_moe_f4_kernel<MOE8_ST>), state(m)->n_sm, TC_F8_THREADS,
+                             MoeLowpCfg<MOE8_ST, true>::smem_bytes(d, I), st, 1, wg, wu, x, wd,
+                             h, sc, ws.tile_e, ws.tile_m0, ws.n_tiles, ws.offsets, I, d, hb, yb,
+                             (const float*)ws.gate_of, ws.ready, ws.err);
+  ++m->launches;
+  if (e != cudaSuccess) {
+    set_error("tc_moe_f4 launch: %s", cudaGetErrorString(e));
     return DG_ERR_CUDA;
   }
   return DG_OK;

@@ -56,8 +56,12 @@ def forward_cost(cfg, batch: int, window: int, unique_experts=None):
     Hq, Hkv, E, k = cfg.n_q_heads, cfg.n_kv_heads, cfg.n_experts, cfg.top_k
     I, Is, V, C = cfg.expert_inter, cfg.shared_inter, cfg.vocab, cfg.canvas
     wb = 4 if cfg.dtype == 0 else 2
-    ewb = 1 if cfg.dtype == 2 else wb
-    expert_bytes = 3 * I * d * ewb + (3 * I * d // 128 * 4 if cfg.dtype == 2 else 0)
+    if cfg.dtype == 2:    # FP8 codes + an fp32 scale per 128 inputs
+        expert_bytes = 3 * I * d + 3 * I * d // 128 * 4
+    elif cfg.dtype == 3:  # NVFP4 codes (half a byte) + an E4M3 scale per 16 inputs
+        expert_bytes = 3 * I * d // 2 + 3 * I * d // 16
+    else:
+        expert_bytes = 3 * I * d * wb
     qkv = (Hq + 2 * Hkv) * h
     dense = (qkv * d + d * Hq * h + E * d + 3 * Is * d) * wb
     if unique_experts is None:

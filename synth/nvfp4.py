@@ -17,10 +17,9 @@ NaN; the eight magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6 are codes 0..7 in order.  T
 represented weight is e2m1(code) * s_b * s_t, exact in fp32 (at most 2 significant
 bits times 4 times a power of two).
 
-Every step is exact in fp64 (scales are powers of two or E4M3 values, the divisions
-by them are exact up to the final rounding, which is done on the fp64 quotient), so
-the host computes each byte and scale once.  This is a weight format; it holds none
-of the model's arithmetic.
+Every step is exact in fp64 or a correctly rounded fp64 division followed by a
+rounding to the grid, so the bytes and scales are the same on the host and on a GPU.
+This is a weight format; it holds none of the model's arithmetic.
 """
 from __future__ import annotations
 
@@ -107,9 +106,10 @@ def quantised(w: Workload, name: str, shape, sigma: float, device="cpu"):
     step = max(1, (1 << 22) // K)
     for r in range(0, R, step):
         n = min(step, R - r)
-        v = gen.normal_values(w.seed, name, r * K, n * K, sigma, "cpu").reshape(n, K)
-        p, s = quantize_rows(v, s_t)
-        packed[r:r + n], scales[r:r + n] = p.to(device), s.to(device)
+        # on the target device: every step is exact or a correctly rounded fp64
+        # division, so the bytes are the same wherever they are computed
+        v = gen.normal_values(w.seed, name, r * K, n * K, sigma, device).reshape(n, K)
+        packed[r:r + n], scales[r:r + n] = quantize_rows(v, s_t)
     st = torch.tensor([s_t], dtype=torch.float32, device=device)
     return (packed.reshape(tuple(shape[:-1]) + (K // 2,)),
             scales.reshape(tuple(shape[:-1]) + (K // BLOCK,)), st)
