@@ -90,7 +90,7 @@ __device__ __forceinline__ void moe_lowp_body(
     const int32_t* __restrict__ chunk_e, const int32_t* __restrict__ chunk_r0,
     const int32_t* __restrict__ n_chunks, const int32_t* __restrict__ offsets, int I, int d,
     bf16* __restrict__ hb, float* __restrict__ yb, const float* __restrict__ gate_of,
-    int32_t* __restrict__ ready, int32_t* err) {
+    int32_t* __restrict__ ready, int32_t* __restrict__ next, int32_t* err) {
   typedef MoeLowpCfg<ST, FP4> Cfg;
   pdl_enter();  // the routing tables come from the preceding kernels
   extern __shared__ uint8_t smem_raw[];
@@ -100,7 +100,15 @@ __device__ __forceinline__ void moe_lowp_body(
   uint64_t* empty = conv + ST;
   uint64_t* tfull = empty + ST;
   uint64_t* tempty = tfull + 1;   // 8 epilogue arrivals
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(tempty + 1);
+  // units taken by the TMA thread, in order, for the MMA thread, the epilogue leader and
+  // the converter leader (the schedule of tc_moe_kernel)
+  constexpr int QD = 4;
+  uint64_t* qfull = tempty + 1;   // [QD] unit id written (TMA thread)
+  uint64_t* qempty = qfull + QD;  // [QD] unit id read (three readers)
+  int32_t* qid = reinterpret_cast<int32_t*>(qempty + QD);  // [QD]
+  int32_t* ubc = qid + QD;        // the epilogue leader's broadcast of the unit id
+  int32_t* cbc = ubc + 1;         // the converter leader's broadcast
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(cbc + 1);
   float* sscl = reinterpret_cast<float*>(smem + ST * Cfg::STAGE + 512);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nc = *n_chunks;
@@ -115,6 +123,10 @@ __device__ __forceinline__ void moe_lowp_body(
     }
     tc::mbar_init(tfull, 1);
     tc::mbar_init(tempty, 8);
+    for (int k = 0; k < QD; ++k) {
+      tc::mbar_init(qfull + k, 1);
+      tc::mbar_init(qempty + k, 3);
+    }
     tc::fence_mbar_init();
   }
   if (warp == 1) tc::tmem_alloc(tslot, Cfg::TCOLS);
@@ -148,6 +160,18 @@ __device__ __forceinline__ void moe_lowp_body(
     x.nk = (x.down ? I : d) / TC_KB;
     return x;
   };
+  // the ui-th unit id of this block (n_units when there is none, or on a timeout)
+  auto take = [&](int ui) -> int {
+    const int k = ui % QD;
+    if (!tc::mbar_wait(qfull + k, (ui / QD) & 1)) {
+      atomicOr(err, ERR_TIMEOUT);
+      return n_units;
+    }
+    const int u = *reinterpret_cast<volatile int32_t*>(qid + k);
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(tc::smem_addr(qempty + k))
+                 : "memory");
+    return u;
+  };
   auto f8_at = [&](int s, int w) { return smem + s * Cfg::STAGE + w * Cfg::F8_TILE; };
   auto bf_at = [&](int s, int w) { return smem + s * Cfg::STAGE + 2 * Cfg::F8_TILE + w * TC_SUB_A; };
   auto x_at = [&](int s) { return smem + s * Cfg::STAGE + 2 * Cfg::F8_TILE + 2 * TC_SUB_A; };
@@ -161,7 +185,19 @@ __device__ __forceinline__ void moe_lowp_body(
       tc::prefetch_tmap(&mH);
       int it = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      for (int qi = 0;; ++qi) {
+        // blocks take the next unit when they are ready for it (gate/up units first,
+        // so a down unit only ever waits for units that running blocks have taken)
+        const int k = qi % QD;
+        if (qi >= QD && !tc::mbar_wait(qempty + k, ((qi / QD) & 1) ^ 1)) {
+          atomicOr(err, ERR_TIMEOUT);
+          break;  // the readers give up on their own bounded waits
+        }
+        const int u = ok ? atomicAdd(next, 1) : n_units;
+        qid[k] = u < n_units ? u : n_units;
+        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(tc::smem_addr(qfull + k))
+                     : "memory");
+        if (u >= n_units) break;
         const Unit x = unit_of(u);
         if (x.down) {
           const uint64_t t0 = tc::global_ns();
@@ -173,7 +209,7 @@ __device__ __forceinline__ void moe_lowp_body(
               break;
             }
           }
-          if (!ok) break;
+          if (!ok) continue;  // publish the end of the work next
           asm volatile("fence.proxy.async.global;" ::: "memory");  // before the TMA reads
         }
         const int nb = (x.n + 31) >> 5;
@@ -205,9 +241,11 @@ __device__ __forceinline__ void moe_lowp_body(
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      int it = 0, ui = 0;
+      int it = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++ui) {
+      for (int ui = 0; ok; ++ui) {
+        const int u = take(ui);
+        if (u >= n_units) break;
         const Unit x = unit_of(u);
         const int npad = ((x.n + 31) >> 5) << 5;
         const uint32_t idesc = tc::idesc_bf16(128, npad);
@@ -248,12 +286,17 @@ __device__ __forceinline__ void moe_lowp_body(
     int it = 0;
     bool dead = false;
     uint8_t* sscl8 = reinterpret_cast<uint8_t*>(sscl);
-    for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+    for (int ui = 0;; ++ui) {
+      // warp 10 takes the unit id for the eight converter warps; the barrier also keeps
+      // the previous unit's scales until every converter has read them
+      if (warp == 10 && lane == 0) *reinterpret_cast<volatile int32_t*>(cbc) = take(ui);
+      asm volatile("bar.sync 2, 256;" ::: "memory");
+      const int u = *reinterpret_cast<volatile int32_t*>(cbc);
+      if (u >= n_units) break;
       const Unit x = unit_of(u);
       const int kscale = (x.down ? I : d) / (FP4 ? 16 : 128);
       const int half = 128 * kscale;
       float tsc[2] = {1.f, 1.f};
-      asm volatile("bar.sync 2, 256;" ::: "memory");  // the previous unit's scales are read
       if constexpr (FP4) {
         // E4M3 bytes: gate rows then up rows, or the 256 down rows (16 bytes at a time)
         for (int i = 16 * t; i < 2 * half; i += 4096) {
@@ -354,8 +397,13 @@ __device__ __forceinline__ void moe_lowp_body(
     // epilogue warps 2..9 -> TMEM lane quarter (warp % 4), token chunks of parity hf
     const int q = warp & 3, hf = (warp - 2) >> 2;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-    int ui = 0;
-    for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++ui) {
+    for (int ui = 0;; ++ui) {
+      // warp 2 takes the unit id for the eight epilogue warps
+      if (warp == 2 && lane == 0) *reinterpret_cast<volatile int32_t*>(ubc) = take(ui);
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      const int u = *reinterpret_cast<volatile int32_t*>(ubc);
+      asm volatile("bar.sync 1, 256;" ::: "memory");  // read by all before the next take
+      if (u >= n_units) break;
       const Unit x = unit_of(u);
       bool rdy = true;
       if (lane == 0) rdy = tc::mbar_wait(tfull, ui & 1);
@@ -418,9 +466,9 @@ __global__ void __launch_bounds__(TC_F8_THREADS, 1)
                      const int32_t* __restrict__ n_chunks, const int32_t* __restrict__ offsets,
                      int I, int d, bf16* __restrict__ hb, float* __restrict__ yb,
                      const float* __restrict__ gate_of, int32_t* __restrict__ ready,
-                     int32_t* err) {
+                     int32_t* __restrict__ next, int32_t* err) {
   moe_lowp_body<ST, false>(mWg, mWu, mX, mWd, mH, sWg, sWu, sWd, F4Scales{}, chunk_e, chunk_r0,
-                           n_chunks, offsets, I, d, hb, yb, gate_of, ready, err);
+                           n_chunks, offsets, I, d, hb, yb, gate_of, ready, next, err);
 }
 
 template <int ST>
@@ -432,9 +480,9 @@ __global__ void __launch_bounds__(TC_F8_THREADS, 1)
                      const int32_t* __restrict__ n_chunks, const int32_t* __restrict__ offsets,
                      int I, int d, bf16* __restrict__ hb, float* __restrict__ yb,
                      const float* __restrict__ gate_of, int32_t* __restrict__ ready,
-                     int32_t* err) {
+                     int32_t* __restrict__ next, int32_t* err) {
   moe_lowp_body<ST, true>(mWg, mWu, mX, mWd, mH, nullptr, nullptr, nullptr, f4, chunk_e,
-                          chunk_r0, n_chunks, offsets, I, d, hb, yb, gate_of, ready, err);
+                          chunk_r0, n_chunks, offsets, I, d, hb, yb, gate_of, ready, next, err);
 }
 
 }  // namespace dg

@@ -352,7 +352,7 @@ dg_status tc_moe_experts_f8(dg_model* m, int l, const bf16* X, bf16* hb, float* 
                              (const float*)L.gate_scale, (const float*)L.up_scale,
                              (const float*)L.down_scale, ws.tile_e, ws.tile_m0, ws.n_tiles,
                              ws.offsets, I, d, hb, yb, (const float*)ws.gate_of, ws.ready,
-                             ws.err);
+                             ws.ready + ws.max_tiles, ws.err);
   ++m->launches;
   if (e != cudaSuccess) {
     set_error("tc_moe_f8 launch: %s", cudaGetErrorString(e));
@@ -381,7 +381,7 @@ dg_status tc_moe_experts_f4(dg_model* m, int l, const bf16* X, bf16* hb, float* 
   cudaError_t e = launch_pdl((tc_moe_f4_kernel<MOE8_ST>), state(m)->n_sm, TC_F8_THREADS,
                              MoeLowpCfg<MOE8_ST, true>::smem_bytes(d, I), st, 1, wg, wu, x, wd,
                              h, sc, ws.tile_e, ws.tile_m0, ws.n_tiles, ws.offsets, I, d, hb, yb,
-                             (const float*)ws.gate_of, ws.ready, ws.err);
+                             (const float*)ws.gate_of, ws.ready, ws.ready + ws.max_tiles, ws.err);
   ++m->launches;
   if (e != cudaSuccess) {
     set_error("tc_moe_f4 launch: %s", cudaGetErrorString(e));
