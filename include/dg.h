@@ -86,7 +86,8 @@ typedef struct dg_config {
  * input columns) in the *_scale fields and one fp32 tensor scale per tensor in the
  * *_tscale fields: w = e2m1(code) * block scale * tensor scale.  The kernel widens
  * the codes to bf16 in shared memory, so a weight must be exact in fp32: the
- * tensor scale must be a power of two. */
+ * tensor scale must be a positive power of two (read at model creation;
+ * DG_ERR_INVALID_ARG otherwise). */
 typedef struct dg_layer_weights {
   const void* wqkv;   /* [(Hq + 2 Hkv) h, d]: query heads, key heads, value heads */
   const void* wo;     /* [d, Hq h]                                                */

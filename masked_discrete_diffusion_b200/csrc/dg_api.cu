@@ -748,6 +748,17 @@ dg_status dg_model_create(const dg_config* cfg, const dg_weights* w, dg_model** 
     DG_REQUIRE(L.wqkv && L.wo && L.router && L.gate && L.up && L.down && L.sgate && L.sup &&
                    L.sdown,
                "null weight pointer in layer %d", l);
+    if (c.dtype == DG_BF16_FP4EXP && L.gate_tscale && L.up_tscale && L.down_tscale) {
+      // the widened weights are exact only with power-of-two tensor scales (read once here)
+      const float* ts[3] = {L.gate_tscale, L.up_tscale, L.down_tscale};
+      for (int i = 0; i < 3; ++i) {
+        float v = 0.f;
+        DG_TRY_CUDA(cudaMemcpy(&v, ts[i], sizeof(float), cudaMemcpyDeviceToHost));
+        int ex = 0;
+        DG_REQUIRE(std::isfinite(v) && v > 0.f && std::frexp(v, &ex) == 0.5f,
+                   "NVFP4 tensor scale %g of layer %d is not a positive power of two", v, l);
+      }
+    }
     if (c.dtype == DG_BF16_FP8EXP)
       DG_REQUIRE(L.gate_scale && L.up_scale && L.down_scale, "null FP8 scale pointer in layer %d", l);
     if (c.dtype == DG_BF16_FP4EXP)

@@ -103,10 +103,15 @@ def test_fp4_needs_its_scales():
     from masked_discrete_diffusion_b200 import binding
     w = W.with_(n_layers=1)
     t = model_inputs.weight_set(w, "cuda")
-    del t["l0.up_tscale"]
+    up_ts = t.pop("l0.up_tscale")
     with pytest.raises(binding.DGError) as e:
         binding.Model(binding.make_config(w), t)
     assert "NVFP4 scale" in str(e.value)
+    # a tensor scale that is not a power of two would make the widened weights inexact
+    t["l0.up_tscale"] = up_ts * 3
+    with pytest.raises(binding.DGError) as e:
+        binding.Model(binding.make_config(w), t)
+    assert "power of two" in str(e.value)
 
 
 GOLD = os.path.join(os.path.dirname(__file__), "golden", "layer1-fp4exp.npz")
