@@ -21,7 +21,7 @@ norm gains, router normalisation, joint softmax over window and canvas, ...)
 are fixed in the docstrings below and listed in the design notes.
 
 Precision: weights are read as their stored values (fp32 / bf16 / dequantised
-FP8) and widened to fp64; every activation and reduction is fp64.  Per-row
+FP8 / dequantised NVFP4) and widened to fp64; every activation and reduction is fp64.  Per-row
 entropies are rounded to fp32 at the end, which is the precision the sampler
 decides in.
 
@@ -29,7 +29,8 @@ Storage variant (Weights(..., storage="bf16")): the same forward with every
 tensor a bf16 model multiplies kept in bf16: the activations rounded where they
 are stored (normalised rows entering a projection, q / k / v after RoPE, the
 attention output, the SwiGLU hidden rows) and FP8 expert weights dequantised to
-bf16 (bf16 weights are already exact); residual stream, router and every sum
+bf16 (bf16 weights and dequantised NVFP4 weights are already exact in bf16); residual
+stream, router and every sum
 stay fp64.  It measures how far bf16 storage alone moves the outputs of a
 workload (its sensitivity), from which the tolerances of the deep workloads are
 derived.
