@@ -309,63 +309,76 @@ struct EpiRouterTopk {
   int32_t* idx;
   float* gate;
   int E, top_k;
+  // the warp's RB rows side by side (each row's arithmetic as for a single row), so that
+  // the warp reductions of the rows overlap
   template <int NQ, int RB>
   __device__ void warp_rows(int row0, int M, int n0, const float (*v)[NQ], int lane,
                             const uint8_t*, int, int, uint8_t*) const {
-#pragma unroll 1
-    for (int r = 0; r < RB; ++r)
-      if (row0 + r < M) warp_row<NQ>(row0 + r, v[r], lane);
-  }
-  template <int NQ>
-  __device__ void warp_row(int row, const float* v, int lane) const {
-    float p[NQ];
-    float mx = -INFINITY;
+    float p[RB][NQ];
 #pragma unroll
-    for (int q2 = 0; q2 < NQ; ++q2) {
-      p[q2] = lane + 32 * q2 < E ? v[q2] : -INFINITY;
-      mx = fmaxf(mx, p[q2]);
-    }
-    mx = warp_max(mx);
-    float z = 0.f;
-#pragma unroll
-    for (int q2 = 0; q2 < NQ; ++q2) {
-      p[q2] = lane + 32 * q2 < E ? expf(p[q2] - mx) : 0.f;
-      z += p[q2];
-    }
-    z = warp_sum(z);
-#pragma unroll
-    for (int q2 = 0; q2 < NQ; ++q2) p[q2] /= z;
-    unsigned taken = 0;
-    float gsum = 0.f, my_p = 0.f;
-    int my_e = 0;
-    for (int k = 0; k < top_k; ++k) {
-      // this lane's best untaken probability (lowest id on ties), then the warp's: the
-      // probabilities are >= 0, so their bit patterns order like the values
-      float bp = -1.f;
-      int be = 0x7fffffff;
+    for (int r = 0; r < RB; ++r) {
+      float mx = -INFINITY;
 #pragma unroll
       for (int q2 = 0; q2 < NQ; ++q2) {
-        const int e = lane + 32 * q2;
-        if (e < E && !((taken >> q2) & 1u) && p[q2] > bp) {
-          bp = p[q2];
-          be = e;
-        }
+        p[r][q2] = lane + 32 * q2 < E ? v[r][q2] : -INFINITY;
+        mx = fmaxf(mx, p[r][q2]);
       }
-      const unsigned bits = bp >= 0.f ? __float_as_uint(bp) : 0u;
-      const unsigned top = __reduce_max_sync(0xffffffffu, bits);
-      be = (unsigned)__reduce_min_sync(0xffffffffu, bits == top && bp >= 0.f ? (unsigned)be
-                                                                              : 0x7fffffffu);
-      bp = __uint_as_float(top);
-      if ((be & 31) == lane) taken |= 1u << (be >> 5);
-      if (lane == k) {
-        my_e = be;
-        my_p = bp;
+      mx = warp_max(mx);
+      float z = 0.f;
+#pragma unroll
+      for (int q2 = 0; q2 < NQ; ++q2) {
+        p[r][q2] = lane + 32 * q2 < E ? expf(p[r][q2] - mx) : 0.f;
+        z += p[r][q2];
       }
-      gsum += bp;
+      z = warp_sum(z);
+#pragma unroll
+      for (int q2 = 0; q2 < NQ; ++q2) p[r][q2] /= z;
     }
-    if (lane < top_k) {
-      idx[(size_t)row * top_k + lane] = my_e;
-      gate[(size_t)row * top_k + lane] = my_p / gsum;
+    unsigned taken[RB];
+    float gsum[RB], my_p[RB];
+    int my_e[RB];
+#pragma unroll
+    for (int r = 0; r < RB; ++r) {
+      taken[r] = 0;
+      gsum[r] = 0.f;
+      my_p[r] = 0.f;
+      my_e[r] = 0;
+    }
+    for (int k = 0; k < top_k; ++k) {
+#pragma unroll
+      for (int r = 0; r < RB; ++r) {
+        // this lane's best untaken probability (lowest id on ties), then the warp's: the
+        // probabilities are >= 0, so their bit patterns order like the values
+        float bp = -1.f;
+        int be = 0x7fffffff;
+#pragma unroll
+        for (int q2 = 0; q2 < NQ; ++q2) {
+          const int e = lane + 32 * q2;
+          if (e < E && !((taken[r] >> q2) & 1u) && p[r][q2] > bp) {
+            bp = p[r][q2];
+            be = e;
+          }
+        }
+        const unsigned bits = bp >= 0.f ? __float_as_uint(bp) : 0u;
+        const unsigned top = __reduce_max_sync(0xffffffffu, bits);
+        be = (unsigned)__reduce_min_sync(0xffffffffu, bits == top && bp >= 0.f ? (unsigned)be
+                                                                                : 0x7fffffffu);
+        bp = __uint_as_float(top);
+        if ((be & 31) == lane) taken[r] |= 1u << (be >> 5);
+        if (lane == k) {
+          my_e[r] = be;
+          my_p[r] = bp;
+        }
+        gsum[r] += bp;
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < RB; ++r) {
+      const int row = row0 + r;
+      if (row < M && lane < top_k) {
+        idx[(size_t)row * top_k + lane] = my_e[r];
+        gate[(size_t)row * top_k + lane] = my_p[r] / gsum[r];
+      }
     }
   }
 };
