@@ -130,3 +130,33 @@ def test_noalloc_binding_rejects_bad_tensors_before_any_launch():
     for h, w, what in bad:
         with pytest.raises(ValueError, match=what):
             binding.dg_lmhead_entropy_noalloc(h, w, 1e-6, 8.0)
+
+
+def _header_struct_fields(name: str) -> list[str]:
+    """Field names, in order, of `typedef struct name { ... } name;` in include/dg.h
+    (comments stripped; one declaration per field, several names per line allowed)."""
+    import os
+    import re
+    src = open(os.path.join(os.path.dirname(__file__), "..", "include", "dg.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    body = re.search(r"typedef struct %s \{(.*?)\} %s;" % (name, name), src, flags=re.S).group(1)
+    fields = []
+    for decl in body.split(";"):
+        decl = decl.strip()
+        if not decl:
+            continue
+        # "int32_t a, b, c", "const void* p" or "float x": the first name ends the type
+        first, *others = [p.strip() for p in decl.split(",")]
+        fields += [first.split()[-1].lstrip("*")] + [o.lstrip("*") for o in others]
+    return fields
+
+
+def test_binding_structs_match_the_header():
+    """The ctypes structs pass field offsets by declaration order: a field out of order
+    or missing would hand the library a wrong pointer or size."""
+    from masked_discrete_diffusion_b200 import binding
+    assert [f for f, _ in binding.dg_config._fields_] == _header_struct_fields("dg_config")
+    assert list(binding._LAYER_FIELDS) == _header_struct_fields("dg_layer_weights")
+    assert [f for f, _ in binding.dg_weights._fields_] == _header_struct_fields("dg_weights")
+    assert [f for f, _ in binding.dg_anneal_params._fields_] == \
+        _header_struct_fields("dg_anneal_params")
