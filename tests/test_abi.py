@@ -132,6 +132,25 @@ def test_noalloc_binding_rejects_bad_tensors_before_any_launch():
             binding.dg_lmhead_entropy_noalloc(h, w, 1e-6, 8.0)
 
 
+def _header_struct_types(name: str) -> list[str]:
+    """The C type of each field of `name`, in order (as _header_struct_fields)."""
+    import os
+    import re
+    src = open(os.path.join(os.path.dirname(__file__), "..", "include", "dg.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    body = re.search(r"typedef struct %s \{(.*?)\} %s;" % (name, name), src, flags=re.S).group(1)
+    types = []
+    for decl in body.split(";"):
+        decl = decl.strip()
+        if not decl:
+            continue
+        first, *others = [p.strip() for p in decl.split(",")]
+        words = first.split()
+        t = " ".join(words[:-1]) + ("*" if words[-1].startswith("*") else "")
+        types += [t] * (1 + len(others))
+    return types
+
+
 def _header_struct_fields(name: str) -> list[str]:
     """Field names, in order, of `typedef struct name { ... } name;` in include/dg.h
     (comments stripped; one declaration per field, several names per line allowed)."""
@@ -160,3 +179,10 @@ def test_binding_structs_match_the_header():
     assert [f for f, _ in binding.dg_weights._fields_] == _header_struct_fields("dg_weights")
     assert [f for f, _ in binding.dg_anneal_params._fields_] == \
         _header_struct_fields("dg_anneal_params")
+    # and the scalar structs' field types
+    import ctypes
+    ctype_of = {"int32_t": ctypes.c_int32, "float": ctypes.c_float}
+    for st, name in ((binding.dg_config, "dg_config"),
+                     (binding.dg_anneal_params, "dg_anneal_params")):
+        want = [ctype_of[t] for t in _header_struct_types(name)]
+        assert [t for _, t in st._fields_] == want, name
