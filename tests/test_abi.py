@@ -59,6 +59,22 @@ def test_host_validation_without_device(lib):
     w = binding.dg_weights()
     assert lib.dg_model_create(ctypes.byref(cfg), ctypes.byref(w), ctypes.byref(out)) == 1
     assert b"multiple" in lib.dg_last_error()
+    # NVFP4 expert weights: d and I multiples of 32 and at most 2048 (a unit's block scales
+    # are staged in shared memory), checked before any weight pointer or device call
+    for d, inter in ((2048 + 32, 768), (2048, 48), (2056, 768)):
+        cfg4 = binding.dg_config(n_layers=1, d_model=d, n_q_heads=16, n_kv_heads=8,
+                                 head_dim=128, n_experts=8, top_k=2, expert_inter=inter,
+                                 shared_inter=64, vocab=16, window=4, canvas=8,
+                                 rope_base=1e4, rms_eps=1e-6, logit_scale=8,
+                                 dtype=binding.DG_BF16_FP4EXP, max_batch=1, max_prompt=8)
+        assert lib.dg_model_create(ctypes.byref(cfg4), ctypes.byref(w), ctypes.byref(out)) == 1
+        assert b"NVFP4" in lib.dg_last_error(), (d, inter, lib.dg_last_error())
+    cfg5 = binding.dg_config(n_layers=1, d_model=64, n_q_heads=4, n_kv_heads=2, head_dim=16,
+                             n_experts=8, top_k=2, expert_inter=64, shared_inter=64, vocab=16,
+                             window=4, canvas=8, rope_base=1e4, rms_eps=1e-6, logit_scale=8,
+                             dtype=4, max_batch=1, max_prompt=8)
+    assert lib.dg_model_create(ctypes.byref(cfg5), ctypes.byref(w), ctypes.byref(out)) == 1
+    assert b"dtype" in lib.dg_last_error()
     assert lib.dg_model_destroy(None) == 0 and lib.dg_kv_destroy(None) == 0
 
 
